@@ -1,0 +1,495 @@
+#!/usr/bin/env python
+"""KDA recurrence benchmark: one JSON line on rank 0.
+
+Default workload (the step): one chunked prefill over the layer-shape batch
+(B=1, H=96, T=8192, dk=dv=128, bf16 q/k/v/g/beta, fp32 state, chunk 64), all of
+it in the library's kernels, inputs resident in HBM. The same line carries the
+decode step (256 requests x 96 heads, fp32 states in place) as a second
+measurement, the end-to-end figure through host buffers, the roofline of the
+dominant kernel, the SM clocks seen while timing, and the fp64 oracle timed on
+the host cores as the CPU baseline.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload prefill|varlen|b2|decode] [--path auto|simt|tc]
+
+Multi-GPU (torchrun, one rank per GPU): (sequence, head) units are independent,
+so every rank runs its own batch (weak scaling, no collective on the data path);
+value = all ranks' tokens / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s (H=96,d=128) & % tensor peak; decode GB/s vs HBM"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+WORKLOAD_ALIASES = {"prefill": "prefill_h96_T8192_d128_bf16", "varlen": "varlen_h96_8seq_d128_bf16",
+                    "b2": "b2_h4_T2048_d128_bf16", "small": "small_f32_T256_d32",
+                    "decode": "decode_n256_h96_d128"}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--workload", default="prefill", choices=sorted(WORKLOAD_ALIASES))
+    p.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    p.add_argument("--decode-steps", type=int, default=50)
+    p.add_argument("--decode-requests", type=int, default=256,
+                   help="requests in the decode batch (smaller only for profiling captures)")
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU-baseline sample time")
+    return p.parse_args()
+
+
+# ----------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def source_sha(relpath):
+    with open(os.path.join(ROOT, relpath), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def traffic_for(kernel_src, workload_name):
+    """DRAM bytes per launch from the committed ncu summary, or None if the
+    summary is missing or was taken on a different version of the kernel."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[workload_name]
+        if e.get("source_sha") != source_sha(kernel_src):
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = str(device_index)
+        self.proc = None
+        self.out = None
+
+    def __enter__(self):
+        try:
+            self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.out is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.out.flush()
+        rows = []
+        with open(self.out.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9 and parts[0] == self.idx:
+                    rows.append(parts)
+        os.unlink(self.out.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def prefill_algorithmic(w, elem):
+    """Algorithmic bytes and flops of one prefill over workload w.
+
+    bytes: q, k, g (dk each), v and o (dv each), beta, per token-head, in the
+    storage dtype; plus the fp32 initial state read (when present) and the
+    final state written, once per (sequence, head).
+    flops per token-head (chunk C): 6 dk dv for the three state contractions
+    (W S, (Gamma q) S, Kh^T U), C (3 dk + 2 dv) for the lower-triangular chunk
+    products (A and P Grams, W, Ut, P U), C^2/3 for the triangular solve."""
+    th = w.total_tokens * w.H
+    units = w.num_seqs * w.H
+    b = th * ((3 * w.dk + 2 * w.dv) * elem + elem) + units * w.dk * w.dv * 4 * (2 if w.s0_std > 0 else 1)
+    C = w.chunk
+    f = th * (6 * w.dk * w.dv + C * (3 * w.dk + 2 * w.dv) + C * C / 3.0)
+    return float(b), float(f)
+
+
+def decode_algorithmic(N, H, dk, dv, elem):
+    per_head = 2 * dk * dv * 4 + (3 * dk + dv) * elem + elem + dv * elem
+    return float(N * H * per_head), float(N * H * 7 * dk * dv)
+
+
+# --------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, device):
+    import torch
+    from linear_attention_recurrence_11_b200 import kda
+    from linear_attention_recurrence_11_b200.inputs import WORKLOADS, workload_inputs
+    import dataclasses
+
+    wname = WORKLOAD_ALIASES[args.workload]
+    w = WORKLOADS[wname]
+    peaks = load_peaks()
+    res = {}
+    stream = torch.cuda.current_stream(device)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    if w.decode_steps:
+        return run_decode_main(args, rank, world, device, w, peaks, barrier, max_over_ranks)
+
+    # every rank draws its own batch (independent sequences)
+    w_rank = dataclasses.replace(w, seed=w.seed + 7919 * rank)
+    inp = workload_inputs(w_rank, device=device)
+    B = 1 if w.seqlens else w.B
+    T = w.total_tokens if w.seqlens else w.T
+    N = w.num_seqs
+    dt = inp["k"].dtype
+    elem = inp["k"].element_size()
+    o = torch.empty((B, T, w.H, w.dv), dtype=dt, device=device)
+    ST = torch.empty((N, w.H, w.dv, w.dk), dtype=torch.float32, device=device)
+    ws_n = kda.kda_forward_workspace_size(B, T, w.H, w.dk, w.dv, w.chunk, N, dt)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=device)
+    cu = inp.get("cu_seqlens")
+    launches = kda.kda_forward_launches(B, T, w.H, w.dk, w.dv, w.chunk, dt, cu is not None, N, args.path)
+    tc_ok = kda.kda_forward_launches(B, T, w.H, w.dk, w.dv, w.chunk, dt, cu is not None, N, "tc") > 0
+    path_used = "tc" if (args.path != "simt" and tc_ok) else "simt"
+
+    def step():
+        kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"],
+                        chunk=w.chunk, cu_seqlens=cu, o=o, S_T=ST, workspace=ws, path=args.path)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    barrier()
+    torch.cuda.synchronize(device)
+    K = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index) as clk:
+        t0.record(stream)
+        for i in range(K):
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize(device)
+    barrier()
+    torch.cuda.synchronize(device)
+    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    kern_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
+    ms_step = ms_total / K
+    tokens = w.total_tokens
+    value = world * tokens * K / (ms_total / 1e3)
+    alg_bytes, alg_flops = prefill_algorithmic(w, elem)
+    kern_src = ("linear_attention_recurrence_11_b200/csrc/kda_prefill_tc.cu" if path_used == "tc"
+                else "linear_attention_recurrence_11_b200/csrc/kda_prefill_simt.cu")
+    achieved = alg_bytes / (kern_ms / 1e3) / 1e9
+    traffic = traffic_for(kern_src, wname)
+    res.update({
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16" if path_used == "tc" else ("f32" if elem == 4 else "bf16-storage/f32-compute"),
+        "data": "synthetic (seeded: q,k unit-norm N(0,1); v N(0,1); beta sigmoid(N); g -5*sigmoid(N))",
+        "config": {"workload": wname, "B": B, "T": T, "H": w.H, "dk": w.dk, "dv": w.dv,
+                   "chunk": w.chunk, "num_seqs": N, "kernel_path": path_used,
+                   "l2": f"inputs larger than L2 ({(inp['q'].numel() * elem * 4) / 1e6:.0f} MB read per step)",
+                   "parallelism": f"dp{world} over independent (sequence, head) units"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
+                     "kernel": os.path.basename(kern_src), "kernel_ms": kern_ms,
+                     "algorithmic_bytes_per_launch": alg_bytes, "peak_source": peaks["source"] + " (hbm_gbs)"},
+        "tensor": {"achieved_tflops": alg_flops / (kern_ms / 1e3) / 1e12,
+                   "peak_tflops": peaks["bf16_tflops"],
+                   "frac": alg_flops / (kern_ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                   "algorithmic_flops_per_launch": alg_flops, "peak_source": peaks["source"] + " (bf16_tflops)"},
+        "gpu_launches": K * launches,
+        "clocks": clk.summary(),
+    })
+
+    if not args.no_e2e:
+        res["e2e"] = e2e_prefill(args, device, inp, w, o, ST, ws, cu, world, barrier, max_over_ranks)
+    if not args.no_decode and args.workload == "prefill":
+        res["decode"] = decode_measure(args, device, peaks, barrier, max_over_ranks, world,
+                                       steps=args.decode_steps)
+        res["gpu_launches"] += res["decode"]["gpu_launches"]
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_prefill(inp, w, args.cpu_seconds)
+    return res
+
+
+def e2e_prefill(args, device, inp, w, o, ST, ws, cu, world, barrier, max_over_ranks):
+    """Same metric through the public API from pinned host buffers: per step,
+    H2D of q,k,v,g,beta(,S0), the prefill, D2H of o and S_T."""
+    import torch
+    from linear_attention_recurrence_11_b200 import kda
+    names = [n for n in ("q", "k", "v", "g", "beta", "S0") if inp.get(n) is not None]
+    host = {n: inp[n].to("cpu").pin_memory() for n in names}
+    dev = {n: torch.empty_like(inp[n]) for n in names}
+    o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    S_h = torch.empty(ST.shape, dtype=ST.dtype, pin_memory=True)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = o_h.numel() * o_h.element_size() + S_h.numel() * S_h.element_size()
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        for n in names:
+            dev[n].copy_(host[n], non_blocking=True)
+        kda.kda_forward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev.get("S0"),
+                        chunk=w.chunk, cu_seqlens=cu, o=o, S_T=ST, workspace=ws, path=args.path)
+        o_h.copy_(o, non_blocking=True)
+        S_h.copy_(ST, non_blocking=True)
+
+    K = max(3, min(args.steps, 10))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(device)
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(K):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_over_ranks(a.elapsed_time(b))
+    return {"value": world * w.total_tokens * K / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
+            "ms_per_step": ms / K}
+
+
+def decode_measure(args, device, peaks, barrier, max_over_ranks, world, steps):
+    """Decode step over 256 requests x 96 heads (1.61 GB of fp32 state, larger
+    than L2), states updated in place; per-step inputs cycle over 8 pre-drawn
+    sets."""
+    import torch
+    from linear_attention_recurrence_11_b200 import kda
+    from linear_attention_recurrence_11_b200.inputs import WORKLOADS, workload_inputs
+    import dataclasses
+    w = WORKLOADS["decode_n256_h96_d128"]
+    if args.decode_requests != w.B:
+        w = dataclasses.replace(w, B=args.decode_requests)
+    S = workload_inputs(w, device=device, step=0)["S0"]
+    sets = []
+    for s in range(8):
+        d = workload_inputs(w, device=device, step=s)
+        sets.append({k: d[k][:, 0].contiguous() for k in ("q", "k", "v", "g", "beta")})
+    o = torch.empty((w.B, w.H, w.dv), dtype=sets[0]["k"].dtype, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step(i):
+        d = sets[i % 8]
+        kda.kda_decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], S, o)
+
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize(device)
+    barrier()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(device.index) as clk:
+        a.record(stream)
+        for i in range(steps):
+            step(i)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+    ms = max_over_ranks(a.elapsed_time(b)) / steps
+    elem = sets[0]["k"].element_size()
+    alg_bytes, _ = decode_algorithmic(w.B, w.H, w.dk, w.dv, elem)
+    gbs = alg_bytes / (ms / 1e3) / 1e9
+    return {"metric": f"KDA decode step GB/s ({w.B} req x {w.H} heads, fp32 state)",
+            "value": gbs * world, "unit": "GB/s", "ms_per_step": ms,
+            "tokens_per_s": world * w.B / (ms / 1e3), "steps": steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "kernel": "kda_decode.cu",
+                         "traffic": traffic_for("linear_attention_recurrence_11_b200/csrc/kda_decode.cu",
+                                                "decode_n256_h96_d128"),
+                         "algorithmic_bytes_per_launch": alg_bytes,
+                         "peak_source": peaks["source"] + " (hbm_gbs)"},
+            "gpu_launches": steps, "clocks": clk.summary(),
+            "requests": w.B, "l2": f"state {w.B * w.H * w.dk * w.dv * 4 / 1e9:.2f} GB per step, larger than L2"}
+
+
+def run_decode_main(args, rank, world, device, w, peaks, barrier, max_over_ranks):
+    d = decode_measure(args, device, peaks, barrier, max_over_ranks, world, steps=args.steps)
+    return {"metric": d["metric"], "value": d["value"], "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": d["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": {"workload": w.name, "N": d["requests"], "H": w.H, "dk": w.dk,
+                                            "dv": w.dv, "l2": d["l2"]},
+            "roofline": d["roofline"], "gpu_launches": d["gpu_launches"], "clocks": d["clocks"]}
+
+
+# ---------------------------------------------------------- CPU baseline
+
+def _oracle_sample(inp, w, seconds, max_heads=None):
+    """Time the fp64 oracle (sequential form, one host core) on whole heads of
+    the workload until about ``seconds`` have elapsed. Returns
+    (token-heads processed, elapsed seconds, heads)."""
+    import oracle
+    from linear_attention_recurrence_11_b200.inputs import to_f64
+    oracle.build()
+    T = w.total_tokens if w.seqlens else w.T
+    T = min(T, 8192)
+    done, el, heads = 0, 0.0, 0
+    h = 0
+    while el < seconds and (max_heads is None or heads < max_heads):
+        a = [to_f64(inp[x][0, :T, h % w.H]) for x in ("q", "k", "v", "g", "beta")]
+        t = time.perf_counter()
+        oracle.forward(*a)
+        el += time.perf_counter() - t
+        done += T
+        heads += 1
+        h += 1
+    return done, el, heads, T
+
+
+def cpu_baseline_prefill(inp, w, seconds):
+    done, el, heads, T = _oracle_sample(inp, w, seconds)
+    return {"value": done / w.H / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{heads} of {w.H} heads x {T} tokens of {w.name}, sequential fp64 oracle, "
+                      f"one thread; tokens/s = token-heads/s / {w.H}",
+            "host_cpus": os.cpu_count(), "seconds": el}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the oracle as it stands, on host cores, on a bounded
+    sample of the same workload per step."""
+    if rank != 0:
+        return None
+    import torch
+    from linear_attention_recurrence_11_b200.inputs import WORKLOADS, workload_inputs
+    w = WORKLOADS[WORKLOAD_ALIASES[args.workload]]
+    if w.decode_steps:
+        w_in = workload_inputs(w, device="cpu", step=0)
+    else:
+        import dataclasses
+        small = dataclasses.replace(w, T=min(w.T or 8192, 8192), seqlens=(), B=1, H=2)
+        w_in = workload_inputs(small, device="cpu")
+    per_step = max(1.0, min(8.0, 150.0 / max(1, args.steps + args.warmup)))
+    tot_done, tot_el = 0, 0.0
+    heads = T = 0
+    for i in range(args.warmup + args.steps):
+        if w.decode_steps:
+            import numpy as np
+            import oracle
+            from linear_attention_recurrence_11_b200.inputs import to_f64
+            d = {k: to_f64(w_in[k][:, 0]) for k in ("q", "k", "v", "g", "beta")}
+            S = to_f64(w_in["S0"])
+            t = time.perf_counter()
+            n_units = 0
+            while time.perf_counter() - t < per_step:
+                n, h = n_units % w.B, (n_units // w.B) % w.H
+                St = np.ascontiguousarray(S[n, h])
+                oracle.decode_step(d["q"][n, h], d["k"][n, h], d["v"][n, h], d["g"][n, h],
+                                   d["beta"][n, h], St)
+                n_units += 1
+            done, el = n_units, time.perf_counter() - t
+        else:
+            done, el, heads, T = _oracle_sample(w_in, small, per_step, max_heads=2)
+        if i >= args.warmup:
+            tot_done += done
+            tot_el += el
+    if w.decode_steps:
+        alg, _ = decode_algorithmic(1, 1, w.dk, w.dv, 2)
+        value, unit = tot_done * alg / tot_el / 1e9, "GB/s"
+        metric = "KDA decode step GB/s (256 req x 96 heads, fp32 state)"
+        sample = f"(request, head) units of one decode step, fp64 oracle, one thread, ~{per_step:.0f} s per step"
+    else:
+        value, unit = tot_done / w.H / tot_el, "tokens/s"
+        metric = METRIC
+        sample = (f"up to 2 heads x {T} tokens per step (same distributions as {w.name}), "
+                  f"sequential fp64 oracle, one thread; tokens/s = token-heads/s / {w.H}")
+    ms = tot_el / max(1, args.steps) * 1e3
+    return {"impl": "reference", "metric": metric, "value": value, "unit": unit, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    import torch
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=device)
+    try:
+        res = run_ours(args, rank, world, device)
+    finally:
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,139 @@
+/*
+ * kda.h — C ABI of libkda.so, a B200 (sm_100a) implementation of the KDA
+ * (Kimi Delta Attention) token-mixing recurrence.
+ *
+ * The operation (Kimi K3 wiki, "Exercices", Q7; the report's eq. 1 as listed
+ * on "Ce qui est public et ce qui ne l'est pas"): for every (sequence, head),
+ * with state S in R^{dk x dv},
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(exp(g_t)) S_{t-1} + beta_t k_t v_t^T,
+ *     o_t = S_t^T q_t,
+ *
+ * with a per-channel log-decay g_t in [g_min, 0], g_min = -5 ("Exercices",
+ * Q8) and an L2-normalised key ("Exercices", Q9). Prefill evaluates it in
+ * chunks; the state is carried from chunk to chunk by the KCP pair
+ * (cumulative transition, local state) and its composition ("Exercices",
+ * Q21-Q22; report eq. 14).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Every pointer argument is DEVICE memory owned by the caller unless the
+ *    comment says otherwise. The library never allocates, frees or
+ *    synchronises: work is enqueued on `stream` (a cudaStream_t; NULL = the
+ *    legacy default stream) and the call returns once it is launched.
+ *  - Activations are token-major and contiguous:
+ *        q, k, g : [B, T, H, dk]      v, o : [B, T, H, dv]      beta : [B, T, H]
+ *    all of the element type `dtype` (o is written in that type too).
+ *  - States are fp32, layout [N, H, dv, dk]: element (i, j) of S for unit
+ *    (n, h) sits at ((n*H + h)*dv + j)*dk + i (a column of S is contiguous).
+ *    Prefill's S_T feeds kda_decode_step's S directly.
+ *  - Supported: dk, dv in {32, 64, 128}; chunk in {16, 32, 64}; every pointer
+ *    16-byte aligned.
+ *  - Preconditions that are documented, not checked: g in [-5, 0],
+ *    beta in [0, 1], ||k_t||_2 = 1 (q and k normalised upstream; the kernels
+ *    do not renormalise and apply no 1/sqrt(dk) scale). A g below -5 may
+ *    overflow the 16-token exponent factorisation.
+ *  - Errors: a call whose arguments fail validation returns a non-zero
+ *    kda_status and launches nothing. A launch failure returns
+ *    KDA_ERR_CUDA. Faults inside a kernel surface at the caller's next
+ *    synchronisation of `stream`.
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1, /* null required pointer, non-positive or inconsistent sizes */
+    KDA_ERR_UNSUPPORTED = 2, /* dk/dv/chunk/dtype/path combination not built            */
+    KDA_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned                         */
+    KDA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required               */
+    KDA_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed               */
+    KDA_ERR_TIMEOUT = 6      /* (device status word) a bounded wait gave up              */
+} kda_status;
+
+typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype;
+
+/* Which prefill kernel kda_forward_ex runs. AUTO picks the tensor-core kernel
+ * where it is built (bf16, dk = dv = 128, chunk = 64) and the SIMT kernel
+ * otherwise. */
+typedef enum { KDA_PATH_AUTO = 0, KDA_PATH_SIMT = 1, KDA_PATH_TC = 2 } kda_path;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *kda_status_string(int status);
+
+/* ABI version of this header (bumped when a signature changes). */
+int kda_abi_version(void);
+
+/*
+ * Bytes of device workspace kda_forward needs for these sizes (0 if none).
+ * num_seqs is the number of packed sequences when cu_seqlens is used, else B.
+ * Returns (size_t)-1 if the sizes are invalid.
+ */
+size_t kda_forward_workspace_size(int B, int T, int H, int dk, int dv, int chunk,
+                                  int num_seqs, int dtype);
+
+/*
+ * Chunked prefill with KCP inter-chunk state composition.
+ *
+ *   q, k, g, v, beta : inputs (layouts above).
+ *   S0   : [N, H, dv, dk] fp32 initial states, or NULL for zeros.
+ *   o    : [B, T, H, dv] output, dtype.
+ *   S_T  : [N, H, dv, dk] fp32 final states, or NULL to skip; may alias S0
+ *          (each unit reads its S0 fully before writing its S_T).
+ *   B, T, H, dk, dv : sizes; T = 0 is allowed (S_T = S0, nothing else).
+ *   chunk : tokens per chunk (16, 32 or 64).
+ *   cu_seqlens : NULL for B dense sequences of T tokens (N = B), or device
+ *          int32 [num_seqs + 1] offsets of packed sequences (B must be 1,
+ *          cu_seqlens[0] = 0, non-decreasing, cu_seqlens[num_seqs] = T;
+ *          chunks never straddle sequences; N = num_seqs).
+ *   workspace / workspace_bytes : device scratch of at least
+ *          kda_forward_workspace_size(...) bytes (may be NULL when that is 0).
+ *   dev_status : NULL, or a device int the kernels set to KDA_ERR_TIMEOUT if
+ *          a bounded wait gives up (the caller zeroes it and reads it after
+ *          synchronising).
+ *   stream : cudaStream_t to enqueue on.
+ */
+int kda_forward(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                const float *S0, void *o, float *S_T, int B, int T, int H, int dk, int dv,
+                int chunk, int dtype, const int32_t *cu_seqlens, int num_seqs,
+                void *workspace, size_t workspace_bytes, int *dev_status, void *stream);
+
+/* kda_forward with an explicit kernel choice (kda_path). KDA_PATH_TC on a
+ * combination the tensor-core kernel does not cover returns
+ * KDA_ERR_UNSUPPORTED. */
+int kda_forward_ex(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                   const float *S0, void *o, float *S_T, int B, int T, int H, int dk, int dv,
+                   int chunk, int dtype, const int32_t *cu_seqlens, int num_seqs,
+                   void *workspace, size_t workspace_bytes, int *dev_status, void *stream,
+                   int path);
+
+/* Number of kernel launches one kda_forward_ex call with these arguments
+ * enqueues (0 when T = 0 and no state is copied), or -1 if invalid. */
+int kda_forward_launches(int B, int T, int H, int dk, int dv, int chunk, int dtype,
+                         int has_cu_seqlens, int num_seqs, int path);
+
+/*
+ * One decode step: one new token for each of N requests, states in place.
+ * Same recurrence with T = 1 ("Exercices", Q4: decode is bound by memory
+ * bandwidth; each state is read and written exactly once).
+ *
+ *   q, k, g : [N, H, dk];  v : [N, H, dv];  beta : [N, H]   (dtype)
+ *   S       : [N, H, dv, dk] fp32, read and overwritten in place.
+ *   o       : [N, H, dv] output, dtype.
+ */
+int kda_decode_step(const void *q, const void *k, const void *v, const void *g,
+                    const void *beta, float *S, void *o, int N, int H, int dk, int dv,
+                    int dtype, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */

@@ -6,14 +6,12 @@ C ABI declared in ``include/kda.h``); ``kda`` is its thin Python binding and
 ``inputs`` the seeded synthetic-input generator. Importing the binding raises
 if the shared library has not been built: there is no CPU fallback.
 """
-__all__ = ["kda", "inputs"]
+import importlib
+
+__all__ = ["kda", "inputs", "build"]
 
 
 def __getattr__(name):
-    if name == "kda":
-        from . import kda
-        return kda
-    if name == "inputs":
-        from . import inputs
-        return inputs
+    if name in __all__:
+        return importlib.import_module(f"{__name__}.{name}")
     raise AttributeError(name)

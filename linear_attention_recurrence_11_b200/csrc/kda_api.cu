@@ -1,0 +1,120 @@
+// C ABI of libkda.so: argument validation and kernel dispatch (include/kda.h).
+#include <stdint.h>
+
+#include "kda_internal.cuh"
+
+namespace {
+
+bool aligned16(const void *p) { return p == nullptr || (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool head_dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+bool chunk_ok(int c) { return c == 16 || c == 32 || c == 64; }
+bool dtype_ok(int t) { return t == KDA_DTYPE_F32 || t == KDA_DTYPE_BF16; }
+
+// Validates the shape arguments shared by kda_forward_* and fills the sizes.
+int check_prefill_sizes(int B, int T, int H, int dk, int dv, int chunk, int dtype,
+                        bool has_cu, int num_seqs, int path, kda::PrefillArgs *a) {
+    if (B <= 0 || T < 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if (!dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv) || !chunk_ok(chunk)) return KDA_ERR_UNSUPPORTED;
+    if (has_cu && (B != 1 || num_seqs <= 0)) return KDA_ERR_INVALID_ARG;
+    if (path != KDA_PATH_AUTO && path != KDA_PATH_SIMT && path != KDA_PATH_TC) return KDA_ERR_INVALID_ARG;
+    if (path == KDA_PATH_TC && !kda::prefill_tc_supported(dk, dv, chunk, dtype)) return KDA_ERR_UNSUPPORTED;
+    // the kernels index tokens with size_t and units with 32-bit grid indices
+    const size_t units = (size_t)(has_cu ? num_seqs : B) * (size_t)H;
+    if (units * (size_t)(dv / 32) > 0x7fffffffu) return KDA_ERR_UNSUPPORTED;
+    a->B = B; a->T = T; a->H = H; a->dk = dk; a->dv = dv; a->chunk = chunk; a->dtype = dtype;
+    a->num_units = has_cu ? num_seqs : B;
+    return KDA_OK;
+}
+
+bool use_tc(const kda::PrefillArgs &a, int path) {
+    if (path == KDA_PATH_SIMT) return false;
+    return kda::prefill_tc_supported(a.dk, a.dv, a.chunk, a.dtype);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *kda_status_string(int status) {
+    switch (status) {
+        case KDA_OK: return "ok";
+        case KDA_ERR_INVALID_ARG: return "invalid argument";
+        case KDA_ERR_UNSUPPORTED: return "unsupported size, dtype or path";
+        case KDA_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+        case KDA_ERR_WORKSPACE: return "workspace missing or too small";
+        case KDA_ERR_CUDA: return "CUDA error";
+        case KDA_ERR_TIMEOUT: return "bounded wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int kda_abi_version(void) { return 1; }
+
+size_t kda_forward_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int num_seqs,
+                                  int dtype) {
+    kda::PrefillArgs a{};
+    const bool has_cu = num_seqs > 0 && B == 1 && num_seqs != B;
+    if (check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, has_cu, num_seqs, KDA_PATH_AUTO, &a))
+        return (size_t)-1;
+    a.num_units = num_seqs > 0 ? num_seqs : B;
+    size_t ws = kda::prefill_simt_workspace(a);
+    if (kda::prefill_tc_supported(dk, dv, chunk, dtype)) {
+        const size_t t = kda::prefill_tc_workspace(a);
+        ws = t > ws ? t : ws;
+    }
+    return ws;
+}
+
+int kda_forward_launches(int B, int T, int H, int dk, int dv, int chunk, int dtype,
+                         int has_cu_seqlens, int num_seqs, int path) {
+    kda::PrefillArgs a{};
+    if (check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, has_cu_seqlens != 0, num_seqs, path, &a))
+        return -1;
+    return use_tc(a, path) ? kda::prefill_tc_launches(a) : kda::prefill_simt_launches(a);
+}
+
+int kda_forward_ex(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                   const float *S0, void *o, float *S_T, int B, int T, int H, int dk, int dv,
+                   int chunk, int dtype, const int32_t *cu_seqlens, int num_seqs, void *workspace,
+                   size_t workspace_bytes, int *dev_status, void *stream, int path) {
+    kda::PrefillArgs a{};
+    int st = check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, cu_seqlens != nullptr, num_seqs,
+                                 path, &a);
+    if (st) return st;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    for (const void *p : {q, k, v, g, beta, (const void *)S0, (const void *)o, (const void *)S_T,
+                          (const void *)cu_seqlens, (const void *)workspace, (const void *)dev_status})
+        if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;
+    a.S0 = S0; a.o = o; a.ST = S_T; a.cu_seqlens = cu_seqlens;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.dev_status = dev_status;
+    a.stream = static_cast<cudaStream_t>(stream);
+    const bool tc = use_tc(a, path);
+    const size_t need = tc ? kda::prefill_tc_workspace(a) : kda::prefill_simt_workspace(a);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
+    const cudaError_t e = tc ? kda::launch_prefill_tc(a) : kda::launch_prefill_simt(a);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_forward(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                const float *S0, void *o, float *S_T, int B, int T, int H, int dk, int dv,
+                int chunk, int dtype, const int32_t *cu_seqlens, int num_seqs, void *workspace,
+                size_t workspace_bytes, int *dev_status, void *stream) {
+    return kda_forward_ex(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, dtype, cu_seqlens,
+                          num_seqs, workspace, workspace_bytes, dev_status, stream, KDA_PATH_AUTO);
+}
+
+int kda_decode_step(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                    float *S, void *o, int N, int H, int dk, int dv, int dtype, void *stream) {
+    if (N <= 0 || H <= 0 || !dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if ((size_t)N * (size_t)H > 0x7fffffffu) return KDA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !g || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+    for (const void *p : {q, k, v, g, beta, (const void *)S, (const void *)o})
+        if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
+    kda::DecodeArgs a{q, k, v, g, beta, S, o, N, H, dk, dv, dtype, static_cast<cudaStream_t>(stream)};
+    return kda::launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// Internal declarations shared by the libkda.so translation units.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+// Arguments of one prefill call, as validated by the C ABI layer.
+struct PrefillArgs {
+    const void *q, *k, *v, *g, *beta;
+    const float *S0;
+    void *o;
+    float *ST;
+    const int32_t *cu_seqlens;  // device offsets or nullptr
+    int B, T, H, dk, dv, chunk, dtype;
+    int num_units;              // N: sequences (B, or num_seqs with cu_seqlens)
+    void *workspace;
+    size_t workspace_bytes;
+    int *dev_status;
+    cudaStream_t stream;
+};
+
+struct DecodeArgs {
+    const void *q, *k, *v, *g, *beta;
+    float *S;
+    void *o;
+    int N, H, dk, dv, dtype;
+    cudaStream_t stream;
+};
+
+// Element loads/stores in the storage dtype, computed in fp32.
+__device__ __forceinline__ float ld_elem(const float *p, size_t i) { return p[i]; }
+__device__ __forceinline__ float ld_elem(const __nv_bfloat16 *p, size_t i) {
+    return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void st_elem(float *p, size_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void st_elem(__nv_bfloat16 *p, size_t i, float x) {
+    p[i] = __float2bfloat16_rn(x);
+}
+
+// Launchers (return cudaSuccess or the launch error).
+cudaError_t launch_prefill_simt(const PrefillArgs &a);
+size_t prefill_simt_workspace(const PrefillArgs &a);
+int prefill_simt_launches(const PrefillArgs &a);
+
+bool prefill_tc_supported(int dk, int dv, int chunk, int dtype);
+cudaError_t launch_prefill_tc(const PrefillArgs &a);
+size_t prefill_tc_workspace(const PrefillArgs &a);
+int prefill_tc_launches(const PrefillArgs &a);
+
+cudaError_t launch_decode(const DecodeArgs &a);
+
+}  // namespace kda

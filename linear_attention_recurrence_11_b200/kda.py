@@ -1,0 +1,161 @@
+"""Python binding of libkda.so (declared in include/kda.h).
+
+Argument marshalling only: torch tensors (CUDA, contiguous) are checked for
+shape/dtype and passed to the C ABI as raw device pointers with the current
+(or given) CUDA stream; every step of the computation runs in the library's
+kernels. Output tensors are allocated here with torch when the caller does not
+pass them. There is no CPU fallback: importing this module raises if
+``libkda.so`` has not been built.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"libkda.so is not built ({LIB_PATH}); run "
+                      "`python -m linear_attention_recurrence_11_b200.build`")
+
+_lib = ctypes.CDLL(LIB_PATH)
+_vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_lib.kda_status_string.argtypes = [_i]
+_lib.kda_status_string.restype = ctypes.c_char_p
+_lib.kda_abi_version.restype = _i
+_lib.kda_forward_workspace_size.argtypes = [_i] * 8
+_lib.kda_forward_workspace_size.restype = _sz
+_lib.kda_forward_launches.argtypes = [_i] * 10
+_lib.kda_forward_launches.restype = _i
+_FWD = [_vp] * 8 + [_i] * 7 + [_vp, _i, _vp, _sz, _vp, _vp]
+_lib.kda_forward.argtypes = _FWD
+_lib.kda_forward.restype = _i
+_lib.kda_forward_ex.argtypes = _FWD + [_i]
+_lib.kda_forward_ex.restype = _i
+_lib.kda_decode_step.argtypes = [_vp] * 7 + [_i] * 5 + [_vp]
+_lib.kda_decode_step.restype = _i
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT = 0, 1, 2, 3
+KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = 4, 5, 6
+DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+PATHS = {"auto": 0, "simt": 1, "tc": 2}
+
+
+class KdaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {kda_status_string(code)} (status {code})")
+
+
+def kda_status_string(code: int) -> str:
+    return _lib.kda_status_string(int(code)).decode()
+
+
+def kda_abi_version() -> int:
+    return _lib.kda_abi_version()
+
+
+def kda_forward_workspace_size(B, T, H, dk, dv, chunk, num_seqs, dtype) -> int:
+    n = _lib.kda_forward_workspace_size(B, T, H, dk, dv, chunk, num_seqs, DTYPES.get(dtype, dtype))
+    if n == ctypes.c_size_t(-1).value:
+        raise KdaError(KDA_ERR_INVALID_ARG, "kda_forward_workspace_size")
+    return int(n)
+
+
+def kda_forward_launches(B, T, H, dk, dv, chunk, dtype, has_cu_seqlens, num_seqs, path="auto") -> int:
+    return _lib.kda_forward_launches(B, T, H, dk, dv, chunk, DTYPES.get(dtype, dtype),
+                                     int(bool(has_cu_seqlens)), num_seqs, PATHS[path])
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream, device):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, dtype=None, shape=None, device=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def kda_forward(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=None, o=None,
+                S_T=None, return_state: bool = True, workspace=None, dev_status=None,
+                stream=None, path: str = "auto"):
+    """Chunked KDA prefill. q, k, g ``[B, T, H, dk]``; v ``[B, T, H, dv]``;
+    beta ``[B, T, H]`` (fp32 or bf16, all the same); S0 ``[N, H, dv, dk]`` fp32
+    or None; cu_seqlens int32 ``[N+1]`` (B must be 1) or None.
+    Returns ``(o, S_T)`` (S_T None when ``return_state`` is False)."""
+    _need(k, "k")
+    dtype, dev = k.dtype, k.device
+    if dtype not in DTYPES:
+        raise ValueError(f"unsupported dtype {dtype}")
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    _need(q, "q", dtype, (B, T, H, dk), dev)
+    _need(g, "g", dtype, (B, T, H, dk), dev)
+    _need(v, "v", dtype, (B, T, H, dv), dev)
+    _need(beta, "beta", dtype, (B, T, H), dev)
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, None, dev)
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (N, H, dv, dk), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dtype, device=dev)
+    _need(o, "o", dtype, (B, T, H, dv), dev)
+    if return_state and S_T is None:
+        S_T = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, (N, H, dv, dk), dev)
+    ws_need = kda_forward_workspace_size(B, T, H, dk, dv, chunk, N, dtype)
+    if workspace is None and ws_need > 0:
+        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = _lib.kda_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                             _ptr(S_T), B, T, H, dk, dv, int(chunk), DTYPES[dtype],
+                             _ptr(cu_seqlens), N if cu_seqlens is not None else 0,
+                             _ptr(workspace), ws_bytes, _ptr(dev_status),
+                             _stream_handle(stream, dev), PATHS[path])
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_forward")
+    return o, S_T
+
+
+def kda_decode_step(q, k, v, g, beta, S, o=None, *, stream=None):
+    """One decode token per request. q, k, g ``[N, H, dk]``; v ``[N, H, dv]``;
+    beta ``[N, H]``; S ``[N, H, dv, dk]`` fp32 updated in place. Returns o."""
+    _need(k, "k")
+    dtype, dev = k.dtype, k.device
+    N, H, dk = k.shape
+    dv = v.shape[-1]
+    _need(q, "q", dtype, (N, H, dk), dev)
+    _need(g, "g", dtype, (N, H, dk), dev)
+    _need(v, "v", dtype, (N, H, dv), dev)
+    _need(beta, "beta", dtype, (N, H), dev)
+    _need(S, "S", torch.float32, (N, H, dv, dk), dev)
+    if o is None:
+        o = torch.empty((N, H, dv), dtype=dtype, device=dev)
+    _need(o, "o", dtype, (N, H, dv), dev)
+    rc = _lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                              N, H, dk, dv, DTYPES[dtype], _stream_handle(stream, dev))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_decode_step")
+    return o

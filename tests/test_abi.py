@@ -1,0 +1,121 @@
+"""The C ABI on CPU: the library loads, exports every function include/kda.h
+declares, and rejects bad arguments before touching the GPU (validation runs
+on the host; none of these calls reaches a CUDA API)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def K():
+    from linear_attention_recurrence_11_b200 import build
+    build.build()
+    from linear_attention_recurrence_11_b200 import kda
+    return kda
+
+
+def declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"^[A-Za-z_][\w \*]*?\b(kda_\w+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for f in ("kda_forward", "kda_forward_ex", "kda_decode_step", "kda_forward_workspace_size",
+              "kda_status_string", "kda_forward_launches", "kda_abi_version"):
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol(K):
+    lib = ctypes.CDLL(K.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings(K):
+    assert K.kda_status_string(0) == "ok"
+    for c in range(1, 7):
+        assert K.kda_status_string(c) not in ("ok", "unknown status")
+    assert K.kda_status_string(99) == "unknown status"
+    assert K.kda_abi_version() >= 1
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null address; never dereferenced
+
+
+def fwd(K, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, S0=None, o=FAKE, S_T=None, B=1, T=64, H=2,
+             dk=128, dv=128, chunk=64, dtype=1, cu=None, num_seqs=0, ws=None, ws_bytes=0,
+             status=None, stream=None, path=0)
+    a.update(kw)
+    return K._lib.kda_forward_ex(a["q"], a["k"], a["v"], a["g"], a["beta"], a["S0"], a["o"], a["S_T"],
+                                 a["B"], a["T"], a["H"], a["dk"], a["dv"], a["chunk"], a["dtype"],
+                                 a["cu"], a["num_seqs"], a["ws"], a["ws_bytes"], a["status"],
+                                 a["stream"], a["path"])
+
+
+def test_forward_rejects_bad_sizes(K):
+    assert fwd(K, B=0) == K.KDA_ERR_INVALID_ARG
+    assert fwd(K, T=-1) == K.KDA_ERR_INVALID_ARG
+    assert fwd(K, H=0) == K.KDA_ERR_INVALID_ARG
+    assert fwd(K, dtype=7) == K.KDA_ERR_INVALID_ARG
+    assert fwd(K, dk=48) == K.KDA_ERR_UNSUPPORTED
+    assert fwd(K, dv=256) == K.KDA_ERR_UNSUPPORTED
+    assert fwd(K, chunk=128) == K.KDA_ERR_UNSUPPORTED
+    assert fwd(K, chunk=0) == K.KDA_ERR_UNSUPPORTED
+    assert fwd(K, path=9) == K.KDA_ERR_INVALID_ARG
+
+
+def test_forward_rejects_bad_pointers(K):
+    for name in ("q", "k", "v", "g", "beta", "o"):
+        assert fwd(K, **{name: None}) == K.KDA_ERR_INVALID_ARG, name
+    for name in ("q", "k", "v", "g", "beta", "o", "S0", "S_T", "cu", "status"):
+        kw = {name: FAKE + 4}
+        if name == "cu":
+            kw["num_seqs"] = 1
+        assert fwd(K, **kw) == K.KDA_ERR_ALIGNMENT, name
+
+
+def test_forward_varlen_rules(K):
+    assert fwd(K, cu=FAKE, num_seqs=0) == K.KDA_ERR_INVALID_ARG
+    assert fwd(K, cu=FAKE, num_seqs=2, B=2) == K.KDA_ERR_INVALID_ARG
+
+
+def test_tc_path_only_where_built(K):
+    # fp32 never takes the tensor-core kernel
+    assert fwd(K, dtype=0, path=K.PATHS["tc"]) == K.KDA_ERR_UNSUPPORTED
+    assert fwd(K, dk=64, path=K.PATHS["tc"]) == K.KDA_ERR_UNSUPPORTED
+
+
+def test_decode_rejects_bad_args(K):
+    d = K._lib.kda_decode_step
+    assert d(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0, 96, 128, 128, 1, None) == K.KDA_ERR_INVALID_ARG
+    assert d(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 96, 96, 128, 1, None) == K.KDA_ERR_UNSUPPORTED
+    assert d(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 4, 96, 128, 128, 1, None) == K.KDA_ERR_INVALID_ARG
+    assert d(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 8, FAKE, 4, 96, 128, 128, 1, None) == K.KDA_ERR_ALIGNMENT
+    assert d(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 96, 128, 128, 3, None) == K.KDA_ERR_INVALID_ARG
+
+
+def test_workspace_and_launch_queries(K):
+    assert K.kda_forward_workspace_size(1, 8192, 96, 128, 128, 64, 1, 1) >= 0
+    with pytest.raises(K.KdaError):
+        K.kda_forward_workspace_size(1, 8192, 96, 100, 128, 64, 1, 1)
+    assert K.kda_forward_launches(1, 8192, 96, 128, 128, 64, 1, 0, 1) >= 1
+    assert K.kda_forward_launches(1, 256, 1, 32, 32, 16, 0, 0, 1, "simt") == 1
+    assert K.kda_forward_launches(1, 256, 1, 48, 32, 16, 0, 0, 1) == -1
+
+
+def test_python_binding_refuses_cpu_tensors(K):
+    import torch
+    x = torch.zeros(1, 4, 1, 32)
+    with pytest.raises(ValueError, match="CUDA"):
+        K.kda_forward(x, x, x, x, torch.zeros(1, 4, 1))
