@@ -24,9 +24,12 @@ def K():
 
 
 def run(K, inp, chunk, path="auto", **kw):
+    status = torch.zeros(4, dtype=torch.int32, device=inp["k"].device)
     o, ST = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp.get("S0"),
-                          chunk=chunk, cu_seqlens=inp.get("cu_seqlens"), path=path, **kw)
+                          chunk=chunk, cu_seqlens=inp.get("cu_seqlens"), path=path,
+                          dev_status=status, **kw)
     torch.cuda.synchronize()
+    assert int(status[0]) == 0, f"device status {int(status[0])}"
     return o, ST
 
 
