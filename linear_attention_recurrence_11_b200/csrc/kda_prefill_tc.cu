@@ -1,7 +1,7 @@
 // Chunked KDA prefill on the 5th-generation tensor cores (sm_100a):
 // bf16 q/k/v/g/beta, fp32 state, dk = dv = 128, chunks of C = 64 tokens.
 //
-// One CTA (256 threads, ~220 KB shared memory, 448 TMEM columns) owns one
+// One CTA (256 threads, ~220 KB shared memory, all 512 TMEM columns) owns one
 // (sequence, head) unit and walks its chunks in order, carrying the state
 // from chunk to chunk with the KCP composition ("Exercices", Q21-Q22): per
 // chunk the incoming state S is mapped to Diag(Gamma_C) S + Kh^T (Ut - W S),
@@ -25,8 +25,11 @@
 //  6. tcgen05.mma: [U ; Qt S] = [Ut ; 0] + [-W ; Gamma*Q] S          (M=128, K=128)
 //  7. tcgen05.mma: O = Qt S + P U (rows 64..127),  dS = Kh^T U       (K=64)
 //     with Kh_s = e^{G_C - G_s} k_s; then S <- Diag(Gamma_C) S + dS in fp32
-//     registers (the state never leaves the SM between chunks; its bf16 copy
+//     in TMEM (the state never leaves the SM between chunks; its bf16 copy
 //     feeds step 6 of the next chunk).
+// The next chunk's tiles are requested as soon as each staging tile has been
+// consumed (g after step 2's cumulative sums, k after step 4, v after step 5,
+// q after step 6), so their HBM latency overlaps the rest of the chunk.
 // All matrices in shared memory use the 128-byte swizzled layout the TMA
 // writes and the tcgen05 descriptors read. No cluster multicast is used.
 #include "kda_internal.cuh"
@@ -44,41 +47,45 @@ constexpr int SUB = 16, NSUB = C / SUB;
 
 // ---------------------------------------------------------- smem layout
 constexpr uint32_t KB = 1024;
-constexpr uint32_t OFF_WQ = 0;          // 32 KB  A operand [-W ; Qt], K-major, 128 rows x 128 (2 K-blocks)
+constexpr uint32_t OFF_WQ = 0;          // 32 KB  A operand [-W ; Qt], K-major, 128 rows x 128 (2 K-blocks); q lands in rows 64..127
 constexpr uint32_t OFF_SB = 32 * KB;    // 32 KB  B operand S (bf16), MN-major [dk rows][dv] (2 N-blocks)
-constexpr uint32_t OFF_KH = 64 * KB;    // 16 KB  k, then Kh: A operand MN-major [tok rows][dk] (2 M-blocks)
+constexpr uint32_t OFF_KS = 64 * KB;    // 16 KB  k tile, [tok rows][dk] (2 blocks of 64 channels)
 constexpr uint32_t OFF_V = 80 * KB;     // 16 KB  v: B operand MN-major [tok rows][dv] (2 N-blocks)
 constexpr uint32_t OFF_G = 96 * KB;     // 16 KB  g, plain [64][128] bf16
 constexpr uint32_t OFF_R = 112 * KB;    // 16 KB  Gram right operand, K-major [s rows][dk]; later U (MN-major B)
 constexpr uint32_t OFF_PB = 128 * KB;   // 8 KB   rows 64..127 of the A operand [junk ; P], K-major, K = 64
-constexpr uint32_t OFF_L = 136 * KB;    // 80 KB  Gram left operands L3, L2, L1, L0 (compact), then phase-4 scratch
+constexpr uint32_t OFF_L = 136 * KB;    // 80 KB  Gram left operands L3, L2, L1, L0 (compact), then the aliases below
 constexpr uint32_t OFF_MISC = 216 * KB;
 // L region: compact left operands, L_j has 2 (64 - 16 j) rows (K part, then Q part).
 __host__ __device__ constexpr uint32_t l_rows(int j) { return 2u * (64u - 16u * j); }
 __host__ __device__ constexpr uint32_t l_off(int j) {
     return j == 3 ? 0u : j == 2 ? 8u * KB : j == 1 ? 24u * KB : 48u * KB;
 }
-// phase-4 aliases inside the L region
-constexpr uint32_t OFF_TB = OFF_L + 0;           // 16 KB  A operand T Diag(beta), K-major, 128 rows x 64
-constexpr uint32_t OFF_KT = OFF_L + 16 * KB;     // 16 KB  B operand Gamma*K, MN-major [tok][dk]
-constexpr uint32_t OFF_AF = OFF_L + 32 * KB;     // 64 x 65 fp32  A
-constexpr uint32_t OFF_TF = OFF_AF + 64 * 65 * 4; // 64 x 65 fp32  T
-constexpr uint32_t OFF_XS = OFF_TF + 64 * 65 * 4; // 3 x 16 x 17 fp32 scratch
-static_assert(OFF_XS + 3 * 16 * 17 * 4 <= OFF_MISC, "phase-4 scratch overflows the L region");
+// aliases inside the L region once the Gram MMAs are done
+constexpr uint32_t OFF_TB = OFF_L + 0;             // 16 KB  A operand T Diag(beta), K-major, 128 rows x 64
+constexpr uint32_t OFF_KT = OFF_L + 16 * KB;       // 16 KB  B operand Gamma*K, MN-major [tok][dk]
+constexpr uint32_t OFF_AF = OFF_L + 32 * KB;       // 64 x 65 fp32  A (dead once T is known)
+constexpr uint32_t OFF_KHAT = OFF_L + 32 * KB;     // 16 KB  A operand Kh, MN-major [tok][dk] (written after A is dead)
+constexpr uint32_t OFF_TF = OFF_L + 49 * KB;       // 64 x 68 fp32  T
+constexpr uint32_t OFF_XS = OFF_TF + 64 * 68 * 4;  // 3 x 16 x 20 fp32 scratch
+static_assert(OFF_AF + 64 * 65 * 4 <= OFF_TF, "A overlaps T");
+static_assert(OFF_XS + 3 * 16 * 20 * 4 <= OFF_MISC, "scratch overflows the L region");
 // misc
 constexpr uint32_t OFF_BAR = OFF_MISC;              // 2 mbarriers
 constexpr uint32_t OFF_TMEMADDR = OFF_MISC + 16;
 constexpr uint32_t OFF_BETA = OFF_MISC + 64;        // 64 fp32
-constexpr uint32_t OFF_DSUM = OFF_BETA + 256;       // 4 x 128 fp32 subtile totals of g
+constexpr uint32_t OFF_DSUM = OFF_BETA + 256;       // 4 x 128 fp32 subtile totals of g (log2 units)
 constexpr uint32_t OFF_GAMC = OFF_DSUM + 2048;      // 128 fp32 Gamma_C
 constexpr uint32_t SMEM_USED = OFF_GAMC + 512;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;   // slack for 1024-byte alignment
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// TMEM columns
-constexpr uint32_t TM_GRAM = 0, TM_W = 64, TM_U = 192, TM_KU = 320, TM_COLS = 512;
+// TMEM columns (512 allocated): the Gram accumulators use the first 64 columns
+// of the W region (read out before the W product is issued).
+constexpr uint32_t TM_GRAM = 0, TM_W = 0, TM_U = 128, TM_KU = 256, TM_S = 384, TM_COLS = 512;
 constexpr uint32_t TMA_BYTES = 6 * 8 * KB + 16 * KB;  // q, k, v: 2 boxes of 8 KB each; g: 1 box of 16 KB
-constexpr long long kWaitCycles = 2000000000LL;  // ~1 s at 2 GHz
+constexpr long long kWaitCycles = 2000000000LL;        // ~1 s at 2 GHz
+constexpr float kLog2e = 1.4426950408889634f;
 
 struct TcParams {
     PrefillArgs a;
@@ -96,39 +103,26 @@ __device__ __forceinline__ uint32_t pack_bf2(float x, float y) {
 }
 
 // ------------------------------------------------------------- MMA issue
-// A, B: K-major (kmaj) or MN-major operand tiles; see the layout notes above.
+// Operand tile in shared memory (128-byte swizzled rows): K-major tiles keep
+// 64-wide K blocks `kblk` bytes apart; MN-major tiles keep 64-wide M/N blocks
+// `lbo` bytes apart and advance 16 K-rows (2 KB) per MMA step.
 struct Opnd {
-    uint32_t base;    // shared address
-    bool mn;          // MN-major?
-    uint32_t kblk;    // K-major: byte stride between 64-wide K blocks
-    uint32_t lbo;     // MN-major: byte stride between 64-wide MN blocks
+    uint32_t base;
+    bool mn;
+    uint32_t kblk;
+    uint32_t lbo;
 };
 
-__device__ __forceinline__ uint64_t opnd_desc(const Opnd &o, int k) {
-    // k = index of the 16-wide K step
-    if (!o.mn) {
-        const uint32_t a = o.base + (uint32_t)(k >> 2) * o.kblk + (uint32_t)(k & 3) * 32u;
-        return smem_desc_sw128(a, 16u, 1024u);
-    }
-    const uint32_t a = o.base + (uint32_t)k * 2048u;  // 16 K-rows of 128 bytes
-    return smem_desc_sw128(a, o.lbo, 1024u);
-}
-
-__device__ __forceinline__ void mma_chain(uint32_t d_tmem, const Opnd &A, const Opnd &B, int N, int ksteps,
+template <int KSTEPS>
+__device__ __forceinline__ void mma_chain(uint32_t d_tmem, const Opnd &A, const Opnd &B, uint32_t idesc,
                                           bool accumulate) {
-    const uint32_t id = idesc_bf16_f32(128, N, A.mn ? 1 : 0, B.mn ? 1 : 0);
-    for (int k = 0; k < ksteps; ++k)
-        mma_bf16_ss(d_tmem, opnd_desc(A, k), opnd_desc(B, k), id, (accumulate || k > 0) ? 1u : 0u);
-}
-
-// 64 fp32 TMEM columns of this warp's 32 lanes.
-__device__ __forceinline__ void tmem_ld64(uint32_t taddr, float (&v)[64]) {
-    float t[16];
+    const uint64_t da = smem_desc_sw128(A.base, A.mn ? A.lbo : 16u, 1024u);
+    const uint64_t db = smem_desc_sw128(B.base, B.mn ? B.lbo : 16u, 1024u);
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        tmem_ld16(taddr + 16u * c, t);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) v[16 * c + i] = t[i];
+    for (int k = 0; k < KSTEPS; ++k) {
+        const uint32_t oa = A.mn ? (uint32_t)k * 2048u : (uint32_t)(k >> 2) * A.kblk + (uint32_t)(k & 3) * 32u;
+        const uint32_t ob = B.mn ? (uint32_t)k * 2048u : (uint32_t)(k >> 2) * B.kblk + (uint32_t)(k & 3) * 32u;
+        mma_bf16_ss(d_tmem, da + (oa >> 4), db + (ob >> 4), idesc, (accumulate || k > 0) ? 1u : 0u);
     }
 }
 
@@ -167,6 +161,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const __nv_bfloat16 *beta = static_cast<const __nv_bfloat16 *>(p.beta);
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
     const size_t state_base = ((size_t)n * H + h) * (size_t)(D * D);
+    const long long nchunks = (len + C - 1) / C;
 
     if (tid == 0) {
         mbar_init(bar_tma, 1);
@@ -181,51 +176,67 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tmem_alloc(s_tmem, TM_COLS);
         tmem_relinquish();
     }
+    __syncthreads();
 
-    // Incoming state: thread owns dk row i = 32*quarter + lane, dv columns 64*half .. +63.
-    const int si = 32 * quarter + lane;
-    float S[64];
-#pragma unroll
-    for (int jj = 0; jj < 64; ++jj) {
-        const int j = 64 * half + jj;
-        S[jj] = p.S0 ? p.S0[state_base + (size_t)j * D + si] : 0.f;
-    }
-    // bf16 copy: B operand, MN-major: row = dk index, 64 dv per 128-byte row, N-block = half
-    auto write_state_bf16 = [&]() {
-        uint8_t *base = sm + OFF_SB + half * 16 * KB;
-#pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
-            uint4 w;
-            w.x = pack_bf2(S[8 * cc + 0], S[8 * cc + 1]);
-            w.y = pack_bf2(S[8 * cc + 2], S[8 * cc + 3]);
-            w.z = pack_bf2(S[8 * cc + 4], S[8 * cc + 5]);
-            w.w = pack_bf2(S[8 * cc + 6], S[8 * cc + 7]);
-            *reinterpret_cast<uint4 *>(base + sw128_offset(si, 8 * cc)) = w;
-        }
+    auto issue_q = [&](long long tok) {
+        tma_load_3d(sm + OFF_WQ + 8 * KB, &tm_q, bar_tma, 0, h, (int)tok);
+        tma_load_3d(sm + OFF_WQ + 24 * KB, &tm_q, bar_tma, 64, h, (int)tok);
     };
-    write_state_bf16();
+    auto issue_k = [&](long long tok) {
+        tma_load_3d(sm + OFF_KS, &tm_k, bar_tma, 0, h, (int)tok);
+        tma_load_3d(sm + OFF_KS + 8 * KB, &tm_k, bar_tma, 64, h, (int)tok);
+    };
+    auto issue_v = [&](long long tok) {
+        tma_load_3d(sm + OFF_V, &tm_v, bar_tma, 0, h, (int)tok);
+        tma_load_3d(sm + OFF_V + 8 * KB, &tm_v, bar_tma, 64, h, (int)tok);
+    };
+    auto issue_g = [&](long long tok) { tma_load_3d(sm + OFF_G, &tm_g, bar_tma, 0, h, (int)tok); };
+    if (nchunks > 0 && tid == 0) {
+        mbar_arrive_expect_tx(bar_tma, TMA_BYTES);
+        issue_g(t_begin);
+        issue_k(t_begin);
+        issue_v(t_begin);
+        issue_q(t_begin);
+    }
+    float bnext = 0.f;  // beta of this thread's row in the next chunk (prefetched)
+    if (tid < C && tid < len) bnext = __bfloat162float(beta[(size_t)(t_begin + tid) * H + h]);
+
+    // Incoming state -> TMEM (fp32, lane = dk row, column = dv) and its bf16 copy
+    // (B operand, MN-major: row = dk index, 64 dv per 128-byte row, N-block = half).
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t tlane = (uint32_t)(32 * quarter) << 16;
+    const int si = 32 * quarter + lane;
+    {
+        uint8_t *sb = sm + OFF_SB + half * 16 * KB;
+#pragma unroll
+        for (int gq = 0; gq < 4; ++gq) {
+            float v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int j = 64 * half + 16 * gq + e;
+                v[e] = p.S0 ? p.S0[state_base + (size_t)j * D + si] : 0.f;
+            }
+            tmem_st16(tmem + tlane + TM_S + 64u * half + 16u * gq, v);
+#pragma unroll
+            for (int cc = 0; cc < 2; ++cc) {
+                uint4 w;
+                w.x = pack_bf2(v[8 * cc + 0], v[8 * cc + 1]);
+                w.y = pack_bf2(v[8 * cc + 2], v[8 * cc + 3]);
+                w.z = pack_bf2(v[8 * cc + 4], v[8 * cc + 5]);
+                w.w = pack_bf2(v[8 * cc + 6], v[8 * cc + 7]);
+                *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq + 8 * cc)) = w;
+            }
+        }
+        tmem_wait_st();
+    }
     fence_proxy_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *s_tmem;
-    const uint32_t tlane = (uint32_t)(32 * quarter) << 16;
 
-    const long long nchunks = (len + C - 1) / C;
     uint32_t tma_phase = 0, mma_phase = 0;
-    bool aborted = false;
-
-    auto issue_qk = [&](long long tok) {
-        tma_load_3d(sm + OFF_WQ + 8 * KB, &tm_q, bar_tma, 0, h, (int)tok);
-        tma_load_3d(sm + OFF_WQ + 24 * KB, &tm_q, bar_tma, 64, h, (int)tok);
-        tma_load_3d(sm + OFF_KH, &tm_k, bar_tma, 0, h, (int)tok);
-        tma_load_3d(sm + OFF_KH + 8 * KB, &tm_k, bar_tma, 64, h, (int)tok);
-    };
-    auto issue_vg = [&](long long tok) {
-        tma_load_3d(sm + OFF_V, &tm_v, bar_tma, 0, h, (int)tok);
-        tma_load_3d(sm + OFF_V + 8 * KB, &tm_v, bar_tma, 64, h, (int)tok);
-        tma_load_3d(sm + OFF_G, &tm_g, bar_tma, 0, h, (int)tok);
-    };
+    bool aborted = false, tma_pending = nchunks > 0;
     // wait for an MMA commit; every thread takes part
     auto wait_mma = [&]() -> bool {
         const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
@@ -234,24 +245,21 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         return __syncthreads_or(!ok) == 0;
     };
 
-    if (nchunks > 0 && tid == 0) {
-        mbar_arrive_expect_tx(bar_tma, TMA_BYTES);
-        issue_vg(t_begin);
-        issue_qk(t_begin);
-    }
-    bool tma_pending = nchunks > 0;
-
-    // thread roles for the token-parallel passes: subtile i, channel pair cp
+    // thread roles for the token-parallel passes: subtile ti, channel pair cp
     const int ti = tid >> 6;          // subtile 0..3
     const int cp = tid & 63;          // channel pair
     const int c0 = 2 * cp;            // first channel
     const int cblk = c0 >> 6;         // 64-wide block of the channel
     const int cin = c0 & 63;          // channel inside the block
-    float gl[SUB][2];                 // in-subtile inclusive cumulative log-decay
+    constexpr uint32_t idG = idesc_bf16_f32(128, 16, 0, 0);     // Gram: K-major x K-major, N = 16
+    constexpr uint32_t idKM = idesc_bf16_f32(128, 128, 0, 1);   // K-major A, MN-major B, N = 128
+    constexpr uint32_t idMM = idesc_bf16_f32(128, 128, 1, 1);   // MN-major A and B, N = 128
 
     for (long long ch = 0; ch < nchunks; ++ch) {
         const long long tok0 = t_begin + ch * C;
         const int Lc = (int)((len - ch * C) < C ? (len - ch * C) : C);
+        const bool more = ch + 1 < nchunks;
+        const long long tokn = tok0 + C;
 
         // ---- wait for this chunk's tiles
         {
@@ -260,28 +268,32 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tma_pending = false;
             if (__syncthreads_or(!ok)) { aborted = true; break; }
         }
-        if (tid < C) sBeta[tid] = (tid < Lc) ? __bfloat162float(beta[(size_t)(tok0 + tid) * H + h]) : 0.f;
+        if (tid < C) {
+            sBeta[tid] = (tid < Lc) ? bnext : 0.f;
+            if (more && tid < len - (ch + 1) * C) bnext = __bfloat162float(beta[(size_t)(tokn + tid) * H + h]);
+        }
         if (Lc < C) {  // zero the rows past the end of the sequence
             for (int idx = tid; idx < (C - Lc) * 16; idx += NT) {
                 const int r = Lc + idx / 16, q16 = idx % 16;  // 16-byte piece of a 256-byte row
                 const uint4 z = make_uint4(0, 0, 0, 0);
                 const int blk = q16 >> 3, pc = (q16 & 7) * 8;
                 *reinterpret_cast<uint4 *>(sm + OFF_WQ + blk * 16 * KB + sw128_offset(64 + r, pc)) = z;
-                *reinterpret_cast<uint4 *>(sm + OFF_KH + blk * 8 * KB + sw128_offset(r, pc)) = z;
+                *reinterpret_cast<uint4 *>(sm + OFF_KS + blk * 8 * KB + sw128_offset(r, pc)) = z;
                 *reinterpret_cast<uint4 *>(sm + OFF_V + blk * 8 * KB + sw128_offset(r, pc)) = z;
                 *reinterpret_cast<uint4 *>(sm + OFF_G + r * 256 + q16 * 16) = z;
             }
         }
         __syncthreads();
 
-        // ---- phase 1a: cumulative log-decay inside subtile ti for channels c0, c0+1
+        // ---- phase 1a: cumulative log2-decay inside subtile ti for channels c0, c0+1
+        float gl[SUB][2];
         {
             float a0 = 0.f, a1 = 0.f;
 #pragma unroll
             for (int rr = 0; rr < SUB; ++rr) {
                 const float2 gv = ld_bf2(sm + OFF_G + (SUB * ti + rr) * 256 + c0 * 2);
-                a0 += gv.x;
-                a1 += gv.y;
+                a0 = fmaf(gv.x, kLog2e, a0);
+                a1 = fmaf(gv.y, kLog2e, a1);
                 gl[rr][0] = a0;
                 gl[rr][1] = a1;
             }
@@ -289,30 +301,38 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             sD[ti * D + c0 + 1] = a1;
         }
         __syncthreads();
+        if (more && tid == 0) {  // g tile consumed: start the next chunk's loads
+            mbar_arrive_expect_tx(bar_tma, TMA_BYTES);
+            issue_g(tokn);
+        }
 
-        // ---- phase 1b: Gram operands and Gamma * q
-        float Dm[NSUB][2], ed[NSUB][2];
-#pragma unroll
-        for (int m = 0; m < NSUB; ++m)
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                Dm[m][e] = sD[m * D + c0 + e];
-                ed[m][e] = __expf(Dm[m][e]);
-            }
-        float pg[2];  // exp(G at the start of subtile ti) relative to the chunk start
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-            float acc = 1.f;
+        // ---- phase 1b: Gram operands and Gamma * q; keep the exp factors for phase 3
+        float F[SUB][2], Rf[SUB][2];
+        float ed[NSUB][2], pg[2], post[2];
+        {
+            float Dm[NSUB][2];
 #pragma unroll
             for (int m = 0; m < NSUB; ++m)
-                if (m < ti) acc *= ed[m][e];
-            pg[e] = acc;
-        }
-        if (ti == 0) {
 #pragma unroll
-            for (int e = 0; e < 2; ++e) sGamC[c0 + e] = ed[0][e] * ed[1][e] * ed[2][e] * ed[3][e];
-        }
-        {
+                for (int e = 0; e < 2; ++e) {
+                    Dm[m][e] = sD[m * D + c0 + e];
+                    ed[m][e] = ex2(Dm[m][e]);
+                }
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+                float a = 1.f, b = 1.f;
+#pragma unroll
+                for (int m = 0; m < NSUB; ++m) {
+                    if (m < ti) a *= ed[m][e];
+                    if (m > ti) b *= ed[m][e];
+                }
+                pg[e] = a;     // Gamma at the start of subtile ti (relative to the chunk start)
+                post[e] = b;   // decay from the end of subtile ti to the end of the chunk
+            }
+            if (ti == 0) {
+#pragma unroll
+                for (int e = 0; e < 2; ++e) sGamC[c0 + e] = ed[0][e] * ed[1][e] * ed[2][e] * ed[3][e];
+            }
             float E[NSUB][2];  // E[j] = exp(G_start(ti) - G_end(j)) for j < ti, exp(-D_ti) for j = ti
 #pragma unroll
             for (int j = 0; j < NSUB; ++j)
@@ -322,30 +342,40 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
                     for (int m = 0; m < NSUB; ++m)
                         if (m > j && m < ti) acc *= ed[m][e];
-                    E[j][e] = (j == ti) ? __expf(-Dm[ti][e]) : acc;
+                    E[j][e] = (j == ti) ? ex2(-Dm[ti][e]) : acc;
                 }
-#pragma unroll 4
+            float dti[2];
+#pragma unroll
+            for (int e = 0; e < 2; ++e) dti[e] = (ti == 0) ? Dm[0][e] : (ti == 1) ? Dm[1][e] : (ti == 2) ? Dm[2][e] : Dm[3][e];
+#pragma unroll
+            for (int rr = 0; rr < SUB; ++rr)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    F[rr][e] = ex2(gl[rr][e]);
+                    Rf[rr][e] = ex2(dti[e] - gl[rr][e]);
+                }
+            uint8_t *const qrow = sm + OFF_WQ + cblk * 16 * KB;
+            uint8_t *const krow = sm + OFF_KS + cblk * 8 * KB;
+            uint8_t *const rrow = sm + OFF_R + cblk * 8 * KB;
+#pragma unroll
             for (int rr = 0; rr < SUB; ++rr) {
                 const int r = SUB * ti + rr;
-                const uint32_t qoff = OFF_WQ + cblk * 16 * KB + sw128_offset(64 + r, cin);
-                const uint32_t koff = OFF_KH + cblk * 8 * KB + sw128_offset(r, cin);
-                const float2 kx = ld_bf2(sm + koff);
-                const float2 qx = ld_bf2(sm + qoff);
-                const float F0 = __expf(gl[rr][0]), F1 = __expf(gl[rr][1]);
-                const float R0 = __expf(Dm[ti][0] - gl[rr][0]), R1 = __expf(Dm[ti][1] - gl[rr][1]);
-                // right operand row r (column block ti)
-                st_bf2(sm + OFF_R + cblk * 8 * KB + sw128_offset(r, cin), kx.x * R0, kx.y * R1);
-                const float kf0 = kx.x * F0, kf1 = kx.y * F1, qf0 = qx.x * F0, qf1 = qx.y * F1;
+                const uint32_t off_r = sw128_offset(r, cin);       // (r & 7) == (rr & 7)
+                const uint32_t off_q = sw128_offset(64 + r, cin);
+                const float2 kx = ld_bf2(krow + off_r);
+                const float2 qx = ld_bf2(qrow + off_q);
+                st_bf2(rrow + off_r, kx.x * Rf[rr][0], kx.y * Rf[rr][1]);
+                const float kf0 = kx.x * F[rr][0], kf1 = kx.y * F[rr][1];
+                const float qf0 = qx.x * F[rr][0], qf1 = qx.y * F[rr][1];
 #pragma unroll
                 for (int j = 0; j < NSUB; ++j) {
                     if (j > ti) continue;
-                    const uint32_t rows = l_rows(j), half_rows = rows / 2;
+                    const uint32_t rows = l_rows(j), hr = rows / 2;
                     uint8_t *Lb = sm + OFF_L + l_off(j) + cblk * rows * 128;
                     st_bf2(Lb + sw128_offset(r - 16 * j, cin), kf0 * E[j][0], kf1 * E[j][1]);
-                    st_bf2(Lb + sw128_offset(half_rows + r - 16 * j, cin), qf0 * E[j][0], qf1 * E[j][1]);
+                    st_bf2(Lb + sw128_offset(hr + r - 16 * j, cin), qf0 * E[j][0], qf1 * E[j][1]);
                 }
-                // Gamma * q in place (rows 64..127 of the [-W ; Qt] operand)
-                st_bf2(sm + qoff, qf0 * pg[0], qf1 * pg[1]);
+                st_bf2(qrow + off_q, qf0 * pg[0], qf1 * pg[1]);  // Gamma * q in place
             }
         }
         fence_proxy_async_smem();
@@ -358,7 +388,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             for (int j = 0; j < NSUB; ++j) {
                 Opnd A{sbase + OFF_L + l_off(j), false, l_rows(j) * 128u, 0};
                 Opnd B{sbase + OFF_R + 16u * j * 128u, false, 8 * KB, 0};
-                mma_chain(tmem + TM_GRAM + 16u * j, A, B, 16, D / 16, false);
+                mma_chain<D / 16>(tmem + TM_GRAM + 16u * j, A, B, idG, false);
             }
             mma_commit(bar_mma);
         }
@@ -391,7 +421,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         st_bf2(prow + sw128_offset(r, s), (s <= r) ? v[s2] : 0.f, (s + 1 <= r) ? v[s2 + 1] : 0.f);
                     }
                     if (r < 16 * (j + 1)) {  // diagonal block: zero the blocks to its right
-                        for (int s = 16 * (j + 1); s < C; s += 2) st_bf2(prow + sw128_offset(r, s), 0.f, 0.f);
+                        for (int s = 16 * (j + 1); s < C; s += 8)
+                            *reinterpret_cast<uint4 *>(prow + sw128_offset(r, s)) = make_uint4(0, 0, 0, 0);
                     }
                 }
             }
@@ -399,43 +430,55 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tc_fence_before();
         __syncthreads();
 
-        // ---- phase 3: T = (I + A)^{-1}, lower unit triangular, by 16 x 16 blocks
-        if (tid < 64) {  // diagonal blocks: forward substitution, one column per thread
+        // ---- phase 3: T = (I + A)^{-1} (unit lower triangular) by 16 x 16 blocks
+        if (tid < 64) {  // diagonal blocks: forward substitution, one column per thread, in registers
             const int bi = tid >> 4, cc = tid & 15, o0 = 16 * bi;
             float x[16];
 #pragma unroll
             for (int rr = 0; rr < 16; ++rr) {
                 float acc = (rr == cc) ? 1.f : 0.f;
-                if (rr > cc) {
 #pragma unroll
-                    for (int ss = 0; ss < 16; ++ss)
-                        if (ss >= cc && ss < rr) acc = fmaf(-AF[(o0 + rr) * 65 + o0 + ss], x[ss], acc);
-                }
-                x[rr] = acc;
-                TF[(o0 + rr) * 65 + o0 + cc] = acc;
+                for (int ss = 0; ss < rr; ++ss) acc = fmaf(-AF[(o0 + rr) * 65 + o0 + ss], x[ss], acc);
+                x[rr] = acc;  // zero above the diagonal since x[ss < cc] = 0
+                TF[(o0 + rr) * 68 + o0 + cc] = acc;
             }
         }
         __syncthreads();
+        // off-diagonal blocks by distance: X = sum_{m=j}^{i-1} A_im T_mj, then T_ij = -T_ii X
+#pragma unroll
         for (int dist = 1; dist < NSUB; ++dist) {
             const int nblk = NSUB - dist;
-            // X = sum_{m=j}^{i-1} A_im T_mj  for blocks (i, j = i - dist)
-            for (int idx = tid; idx < nblk * 256; idx += NT) {
-                const int b = idx >> 8, rr = (idx >> 4) & 15, cc = idx & 15;
-                const int bi = dist + b, bj = b;
-                float acc = 0.f;
-                for (int kk = 16 * bj + cc; kk < 16 * bi; ++kk)
-                    acc = fmaf(AF[(16 * bi + rr) * 65 + kk], TF[kk * 65 + 16 * bj + cc], acc);
-                XS[b * 272 + rr * 17 + cc] = acc;
+            const int b = tid >> 6, r = (tid & 63) >> 2, q0 = (tid & 3) * 4;
+            const int bi = dist + b, bj = b;
+            if (b < nblk) {
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int m = bj; m < bi; ++m) {
+#pragma unroll
+                    for (int kk = 0; kk < 16; ++kk) {
+                        const float a = AF[(16 * bi + r) * 65 + 16 * m + kk];
+                        const float4 t = *reinterpret_cast<const float4 *>(TF + (16 * m + kk) * 68 + 16 * bj + q0);
+                        acc.x = fmaf(a, t.x, acc.x);
+                        acc.y = fmaf(a, t.y, acc.y);
+                        acc.z = fmaf(a, t.z, acc.z);
+                        acc.w = fmaf(a, t.w, acc.w);
+                    }
+                }
+                *reinterpret_cast<float4 *>(XS + b * 320 + r * 20 + q0) = acc;
             }
             __syncthreads();
-            // T_ij = -T_ii X
-            for (int idx = tid; idx < nblk * 256; idx += NT) {
-                const int b = idx >> 8, rr = (idx >> 4) & 15, cc = idx & 15;
-                const int bi = dist + b, bj = b;
-                float acc = 0.f;
-                for (int kk = 0; kk <= rr; ++kk)
-                    acc = fmaf(TF[(16 * bi + rr) * 65 + 16 * bi + kk], XS[b * 272 + kk * 17 + cc], acc);
-                TF[(16 * bi + rr) * 65 + 16 * bj + cc] = -acc;
+            if (b < nblk) {
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                for (int kk = 0; kk < 16; ++kk) {
+                    const float a = TF[(16 * bi + r) * 68 + 16 * bi + kk];
+                    const float4 t = *reinterpret_cast<const float4 *>(XS + b * 320 + kk * 20 + q0);
+                    acc.x = fmaf(a, t.x, acc.x);
+                    acc.y = fmaf(a, t.y, acc.y);
+                    acc.z = fmaf(a, t.z, acc.z);
+                    acc.w = fmaf(a, t.w, acc.w);
+                }
+                *reinterpret_cast<float4 *>(TF + (16 * bi + r) * 68 + 16 * bj + q0) =
+                    make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
             }
             __syncthreads();
         }
@@ -444,42 +487,30 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const int r = idx >> 3, pc = (idx & 7) * 8;
             uint4 w = make_uint4(0, 0, 0, 0);
             if (r < C) {
-                float t[8];
+                const float4 t0 = *reinterpret_cast<const float4 *>(TF + r * 68 + pc);
+                const float4 t1 = *reinterpret_cast<const float4 *>(TF + r * 68 + pc + 4);
+                const float t[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+                float u[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int s = pc + e;
-                    t[e] = (s <= r) ? TF[r * 65 + s] * sBeta[s] : 0.f;
-                }
-                w.x = pack_bf2(t[0], t[1]);
-                w.y = pack_bf2(t[2], t[3]);
-                w.z = pack_bf2(t[4], t[5]);
-                w.w = pack_bf2(t[6], t[7]);
+                for (int e = 0; e < 8; ++e) u[e] = (pc + e <= r) ? t[e] * sBeta[pc + e] : 0.f;
+                w.x = pack_bf2(u[0], u[1]);
+                w.y = pack_bf2(u[2], u[3]);
+                w.z = pack_bf2(u[4], u[5]);
+                w.w = pack_bf2(u[6], u[7]);
             }
             *reinterpret_cast<uint4 *>(sm + OFF_TB + sw128_offset(r, pc)) = w;
         }
-        // Gamma * k -> KT, and Kh = exp(G_C - G_s) * k_s in place of k
+        // Gamma * k -> KT and Kh = exp(G_C - G_s) * k_s -> KHAT (A is dead now)
         {
-            float sumD[2];
+            const uint8_t *krow = sm + OFF_KS + cblk * 8 * KB;
+            uint8_t *ktrow = sm + OFF_KT + cblk * 8 * KB;
+            uint8_t *khrow = sm + OFF_KHAT + cblk * 8 * KB;
 #pragma unroll
-            for (int e = 0; e < 2; ++e) sumD[e] = Dm[0][e] + Dm[1][e] + Dm[2][e] + Dm[3][e];
-            float Gs[2];
-#pragma unroll
-            for (int e = 0; e < 2; ++e) {
-                float acc = 0.f;
-#pragma unroll
-                for (int m = 0; m < NSUB; ++m)
-                    if (m < ti) acc += Dm[m][e];
-                Gs[e] = acc;
-            }
-#pragma unroll 4
             for (int rr = 0; rr < SUB; ++rr) {
-                const int r = SUB * ti + rr;
-                const uint32_t koff = OFF_KH + cblk * 8 * KB + sw128_offset(r, cin);
-                const float2 kx = ld_bf2(sm + koff);
-                const float F0 = __expf(gl[rr][0]), F1 = __expf(gl[rr][1]);
-                st_bf2(sm + OFF_KT + cblk * 8 * KB + sw128_offset(r, cin), kx.x * F0 * pg[0], kx.y * F1 * pg[1]);
-                const float h0 = __expf(sumD[0] - Gs[0] - gl[rr][0]), h1 = __expf(sumD[1] - Gs[1] - gl[rr][1]);
-                st_bf2(sm + koff, kx.x * h0, kx.y * h1);
+                const uint32_t off_r = sw128_offset(SUB * ti + rr, cin);
+                const float2 kx = ld_bf2(krow + off_r);
+                st_bf2(ktrow + off_r, kx.x * F[rr][0] * pg[0], kx.y * F[rr][1] * pg[1]);
+                st_bf2(khrow + off_r, kx.x * Rf[rr][0] * post[0], kx.y * Rf[rr][1] * post[1]);
             }
         }
         fence_proxy_async_smem();
@@ -487,37 +518,37 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
         // ---- [W | Ut] = T Diag(beta) [Gamma*K | V]
         if (tid == 0) {
+            if (more) issue_k(tokn);  // the k tile is consumed
             tc_fence_after();
             Opnd A{sbase + OFF_TB, false, 16 * KB, 0};
             Opnd BK{sbase + OFF_KT, true, 0, 8 * KB};
             Opnd BV{sbase + OFF_V, true, 0, 8 * KB};
-            mma_chain(tmem + TM_W, A, BK, 128, C / 16, false);
-            mma_chain(tmem + TM_U, A, BV, 128, C / 16, false);
+            mma_chain<C / 16>(tmem + TM_W, A, BK, idKM, false);
+            mma_chain<C / 16>(tmem + TM_U, A, BV, idKM, false);
             mma_commit(bar_mma);
         }
         if (!wait_mma()) { aborted = true; break; }
-        const bool more = ch + 1 < nchunks;
-        if (more && tid == 0) {  // v, g tiles are free: start the next chunk's loads
-            mbar_arrive_expect_tx(bar_tma, TMA_BYTES);
-            issue_vg(tok0 + C);
-        }
+        if (more && tid == 0) issue_v(tokn);
         tma_pending = more;
 
         // ---- phase 4: -W (rows 0..63) into the [-W ; Qt] operand
         if (quarter < 2) {
-            float v[64];
-            tmem_ld64(tmem + tlane + TM_W + 64u * half, v);
-            tmem_wait_ld();
             const int r = 32 * quarter + lane;
             uint8_t *base = sm + OFF_WQ + half * 16 * KB;
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                uint4 w;
-                w.x = pack_bf2(-v[8 * cc + 0], -v[8 * cc + 1]);
-                w.y = pack_bf2(-v[8 * cc + 2], -v[8 * cc + 3]);
-                w.z = pack_bf2(-v[8 * cc + 4], -v[8 * cc + 5]);
-                w.w = pack_bf2(-v[8 * cc + 6], -v[8 * cc + 7]);
-                *reinterpret_cast<uint4 *>(base + sw128_offset(r, 8 * cc)) = w;
+            for (int gq = 0; gq < 4; ++gq) {
+                float v[16];
+                tmem_ld16(tmem + tlane + TM_W + 64u * half + 16u * gq, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint4 w;
+                    w.x = pack_bf2(-v[8 * cc + 0], -v[8 * cc + 1]);
+                    w.y = pack_bf2(-v[8 * cc + 2], -v[8 * cc + 3]);
+                    w.z = pack_bf2(-v[8 * cc + 4], -v[8 * cc + 5]);
+                    w.w = pack_bf2(-v[8 * cc + 6], -v[8 * cc + 7]);
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, 16 * gq + 8 * cc)) = w;
+                }
             }
         }
         fence_proxy_async_smem();
@@ -529,26 +560,30 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_fence_after();
             Opnd A{sbase + OFF_WQ, false, 16 * KB, 0};
             Opnd B{sbase + OFF_SB, true, 0, 16 * KB};
-            mma_chain(tmem + TM_U, A, B, 128, D / 16, true);
+            mma_chain<D / 16>(tmem + TM_U, A, B, idKM, true);
             mma_commit(bar_mma);
         }
         if (!wait_mma()) { aborted = true; break; }
+        if (more && tid == 0) issue_q(tokn);  // rows 64..127 of the [-W ; Qt] operand are free
 
         // ---- phase 5: U (rows 0..63) -> bf16 B operand, MN-major [tok][dv]
         if (quarter < 2) {
-            float v[64];
-            tmem_ld64(tmem + tlane + TM_U + 64u * half, v);
-            tmem_wait_ld();
             const int r = 32 * quarter + lane;
             uint8_t *base = sm + OFF_R + half * 8 * KB;
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                uint4 w;
-                w.x = pack_bf2(v[8 * cc + 0], v[8 * cc + 1]);
-                w.y = pack_bf2(v[8 * cc + 2], v[8 * cc + 3]);
-                w.z = pack_bf2(v[8 * cc + 4], v[8 * cc + 5]);
-                w.w = pack_bf2(v[8 * cc + 6], v[8 * cc + 7]);
-                *reinterpret_cast<uint4 *>(base + sw128_offset(r, 8 * cc)) = w;
+            for (int gq = 0; gq < 4; ++gq) {
+                float v[16];
+                tmem_ld16(tmem + tlane + TM_U + 64u * half + 16u * gq, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint4 w;
+                    w.x = pack_bf2(v[8 * cc + 0], v[8 * cc + 1]);
+                    w.y = pack_bf2(v[8 * cc + 2], v[8 * cc + 3]);
+                    w.z = pack_bf2(v[8 * cc + 4], v[8 * cc + 5]);
+                    w.w = pack_bf2(v[8 * cc + 6], v[8 * cc + 7]);
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, 16 * gq + 8 * cc)) = w;
+                }
             }
         }
         fence_proxy_async_smem();
@@ -560,41 +595,59 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_fence_after();
             Opnd AP{sbase + OFF_PB - 8 * KB, false, 16 * KB, 0};
             Opnd BU{sbase + OFF_R, true, 0, 8 * KB};
-            Opnd AK{sbase + OFF_KH, true, 0, 8 * KB};
-            mma_chain(tmem + TM_U, AP, BU, 128, C / 16, true);
-            mma_chain(tmem + TM_KU, AK, BU, 128, C / 16, false);
+            Opnd AK{sbase + OFF_KHAT, true, 0, 8 * KB};
+            mma_chain<C / 16>(tmem + TM_KU, AK, BU, idMM, false);
+            mma_chain<C / 16>(tmem + TM_U, AP, BU, idKM, true);
             mma_commit(bar_mma);
         }
         if (!wait_mma()) { aborted = true; break; }
-        if (more && tid == 0) issue_qk(tok0 + C);
 
-        // ---- phase 6: outputs and the state update
+        // ---- phase 6: outputs and the state update S <- Diag(Gamma_C) S + dS
         if (quarter >= 2) {
-            float v[64];
-            tmem_ld64(tmem + tlane + TM_U + 64u * half, v);
-            tmem_wait_ld();
             const int r = 32 * quarter + lane - 64;
-            if (r < Lc) {
-                uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(tok0 + r) * H + h) * D + 64 * half);
+            uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(tok0 + r) * H + h) * D + 64 * half);
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc) {
-                    uint4 w;
-                    w.x = pack_bf2(v[8 * cc + 0], v[8 * cc + 1]);
-                    w.y = pack_bf2(v[8 * cc + 2], v[8 * cc + 3]);
-                    w.z = pack_bf2(v[8 * cc + 4], v[8 * cc + 5]);
-                    w.w = pack_bf2(v[8 * cc + 6], v[8 * cc + 7]);
-                    dst[cc] = w;
+            for (int gq = 0; gq < 4; ++gq) {
+                float v[16];
+                tmem_ld16(tmem + tlane + TM_U + 64u * half + 16u * gq, v);
+                tmem_wait_ld();
+                if (r < Lc) {
+#pragma unroll
+                    for (int cc = 0; cc < 2; ++cc) {
+                        uint4 w;
+                        w.x = pack_bf2(v[8 * cc + 0], v[8 * cc + 1]);
+                        w.y = pack_bf2(v[8 * cc + 2], v[8 * cc + 3]);
+                        w.z = pack_bf2(v[8 * cc + 4], v[8 * cc + 5]);
+                        w.w = pack_bf2(v[8 * cc + 6], v[8 * cc + 7]);
+                        dst[2 * gq + cc] = w;
+                    }
                 }
             }
         }
         {
-            float v[64];
-            tmem_ld64(tmem + tlane + TM_KU + 64u * half, v);
-            tmem_wait_ld();
             const float gam = sGamC[si];
+            uint8_t *sb = sm + OFF_SB + half * 16 * KB;
 #pragma unroll
-            for (int jj = 0; jj < 64; ++jj) S[jj] = fmaf(gam, S[jj], v[jj]);
-            write_state_bf16();
+            for (int gq = 0; gq < 4; ++gq) {
+                float sv[16], dv[16];
+                const uint32_t col = 64u * half + 16u * gq;
+                tmem_ld16(tmem + tlane + TM_S + col, sv);
+                tmem_ld16(tmem + tlane + TM_KU + col, dv);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) sv[e] = fmaf(gam, sv[e], dv[e]);
+                tmem_st16(tmem + tlane + TM_S + col, sv);
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    uint4 w;
+                    w.x = pack_bf2(sv[8 * cc + 0], sv[8 * cc + 1]);
+                    w.y = pack_bf2(sv[8 * cc + 2], sv[8 * cc + 3]);
+                    w.z = pack_bf2(sv[8 * cc + 4], sv[8 * cc + 5]);
+                    w.w = pack_bf2(sv[8 * cc + 6], sv[8 * cc + 7]);
+                    *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq + 8 * cc)) = w;
+                }
+            }
+            tmem_wait_st();
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -605,10 +658,17 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (tid == 0 && p.dev_status) atomicExch(p.dev_status, (int)KDA_ERR_TIMEOUT);
         if (tma_pending && tid == 0) mbar_wait_bounded(bar_tma, tma_phase, kWaitCycles);
     } else if (p.ST) {
+        tc_fence_after();
 #pragma unroll
-        for (int jj = 0; jj < 64; ++jj) {
-            const int j = 64 * half + jj;
-            p.ST[state_base + (size_t)j * D + si] = S[jj];
+        for (int gq = 0; gq < 4; ++gq) {
+            float sv[16];
+            tmem_ld16(tmem + tlane + TM_S + 64u * half + 16u * gq, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int j = 64 * half + 16 * gq + e;
+                p.ST[state_base + (size_t)j * D + si] = sv[e];
+            }
         }
     }
     tc_fence_before();
