@@ -67,12 +67,12 @@ constexpr uint32_t OFF_KT = OFF_L + 16 * KB;       // 16 KB  B operand Gamma*K, 
 constexpr uint32_t OFF_AF = OFF_L + 32 * KB;       // 64 x 65 fp32  A (dead once T is known)
 constexpr uint32_t OFF_KHAT = OFF_L + 32 * KB;     // 16 KB  A operand Kh, MN-major [tok][dk] (written after A is dead)
 constexpr uint32_t OFF_TF = OFF_L + 49 * KB;       // 64 x 68 fp32  T
-constexpr uint32_t OFF_XS = OFF_TF + 64 * 68 * 4;  // 3 x 16 x 20 fp32 scratch
+constexpr uint32_t OFF_XS = OFF_TF + 64 * 68 * 4;  // 32 x 36 fp32 scratch
 static_assert(OFF_AF + 64 * 65 * 4 <= OFF_TF, "A overlaps T");
-static_assert(OFF_XS + 3 * 16 * 20 * 4 <= OFF_MISC, "scratch overflows the L region");
+static_assert(OFF_XS + 32 * 36 * 4 <= OFF_MISC, "scratch overflows the L region");
 // misc
-constexpr uint32_t OFF_BAR = OFF_MISC;              // 2 mbarriers
-constexpr uint32_t OFF_TMEMADDR = OFF_MISC + 16;
+constexpr uint32_t OFF_BAR = OFF_MISC;              // 3 mbarriers
+constexpr uint32_t OFF_TMEMADDR = OFF_MISC + 32;
 constexpr uint32_t OFF_BETA = OFF_MISC + 64;        // 64 fp32
 constexpr uint32_t OFF_DSUM = OFF_BETA + 256;       // 4 x 128 fp32 subtile totals of g (log2 units)
 constexpr uint32_t OFF_GAMC = OFF_DSUM + 2048;      // 128 fp32 Gamma_C
@@ -126,6 +126,70 @@ __device__ __forceinline__ void mma_chain(uint32_t d_tmem, const Opnd &A, const 
     }
 }
 
+
+// Off-diagonal part of T = (I + A)^{-1} (64 x 64 unit lower triangular) once the
+// four 16 x 16 diagonal blocks T_ii are in place (zero above their diagonal):
+//   level 1:  T_10 = -T_11 A_10 T_00,  T_32 = -T_33 A_32 T_22            (16 x 16)
+//   level 2:  T[32:64, 0:32] = -T[32:64, 32:64] A[32:64, 0:32] T[0:32, 0:32] (32 x 32)
+// i.e. the 2 x 2 block inverse applied twice. Each product is spread over all
+// 256 threads with 2 (level 1) or 4 (level 2) outputs per thread.
+// A: 64 x 65 fp32 (strictly lower), T: 64 x 68 fp32, XS: scratch of 32 x 36 fp32.
+__device__ __forceinline__ void tri_inverse_offdiag(const float *AF, float *TF, float *XS, int tid) {
+    {   // level 1, X = A_ij T_jj for (i, j) = (1, 0), (3, 2); 2 blocks x 16 x 16 outputs
+        const int b = tid >> 7, r = (tid & 127) >> 3, c = (tid & 7) * 2;
+        const int i = 2 * b + 1, j = 2 * b;
+        float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float a = AF[(16 * i + r) * 65 + 16 * j + k];
+            const float2 t = *reinterpret_cast<const float2 *>(TF + (16 * j + k) * 68 + 16 * j + c);
+            x0 = fmaf(a, t.x, x0);
+            x1 = fmaf(a, t.y, x1);
+        }
+        *reinterpret_cast<float2 *>(XS + b * 16 * 18 + r * 18 + c) = make_float2(x0, x1);
+        __syncthreads();
+        // T_ij = -T_ii X
+        float y0 = 0.f, y1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float a = TF[(16 * i + r) * 68 + 16 * i + k];
+            const float2 x = *reinterpret_cast<const float2 *>(XS + b * 16 * 18 + k * 18 + c);
+            y0 = fmaf(a, x.x, y0);
+            y1 = fmaf(a, x.y, y1);
+        }
+        *reinterpret_cast<float2 *>(TF + (16 * i + r) * 68 + 16 * j + c) = make_float2(-y0, -y1);
+        __syncthreads();
+    }
+    {   // level 2, X = A[32:64, 0:32] T[0:32, 0:32]; 32 x 32 outputs, 4 per thread
+        const int r = tid >> 3, c = (tid & 7) * 4;
+        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const float a = AF[(32 + r) * 65 + k];
+            const float4 t = *reinterpret_cast<const float4 *>(TF + k * 68 + c);
+            x.x = fmaf(a, t.x, x.x);
+            x.y = fmaf(a, t.y, x.y);
+            x.z = fmaf(a, t.z, x.z);
+            x.w = fmaf(a, t.w, x.w);
+        }
+        *reinterpret_cast<float4 *>(XS + r * 36 + c) = x;
+        __syncthreads();
+        // T[32:64, 0:32] = -T[32:64, 32:64] X
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const float a = TF[(32 + r) * 68 + 32 + k];
+            const float4 t = *reinterpret_cast<const float4 *>(XS + k * 36 + c);
+            y.x = fmaf(a, t.x, y.x);
+            y.y = fmaf(a, t.y, y.y);
+            y.z = fmaf(a, t.z, y.z);
+            y.w = fmaf(a, t.w, y.w);
+        }
+        *reinterpret_cast<float4 *>(TF + (32 + r) * 68 + c) = make_float4(-y.x, -y.y, -y.z, -y.w);
+        __syncthreads();
+    }
+}
+
 __global__ void __launch_bounds__(NT, 1)
 kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -137,6 +201,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t sbase = smem_u32(sm);
     uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint64_t *bar_mma = bar_tma + 1;
+    uint64_t *bar_gram = bar_tma + 2;  // 4 arrivals: one commit per Gram column block
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + OFF_TMEMADDR);
     float *sBeta = reinterpret_cast<float *>(sm + OFF_BETA);
     float *sD = reinterpret_cast<float *>(sm + OFF_DSUM);
@@ -166,6 +231,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (tid == 0) {
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
+        mbar_init(bar_gram, NSUB);
         fence_mbar_init();
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
@@ -198,8 +264,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         issue_v(t_begin);
         issue_q(t_begin);
     }
-    float bnext = 0.f;  // beta of this thread's row in the next chunk (prefetched)
-    if (tid < C && tid < len) bnext = __bfloat162float(beta[(size_t)(t_begin + tid) * H + h]);
+    // beta of this thread's row in the next chunk, prefetched as raw bf16 (converted when used)
+    __nv_bfloat16 bnext = __float2bfloat16(0.f);
+    if (tid < C && tid < len) bnext = beta[(size_t)(t_begin + tid) * H + h];
 
     // Incoming state -> TMEM (fp32, lane = dk row, column = dv) and its bf16 copy
     // (B operand, MN-major: row = dk index, 64 dv per 128-byte row, N-block = half).
@@ -235,7 +302,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __syncthreads();
     tc_fence_after();
 
-    uint32_t tma_phase = 0, mma_phase = 0;
+    uint32_t tma_phase = 0, mma_phase = 0, gram_phase = 0;
     bool aborted = false, tma_pending = nchunks > 0;
     // wait for an MMA commit; every thread takes part
     auto wait_mma = [&]() -> bool {
@@ -245,12 +312,15 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         return __syncthreads_or(!ok) == 0;
     };
 
-    // thread roles for the token-parallel passes: subtile ti, channel pair cp
-    const int ti = tid >> 6;          // subtile 0..3
-    const int cp = tid & 63;          // channel pair
-    const int c0 = 2 * cp;            // first channel
-    const int cblk = c0 >> 6;         // 64-wide block of the channel
-    const int cin = c0 & 63;          // channel inside the block
+    // thread roles for the token-parallel passes: subtile ti (warps 2ti, 2ti+1), half hh of
+    // the subtile (rows 8hh..8hh+7), and a quad of channels (4 consecutive channels, 8 bytes)
+    const int ti = warp >> 1;                     // subtile 0..3
+    const int hh = lane >> 4;                     // which 8 rows of the subtile
+    const int cq = (warp & 1) * 16 + (lane & 15); // channel quad 0..31
+    const int c0 = 4 * cq;                        // first channel
+    const int cblk = c0 >> 6;                     // 64-wide block of the channel
+    const int cin = c0 & 63;                      // channel inside the block
+    constexpr int HR = SUB / 2;                   // rows per thread
     constexpr uint32_t idG = idesc_bf16_f32(128, 16, 0, 0);     // Gram: K-major x K-major, N = 16
     constexpr uint32_t idKM = idesc_bf16_f32(128, 128, 0, 1);   // K-major A, MN-major B, N = 128
     constexpr uint32_t idMM = idesc_bf16_f32(128, 128, 1, 1);   // MN-major A and B, N = 128
@@ -269,8 +339,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (__syncthreads_or(!ok)) { aborted = true; break; }
         }
         if (tid < C) {
-            sBeta[tid] = (tid < Lc) ? bnext : 0.f;
-            if (more && tid < len - (ch + 1) * C) bnext = __bfloat162float(beta[(size_t)(tokn + tid) * H + h]);
+            sBeta[tid] = (tid < Lc) ? __bfloat162float(bnext) : 0.f;
+            if (more && tid < len - (ch + 1) * C) bnext = beta[(size_t)(tokn + tid) * H + h];
         }
         if (Lc < C) {  // zero the rows past the end of the sequence
             for (int idx = tid; idx < (C - Lc) * 16; idx += NT) {
@@ -285,20 +355,35 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         __syncthreads();
 
-        // ---- phase 1a: cumulative log2-decay inside subtile ti for channels c0, c0+1
-        float gl[SUB][2];
+        // ---- phase 1a: cumulative log2-decay inside subtile ti for channels c0..c0+3
+        float gl[HR][4];
         {
-            float a0 = 0.f, a1 = 0.f;
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int rr = 0; rr < SUB; ++rr) {
-                const float2 gv = ld_bf2(sm + OFF_G + (SUB * ti + rr) * 256 + c0 * 2);
-                a0 = fmaf(gv.x, kLog2e, a0);
-                a1 = fmaf(gv.y, kLog2e, a1);
-                gl[rr][0] = a0;
-                gl[rr][1] = a1;
+            for (int rr = 0; rr < HR; ++rr) {
+                const uint2 raw = *reinterpret_cast<const uint2 *>(sm + OFF_G + (SUB * ti + HR * hh + rr) * 256 + c0 * 2);
+                const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+                const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+                a[0] = fmaf(g01.x, kLog2e, a[0]);
+                a[1] = fmaf(g01.y, kLog2e, a[1]);
+                a[2] = fmaf(g23.x, kLog2e, a[2]);
+                a[3] = fmaf(g23.y, kLog2e, a[3]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) gl[rr][e] = a[e];
             }
-            sD[ti * D + c0] = a0;
-            sD[ti * D + c0 + 1] = a1;
+            // the upper half adds the lower half's total (lane - 16 holds the same channels)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float lo = __shfl_sync(0xffffffffu, a[e], lane & 15);
+                if (hh) {
+#pragma unroll
+                    for (int rr = 0; rr < HR; ++rr) gl[rr][e] += lo;
+                }
+            }
+            if (hh) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sD[ti * D + c0 + e] = gl[HR - 1][e];
+            }
         }
         __syncthreads();
         if (more && tid == 0) {  // g tile consumed: start the next chunk's loads
@@ -307,19 +392,19 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
 
         // ---- phase 1b: Gram operands and Gamma * q; keep the exp factors for phase 3
-        float F[SUB][2], Rf[SUB][2];
-        float ed[NSUB][2], pg[2], post[2];
+        float F[HR][4], Rf[HR][4];
+        float pg[4], post[4];
         {
-            float Dm[NSUB][2];
+            float Dm[NSUB][4], ed[NSUB][4];
 #pragma unroll
-            for (int m = 0; m < NSUB; ++m)
+            for (int m = 0; m < NSUB; ++m) {
+                const float4 d4 = *reinterpret_cast<const float4 *>(sD + m * D + c0);
+                Dm[m][0] = d4.x; Dm[m][1] = d4.y; Dm[m][2] = d4.z; Dm[m][3] = d4.w;
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
-                    Dm[m][e] = sD[m * D + c0 + e];
-                    ed[m][e] = ex2(Dm[m][e]);
-                }
+                for (int e = 0; e < 4; ++e) ed[m][e] = ex2(Dm[m][e]);
+            }
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
+            for (int e = 0; e < 4; ++e) {
                 float a = 1.f, b = 1.f;
 #pragma unroll
                 for (int m = 0; m < NSUB; ++m) {
@@ -329,70 +414,89 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 pg[e] = a;     // Gamma at the start of subtile ti (relative to the chunk start)
                 post[e] = b;   // decay from the end of subtile ti to the end of the chunk
             }
-            if (ti == 0) {
-#pragma unroll
-                for (int e = 0; e < 2; ++e) sGamC[c0 + e] = ed[0][e] * ed[1][e] * ed[2][e] * ed[3][e];
+            if (ti == 0 && hh == 0) {
+                *reinterpret_cast<float4 *>(sGamC + c0) =
+                    make_float4(ed[0][0] * ed[1][0] * ed[2][0] * ed[3][0], ed[0][1] * ed[1][1] * ed[2][1] * ed[3][1],
+                                ed[0][2] * ed[1][2] * ed[2][2] * ed[3][2], ed[0][3] * ed[1][3] * ed[2][3] * ed[3][3]);
             }
-            float E[NSUB][2];  // E[j] = exp(G_start(ti) - G_end(j)) for j < ti, exp(-D_ti) for j = ti
+            float E[NSUB][4];  // E[j] = exp(G_start(ti) - G_end(j)) for j < ti, exp(-D_ti) for j = ti
+            float dti[4];
 #pragma unroll
-            for (int j = 0; j < NSUB; ++j)
+            for (int e = 0; e < 4; ++e) {
+                dti[e] = (ti == 0) ? Dm[0][e] : (ti == 1) ? Dm[1][e] : (ti == 2) ? Dm[2][e] : Dm[3][e];
 #pragma unroll
-                for (int e = 0; e < 2; ++e) {
+                for (int j = 0; j < NSUB; ++j) {
                     float acc = 1.f;
 #pragma unroll
                     for (int m = 0; m < NSUB; ++m)
                         if (m > j && m < ti) acc *= ed[m][e];
-                    E[j][e] = (j == ti) ? ex2(-Dm[ti][e]) : acc;
+                    E[j][e] = (j == ti) ? ex2(-dti[e]) : acc;
                 }
-            float dti[2];
+            }
 #pragma unroll
-            for (int e = 0; e < 2; ++e) dti[e] = (ti == 0) ? Dm[0][e] : (ti == 1) ? Dm[1][e] : (ti == 2) ? Dm[2][e] : Dm[3][e];
+            for (int rr = 0; rr < HR; ++rr)
 #pragma unroll
-            for (int rr = 0; rr < SUB; ++rr)
-#pragma unroll
-                for (int e = 0; e < 2; ++e) {
+                for (int e = 0; e < 4; ++e) {
                     F[rr][e] = ex2(gl[rr][e]);
                     Rf[rr][e] = ex2(dti[e] - gl[rr][e]);
                 }
             uint8_t *const qrow = sm + OFF_WQ + cblk * 16 * KB;
             uint8_t *const krow = sm + OFF_KS + cblk * 8 * KB;
             uint8_t *const rrow = sm + OFF_R + cblk * 8 * KB;
+            auto st4 = [](uint8_t *p, float a, float b, float c, float d) {
+                *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf2(a, b), pack_bf2(c, d));
+            };
+            auto ld4 = [](const uint8_t *p, float (&v)[4]) {
+                const uint2 raw = *reinterpret_cast<const uint2 *>(p);
+                const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+                const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+                v[0] = x.x; v[1] = x.y; v[2] = y.x; v[3] = y.y;
+            };
 #pragma unroll
-            for (int rr = 0; rr < SUB; ++rr) {
-                const int r = SUB * ti + rr;
-                const uint32_t off_r = sw128_offset(r, cin);       // (r & 7) == (rr & 7)
+            for (int rr = 0; rr < HR; ++rr) {
+                const int r = SUB * ti + HR * hh + rr;
+                const uint32_t off_r = sw128_offset(r, cin);       // (r & 7) == rr
                 const uint32_t off_q = sw128_offset(64 + r, cin);
-                const float2 kx = ld_bf2(krow + off_r);
-                const float2 qx = ld_bf2(qrow + off_q);
-                st_bf2(rrow + off_r, kx.x * Rf[rr][0], kx.y * Rf[rr][1]);
-                const float kf0 = kx.x * F[rr][0], kf1 = kx.y * F[rr][1];
-                const float qf0 = qx.x * F[rr][0], qf1 = qx.y * F[rr][1];
+                float kx[4], qx[4], kf[4], qf[4];
+                ld4(krow + off_r, kx);
+                ld4(qrow + off_q, qx);
+                st4(rrow + off_r, kx[0] * Rf[rr][0], kx[1] * Rf[rr][1], kx[2] * Rf[rr][2], kx[3] * Rf[rr][3]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    kf[e] = kx[e] * F[rr][e];
+                    qf[e] = qx[e] * F[rr][e];
+                }
 #pragma unroll
                 for (int j = 0; j < NSUB; ++j) {
                     if (j > ti) continue;
                     const uint32_t rows = l_rows(j), hr = rows / 2;
                     uint8_t *Lb = sm + OFF_L + l_off(j) + cblk * rows * 128;
-                    st_bf2(Lb + sw128_offset(r - 16 * j, cin), kf0 * E[j][0], kf1 * E[j][1]);
-                    st_bf2(Lb + sw128_offset(hr + r - 16 * j, cin), qf0 * E[j][0], qf1 * E[j][1]);
+                    st4(Lb + sw128_offset(r - 16 * j, cin), kf[0] * E[j][0], kf[1] * E[j][1], kf[2] * E[j][2],
+                        kf[3] * E[j][3]);
+                    st4(Lb + sw128_offset(hr + r - 16 * j, cin), qf[0] * E[j][0], qf[1] * E[j][1],
+                        qf[2] * E[j][2], qf[3] * E[j][3]);
                 }
-                st_bf2(qrow + off_q, qf0 * pg[0], qf1 * pg[1]);  // Gamma * q in place
+                st4(qrow + off_q, qf[0] * pg[0], qf[1] * pg[1], qf[2] * pg[2], qf[3] * pg[3]);  // Gamma * q
             }
         }
         fence_proxy_async_smem();
         __syncthreads();
 
-        // ---- Gram MMAs: column block j -> TMEM columns 16j..16j+15
-        if (tid == 0) {
+        // ---- Gram MMAs: column block j -> TMEM columns 16j..16j+15, issued by lane 0 of warp j
+        if (lane == 0 && warp < NSUB) {
+            const int j = warp;
             tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < NSUB; ++j) {
-                Opnd A{sbase + OFF_L + l_off(j), false, l_rows(j) * 128u, 0};
-                Opnd B{sbase + OFF_R + 16u * j * 128u, false, 8 * KB, 0};
-                mma_chain<D / 16>(tmem + TM_GRAM + 16u * j, A, B, idG, false);
-            }
-            mma_commit(bar_mma);
+            Opnd A{sbase + OFF_L + l_off(j), false, l_rows(j) * 128u, 0};
+            Opnd B{sbase + OFF_R + 16u * j * 128u, false, 8 * KB, 0};
+            mma_chain<D / 16>(tmem + TM_GRAM + 16u * j, A, B, idG, false);
+            mma_commit(bar_gram);
         }
-        if (!wait_mma()) { aborted = true; break; }
+        {
+            const bool ok = mbar_wait_bounded(bar_gram, gram_phase, kWaitCycles);
+            gram_phase ^= 1u;
+            tc_fence_after();
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+        }
 
         // ---- phase 2: Gram readout -> A (fp32, strictly lower, times beta_r), P (bf16, lower)
         {
@@ -431,57 +535,26 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         __syncthreads();
 
         // ---- phase 3: T = (I + A)^{-1} (unit lower triangular) by 16 x 16 blocks
-        if (tid < 64) {  // diagonal blocks: forward substitution, one column per thread, in registers
+        if (tid < 64) {  // diagonal blocks: right-looking substitution, one column per thread, in registers
             const int bi = tid >> 4, cc = tid & 15, o0 = 16 * bi;
             float x[16];
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) {
-                float acc = (rr == cc) ? 1.f : 0.f;
+            for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == cc) ? 1.f : 0.f;
 #pragma unroll
-                for (int ss = 0; ss < rr; ++ss) acc = fmaf(-AF[(o0 + rr) * 65 + o0 + ss], x[ss], acc);
-                x[rr] = acc;  // zero above the diagonal since x[ss < cc] = 0
-                TF[(o0 + rr) * 68 + o0 + cc] = acc;
+            for (int ss = 0; ss < 16; ++ss) {
+                // x[ss] is final; entries above the diagonal stay 0 because x[ss < cc] = 0
+#pragma unroll
+                for (int rr = ss + 1; rr < 16; ++rr) x[rr] = fmaf(-AF[(o0 + rr) * 65 + o0 + ss], x[ss], x[rr]);
+            }
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) TF[(o0 + rr) * 68 + o0 + cc] = x[rr];
+            if ((bi & 1) == 0) {  // the 16 x 16 block right of it, inside its 32 x 32 diagonal block
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) TF[(o0 + rr) * 68 + o0 + 16 + cc] = 0.f;
             }
         }
         __syncthreads();
-        // off-diagonal blocks by distance: X = sum_{m=j}^{i-1} A_im T_mj, then T_ij = -T_ii X
-#pragma unroll
-        for (int dist = 1; dist < NSUB; ++dist) {
-            const int nblk = NSUB - dist;
-            const int b = tid >> 6, r = (tid & 63) >> 2, q0 = (tid & 3) * 4;
-            const int bi = dist + b, bj = b;
-            if (b < nblk) {
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int m = bj; m < bi; ++m) {
-#pragma unroll
-                    for (int kk = 0; kk < 16; ++kk) {
-                        const float a = AF[(16 * bi + r) * 65 + 16 * m + kk];
-                        const float4 t = *reinterpret_cast<const float4 *>(TF + (16 * m + kk) * 68 + 16 * bj + q0);
-                        acc.x = fmaf(a, t.x, acc.x);
-                        acc.y = fmaf(a, t.y, acc.y);
-                        acc.z = fmaf(a, t.z, acc.z);
-                        acc.w = fmaf(a, t.w, acc.w);
-                    }
-                }
-                *reinterpret_cast<float4 *>(XS + b * 320 + r * 20 + q0) = acc;
-            }
-            __syncthreads();
-            if (b < nblk) {
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                for (int kk = 0; kk < 16; ++kk) {
-                    const float a = TF[(16 * bi + r) * 68 + 16 * bi + kk];
-                    const float4 t = *reinterpret_cast<const float4 *>(XS + b * 320 + kk * 20 + q0);
-                    acc.x = fmaf(a, t.x, acc.x);
-                    acc.y = fmaf(a, t.y, acc.y);
-                    acc.z = fmaf(a, t.z, acc.z);
-                    acc.w = fmaf(a, t.w, acc.w);
-                }
-                *reinterpret_cast<float4 *>(TF + (16 * bi + r) * 68 + 16 * bj + q0) =
-                    make_float4(-acc.x, -acc.y, -acc.z, -acc.w);
-            }
-            __syncthreads();
-        }
+        tri_inverse_offdiag(AF, TF, XS, tid);
         // T Diag(beta) -> bf16 A operand (rows 0..63), zero rows 64..127
         for (int idx = tid; idx < 128 * 8; idx += NT) {
             const int r = idx >> 3, pc = (idx & 7) * 8;
@@ -506,11 +579,20 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             uint8_t *ktrow = sm + OFF_KT + cblk * 8 * KB;
             uint8_t *khrow = sm + OFF_KHAT + cblk * 8 * KB;
 #pragma unroll
-            for (int rr = 0; rr < SUB; ++rr) {
-                const uint32_t off_r = sw128_offset(SUB * ti + rr, cin);
-                const float2 kx = ld_bf2(krow + off_r);
-                st_bf2(ktrow + off_r, kx.x * F[rr][0] * pg[0], kx.y * F[rr][1] * pg[1]);
-                st_bf2(khrow + off_r, kx.x * Rf[rr][0] * post[0], kx.y * Rf[rr][1] * post[1]);
+            for (int rr = 0; rr < HR; ++rr) {
+                const uint32_t off_r = sw128_offset(SUB * ti + HR * hh + rr, cin);
+                const uint2 raw = *reinterpret_cast<const uint2 *>(krow + off_r);
+                const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+                const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+                const float kx[4] = {x.x, x.y, y.x, y.y};
+                float a[4], b[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    a[e] = kx[e] * F[rr][e] * pg[e];
+                    b[e] = kx[e] * Rf[rr][e] * post[e];
+                }
+                *reinterpret_cast<uint2 *>(ktrow + off_r) = make_uint2(pack_bf2(a[0], a[1]), pack_bf2(a[2], a[3]));
+                *reinterpret_cast<uint2 *>(khrow + off_r) = make_uint2(pack_bf2(b[0], b[1]), pack_bf2(b[2], b[3]));
             }
         }
         fence_proxy_async_smem();
