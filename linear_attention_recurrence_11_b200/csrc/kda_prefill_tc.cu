@@ -52,7 +52,7 @@ constexpr uint32_t OFF_SB = 32 * KB;    // 32 KB  B operand S (bf16), MN-major [
 constexpr uint32_t OFF_KS = 64 * KB;    // 16 KB  k tile, [tok rows][dk] (2 blocks of 64 channels)
 constexpr uint32_t OFF_V = 80 * KB;     // 16 KB  v: B operand MN-major [tok rows][dv] (2 N-blocks)
 constexpr uint32_t OFF_G = 96 * KB;     // 16 KB  g, plain [64][128] bf16
-constexpr uint32_t OFF_R = 112 * KB;    // 16 KB  Gram right operand, K-major [s rows][dk]; later U (MN-major B)
+constexpr uint32_t OFF_R = 112 * KB;    // 16 KB  Gram right operand, K-major [s rows][dk]; later Kh (MN-major A)
 constexpr uint32_t OFF_PB = 128 * KB;   // 8 KB   rows 64..127 of the A operand [junk ; P], K-major, K = 64
 constexpr uint32_t OFF_L = 136 * KB;    // 80 KB  Gram left operands L3, L2, L1, L0 (compact), then the aliases below
 constexpr uint32_t OFF_MISC = 216 * KB;
@@ -64,8 +64,9 @@ __host__ __device__ constexpr uint32_t l_off(int j) {
 // aliases inside the L region once the Gram MMAs are done
 constexpr uint32_t OFF_TB = OFF_L + 0;             // 16 KB  A operand T Diag(beta), K-major, 128 rows x 64
 constexpr uint32_t OFF_KT = OFF_L + 16 * KB;       // 16 KB  B operand Gamma*K, MN-major [tok][dk]
-constexpr uint32_t OFF_AF = OFF_L + 32 * KB;       // 64 x 65 fp32  A (dead once T is known)
-constexpr uint32_t OFF_KHAT = OFF_L + 32 * KB;     // 16 KB  A operand Kh, MN-major [tok][dk] (written after A is dead)
+constexpr uint32_t OFF_AF = OFF_L + 32 * KB;       // 64 x 65 fp32  A
+constexpr uint32_t OFF_KHAT = OFF_R;               // 16 KB  A operand Kh, MN-major [tok][dk] (the Gram is done)
+constexpr uint32_t OFF_UB = OFF_L + 0;             // 16 KB  B operand U, MN-major [tok][dv] (T Diag(beta) is done)
 constexpr uint32_t OFF_TF = OFF_L + 49 * KB;       // 64 x 68 fp32  T
 constexpr uint32_t OFF_XS = OFF_TF + 64 * 68 * 4;  // 32 x 36 fp32 scratch
 static_assert(OFF_AF + 64 * 65 * 4 <= OFF_TF, "A overlaps T");
@@ -127,67 +128,78 @@ __device__ __forceinline__ void mma_chain(uint32_t d_tmem, const Opnd &A, const 
 }
 
 
+// fp32 -> tf32 (round to nearest, ties away), for the warp-level MMAs below.
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+    uint32_t y;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(y) : "f"(x));
+    return y;
+}
+
+// One warp: C[16 x 8] = sum_k A[ar + 0..15][ac + k] * B[br + k][bc + 0..7], k < K,
+// A and B fp32 in shared memory (row strides lda, ldb), with mma.sync m16n8k8 TF32
+// (fp32 accumulation). Fragment (g = lane / 4, t = lane % 4): A rows g, g + 8 and
+// columns t, t + 4; B rows t, t + 4 and column g; C rows g, g + 8, columns 2t, 2t + 1.
+template <int K>
+__device__ __forceinline__ void warp_mma_16x8(const float *A, int lda, int ar, int ac, const float *B, int ldb,
+                                              int br, int bc, float (&c)[4]) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    c[0] = c[1] = c[2] = c[3] = 0.f;
+#pragma unroll
+    for (int k0 = 0; k0 < K; k0 += 8) {
+        const uint32_t a0 = to_tf32(A[(ar + g) * lda + ac + k0 + t]);
+        const uint32_t a1 = to_tf32(A[(ar + g + 8) * lda + ac + k0 + t]);
+        const uint32_t a2 = to_tf32(A[(ar + g) * lda + ac + k0 + t + 4]);
+        const uint32_t a3 = to_tf32(A[(ar + g + 8) * lda + ac + k0 + t + 4]);
+        const uint32_t b0 = to_tf32(B[(br + k0 + t) * ldb + bc + g]);
+        const uint32_t b1 = to_tf32(B[(br + k0 + t + 4) * ldb + bc + g]);
+        asm volatile(
+            "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+            "{%0,%1,%2,%3};"
+            : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+}
+
+// Store a C fragment of warp_mma_16x8 (times `scale`) at D[dr + .., dc + ..].
+__device__ __forceinline__ void warp_store_16x8(float *Dm, int ldd, int dr, int dc, const float (&c)[4],
+                                                float scale) {
+    const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+    *reinterpret_cast<float2 *>(Dm + (dr + g) * ldd + dc + 2 * t) = make_float2(scale * c[0], scale * c[1]);
+    *reinterpret_cast<float2 *>(Dm + (dr + g + 8) * ldd + dc + 2 * t) = make_float2(scale * c[2], scale * c[3]);
+}
+
 // Off-diagonal part of T = (I + A)^{-1} (64 x 64 unit lower triangular) once the
-// four 16 x 16 diagonal blocks T_ii are in place (zero above their diagonal):
-//   level 1:  T_10 = -T_11 A_10 T_00,  T_32 = -T_33 A_32 T_22            (16 x 16)
-//   level 2:  T[32:64, 0:32] = -T[32:64, 32:64] A[32:64, 0:32] T[0:32, 0:32] (32 x 32)
-// i.e. the 2 x 2 block inverse applied twice. Each product is spread over all
-// 256 threads with 2 (level 1) or 4 (level 2) outputs per thread.
-// A: 64 x 65 fp32 (strictly lower), T: 64 x 68 fp32, XS: scratch of 32 x 36 fp32.
+// four 16 x 16 diagonal blocks T_ii are in place (zero above their diagonal, and
+// zero in the 16 x 16 block to the right of T_00 and T_22):
+//   level 1:  T_10 = -T_11 A_10 T_00,  T_32 = -T_33 A_32 T_22                 (16 x 16)
+//   level 2:  T[32:64, 0:32] = -T[32:64, 32:64] A[32:64, 0:32] T[0:32, 0:32]  (32 x 32)
+// i.e. the 2 x 2 block inverse applied twice; each product is a handful of
+// warp-level TF32 MMAs. A: 64 x 65 fp32 (strictly lower), T: 64 x 68 fp32,
+// XS: scratch of 32 x 36 fp32.
 __device__ __forceinline__ void tri_inverse_offdiag(const float *AF, float *TF, float *XS, int tid) {
-    {   // level 1, X = A_ij T_jj for (i, j) = (1, 0), (3, 2); 2 blocks x 16 x 16 outputs
-        const int b = tid >> 7, r = (tid & 127) >> 3, c = (tid & 7) * 2;
-        const int i = 2 * b + 1, j = 2 * b;
-        float x0 = 0.f, x1 = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const float a = AF[(16 * i + r) * 65 + 16 * j + k];
-            const float2 t = *reinterpret_cast<const float2 *>(TF + (16 * j + k) * 68 + 16 * j + c);
-            x0 = fmaf(a, t.x, x0);
-            x1 = fmaf(a, t.y, x1);
-        }
-        *reinterpret_cast<float2 *>(XS + b * 16 * 18 + r * 18 + c) = make_float2(x0, x1);
-        __syncthreads();
-        // T_ij = -T_ii X
-        float y0 = 0.f, y1 = 0.f;
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-            const float a = TF[(16 * i + r) * 68 + 16 * i + k];
-            const float2 x = *reinterpret_cast<const float2 *>(XS + b * 16 * 18 + k * 18 + c);
-            y0 = fmaf(a, x.x, y0);
-            y1 = fmaf(a, x.y, y1);
-        }
-        *reinterpret_cast<float2 *>(TF + (16 * i + r) * 68 + 16 * j + c) = make_float2(-y0, -y1);
-        __syncthreads();
+    const int warp = tid >> 5;
+    float c[4];
+    // level 1: 2 blocks x 2 column tiles of 8 -> warps 0..3
+    const int b = (warp >> 1) & 1, nt = warp & 1;
+    const int i1 = 16 * (2 * b + 1), j1 = 16 * (2 * b);
+    if (warp < 4) {
+        warp_mma_16x8<16>(AF, 65, i1, j1, TF, 68, j1, j1 + 8 * nt, c);     // X = A_ij T_jj
+        warp_store_16x8(XS, 36, 16 * b, 8 * nt, c, 1.f);
     }
-    {   // level 2, X = A[32:64, 0:32] T[0:32, 0:32]; 32 x 32 outputs, 4 per thread
-        const int r = tid >> 3, c = (tid & 7) * 4;
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const float a = AF[(32 + r) * 65 + k];
-            const float4 t = *reinterpret_cast<const float4 *>(TF + k * 68 + c);
-            x.x = fmaf(a, t.x, x.x);
-            x.y = fmaf(a, t.y, x.y);
-            x.z = fmaf(a, t.z, x.z);
-            x.w = fmaf(a, t.w, x.w);
-        }
-        *reinterpret_cast<float4 *>(XS + r * 36 + c) = x;
-        __syncthreads();
-        // T[32:64, 0:32] = -T[32:64, 32:64] X
-        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int k = 0; k < 32; ++k) {
-            const float a = TF[(32 + r) * 68 + 32 + k];
-            const float4 t = *reinterpret_cast<const float4 *>(XS + k * 36 + c);
-            y.x = fmaf(a, t.x, y.x);
-            y.y = fmaf(a, t.y, y.y);
-            y.z = fmaf(a, t.z, y.z);
-            y.w = fmaf(a, t.w, y.w);
-        }
-        *reinterpret_cast<float4 *>(TF + (32 + r) * 68 + c) = make_float4(-y.x, -y.y, -y.z, -y.w);
-        __syncthreads();
+    __syncthreads();
+    if (warp < 4) {
+        warp_mma_16x8<16>(TF, 68, i1, i1, XS, 36, 16 * b, 8 * nt, c);       // T_ij = -T_ii X
+        warp_store_16x8(TF, 68, i1, j1 + 8 * nt, c, -1.f);
     }
+    __syncthreads();
+    // level 2: 2 row tiles x 4 column tiles -> warps 0..7
+    const int mt = warp >> 2, n2 = warp & 3;
+    warp_mma_16x8<32>(AF, 65, 32 + 16 * mt, 0, TF, 68, 0, 8 * n2, c);        // X = A21 T_lo
+    warp_store_16x8(XS, 36, 16 * mt, 8 * n2, c, 1.f);
+    __syncthreads();
+    warp_mma_16x8<32>(TF, 68, 32 + 16 * mt, 32, XS, 36, 0, 8 * n2, c);       // T21 = -T_hi X
+    warp_store_16x8(TF, 68, 32 + 16 * mt, 8 * n2, c, -1.f);
+    __syncthreads();
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -312,11 +324,13 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         return __syncthreads_or(!ok) == 0;
     };
 
-    // thread roles for the token-parallel passes: subtile ti (warps 2ti, 2ti+1), half hh of
+    // thread roles for the token-parallel passes: subtile ti (a pair of warps), half hh of
     // the subtile (rows 8hh..8hh+7), and a quad of channels (4 consecutive channels, 8 bytes)
-    const int ti = warp >> 1;                     // subtile 0..3
+    // subtile of each warp pair; warps w and w + 4 share a scheduler, and subtile i
+    // writes i + 1 Gram left-operand rows per token, so pair subtiles 0 with 3 and 1 with 2
+    const int ti = (0x22331100 >> (4 * warp)) & 0xF;  // warps 0..7 -> 0,0,1,1,3,3,2,2
     const int hh = lane >> 4;                     // which 8 rows of the subtile
-    const int cq = (warp & 1) * 16 + (lane & 15); // channel quad 0..31
+    const int cq = (warp & 1) * 16 + (lane & 15); // channel quad 0..31 (the two warps of a pair)
     const int c0 = 4 * cq;                        // first channel
     const int cblk = c0 >> 6;                     // 64-wide block of the channel
     const int cin = c0 & 63;                      // channel inside the block
@@ -535,6 +549,28 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         __syncthreads();
 
         // ---- phase 3: T = (I + A)^{-1} (unit lower triangular) by 16 x 16 blocks
+        // Gamma * k -> KT and Kh = exp(G_C - G_s) * k_s -> KHAT (first, so the exp factors die early)
+        {
+            const uint8_t *krow = sm + OFF_KS + cblk * 8 * KB;
+            uint8_t *ktrow = sm + OFF_KT + cblk * 8 * KB;
+            uint8_t *khrow = sm + OFF_KHAT + cblk * 8 * KB;
+#pragma unroll
+            for (int rr = 0; rr < HR; ++rr) {
+                const uint32_t off_r = sw128_offset(SUB * ti + HR * hh + rr, cin);
+                const uint2 raw = *reinterpret_cast<const uint2 *>(krow + off_r);
+                const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+                const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+                const float kx[4] = {x.x, x.y, y.x, y.y};
+                float a[4], b[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    a[e] = kx[e] * F[rr][e] * pg[e];
+                    b[e] = kx[e] * Rf[rr][e] * post[e];
+                }
+                *reinterpret_cast<uint2 *>(ktrow + off_r) = make_uint2(pack_bf2(a[0], a[1]), pack_bf2(a[2], a[3]));
+                *reinterpret_cast<uint2 *>(khrow + off_r) = make_uint2(pack_bf2(b[0], b[1]), pack_bf2(b[2], b[3]));
+            }
+        }
         if (tid < 64) {  // diagonal blocks: right-looking substitution, one column per thread, in registers
             const int bi = tid >> 4, cc = tid & 15, o0 = 16 * bi;
             float x[16];
@@ -572,28 +608,6 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 w.w = pack_bf2(u[6], u[7]);
             }
             *reinterpret_cast<uint4 *>(sm + OFF_TB + sw128_offset(r, pc)) = w;
-        }
-        // Gamma * k -> KT and Kh = exp(G_C - G_s) * k_s -> KHAT (A is dead now)
-        {
-            const uint8_t *krow = sm + OFF_KS + cblk * 8 * KB;
-            uint8_t *ktrow = sm + OFF_KT + cblk * 8 * KB;
-            uint8_t *khrow = sm + OFF_KHAT + cblk * 8 * KB;
-#pragma unroll
-            for (int rr = 0; rr < HR; ++rr) {
-                const uint32_t off_r = sw128_offset(SUB * ti + HR * hh + rr, cin);
-                const uint2 raw = *reinterpret_cast<const uint2 *>(krow + off_r);
-                const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
-                const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
-                const float kx[4] = {x.x, x.y, y.x, y.y};
-                float a[4], b[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    a[e] = kx[e] * F[rr][e] * pg[e];
-                    b[e] = kx[e] * Rf[rr][e] * post[e];
-                }
-                *reinterpret_cast<uint2 *>(ktrow + off_r) = make_uint2(pack_bf2(a[0], a[1]), pack_bf2(a[2], a[3]));
-                *reinterpret_cast<uint2 *>(khrow + off_r) = make_uint2(pack_bf2(b[0], b[1]), pack_bf2(b[2], b[3]));
-            }
         }
         fence_proxy_async_smem();
         __syncthreads();
@@ -651,7 +665,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // ---- phase 5: U (rows 0..63) -> bf16 B operand, MN-major [tok][dv]
         if (quarter < 2) {
             const int r = 32 * quarter + lane;
-            uint8_t *base = sm + OFF_R + half * 8 * KB;
+            uint8_t *base = sm + OFF_UB + half * 8 * KB;
 #pragma unroll
             for (int gq = 0; gq < 4; ++gq) {
                 float v[16];
@@ -676,7 +690,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (tid == 0) {
             tc_fence_after();
             Opnd AP{sbase + OFF_PB - 8 * KB, false, 16 * KB, 0};
-            Opnd BU{sbase + OFF_R, true, 0, 8 * KB};
+            Opnd BU{sbase + OFF_UB, true, 0, 8 * KB};
             Opnd AK{sbase + OFF_KHAT, true, 0, 8 * KB};
             mma_chain<C / 16>(tmem + TM_KU, AK, BU, idMM, false);
             mma_chain<C / 16>(tmem + TM_U, AP, BU, idKM, true);
