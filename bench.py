@@ -48,6 +48,8 @@ def parse_args():
     p.add_argument("--workload", default="prefill", choices=sorted(WORKLOAD_ALIASES))
     p.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
     p.add_argument("--decode-steps", type=int, default=50)
+    p.add_argument("--tokens", type=int, default=0,
+                   help="override T of the dense prefill workload (smaller only for profiling captures)")
     p.add_argument("--decode-requests", type=int, default=256,
                    help="requests in the decode batch (smaller only for profiling captures)")
     p.add_argument("--no-decode", action="store_true")
@@ -172,9 +174,11 @@ def run_ours(args, rank, world, device):
     from linear_attention_recurrence_11_b200 import kda
     from linear_attention_recurrence_11_b200.inputs import WORKLOADS, workload_inputs
     import dataclasses
-
     wname = WORKLOAD_ALIASES[args.workload]
     w = WORKLOADS[wname]
+    if args.tokens and not w.seqlens and not w.decode_steps:
+        w = dataclasses.replace(w, T=args.tokens)
+        wname = f"{wname}@T{args.tokens}"
     peaks = load_peaks()
     res = {}
     stream = torch.cuda.current_stream(device)

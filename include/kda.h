@@ -73,8 +73,13 @@ int kda_abi_version(void);
 
 /*
  * Bytes of device workspace kda_forward needs for these sizes (0 if none).
- * num_seqs is the number of packed sequences when cu_seqlens is used, else B.
- * Returns (size_t)-1 if the sizes are invalid.
+ * num_seqs is the number of packed sequences when cu_seqlens is used, else B
+ * (B == 1 with num_seqs > 1 means packed sequences). Packed batches of 2 to
+ * 2048 sequences use a few bytes per sequence for a longest-first schedule
+ * (a small kernel ranks the sequences by length so the longest start first);
+ * nothing else needs workspace. The workspace is scratch: its contents on
+ * entry do not matter and it may be reused after the stream reaches the end
+ * of the call. Returns (size_t)-1 if the sizes are invalid.
  */
 size_t kda_forward_workspace_size(int B, int T, int H, int dk, int dv, int chunk,
                                   int num_seqs, int dtype);

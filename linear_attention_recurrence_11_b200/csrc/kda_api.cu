@@ -27,6 +27,10 @@ int check_prefill_sizes(int B, int T, int H, int dk, int dv, int chunk, int dtyp
     return KDA_OK;
 }
 
+// Marks "packed sequences are used" in size-only queries, where the real device
+// pointer is not at hand; it is compared against null and never dereferenced.
+const int32_t kPackedMarker = 0;
+
 bool use_tc(const kda::PrefillArgs &a, int path) {
     if (path == KDA_PATH_SIMT) return false;
     return kda::prefill_tc_supported(a.dk, a.dv, a.chunk, a.dtype);
@@ -54,10 +58,11 @@ int kda_abi_version(void) { return 1; }
 size_t kda_forward_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int num_seqs,
                                   int dtype) {
     kda::PrefillArgs a{};
-    const bool has_cu = num_seqs > 0 && B == 1 && num_seqs != B;
+    // packed sequences (cu_seqlens) are recognised by B == 1 and num_seqs > 1
+    const bool has_cu = B == 1 && num_seqs > 1;
     if (check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, has_cu, num_seqs, KDA_PATH_AUTO, &a))
         return (size_t)-1;
-    a.num_units = num_seqs > 0 ? num_seqs : B;
+    a.cu_seqlens = has_cu ? &kPackedMarker : nullptr;
     size_t ws = kda::prefill_simt_workspace(a);
     if (kda::prefill_tc_supported(dk, dv, chunk, dtype)) {
         const size_t t = kda::prefill_tc_workspace(a);
@@ -71,6 +76,7 @@ int kda_forward_launches(int B, int T, int H, int dk, int dv, int chunk, int dty
     kda::PrefillArgs a{};
     if (check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, has_cu_seqlens != 0, num_seqs, path, &a))
         return -1;
+    a.cu_seqlens = has_cu_seqlens ? &kPackedMarker : nullptr;
     return use_tc(a, path) ? kda::prefill_tc_launches(a) : kda::prefill_simt_launches(a);
 }
 

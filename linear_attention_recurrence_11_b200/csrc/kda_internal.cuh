@@ -17,6 +17,7 @@ struct PrefillArgs {
     void *o;
     float *ST;
     const int32_t *cu_seqlens;  // device offsets or nullptr
+    const int32_t *seq_order;   // device: block b runs sequence seq_order[b / H] (nullptr: b / H)
     int B, T, H, dk, dv, chunk, dtype;
     int num_units;              // N: sequences (B, or num_seqs with cu_seqlens)
     void *workspace;
@@ -41,6 +42,16 @@ __device__ __forceinline__ float ld_elem(const __nv_bfloat16 *p, size_t i) {
 __device__ __forceinline__ void st_elem(float *p, size_t i, float x) { p[i] = x; }
 __device__ __forceinline__ void st_elem(__nv_bfloat16 *p, size_t i, float x) {
     p[i] = __float2bfloat16_rn(x);
+}
+
+// Longest-first ordering of packed sequences (workspace-backed, up to this many).
+constexpr int kMaxOrderedSeqs = 2048;
+size_t seq_order_bytes(int num_seqs);  // 0 when no ordering is done
+cudaError_t launch_seq_order(const int32_t *cu_seqlens, int num_seqs, int32_t *order, cudaStream_t stream);
+
+// Sequence index run by prefill block `b` (one block per (sequence, head) unit).
+__device__ __forceinline__ int unit_seq(const PrefillArgs &p, int b_over_h) {
+    return p.seq_order ? p.seq_order[b_over_h] : b_over_h;
 }
 
 // Launchers (return cudaSuccess or the launch error).

@@ -60,7 +60,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_simt_kernel(const Pre
     const int nblk = p.dv / DVB;
     const int dvb = blockIdx.x % nblk;
     const int h = (blockIdx.x / nblk) % p.H;
-    const int n = blockIdx.x / (nblk * p.H);
+    const int n = unit_seq(p, blockIdx.x / (nblk * p.H));
     const size_t H = (size_t)p.H, dv = (size_t)p.dv;
     size_t t_begin, len;
     if (p.cu_seqlens) {
@@ -241,13 +241,23 @@ cudaError_t launch_dtype(const PrefillArgs &a) {
 
 }  // namespace
 
-cudaError_t launch_prefill_simt(const PrefillArgs &a) {
-    if (a.num_units == 0 || a.H == 0) return cudaSuccess;
+cudaError_t launch_prefill_simt(const PrefillArgs &a_in) {
+    if (a_in.num_units == 0 || a_in.H == 0) return cudaSuccess;
+    PrefillArgs a = a_in;
+    if (a.cu_seqlens && seq_order_bytes(a.num_units) > 0) {
+        int32_t *order = static_cast<int32_t *>(a.workspace);
+        const cudaError_t e = launch_seq_order(a.cu_seqlens, a.num_units, order, a.stream);
+        if (e != cudaSuccess) return e;
+        a.seq_order = order;
+    }
     return a.dtype == KDA_DTYPE_BF16 ? launch_dtype<__nv_bfloat16>(a) : launch_dtype<float>(a);
 }
 
-size_t prefill_simt_workspace(const PrefillArgs &) { return 0; }
+size_t prefill_simt_workspace(const PrefillArgs &a) { return a.cu_seqlens ? seq_order_bytes(a.num_units) : 0; }
 
-int prefill_simt_launches(const PrefillArgs &a) { return (a.num_units > 0 && a.H > 0) ? 1 : 0; }
+int prefill_simt_launches(const PrefillArgs &a) {
+    if (a.num_units <= 0 || a.H <= 0) return 0;
+    return 1 + ((a.cu_seqlens && seq_order_bytes(a.num_units) > 0) ? 1 : 0);
+}
 
 }  // namespace kda

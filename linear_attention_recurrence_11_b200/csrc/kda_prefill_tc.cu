@@ -225,7 +225,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, half = warp >> 2;  // TMEM lane quarter, column half
     const int h = blockIdx.x % p.H;
-    const int n = blockIdx.x / p.H;
+    const int n = unit_seq(p, blockIdx.x / p.H);
     const size_t H = (size_t)p.H;
     long long t_begin, len;
     if (p.cu_seqlens) {
@@ -809,9 +809,12 @@ bool prefill_tc_supported(int dk, int dv, int chunk, int dtype) {
     return dk == D && dv == D && chunk == C && dtype == KDA_DTYPE_BF16;
 }
 
-size_t prefill_tc_workspace(const PrefillArgs &) { return 0; }
+size_t prefill_tc_workspace(const PrefillArgs &a) { return a.cu_seqlens ? seq_order_bytes(a.num_units) : 0; }
 
-int prefill_tc_launches(const PrefillArgs &a) { return (a.num_units > 0 && a.H > 0) ? 1 : 0; }
+int prefill_tc_launches(const PrefillArgs &a) {
+    if (a.num_units <= 0 || a.H <= 0) return 0;
+    return 1 + ((a.cu_seqlens && seq_order_bytes(a.num_units) > 0) ? 1 : 0);
+}
 
 cudaError_t launch_prefill_tc(const PrefillArgs &a) {
     if (a.num_units == 0) return cudaSuccess;
@@ -826,6 +829,12 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a) {
                                          (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     TcParams prm{a};
+    if (a.cu_seqlens && seq_order_bytes(a.num_units) > 0) {
+        int32_t *order = static_cast<int32_t *>(a.workspace);
+        e = launch_seq_order(a.cu_seqlens, a.num_units, order, a.stream);
+        if (e != cudaSuccess) return e;
+        prm.a.seq_order = order;
+    }
     const unsigned grid = (unsigned)((size_t)a.num_units * a.H);
     kda_prefill_tc_kernel<<<grid, NT, SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, prm);
     return cudaGetLastError();

@@ -88,6 +88,10 @@ def test_forward_rejects_bad_pointers(K):
 def test_forward_varlen_rules(K):
     assert fwd(K, cu=FAKE, num_seqs=0) == K.KDA_ERR_INVALID_ARG
     assert fwd(K, cu=FAKE, num_seqs=2, B=2) == K.KDA_ERR_INVALID_ARG
+    # the longest-first schedule needs its workspace; missing or short -> rejected before launch
+    for path in (0, 1, 2):
+        assert fwd(K, cu=FAKE, num_seqs=8, path=path) == K.KDA_ERR_WORKSPACE
+        assert fwd(K, cu=FAKE, num_seqs=8, ws=FAKE, ws_bytes=16, path=path) == K.KDA_ERR_WORKSPACE
 
 
 def test_tc_path_only_where_built(K):
@@ -106,7 +110,15 @@ def test_decode_rejects_bad_args(K):
 
 
 def test_workspace_and_launch_queries(K):
-    assert K.kda_forward_workspace_size(1, 8192, 96, 128, 128, 64, 1, 1) >= 0
+    assert K.kda_forward_workspace_size(1, 8192, 96, 128, 128, 64, 1, 1) == 0
+    assert K.kda_forward_workspace_size(2, 8192, 96, 128, 128, 64, 2, 1) == 0
+    # packed sequences: a small longest-first schedule (up to 2048 sequences)
+    assert K.kda_forward_workspace_size(1, 352549, 96, 128, 128, 64, 8, 1) == 256
+    assert K.kda_forward_workspace_size(1, 100000, 2, 64, 64, 32, 2048, 0) == 8192
+    assert K.kda_forward_workspace_size(1, 100000, 2, 64, 64, 32, 2049, 0) == 0
+    assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8) == 2
+    assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8, "simt") == 2
+    assert K.kda_forward_launches(1, 8192, 96, 128, 128, 64, 1, 0, 1) == 1
     with pytest.raises(K.KdaError):
         K.kda_forward_workspace_size(1, 8192, 96, 100, 128, 64, 1, 1)
     assert K.kda_forward_launches(1, 8192, 96, 128, 128, 64, 1, 0, 1) >= 1

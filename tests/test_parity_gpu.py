@@ -85,6 +85,30 @@ def test_varlen_with_edge_lengths(K, oracle_mod, path):
     assert torch.equal(ST[3], inp["S0"][3])
 
 
+@pytest.mark.parametrize("nseq", [40, 2100])
+def test_varlen_many_sequences(K, oracle_mod, nseq):
+    """Many packed sequences of mixed lengths (zeros included): with up to 2048
+    sequences a longest-first schedule runs first; above that, natural order."""
+    rng = np.random.default_rng(nseq)
+    if nseq <= 2048:
+        lens = rng.integers(0, 300, size=nseq)
+    else:
+        lens = rng.integers(0, 4, size=nseq)
+    lens[::7] = 0
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    H = 2
+    inp = case(1, int(cu[-1]), H, 128, 128, "bf16", seed=nseq, s0_std=0.1, num_states=nseq)
+    inp["cu_seqlens"] = torch.tensor(cu, device="cuda")
+    o, ST = run(K, inp, 64, "auto")
+    picks = [int(i) for i in np.argsort(-lens)[:3]] + [int(np.argmin(lens)), nseq - 1]
+    units = [(n, h) for n in picks for h in range(H)]
+    o_ref, ST_ref = oracle_forward(oracle_mod, inp, units=units)
+    e_o, e_s = compare_units(o, ST, o_ref, ST_ref, units, cu)
+    assert e_o < TOL["bf16"] and e_s < TOL["bf16"], (e_o, e_s)
+    zero = np.nonzero(lens == 0)[0]
+    assert torch.equal(ST[zero], inp["S0"][zero])
+
+
 @pytest.mark.parametrize("path", PATHS)
 def test_identity_transition_is_exact(K, path):
     """beta = 0, g = 0: S_T = S0 bit for bit and o_t = S0^T q_t."""
