@@ -167,6 +167,30 @@ def decode_algorithmic(N, H, dk, dv, elem):
     return float(N * H * per_head), float(N * H * 7 * dk * dv)
 
 
+# ----------------------------------------------------- multi-rank helpers
+
+def rank_workload(w, rank: int):
+    """Each rank runs its own batch of independent sequences (weak scaling):
+    the same shapes and distributions, a rank-specific seed."""
+    import dataclasses
+    return dataclasses.replace(w, seed=w.seed + 7919 * rank)
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The slowest rank's time: an all-reduce MAX (no-op for one rank)."""
+    if world == 1:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(units_per_rank: float, steps: int, ms_total_max: float, world: int) -> float:
+    """Whole-job throughput: all ranks' units over the slowest rank's time."""
+    return world * units_per_rank * steps / (ms_total_max / 1e3)
+
+
 # --------------------------------------------------------------- our arm
 
 def run_ours(args, rank, world, device):
@@ -187,19 +211,14 @@ def run_ours(args, rank, world, device):
         if world > 1:
             torch.distributed.barrier()
 
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+    def max_ranks(x):
+        return max_over_ranks(x, world, device)
 
     if w.decode_steps:
-        return run_decode_main(args, rank, world, device, w, peaks, barrier, max_over_ranks)
+        return run_decode_main(args, rank, world, device, w, peaks, barrier, max_ranks)
 
     # every rank draws its own batch (independent sequences)
-    w_rank = dataclasses.replace(w, seed=w.seed + 7919 * rank)
-    inp = workload_inputs(w_rank, device=device)
+    inp = workload_inputs(rank_workload(w, rank), device=device)
     B = 1 if w.seqlens else w.B
     T = w.total_tokens if w.seqlens else w.T
     N = w.num_seqs
@@ -236,11 +255,11 @@ def run_ours(args, rank, world, device):
         torch.cuda.synchronize(device)
     barrier()
     torch.cuda.synchronize(device)
-    ms_total = max_over_ranks(t0.elapsed_time(t1))
+    ms_total = max_ranks(t0.elapsed_time(t1))
     kern_ms = statistics.mean(a.elapsed_time(b) for a, b in evs)
     ms_step = ms_total / K
     tokens = w.total_tokens
-    value = world * tokens * K / (ms_total / 1e3)
+    value = weak_scaling_value(tokens, K, ms_total, world)
     alg_bytes, alg_flops = prefill_algorithmic(w, elem)
     kern_src = ("linear_attention_recurrence_11_b200/csrc/kda_prefill_tc.cu" if path_used == "tc"
                 else "linear_attention_recurrence_11_b200/csrc/kda_prefill_simt.cu")
@@ -268,9 +287,9 @@ def run_ours(args, rank, world, device):
     })
 
     if not args.no_e2e:
-        res["e2e"] = e2e_prefill(args, device, inp, w, o, ST, ws, cu, world, barrier, max_over_ranks)
+        res["e2e"] = e2e_prefill(args, device, inp, w, o, ST, ws, cu, world, barrier, max_ranks)
     if not args.no_decode and args.workload == "prefill":
-        res["decode"] = decode_measure(args, device, peaks, barrier, max_over_ranks, world,
+        res["decode"] = decode_measure(args, device, peaks, barrier, max_ranks, world,
                                        steps=args.decode_steps)
         res["gpu_launches"] += res["decode"]["gpu_launches"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -278,7 +297,7 @@ def run_ours(args, rank, world, device):
     return res
 
 
-def e2e_prefill(args, device, inp, w, o, ST, ws, cu, world, barrier, max_over_ranks):
+def e2e_prefill(args, device, inp, w, o, ST, ws, cu, world, barrier, max_ranks):
     """Same metric through the public API from pinned host buffers: per step,
     H2D of q,k,v,g,beta(,S0), the prefill, D2H of o and S_T."""
     import torch
@@ -311,13 +330,13 @@ def e2e_prefill(args, device, inp, w, o, ST, ws, cu, world, barrier, max_over_ra
         step()
     b.record(stream)
     torch.cuda.synchronize(device)
-    ms = max_over_ranks(a.elapsed_time(b))
+    ms = max_ranks(a.elapsed_time(b))
     return {"value": world * w.total_tokens * K / (ms / 1e3), "unit": "tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
             "ms_per_step": ms / K}
 
 
-def decode_measure(args, device, peaks, barrier, max_over_ranks, world, steps):
+def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):
     """Decode step over 256 requests x 96 heads (1.61 GB of fp32 state, larger
     than L2), states updated in place; per-step inputs cycle over 8 pre-drawn
     sets."""
@@ -351,7 +370,7 @@ def decode_measure(args, device, peaks, barrier, max_over_ranks, world, steps):
             step(i)
         b.record(stream)
         torch.cuda.synchronize(device)
-    ms = max_over_ranks(a.elapsed_time(b)) / steps
+    ms = max_ranks(a.elapsed_time(b)) / steps
     elem = sets[0]["k"].element_size()
     alg_bytes, _ = decode_algorithmic(w.B, w.H, w.dk, w.dv, elem)
     gbs = alg_bytes / (ms / 1e3) / 1e9
@@ -368,8 +387,8 @@ def decode_measure(args, device, peaks, barrier, max_over_ranks, world, steps):
             "requests": w.B, "l2": f"state {w.B * w.H * w.dk * w.dv * 4 / 1e9:.2f} GB per step, larger than L2"}
 
 
-def run_decode_main(args, rank, world, device, w, peaks, barrier, max_over_ranks):
-    d = decode_measure(args, device, peaks, barrier, max_over_ranks, world, steps=args.steps)
+def run_decode_main(args, rank, world, device, w, peaks, barrier, max_ranks):
+    d = decode_measure(args, device, peaks, barrier, max_ranks, world, steps=args.steps)
     return {"metric": d["metric"], "value": d["value"], "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": d["ms_per_step"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
