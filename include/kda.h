@@ -55,7 +55,8 @@ typedef enum {
     KDA_ERR_ALIGNMENT = 3,   /* a pointer is not 16-byte aligned                         */
     KDA_ERR_WORKSPACE = 4,   /* workspace missing or smaller than required               */
     KDA_ERR_CUDA = 5,        /* a CUDA runtime call or kernel launch failed               */
-    KDA_ERR_TIMEOUT = 6      /* (device status word) a bounded wait gave up              */
+    KDA_ERR_TIMEOUT = 6,     /* (device status word) a bounded wait gave up              */
+    KDA_ERR_SCRATCH_LIMIT = 7 /* kda_forward_noalloc: more packed sequences than its fixed scratch holds */
 } kda_status;
 
 typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype;
@@ -123,6 +124,34 @@ int kda_forward_ex(const void *q, const void *k, const void *v, const void *g, c
  * enqueues (0 when T = 0 and no state is copied), or -1 if invalid. */
 int kda_forward_launches(int B, int T, int H, int dk, int dv, int chunk, int dtype,
                          int has_cu_seqlens, int num_seqs, int path);
+
+/*
+ * kda_forward without a workspace argument, for callers that cannot allocate
+ * device memory: engines that reserve all device memory in their own pools at
+ * start-up and treat any other allocation as an error, hosts that hand a
+ * library raw device pointers but no allocator, and latency-critical paths
+ * where an allocation could block. (The Kimi K3 pages have no counterpart; it
+ * is an interface convenience, not part of the method.)
+ *
+ * Same arguments and results as kda_forward, minus workspace. The only
+ * scratch the computation uses, the longest-first schedule of a packed batch,
+ * lives in a fixed array of this library's own device memory: 2048 int32
+ * (8 KiB), held by every GPU that loads the library until the process exits.
+ * Hence the limit: a packed batch (cu_seqlens != NULL) of more than 2048
+ * sequences returns KDA_ERR_SCRATCH_LIMIT and launches nothing; dense batches
+ * have no limit. This entry point itself allocates nothing.
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any stream
+ * capture. Every call shares the one array per device and leaves its contents
+ * behind (each call overwrites what it reads, so stale contents are harmless);
+ * calls that overlap on the GPU race on it, so do not run two at once on one
+ * device.
+ */
+int kda_forward_noalloc(const void *q, const void *k, const void *v, const void *g,
+                        const void *beta, const float *S0, void *o, float *S_T, int B, int T,
+                        int H, int dk, int dv, int chunk, int dtype, const int32_t *cu_seqlens,
+                        int num_seqs, int *dev_status, void *stream);
 
 /*
  * One decode step: one new token for each of N requests, states in place.

@@ -49,6 +49,7 @@ const char *kda_status_string(int status) {
         case KDA_ERR_WORKSPACE: return "workspace missing or too small";
         case KDA_ERR_CUDA: return "CUDA error";
         case KDA_ERR_TIMEOUT: return "bounded wait timed out";
+        case KDA_ERR_SCRATCH_LIMIT: return "more packed sequences than the no-alloc entry point's fixed scratch holds";
         default: return "unknown status";
     }
 }

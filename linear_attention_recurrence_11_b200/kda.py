@@ -37,9 +37,11 @@ _lib.kda_forward_ex.argtypes = _FWD + [_i]
 _lib.kda_forward_ex.restype = _i
 _lib.kda_decode_step.argtypes = [_vp] * 7 + [_i] * 5 + [_vp]
 _lib.kda_decode_step.restype = _i
+_lib.kda_forward_noalloc.argtypes = [_vp] * 8 + [_i] * 7 + [_vp, _i, _vp, _vp]
+_lib.kda_forward_noalloc.restype = _i
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT = 0, 1, 2, 3
-KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = 4, 5, 6
+KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_SCRATCH_LIMIT = 4, 5, 6, 7
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 PATHS = {"auto": 0, "simt": 1, "tc": 2}
 
@@ -136,6 +138,41 @@ def kda_forward(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=None, 
                              _stream_handle(stream, dev), PATHS[path])
     if rc != KDA_OK:
         raise KdaError(rc, "kda_forward")
+    return o, S_T
+
+
+def kda_forward_noalloc(q, k, v, g, beta, S0, o, S_T, *, chunk: int = 64, cu_seqlens=None,
+                        dev_status=None, stream=None):
+    """kda_forward for callers that cannot allocate device memory: no workspace
+    argument (the library keeps a fixed 8 KiB schedule array per device) and no
+    allocation here either, so o and S_T must be passed in (S_T may be None).
+    Packed batches are limited to 2048 sequences (KdaError KDA_ERR_SCRATCH_LIMIT
+    beyond that). Calls that overlap on one device race on that array."""
+    _need(k, "k")
+    dtype, dev = k.dtype, k.device
+    if dtype not in DTYPES:
+        raise ValueError(f"unsupported dtype {dtype}")
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    _need(q, "q", dtype, (B, T, H, dk), dev)
+    _need(g, "g", dtype, (B, T, H, dk), dev)
+    _need(v, "v", dtype, (B, T, H, dv), dev)
+    _need(beta, "beta", dtype, (B, T, H), dev)
+    N = B
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, None, dev)
+        N = cu_seqlens.numel() - 1
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (N, H, dv, dk), dev)
+    _need(o, "o", dtype, (B, T, H, dv), dev)
+    if S_T is not None:
+        _need(S_T, "S_T", torch.float32, (N, H, dv, dk), dev)
+    rc = _lib.kda_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                  _ptr(S_T), B, T, H, dk, dv, int(chunk), DTYPES[dtype],
+                                  _ptr(cu_seqlens), N if cu_seqlens is not None else 0,
+                                  _ptr(dev_status), _stream_handle(stream, dev))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_forward_noalloc")
     return o, S_T
 
 
