@@ -15,9 +15,11 @@
 //     exponent factor below is <= e^80) and the scaled bf16 operands of the
 //     decayed Grams. Column block j (tokens 16j..16j+15) of
 //        A_rs = beta_r sum_c k_rc k_sc e^{G_rc - G_sc},  P_rs = sum_c q_rc k_sc e^{G_rc - G_sc}
-//     is the product of a left operand k_r e^{G_r - G_end(j)} (stacked with
-//     q_r e^{G_r - G_end(j)}) and a right operand k_s e^{G_end(j) - G_s}; both
-//     factors stay in [0, e^80].
+//     is the product of a left operand k_r e^{G_r - G_start(j)} (stacked with
+//     q_r e^{G_r - G_start(j)}, rows r >= 16j) and a right operand
+//     k_s e^{G_start(j) - G_s}; the left factor is <= 1, the right one in
+//     [1, e^80]. For j = 0 the left operand is [Gamma*k ; Gamma*q] itself, the
+//     tile the state products use anyway.
 //  3. tcgen05.mma (M=128, N=16, K=128) x 4 -> TMEM; readout to A (fp32) and P (bf16).
 //  4. CUDA cores: T = (I + A)^{-1} by 16 x 16 blocks (forward substitution on
 //     the diagonal blocks, then block rows by distance).
@@ -47,7 +49,7 @@ constexpr int SUB = 16, NSUB = C / SUB;
 
 // ---------------------------------------------------------- smem layout
 constexpr uint32_t KB = 1024;
-constexpr uint32_t OFF_WQ = 0;          // 32 KB  A operand [-W ; Qt], K-major, 128 rows x 128 (2 K-blocks); q lands in rows 64..127
+constexpr uint32_t OFF_WQ = 0;          // 32 KB  [Gamma*K, then -W ; Gamma*Q], K-major, 128 rows x 128 (2 K-blocks); q lands in rows 64..127
 constexpr uint32_t OFF_SB = 32 * KB;    // 32 KB  B operand S (bf16), MN-major [dk rows][dv] (2 N-blocks)
 constexpr uint32_t OFF_KS = 64 * KB;    // 16 KB  k tile, [tok rows][dk] (2 blocks of 64 channels)
 constexpr uint32_t OFF_V = 80 * KB;     // 16 KB  v: B operand MN-major [tok rows][dv] (2 N-blocks)
@@ -56,14 +58,16 @@ constexpr uint32_t OFF_R = 112 * KB;    // 16 KB  Gram right operand, K-major [s
 constexpr uint32_t OFF_PB = 128 * KB;   // 8 KB   rows 64..127 of the A operand [junk ; P], K-major, K = 64
 constexpr uint32_t OFF_L = 136 * KB;    // 80 KB  Gram left operands L3, L2, L1, L0 (compact), then the aliases below
 constexpr uint32_t OFF_MISC = 216 * KB;
-// L region: compact left operands, L_j has 2 (64 - 16 j) rows (K part, then Q part).
+// L region: compact left operands of column blocks 1..3, L_j has 2 (64 - 16 j) rows (K part,
+// then Q part); block 0's left operand is the [Gamma*K ; Gamma*Q] tile at OFF_WQ. The order
+// keeps every 128-row operand read (from each K-block start) inside the region.
 __host__ __device__ constexpr uint32_t l_rows(int j) { return 2u * (64u - 16u * j); }
-__host__ __device__ constexpr uint32_t l_off(int j) {
-    return j == 3 ? 0u : j == 2 ? 8u * KB : j == 1 ? 24u * KB : 48u * KB;
-}
+__host__ __device__ constexpr uint32_t l_off(int j) { return j == 3 ? 0u : j == 2 ? 8u * KB : 24u * KB; }
 // aliases inside the L region once the Gram MMAs are done
 constexpr uint32_t OFF_TB = OFF_L + 0;             // 16 KB  A operand T Diag(beta), K-major, 128 rows x 64
-constexpr uint32_t OFF_KT = OFF_L + 16 * KB;       // 16 KB  B operand Gamma*K, MN-major [tok][dk]
+// Gamma*K sits in rows 0..63 of the [-W ; Gamma*Q] tile until the W product is read out:
+// the same bytes are block 0's Gram operand (K-major A) and the W product's B (MN-major).
+constexpr uint32_t OFF_KT = OFF_WQ;
 constexpr uint32_t OFF_AF = OFF_L + 32 * KB;       // 64 x 65 fp32  A
 constexpr uint32_t OFF_KHAT = OFF_R;               // 16 KB  A operand Kh, MN-major [tok][dk] (the Gram is done)
 constexpr uint32_t OFF_UB = OFF_L + 0;             // 16 KB  B operand U, MN-major [tok][dv] (T Diag(beta) is done)
@@ -405,8 +409,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             issue_g(tokn);
         }
 
-        // ---- phase 1b: Gram operands and Gamma * q; keep the exp factors for phase 3
-        float F[HR][4], Rf[HR][4];
+        // ---- phase 1b: Gram operands, Gamma * q and Gamma * k; keep the factors for Kh
+        float F[HR][4], Fi[HR][4];
         float pg[4], post[4];
         {
             float Dm[NSUB][4], ed[NSUB][4];
@@ -423,36 +427,33 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 #pragma unroll
                 for (int m = 0; m < NSUB; ++m) {
                     if (m < ti) a *= ed[m][e];
-                    if (m > ti) b *= ed[m][e];
+                    if (m >= ti) b *= ed[m][e];
                 }
                 pg[e] = a;     // Gamma at the start of subtile ti (relative to the chunk start)
-                post[e] = b;   // decay from the end of subtile ti to the end of the chunk
+                post[e] = b;   // decay from the start of subtile ti to the end of the chunk
             }
             if (ti == 0 && hh == 0) {
                 *reinterpret_cast<float4 *>(sGamC + c0) =
                     make_float4(ed[0][0] * ed[1][0] * ed[2][0] * ed[3][0], ed[0][1] * ed[1][1] * ed[2][1] * ed[3][1],
                                 ed[0][2] * ed[1][2] * ed[2][2] * ed[3][2], ed[0][3] * ed[1][3] * ed[2][3] * ed[3][3]);
             }
-            float E[NSUB][4];  // E[j] = exp(G_start(ti) - G_end(j)) for j < ti, exp(-D_ti) for j = ti
-            float dti[4];
+            float E[NSUB][4];  // E[j] = exp(G_start(ti) - G_start(j)) for j = 1..ti (1 for j = ti)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                dti[e] = (ti == 0) ? Dm[0][e] : (ti == 1) ? Dm[1][e] : (ti == 2) ? Dm[2][e] : Dm[3][e];
+            for (int j = 0; j < NSUB; ++j)
 #pragma unroll
-                for (int j = 0; j < NSUB; ++j) {
+                for (int e = 0; e < 4; ++e) {
                     float acc = 1.f;
 #pragma unroll
                     for (int m = 0; m < NSUB; ++m)
-                        if (m > j && m < ti) acc *= ed[m][e];
-                    E[j][e] = (j == ti) ? ex2(-dti[e]) : acc;
+                        if (m >= j && m < ti) acc *= ed[m][e];
+                    E[j][e] = acc;
                 }
-            }
 #pragma unroll
             for (int rr = 0; rr < HR; ++rr)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    F[rr][e] = ex2(gl[rr][e]);
-                    Rf[rr][e] = ex2(dti[e] - gl[rr][e]);
+                    F[rr][e] = ex2(gl[rr][e]);    // e^{G_r - G_start(ti)}, in [e^-80, 1]
+                    Fi[rr][e] = ex2(-gl[rr][e]);  // e^{G_start(ti) - G_r}, in [1, e^80]
                 }
             uint8_t *const qrow = sm + OFF_WQ + cblk * 16 * KB;
             uint8_t *const krow = sm + OFF_KS + cblk * 8 * KB;
@@ -474,14 +475,15 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 float kx[4], qx[4], kf[4], qf[4];
                 ld4(krow + off_r, kx);
                 ld4(qrow + off_q, qx);
-                st4(rrow + off_r, kx[0] * Rf[rr][0], kx[1] * Rf[rr][1], kx[2] * Rf[rr][2], kx[3] * Rf[rr][3]);
+                // right operand row r (column block ti): k_r e^{G_start(ti) - G_r}
+                st4(rrow + off_r, kx[0] * Fi[rr][0], kx[1] * Fi[rr][1], kx[2] * Fi[rr][2], kx[3] * Fi[rr][3]);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     kf[e] = kx[e] * F[rr][e];
                     qf[e] = qx[e] * F[rr][e];
                 }
 #pragma unroll
-                for (int j = 0; j < NSUB; ++j) {
+                for (int j = 1; j < NSUB; ++j) {
                     if (j > ti) continue;
                     const uint32_t rows = l_rows(j), hr = rows / 2;
                     uint8_t *Lb = sm + OFF_L + l_off(j) + cblk * rows * 128;
@@ -491,6 +493,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         qf[2] * E[j][2], qf[3] * E[j][3]);
                 }
                 st4(qrow + off_q, qf[0] * pg[0], qf[1] * pg[1], qf[2] * pg[2], qf[3] * pg[3]);  // Gamma * q
+                st4(qrow + off_r, kf[0] * pg[0], kf[1] * pg[1], kf[2] * pg[2], kf[3] * pg[3]);  // Gamma * k, row r
             }
         }
         fence_proxy_async_smem();
@@ -500,7 +503,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (lane == 0 && warp < NSUB) {
             const int j = warp;
             tc_fence_after();
-            Opnd A{sbase + OFF_L + l_off(j), false, l_rows(j) * 128u, 0};
+            Opnd A = (j == 0) ? Opnd{sbase + OFF_WQ, false, 16 * KB, 0}
+                              : Opnd{sbase + OFF_L + l_off(j), false, l_rows(j) * 128u, 0};
             Opnd B{sbase + OFF_R + 16u * j * 128u, false, 8 * KB, 0};
             mma_chain<D / 16>(tmem + TM_GRAM + 16u * j, A, B, idG, false);
             mma_commit(bar_gram);
@@ -549,10 +553,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         __syncthreads();
 
         // ---- phase 3: T = (I + A)^{-1} (unit lower triangular) by 16 x 16 blocks
-        // Gamma * k -> KT and Kh = exp(G_C - G_s) * k_s -> KHAT (first, so the exp factors die early)
+        // Kh = exp(G_C - G_s) * k_s -> KHAT (first, so the exp factors die early)
         {
             const uint8_t *krow = sm + OFF_KS + cblk * 8 * KB;
-            uint8_t *ktrow = sm + OFF_KT + cblk * 8 * KB;
             uint8_t *khrow = sm + OFF_KHAT + cblk * 8 * KB;
 #pragma unroll
             for (int rr = 0; rr < HR; ++rr) {
@@ -560,15 +563,10 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 const uint2 raw = *reinterpret_cast<const uint2 *>(krow + off_r);
                 const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
                 const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
-                const float kx[4] = {x.x, x.y, y.x, y.y};
-                float a[4], b[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    a[e] = kx[e] * F[rr][e] * pg[e];
-                    b[e] = kx[e] * Rf[rr][e] * post[e];
-                }
-                *reinterpret_cast<uint2 *>(ktrow + off_r) = make_uint2(pack_bf2(a[0], a[1]), pack_bf2(a[2], a[3]));
-                *reinterpret_cast<uint2 *>(khrow + off_r) = make_uint2(pack_bf2(b[0], b[1]), pack_bf2(b[2], b[3]));
+                // e^{G_C - G_s} = e^{G_start(ti) - G_s} e^{G_C - G_start(ti)}, both factors bounded
+                const float b0 = x.x * Fi[rr][0] * post[0], b1 = x.y * Fi[rr][1] * post[1];
+                const float b2 = y.x * Fi[rr][2] * post[2], b3 = y.y * Fi[rr][3] * post[3];
+                *reinterpret_cast<uint2 *>(khrow + off_r) = make_uint2(pack_bf2(b0, b1), pack_bf2(b2, b3));
             }
         }
         if (tid < 64) {  // diagonal blocks: right-looking substitution, one column per thread, in registers
@@ -617,7 +615,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (more) issue_k(tokn);  // the k tile is consumed
             tc_fence_after();
             Opnd A{sbase + OFF_TB, false, 16 * KB, 0};
-            Opnd BK{sbase + OFF_KT, true, 0, 8 * KB};
+            Opnd BK{sbase + OFF_KT, true, 0, 16 * KB};
             Opnd BV{sbase + OFF_V, true, 0, 8 * KB};
             mma_chain<C / 16>(tmem + TM_W, A, BK, idKM, false);
             mma_chain<C / 16>(tmem + TM_U, A, BV, idKM, false);
