@@ -68,13 +68,17 @@ constexpr uint32_t OFF_TB = OFF_L + 0;             // 16 KB  A operand T Diag(be
 // Gamma*K sits in rows 0..63 of the [-W ; Gamma*Q] tile until the W product is read out:
 // the same bytes are block 0's Gram operand (K-major A) and the W product's B (MN-major).
 constexpr uint32_t OFF_KT = OFF_WQ;
-constexpr uint32_t OFF_AF = OFF_L + 32 * KB;       // 64 x 65 fp32  A
+// fp32 row strides (in floats) of the small matrices of the triangular inverse, chosen so that
+// the warp-level MMA fragments below read shared memory without bank conflicts: rows of an A
+// fragment are LDA apart (LDA = 4 mod 32), rows of a B fragment LDX apart (LDX = 8 mod 32).
+constexpr int LDA = 68, LDT = 68, LDX = 40;
+constexpr uint32_t OFF_AF = OFF_L + 32 * KB;       // 64 x LDA fp32  A
 constexpr uint32_t OFF_KHAT = OFF_R;               // 16 KB  A operand Kh, MN-major [tok][dk] (the Gram is done)
 constexpr uint32_t OFF_UB = OFF_L + 0;             // 16 KB  B operand U, MN-major [tok][dv] (T Diag(beta) is done)
-constexpr uint32_t OFF_TF = OFF_L + 49 * KB;       // 64 x 68 fp32  T
-constexpr uint32_t OFF_XS = OFF_TF + 64 * 68 * 4;  // 32 x 36 fp32 scratch
-static_assert(OFF_AF + 64 * 65 * 4 <= OFF_TF, "A overlaps T");
-static_assert(OFF_XS + 32 * 36 * 4 <= OFF_MISC, "scratch overflows the L region");
+constexpr uint32_t OFF_TF = OFF_L + 49 * KB;       // 64 x LDT fp32  T
+constexpr uint32_t OFF_XS = OFF_TF + 64 * LDT * 4;  // 32 x LDX fp32 scratch
+static_assert(OFF_AF + 64 * LDA * 4 <= OFF_TF, "A overlaps T");
+static_assert(OFF_XS + 32 * LDX * 4 <= OFF_MISC, "scratch overflows the L region");
 // misc
 constexpr uint32_t OFF_BAR = OFF_MISC;              // 3 mbarriers
 constexpr uint32_t OFF_TMEMADDR = OFF_MISC + 32;
@@ -105,6 +109,18 @@ __device__ __forceinline__ void st_bf2(uint8_t *p, float x, float y) {
 __device__ __forceinline__ uint32_t pack_bf2(float x, float y) {
     __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
     return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// 16 fp32 values (times `scale`) -> 16 bf16 in two 16-byte words
+__device__ __forceinline__ void pack16(const float *v, float scale, uint4 &w0, uint4 &w1) {
+    w0.x = pack_bf2(scale * v[0], scale * v[1]);
+    w0.y = pack_bf2(scale * v[2], scale * v[3]);
+    w0.z = pack_bf2(scale * v[4], scale * v[5]);
+    w0.w = pack_bf2(scale * v[6], scale * v[7]);
+    w1.x = pack_bf2(scale * v[8], scale * v[9]);
+    w1.y = pack_bf2(scale * v[10], scale * v[11]);
+    w1.z = pack_bf2(scale * v[12], scale * v[13]);
+    w1.w = pack_bf2(scale * v[14], scale * v[15]);
 }
 
 // ------------------------------------------------------------- MMA issue
@@ -178,7 +194,7 @@ __device__ __forceinline__ void warp_store_16x8(float *Dm, int ldd, int dr, int 
 //   level 1:  T_10 = -T_11 A_10 T_00,  T_32 = -T_33 A_32 T_22                 (16 x 16)
 //   level 2:  T[32:64, 0:32] = -T[32:64, 32:64] A[32:64, 0:32] T[0:32, 0:32]  (32 x 32)
 // i.e. the 2 x 2 block inverse applied twice; each product is a handful of
-// warp-level TF32 MMAs. A: 64 x 65 fp32 (strictly lower), T: 64 x 68 fp32,
+// warp-level TF32 MMAs. A: 64 x LDA fp32 (strictly lower), T: 64 x LDT fp32,
 // XS: scratch of 32 x 36 fp32.
 __device__ __forceinline__ void tri_inverse_offdiag(const float *AF, float *TF, float *XS, int tid) {
     const int warp = tid >> 5;
@@ -187,22 +203,22 @@ __device__ __forceinline__ void tri_inverse_offdiag(const float *AF, float *TF, 
     const int b = (warp >> 1) & 1, nt = warp & 1;
     const int i1 = 16 * (2 * b + 1), j1 = 16 * (2 * b);
     if (warp < 4) {
-        warp_mma_16x8<16>(AF, 65, i1, j1, TF, 68, j1, j1 + 8 * nt, c);     // X = A_ij T_jj
-        warp_store_16x8(XS, 36, 16 * b, 8 * nt, c, 1.f);
+        warp_mma_16x8<16>(AF, LDA, i1, j1, TF, LDT, j1, j1 + 8 * nt, c);     // X = A_ij T_jj
+        warp_store_16x8(XS, LDX, 16 * b, 8 * nt, c, 1.f);
     }
     __syncthreads();
     if (warp < 4) {
-        warp_mma_16x8<16>(TF, 68, i1, i1, XS, 36, 16 * b, 8 * nt, c);       // T_ij = -T_ii X
-        warp_store_16x8(TF, 68, i1, j1 + 8 * nt, c, -1.f);
+        warp_mma_16x8<16>(TF, LDT, i1, i1, XS, LDX, 16 * b, 8 * nt, c);       // T_ij = -T_ii X
+        warp_store_16x8(TF, LDT, i1, j1 + 8 * nt, c, -1.f);
     }
     __syncthreads();
     // level 2: 2 row tiles x 4 column tiles -> warps 0..7
     const int mt = warp >> 2, n2 = warp & 3;
-    warp_mma_16x8<32>(AF, 65, 32 + 16 * mt, 0, TF, 68, 0, 8 * n2, c);        // X = A21 T_lo
-    warp_store_16x8(XS, 36, 16 * mt, 8 * n2, c, 1.f);
+    warp_mma_16x8<32>(AF, LDA, 32 + 16 * mt, 0, TF, LDT, 0, 8 * n2, c);        // X = A21 T_lo
+    warp_store_16x8(XS, LDX, 16 * mt, 8 * n2, c, 1.f);
     __syncthreads();
-    warp_mma_16x8<32>(TF, 68, 32 + 16 * mt, 32, XS, 36, 0, 8 * n2, c);       // T21 = -T_hi X
-    warp_store_16x8(TF, 68, 32 + 16 * mt, 8 * n2, c, -1.f);
+    warp_mma_16x8<32>(TF, LDT, 32 + 16 * mt, 32, XS, LDX, 0, 8 * n2, c);       // T21 = -T_hi X
+    warp_store_16x8(TF, LDT, 32 + 16 * mt, 8 * n2, c, -1.f);
     __syncthreads();
 }
 
@@ -518,21 +534,25 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
         // ---- phase 2: Gram readout -> A (fp32, strictly lower, times beta_r), P (bf16, lower)
         {
+            float v2[2][16];
+            tmem_ld16(tmem + tlane + TM_GRAM + 16u * (2 * half), v2[0]);
+            tmem_ld16(tmem + tlane + TM_GRAM + 16u * (2 * half + 1), v2[1]);
+            tmem_wait_ld();
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
                 const int j = 2 * half + jj;
-                float v[16];
-                tmem_ld16(tmem + tlane + TM_GRAM + 16u * j, v);
-                tmem_wait_ld();
+                const float *v = v2[jj];
                 const int m = 32 * quarter + lane;
                 const int kr = 64 - 16 * j;
                 if (m < kr) {
                     const int r = 16 * j + m;
                     const float b = sBeta[r];
+                    float4 *arow = reinterpret_cast<float4 *>(AF + r * LDA + 16 * j);
 #pragma unroll
-                    for (int s2 = 0; s2 < 16; ++s2) {
-                        const int s = 16 * j + s2;
-                        AF[r * 65 + s] = (s < r) ? b * v[s2] : 0.f;
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        const int s = 16 * j + 4 * q4;
+                        arow[q4] = make_float4((s < r) ? b * v[4 * q4] : 0.f, (s + 1 < r) ? b * v[4 * q4 + 1] : 0.f,
+                                               (s + 2 < r) ? b * v[4 * q4 + 2] : 0.f, (s + 3 < r) ? b * v[4 * q4 + 3] : 0.f);
                     }
                 } else if (m < 2 * kr) {
                     const int r = 16 * j + (m - kr);
@@ -569,22 +589,33 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 *reinterpret_cast<uint2 *>(khrow + off_r) = make_uint2(pack_bf2(b0, b1), pack_bf2(b2, b3));
             }
         }
-        if (tid < 64) {  // diagonal blocks: right-looking substitution, one column per thread, in registers
-            const int bi = tid >> 4, cc = tid & 15, o0 = 16 * bi;
+        if (warp < NSUB && lane < 16) {
+            // diagonal block `warp`: forward substitution by rows (left-looking), one column of
+            // T_ii per lane; each row of A_ii is one broadcast read shared by the 16 lanes
+            const int o0 = 16 * warp, cc = lane;
             float x[16];
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) x[rr] = (rr == cc) ? 1.f : 0.f;
+            for (int rr = 0; rr < 16; ++rr) {
+                float a[16];
+                const float4 *arow = reinterpret_cast<const float4 *>(AF + (o0 + rr) * LDA + o0);
 #pragma unroll
-            for (int ss = 0; ss < 16; ++ss) {
-                // x[ss] is final; entries above the diagonal stay 0 because x[ss < cc] = 0
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    if (4 * q4 < rr) {
+                        const float4 t = arow[q4];
+                        a[4 * q4] = t.x; a[4 * q4 + 1] = t.y; a[4 * q4 + 2] = t.z; a[4 * q4 + 3] = t.w;
+                    }
+                }
+                // x[rr] = [rr == cc] - sum_{ss < rr} A[rr][ss] x[ss], four partial sums
+                float acc[4] = {(rr == cc) ? 1.f : 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int rr = ss + 1; rr < 16; ++rr) x[rr] = fmaf(-AF[(o0 + rr) * 65 + o0 + ss], x[ss], x[rr]);
+                for (int ss = 0; ss < rr; ++ss) acc[ss & 3] = fmaf(-a[ss], x[ss], acc[ss & 3]);
+                x[rr] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             }
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) TF[(o0 + rr) * 68 + o0 + cc] = x[rr];
-            if ((bi & 1) == 0) {  // the 16 x 16 block right of it, inside its 32 x 32 diagonal block
+            for (int rr = 0; rr < 16; ++rr) TF[(o0 + rr) * LDT + o0 + cc] = x[rr];
+            if ((warp & 1) == 0) {  // the 16 x 16 block right of it, inside its 32 x 32 diagonal block
 #pragma unroll
-                for (int rr = 0; rr < 16; ++rr) TF[(o0 + rr) * 68 + o0 + 16 + cc] = 0.f;
+                for (int rr = 0; rr < 16; ++rr) TF[(o0 + rr) * LDT + o0 + 16 + cc] = 0.f;
             }
         }
         __syncthreads();
@@ -594,8 +625,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const int r = idx >> 3, pc = (idx & 7) * 8;
             uint4 w = make_uint4(0, 0, 0, 0);
             if (r < C) {
-                const float4 t0 = *reinterpret_cast<const float4 *>(TF + r * 68 + pc);
-                const float4 t1 = *reinterpret_cast<const float4 *>(TF + r * 68 + pc + 4);
+                const float4 t0 = *reinterpret_cast<const float4 *>(TF + r * LDT + pc);
+                const float4 t1 = *reinterpret_cast<const float4 *>(TF + r * LDT + pc + 4);
                 const float t[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
                 float u[8];
 #pragma unroll
@@ -629,20 +660,16 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (quarter < 2) {
             const int r = 32 * quarter + lane;
             uint8_t *base = sm + OFF_WQ + half * 16 * KB;
+            float v[4][16];
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + TM_W + 64u * half + 16u * gq, v[gq]);
+            tmem_wait_ld();
 #pragma unroll
             for (int gq = 0; gq < 4; ++gq) {
-                float v[16];
-                tmem_ld16(tmem + tlane + TM_W + 64u * half + 16u * gq, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    uint4 w;
-                    w.x = pack_bf2(-v[8 * cc + 0], -v[8 * cc + 1]);
-                    w.y = pack_bf2(-v[8 * cc + 2], -v[8 * cc + 3]);
-                    w.z = pack_bf2(-v[8 * cc + 4], -v[8 * cc + 5]);
-                    w.w = pack_bf2(-v[8 * cc + 6], -v[8 * cc + 7]);
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, 16 * gq + 8 * cc)) = w;
-                }
+                uint4 w0, w1;
+                pack16(v[gq], -1.f, w0, w1);
+                *reinterpret_cast<uint4 *>(base + sw128_offset(r, 16 * gq)) = w0;
+                *reinterpret_cast<uint4 *>(base + sw128_offset(r, 16 * gq + 8)) = w1;
             }
         }
         fence_proxy_async_smem();
@@ -664,20 +691,16 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (quarter < 2) {
             const int r = 32 * quarter + lane;
             uint8_t *base = sm + OFF_UB + half * 8 * KB;
+            float v[4][16];
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + TM_U + 64u * half + 16u * gq, v[gq]);
+            tmem_wait_ld();
 #pragma unroll
             for (int gq = 0; gq < 4; ++gq) {
-                float v[16];
-                tmem_ld16(tmem + tlane + TM_U + 64u * half + 16u * gq, v);
-                tmem_wait_ld();
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    uint4 w;
-                    w.x = pack_bf2(v[8 * cc + 0], v[8 * cc + 1]);
-                    w.y = pack_bf2(v[8 * cc + 2], v[8 * cc + 3]);
-                    w.z = pack_bf2(v[8 * cc + 4], v[8 * cc + 5]);
-                    w.w = pack_bf2(v[8 * cc + 6], v[8 * cc + 7]);
-                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, 16 * gq + 8 * cc)) = w;
-                }
+                uint4 w0, w1;
+                pack16(v[gq], 1.f, w0, w1);
+                *reinterpret_cast<uint4 *>(base + sw128_offset(r, 16 * gq)) = w0;
+                *reinterpret_cast<uint4 *>(base + sw128_offset(r, 16 * gq + 8)) = w1;
             }
         }
         fence_proxy_async_smem();
@@ -700,21 +723,17 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (quarter >= 2) {
             const int r = 32 * quarter + lane - 64;
             uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(tok0 + r) * H + h) * D + 64 * half);
+            float v[4][16];
 #pragma unroll
-            for (int gq = 0; gq < 4; ++gq) {
-                float v[16];
-                tmem_ld16(tmem + tlane + TM_U + 64u * half + 16u * gq, v);
-                tmem_wait_ld();
-                if (r < Lc) {
+            for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + TM_U + 64u * half + 16u * gq, v[gq]);
+            tmem_wait_ld();
+            if (r < Lc) {
 #pragma unroll
-                    for (int cc = 0; cc < 2; ++cc) {
-                        uint4 w;
-                        w.x = pack_bf2(v[8 * cc + 0], v[8 * cc + 1]);
-                        w.y = pack_bf2(v[8 * cc + 2], v[8 * cc + 3]);
-                        w.z = pack_bf2(v[8 * cc + 4], v[8 * cc + 5]);
-                        w.w = pack_bf2(v[8 * cc + 6], v[8 * cc + 7]);
-                        dst[2 * gq + cc] = w;
-                    }
+                for (int gq = 0; gq < 4; ++gq) {
+                    uint4 w0, w1;
+                    pack16(v[gq], 1.f, w0, w1);
+                    dst[2 * gq] = w0;
+                    dst[2 * gq + 1] = w1;
                 }
             }
         }
@@ -722,23 +741,25 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const float gam = sGamC[si];
             uint8_t *sb = sm + OFF_SB + half * 16 * KB;
 #pragma unroll
-            for (int gq = 0; gq < 4; ++gq) {
-                float sv[16], dv[16];
-                const uint32_t col = 64u * half + 16u * gq;
-                tmem_ld16(tmem + tlane + TM_S + col, sv);
-                tmem_ld16(tmem + tlane + TM_KU + col, dv);
+            for (int gp = 0; gp < 2; ++gp) {
+                float sv[2][16], dv[2][16];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const uint32_t col = 64u * half + 16u * (2 * gp + i);
+                    tmem_ld16(tmem + tlane + TM_S + col, sv[i]);
+                    tmem_ld16(tmem + tlane + TM_KU + col, dv[i]);
+                }
                 tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 16; ++e) sv[e] = fmaf(gam, sv[e], dv[e]);
-                tmem_st16(tmem + tlane + TM_S + col, sv);
+                for (int i = 0; i < 2; ++i) {
+                    const int gq = 2 * gp + i;
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    uint4 w;
-                    w.x = pack_bf2(sv[8 * cc + 0], sv[8 * cc + 1]);
-                    w.y = pack_bf2(sv[8 * cc + 2], sv[8 * cc + 3]);
-                    w.z = pack_bf2(sv[8 * cc + 4], sv[8 * cc + 5]);
-                    w.w = pack_bf2(sv[8 * cc + 6], sv[8 * cc + 7]);
-                    *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq + 8 * cc)) = w;
+                    for (int e = 0; e < 16; ++e) sv[i][e] = fmaf(gam, sv[i][e], dv[i][e]);
+                    tmem_st16(tmem + tlane + TM_S + 64u * half + 16u * gq, sv[i]);
+                    uint4 w0, w1;
+                    pack16(sv[i], 1.f, w0, w1);
+                    *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq)) = w0;
+                    *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq + 8)) = w1;
                 }
             }
             tmem_wait_st();
