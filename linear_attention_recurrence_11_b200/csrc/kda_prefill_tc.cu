@@ -25,10 +25,11 @@
 //     the diagonal blocks, then block rows by distance).
 //  5. tcgen05.mma: [W | Ut] = T Diag(beta) [Gamma*K | V]           (M=128 padded, K=64)
 //  6. tcgen05.mma: [U ; Qt S] = [Ut ; 0] + [-W ; Gamma*Q] S          (M=128, K=128)
-//  7. tcgen05.mma: O = Qt S + P U (rows 64..127),  dS = Kh^T U       (K=64)
-//     with Kh_s = e^{G_C - G_s} k_s; then S <- Diag(Gamma_C) S + dS in fp32
-//     in TMEM (the state never leaves the SM between chunks; its bf16 copy
-//     feeds step 6 of the next chunk).
+//  7. tcgen05.mma: O = Qt S + P U (rows 64..127),  S += Kh^T U      (K=64)
+//     with Kh_s = e^{G_C - G_s} k_s, onto the fp32 state in TMEM that was
+//     scaled by Diag(Gamma_C) while step 6 ran (the state never leaves the SM
+//     between chunks; its bf16 copy feeds step 6 of the next chunk). The
+//     outputs are staged in shared memory and written by TMA tensor stores.
 // The next chunk's tiles are requested as soon as each staging tile has been
 // consumed (g after step 2's cumulative sums, k after step 4, v after step 5,
 // q after step 6), so their HBM latency overlaps the rest of the chunk.
@@ -91,7 +92,7 @@ static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // TMEM columns (512 allocated): the Gram accumulators use the first 64 columns
 // of the W region (read out before the W product is issued).
-constexpr uint32_t TM_GRAM = 0, TM_W = 0, TM_U = 128, TM_KU = 256, TM_S = 384, TM_COLS = 512;
+constexpr uint32_t TM_GRAM = 0, TM_W = 0, TM_U = 128, TM_S = 384, TM_COLS = 512;
 constexpr uint32_t TMA_BYTES = 6 * 8 * KB + 16 * KB;  // q, k, v: 2 boxes of 8 KB each; g: 1 box of 16 KB
 constexpr long long kWaitCycles = 2000000000LL;        // ~1 s at 2 GHz
 constexpr float kLog2e = 1.4426950408889634f;
@@ -225,7 +226,7 @@ __device__ __forceinline__ void tri_inverse_offdiag(const float *AF, float *TF, 
 __global__ void __launch_bounds__(NT, 1)
 kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                      const TcParams prm) {
+                      const __grid_constant__ CUtensorMap tm_o, const TcParams prm) {
     const PrefillArgs &p = prm.a;
     extern __shared__ uint8_t smem_raw[];
     // 1024-byte alignment of the shared-window address (the swizzle patterns key on it)
@@ -269,6 +270,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tma_prefetch_desc(&tm_k);
         tma_prefetch_desc(&tm_v);
         tma_prefetch_desc(&tm_g);
+        tma_prefetch_desc(&tm_o);
     }
     if (warp == 0) {
         tmem_alloc(s_tmem, TM_COLS);
@@ -376,7 +378,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             sBeta[tid] = (tid < Lc) ? __bfloat162float(bnext) : 0.f;
             if (more && tid < len - (ch + 1) * C) bnext = beta[(size_t)(tokn + tid) * H + h];
         }
-        if (Lc < C) {  // zero the rows past the end of the sequence
+        if (Lc < C) {  // zero the q, k, v rows past the end of the sequence (read after the next barrier)
             for (int idx = tid; idx < (C - Lc) * 16; idx += NT) {
                 const int r = Lc + idx / 16, q16 = idx % 16;  // 16-byte piece of a 256-byte row
                 const uint4 z = make_uint4(0, 0, 0, 0);
@@ -384,10 +386,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 *reinterpret_cast<uint4 *>(sm + OFF_WQ + blk * 16 * KB + sw128_offset(64 + r, pc)) = z;
                 *reinterpret_cast<uint4 *>(sm + OFF_KS + blk * 8 * KB + sw128_offset(r, pc)) = z;
                 *reinterpret_cast<uint4 *>(sm + OFF_V + blk * 8 * KB + sw128_offset(r, pc)) = z;
-                *reinterpret_cast<uint4 *>(sm + OFF_G + r * 256 + q16 * 16) = z;
             }
         }
-        __syncthreads();
 
         // ---- phase 1a: cumulative log2-decay inside subtile ti for channels c0..c0+3
         float gl[HR][4];
@@ -395,7 +395,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             float a[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int rr = 0; rr < HR; ++rr) {
-                const uint2 raw = *reinterpret_cast<const uint2 *>(sm + OFF_G + (SUB * ti + HR * hh + rr) * 256 + c0 * 2);
+                const int row = SUB * ti + HR * hh + rr;  // rows past the end of the sequence decay by 1
+                const uint2 raw = row < Lc ? *reinterpret_cast<const uint2 *>(sm + OFF_G + row * 256 + c0 * 2) : make_uint2(0, 0);
                 const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
                 const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
                 a[0] = fmaf(g01.x, kLog2e, a[0]);
@@ -419,6 +420,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int e = 0; e < 4; ++e) sD[ti * D + c0 + e] = gl[HR - 1][e];
             }
         }
+        if (tid == 0) bulk_wait_read_all();  // the previous chunk's staged outputs have been read
         __syncthreads();
         if (more && tid == 0) {  // g tile consumed: start the next chunk's loads
             mbar_arrive_expect_tx(bar_tma, TMA_BYTES);
@@ -620,23 +622,34 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         __syncthreads();
         tri_inverse_offdiag(AF, TF, XS, tid);
-        // T Diag(beta) -> bf16 A operand (rows 0..63), zero rows 64..127
-        for (int idx = tid; idx < 128 * 8; idx += NT) {
-            const int r = idx >> 3, pc = (idx & 7) * 8;
-            uint4 w = make_uint4(0, 0, 0, 0);
-            if (r < C) {
-                const float4 t0 = *reinterpret_cast<const float4 *>(TF + r * LDT + pc);
-                const float4 t1 = *reinterpret_cast<const float4 *>(TF + r * LDT + pc + 4);
-                const float t[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+        // T Diag(beta) -> bf16 A operand (rows 0..63), zero rows 64..127: every thread converts
+        // two 8-column pieces of T (rows r and r + 32, same columns) and zeroes two pieces
+        {
+            const int r = tid >> 3, pc = (tid & 7) * 8;
+            const float4 b0 = *reinterpret_cast<const float4 *>(sBeta + pc);
+            const float4 b1 = *reinterpret_cast<const float4 *>(sBeta + pc + 4);
+            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+            float4 t[2][2];
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                t[i][0] = *reinterpret_cast<const float4 *>(TF + (r + 32 * i) * LDT + pc);
+                t[i][1] = *reinterpret_cast<const float4 *>(TF + (r + 32 * i) * LDT + pc + 4);
+            }
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int ri = r + 32 * i;
+                const float tv[8] = {t[i][0].x, t[i][0].y, t[i][0].z, t[i][0].w, t[i][1].x, t[i][1].y, t[i][1].z, t[i][1].w};
                 float u[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) u[e] = (pc + e <= r) ? t[e] * sBeta[pc + e] : 0.f;
+                for (int e = 0; e < 8; ++e) u[e] = (pc + e <= ri) ? tv[e] * bb[e] : 0.f;
+                uint4 w;
                 w.x = pack_bf2(u[0], u[1]);
                 w.y = pack_bf2(u[2], u[3]);
                 w.z = pack_bf2(u[4], u[5]);
                 w.w = pack_bf2(u[6], u[7]);
+                *reinterpret_cast<uint4 *>(sm + OFF_TB + sw128_offset(ri, pc)) = w;
+                *reinterpret_cast<uint4 *>(sm + OFF_TB + sw128_offset(ri + 64, pc)) = make_uint4(0, 0, 0, 0);
             }
-            *reinterpret_cast<uint4 *>(sm + OFF_TB + sw128_offset(r, pc)) = w;
         }
         fence_proxy_async_smem();
         __syncthreads();
@@ -684,6 +697,23 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mma_chain<D / 16>(tmem + TM_U, A, B, idKM, true);
             mma_commit(bar_mma);
         }
+        // while it runs: S <- Diag(Gamma_C) S in TMEM, so that the dS product below can
+        // accumulate onto the state directly
+        {
+            const float gam = sGamC[si];
+            float sv[4][16];
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + TM_S + 64u * half + 16u * gq, sv[gq]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) sv[gq][e] *= gam;
+                tmem_st16(tmem + tlane + TM_S + 64u * half + 16u * gq, sv[gq]);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+        }
         if (!wait_mma()) { aborted = true; break; }
         if (more && tid == 0) issue_q(tokn);  // rows 64..127 of the [-W ; Qt] operand are free
 
@@ -707,27 +737,39 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tc_fence_before();
         __syncthreads();
 
-        // ---- O = Qt S + P U (rows 64..127 of the same accumulator), dS = Kh^T U
+        // ---- O = Qt S + P U (rows 64..127 of the same accumulator), S += dS = Kh^T U
         if (tid == 0) {
             tc_fence_after();
             Opnd AP{sbase + OFF_PB - 8 * KB, false, 16 * KB, 0};
             Opnd BU{sbase + OFF_UB, true, 0, 8 * KB};
             Opnd AK{sbase + OFF_KHAT, true, 0, 8 * KB};
-            mma_chain<C / 16>(tmem + TM_KU, AK, BU, idMM, false);
+            mma_chain<C / 16>(tmem + TM_S, AK, BU, idMM, true);
             mma_chain<C / 16>(tmem + TM_U, AP, BU, idKM, true);
             mma_commit(bar_mma);
         }
         if (!wait_mma()) { aborted = true; break; }
 
-        // ---- phase 6: outputs and the state update S <- Diag(Gamma_C) S + dS
+        // ---- phase 6: outputs, and the bf16 copy of the updated state. A full chunk of
+        // outputs is staged in the U tile (free now, and already in the 128-byte swizzled
+        // [token][dv] layout a tensor store reads) and written by two TMA stores; the
+        // rows of a partial chunk are stored directly, so nothing lands past the sequence.
         if (quarter >= 2) {
             const int r = 32 * quarter + lane - 64;
-            uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(tok0 + r) * H + h) * D + 64 * half);
             float v[4][16];
 #pragma unroll
             for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + TM_U + 64u * half + 16u * gq, v[gq]);
             tmem_wait_ld();
-            if (r < Lc) {
+            if (Lc == C) {
+                uint8_t *base = sm + OFF_UB + half * 8 * KB;
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) {
+                    uint4 w0, w1;
+                    pack16(v[gq], 1.f, w0, w1);
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, 16 * gq)) = w0;
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, 16 * gq + 8)) = w1;
+                }
+            } else if (r < Lc) {
+                uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(tok0 + r) * H + h) * D + 64 * half);
 #pragma unroll
                 for (int gq = 0; gq < 4; ++gq) {
                     uint4 w0, w1;
@@ -738,36 +780,29 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
         }
         {
-            const float gam = sGamC[si];
             uint8_t *sb = sm + OFF_SB + half * 16 * KB;
+            float sv[4][16];
 #pragma unroll
-            for (int gp = 0; gp < 2; ++gp) {
-                float sv[2][16], dv[2][16];
+            for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + TM_S + 64u * half + 16u * gq, sv[gq]);
+            tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const uint32_t col = 64u * half + 16u * (2 * gp + i);
-                    tmem_ld16(tmem + tlane + TM_S + col, sv[i]);
-                    tmem_ld16(tmem + tlane + TM_KU + col, dv[i]);
-                }
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    const int gq = 2 * gp + i;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) sv[i][e] = fmaf(gam, sv[i][e], dv[i][e]);
-                    tmem_st16(tmem + tlane + TM_S + 64u * half + 16u * gq, sv[i]);
-                    uint4 w0, w1;
-                    pack16(sv[i], 1.f, w0, w1);
-                    *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq)) = w0;
-                    *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq + 8)) = w1;
-                }
+            for (int gq = 0; gq < 4; ++gq) {
+                uint4 w0, w1;
+                pack16(sv[gq], 1.f, w0, w1);
+                *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq)) = w0;
+                *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq + 8)) = w1;
             }
-            tmem_wait_st();
         }
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
+        if (Lc == C && tid == 0) {
+            tma_store_3d(&tm_o, sm + OFF_UB, 0, h, (int)tok0);
+            tma_store_3d(&tm_o, sm + OFF_UB + 8 * KB, 64, h, (int)tok0);
+            bulk_commit();
+        }
     }
+    if (tid == 0) bulk_wait_all();  // the output stores are complete before the CTA exits
 
     if (aborted) {
         if (tid == 0 && p.dev_status) atomicExch(p.dev_status, (int)KDA_ERR_TIMEOUT);
@@ -840,9 +875,10 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a) {
     const size_t tokens = a.cu_seqlens ? (size_t)a.T : (size_t)a.B * (size_t)a.T;
     // A batch without tokens only copies S0 to S_T; the SIMT kernel does that.
     if (tokens == 0) return launch_prefill_simt(a);
-    CUtensorMap mq, mk, mv, mg;
+    CUtensorMap mq, mk, mv, mg, mo;
     if (!make_map(&mq, a.q, tokens, a.H, 64, true) || !make_map(&mk, a.k, tokens, a.H, 64, true) ||
-        !make_map(&mv, a.v, tokens, a.H, 64, true) || !make_map(&mg, a.g, tokens, a.H, 128, false))
+        !make_map(&mv, a.v, tokens, a.H, 64, true) || !make_map(&mg, a.g, tokens, a.H, 128, false) ||
+        !make_map(&mo, a.o, tokens, a.H, 64, true))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(kda_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
@@ -855,7 +891,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a) {
         prm.a.seq_order = order;
     }
     const unsigned grid = (unsigned)((size_t)a.num_units * a.H);
-    kda_prefill_tc_kernel<<<grid, NT, SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, prm);
+    kda_prefill_tc_kernel<<<grid, NT, SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, mo, prm);
     return cudaGetLastError();
 }
 
