@@ -55,13 +55,15 @@ constexpr uint32_t OFF_SB = 32 * KB;    // 32 KB  B operand S (bf16), MN-major [
 constexpr uint32_t OFF_KS = 64 * KB;    // 16 KB  k tile, [tok rows][dk] (2 blocks of 64 channels)
 constexpr uint32_t OFF_V = 80 * KB;     // 16 KB  v: B operand MN-major [tok rows][dv] (2 N-blocks)
 constexpr uint32_t OFF_G = 96 * KB;     // 16 KB  g, plain [64][128] bf16
-constexpr uint32_t OFF_R = 112 * KB;    // 16 KB  Gram right operand, K-major [s rows][dk]; later Kh (MN-major A)
+constexpr uint32_t OFF_R = 112 * KB;    // 16 KB  Gram right operand, K-major [s rows][dk]; then scratch of the inverse
 constexpr uint32_t OFF_PB = 128 * KB;   // 8 KB   rows 64..127 of the A operand [junk ; P], K-major, K = 64
-constexpr uint32_t OFF_L = 136 * KB;    // 80 KB  Gram left operands L3, L2, L1, L0 (compact), then the aliases below
+constexpr uint32_t OFF_L = 136 * KB;    // 80 KB  Gram left operands L3, L2, L1 (compact), Kh, then the aliases below
 constexpr uint32_t OFF_MISC = 216 * KB;
 // L region: compact left operands of column blocks 1..3, L_j has 2 (64 - 16 j) rows (K part,
-// then Q part); block 0's left operand is the [Gamma*K ; Gamma*Q] tile at OFF_WQ. The order
-// keeps every 128-row operand read (from each K-block start) inside the region.
+// then Q part); block 0's left operand is the [Gamma*K ; Gamma*Q] tile at OFF_WQ. A 128-row
+// operand read from a K-block start ends at most 52 KB into the region (block 1, K-block 1;
+// the rows past its own land in accumulator lanes that are never read). Kh, written with the
+// Gram operands and read by the last product of the chunk, sits past that point.
 __host__ __device__ constexpr uint32_t l_rows(int j) { return 2u * (64u - 16u * j); }
 __host__ __device__ constexpr uint32_t l_off(int j) { return j == 3 ? 0u : j == 2 ? 8u * KB : 24u * KB; }
 // aliases inside the L region once the Gram MMAs are done
@@ -73,13 +75,16 @@ constexpr uint32_t OFF_KT = OFF_WQ;
 // the warp-level MMA fragments below read shared memory without bank conflicts: rows of an A
 // fragment are LDA apart (LDA = 4 mod 32), rows of a B fragment LDX apart (LDX = 8 mod 32).
 constexpr int LDA = 68, LDT = 68, LDX = 40;
-constexpr uint32_t OFF_AF = OFF_L + 32 * KB;       // 64 x LDA fp32  A
-constexpr uint32_t OFF_KHAT = OFF_R;               // 16 KB  A operand Kh, MN-major [tok][dk] (the Gram is done)
+constexpr uint32_t OFF_KHAT = OFF_L + 56 * KB;     // 16 KB  A operand Kh, MN-major [tok][dk]
+constexpr uint32_t OFF_AF = OFF_L + 16 * KB;       // 64 x LDA fp32  A          (the Gram is done)
 constexpr uint32_t OFF_UB = OFF_L + 0;             // 16 KB  B operand U, MN-major [tok][dv] (T Diag(beta) is done)
-constexpr uint32_t OFF_TF = OFF_L + 49 * KB;       // 64 x LDT fp32  T
-constexpr uint32_t OFF_XS = OFF_TF + 64 * LDT * 4;  // 32 x LDX fp32 scratch
-static_assert(OFF_AF + 64 * LDA * 4 <= OFF_TF, "A overlaps T");
-static_assert(OFF_XS + 32 * LDX * 4 <= OFF_MISC, "scratch overflows the L region");
+constexpr uint32_t OFF_TF = OFF_L + 33 * KB;       // 64 x LDT fp32  T
+constexpr uint32_t OFF_XS = OFF_R;                 // 32 x LDX fp32 scratch (the Gram is done)
+static_assert(OFF_L + l_off(1) + l_rows(1) * 128 + 16 * KB <= OFF_KHAT, "Gram operand reads reach Kh");
+static_assert(OFF_AF >= OFF_TB + 16 * KB && OFF_AF + 64 * LDA * 4 <= OFF_TF, "A overlaps T Diag(beta) or T");
+static_assert(OFF_TF + 64 * LDT * 4 <= OFF_KHAT, "T overlaps Kh");
+static_assert(OFF_KHAT + 16 * KB <= OFF_MISC, "Kh overflows the L region");
+static_assert(32 * LDX * 4 <= 16 * KB, "scratch overflows the right-operand tile");
 // misc
 constexpr uint32_t OFF_BAR = OFF_MISC;              // 3 mbarriers
 constexpr uint32_t OFF_TMEMADDR = OFF_MISC + 32;
@@ -476,6 +481,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             uint8_t *const qrow = sm + OFF_WQ + cblk * 16 * KB;
             uint8_t *const krow = sm + OFF_KS + cblk * 8 * KB;
             uint8_t *const rrow = sm + OFF_R + cblk * 8 * KB;
+            uint8_t *const khrow = sm + OFF_KHAT + cblk * 8 * KB;
             auto st4 = [](uint8_t *p, float a, float b, float c, float d) {
                 *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf2(a, b), pack_bf2(c, d));
             };
@@ -493,8 +499,13 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 float kx[4], qx[4], kf[4], qf[4];
                 ld4(krow + off_r, kx);
                 ld4(qrow + off_q, qx);
-                // right operand row r (column block ti): k_r e^{G_start(ti) - G_r}
-                st4(rrow + off_r, kx[0] * Fi[rr][0], kx[1] * Fi[rr][1], kx[2] * Fi[rr][2], kx[3] * Fi[rr][3]);
+                // right operand row r (column block ti): k_r e^{G_start(ti) - G_r}; and Kh row r:
+                // k_r e^{G_C - G_r} = (k_r e^{G_start(ti) - G_r}) e^{G_C - G_start(ti)}, both factors bounded
+                float kr[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) kr[e] = kx[e] * Fi[rr][e];
+                st4(rrow + off_r, kr[0], kr[1], kr[2], kr[3]);
+                st4(khrow + off_r, kr[0] * post[0], kr[1] * post[1], kr[2] * post[2], kr[3] * post[3]);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     kf[e] = kx[e] * F[rr][e];
@@ -527,6 +538,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mma_chain<D / 16>(tmem + TM_GRAM + 16u * j, A, B, idG, false);
             mma_commit(bar_gram);
         }
+        if (more && tid == 0) issue_k(tokn);  // the k tile is consumed (Kh is written with the Gram operands)
         {
             const bool ok = mbar_wait_bounded(bar_gram, gram_phase, kWaitCycles);
             gram_phase ^= 1u;
@@ -575,22 +587,6 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         __syncthreads();
 
         // ---- phase 3: T = (I + A)^{-1} (unit lower triangular) by 16 x 16 blocks
-        // Kh = exp(G_C - G_s) * k_s -> KHAT (first, so the exp factors die early)
-        {
-            const uint8_t *krow = sm + OFF_KS + cblk * 8 * KB;
-            uint8_t *khrow = sm + OFF_KHAT + cblk * 8 * KB;
-#pragma unroll
-            for (int rr = 0; rr < HR; ++rr) {
-                const uint32_t off_r = sw128_offset(SUB * ti + HR * hh + rr, cin);
-                const uint2 raw = *reinterpret_cast<const uint2 *>(krow + off_r);
-                const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
-                const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
-                // e^{G_C - G_s} = e^{G_start(ti) - G_s} e^{G_C - G_start(ti)}, both factors bounded
-                const float b0 = x.x * Fi[rr][0] * post[0], b1 = x.y * Fi[rr][1] * post[1];
-                const float b2 = y.x * Fi[rr][2] * post[2], b3 = y.y * Fi[rr][3] * post[3];
-                *reinterpret_cast<uint2 *>(khrow + off_r) = make_uint2(pack_bf2(b0, b1), pack_bf2(b2, b3));
-            }
-        }
         if (warp < NSUB && lane < 16) {
             // diagonal block `warp`: forward substitution by rows (left-looking), one column of
             // T_ii per lane; each row of A_ii is one broadcast read shared by the 16 lanes
@@ -656,7 +652,6 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
         // ---- [W | Ut] = T Diag(beta) [Gamma*K | V]
         if (tid == 0) {
-            if (more) issue_k(tokn);  // the k tile is consumed
             tc_fence_after();
             Opnd A{sbase + OFF_TB, false, 16 * KB, 0};
             Opnd BK{sbase + OFF_KT, true, 0, 16 * KB};
