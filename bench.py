@@ -36,7 +36,7 @@ METRIC = "KDA prefill tokens/s (H=96,d=128) & % tensor peak; decode GB/s vs HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 WORKLOAD_ALIASES = {"prefill": "prefill_h96_T8192_d128_bf16", "varlen": "varlen_h96_8seq_d128_bf16",
                     "b2": "b2_h4_T2048_d128_bf16", "small": "small_f32_T256_d32",
-                    "decode": "decode_n256_h96_d128"}
+                    "decode": "decode_n256_h96_d128", "long": "long_h8_T65536_d128_bf16"}
 
 
 def parse_args():
@@ -226,16 +226,28 @@ def run_ours(args, rank, world, device):
     elem = inp["k"].element_size()
     o = torch.empty((B, T, w.H, w.dv), dtype=dt, device=device)
     ST = torch.empty((N, w.H, w.dv, w.dk), dtype=torch.float32, device=device)
-    ws_n = kda.kda_forward_workspace_size(B, T, w.H, w.dk, w.dv, w.chunk, N, dt)
-    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=device)
     cu = inp.get("cu_seqlens")
-    launches = kda.kda_forward_launches(B, T, w.H, w.dk, w.dv, w.chunk, dt, cu is not None, N, args.path)
+    seg = w.seg_len if (w.seg_len and not w.seqlens) else 0
+    if seg:  # long sequences with few heads: segment-parallel (pairs, scan, replay)
+        ws_n = kda.kda_forward_segmented_workspace_size(B, T, w.H, w.dk, w.dv, w.chunk, dt, seg)
+        launches = kda.kda_forward_segmented_launches(B, T, w.H, w.dk, w.dv, w.chunk, dt, seg, args.path)
+    else:
+        ws_n = kda.kda_forward_workspace_size(B, T, w.H, w.dk, w.dv, w.chunk, N, dt)
+        launches = kda.kda_forward_launches(B, T, w.H, w.dk, w.dv, w.chunk, dt, cu is not None, N, args.path)
+    ws = torch.empty(max(ws_n, 1), dtype=torch.uint8, device=device)
     tc_ok = kda.kda_forward_launches(B, T, w.H, w.dk, w.dv, w.chunk, dt, cu is not None, N, "tc") > 0
     path_used = "tc" if (args.path != "simt" and tc_ok) else "simt"
 
+    def forward(q, k, v, g, beta, S0):
+        if seg:
+            kda.kda_forward_segmented(q, k, v, g, beta, S0, seg_len=seg, chunk=w.chunk, o=o, S_T=ST,
+                                      workspace=ws, path=args.path)
+        else:
+            kda.kda_forward(q, k, v, g, beta, S0, chunk=w.chunk, cu_seqlens=cu, o=o, S_T=ST,
+                            workspace=ws, path=args.path)
+
     def step():
-        kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"],
-                        chunk=w.chunk, cu_seqlens=cu, o=o, S_T=ST, workspace=ws, path=args.path)
+        forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"])
 
     for _ in range(args.warmup):
         step()
@@ -272,8 +284,10 @@ def run_ours(args, rank, world, device):
         "data": "synthetic (seeded: q,k unit-norm N(0,1); v N(0,1); beta sigmoid(N); g -5*sigmoid(N))",
         "config": {"workload": wname, "B": B, "T": T, "H": w.H, "dk": w.dk, "dv": w.dv,
                    "chunk": w.chunk, "num_seqs": N, "kernel_path": path_used,
+                   **({"seg_len": seg, "segments": -(-T // seg) * B} if seg else {}),
                    "l2": f"inputs larger than L2 ({(inp['q'].numel() * elem * 4) / 1e6:.0f} MB read per step)",
-                   "parallelism": f"dp{world} over independent (sequence, head) units"},
+                   "parallelism": f"dp{world} over independent (sequence, head) units"
+                                  + (" (segments of a sequence run as units: KCP pairs, scan, replay)" if seg else "")},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / peaks["hbm_gbs"], "traffic": traffic,
                      "kernel": os.path.basename(kern_src), "kernel_ms": kern_ms,
@@ -286,8 +300,26 @@ def run_ours(args, rank, world, device):
         "clocks": clk.summary(),
     })
 
+    if seg:  # context: the plain prefill on the same workload (one unit per (sequence, head))
+        ws_p = torch.empty(max(kda.kda_forward_workspace_size(B, T, w.H, w.dk, w.dv, w.chunk, N, dt), 1),
+                           dtype=torch.uint8, device=device)
+
+        def plain():
+            kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], chunk=w.chunk,
+                            o=o, S_T=ST, workspace=ws_p, path=args.path)
+        plain()
+        torch.cuda.synchronize(device)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(3):
+            plain()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        res["plain_prefill"] = {"ms_per_step": a.elapsed_time(b) / 3,
+                                "tokens_per_s": tokens / (a.elapsed_time(b) / 3 / 1e3),
+                                "note": "kda_forward on the same inputs, one unit per (sequence, head); outside the timed region"}
     if not args.no_e2e:
-        res["e2e"] = e2e_prefill(args, device, inp, w, o, ST, ws, cu, world, barrier, max_ranks)
+        res["e2e"] = e2e_prefill(args, device, inp, w, forward, o, ST, world, barrier, max_ranks)
     if not args.no_decode and args.workload == "prefill":
         res["decode"] = decode_measure(args, device, peaks, barrier, max_ranks, world,
                                        steps=args.decode_steps)
@@ -297,7 +329,7 @@ def run_ours(args, rank, world, device):
     return res
 
 
-def e2e_prefill(args, device, inp, w, o, ST, ws, cu, world, barrier, max_ranks):
+def e2e_prefill(args, device, inp, w, forward, o, ST, world, barrier, max_ranks):
     """Same metric through the public API from pinned host buffers: per step,
     H2D of q,k,v,g,beta(,S0), the prefill, D2H of o and S_T."""
     import torch
@@ -314,8 +346,7 @@ def e2e_prefill(args, device, inp, w, o, ST, ws, cu, world, barrier, max_ranks):
     def step():
         for n in names:
             dev[n].copy_(host[n], non_blocking=True)
-        kda.kda_forward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev.get("S0"),
-                        chunk=w.chunk, cu_seqlens=cu, o=o, S_T=ST, workspace=ws, path=args.path)
+        forward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev.get("S0"))
         o_h.copy_(o, non_blocking=True)
         S_h.copy_(ST, non_blocking=True)
 

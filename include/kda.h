@@ -154,6 +154,38 @@ int kda_forward_noalloc(const void *q, const void *k, const void *v, const void 
                         int num_seqs, int *dev_status, void *stream);
 
 /*
+ * Segment-parallel prefill for long sequences with few heads (KCP scan, after
+ * "Exercices", Q21-Q22 and the 4-rank scan of the pages' check script).
+ *
+ * Same results as kda_forward on B dense sequences of T tokens (no cu_seqlens),
+ * computed differently: each sequence is cut into P = ceil(T / seg_len)
+ * segments that run as independent (segment, head) units. Pass A computes each
+ * segment's transition M_p (the recurrence from S = I with zero values), pass
+ * B its local state S~_p (from S = 0), an fp32 scan composes
+ * S_in,p+1 = M_p S_in,p + S~_p from S_in,0 = S0 (its last value is S_T), and
+ * pass C replays every segment from S_in,p to write o. The passes read the
+ * inputs three times and add a d x d product per segment, so this only pays
+ * when (sequences x heads) is well below the SM count and T is long.
+ *
+ *   seg_len : tokens per segment, a positive multiple of chunk. With P = 1
+ *             the call is kda_forward_ex.
+ *   workspace / workspace_bytes : device scratch of at least
+ *             kda_forward_segmented_workspace_size(...) bytes: for P > 1,
+ *             3 x B P H x 64 KiB of fp32 states at d = 128 plus a few bytes per
+ *             segment. Scratch only; contents on entry do not matter.
+ *   path    : kda_path, as in kda_forward_ex.
+ * Other arguments, layouts and errors as kda_forward (S_T may alias S0).
+ */
+size_t kda_forward_segmented_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int dtype,
+                                            int seg_len);
+int kda_forward_segmented_launches(int B, int T, int H, int dk, int dv, int chunk, int dtype, int seg_len,
+                                   int path);
+int kda_forward_segmented(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                          const float *S0, void *o, float *S_T, int B, int T, int H, int dk, int dv, int chunk,
+                          int dtype, int seg_len, void *workspace, size_t workspace_bytes, int *dev_status,
+                          void *stream, int path);
+
+/*
  * One decode step: one new token for each of N requests, states in place.
  * Same recurrence with T = 1 ("Exercices", Q4: decode is bound by memory
  * bandwidth; each state is read and written exactly once).

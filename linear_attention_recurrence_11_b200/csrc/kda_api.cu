@@ -112,6 +112,69 @@ int kda_forward(const void *q, const void *k, const void *v, const void *g, cons
                           num_seqs, workspace, workspace_bytes, dev_status, stream, KDA_PATH_AUTO);
 }
 
+namespace {
+// Shared validation of kda_forward_segmented and its queries; fills s (not the pointers).
+int check_segmented(int B, int T, int H, int dk, int dv, int chunk, int dtype, int seg_len, int path,
+                    kda::SegmentedArgs *s, bool *tc_pair, bool *tc_state) {
+    kda::PrefillArgs a{};
+    int st = check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, false, 0, path, &a);
+    if (st) return st;
+    if (seg_len <= 0 || seg_len % chunk != 0) return KDA_ERR_INVALID_ARG;
+    const long long P = T == 0 ? 0 : ((long long)T + seg_len - 1) / seg_len;
+    if (P > 1) {  // the segments run as packed sequences of one flat token axis
+        if ((long long)B * T > 0x7fffffffLL || (long long)B * P > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+        if ((size_t)(B * P) * (size_t)H * (size_t)(dv > dk ? dv : dk) / 32 > 0x7fffffffu) return KDA_ERR_UNSUPPORTED;
+        if (path == KDA_PATH_TC && !kda::prefill_tc_supported(dk, dk, chunk, dtype)) return KDA_ERR_UNSUPPORTED;
+    }
+    *s = kda::SegmentedArgs{};
+    s->B = B; s->T = T; s->H = H; s->dk = dk; s->dv = dv; s->chunk = chunk; s->dtype = dtype;
+    s->seg_len = seg_len; s->P = (int)P;
+    *tc_pair = path != KDA_PATH_SIMT && kda::prefill_tc_supported(dk, dk, chunk, dtype);
+    *tc_state = path != KDA_PATH_SIMT && kda::prefill_tc_supported(dk, dv, chunk, dtype);
+    return KDA_OK;
+}
+}  // namespace
+
+size_t kda_forward_segmented_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int dtype,
+                                            int seg_len) {
+    kda::SegmentedArgs s;
+    bool tp, ts;
+    if (check_segmented(B, T, H, dk, dv, chunk, dtype, seg_len, KDA_PATH_AUTO, &s, &tp, &ts)) return (size_t)-1;
+    if (s.P <= 1) return kda_forward_workspace_size(B, T, H, dk, dv, chunk, B, dtype);
+    return kda::segmented_workspace(s);
+}
+
+int kda_forward_segmented_launches(int B, int T, int H, int dk, int dv, int chunk, int dtype, int seg_len,
+                                   int path) {
+    kda::SegmentedArgs s;
+    bool tp, ts;
+    if (check_segmented(B, T, H, dk, dv, chunk, dtype, seg_len, path, &s, &tp, &ts)) return -1;
+    if (s.P <= 1) return kda_forward_launches(B, T, H, dk, dv, chunk, dtype, 0, B, path);
+    return kda::segmented_launches(s);
+}
+
+int kda_forward_segmented(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                          const float *S0, void *o, float *S_T, int B, int T, int H, int dk, int dv, int chunk,
+                          int dtype, int seg_len, void *workspace, size_t workspace_bytes, int *dev_status,
+                          void *stream, int path) {
+    kda::SegmentedArgs s;
+    bool tc_pair, tc_state;
+    int st = check_segmented(B, T, H, dk, dv, chunk, dtype, seg_len, path, &s, &tc_pair, &tc_state);
+    if (st) return st;
+    if (s.P <= 1)  // one segment: the plain prefill
+        return kda_forward_ex(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, dtype, nullptr, 0, workspace,
+                              workspace_bytes, dev_status, stream, path);
+    if (!q || !k || !v || !g || !beta || !o) return KDA_ERR_INVALID_ARG;
+    for (const void *p : {q, k, v, g, beta, (const void *)S0, (const void *)o, (const void *)S_T,
+                          (const void *)workspace, (const void *)dev_status})
+        if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
+    s.q = q; s.k = k; s.v = v; s.g = g; s.beta = beta; s.S0 = S0; s.o = o; s.ST = S_T;
+    s.workspace = workspace; s.workspace_bytes = workspace_bytes; s.dev_status = dev_status;
+    s.stream = static_cast<cudaStream_t>(stream);
+    if (workspace == nullptr || workspace_bytes < kda::segmented_workspace(s)) return KDA_ERR_WORKSPACE;
+    return kda::launch_segmented(s, tc_pair, tc_state) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 int kda_decode_step(const void *q, const void *k, const void *v, const void *g, const void *beta,
                     float *S, void *o, int N, int H, int dk, int dv, int dtype, void *stream) {
     if (N <= 0 || H <= 0 || !dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;

@@ -11,6 +11,8 @@
 namespace kda {
 
 // Arguments of one prefill call, as validated by the C ABI layer.
+// Prefill arguments. Inside the library (the segment-pair pass of kda_forward_segmented)
+// v may be null, meaning all-zero values, and o may be null, meaning no outputs.
 struct PrefillArgs {
     const void *q, *k, *v, *g, *beta;
     const float *S0;
@@ -20,6 +22,20 @@ struct PrefillArgs {
     const int32_t *seq_order;   // device: block b runs sequence seq_order[b / H] (nullptr: b / H)
     int B, T, H, dk, dv, chunk, dtype;
     int num_units;              // N: sequences (B, or num_seqs with cu_seqlens)
+    void *workspace;
+    size_t workspace_bytes;
+    int *dev_status;
+    cudaStream_t stream;
+};
+
+// kda_forward_segmented: B dense sequences of T tokens, each cut into P = ceil(T / seg_len)
+// segments that run as independent units (kda_segmented.cu).
+struct SegmentedArgs {
+    const void *q, *k, *v, *g, *beta;
+    const float *S0;
+    void *o;
+    float *ST;
+    int B, T, H, dk, dv, chunk, dtype, seg_len, P;
     void *workspace;
     size_t workspace_bytes;
     int *dev_status;
@@ -60,6 +76,10 @@ size_t prefill_simt_workspace(const PrefillArgs &a);
 int prefill_simt_launches(const PrefillArgs &a);
 
 bool prefill_tc_supported(int dk, int dv, int chunk, int dtype);
+size_t segmented_workspace(const SegmentedArgs &s);
+int segmented_launches(const SegmentedArgs &s);
+// tc_pair / tc_state: run the M_p pass (dv = dk) / the other passes on the tensor-core kernel
+cudaError_t launch_segmented(const SegmentedArgs &s, bool tc_pair, bool tc_state);
 cudaError_t launch_prefill_tc(const PrefillArgs &a);
 size_t prefill_tc_workspace(const PrefillArgs &a);
 int prefill_tc_launches(const PrefillArgs &a);

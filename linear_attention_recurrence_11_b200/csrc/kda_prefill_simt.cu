@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_simt_kernel(const Pre
         }
         for (int idx = tid; idx < C * DVB; idx += kThreads) {
             const int r = idx / DVB, j = idx % DVB;
-            sU[r * UP + j] = (r < Lc) ? ld_elem(v, ((t_begin + c0 + r) * H + h) * dv + j0 + j) : 0.f;
+            sU[r * UP + j] = (r < Lc && v) ? ld_elem(v, ((t_begin + c0 + r) * H + h) * dv + j0 + j) : 0.f;
         }
         for (int r = tid; r < C; r += kThreads)
             sB[r] = (r < Lc) ? ld_elem(beta, (t_begin + c0 + r) * H + h) : 0.f;
@@ -174,8 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_simt_kernel(const Pre
         }
         __syncthreads();
 
-        // O = (Gamma * Q) S + P U, rows < Lc stored
-        {
+        // O = (Gamma * Q) S + P U, rows < Lc stored (no outputs when o is null)
+        if (o) {
             const int j = tid % DVB, r0 = tid / DVB;
             constexpr int RS = kThreads / DVB;
             for (int r = r0; r < Lc; r += RS) {

@@ -106,9 +106,6 @@ struct TcParams {
     PrefillArgs a;
 };
 
-__device__ __forceinline__ float2 ld_bf2(const uint8_t *p) {
-    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
-}
 __device__ __forceinline__ void st_bf2(uint8_t *p, float x, float y) {
     *reinterpret_cast<__nv_bfloat162 *>(p) = __floats2bfloat162_rn(x, y);
 }
@@ -292,12 +289,14 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tma_load_3d(sm + OFF_KS + 8 * KB, &tm_k, bar_tma, 64, h, (int)tok);
     };
     auto issue_v = [&](long long tok) {
+        if (!p.v) return;  // all-zero values: the V tile is zeroed once below
         tma_load_3d(sm + OFF_V, &tm_v, bar_tma, 0, h, (int)tok);
         tma_load_3d(sm + OFF_V + 8 * KB, &tm_v, bar_tma, 64, h, (int)tok);
     };
+    const uint32_t tma_bytes = p.v ? TMA_BYTES : TMA_BYTES - 16 * KB;
     auto issue_g = [&](long long tok) { tma_load_3d(sm + OFF_G, &tm_g, bar_tma, 0, h, (int)tok); };
     if (nchunks > 0 && tid == 0) {
-        mbar_arrive_expect_tx(bar_tma, TMA_BYTES);
+        mbar_arrive_expect_tx(bar_tma, tma_bytes);
         issue_g(t_begin);
         issue_k(t_begin);
         issue_v(t_begin);
@@ -307,6 +306,10 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     __nv_bfloat16 bnext = __float2bfloat16(0.f);
     if (tid < C && tid < len) bnext = beta[(size_t)(t_begin + tid) * H + h];
 
+    if (!p.v) {  // all-zero values (the segment-pair pass): zero the V tile once
+        for (int idx = tid; idx < 16 * KB / 16; idx += NT)
+            *reinterpret_cast<uint4 *>(sm + OFF_V + 16 * idx) = make_uint4(0, 0, 0, 0);
+    }
     // Incoming state -> TMEM (fp32, lane = dk row, column = dv) and its bf16 copy
     // (B operand, MN-major: row = dk index, 64 dv per 128-byte row, N-block = half).
     tc_fence_after();
@@ -428,7 +431,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (tid == 0) bulk_wait_read_all();  // the previous chunk's staged outputs have been read
         __syncthreads();
         if (more && tid == 0) {  // g tile consumed: start the next chunk's loads
-            mbar_arrive_expect_tx(bar_tma, TMA_BYTES);
+            mbar_arrive_expect_tx(bar_tma, tma_bytes);
             issue_g(tokn);
         }
 
@@ -748,7 +751,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // outputs is staged in the U tile (free now, and already in the 128-byte swizzled
         // [token][dv] layout a tensor store reads) and written by two TMA stores; the
         // rows of a partial chunk are stored directly, so nothing lands past the sequence.
-        if (quarter >= 2) {
+        if (quarter >= 2 && p.o) {
             const int r = 32 * quarter + lane - 64;
             float v[4][16];
 #pragma unroll
@@ -791,7 +794,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (Lc == C && tid == 0) {
+        if (Lc == C && tid == 0 && p.o) {
             tma_store_3d(&tm_o, sm + OFF_UB, 0, h, (int)tok0);
             tma_store_3d(&tm_o, sm + OFF_UB + 8 * KB, 64, h, (int)tok0);
             bulk_commit();
@@ -870,10 +873,12 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a) {
     const size_t tokens = a.cu_seqlens ? (size_t)a.T : (size_t)a.B * (size_t)a.T;
     // A batch without tokens only copies S0 to S_T; the SIMT kernel does that.
     if (tokens == 0) return launch_prefill_simt(a);
+    // v and o may be null inside the library (zero values, no outputs): their maps are then
+    // copies of q's and are never used
     CUtensorMap mq, mk, mv, mg, mo;
     if (!make_map(&mq, a.q, tokens, a.H, 64, true) || !make_map(&mk, a.k, tokens, a.H, 64, true) ||
-        !make_map(&mv, a.v, tokens, a.H, 64, true) || !make_map(&mg, a.g, tokens, a.H, 128, false) ||
-        !make_map(&mo, a.o, tokens, a.H, 64, true))
+        !make_map(&mv, a.v ? a.v : a.q, tokens, a.H, 64, true) || !make_map(&mg, a.g, tokens, a.H, 128, false) ||
+        !make_map(&mo, a.o ? a.o : a.q, tokens, a.H, 64, true))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(kda_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);

@@ -1,0 +1,196 @@
+// Segment-parallel prefill: the KCP pair of every segment, a scan over the
+// pairs, and a replay of every segment from its true incoming state
+// ("Exercices", Q21-Q22: a segment maps an incoming state S to M S + S~, and
+// pairs compose as (M2, S~2) o (M1, S~1) = (M2 M1, M2 S~1 + S~2); the pages'
+// check script applies the same scan to a sequence split over 4 ranks).
+//
+// A long sequence with few heads has few (sequence, head) units, so the plain
+// prefill leaves most SMs idle while each unit walks its chunks in order. Here
+// each sequence is cut into segments of seg_len tokens that run as independent
+// units in three passes over the tokens:
+//   pass A  M_p  = the segment's transition: the prefill recurrence run from
+//                  S = I with all values v = 0 (then S_out = M_p I + 0);
+//   pass B  S~_p = the segment's local state: the recurrence run from S = 0;
+//   scan    S_in,0 = S0, S_in,p+1 = M_p S_in,p + S~_p (fp32, one CTA per
+//           (sequence, head), sequential over segments; the last one is S_T);
+//   pass C  the recurrence run over every segment from S_in,p, writing o.
+// Passes A-C are the ordinary prefill kernels over the segments laid out as
+// packed sequences. M_p is a dk x dk matrix kept in the state layout
+// ([column][dk], so pass A runs with dv = dk).
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kSegThreads = 256;
+
+// cu_seg[u] for the B * P segments (segment p of sequence b is unit b * P + p) and the
+// identity as the starting "state" of pass A, [B * P, H, dk, dk] in the state layout.
+__global__ void kda_segment_init_kernel(int32_t *cu_seg, float *Mbuf, int B, int T, int P, int seg_len,
+                                        int H, int dk) {
+    const int units = B * P;
+    const size_t gid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const size_t stride = (size_t)gridDim.x * blockDim.x;
+    for (size_t u = gid; u <= (size_t)units; u += stride) {
+        if (u == (size_t)units) {
+            cu_seg[u] = B * T;
+        } else {
+            const int b = (int)(u / P), p = (int)(u % P);
+            cu_seg[u] = b * T + p * seg_len;
+        }
+    }
+    const size_t n = (size_t)units * H * dk * dk;
+    for (size_t i = gid; i < n; i += stride) {
+        const size_t e = i % ((size_t)dk * dk);
+        Mbuf[i] = (e / dk == e % dk) ? 1.f : 0.f;
+    }
+}
+
+// One CTA per (sequence b, head h): X <- S0 (or 0); for p = 0..P-1 { Sin[p] = X;
+// X = X Ms_p + Zs_p }; S_T = X. In the state layout X is [dv][dk] (X[j][i] = S[i][j]),
+// Ms_p is [dk][dk] (Ms[a][i] = M_p[i][a]) and Zs_p is [dv][dk], so M_p S + S~_p is
+// the plain row-major product X Ms + Zs, in fp32. Thread (tj, ti) owns rows
+// j = tj + 16 r and columns i = ti + 16 c, so that a warp's shared-memory reads of
+// Ms are consecutive; X is kept transposed with an odd row stride (no bank conflicts
+// on its column-wise writes).
+template <int DK, int DV>
+__global__ void __launch_bounds__(kSegThreads)
+kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float *Sin, float *ST, int P, int H) {
+    constexpr int TJ = DV / 16, TI = DK / 16, XS = DV + 1;
+    extern __shared__ float smem[];
+    float *XT = smem;            // XT[a * XS + j] = X[j][a]
+    float *Ms = smem + DK * XS;  // Ms[a * DK + i]
+    const int b = blockIdx.x / H, h = blockIdx.x % H, tid = threadIdx.x;
+    const int tj = tid / 16, ti = tid % 16;
+    const size_t sbase = ((size_t)b * H + h) * DV * DK;
+    for (int e = tid; e < DV * DK; e += kSegThreads) XT[(e % DK) * XS + e / DK] = S0 ? S0[sbase + e] : 0.f;
+    for (int p = 0; p < P; ++p) {
+        const size_t u = (size_t)b * P + p;
+        const size_t xbase = (u * H + h) * DV * DK, mbase = (u * H + h) * DK * DK;
+        for (int e = tid; e < DK * DK; e += kSegThreads) Ms[e] = Mbuf[mbase + e];
+        __syncthreads();
+        for (int e = tid; e < DV * DK; e += kSegThreads) Sin[xbase + e] = XT[(e % DK) * XS + e / DK];
+        float acc[TJ][TI];
+#pragma unroll
+        for (int r = 0; r < TJ; ++r)
+#pragma unroll
+            for (int c = 0; c < TI; ++c) acc[r][c] = Zbuf[xbase + (size_t)(tj + 16 * r) * DK + ti + 16 * c];
+#pragma unroll 4
+        for (int a = 0; a < DK; ++a) {
+            float xv[TJ], mv[TI];
+#pragma unroll
+            for (int r = 0; r < TJ; ++r) xv[r] = XT[a * XS + tj + 16 * r];
+#pragma unroll
+            for (int c = 0; c < TI; ++c) mv[c] = Ms[a * DK + ti + 16 * c];
+#pragma unroll
+            for (int r = 0; r < TJ; ++r)
+#pragma unroll
+                for (int c = 0; c < TI; ++c) acc[r][c] = fmaf(xv[r], mv[c], acc[r][c]);
+        }
+        __syncthreads();  // every thread has read X and Ms_p
+#pragma unroll
+        for (int r = 0; r < TJ; ++r)
+#pragma unroll
+            for (int c = 0; c < TI; ++c) XT[(ti + 16 * c) * XS + tj + 16 * r] = acc[r][c];
+        __syncthreads();
+    }
+    if (ST)
+        for (int e = tid; e < DV * DK; e += kSegThreads) ST[sbase + e] = XT[(e % DK) * XS + e / DK];
+}
+
+template <int DK, int DV>
+cudaError_t launch_scan_t(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin) {
+    const size_t smem = (size_t)(DK * (DV + 1) + DK * DK) * sizeof(float);
+    cudaError_t e = cudaFuncSetAttribute(kda_kcp_scan_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    kda_kcp_scan_kernel<DK, DV><<<s.B * s.H, kSegThreads, smem, s.stream>>>(s.S0, Mbuf, Zbuf, Sin, s.ST, s.P, s.H);
+    return cudaGetLastError();
+}
+
+template <int DK>
+cudaError_t launch_scan_dv(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin) {
+    switch (s.dv) {
+        case 32: return launch_scan_t<DK, 32>(s, Mbuf, Zbuf, Sin);
+        case 64: return launch_scan_t<DK, 64>(s, Mbuf, Zbuf, Sin);
+        case 128: return launch_scan_t<DK, 128>(s, Mbuf, Zbuf, Sin);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_scan(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin) {
+    switch (s.dk) {
+        case 32: return launch_scan_dv<32>(s, Mbuf, Zbuf, Sin);
+        case 64: return launch_scan_dv<64>(s, Mbuf, Zbuf, Sin);
+        case 128: return launch_scan_dv<128>(s, Mbuf, Zbuf, Sin);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Workspace carve-up (all pieces 256-byte aligned).
+struct SegLayout {
+    size_t cu, order, M, Z, Sin, total;
+};
+SegLayout seg_layout(const SegmentedArgs &s) {
+    const size_t units = (size_t)s.B * s.P;
+    SegLayout L;
+    L.cu = 0;
+    L.order = L.cu + align256((units + 1) * sizeof(int32_t));
+    L.M = L.order + seq_order_bytes((int)units);
+    L.Z = L.M + align256(units * s.H * s.dk * s.dk * sizeof(float));
+    L.Sin = L.Z + align256(units * s.H * s.dv * s.dk * sizeof(float));
+    L.total = L.Sin + align256(units * s.H * s.dv * s.dk * sizeof(float));
+    return L;
+}
+
+cudaError_t run_pass(const PrefillArgs &a, bool tc) { return tc ? launch_prefill_tc(a) : launch_prefill_simt(a); }
+
+}  // namespace
+
+size_t segmented_workspace(const SegmentedArgs &s) { return s.P <= 1 ? 0 : seg_layout(s).total; }
+
+int segmented_launches(const SegmentedArgs &s) {
+    const int order = seq_order_bytes(s.B * s.P) > 0 ? 1 : 0;
+    return 1 /* init */ + 3 * (1 + order) /* passes A, B, C */ + 1 /* scan */;
+}
+
+cudaError_t launch_segmented(const SegmentedArgs &s, bool tc_pair, bool tc_state) {
+    const SegLayout L = seg_layout(s);
+    uint8_t *ws = static_cast<uint8_t *>(s.workspace);
+    int32_t *cu_seg = reinterpret_cast<int32_t *>(ws + L.cu);
+    float *Mbuf = reinterpret_cast<float *>(ws + L.M);
+    float *Zbuf = reinterpret_cast<float *>(ws + L.Z);
+    float *Sin = reinterpret_cast<float *>(ws + L.Sin);
+    const int units = s.B * s.P;
+
+    kda_segment_init_kernel<<<296, kSegThreads, 0, s.stream>>>(cu_seg, Mbuf, s.B, s.T, s.P, s.seg_len, s.H, s.dk);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    PrefillArgs a{};
+    a.q = s.q; a.k = s.k; a.g = s.g; a.beta = s.beta;
+    a.cu_seqlens = cu_seg;
+    a.B = 1; a.T = s.B * s.T; a.H = s.H; a.dk = s.dk; a.chunk = s.chunk; a.dtype = s.dtype;
+    a.num_units = units;
+    a.workspace = ws + L.order; a.workspace_bytes = seq_order_bytes(units);
+    a.dev_status = s.dev_status; a.stream = s.stream;
+
+    // pass A: M_p, from the identity with zero values (dv = dk: M_p is dk x dk)
+    PrefillArgs pa = a;
+    pa.v = nullptr; pa.o = nullptr; pa.S0 = Mbuf; pa.ST = Mbuf; pa.dv = s.dk;
+    if ((e = run_pass(pa, tc_pair)) != cudaSuccess) return e;
+    // pass B: S~_p, from zero
+    PrefillArgs pb = a;
+    pb.v = s.v; pb.o = nullptr; pb.S0 = nullptr; pb.ST = Zbuf; pb.dv = s.dv;
+    if ((e = run_pass(pb, tc_state)) != cudaSuccess) return e;
+    // scan: incoming state of every segment, and S_T
+    if ((e = launch_scan(s, Mbuf, Zbuf, Sin)) != cudaSuccess) return e;
+    // pass C: outputs, every segment from its incoming state
+    PrefillArgs pc = a;
+    pc.v = s.v; pc.o = s.o; pc.S0 = Sin; pc.ST = nullptr; pc.dv = s.dv;
+    return run_pass(pc, tc_state);
+}
+
+}  // namespace kda

@@ -43,6 +43,7 @@ class Workload:
     s0_std: float = 0.0             # 0 -> no initial state (zeros)
     g_min_frac: float = 0.0         # fraction of g elements set to exactly g_min
     decode_steps: int = 0           # >0: a decode workload (T = 1 per step)
+    seg_len: int = 0                # >0: run segment-parallel (segments of seg_len tokens)
     seed: int = 1000
     notes: str = ""
 
@@ -88,6 +89,11 @@ WORKLOADS = {
         name="varlen_h96_8seq_d128_bf16", B=1, H=96, dk=128, dv=128, dtype="bf16", chunk=64,
         seqlens=varlen_lengths(8, 4096, 131072, seed=1003), seed=1003,
         notes="8 packed sequences, log-uniform lengths in [4096, 131072]"),
+    "long_h8_T65536_d128_bf16": Workload(
+        name="long_h8_T65536_d128_bf16", B=1, H=8, T=65536, dk=128, dv=128, dtype="bf16",
+        chunk=64, g_min_frac=0.10, seg_len=4096, seed=1005,
+        notes="one long sequence with few heads (8 units on a 148-SM GPU): segment-parallel, "
+              "16 segments of 4096 tokens"),
     "decode_n256_h96_d128": Workload(
         name="decode_n256_h96_d128", B=256, H=96, T=1, dk=128, dv=128, dtype="bf16",
         chunk=64, s0_std=0.02, decode_steps=1000, seed=1004,

@@ -131,3 +131,45 @@ def test_python_binding_refuses_cpu_tensors(K):
     x = torch.zeros(1, 4, 1, 32)
     with pytest.raises(ValueError, match="CUDA"):
         K.kda_forward(x, x, x, x, torch.zeros(1, 4, 1))
+
+
+def seg(K, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, S0=None, o=FAKE, S_T=None, B=1, T=1000, H=2,
+             dk=128, dv=128, chunk=64, dtype=1, seg_len=256, ws=None, ws_bytes=0, status=None, stream=None,
+             path=0)
+    a.update(kw)
+    return K._lib.kda_forward_segmented(a["q"], a["k"], a["v"], a["g"], a["beta"], a["S0"], a["o"], a["S_T"],
+                                        a["B"], a["T"], a["H"], a["dk"], a["dv"], a["chunk"], a["dtype"],
+                                        a["seg_len"], a["ws"], a["ws_bytes"], a["status"], a["stream"],
+                                        a["path"])
+
+
+def test_segmented_rejects_bad_arguments(K):
+    assert seg(K, seg_len=0) == K.KDA_ERR_INVALID_ARG
+    assert seg(K, seg_len=100) == K.KDA_ERR_INVALID_ARG          # not a multiple of chunk
+    assert seg(K, seg_len=-64) == K.KDA_ERR_INVALID_ARG
+    assert seg(K, dk=48) == K.KDA_ERR_UNSUPPORTED
+    assert seg(K, v=None) == K.KDA_ERR_INVALID_ARG
+    assert seg(K, o=None) == K.KDA_ERR_INVALID_ARG
+    assert seg(K, q=FAKE + 4) == K.KDA_ERR_ALIGNMENT
+    # four segments need the workspace: missing or short -> rejected before launch
+    assert seg(K) == K.KDA_ERR_WORKSPACE
+    assert seg(K, ws=FAKE, ws_bytes=1024) == K.KDA_ERR_WORKSPACE
+    # fp32 never takes the tensor-core kernel
+    assert seg(K, dtype=0, path=K.PATHS["tc"]) == K.KDA_ERR_UNSUPPORTED
+
+
+def test_segmented_queries(K):
+    # 4 segments x 2 heads: three fp32 128 x 128 states per (segment, head) plus offsets
+    n = K.kda_forward_segmented_workspace_size(1, 1000, 2, 128, 128, 64, 1, 256)
+    assert n >= 3 * 4 * 2 * 128 * 128 * 4 and n < 3 * 4 * 2 * 128 * 128 * 4 + 4096
+    # the transition of a dk = 64 segment is 64 x 64 whatever dv is
+    n2 = K.kda_forward_segmented_workspace_size(1, 1000, 2, 64, 128, 64, 1, 256)
+    assert n2 >= 4 * 2 * (64 * 64 + 2 * 128 * 64) * 4
+    # one segment: the plain prefill's needs (none for a dense batch)
+    assert K.kda_forward_segmented_workspace_size(2, 1000, 2, 128, 128, 64, 1, 1024) == 0
+    assert K.kda_forward_segmented_launches(2, 1000, 2, 128, 128, 64, 1, 1024) == 1
+    # init, three passes each with a longest-first schedule, scan
+    assert K.kda_forward_segmented_launches(1, 1000, 2, 128, 128, 64, 1, 256) == 8
+    with pytest.raises(K.KdaError):
+        K.kda_forward_segmented_workspace_size(1, 1000, 2, 128, 128, 64, 1, 96)
