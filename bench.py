@@ -47,6 +47,8 @@ def parse_args():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="prefill", choices=sorted(WORKLOAD_ALIASES))
     p.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    p.add_argument("--draft-tokens", type=int, default=4,
+                   help="draft tokens per request in the speculative decode leg (0: skip)")
     p.add_argument("--decode-steps", type=int, default=50)
     p.add_argument("--tokens", type=int, default=0,
                    help="override T of the dense prefill workload (smaller only for profiling captures)")
@@ -405,7 +407,7 @@ def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):
     elem = sets[0]["k"].element_size()
     alg_bytes, _ = decode_algorithmic(w.B, w.H, w.dk, w.dv, elem)
     gbs = alg_bytes / (ms / 1e3) / 1e9
-    return {"metric": f"KDA decode step GB/s ({w.B} req x {w.H} heads, fp32 state)",
+    res = {"metric": f"KDA decode step GB/s ({w.B} req x {w.H} heads, fp32 state)",
             "value": gbs * world, "unit": "GB/s", "ms_per_step": ms,
             "tokens_per_s": world * w.B / (ms / 1e3), "steps": steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -416,6 +418,58 @@ def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):
                          "peak_source": peaks["source"] + " (hbm_gbs)"},
             "gpu_launches": steps, "clocks": clk.summary(),
             "requests": w.B, "l2": f"state {w.B * w.H * w.dk * w.dv * 4 / 1e9:.2f} GB per step, larger than L2"}
+    if args.draft_tokens > 0:
+        res["multi_token"] = multi_decode_measure(args, device, peaks, max_ranks, world, w, S)
+        res["gpu_launches"] += res["multi_token"]["gpu_launches"]
+    return res
+
+
+def multi_decode_measure(args, device, peaks, max_ranks, world, w, S, rounds=10):
+    """Speculative decoding rounds on the same states: T draft tokens per request,
+    a verification call (outputs of all T, states untouched) then a commit call
+    (the state after each request's accepted prefix, no outputs). Acceptance
+    counts are seeded draws in [0, T]."""
+    import torch
+    from linear_attention_recurrence_11_b200 import kda
+    from linear_attention_recurrence_11_b200.inputs import make_inputs
+    T = args.draft_tokens
+    inp = make_inputs(w.B, T, w.H, w.dk, w.dv, "bf16", seed=w.seed + 77, device=device)
+    gen = torch.Generator().manual_seed(w.seed + 78)
+    acc = torch.randint(0, T + 1, (w.B,), generator=gen, dtype=torch.int32).to(device)
+    zeros = torch.zeros_like(acc)
+    o = torch.empty((w.B, T, w.H, w.dv), dtype=inp["k"].dtype, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def round_():
+        kda.kda_decode_multi(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S, o, n_accept=zeros)
+        kda.kda_decode_multi(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S, None, n_accept=acc,
+                             outputs=False)
+
+    for _ in range(3):
+        round_()
+    torch.cuda.synchronize(device)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(rounds):
+        round_()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    ms = max_ranks(a.elapsed_time(b)) / rounds
+    state = w.dk * w.dv * 4
+    per_tok = (3 * w.dk + w.dv + 1) * 2
+    written = int((acc > 0).sum().item())
+    bytes_round = (2 * w.B * w.H * state + written * w.H * state       # two state reads, accepted writes
+                   + 2 * w.B * T * w.H * per_tok + w.B * T * w.H * w.dv * 2)  # inputs twice, outputs once
+    gbs = bytes_round / (ms / 1e3) / 1e9
+    accepted = int(acc.sum().item())
+    return {"draft_tokens": T, "ms_per_round": ms, "accepted_tokens_per_round": accepted * world,
+            "accepted_tokens_per_s": world * accepted / (ms / 1e3),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "kernel": "kda_decode_multi.cu",
+                         "algorithmic_bytes_per_round": bytes_round, "peak_source": peaks["source"] + " (hbm_gbs)"},
+            "gpu_launches": 2 * rounds,
+            "note": "per round: verify (outputs of all draft tokens) + commit (accepted prefixes); "
+                    "kda_decode_step would move the state twice per accepted token instead"}
 
 
 def run_decode_main(args, rank, world, device, w, peaks, barrier, max_ranks):

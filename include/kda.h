@@ -198,6 +198,29 @@ int kda_decode_step(const void *q, const void *k, const void *v, const void *g,
                     const void *beta, float *S, void *o, int N, int H, int dk, int dv,
                     int dtype, void *stream);
 
+/*
+ * Multi-token decode with speculative acceptance ("Exercices", Q27: the state
+ * after an accepted prefix of draft tokens is determined by those tokens'
+ * inputs, so only the inputs are kept, the recurrence is replayed on chip and
+ * the verified state is written back).
+ *
+ * For each request n, T tokens are applied in order to its states, each as
+ * one kda_decode_step; o receives all T outputs (when o is not NULL) and the
+ * state after the first n_accept[n] tokens is written back in place
+ * (n_accept NULL: all T; 0: S[n] is left untouched). Every state is read
+ * once and written at most once, whatever T is.
+ * Typical use: verify T draft tokens with n_accept all zero (outputs only),
+ * then commit with the accepted counts and o = NULL.
+ *
+ *   q, k, g : [N, T, H, dk];  v, o : [N, T, H, dv];  beta : [N, T, H]   (dtype)
+ *   S        : [N, H, dv, dk] fp32, read, and written where n_accept > 0.
+ *   n_accept : device int32 [N] (values clamped to [0, T]) or NULL.
+ *   T        : 1..64 (KDA_ERR_UNSUPPORTED above).
+ */
+int kda_decode_multi(const void *q, const void *k, const void *v, const void *g, const void *beta, float *S,
+                     void *o, const int32_t *n_accept, int N, int T, int H, int dk, int dv, int dtype,
+                     void *stream);
+
 #ifdef __cplusplus
 }
 #endif

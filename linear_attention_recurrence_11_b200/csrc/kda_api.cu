@@ -187,4 +187,18 @@ int kda_decode_step(const void *q, const void *k, const void *v, const void *g, 
     return kda::launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+int kda_decode_multi(const void *q, const void *k, const void *v, const void *g, const void *beta, float *S,
+                     void *o, const int32_t *n_accept, int N, int T, int H, int dk, int dv, int dtype,
+                     void *stream) {
+    if (N <= 0 || T <= 0 || H <= 0 || !dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;
+    if (T > kda::kMaxMultiTokens) return KDA_ERR_UNSUPPORTED;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if ((size_t)N * (size_t)H > 0x7fffffffu || (size_t)N * T * H > 0x7fffffffu) return KDA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !g || !beta || !S) return KDA_ERR_INVALID_ARG;
+    for (const void *p : {q, k, v, g, beta, (const void *)S, (const void *)o, (const void *)n_accept})
+        if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
+    kda::MultiDecodeArgs a{q, k, v, g, beta, S, o, n_accept, N, T, H, dk, dv, dtype, static_cast<cudaStream_t>(stream)};
+    return kda::launch_decode_multi(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 }  // extern "C"

@@ -1,0 +1,190 @@
+// Multi-token decode with speculative acceptance ("Exercices", Q27: the state
+// after any accepted prefix of draft tokens is determined by those tokens'
+// inputs, which are far smaller than the state; so keep only the inputs,
+// replay the recurrence on chip and write back the verified state).
+//
+// Per (request n, head h): T tokens t = 0..T-1 are applied in order to the
+// state S (dk x dv, stored [dv][dk] fp32), each exactly as one decode step
+//   S' = Diag(exp g_t) S,  s = S'^T k_t,  u = beta_t (v_t - s),
+//   S <- S' + k_t u^T,     o_t = S'^T q_t + u (k_t^T q_t)
+// and the state after the first n_acc tokens (n_acc = n_accept[n], or T) is
+// written back in place; n_acc = 0 leaves S untouched. Outputs of all T
+// tokens are written when o is given. A verification pass is n_accept = all
+// zeros (outputs only, S read once and not written); the commit that follows
+// is the same call with the accepted counts and o = NULL.
+//
+// Each state is read from HBM once and written at most once, whatever T is.
+// Every column j of S (a contiguous dk-float row of the stored state) evolves
+// independently of the others through all T tokens (the decay, both dot
+// products and the rank-1 update act column by column), so the kernel streams
+// the state like the single-step decode: one CTA of 4 warps per (request,
+// head), 8 lanes per column with 128-bit loads, two columns in flight per
+// lane, all T tokens applied while a column is in registers, the column
+// written back right after token n_acc. The tokens' q, k, exp(g), beta and v
+// are staged in shared memory first; outputs are collected there and written
+// as contiguous rows at the end.
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kMtThreads = 128;
+constexpr int kMtLanesPerRow = 8;
+constexpr int kMtRowsPerPass = (kMtThreads / 32) * (32 / kMtLanesPerRow);  // 16
+constexpr int kMtRowsInFlight = 2;
+
+template <typename Tin, int DK, int DV>
+__global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const MultiDecodeArgs p) {
+    constexpr int F4 = DK / (4 * kMtLanesPerRow);  // float4 per lane per column
+    constexpr int E = 4 * F4;                      // channels per lane
+    // per token: q, k, exp(g) [DK each], v [DV], beta, padded to 16 bytes; then the outputs [T][DV]
+    constexpr int TOK = 3 * DK + DV + 4;
+    extern __shared__ float sIn[];
+    const Tin *q = static_cast<const Tin *>(p.q), *k = static_cast<const Tin *>(p.k);
+    const Tin *v = static_cast<const Tin *>(p.v), *g = static_cast<const Tin *>(p.g);
+    const Tin *beta = static_cast<const Tin *>(p.beta);
+    Tin *o = static_cast<Tin *>(p.o);
+    const int T = p.T, H = p.H;
+    const size_t unit = blockIdx.x;  // n * H + h
+    const int n = (int)(unit / H), h = (int)(unit % H);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int sub = lane & (kMtLanesPerRow - 1), rw = lane / kMtLanesPerRow;
+
+    // the tokens' inputs -> shared memory (input layout [N, T, H, d])
+    for (int idx = tid; idx < T * TOK; idx += kMtThreads) {
+        const int t = idx / TOK, c = idx % TOK;
+        const size_t tok = ((size_t)n * T + t) * H + h;
+        float x;
+        if (c < DK) x = ld_elem(q, tok * DK + c);
+        else if (c < 2 * DK) x = ld_elem(k, tok * DK + (c - DK));
+        else if (c < 3 * DK) x = __expf(ld_elem(g, tok * DK + (c - 2 * DK)));
+        else if (c < 3 * DK + DV) x = ld_elem(v, tok * DV + (c - 3 * DK));
+        else if (c == 3 * DK + DV) x = ld_elem(beta, tok);
+        else continue;
+        sIn[idx] = x;
+    }
+    float *sOut = sIn + T * TOK;
+    int n_acc = p.n_accept ? p.n_accept[n] : T;
+    n_acc = n_acc < 0 ? 0 : (n_acc > T ? T : n_acc);
+    __syncthreads();
+
+    float *Su = p.S + unit * (size_t)DV * DK;
+    for (int jb = warp * (32 / kMtLanesPerRow) + rw; jb < DV; jb += kMtRowsPerPass * kMtRowsInFlight) {
+        float4 s[kMtRowsInFlight][F4];
+#pragma unroll
+        for (int r = 0; r < kMtRowsInFlight; ++r) {
+            const int j = jb + r * kMtRowsPerPass;  // DV is a multiple of 32: always a valid column
+#pragma unroll
+            for (int m = 0; m < F4; ++m)
+                s[r][m] = __ldcs(reinterpret_cast<const float4 *>(Su + (size_t)j * DK + 4 * (sub + kMtLanesPerRow * m)));
+        }
+        for (int t = 0; t < T; ++t) {
+            const float *in = sIn + t * TOK;
+            float kk[E], qq[E], a[E];
+#pragma unroll
+            for (int m = 0; m < F4; ++m) {
+                const int c = 4 * (sub + kMtLanesPerRow * m);
+                const float4 q4 = *reinterpret_cast<const float4 *>(in + c);
+                const float4 k4 = *reinterpret_cast<const float4 *>(in + DK + c);
+                const float4 a4 = *reinterpret_cast<const float4 *>(in + 2 * DK + c);
+                qq[4 * m] = q4.x; qq[4 * m + 1] = q4.y; qq[4 * m + 2] = q4.z; qq[4 * m + 3] = q4.w;
+                kk[4 * m] = k4.x; kk[4 * m + 1] = k4.y; kk[4 * m + 2] = k4.z; kk[4 * m + 3] = k4.w;
+                a[4 * m] = a4.x; a[4 * m + 1] = a4.y; a[4 * m + 2] = a4.z; a[4 * m + 3] = a4.w;
+            }
+            float kq = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) kq = fmaf(kk[e], qq[e], kq);
+#pragma unroll
+            for (int off = 1; off < kMtLanesPerRow; off <<= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+            const float b = in[3 * DK + DV];
+#pragma unroll
+            for (int r = 0; r < kMtRowsInFlight; ++r) {
+                const int j = jb + r * kMtRowsPerPass;
+                // the tokens of a column are sequential, so the dot products keep four
+                // partial sums each (short dependency chains between tokens)
+                float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int m = 0; m < F4; ++m) {
+                    float *x = reinterpret_cast<float *>(&s[r][m]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        x[e] *= a[4 * m + e];
+                        pk[e] = fmaf(x[e], kk[4 * m + e], pk[e]);
+                        pq[e] = fmaf(x[e], qq[4 * m + e], pq[e]);
+                    }
+                }
+                float sk = (pk[0] + pk[1]) + (pk[2] + pk[3]), sq = (pq[0] + pq[1]) + (pq[2] + pq[3]);
+#pragma unroll
+                for (int off = 1; off < kMtLanesPerRow; off <<= 1) {
+                    sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                }
+                const float u = b * (in[3 * DK + j] - sk);
+#pragma unroll
+                for (int m = 0; m < F4; ++m) {
+                    float *x = reinterpret_cast<float *>(&s[r][m]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) x[e] = fmaf(kk[4 * m + e], u, x[e]);
+                }
+                if (sub == 0) sOut[t * DV + j] = fmaf(u, kq, sq);
+            }
+            if (t + 1 == n_acc) {  // the column after the accepted prefix, in place
+#pragma unroll
+                for (int r = 0; r < kMtRowsInFlight; ++r) {
+                    const int j = jb + r * kMtRowsPerPass;
+#pragma unroll
+                    for (int m = 0; m < F4; ++m)
+                        __stcs(reinterpret_cast<float4 *>(Su + (size_t)j * DK + 4 * (sub + kMtLanesPerRow * m)), s[r][m]);
+                }
+            }
+        }
+    }
+    if (o) {  // outputs, one contiguous dv row per token
+        __syncthreads();
+        for (int idx = tid; idx < T * DV; idx += kMtThreads) {
+            const int t = idx / DV, j = idx % DV;
+            st_elem(o, (((size_t)n * T + t) * H + h) * DV + j, sOut[idx]);
+        }
+    }
+}
+
+template <typename Tin, int DK, int DV>
+cudaError_t launch_mt(const MultiDecodeArgs &a) {
+    const size_t smem = (size_t)a.T * (3 * DK + DV + 4 + DV) * sizeof(float);
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kda_decode_multi_kernel<Tin, DK, DV>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    kda_decode_multi_kernel<Tin, DK, DV><<<(unsigned)((size_t)a.N * a.H), kMtThreads, smem, a.stream>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename Tin, int DK>
+cudaError_t launch_mt_dv(const MultiDecodeArgs &a) {
+    switch (a.dv) {
+        case 32: return launch_mt<Tin, DK, 32>(a);
+        case 64: return launch_mt<Tin, DK, 64>(a);
+        case 128: return launch_mt<Tin, DK, 128>(a);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <typename Tin>
+cudaError_t launch_mt_t(const MultiDecodeArgs &a) {
+    switch (a.dk) {
+        case 32: return launch_mt_dv<Tin, 32>(a);
+        case 64: return launch_mt_dv<Tin, 64>(a);
+        case 128: return launch_mt_dv<Tin, 128>(a);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_decode_multi(const MultiDecodeArgs &a) {
+    if ((size_t)a.N * a.H == 0 || a.T == 0) return cudaSuccess;
+    return a.dtype == KDA_DTYPE_BF16 ? launch_mt_t<__nv_bfloat16>(a) : launch_mt_t<float>(a);
+}
+
+}  // namespace kda

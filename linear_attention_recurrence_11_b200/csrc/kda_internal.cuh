@@ -50,6 +50,17 @@ struct DecodeArgs {
     cudaStream_t stream;
 };
 
+// kda_decode_multi: T tokens per request, the state after n_accept[n] of them written back.
+struct MultiDecodeArgs {
+    const void *q, *k, *v, *g, *beta;
+    float *S;
+    void *o;                   // may be null: no outputs
+    const int32_t *n_accept;   // device [N] or null (all T)
+    int N, T, H, dk, dv, dtype;
+    cudaStream_t stream;
+};
+constexpr int kMaxMultiTokens = 64;
+
 // Element loads/stores in the storage dtype, computed in fp32.
 __device__ __forceinline__ float ld_elem(const float *p, size_t i) { return p[i]; }
 __device__ __forceinline__ float ld_elem(const __nv_bfloat16 *p, size_t i) {
@@ -85,5 +96,6 @@ size_t prefill_tc_workspace(const PrefillArgs &a);
 int prefill_tc_launches(const PrefillArgs &a);
 
 cudaError_t launch_decode(const DecodeArgs &a);
+cudaError_t launch_decode_multi(const MultiDecodeArgs &a);
 
 }  // namespace kda

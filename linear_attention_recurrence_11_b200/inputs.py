@@ -91,9 +91,9 @@ WORKLOADS = {
         notes="8 packed sequences, log-uniform lengths in [4096, 131072]"),
     "long_h8_T65536_d128_bf16": Workload(
         name="long_h8_T65536_d128_bf16", B=1, H=8, T=65536, dk=128, dv=128, dtype="bf16",
-        chunk=64, g_min_frac=0.10, seg_len=4096, seed=1005,
+        chunk=64, g_min_frac=0.10, seg_len=3648, seed=1005,
         notes="one long sequence with few heads (8 units on a 148-SM GPU): segment-parallel, "
-              "16 segments of 4096 tokens"),
+              "18 segments of 57 chunks (the last 55), 144 (segment, head) units"),
     "decode_n256_h96_d128": Workload(
         name="decode_n256_h96_d128", B=256, H=96, T=1, dk=128, dv=128, dtype="bf16",
         chunk=64, s0_std=0.02, decode_steps=1000, seed=1004,

@@ -45,6 +45,8 @@ _lib.kda_forward_segmented_launches.argtypes = [_i] * 9
 _lib.kda_forward_segmented_launches.restype = _i
 _lib.kda_forward_segmented.argtypes = [_vp] * 8 + [_i] * 8 + [_vp, _sz, _vp, _vp, _i]
 _lib.kda_forward_segmented.restype = _i
+_lib.kda_decode_multi.argtypes = [_vp] * 8 + [_i] * 6 + [_vp]
+_lib.kda_decode_multi.restype = _i
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT = 0, 1, 2, 3
 KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_SCRATCH_LIMIT = 4, 5, 6, 7
@@ -251,4 +253,32 @@ def kda_decode_step(q, k, v, g, beta, S, o=None, *, stream=None):
                               N, H, dk, dv, DTYPES[dtype], _stream_handle(stream, dev))
     if rc != KDA_OK:
         raise KdaError(rc, "kda_decode_step")
+    return o
+
+
+def kda_decode_multi(q, k, v, g, beta, S, o=None, *, n_accept=None, outputs: bool = True, stream=None):
+    """T tokens per request from the states S (fp32 ``[N, H, dv, dk]``): outputs
+    of all T tokens, and the state after the first ``n_accept[n]`` tokens written
+    back in place (int32 ``[N]`` on the device; None = all T; 0 = untouched).
+    q, k, g ``[N, T, H, dk]``; v ``[N, T, H, dv]``; beta ``[N, T, H]``.
+    Returns o ``[N, T, H, dv]`` (None when ``outputs`` is False and o is None)."""
+    _need(k, "k")
+    dtype, dev = k.dtype, k.device
+    N, T, H, dk = k.shape
+    dv = v.shape[-1]
+    _need(q, "q", dtype, (N, T, H, dk), dev)
+    _need(g, "g", dtype, (N, T, H, dk), dev)
+    _need(v, "v", dtype, (N, T, H, dv), dev)
+    _need(beta, "beta", dtype, (N, T, H), dev)
+    _need(S, "S", torch.float32, (N, H, dv, dk), dev)
+    if n_accept is not None:
+        _need(n_accept, "n_accept", torch.int32, (N,), dev)
+    if o is None and outputs:
+        o = torch.empty((N, T, H, dv), dtype=dtype, device=dev)
+    if o is not None:
+        _need(o, "o", dtype, (N, T, H, dv), dev)
+    rc = _lib.kda_decode_multi(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
+                               _ptr(n_accept), N, T, H, dk, dv, DTYPES[dtype], _stream_handle(stream, dev))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_decode_multi")
     return o

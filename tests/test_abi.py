@@ -173,3 +173,17 @@ def test_segmented_queries(K):
     assert K.kda_forward_segmented_launches(1, 1000, 2, 128, 128, 64, 1, 256) == 8
     with pytest.raises(K.KdaError):
         K.kda_forward_segmented_workspace_size(1, 1000, 2, 128, 128, 64, 1, 96)
+
+
+def test_decode_multi_rejects_bad_args(K):
+    d = K._lib.kda_decode_multi
+    args = lambda **kw: [kw.get(n, FAKE) for n in ("q", "k", "v", "g", "beta", "S", "o", "acc")] + \
+        [kw.get(n, x) for n, x in (("N", 4), ("T", 3), ("H", 2), ("dk", 128), ("dv", 128), ("dt", 1))] + [None]
+    assert d(*args(T=0)) == K.KDA_ERR_INVALID_ARG
+    assert d(*args(N=0)) == K.KDA_ERR_INVALID_ARG
+    assert d(*args(T=65)) == K.KDA_ERR_UNSUPPORTED
+    assert d(*args(dk=96)) == K.KDA_ERR_UNSUPPORTED
+    assert d(*args(S=None)) == K.KDA_ERR_INVALID_ARG
+    assert d(*args(S=FAKE + 8)) == K.KDA_ERR_ALIGNMENT
+    assert d(*args(acc=FAKE + 4)) == K.KDA_ERR_ALIGNMENT
+    assert d(*args(dt=5)) == K.KDA_ERR_INVALID_ARG

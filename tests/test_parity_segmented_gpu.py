@@ -86,7 +86,7 @@ def test_segments_agree_with_plain_prefill(K):
 
 
 def test_long_sequence_few_heads_sampled(K, oracle_mod):
-    """The long-sequence workload (8 heads x 65536 tokens, 16 segments of 4096) in
+    """The long-sequence workload (8 heads x 65536 tokens, 18 segments of 3648) in
     the launch configuration the benchmark times; two heads checked in full."""
     w = WORKLOADS["long_h8_T65536_d128_bf16"]
     inp = workload_inputs(w, device="cuda")
