@@ -154,6 +154,25 @@ int kda_forward_noalloc(const void *q, const void *k, const void *v, const void 
                         int num_seqs, int *dev_status, void *stream);
 
 /*
+ * kda_forward on B dense sequences (no cu_seqlens) that also saves the state
+ * every snap_every tokens, for a prefix cache on a hybrid model ("Exercices",
+ * Q26: a prefix can only be reused where the KDA state was saved, and the
+ * state is large, so it is saved at coarse boundaries).
+ *
+ *   snap_every : tokens between snapshots, a positive multiple of chunk.
+ *   S_snap     : fp32 [B, T / snap_every, H, dv, dk]: slot p of sequence b is
+ *                the state after its first (p + 1) snap_every tokens, in the
+ *                S0 layout of one sequence (it can be passed back as S0 to
+ *                resume from that prefix). May be NULL when T < snap_every.
+ * Other arguments, results and errors as kda_forward_ex (no workspace is
+ * needed for dense batches; pass NULL, 0).
+ */
+int kda_forward_snapshots(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                          const float *S0, void *o, float *S_T, float *S_snap, int snap_every, int B, int T,
+                          int H, int dk, int dv, int chunk, int dtype, void *workspace, size_t workspace_bytes,
+                          int *dev_status, void *stream, int path);
+
+/*
  * Segment-parallel prefill for long sequences with few heads (KCP scan, after
  * "Exercices", Q21-Q22 and the 4-rank scan of the pages' check script).
  *

@@ -104,6 +104,29 @@ int kda_forward_ex(const void *q, const void *k, const void *v, const void *g, c
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+int kda_forward_snapshots(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                          const float *S0, void *o, float *S_T, float *S_snap, int snap_every, int B, int T,
+                          int H, int dk, int dv, int chunk, int dtype, void *workspace, size_t workspace_bytes,
+                          int *dev_status, void *stream, int path) {
+    kda::PrefillArgs a{};
+    int st = check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, false, 0, path, &a);
+    if (st) return st;
+    if (snap_every <= 0 || snap_every % chunk != 0) return KDA_ERR_INVALID_ARG;
+    if (T / snap_every > 0 && !S_snap) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    for (const void *p : {q, k, v, g, beta, (const void *)S0, (const void *)o, (const void *)S_T,
+                          (const void *)S_snap, (const void *)workspace, (const void *)dev_status})
+        if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;
+    a.S0 = S0; a.o = o; a.ST = S_T;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.dev_status = dev_status;
+    a.stream = static_cast<cudaStream_t>(stream);
+    a.S_snap = S_snap; a.snap_every = T / snap_every > 0 ? snap_every : 0;
+    const bool tc = use_tc(a, path);
+    const cudaError_t e = tc ? kda::launch_prefill_tc(a) : kda::launch_prefill_simt(a);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 int kda_forward(const void *q, const void *k, const void *v, const void *g, const void *beta,
                 const float *S0, void *o, float *S_T, int B, int T, int H, int dk, int dv,
                 int chunk, int dtype, const int32_t *cu_seqlens, int num_seqs, void *workspace,

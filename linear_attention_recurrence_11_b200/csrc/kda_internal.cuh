@@ -26,6 +26,10 @@ struct PrefillArgs {
     size_t workspace_bytes;
     int *dev_status;
     cudaStream_t stream;
+    // kda_forward_snapshots (dense batches): every snap_every tokens (a multiple of chunk) the
+    // state after that prefix goes to S_snap [B, T / snap_every, H, dv, dk]; 0 = none
+    float *S_snap = nullptr;
+    int snap_every = 0;
 };
 
 // kda_forward_segmented: B dense sequences of T tokens, each cut into P = ceil(T / seg_len)

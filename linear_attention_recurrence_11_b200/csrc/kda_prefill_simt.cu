@@ -199,6 +199,16 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_simt_kernel(const Pre
                 sS[i * UP + j] = acc;
             }
         }
+        // a snapshot of the state after this chunk (fp32, the S0 layout of one sequence)
+        if (p.snap_every && Lc == C && (c0 + C) % (size_t)p.snap_every == 0) {
+            __syncthreads();
+            const size_t nsnap = (size_t)p.T / p.snap_every, ps = (c0 + C) / p.snap_every - 1;
+            float *dst = p.S_snap + (((size_t)n * nsnap + ps) * H + h) * dv * DK + (size_t)j0 * DK;
+            for (int idx = tid; idx < DK * DVB; idx += kThreads) {
+                const int j = idx / DK, i = idx % DK;
+                dst[(size_t)j * DK + i] = sS[i * UP + j];
+            }
+        }
     }
     __syncthreads();
     if (p.ST)

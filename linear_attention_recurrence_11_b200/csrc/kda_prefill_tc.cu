@@ -790,6 +790,16 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq)) = w0;
                 *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq + 8)) = w1;
             }
+            // a snapshot of the state after this chunk (fp32, the S0 layout of one sequence)
+            const long long done = (ch + 1) * C;
+            if (p.snap_every && Lc == C && done % p.snap_every == 0) {
+                const long long nsnap = p.T / p.snap_every;
+                float *dst = p.S_snap + (((size_t)n * nsnap + (size_t)(done / p.snap_every - 1)) * H + h) * (size_t)(D * D);
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) dst[(size_t)(64 * half + 16 * gq + e) * D + si] = sv[gq][e];
+            }
         }
         fence_proxy_async_smem();
         tc_fence_before();

@@ -47,6 +47,8 @@ _lib.kda_forward_segmented.argtypes = [_vp] * 8 + [_i] * 8 + [_vp, _sz, _vp, _vp
 _lib.kda_forward_segmented.restype = _i
 _lib.kda_decode_multi.argtypes = [_vp] * 8 + [_i] * 6 + [_vp]
 _lib.kda_decode_multi.restype = _i
+_lib.kda_forward_snapshots.argtypes = [_vp] * 9 + [_i] * 8 + [_vp, _sz, _vp, _vp, _i]
+_lib.kda_forward_snapshots.restype = _i
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT = 0, 1, 2, 3
 KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_SCRATCH_LIMIT = 4, 5, 6, 7
@@ -282,3 +284,40 @@ def kda_decode_multi(q, k, v, g, beta, S, o=None, *, n_accept=None, outputs: boo
     if rc != KDA_OK:
         raise KdaError(rc, "kda_decode_multi")
     return o
+
+
+def kda_forward_snapshots(q, k, v, g, beta, S0=None, *, snap_every: int, chunk: int = 64, o=None,
+                          S_T=None, S_snap=None, dev_status=None, stream=None, path: str = "auto"):
+    """kda_forward on B dense sequences that also returns the state every
+    ``snap_every`` tokens: S_snap fp32 ``[B, T // snap_every, H, dv, dk]`` (slot p =
+    the state after (p + 1) * snap_every tokens, usable as S0 of one sequence).
+    Returns ``(o, S_T, S_snap)``."""
+    _need(k, "k")
+    dtype, dev = k.dtype, k.device
+    if dtype not in DTYPES:
+        raise ValueError(f"unsupported dtype {dtype}")
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    _need(q, "q", dtype, (B, T, H, dk), dev)
+    _need(g, "g", dtype, (B, T, H, dk), dev)
+    _need(v, "v", dtype, (B, T, H, dv), dev)
+    _need(beta, "beta", dtype, (B, T, H), dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dv, dk), dev)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dtype, device=dev)
+    _need(o, "o", dtype, (B, T, H, dv), dev)
+    if S_T is None:
+        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    _need(S_T, "S_T", torch.float32, (B, H, dv, dk), dev)
+    nsnap = T // snap_every if snap_every > 0 else 0
+    if S_snap is None:
+        S_snap = torch.empty((B, nsnap, H, dv, dk), dtype=torch.float32, device=dev)
+    _need(S_snap, "S_snap", torch.float32, (B, nsnap, H, dv, dk), dev)
+    rc = _lib.kda_forward_snapshots(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                    _ptr(S_T), _ptr(S_snap) if nsnap > 0 else None, int(snap_every), B, T, H,
+                                    dk, dv, int(chunk), DTYPES[dtype], None, 0, _ptr(dev_status),
+                                    _stream_handle(stream, dev), PATHS[path])
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_forward_snapshots")
+    return o, S_T, S_snap

@@ -187,3 +187,15 @@ def test_decode_multi_rejects_bad_args(K):
     assert d(*args(S=FAKE + 8)) == K.KDA_ERR_ALIGNMENT
     assert d(*args(acc=FAKE + 4)) == K.KDA_ERR_ALIGNMENT
     assert d(*args(dt=5)) == K.KDA_ERR_INVALID_ARG
+
+
+def test_snapshots_reject_bad_arguments(K):
+    f = K._lib.kda_forward_snapshots
+    base = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, S0=None, o=FAKE, S_T=None, snap=FAKE, every=256,
+                B=1, T=1000, H=2, dk=128, dv=128, chunk=64, dt=1, ws=None, wsb=0, st=None, stream=None, path=0)
+    call = lambda **kw: f(*[dict(base, **kw)[n] for n in base])
+    assert call(every=0) == K.KDA_ERR_INVALID_ARG
+    assert call(every=100) == K.KDA_ERR_INVALID_ARG     # not a multiple of chunk
+    assert call(snap=None) == K.KDA_ERR_INVALID_ARG     # 3 snapshots are due
+    assert call(snap=FAKE + 4) == K.KDA_ERR_ALIGNMENT
+    assert call(dk=48) == K.KDA_ERR_UNSUPPORTED
