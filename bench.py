@@ -47,6 +47,8 @@ def parse_args():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="prefill", choices=sorted(WORKLOAD_ALIASES))
     p.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    p.add_argument("--snap-every", type=int, default=1024,
+                   help="prefill leg saving the state every N tokens (0: skip)")
     p.add_argument("--draft-tokens", type=int, default=4,
                    help="draft tokens per request in the speculative decode leg (0: skip)")
     p.add_argument("--decode-steps", type=int, default=50)
@@ -320,6 +322,28 @@ def run_ours(args, rank, world, device):
         res["plain_prefill"] = {"ms_per_step": a.elapsed_time(b) / 3,
                                 "tokens_per_s": tokens / (a.elapsed_time(b) / 3 / 1e3),
                                 "note": "kda_forward on the same inputs, one unit per (sequence, head); outside the timed region"}
+    if args.snap_every > 0 and not seg and not w.seqlens and T >= args.snap_every:
+        # the same prefill saving the state every snap_every tokens (prefix cache)
+        Ssn = torch.empty((B, T // args.snap_every, w.H, w.dv, w.dk), dtype=torch.float32, device=device)
+
+        def snap():
+            kda.kda_forward_snapshots(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"],
+                                      snap_every=args.snap_every, chunk=w.chunk, o=o, S_T=ST, S_snap=Ssn,
+                                      path=args.path)
+        for _ in range(2):
+            snap()
+        torch.cuda.synchronize(device)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(5):
+            snap()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        ms_snap = a.elapsed_time(b) / 5
+        res["snapshots"] = {"snap_every": args.snap_every, "snapshots_per_unit": T // args.snap_every,
+                            "ms_per_step": ms_snap, "overhead_vs_step": ms_snap / kern_ms - 1.0,
+                            "snapshot_bytes_per_step": Ssn.numel() * 4,
+                            "note": "kda_forward_snapshots on the same inputs, outside the timed region"}
     if not args.no_e2e:
         res["e2e"] = e2e_prefill(args, device, inp, w, forward, o, ST, world, barrier, max_ranks)
     if not args.no_decode and args.workload == "prefill":

@@ -218,6 +218,30 @@ int kda_decode_step(const void *q, const void *k, const void *v, const void *g,
                     int dtype, void *stream);
 
 /*
+ * The pieces of the segment-parallel prefill, for callers that place the
+ * segments themselves (one segment per GPU: context parallelism, after the
+ * pages' 4-rank scan).
+ *
+ * kda_segment_pair: the KCP pair of each of B dense sequences of T tokens
+ * ("Exercices", Q21-Q22): M [B, H, dk, dk], the transition (the recurrence
+ * run from S = I with zero values; stored like a state with dv = dk: element
+ * (i, a) of M at a * dk + i), and Z [B, H, dv, dk], the local state (from
+ * S = 0). fp32. Sizes, dtypes and path as kda_forward_ex.
+ *
+ * kda_kcp_scan: for B sequences of P consecutive segments with pairs
+ * M [B, P, H, dk, dk] and Z [B, P, H, dv, dk] (each segment's pair in the
+ * layout above) and incoming states S0 [B, H, dv, dk] (NULL: zeros), writes
+ * S_in [B, P, H, dv, dk], the incoming state of every segment
+ * (S_in,0 = S0, S_in,p+1 = M_p S_in,p + Z_p, fp32), and S_T [B, H, dv, dk]
+ * (NULL to skip), the state after the last segment.
+ */
+int kda_segment_pair(const void *q, const void *k, const void *v, const void *g, const void *beta, float *M,
+                     float *Z, int B, int T, int H, int dk, int dv, int chunk, int dtype, int *dev_status,
+                     void *stream, int path);
+int kda_kcp_scan(const float *S0, const float *M, const float *Z, float *S_in, float *S_T, int B, int P, int H,
+                 int dk, int dv, void *stream);
+
+/*
  * Multi-token decode with speculative acceptance ("Exercices", Q27: the state
  * after an accepted prefix of draft tokens is determined by those tokens'
  * inputs, so only the inputs are kept, the recurrence is replayed on chip and

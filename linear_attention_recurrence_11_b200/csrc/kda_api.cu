@@ -210,6 +210,39 @@ int kda_decode_step(const void *q, const void *k, const void *v, const void *g, 
     return kda::launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+int kda_segment_pair(const void *q, const void *k, const void *v, const void *g, const void *beta, float *M,
+                     float *Z, int B, int T, int H, int dk, int dv, int chunk, int dtype, int *dev_status,
+                     void *stream, int path) {
+    kda::PrefillArgs a{};
+    int st = check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, false, 0, path, &a);
+    if (st) return st;
+    if (path == KDA_PATH_TC && !kda::prefill_tc_supported(dk, dk, chunk, dtype)) return KDA_ERR_UNSUPPORTED;
+    if (!M || !Z || (T > 0 && (!q || !k || !v || !g || !beta))) return KDA_ERR_INVALID_ARG;
+    for (const void *p : {q, k, v, g, beta, (const void *)M, (const void *)Z, (const void *)dev_status})
+        if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
+    kda::SegmentedArgs s{};
+    s.q = q; s.k = k; s.v = v; s.g = g; s.beta = beta;
+    s.B = B; s.T = T; s.H = H; s.dk = dk; s.dv = dv; s.chunk = chunk; s.dtype = dtype; s.P = 1; s.seg_len = T;
+    s.dev_status = dev_status; s.stream = static_cast<cudaStream_t>(stream);
+    const bool tc_pair = path != KDA_PATH_SIMT && kda::prefill_tc_supported(dk, dk, chunk, dtype);
+    const bool tc_state = path != KDA_PATH_SIMT && kda::prefill_tc_supported(dk, dv, chunk, dtype);
+    return kda::launch_segment_pair(s, M, Z, tc_pair, tc_state) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_kcp_scan(const float *S0, const float *M, const float *Z, float *S_in, float *S_T, int B, int P, int H,
+                 int dk, int dv, void *stream) {
+    if (B <= 0 || P <= 0 || H <= 0) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if ((size_t)B * P * H > 0x7fffffffu) return KDA_ERR_UNSUPPORTED;
+    if (!M || !Z || !S_in) return KDA_ERR_INVALID_ARG;
+    for (const void *p : {(const void *)S0, (const void *)M, (const void *)Z, (const void *)S_in, (const void *)S_T})
+        if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
+    kda::SegmentedArgs s{};
+    s.S0 = S0; s.ST = S_T; s.B = B; s.P = P; s.H = H; s.dk = dk; s.dv = dv;
+    s.stream = static_cast<cudaStream_t>(stream);
+    return kda::launch_kcp_scan(s, M, Z, S_in) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 int kda_decode_multi(const void *q, const void *k, const void *v, const void *g, const void *beta, float *S,
                      void *o, const int32_t *n_accept, int N, int T, int H, int dk, int dv, int dtype,
                      void *stream) {

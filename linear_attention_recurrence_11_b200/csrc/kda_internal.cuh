@@ -95,6 +95,10 @@ size_t segmented_workspace(const SegmentedArgs &s);
 int segmented_launches(const SegmentedArgs &s);
 // tc_pair / tc_state: run the M_p pass (dv = dk) / the other passes on the tensor-core kernel
 cudaError_t launch_segmented(const SegmentedArgs &s, bool tc_pair, bool tc_state);
+// one segment per sequence: M [B, H, dk, dk] (from the identity, zero values), Z [B, H, dv, dk] (from 0)
+cudaError_t launch_segment_pair(const SegmentedArgs &s, float *M, float *Z, bool tc_pair, bool tc_state);
+// s.S0 / s.ST / s.B / s.P / s.H / s.dk / s.dv / s.stream: incoming states of P segments per sequence
+cudaError_t launch_kcp_scan(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin);
 cudaError_t launch_prefill_tc(const PrefillArgs &a);
 size_t prefill_tc_workspace(const PrefillArgs &a);
 int prefill_tc_launches(const PrefillArgs &a);

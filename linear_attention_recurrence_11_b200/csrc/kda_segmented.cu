@@ -31,7 +31,7 @@ __global__ void kda_segment_init_kernel(int32_t *cu_seg, float *Mbuf, int B, int
     const int units = B * P;
     const size_t gid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const size_t stride = (size_t)gridDim.x * blockDim.x;
-    for (size_t u = gid; u <= (size_t)units; u += stride) {
+    for (size_t u = gid; cu_seg && u <= (size_t)units; u += stride) {
         if (u == (size_t)units) {
             cu_seg[u] = B * T;
         } else {
@@ -150,6 +150,27 @@ cudaError_t run_pass(const PrefillArgs &a, bool tc) { return tc ? launch_prefill
 }  // namespace
 
 size_t segmented_workspace(const SegmentedArgs &s) { return s.P <= 1 ? 0 : seg_layout(s).total; }
+
+cudaError_t launch_kcp_scan(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin) {
+    return launch_scan(s, Mbuf, Zbuf, Sin);
+}
+
+cudaError_t launch_segment_pair(const SegmentedArgs &s, float *M, float *Z, bool tc_pair, bool tc_state) {
+    // identity start for the transition pass (no offsets needed: one segment per sequence)
+    kda_segment_init_kernel<<<296, kSegThreads, 0, s.stream>>>(nullptr, M, s.B, s.T, 1, s.T, s.H, s.dk);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    PrefillArgs a{};
+    a.q = s.q; a.k = s.k; a.g = s.g; a.beta = s.beta;
+    a.B = s.B; a.T = s.T; a.H = s.H; a.dk = s.dk; a.chunk = s.chunk; a.dtype = s.dtype;
+    a.num_units = s.B; a.dev_status = s.dev_status; a.stream = s.stream;
+    PrefillArgs pa = a;
+    pa.v = nullptr; pa.o = nullptr; pa.S0 = M; pa.ST = M; pa.dv = s.dk;
+    if ((e = run_pass(pa, tc_pair)) != cudaSuccess) return e;
+    PrefillArgs pb = a;
+    pb.v = s.v; pb.o = nullptr; pb.S0 = nullptr; pb.ST = Z; pb.dv = s.dv;
+    return run_pass(pb, tc_state);
+}
 
 int segmented_launches(const SegmentedArgs &s) {
     const int order = seq_order_bytes(s.B * s.P) > 0 ? 1 : 0;

@@ -49,6 +49,10 @@ _lib.kda_decode_multi.argtypes = [_vp] * 8 + [_i] * 6 + [_vp]
 _lib.kda_decode_multi.restype = _i
 _lib.kda_forward_snapshots.argtypes = [_vp] * 9 + [_i] * 8 + [_vp, _sz, _vp, _vp, _i]
 _lib.kda_forward_snapshots.restype = _i
+_lib.kda_segment_pair.argtypes = [_vp] * 7 + [_i] * 7 + [_vp, _vp, _i]
+_lib.kda_segment_pair.restype = _i
+_lib.kda_kcp_scan.argtypes = [_vp] * 5 + [_i] * 5 + [_vp]
+_lib.kda_kcp_scan.restype = _i
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT = 0, 1, 2, 3
 KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_SCRATCH_LIMIT = 4, 5, 6, 7
@@ -321,3 +325,44 @@ def kda_forward_snapshots(q, k, v, g, beta, S0=None, *, snap_every: int, chunk: 
     if rc != KDA_OK:
         raise KdaError(rc, "kda_forward_snapshots")
     return o, S_T, S_snap
+
+
+def kda_segment_pair(q, k, v, g, beta, *, chunk: int = 64, dev_status=None, stream=None, path: str = "auto"):
+    """KCP pair of each of B dense sequences: M fp32 ``[B, H, dk, dk]`` (the transition,
+    stored like a state with dv = dk) and Z fp32 ``[B, H, dv, dk]`` (the local state)."""
+    _need(k, "k")
+    dtype, dev = k.dtype, k.device
+    B, T, H, dk = k.shape
+    dv = v.shape[-1]
+    _need(q, "q", dtype, (B, T, H, dk), dev)
+    _need(g, "g", dtype, (B, T, H, dk), dev)
+    _need(v, "v", dtype, (B, T, H, dv), dev)
+    _need(beta, "beta", dtype, (B, T, H), dev)
+    M = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev)
+    Z = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    rc = _lib.kda_segment_pair(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(M), _ptr(Z), B, T, H, dk,
+                               dv, int(chunk), DTYPES[dtype], _ptr(dev_status), _stream_handle(stream, dev),
+                               PATHS[path])
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_segment_pair")
+    return M, Z
+
+
+def kda_kcp_scan(S0, M, Z, *, stream=None):
+    """Incoming state of every segment from the segments' pairs: M ``[B, P, H, dk, dk]``,
+    Z ``[B, P, H, dv, dk]``, S0 ``[B, H, dv, dk]`` or None. Returns (S_in
+    ``[B, P, H, dv, dk]``, S_T ``[B, H, dv, dk]``), fp32."""
+    _need(M, "M", torch.float32)
+    B, P, H, dk, _ = M.shape
+    dv = Z.shape[3]
+    dev = M.device
+    _need(Z, "Z", torch.float32, (B, P, H, dv, dk), dev)
+    if S0 is not None:
+        _need(S0, "S0", torch.float32, (B, H, dv, dk), dev)
+    S_in = torch.empty((B, P, H, dv, dk), dtype=torch.float32, device=dev)
+    S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    rc = _lib.kda_kcp_scan(_ptr(S0), _ptr(M), _ptr(Z), _ptr(S_in), _ptr(S_T), B, P, H, dk, dv,
+                           _stream_handle(stream, dev))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_kcp_scan")
+    return S_in, S_T

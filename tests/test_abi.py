@@ -199,3 +199,15 @@ def test_snapshots_reject_bad_arguments(K):
     assert call(snap=None) == K.KDA_ERR_INVALID_ARG     # 3 snapshots are due
     assert call(snap=FAKE + 4) == K.KDA_ERR_ALIGNMENT
     assert call(dk=48) == K.KDA_ERR_UNSUPPORTED
+
+
+def test_pair_and_scan_reject_bad_arguments(K):
+    pair = K._lib.kda_segment_pair
+    assert pair(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 1, 64, 2, 128, 128, 64, 1, None, None, 0) == K.KDA_ERR_INVALID_ARG
+    assert pair(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4, FAKE, 1, 64, 2, 128, 128, 64, 1, None, None, 0) == K.KDA_ERR_ALIGNMENT
+    assert pair(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 64, 2, 48, 128, 64, 1, None, None, 0) == K.KDA_ERR_UNSUPPORTED
+    scan = K._lib.kda_kcp_scan
+    assert scan(None, FAKE, FAKE, FAKE, None, 1, 0, 2, 128, 128, None) == K.KDA_ERR_INVALID_ARG
+    assert scan(None, None, FAKE, FAKE, None, 1, 2, 2, 128, 128, None) == K.KDA_ERR_INVALID_ARG
+    assert scan(None, FAKE, FAKE, FAKE, None, 1, 2, 2, 96, 128, None) == K.KDA_ERR_UNSUPPORTED
+    assert scan(FAKE + 8, FAKE, FAKE, FAKE, None, 1, 2, 2, 128, 128, None) == K.KDA_ERR_ALIGNMENT

@@ -96,3 +96,41 @@ def test_long_sequence_few_heads_sampled(K, oracle_mod):
     o_ref, ST_ref = oracle_forward(oracle_mod, inp, units=units)
     e_o, e_s = compare_units(o, ST, o_ref, ST_ref, units)
     assert e_o < TOL["bf16"] and e_s < TOL["bf16"], (e_o, e_s)
+
+
+@pytest.mark.parametrize("path", ["auto", "simt"])
+def test_pairs_scan_replay_by_hand(K, oracle_mod, path):
+    """The context-parallel pieces on one GPU: three segments' pairs, the scan, and
+    each segment replayed from its incoming state, against the oracle's single pass."""
+    inp = case(2, 3 * 192 - 40, 2, 128, 128, "bf16", seed=71, s0_std=0.1)
+    T = inp["k"].shape[1]
+    cuts = [(0, 192), (192, 384), (384, T)]
+    pairs = [K.kda_segment_pair(*(inp[x][:, a:b].contiguous() for x in ("q", "k", "v", "g", "beta")), path=path)
+             for a, b in cuts]
+    M = torch.stack([p[0] for p in pairs], 1)
+    Z = torch.stack([p[1] for p in pairs], 1)
+    S_in, S_T = K.kda_kcp_scan(inp["S0"], M, Z)
+    o = torch.cat([K.kda_forward(*(inp[x][:, a:b].contiguous() for x in ("q", "k", "v", "g", "beta")),
+                                 S_in[:, p].contiguous(), chunk=64, return_state=False, path=path)[0]
+                   for p, (a, b) in enumerate(cuts)], 1)
+    torch.cuda.synchronize()
+    o_ref, ST_ref = oracle_forward(oracle_mod, inp)
+    e_o, e_s = compare_units(o, S_T, o_ref, ST_ref, [(b, h) for b in range(2) for h in range(2)])
+    assert e_o < TOL["bf16"] and e_s < TOL["bf16"], (e_o, e_s)
+
+
+def test_context_parallel_module_one_rank_nccl(K):
+    """The context-parallel module through a real NCCL group of one rank (the
+    collective is the identity there): equals the plain prefill."""
+    import torch.distributed as dist
+    from linear_attention_recurrence_11_b200.context_parallel import context_parallel_forward
+    inp = case(1, 320, 2, 128, 128, "bf16", seed=73, s0_std=0.1)
+    dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1)
+    try:
+        o, S_T = context_parallel_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"])
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    o2, S2 = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], chunk=64)
+    torch.cuda.synchronize()
+    assert rel(to_f64(o), to_f64(o2)) < 1e-5 and rel(to_f64(S_T), to_f64(S2)) < 1e-2
