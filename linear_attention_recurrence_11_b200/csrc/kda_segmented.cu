@@ -46,65 +46,70 @@ __global__ void kda_segment_init_kernel(int32_t *cu_seg, float *Mbuf, int B, int
     }
 }
 
-// One CTA per (sequence b, head h): X <- S0 (or 0); for p = 0..P-1 { Sin[p] = X;
-// X = X Ms_p + Zs_p }; S_T = X. In the state layout X is [dv][dk] (X[j][i] = S[i][j]),
-// Ms_p is [dk][dk] (Ms[a][i] = M_p[i][a]) and Zs_p is [dv][dk], so M_p S + S~_p is
-// the plain row-major product X Ms + Zs, in fp32. Thread (tj, ti) owns rows
-// j = tj + 16 r and columns i = ti + 16 c, so that a warp's shared-memory reads of
-// Ms are consecutive; X is kept transposed with an odd row stride (no bank conflicts
-// on its column-wise writes).
+// Rows of the stored state (X[j][i] = S[i][j], [dv][dk]) evolve independently through
+// S <- M S + S~ (M acts on the dk index): in the stored layout X <- X Ms + Zs with
+// Ms[a][i] = M[i][a]. So one CTA per (sequence b, head h, block of kRowsPerCta rows)
+// runs the whole scan for its rows: X <- S0 rows (or 0); for p = 0..P-1 { Sin[p] = X;
+// X = X Ms_p + Zs_p }; S_T = X. fp32. Thread (r, ci) owns row r of the block and the
+// columns ci + 16 c, so a warp's reads of Ms are consecutive and of X a broadcast.
+constexpr int kRowsPerCta = 16;
+
 template <int DK, int DV>
 __global__ void __launch_bounds__(kSegThreads)
 kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float *Sin, float *ST, int P, int H) {
-    constexpr int TJ = DV / 16, TI = DK / 16, XS = DV + 1;
+    constexpr int TI = DK / 16;                      // columns per thread
+    constexpr int RPI = kSegThreads / 16;            // rows covered per pass of the threads (16)
+    constexpr int RP = kRowsPerCta / RPI;            // rows per thread (1)
     extern __shared__ float smem[];
-    float *XT = smem;            // XT[a * XS + j] = X[j][a]
-    float *Ms = smem + DK * XS;  // Ms[a * DK + i]
-    const int b = blockIdx.x / H, h = blockIdx.x % H, tid = threadIdx.x;
-    const int tj = tid / 16, ti = tid % 16;
-    const size_t sbase = ((size_t)b * H + h) * DV * DK;
-    for (int e = tid; e < DV * DK; e += kSegThreads) XT[(e % DK) * XS + e / DK] = S0 ? S0[sbase + e] : 0.f;
+    float *Xs = smem;                                // [kRowsPerCta][DK]
+    float *Ms = smem + kRowsPerCta * DK;             // [DK][DK]
+    const int b = blockIdx.x / H, h = blockIdx.x % H, j0 = blockIdx.y * kRowsPerCta, tid = threadIdx.x;
+    const int r0 = tid / 16, ci = tid % 16;
+    const size_t sbase = (((size_t)b * H + h) * DV + j0) * DK;
+    for (int e = tid; e < kRowsPerCta * DK; e += kSegThreads) Xs[e] = S0 ? S0[sbase + e] : 0.f;
     for (int p = 0; p < P; ++p) {
         const size_t u = (size_t)b * P + p;
-        const size_t xbase = (u * H + h) * DV * DK, mbase = (u * H + h) * DK * DK;
-        for (int e = tid; e < DK * DK; e += kSegThreads) Ms[e] = Mbuf[mbase + e];
+        const size_t xbase = ((u * H + h) * DV + j0) * DK, mbase = (u * H + h) * DK * DK;
+        for (int e = 4 * tid; e < DK * DK; e += 4 * kSegThreads)
+            *reinterpret_cast<float4 *>(Ms + e) = *reinterpret_cast<const float4 *>(Mbuf + mbase + e);
         __syncthreads();
-        for (int e = tid; e < DV * DK; e += kSegThreads) Sin[xbase + e] = XT[(e % DK) * XS + e / DK];
-        float acc[TJ][TI];
+        for (int e = tid; e < kRowsPerCta * DK; e += kSegThreads) Sin[xbase + e] = Xs[e];
+        float acc[RP][TI];
 #pragma unroll
-        for (int r = 0; r < TJ; ++r)
+        for (int rr = 0; rr < RP; ++rr)
 #pragma unroll
-            for (int c = 0; c < TI; ++c) acc[r][c] = Zbuf[xbase + (size_t)(tj + 16 * r) * DK + ti + 16 * c];
-#pragma unroll 4
+            for (int c = 0; c < TI; ++c) acc[rr][c] = Zbuf[xbase + (size_t)(r0 + RPI * rr) * DK + ci + 16 * c];
+#pragma unroll 8
         for (int a = 0; a < DK; ++a) {
-            float xv[TJ], mv[TI];
+            float mv[TI];
 #pragma unroll
-            for (int r = 0; r < TJ; ++r) xv[r] = XT[a * XS + tj + 16 * r];
+            for (int c = 0; c < TI; ++c) mv[c] = Ms[a * DK + ci + 16 * c];
 #pragma unroll
-            for (int c = 0; c < TI; ++c) mv[c] = Ms[a * DK + ti + 16 * c];
+            for (int rr = 0; rr < RP; ++rr) {
+                const float xv = Xs[(r0 + RPI * rr) * DK + a];
 #pragma unroll
-            for (int r = 0; r < TJ; ++r)
-#pragma unroll
-                for (int c = 0; c < TI; ++c) acc[r][c] = fmaf(xv[r], mv[c], acc[r][c]);
+                for (int c = 0; c < TI; ++c) acc[rr][c] = fmaf(xv, mv[c], acc[rr][c]);
+            }
         }
         __syncthreads();  // every thread has read X and Ms_p
 #pragma unroll
-        for (int r = 0; r < TJ; ++r)
+        for (int rr = 0; rr < RP; ++rr)
 #pragma unroll
-            for (int c = 0; c < TI; ++c) XT[(ti + 16 * c) * XS + tj + 16 * r] = acc[r][c];
+            for (int c = 0; c < TI; ++c) Xs[(r0 + RPI * rr) * DK + ci + 16 * c] = acc[rr][c];
         __syncthreads();
     }
     if (ST)
-        for (int e = tid; e < DV * DK; e += kSegThreads) ST[sbase + e] = XT[(e % DK) * XS + e / DK];
+        for (int e = tid; e < kRowsPerCta * DK; e += kSegThreads) ST[sbase + e] = Xs[e];
 }
 
 template <int DK, int DV>
 cudaError_t launch_scan_t(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin) {
-    const size_t smem = (size_t)(DK * (DV + 1) + DK * DK) * sizeof(float);
+    const size_t smem = (size_t)(kRowsPerCta * DK + DK * DK) * sizeof(float);
     cudaError_t e = cudaFuncSetAttribute(kda_kcp_scan_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    kda_kcp_scan_kernel<DK, DV><<<s.B * s.H, kSegThreads, smem, s.stream>>>(s.S0, Mbuf, Zbuf, Sin, s.ST, s.P, s.H);
+    const dim3 grid((unsigned)(s.B * s.H), DV / kRowsPerCta);
+    kda_kcp_scan_kernel<DK, DV><<<grid, kSegThreads, smem, s.stream>>>(s.S0, Mbuf, Zbuf, Sin, s.ST, s.P, s.H);
     return cudaGetLastError();
 }
 
