@@ -264,6 +264,16 @@ int kda_decode_multi(const void *q, const void *k, const void *v, const void *g,
                      void *o, const int32_t *n_accept, int N, int T, int H, int dk, int dv, int dtype,
                      void *stream);
 
+/*
+ * Diagnostic: one CTA waits, through the same bounded-wait helper the
+ * tensor-core prefill uses for every mbarrier wait, on an mbarrier that
+ * nothing arrives on; after max_cycles SM clocks (1 .. 4e9) it gives up,
+ * stores KDA_ERR_TIMEOUT into *dev_status (device int, 16-byte aligned) and
+ * returns. Nothing faults or hangs and the stream stays usable; used to test
+ * failure reporting without a GPU fault.
+ */
+int kda_selftest_wait_timeout(int *dev_status, long long max_cycles, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

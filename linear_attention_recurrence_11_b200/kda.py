@@ -53,6 +53,8 @@ _lib.kda_segment_pair.argtypes = [_vp] * 7 + [_i] * 7 + [_vp, _vp, _i]
 _lib.kda_segment_pair.restype = _i
 _lib.kda_kcp_scan.argtypes = [_vp] * 5 + [_i] * 5 + [_vp]
 _lib.kda_kcp_scan.restype = _i
+_lib.kda_selftest_wait_timeout.argtypes = [_vp, ctypes.c_longlong, _vp]
+_lib.kda_selftest_wait_timeout.restype = _i
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT = 0, 1, 2, 3
 KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_SCRATCH_LIMIT = 4, 5, 6, 7
@@ -366,3 +368,12 @@ def kda_kcp_scan(S0, M, Z, *, stream=None):
     if rc != KDA_OK:
         raise KdaError(rc, "kda_kcp_scan")
     return S_in, S_T
+
+
+def kda_selftest_wait_timeout(dev_status, max_cycles: int = 20_000_000, *, stream=None):
+    """Run the bounded-wait self-test (a wait that must run out); the caller reads
+    dev_status (int32 on the device) after synchronising: KDA_ERR_TIMEOUT."""
+    _need(dev_status, "dev_status", torch.int32)
+    rc = _lib.kda_selftest_wait_timeout(_ptr(dev_status), int(max_cycles), _stream_handle(stream, dev_status.device))
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_selftest_wait_timeout")
