@@ -61,6 +61,15 @@ typedef enum {
 
 typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype;
 
+/* Pre-operations fused into the kernels (kda_forward_fused, kda_decode_step_fused):
+ * KDA_FUSE_NORM_QK: q and k are raw; each (token, head) row of both is L2-normalised
+ *   inside the kernel ("Exercices", Q9: I - beta k k^T is a well-conditioned projection
+ *   only for ||k||_2 = 1; q is normalised the same way); an all-zero row stays zero.
+ * KDA_FUSE_GATE_LOGITS: g holds gate logits x; the log-decay is g_min sigmoid(x) with
+ *   g_min = -5, which maps onto [g_min, 0] ("Exercices", Q8). The pages bound g but do
+ *   not print its formula; this is the plainest map onto that range. */
+typedef enum { KDA_FUSE_NORM_QK = 1, KDA_FUSE_GATE_LOGITS = 2 } kda_fuse;
+
 /* Which prefill kernel kda_forward_ex runs. AUTO picks the tensor-core kernel
  * where it is built (bf16, dk = dv = 128, chunk = 64) and the SIMT kernel
  * otherwise. */
@@ -119,6 +128,13 @@ int kda_forward_ex(const void *q, const void *k, const void *v, const void *g, c
                    int chunk, int dtype, const int32_t *cu_seqlens, int num_seqs,
                    void *workspace, size_t workspace_bytes, int *dev_status, void *stream,
                    int path);
+
+/* kda_forward_ex with fused pre-operations (flags: kda_fuse bits; 0 = kda_forward_ex).
+ * Unknown bits return KDA_ERR_INVALID_ARG. */
+int kda_forward_fused(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                      const float *S0, void *o, float *S_T, int B, int T, int H, int dk, int dv, int chunk,
+                      int dtype, const int32_t *cu_seqlens, int num_seqs, void *workspace,
+                      size_t workspace_bytes, int *dev_status, void *stream, int path, int flags);
 
 /* Number of kernel launches one kda_forward_ex call with these arguments
  * enqueues (0 when T = 0 and no state is copied), or -1 if invalid. */
@@ -240,6 +256,10 @@ int kda_segment_pair(const void *q, const void *k, const void *v, const void *g,
                      void *stream, int path);
 int kda_kcp_scan(const float *S0, const float *M, const float *Z, float *S_in, float *S_T, int B, int P, int H,
                  int dk, int dv, void *stream);
+
+/* kda_decode_step with fused pre-operations (flags: kda_fuse bits; 0 = kda_decode_step). */
+int kda_decode_step_fused(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                          float *S, void *o, int N, int H, int dk, int dv, int dtype, void *stream, int flags);
 
 /*
  * Multi-token decode with speculative acceptance ("Exercices", Q27: the state

@@ -127,6 +127,30 @@ int kda_forward_snapshots(const void *q, const void *k, const void *v, const voi
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
+int kda_forward_fused(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                      const float *S0, void *o, float *S_T, int B, int T, int H, int dk, int dv, int chunk,
+                      int dtype, const int32_t *cu_seqlens, int num_seqs, void *workspace,
+                      size_t workspace_bytes, int *dev_status, void *stream, int path, int flags) {
+    if (flags & ~(KDA_FUSE_NORM_QK | KDA_FUSE_GATE_LOGITS)) return KDA_ERR_INVALID_ARG;
+    kda::PrefillArgs a{};
+    int st = check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, cu_seqlens != nullptr, num_seqs, path, &a);
+    if (st) return st;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    for (const void *p : {q, k, v, g, beta, (const void *)S0, (const void *)o, (const void *)S_T,
+                          (const void *)cu_seqlens, (const void *)workspace, (const void *)dev_status})
+        if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
+    a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta;
+    a.S0 = S0; a.o = o; a.ST = S_T; a.cu_seqlens = cu_seqlens;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.dev_status = dev_status;
+    a.stream = static_cast<cudaStream_t>(stream);
+    a.fuse = flags;
+    const bool tc = use_tc(a, path);
+    const size_t need = tc ? kda::prefill_tc_workspace(a) : kda::prefill_simt_workspace(a);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
+    const cudaError_t e = tc ? kda::launch_prefill_tc(a) : kda::launch_prefill_simt(a);
+    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
 int kda_forward(const void *q, const void *k, const void *v, const void *g, const void *beta,
                 const float *S0, void *o, float *S_T, int B, int T, int H, int dk, int dv,
                 int chunk, int dtype, const int32_t *cu_seqlens, int num_seqs, void *workspace,
@@ -196,6 +220,20 @@ int kda_forward_segmented(const void *q, const void *k, const void *v, const voi
     s.stream = static_cast<cudaStream_t>(stream);
     if (workspace == nullptr || workspace_bytes < kda::segmented_workspace(s)) return KDA_ERR_WORKSPACE;
     return kda::launch_segmented(s, tc_pair, tc_state) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+}
+
+int kda_decode_step_fused(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                          float *S, void *o, int N, int H, int dk, int dv, int dtype, void *stream, int flags) {
+    if (flags & ~(KDA_FUSE_NORM_QK | KDA_FUSE_GATE_LOGITS)) return KDA_ERR_INVALID_ARG;
+    if (N <= 0 || H <= 0 || !dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if ((size_t)N * (size_t)H > 0x7fffffffu) return KDA_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !g || !beta || !S || !o) return KDA_ERR_INVALID_ARG;
+    for (const void *p : {q, k, v, g, beta, (const void *)S, (const void *)o})
+        if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
+    kda::DecodeArgs a{q, k, v, g, beta, S, o, N, H, dk, dv, dtype, static_cast<cudaStream_t>(stream)};
+    a.fuse = flags;
+    return kda::launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
 int kda_decode_step(const void *q, const void *k, const void *v, const void *g, const void *beta,

@@ -50,10 +50,30 @@ __global__ void __launch_bounds__(kDecThreads) kda_decode_kernel(const DecodeArg
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int i = 4 * (sub + kLanesPerRow * m) + e;
-            a[4 * m + e] = __expf(ld_elem(g, vb + i));
+            const float gi = ld_elem(g, vb + i);
+            a[4 * m + e] = __expf((p.fuse & KDA_FUSE_GATE_LOGITS) ? gate_from_logit(gi) : gi);
             kk[4 * m + e] = ld_elem(k, vb + i);
             qq[4 * m + e] = ld_elem(q, vb + i);
         }
+    if (p.fuse & KDA_FUSE_NORM_QK) {  // q and k normalised (the 8 lanes of a row hold all channels)
+        float sk = 0.f, sq = 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            sk = fmaf(kk[e], kk[e], sk);
+            sq = fmaf(qq[e], qq[e], sq);
+        }
+#pragma unroll
+        for (int off = 1; off < kLanesPerRow; off <<= 1) {
+            sk += __shfl_xor_sync(0xffffffffu, sk, off);
+            sq += __shfl_xor_sync(0xffffffffu, sq, off);
+        }
+        const float ik = sk > 0.f ? rsqrtf(sk) : 0.f, iq = sq > 0.f ? rsqrtf(sq) : 0.f;
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+            kk[e] *= ik;
+            qq[e] *= iq;
+        }
+    }
     float kq = 0.f;
 #pragma unroll
     for (int e = 0; e < E; ++e) kq = fmaf(kk[e], qq[e], kq);

@@ -30,6 +30,7 @@ struct PrefillArgs {
     // state after that prefix goes to S_snap [B, T / snap_every, H, dv, dk]; 0 = none
     float *S_snap = nullptr;
     int snap_every = 0;
+    int fuse = 0;  // KDA_FUSE_* bits: q, k normalised and / or g from gate logits inside the kernel
 };
 
 // kda_forward_segmented: B dense sequences of T tokens, each cut into P = ceil(T / seg_len)
@@ -52,7 +53,11 @@ struct DecodeArgs {
     void *o;
     int N, H, dk, dv, dtype;
     cudaStream_t stream;
+    int fuse = 0;  // KDA_FUSE_* bits
 };
+
+// g from a gate logit x: g_min sigmoid(x) = -5 / (1 + e^{-x}), in [g_min, 0]
+__device__ __forceinline__ float gate_from_logit(float x) { return -5.f / (1.f + __expf(-x)); }
 
 // kda_decode_multi: T tokens per request, the state after n_accept[n] of them written back.
 struct MultiDecodeArgs {

@@ -102,6 +102,34 @@ __global__ void __launch_bounds__(kThreads, 1) kda_prefill_simt_kernel(const Pre
         for (int r = tid; r < C; r += kThreads)
             sB[r] = (r < Lc) ? ld_elem(beta, (t_begin + c0 + r) * H + h) : 0.f;
         __syncthreads();
+        if (p.fuse) {  // fused pre-ops: g from gate logits, q and k normalised per row
+            if (p.fuse & KDA_FUSE_GATE_LOGITS)
+                for (int idx = tid; idx < Lc * DK; idx += kThreads) {
+                    const int r = idx / DK, i = idx % DK;
+                    sG[r * KP + i] = gate_from_logit(sG[r * KP + i]);
+                }
+            if (p.fuse & KDA_FUSE_NORM_QK) {
+                const int lane = tid & 31, w = tid >> 5;
+                for (int r = w; r < Lc; r += kThreads / 32) {
+                    float sk = 0.f, sq = 0.f;
+                    for (int i = lane; i < DK; i += 32) {
+                        sk = fmaf(sK[r * KP + i], sK[r * KP + i], sk);
+                        sq = fmaf(sQ[r * KP + i], sQ[r * KP + i], sq);
+                    }
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) {
+                        sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                        sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                    }
+                    const float ik = sk > 0.f ? rsqrtf(sk) : 0.f, iq = sq > 0.f ? rsqrtf(sq) : 0.f;
+                    for (int i = lane; i < DK; i += 32) {
+                        sK[r * KP + i] *= ik;
+                        sQ[r * KP + i] *= iq;
+                    }
+                }
+            }
+            __syncthreads();
+        }
 
         // cumulative log-decay over the chunk, per channel
         for (int i = tid; i < DK; i += kThreads) {

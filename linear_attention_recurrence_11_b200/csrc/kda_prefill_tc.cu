@@ -91,7 +91,8 @@ constexpr uint32_t OFF_TMEMADDR = OFF_MISC + 32;
 constexpr uint32_t OFF_BETA = OFF_MISC + 64;        // 64 fp32
 constexpr uint32_t OFF_DSUM = OFF_BETA + 256;       // 4 x 128 fp32 subtile totals of g (log2 units)
 constexpr uint32_t OFF_GAMC = OFF_DSUM + 2048;      // 128 fp32 Gamma_C
-constexpr uint32_t SMEM_USED = OFF_GAMC + 512;
+constexpr uint32_t OFF_NORM = OFF_GAMC + 512;       // 2 x 64 x 2 fp32: per-row partial squared norms of k, q
+constexpr uint32_t SMEM_USED = OFF_NORM + 1024;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;   // slack for 1024-byte alignment
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
@@ -225,6 +226,9 @@ __device__ __forceinline__ void tri_inverse_offdiag(const float *AF, float *TF, 
     __syncthreads();
 }
 
+// kFused: the variant with the fused pre-operations (KDA_FUSE_* in p.fuse); the plain
+// variant carries none of their code, so its schedule is not disturbed.
+template <bool kFused>
 __global__ void __launch_bounds__(NT, 1)
 kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -241,6 +245,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     float *sBeta = reinterpret_cast<float *>(sm + OFF_BETA);
     float *sD = reinterpret_cast<float *>(sm + OFF_DSUM);
     float *sGamC = reinterpret_cast<float *>(sm + OFF_GAMC);
+    float *sNorm = reinterpret_cast<float *>(sm + OFF_NORM);
+    const bool fuse_gate = kFused && (p.fuse & KDA_FUSE_GATE_LOGITS) != 0;
+    const bool fuse_norm = kFused && (p.fuse & KDA_FUSE_NORM_QK) != 0;
     float *AF = reinterpret_cast<float *>(sm + OFF_AF);
     float *TF = reinterpret_cast<float *>(sm + OFF_TF);
     float *XS = reinterpret_cast<float *>(sm + OFF_XS);
@@ -405,8 +412,12 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             for (int rr = 0; rr < HR; ++rr) {
                 const int row = SUB * ti + HR * hh + rr;  // rows past the end of the sequence decay by 1
                 const uint2 raw = row < Lc ? *reinterpret_cast<const uint2 *>(sm + OFF_G + row * 256 + c0 * 2) : make_uint2(0, 0);
-                const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
-                const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+                float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+                float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+                if (fuse_gate && row < Lc) {  // g holds gate logits
+                    g01 = make_float2(gate_from_logit(g01.x), gate_from_logit(g01.y));
+                    g23 = make_float2(gate_from_logit(g23.x), gate_from_logit(g23.y));
+                }
                 a[0] = fmaf(g01.x, kLog2e, a[0]);
                 a[1] = fmaf(g01.y, kLog2e, a[1]);
                 a[2] = fmaf(g23.x, kLog2e, a[2]);
@@ -426,6 +437,34 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (hh) {
 #pragma unroll
                 for (int e = 0; e < 4; ++e) sD[ti * D + c0 + e] = gl[HR - 1][e];
+            }
+        }
+        if (fuse_norm) {
+            // squared norms of this thread's k and q rows over its 4 channels, summed over the
+            // 16 lanes of the half-warp (64 channels); the partner warp holds the other 64
+            const uint8_t *krow = sm + OFF_KS + cblk * 8 * KB;
+            const uint8_t *qrow = sm + OFF_WQ + cblk * 16 * KB;
+#pragma unroll
+            for (int rr = 0; rr < HR; ++rr) {
+                const int r = SUB * ti + HR * hh + rr;
+                const uint2 kr = *reinterpret_cast<const uint2 *>(krow + sw128_offset(r, cin));
+                const uint2 qr = *reinterpret_cast<const uint2 *>(qrow + sw128_offset(64 + r, cin));
+                const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kr.x));
+                const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kr.y));
+                const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qr.x));
+                const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qr.y));
+                // rows past the end are being zeroed in this same phase: count them as zero
+                float sk = r < Lc ? k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y : 0.f;
+                float sq = r < Lc ? q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y : 0.f;
+#pragma unroll
+                for (int off = 1; off < 16; off <<= 1) {
+                    sk += __shfl_xor_sync(0xffffffffu, sk, off);
+                    sq += __shfl_xor_sync(0xffffffffu, sq, off);
+                }
+                if ((lane & 15) == rr) {
+                    sNorm[(0 * C + r) * 2 + (warp & 1)] = sk;
+                    sNorm[(1 * C + r) * 2 + (warp & 1)] = sq;
+                }
             }
         }
         if (tid == 0) bulk_wait_read_all();  // the previous chunk's staged outputs have been read
@@ -502,6 +541,16 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 float kx[4], qx[4], kf[4], qf[4];
                 ld4(krow + off_r, kx);
                 ld4(qrow + off_q, qx);
+                if (fuse_norm) {  // k and q normalised per row (rows past the end stay zero)
+                    const float nk = sNorm[(0 * C + r) * 2] + sNorm[(0 * C + r) * 2 + 1];
+                    const float nq = sNorm[(1 * C + r) * 2] + sNorm[(1 * C + r) * 2 + 1];
+                    const float ik = nk > 0.f ? rsqrtf(nk) : 0.f, iq = nq > 0.f ? rsqrtf(nq) : 0.f;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        kx[e] *= ik;
+                        qx[e] *= iq;
+                    }
+                }
                 // right operand row r (column block ti): k_r e^{G_start(ti) - G_r}; and Kh row r:
                 // k_r e^{G_C - G_r} = (k_r e^{G_start(ti) - G_r}) e^{G_C - G_start(ti)}, both factors bounded
                 float kr[4];
@@ -890,8 +939,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a) {
         !make_map(&mv, a.v ? a.v : a.q, tokens, a.H, 64, true) || !make_map(&mg, a.g, tokens, a.H, 128, false) ||
         !make_map(&mo, a.o ? a.o : a.q, tokens, a.H, 64, true))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(kda_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
+    const auto kern = a.fuse ? kda_prefill_tc_kernel<true> : kda_prefill_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     TcParams prm{a};
     if (a.cu_seqlens && seq_order_bytes(a.num_units) > 0) {
@@ -901,7 +950,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a) {
         prm.a.seq_order = order;
     }
     const unsigned grid = (unsigned)((size_t)a.num_units * a.H);
-    kda_prefill_tc_kernel<<<grid, NT, SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, mo, prm);
+    kern<<<grid, NT, SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, mo, prm);
     return cudaGetLastError();
 }
 

@@ -55,11 +55,16 @@ _lib.kda_kcp_scan.argtypes = [_vp] * 5 + [_i] * 5 + [_vp]
 _lib.kda_kcp_scan.restype = _i
 _lib.kda_selftest_wait_timeout.argtypes = [_vp, ctypes.c_longlong, _vp]
 _lib.kda_selftest_wait_timeout.restype = _i
+_lib.kda_forward_fused.argtypes = _FWD + [_i, _i]
+_lib.kda_forward_fused.restype = _i
+_lib.kda_decode_step_fused.argtypes = [_vp] * 7 + [_i] * 5 + [_vp, _i]
+_lib.kda_decode_step_fused.restype = _i
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT = 0, 1, 2, 3
 KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_SCRATCH_LIMIT = 4, 5, 6, 7
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 PATHS = {"auto": 0, "simt": 1, "tc": 2}
+KDA_FUSE_NORM_QK, KDA_FUSE_GATE_LOGITS = 1, 2  # fused pre-operations (see include/kda.h)
 
 
 class KdaError(RuntimeError):
@@ -114,10 +119,11 @@ def _need(t, name, dtype=None, shape=None, device=None):
 
 def kda_forward(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=None, o=None,
                 S_T=None, return_state: bool = True, workspace=None, dev_status=None,
-                stream=None, path: str = "auto"):
+                stream=None, path: str = "auto", fuse: int = 0):
     """Chunked KDA prefill. q, k, g ``[B, T, H, dk]``; v ``[B, T, H, dv]``;
     beta ``[B, T, H]`` (fp32 or bf16, all the same); S0 ``[N, H, dv, dk]`` fp32
-    or None; cu_seqlens int32 ``[N+1]`` (B must be 1) or None.
+    or None; cu_seqlens int32 ``[N+1]`` (B must be 1) or None. ``fuse``:
+    KDA_FUSE_* bits (raw q, k normalised in the kernel; g as gate logits).
     Returns ``(o, S_T)`` (S_T None when ``return_state`` is False)."""
     _need(k, "k")
     dtype, dev = k.dtype, k.device
@@ -147,11 +153,10 @@ def kda_forward(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=None, 
     if workspace is None and ws_need > 0:
         workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = _lib.kda_forward_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
-                             _ptr(S_T), B, T, H, dk, dv, int(chunk), DTYPES[dtype],
-                             _ptr(cu_seqlens), N if cu_seqlens is not None else 0,
-                             _ptr(workspace), ws_bytes, _ptr(dev_status),
-                             _stream_handle(stream, dev), PATHS[path])
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv,
+            int(chunk), DTYPES[dtype], _ptr(cu_seqlens), N if cu_seqlens is not None else 0,
+            _ptr(workspace), ws_bytes, _ptr(dev_status), _stream_handle(stream, dev), PATHS[path])
+    rc = _lib.kda_forward_fused(*args, int(fuse)) if fuse else _lib.kda_forward_ex(*args)
     if rc != KDA_OK:
         raise KdaError(rc, "kda_forward")
     return o, S_T
@@ -242,9 +247,10 @@ def kda_forward_segmented(q, k, v, g, beta, S0=None, *, seg_len: int, chunk: int
     return o, S_T
 
 
-def kda_decode_step(q, k, v, g, beta, S, o=None, *, stream=None):
+def kda_decode_step(q, k, v, g, beta, S, o=None, *, stream=None, fuse: int = 0):
     """One decode token per request. q, k, g ``[N, H, dk]``; v ``[N, H, dv]``;
-    beta ``[N, H]``; S ``[N, H, dv, dk]`` fp32 updated in place. Returns o."""
+    beta ``[N, H]``; S ``[N, H, dv, dk]`` fp32 updated in place. ``fuse``:
+    KDA_FUSE_* bits. Returns o."""
     _need(k, "k")
     dtype, dev = k.dtype, k.device
     N, H, dk = k.shape
@@ -257,8 +263,9 @@ def kda_decode_step(q, k, v, g, beta, S, o=None, *, stream=None):
     if o is None:
         o = torch.empty((N, H, dv), dtype=dtype, device=dev)
     _need(o, "o", dtype, (N, H, dv), dev)
-    rc = _lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
-                              N, H, dk, dv, DTYPES[dtype], _stream_handle(stream, dev))
+    args = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o), N, H, dk, dv, DTYPES[dtype],
+            _stream_handle(stream, dev))
+    rc = _lib.kda_decode_step_fused(*args, int(fuse)) if fuse else _lib.kda_decode_step(*args)
     if rc != KDA_OK:
         raise KdaError(rc, "kda_decode_step")
     return o

@@ -211,3 +211,12 @@ def test_pair_and_scan_reject_bad_arguments(K):
     assert scan(None, None, FAKE, FAKE, None, 1, 2, 2, 128, 128, None) == K.KDA_ERR_INVALID_ARG
     assert scan(None, FAKE, FAKE, FAKE, None, 1, 2, 2, 96, 128, None) == K.KDA_ERR_UNSUPPORTED
     assert scan(FAKE + 8, FAKE, FAKE, FAKE, None, 1, 2, 2, 128, 128, None) == K.KDA_ERR_ALIGNMENT
+
+
+def test_fused_entry_points_reject_unknown_flags(K):
+    f = K._lib.kda_forward_fused
+    base = [FAKE] * 5 + [None, FAKE, None, 1, 64, 2, 128, 128, 64, 1, None, 0, None, 0, None, None, 0]
+    assert f(*base, 4) == K.KDA_ERR_INVALID_ARG
+    assert f(*(base[:8] + [0] + base[9:]), 1) == K.KDA_ERR_INVALID_ARG  # B = 0
+    d = K._lib.kda_decode_step_fused
+    assert d(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 96, 128, 128, 1, None, 8) == K.KDA_ERR_INVALID_ARG
