@@ -58,6 +58,8 @@ def parse_args():
                    help="requests in the decode batch (smaller only for profiling captures)")
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--e2e-piece", type=int, default=1024,
+                   help="tokens per piece of kda_forward_host in the end-to-end leg (0: library default)")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU-baseline sample time")
     return p.parse_args()
@@ -345,7 +347,8 @@ def run_ours(args, rank, world, device):
                             "snapshot_bytes_per_step": Ssn.numel() * 4,
                             "note": "kda_forward_snapshots on the same inputs, outside the timed region"}
     if not args.no_e2e:
-        res["e2e"] = e2e_prefill(args, device, inp, w, forward, o, ST, world, barrier, max_ranks)
+        res["e2e"] = e2e_prefill(args, device, inp, w, forward, o, ST, world, barrier, max_ranks,
+                                 dense=not seg and not w.seqlens)
     if not args.no_decode and args.workload == "prefill":
         res["decode"] = decode_measure(args, device, peaks, barrier, max_ranks, world,
                                        steps=args.decode_steps)
@@ -355,9 +358,14 @@ def run_ours(args, rank, world, device):
     return res
 
 
-def e2e_prefill(args, device, inp, w, forward, o, ST, world, barrier, max_ranks):
-    """Same metric through the public API from pinned host buffers: per step,
-    H2D of q,k,v,g,beta(,S0), the prefill, D2H of o and S_T."""
+def e2e_prefill(args, device, inp, w, forward, o, ST, world, barrier, max_ranks, dense):
+    """Same metric from pinned host buffers, host<->device copies inside the
+    timed region: per step the inputs q,k,v,g,beta(,S0) go up and o and S_T come
+    back. Dense batches go through the C ABI's host entry point
+    (kda_forward_host: pieces of --e2e-piece tokens, uploads, launches and
+    downloads overlapped); packed or segmented workloads copy whole tensors
+    around the device call. For dense batches the serial form (whole-tensor
+    copies around kda_forward) is timed too, for comparison."""
     import torch
     from linear_attention_recurrence_11_b200 import kda
     names = [n for n in ("q", "k", "v", "g", "beta", "S0") if inp.get(n) is not None]
@@ -369,28 +377,49 @@ def e2e_prefill(args, device, inp, w, forward, o, ST, world, barrier, max_ranks)
     d2h = o_h.numel() * o_h.element_size() + S_h.numel() * S_h.element_size()
     stream = torch.cuda.current_stream(device)
 
-    def step():
+    def serial_step():
         for n in names:
             dev[n].copy_(host[n], non_blocking=True)
         forward(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], dev.get("S0"))
         o_h.copy_(o, non_blocking=True)
         S_h.copy_(ST, non_blocking=True)
 
-    K = max(3, min(args.steps, 10))
-    for _ in range(2):
-        step()
-    torch.cuda.synchronize(device)
-    barrier()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(K):
-        step()
-    b.record(stream)
-    torch.cuda.synchronize(device)
-    ms = max_ranks(a.elapsed_time(b))
-    return {"value": world * w.total_tokens * K / (ms / 1e3), "unit": "tokens/s",
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
-            "ms_per_step": ms / K}
+    if dense:
+        B, T, H, dk = inp["k"].shape
+        ws = torch.empty(kda.kda_forward_host_workspace_size(B, T, H, dk, inp["v"].shape[-1], w.chunk,
+                                                             inp["k"].dtype, args.e2e_piece),
+                         dtype=torch.uint8, device=device)
+
+        def host_step():
+            kda.kda_forward_host(host["q"], host["k"], host["v"], host["g"], host["beta"], host.get("S0"),
+                                 chunk=w.chunk, piece_len=args.e2e_piece, o=o_h, S_T=S_h, workspace=ws,
+                                 device=device, stream=stream, path=args.path)
+
+    def timed(step):
+        K = max(3, min(args.steps, 10))
+        for _ in range(2):
+            step()
+        torch.cuda.synchronize(device)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(K):
+            step()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        return max_ranks(a.elapsed_time(b)), K
+
+    ms, K = timed(host_step if dense else serial_step)
+    res = {"value": world * w.total_tokens * K / (ms / 1e3), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
+           "ms_per_step": ms / K}
+    if dense:
+        ms_serial, K_s = timed(serial_step)
+        res["api"] = f"kda_forward_host (pieces of {args.e2e_piece or 'T/8'} tokens)"
+        res["serial_ms_per_step"] = ms_serial / K_s
+    else:
+        res["api"] = "whole-tensor copies around the device call"
+    return res
 
 
 def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):

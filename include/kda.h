@@ -142,6 +142,43 @@ int kda_forward_launches(int B, int T, int H, int dk, int dv, int chunk, int dty
                          int has_cu_seqlens, int num_seqs, int path);
 
 /*
+ * Prefill of dense batches whose inputs and outputs are in HOST memory.
+ * The state is a fixed-size summary of the whole past ("Exercices", Q6), and
+ * a part of a sequence acts only on the state it receives ("Exercices", Q21).
+ * So the call cuts every sequence into pieces of piece_len tokens and runs
+ * each piece as one kda_forward_ex launch from the fp32 state the previous
+ * piece left on the device. Piece p's inputs are uploaded while piece p-1
+ * runs and piece p-2's outputs are downloaded, on two side streams of the
+ * library. With piece_len a multiple of chunk, o and S_T equal those of one
+ * kda_forward_ex call over all T tokens bit for bit.
+ *
+ *   q, k, g : host [B, T, H, dk]; v : host [B, T, H, dv]; beta : host [B, T, H];
+ *          all of dtype. Page-locked (pinned) memory lets the copies run
+ *          asynchronously and overlap; pageable memory works but serialises.
+ *   S0   : host [B, H, dv, dk] fp32, or NULL for zeros.
+ *   o    : host [B, T, H, dv] output, dtype. S_T : host [B, H, dv, dk] fp32, or NULL.
+ *   piece_len : tokens per piece, a positive multiple of chunk, or 0 for
+ *          about T / 8 rounded up to whole chunks.
+ *   workspace / workspace_bytes : DEVICE memory, 256-byte aligned, of at least
+ *          kda_forward_host_workspace_size(...) bytes: two slots for one
+ *          piece's inputs and outputs, and the state.
+ *   dev_status, path : as for kda_forward_ex. stream : the caller's stream;
+ *          the launches run on it, and it is made to wait for the last
+ *          download, so the host outputs are complete once the stream is.
+ * Host buffers and the workspace must stay valid until then. Ownership stays
+ * with the caller. Returns KDA_OK, a validation status (nothing enqueued), or
+ * KDA_ERR_CUDA (a CUDA call failed; work may have been enqueued). Calls on
+ * one device serialise while they enqueue (a mutex); the side streams and
+ * events are created on a device's first call and kept until process exit.
+ */
+size_t kda_forward_host_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int dtype,
+                                       int piece_len);
+int kda_forward_host(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                     const float *S0, void *o, float *S_T, int B, int T, int H, int dk, int dv,
+                     int chunk, int dtype, int piece_len, void *workspace, size_t workspace_bytes,
+                     int *dev_status, void *stream, int path);
+
+/*
  * kda_forward without a workspace argument, for callers that cannot allocate
  * device memory: engines that reserve all device memory in their own pools at
  * start-up and treat any other allocation as an error, hosts that hand a

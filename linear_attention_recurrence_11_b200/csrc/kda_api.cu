@@ -38,6 +38,13 @@ bool use_tc(const kda::PrefillArgs &a, int path) {
 
 }  // namespace
 
+namespace kda {
+int validate_prefill(int B, int T, int H, int dk, int dv, int chunk, int dtype, int path) {
+    PrefillArgs a{};
+    return check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, false, 0, path, &a);
+}
+}  // namespace kda
+
 extern "C" {
 
 const char *kda_status_string(int status) {

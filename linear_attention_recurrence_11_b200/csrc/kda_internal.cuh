@@ -110,5 +110,7 @@ int prefill_tc_launches(const PrefillArgs &a);
 
 cudaError_t launch_decode(const DecodeArgs &a);
 cudaError_t launch_decode_multi(const MultiDecodeArgs &a);
+// KDA_OK, or the status kda_forward_ex returns for these sizes (dense batches)
+int validate_prefill(int B, int T, int H, int dk, int dv, int chunk, int dtype, int path);
 
 }  // namespace kda

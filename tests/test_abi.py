@@ -220,3 +220,44 @@ def test_fused_entry_points_reject_unknown_flags(K):
     assert f(*(base[:8] + [0] + base[9:]), 1) == K.KDA_ERR_INVALID_ARG  # B = 0
     d = K._lib.kda_decode_step_fused
     assert d(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 96, 128, 128, 1, None, 8) == K.KDA_ERR_INVALID_ARG
+
+
+def test_host_entry_point_validates_before_any_cuda_call(K):
+    f = K._lib.kda_forward_host
+
+    def call(**kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, S0=None, o=FAKE, S_T=None, B=1, T=256, H=2,
+                 dk=128, dv=128, chunk=64, dtype=1, piece=128, ws=FAKE, ws_bytes=1 << 40, status=None,
+                 stream=None, path=0)
+        a.update(kw)
+        return f(a["q"], a["k"], a["v"], a["g"], a["beta"], a["S0"], a["o"], a["S_T"], a["B"], a["T"], a["H"],
+                 a["dk"], a["dv"], a["chunk"], a["dtype"], a["piece"], a["ws"], a["ws_bytes"], a["status"],
+                 a["stream"], a["path"])
+
+    assert call(piece=100) == K.KDA_ERR_INVALID_ARG      # not whole chunks
+    assert call(piece=-64) == K.KDA_ERR_INVALID_ARG
+    assert call(dk=48) == K.KDA_ERR_UNSUPPORTED
+    assert call(B=0) == K.KDA_ERR_INVALID_ARG
+    assert call(dtype=0, path=K.PATHS["tc"]) == K.KDA_ERR_UNSUPPORTED
+    for name in ("q", "k", "v", "g", "beta", "o"):
+        assert call(**{name: None}) == K.KDA_ERR_INVALID_ARG, name
+    assert call(ws=None) == K.KDA_ERR_WORKSPACE
+    assert call(ws_bytes=1024) == K.KDA_ERR_WORKSPACE
+    assert call(ws=FAKE + 16) == K.KDA_ERR_ALIGNMENT    # device workspace: 256-byte aligned
+
+
+def test_host_workspace_size_is_two_piece_slots_and_the_state(K):
+    # two slots of one piece's q, k, v, g, beta and o (each rounded up to 256 bytes) plus the fp32 state
+    B, T, H, d, L = 1, 8192, 96, 128, 1024
+    piece = B * L * H * d * 2
+    slot = 5 * piece + B * L * H * 2
+    state = B * H * d * d * 4
+    assert K.kda_forward_host_workspace_size(B, T, H, d, d, 64, 1, L) == 2 * slot + state
+    # piece_len 0: about T / 8 in whole chunks; a piece never exceeds the sequence
+    assert K.kda_forward_host_workspace_size(B, T, H, d, d, 64, 1, 0) == 2 * slot + state
+    small = K.kda_forward_host_workspace_size(2, 100, 3, 64, 32, 32, 0, 256)
+    tok = 2 * 100 * 3
+    rnd = lambda x: (x + 255) // 256 * 256
+    assert small == 2 * (3 * rnd(tok * 64 * 4) + 2 * rnd(tok * 32 * 4) + rnd(tok * 4)) + rnd(2 * 3 * 32 * 64 * 4)
+    with pytest.raises(K.KdaError):
+        K.kda_forward_host_workspace_size(1, 64, 2, 128, 128, 64, 1, 96)
