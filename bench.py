@@ -511,10 +511,12 @@ def multi_decode_measure(args, device, peaks, max_ranks, world, w, S, rounds=10)
     state = w.dk * w.dv * 4
     per_tok = (3 * w.dk + w.dv + 1) * 2
     written = int((acc > 0).sum().item())
-    bytes_round = (2 * w.B * w.H * state + written * w.H * state       # two state reads, accepted writes
-                   + 2 * w.B * T * w.H * per_tok + w.B * T * w.H * w.dv * 2)  # inputs twice, outputs once
-    gbs = bytes_round / (ms / 1e3) / 1e9
     accepted = int(acc.sum().item())
+    # verify: every state read, the inputs of all T tokens, all outputs; commit: the states of
+    # requests with an accepted token read and written, the inputs of the accepted tokens
+    bytes_round = ((w.B + 2 * written) * w.H * state
+                   + (w.B * T + accepted) * w.H * per_tok + w.B * T * w.H * w.dv * 2)
+    gbs = bytes_round / (ms / 1e3) / 1e9
     return {"draft_tokens": T, "ms_per_round": ms, "accepted_tokens_per_round": accepted * world,
             "accepted_tokens_per_s": world * accepted / (ms / 1e3),
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",

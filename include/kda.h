@@ -18,9 +18,12 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  *  - Every pointer argument is DEVICE memory owned by the caller unless the
- *    comment says otherwise. The library never allocates, frees or
- *    synchronises: work is enqueued on `stream` (a cudaStream_t; NULL = the
- *    legacy default stream) and the call returns once it is launched.
+ *    comment says otherwise (kda_forward_host takes host buffers). The
+ *    library never allocates or frees device memory and never synchronises:
+ *    work is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *    stream) and the call returns once it is launched. kda_forward_host also
+ *    keeps two side streams and eight events per device, made on its first
+ *    call there.
  *  - Activations are token-major and contiguous:
  *        q, k, g : [B, T, H, dk]      v, o : [B, T, H, dv]      beta : [B, T, H]
  *    all of the element type `dtype` (o is written in that type too).
@@ -316,10 +319,13 @@ int kda_decode_step_fused(const void *q, const void *k, const void *v, const voi
  *   S        : [N, H, dv, dk] fp32, read, and written where n_accept > 0.
  *   n_accept : device int32 [N] (values clamped to [0, T]) or NULL.
  *   T        : 1..64 (KDA_ERR_UNSUPPORTED above).
+ *   dev_status : NULL, or a device int set to KDA_ERR_TIMEOUT if a bounded
+ *          wait for the state's staging copies gives up (the outputs and the
+ *          states of that request and head are then left unwritten).
  */
 int kda_decode_multi(const void *q, const void *k, const void *v, const void *g, const void *beta, float *S,
                      void *o, const int32_t *n_accept, int N, int T, int H, int dk, int dv, int dtype,
-                     void *stream);
+                     int *dev_status, void *stream);
 
 /*
  * Diagnostic: one CTA waits, through the same bounded-wait helper the

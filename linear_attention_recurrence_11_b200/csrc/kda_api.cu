@@ -61,7 +61,7 @@ const char *kda_status_string(int status) {
     }
 }
 
-int kda_abi_version(void) { return 1; }
+int kda_abi_version(void) { return 2; }
 
 size_t kda_forward_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int num_seqs,
                                   int dtype) {
@@ -290,15 +290,17 @@ int kda_kcp_scan(const float *S0, const float *M, const float *Z, float *S_in, f
 
 int kda_decode_multi(const void *q, const void *k, const void *v, const void *g, const void *beta, float *S,
                      void *o, const int32_t *n_accept, int N, int T, int H, int dk, int dv, int dtype,
-                     void *stream) {
+                     int *dev_status, void *stream) {
     if (N <= 0 || T <= 0 || H <= 0 || !dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;
     if (T > kda::kMaxMultiTokens) return KDA_ERR_UNSUPPORTED;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
     if ((size_t)N * (size_t)H > 0x7fffffffu || (size_t)N * T * H > 0x7fffffffu) return KDA_ERR_UNSUPPORTED;
     if (!q || !k || !v || !g || !beta || !S) return KDA_ERR_INVALID_ARG;
-    for (const void *p : {q, k, v, g, beta, (const void *)S, (const void *)o, (const void *)n_accept})
+    for (const void *p : {q, k, v, g, beta, (const void *)S, (const void *)o, (const void *)n_accept,
+                          (const void *)dev_status})
         if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
-    kda::MultiDecodeArgs a{q, k, v, g, beta, S, o, n_accept, N, T, H, dk, dv, dtype, static_cast<cudaStream_t>(stream)};
+    kda::MultiDecodeArgs a{q, k, v, g, beta, S, o, n_accept, dev_status, N, T, H, dk, dv, dtype,
+                           static_cast<cudaStream_t>(stream)};
     return kda::launch_decode_multi(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 

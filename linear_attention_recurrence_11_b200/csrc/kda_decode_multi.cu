@@ -16,22 +16,31 @@
 // Each state is read from HBM once and written at most once, whatever T is.
 // Every column j of S (a contiguous dk-float row of the stored state) evolves
 // independently of the others through all T tokens (the decay, both dot
-// products and the rank-1 update act column by column), so the kernel streams
-// the state like the single-step decode: one CTA of 4 warps per (request,
-// head), 8 lanes per column with 128-bit loads, two columns in flight per
-// lane, all T tokens applied while a column is in registers, the column
-// written back right after token n_acc. The tokens' q, k, exp(g), beta and v
-// are staged in shared memory first; outputs are collected there and written
-// as contiguous rows at the end.
+// products and the rank-1 update act column by column). One CTA of 4 warps
+// per (request, head) walks the state in passes of 32 columns, each pass one
+// contiguous block (32 dk floats) that a bulk copy brings into shared memory:
+// two buffers, so the copy of pass p + 1 (and p + 2) is in flight while pass p
+// computes. In a pass, 8 lanes cover a column with 128-bit reads and each lane
+// holds two columns; all T tokens are applied while the columns are in
+// registers and a column goes back to HBM right after token n_acc. The
+// tokens' q, k, exp(g), beta and v are staged in shared memory first; outputs
+// are collected there and written as contiguous rows at the end. Without
+// outputs (o = NULL) only the first n_acc tokens are applied, and a request
+// with n_acc = 0 reads nothing.
 #include "kda_internal.cuh"
+#include "kda_sm100.cuh"
 
 namespace kda {
 namespace {
+
+using namespace sm100;
 
 constexpr int kMtThreads = 128;
 constexpr int kMtLanesPerRow = 8;
 constexpr int kMtRowsPerPass = (kMtThreads / 32) * (32 / kMtLanesPerRow);  // 16
 constexpr int kMtRowsInFlight = 2;
+constexpr int kMtCols = kMtRowsPerPass * kMtRowsInFlight;                  // 32 columns per pass
+constexpr long long kMtWaitCycles = 2000000000LL;                          // ~1 s at 2 GHz
 
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const MultiDecodeArgs p) {
@@ -39,7 +48,13 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
     constexpr int E = 4 * F4;                      // channels per lane
     // per token: q, k, exp(g) [DK each], v [DV], beta, padded to 16 bytes; then the outputs [T][DV]
     constexpr int TOK = 3 * DK + DV + 4;
-    extern __shared__ float sIn[];
+    constexpr int kPasses = DV / kMtCols;
+    constexpr uint32_t kPassBytes = kMtCols * DK * sizeof(float);
+    // shared: two pass buffers, two mbarriers (16 bytes), the tokens, the outputs
+    extern __shared__ __align__(16) float smem_mt[];
+    float *sBuf = smem_mt;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sBuf + 2 * kMtCols * DK);
+    float *sIn = reinterpret_cast<float *>(bar + 2);
     const Tin *q = static_cast<const Tin *>(p.q), *k = static_cast<const Tin *>(p.k);
     const Tin *v = static_cast<const Tin *>(p.v), *g = static_cast<const Tin *>(p.g);
     const Tin *beta = static_cast<const Tin *>(p.beta);
@@ -50,8 +65,24 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int sub = lane & (kMtLanesPerRow - 1), rw = lane / kMtLanesPerRow;
 
+    int n_acc = p.n_accept ? p.n_accept[n] : T;
+    n_acc = n_acc < 0 ? 0 : (n_acc > T ? T : n_acc);
+    const int t_end = o ? T : n_acc;  // tokens whose effect is needed
+    float *Su = p.S + unit * (size_t)DV * DK;
+    if (t_end > 0 && tid == 0) {  // the first two passes' columns -> shared memory
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_mbar_init();
+#pragma unroll
+        for (int b = 0; b < 2 && b < kPasses; ++b) {
+            mbar_arrive_expect_tx(&bar[b], kPassBytes);
+            bulk_load(sBuf + b * kMtCols * DK, Su + (size_t)b * kMtCols * DK, kPassBytes, &bar[b]);
+        }
+    }
+    if (t_end == 0) return;  // nothing to apply, nothing to write
+
     // the tokens' inputs -> shared memory (input layout [N, T, H, d])
-    for (int idx = tid; idx < T * TOK; idx += kMtThreads) {
+    for (int idx = tid; idx < t_end * TOK; idx += kMtThreads) {
         const int t = idx / TOK, c = idx % TOK;
         const size_t tok = ((size_t)n * T + t) * H + h;
         float x;
@@ -64,21 +95,30 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
         sIn[idx] = x;
     }
     float *sOut = sIn + T * TOK;
-    int n_acc = p.n_accept ? p.n_accept[n] : T;
-    n_acc = n_acc < 0 ? 0 : (n_acc > T ? T : n_acc);
     __syncthreads();
 
-    float *Su = p.S + unit * (size_t)DV * DK;
-    for (int jb = warp * (32 / kMtLanesPerRow) + rw; jb < DV; jb += kMtRowsPerPass * kMtRowsInFlight) {
+    int pass = 0;
+    bool ok = true;
+    for (; pass < kPasses; ++pass) {
+        const int b = pass & 1;
+        const float *buf = sBuf + b * kMtCols * DK;
+        const bool got = mbar_wait_bounded(&bar[b], (uint32_t)(pass >> 1) & 1u, kMtWaitCycles);
         float4 s[kMtRowsInFlight][F4];
 #pragma unroll
         for (int r = 0; r < kMtRowsInFlight; ++r) {
-            const int j = jb + r * kMtRowsPerPass;  // DV is a multiple of 32: always a valid column
+            const int jl = warp * (32 / kMtLanesPerRow) + rw + r * kMtRowsPerPass;  // column inside the pass
 #pragma unroll
             for (int m = 0; m < F4; ++m)
-                s[r][m] = __ldcs(reinterpret_cast<const float4 *>(Su + (size_t)j * DK + 4 * (sub + kMtLanesPerRow * m)));
+                s[r][m] = *reinterpret_cast<const float4 *>(buf + jl * DK + 4 * (sub + kMtLanesPerRow * m));
         }
-        for (int t = 0; t < T; ++t) {
+        // every thread holds its columns (or a wait gave up): the buffer can be refilled
+        if (__syncthreads_or(!got)) { ok = false; break; }
+        if (tid == 0 && pass + 2 < kPasses) {
+            fence_proxy_async_smem();
+            mbar_arrive_expect_tx(&bar[b], kPassBytes);
+            bulk_load(sBuf + b * kMtCols * DK, Su + (size_t)(pass + 2) * kMtCols * DK, kPassBytes, &bar[b]);
+        }
+        for (int t = 0; t < t_end; ++t) {
             const float *in = sIn + t * TOK;
             float kk[E], qq[E], a[E];
 #pragma unroll
@@ -96,10 +136,10 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
             for (int e = 0; e < E; ++e) kq = fmaf(kk[e], qq[e], kq);
 #pragma unroll
             for (int off = 1; off < kMtLanesPerRow; off <<= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
-            const float b = in[3 * DK + DV];
+            const float bt = in[3 * DK + DV];
 #pragma unroll
             for (int r = 0; r < kMtRowsInFlight; ++r) {
-                const int j = jb + r * kMtRowsPerPass;
+                const int j = pass * kMtCols + warp * (32 / kMtLanesPerRow) + rw + r * kMtRowsPerPass;
                 // the tokens of a column are sequential, so the dot products keep four
                 // partial sums each (short dependency chains between tokens)
                 float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
@@ -119,25 +159,36 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
                     sk += __shfl_xor_sync(0xffffffffu, sk, off);
                     sq += __shfl_xor_sync(0xffffffffu, sq, off);
                 }
-                const float u = b * (in[3 * DK + j] - sk);
+                const float u = bt * (in[3 * DK + j] - sk);
 #pragma unroll
                 for (int m = 0; m < F4; ++m) {
                     float *x = reinterpret_cast<float *>(&s[r][m]);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) x[e] = fmaf(kk[4 * m + e], u, x[e]);
                 }
-                if (sub == 0) sOut[t * DV + j] = fmaf(u, kq, sq);
+                if (o && sub == 0) sOut[t * DV + j] = fmaf(u, kq, sq);
             }
             if (t + 1 == n_acc) {  // the column after the accepted prefix, in place
 #pragma unroll
                 for (int r = 0; r < kMtRowsInFlight; ++r) {
-                    const int j = jb + r * kMtRowsPerPass;
+                    const int j = pass * kMtCols + warp * (32 / kMtLanesPerRow) + rw + r * kMtRowsPerPass;
 #pragma unroll
                     for (int m = 0; m < F4; ++m)
                         __stcs(reinterpret_cast<float4 *>(Su + (size_t)j * DK + 4 * (sub + kMtLanesPerRow * m)), s[r][m]);
                 }
             }
         }
+    }
+    if (!ok) {
+        // a staging copy did not arrive in time: report it, and let the copies still in
+        // flight (passes `pass` .. issued - 1) land before the CTA's shared memory is released
+        if (tid == 0) {
+            if (p.dev_status) atomicExch(p.dev_status, (int)KDA_ERR_TIMEOUT);
+            const int issued = pass + 2 < kPasses ? pass + 2 : kPasses;
+            for (int i = pass; i < issued; ++i)
+                mbar_wait_bounded(&bar[i & 1], (uint32_t)(i >> 1) & 1u, kMtWaitCycles);
+        }
+        return;
     }
     if (o) {  // outputs, one contiguous dv row per token
         __syncthreads();
@@ -150,7 +201,8 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
 
 template <typename Tin, int DK, int DV>
 cudaError_t launch_mt(const MultiDecodeArgs &a) {
-    const size_t smem = (size_t)a.T * (3 * DK + DV + 4 + DV) * sizeof(float);
+    const size_t smem = 2 * (size_t)kMtCols * DK * sizeof(float) + 16 +
+                        (size_t)a.T * (3 * DK + DV + 4 + DV) * sizeof(float);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kda_decode_multi_kernel<Tin, DK, DV>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

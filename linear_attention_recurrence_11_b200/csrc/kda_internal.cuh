@@ -65,6 +65,7 @@ struct MultiDecodeArgs {
     float *S;
     void *o;                   // may be null: no outputs
     const int32_t *n_accept;   // device [N] or null (all T)
+    int *dev_status;           // device status word or null
     int N, T, H, dk, dv, dtype;
     cudaStream_t stream;
 };

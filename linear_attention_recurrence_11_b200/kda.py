@@ -45,7 +45,7 @@ _lib.kda_forward_segmented_launches.argtypes = [_i] * 9
 _lib.kda_forward_segmented_launches.restype = _i
 _lib.kda_forward_segmented.argtypes = [_vp] * 8 + [_i] * 8 + [_vp, _sz, _vp, _vp, _i]
 _lib.kda_forward_segmented.restype = _i
-_lib.kda_decode_multi.argtypes = [_vp] * 8 + [_i] * 6 + [_vp]
+_lib.kda_decode_multi.argtypes = [_vp] * 8 + [_i] * 6 + [_vp, _vp]
 _lib.kda_decode_multi.restype = _i
 _lib.kda_forward_snapshots.argtypes = [_vp] * 9 + [_i] * 8 + [_vp, _sz, _vp, _vp, _i]
 _lib.kda_forward_snapshots.restype = _i
@@ -340,7 +340,8 @@ def kda_decode_step(q, k, v, g, beta, S, o=None, *, stream=None, fuse: int = 0):
     return o
 
 
-def kda_decode_multi(q, k, v, g, beta, S, o=None, *, n_accept=None, outputs: bool = True, stream=None):
+def kda_decode_multi(q, k, v, g, beta, S, o=None, *, n_accept=None, outputs: bool = True, dev_status=None,
+                     stream=None):
     """T tokens per request from the states S (fp32 ``[N, H, dv, dk]``): outputs
     of all T tokens, and the state after the first ``n_accept[n]`` tokens written
     back in place (int32 ``[N]`` on the device; None = all T; 0 = untouched).
@@ -361,8 +362,11 @@ def kda_decode_multi(q, k, v, g, beta, S, o=None, *, n_accept=None, outputs: boo
         o = torch.empty((N, T, H, dv), dtype=dtype, device=dev)
     if o is not None:
         _need(o, "o", dtype, (N, T, H, dv), dev)
+    if dev_status is not None:
+        _need(dev_status, "dev_status", torch.int32, None, dev)
     rc = _lib.kda_decode_multi(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S), _ptr(o),
-                               _ptr(n_accept), N, T, H, dk, dv, DTYPES[dtype], _stream_handle(stream, dev))
+                               _ptr(n_accept), N, T, H, dk, dv, DTYPES[dtype], _ptr(dev_status),
+                               _stream_handle(stream, dev))
     if rc != KDA_OK:
         raise KdaError(rc, "kda_decode_multi")
     return o

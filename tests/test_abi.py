@@ -178,7 +178,8 @@ def test_segmented_queries(K):
 def test_decode_multi_rejects_bad_args(K):
     d = K._lib.kda_decode_multi
     args = lambda **kw: [kw.get(n, FAKE) for n in ("q", "k", "v", "g", "beta", "S", "o", "acc")] + \
-        [kw.get(n, x) for n, x in (("N", 4), ("T", 3), ("H", 2), ("dk", 128), ("dv", 128), ("dt", 1))] + [None]
+        [kw.get(n, x) for n, x in (("N", 4), ("T", 3), ("H", 2), ("dk", 128), ("dv", 128), ("dt", 1))] + \
+        [kw.get("status"), None]
     assert d(*args(T=0)) == K.KDA_ERR_INVALID_ARG
     assert d(*args(N=0)) == K.KDA_ERR_INVALID_ARG
     assert d(*args(T=65)) == K.KDA_ERR_UNSUPPORTED
@@ -187,6 +188,7 @@ def test_decode_multi_rejects_bad_args(K):
     assert d(*args(S=FAKE + 8)) == K.KDA_ERR_ALIGNMENT
     assert d(*args(acc=FAKE + 4)) == K.KDA_ERR_ALIGNMENT
     assert d(*args(dt=5)) == K.KDA_ERR_INVALID_ARG
+    assert d(*args(status=FAKE + 4)) == K.KDA_ERR_ALIGNMENT
 
 
 def test_snapshots_reject_bad_arguments(K):

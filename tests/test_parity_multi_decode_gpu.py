@@ -87,3 +87,20 @@ def test_verify_then_commit(K, oracle_mod):
                               n_accept=torch.tensor(n_acc, device="cuda"), outputs=False) is None
     torch.cuda.synchronize()
     assert rel(to_f64(S), S_ref) < TOL["bf16"]
+
+
+def test_commit_without_outputs_equals_the_full_call(K):
+    """Without outputs only the accepted tokens are applied (and a request with
+    none accepted reads nothing): the states equal, bit for bit, those of the
+    call that also produces every output; the status word stays clear."""
+    N, T, H = 7, 6, 3
+    inp = make_inputs(N, T, H, 128, 64, "bf16", seed=43, device="cuda")
+    S1 = (0.02 * torch.randn(N, H, 64, 128, generator=torch.Generator().manual_seed(7))).cuda()
+    S2 = S1.clone()
+    acc = torch.tensor([0, 1, 2, 3, 6, 5, 4], dtype=torch.int32, device="cuda")
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    args = [inp[x] for x in ("q", "k", "v", "g", "beta")]
+    K.kda_decode_multi(*args, S1, n_accept=acc, dev_status=status)
+    assert K.kda_decode_multi(*args, S2, n_accept=acc, outputs=False, dev_status=status) is None
+    torch.cuda.synchronize()
+    assert torch.equal(S1, S2) and int(status[0]) == 0
