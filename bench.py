@@ -465,8 +465,9 @@ def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):
             "tokens_per_s": world * w.B / (ms / 1e3), "steps": steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "kernel": "kda_decode.cu",
+                         # the committed capture is scaled to the full 256-request batch only
                          "traffic": traffic_for("linear_attention_recurrence_11_b200/csrc/kda_decode.cu",
-                                                "decode_n256_h96_d128"),
+                                                "decode_n256_h96_d128") if w.B == 256 else None,
                          "algorithmic_bytes_per_launch": alg_bytes,
                          "peak_source": peaks["source"] + " (hbm_gbs)"},
             "gpu_launches": steps, "clocks": clk.summary(),

@@ -42,10 +42,24 @@ constexpr int kMtRowsInFlight = 2;
 constexpr int kMtCols = kMtRowsPerPass * kMtRowsInFlight;                  // 32 columns per pass
 constexpr long long kMtWaitCycles = 2000000000LL;                          // ~1 s at 2 GHz
 
+// 16 bytes of elements -> floats (8 bf16 or 4 fp32)
+__device__ __forceinline__ void unpack16(const uint4 &r, float (&x)[8]) {
+    const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w[i]));
+        x[2 * i] = f.x;
+        x[2 * i + 1] = f.y;
+    }
+}
+__device__ __forceinline__ void unpack16(const uint4 &r, float (&x)[4]) {
+    x[0] = __uint_as_float(r.x); x[1] = __uint_as_float(r.y);
+    x[2] = __uint_as_float(r.z); x[3] = __uint_as_float(r.w);
+}
+
 template <typename Tin, int DK, int DV>
 __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const MultiDecodeArgs p) {
     constexpr int F4 = DK / (4 * kMtLanesPerRow);  // float4 per lane per column
-    constexpr int E = 4 * F4;                      // channels per lane
     // per token: q, k, exp(g) [DK each], v [DV], beta, padded to 16 bytes; then the outputs [T][DV]
     constexpr int TOK = 3 * DK + DV + 4;
     constexpr int kPasses = DV / kMtCols;
@@ -81,18 +95,48 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
     }
     if (t_end == 0) return;  // nothing to apply, nothing to write
 
-    // the tokens' inputs -> shared memory (input layout [N, T, H, d])
-    for (int idx = tid; idx < t_end * TOK; idx += kMtThreads) {
-        const int t = idx / TOK, c = idx % TOK;
-        const size_t tok = ((size_t)n * T + t) * H + h;
-        float x;
-        if (c < DK) x = ld_elem(q, tok * DK + c);
-        else if (c < 2 * DK) x = ld_elem(k, tok * DK + (c - DK));
-        else if (c < 3 * DK) x = __expf(ld_elem(g, tok * DK + (c - 2 * DK)));
-        else if (c < 3 * DK + DV) x = ld_elem(v, tok * DV + (c - 3 * DK));
-        else if (c == 3 * DK + DV) x = ld_elem(beta, tok);
-        else continue;
-        sIn[idx] = x;
+    // the tokens' inputs -> shared memory (input layout [N, T, H, d]): 16-byte pieces of the
+    // q, k, g and v rows, four per thread in flight before any is used
+    {
+        constexpr int VEC = 16 / (int)sizeof(Tin);      // elements per piece
+        constexpr int NK = DK / VEC, NVV = DV / VEC;    // pieces per row
+        constexpr int PER_TOK = 3 * NK + NVV;
+        constexpr int UNR = 4;
+        const int total = t_end * PER_TOK;
+        for (int base = tid; base < total; base += UNR * kMtThreads) {
+            uint4 raw[UNR];
+            int dst[UNR];
+            bool is_g[UNR];
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                const int idx = base + u * kMtThreads;
+                if (idx >= total) continue;
+                const int t = idx / PER_TOK, c = idx % PER_TOK;
+                const size_t tok = ((size_t)n * T + t) * H + h;
+                const Tin *src;
+                if (c < NK) { src = q + tok * DK + c * VEC; dst[u] = c * VEC; }
+                else if (c < 2 * NK) { src = k + tok * DK + (c - NK) * VEC; dst[u] = DK + (c - NK) * VEC; }
+                else if (c < 3 * NK) { src = g + tok * DK + (c - 2 * NK) * VEC; dst[u] = 2 * DK + (c - 2 * NK) * VEC; }
+                else { src = v + tok * DV + (c - 3 * NK) * VEC; dst[u] = 3 * DK + (c - 3 * NK) * VEC; }
+                is_g[u] = c >= 2 * NK && c < 3 * NK;
+                dst[u] += t * TOK;
+                raw[u] = __ldg(reinterpret_cast<const uint4 *>(src));
+            }
+#pragma unroll
+            for (int u = 0; u < UNR; ++u) {
+                if (base + u * kMtThreads >= total) continue;
+                float x[VEC];
+                unpack16(raw[u], x);
+                if (is_g[u]) {
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) x[e] = __expf(x[e]);
+                }
+#pragma unroll
+                for (int e = 0; e < VEC; e += 4)
+                    *reinterpret_cast<float4 *>(sIn + dst[u] + e) = make_float4(x[e], x[e + 1], x[e + 2], x[e + 3]);
+            }
+        }
+        if (tid < t_end) sIn[tid * TOK + 3 * DK + DV] = ld_elem(beta, ((size_t)n * T + tid) * H + h);
     }
     float *sOut = sIn + T * TOK;
     __syncthreads();
@@ -120,20 +164,26 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
         }
         for (int t = 0; t < t_end; ++t) {
             const float *in = sIn + t * TOK;
-            float kk[E], qq[E], a[E];
+            // this lane's channels as pairs: the element-wise work runs on the paired fp32
+            // pipe (__fmul2_rn / __ffma2_rn: per element the same IEEE operations, in the
+            // same order, as scalar code)
+            float2 kk[2 * F4], qq[2 * F4], a[2 * F4];
 #pragma unroll
             for (int m = 0; m < F4; ++m) {
                 const int c = 4 * (sub + kMtLanesPerRow * m);
                 const float4 q4 = *reinterpret_cast<const float4 *>(in + c);
                 const float4 k4 = *reinterpret_cast<const float4 *>(in + DK + c);
                 const float4 a4 = *reinterpret_cast<const float4 *>(in + 2 * DK + c);
-                qq[4 * m] = q4.x; qq[4 * m + 1] = q4.y; qq[4 * m + 2] = q4.z; qq[4 * m + 3] = q4.w;
-                kk[4 * m] = k4.x; kk[4 * m + 1] = k4.y; kk[4 * m + 2] = k4.z; kk[4 * m + 3] = k4.w;
-                a[4 * m] = a4.x; a[4 * m + 1] = a4.y; a[4 * m + 2] = a4.z; a[4 * m + 3] = a4.w;
+                qq[2 * m] = make_float2(q4.x, q4.y); qq[2 * m + 1] = make_float2(q4.z, q4.w);
+                kk[2 * m] = make_float2(k4.x, k4.y); kk[2 * m + 1] = make_float2(k4.z, k4.w);
+                a[2 * m] = make_float2(a4.x, a4.y); a[2 * m + 1] = make_float2(a4.z, a4.w);
             }
             float kq = 0.f;
 #pragma unroll
-            for (int e = 0; e < E; ++e) kq = fmaf(kk[e], qq[e], kq);
+            for (int e = 0; e < 2 * F4; ++e) {
+                kq = fmaf(kk[e].x, qq[e].x, kq);
+                kq = fmaf(kk[e].y, qq[e].y, kq);
+            }
 #pragma unroll
             for (int off = 1; off < kMtLanesPerRow; off <<= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
             const float bt = in[3 * DK + DV];
@@ -142,30 +192,33 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
                 const int j = pass * kMtCols + warp * (32 / kMtLanesPerRow) + rw + r * kMtRowsPerPass;
                 // the tokens of a column are sequential, so the dot products keep four
                 // partial sums each (short dependency chains between tokens)
-                float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
+                float2 pk[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                float2 pq[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+                float2 x[2 * F4];
 #pragma unroll
                 for (int m = 0; m < F4; ++m) {
-                    float *x = reinterpret_cast<float *>(&s[r][m]);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        x[e] *= a[4 * m + e];
-                        pk[e] = fmaf(x[e], kk[4 * m + e], pk[e]);
-                        pq[e] = fmaf(x[e], qq[4 * m + e], pq[e]);
-                    }
+                    x[2 * m] = make_float2(s[r][m].x, s[r][m].y);
+                    x[2 * m + 1] = make_float2(s[r][m].z, s[r][m].w);
                 }
-                float sk = (pk[0] + pk[1]) + (pk[2] + pk[3]), sq = (pq[0] + pq[1]) + (pq[2] + pq[3]);
+#pragma unroll
+                for (int e = 0; e < 2 * F4; ++e) {
+                    x[e] = __fmul2_rn(x[e], a[e]);
+                    pk[e & 1] = __ffma2_rn(x[e], kk[e], pk[e & 1]);
+                    pq[e & 1] = __ffma2_rn(x[e], qq[e], pq[e & 1]);
+                }
+                float sk = (pk[0].x + pk[0].y) + (pk[1].x + pk[1].y);
+                float sq = (pq[0].x + pq[0].y) + (pq[1].x + pq[1].y);
 #pragma unroll
                 for (int off = 1; off < kMtLanesPerRow; off <<= 1) {
                     sk += __shfl_xor_sync(0xffffffffu, sk, off);
                     sq += __shfl_xor_sync(0xffffffffu, sq, off);
                 }
                 const float u = bt * (in[3 * DK + j] - sk);
+                const float2 uu = make_float2(u, u);
 #pragma unroll
-                for (int m = 0; m < F4; ++m) {
-                    float *x = reinterpret_cast<float *>(&s[r][m]);
+                for (int e = 0; e < 2 * F4; ++e) x[e] = __ffma2_rn(kk[e], uu, x[e]);
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) x[e] = fmaf(kk[4 * m + e], u, x[e]);
-                }
+                for (int m = 0; m < F4; ++m) s[r][m] = make_float4(x[2 * m].x, x[2 * m].y, x[2 * m + 1].x, x[2 * m + 1].y);
                 if (o && sub == 0) sOut[t * DV + j] = fmaf(u, kq, sq);
             }
             if (t + 1 == n_acc) {  // the column after the accepted prefix, in place
