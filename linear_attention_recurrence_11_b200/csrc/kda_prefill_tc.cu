@@ -10,17 +10,18 @@
 // Per chunk (G = per-channel cumulative log-decay, Gamma = exp(G)):
 //  1. TMA brings q, k, v (128-byte swizzled, straight into the operand tiles
 //     they become) and g (plain) into shared memory.
-//  2. CUDA cores: cumulative sums of g inside each 16-token subtile (the
-//     pages' g_min = -5 bound: 16 x 5 = 80, e^80 fits bf16 and fp32, so every
-//     exponent factor below is <= e^80) and the scaled bf16 operands of the
-//     decayed Grams. Column block j (tokens 16j..16j+15) of
+//  2. CUDA cores: cumulative sums of g inside each 16-token subtile and the
+//     scaled bf16 operands of the decayed Grams. Column block j (tokens
+//     32j..32j+31) of
 //        A_rs = beta_r sum_c k_rc k_sc e^{G_rc - G_sc},  P_rs = sum_c q_rc k_sc e^{G_rc - G_sc}
-//     is the product of a left operand k_r e^{G_r - G_start(j)} (stacked with
-//     q_r e^{G_r - G_start(j)}, rows r >= 16j) and a right operand
-//     k_s e^{G_start(j) - G_s}; the left factor is <= 1, the right one in
-//     [1, e^80]. For j = 0 the left operand is [Gamma*k ; Gamma*q] itself, the
-//     tile the state products use anyway.
-//  3. tcgen05.mma (M=128, N=16, K=128) x 4 -> TMEM; readout to A (fp32) and P (bf16).
+//     is the product of a left operand k_r e^{G_r - G_mid(j)} (stacked with
+//     q_r e^{G_r - G_mid(j)}, rows r >= 32j) and a right operand
+//     k_s e^{G_mid(j) - G_s}, referenced to the block's middle token
+//     mid(j) = 32j + 16. The pages' g_min = -5 bound keeps every factor within
+//     e^{+-80} (16 tokens x 5), which bf16 and fp32 hold; entries r < s of the
+//     product may overflow, and the readout drops them by selection. A left
+//     factor that underflows belongs to an entry below e^-12.
+//  3. tcgen05.mma (M=128, N=32, K=128) x 2 -> TMEM; readout to A (fp32) and P (bf16).
 //  4. CUDA cores: T = (I + A)^{-1} by 16 x 16 blocks (forward substitution on
 //     the diagonal blocks, then block rows by distance).
 //  5. tcgen05.mma: [W | Ut] = T Diag(beta) [Gamma*K | V]           (M=128 padded, K=64)
@@ -59,17 +60,18 @@ constexpr uint32_t OFF_R = 112 * KB;    // 16 KB  Gram right operand, K-major [s
 constexpr uint32_t OFF_PB = 128 * KB;   // 8 KB   rows 64..127 of the A operand [junk ; P], K-major, K = 64
 constexpr uint32_t OFF_L = 136 * KB;    // 80 KB  Gram left operands L3, L2, L1 (compact), Kh, then the aliases below
 constexpr uint32_t OFF_MISC = 216 * KB;
-// L region: compact left operands of column blocks 1..3, L_j has 2 (64 - 16 j) rows (K part,
-// then Q part); block 0's left operand is the [Gamma*K ; Gamma*Q] tile at OFF_WQ. A 128-row
-// operand read from a K-block start ends at most 52 KB into the region (block 1, K-block 1;
-// the rows past its own land in accumulator lanes that are never read). Kh, written with the
-// Gram operands and read by the last product of the chunk, sits past that point.
-__host__ __device__ constexpr uint32_t l_rows(int j) { return 2u * (64u - 16u * j); }
-__host__ __device__ constexpr uint32_t l_off(int j) { return j == 3 ? 0u : j == 2 ? 8u * KB : 24u * KB; }
+// L region: left operands of the two 32-token column blocks of the Gram, each referenced to
+// the block's middle token: L0 = [k ; q] rows 0..63 (128 rows, K-blocks 16 KB apart), L1 =
+// [k ; q] rows 32..63 (64 rows, K-blocks 8 KB apart). Read as 128-row operands, L1's second
+// K-block ends 24 KB past L1 (the rows past its own land in accumulator lanes that are never
+// read); Kh, written with the Gram operands and read by the last product of the chunk, starts
+// there.
+constexpr int kGramChains = 2;
+constexpr uint32_t L0_OFF = 0, L1_OFF = 32 * KB;
 // aliases inside the L region once the Gram MMAs are done
 constexpr uint32_t OFF_TB = OFF_L + 0;             // 16 KB  A operand T Diag(beta), K-major, 128 rows x 64
 // Gamma*K sits in rows 0..63 of the [-W ; Gamma*Q] tile until the W product is read out:
-// the same bytes are block 0's Gram operand (K-major A) and the W product's B (MN-major).
+// the W product reads it as its B operand (MN-major).
 constexpr uint32_t OFF_KT = OFF_WQ;
 // fp32 row strides (in floats) of the small matrices of the triangular inverse, chosen so that
 // the warp-level MMA fragments below read shared memory without bank conflicts: rows of an A
@@ -80,7 +82,7 @@ constexpr uint32_t OFF_AF = OFF_L + 16 * KB;       // 64 x LDA fp32  A          
 constexpr uint32_t OFF_UB = OFF_L + 0;             // 16 KB  B operand U, MN-major [tok][dv] (T Diag(beta) is done)
 constexpr uint32_t OFF_TF = OFF_L + 33 * KB;       // 64 x LDT fp32  T
 constexpr uint32_t OFF_XS = OFF_R;                 // 32 x LDX fp32 scratch (the Gram is done)
-static_assert(OFF_L + l_off(1) + l_rows(1) * 128 + 16 * KB <= OFF_KHAT, "Gram operand reads reach Kh");
+static_assert(OFF_L + L1_OFF + 8 * KB + 16 * KB <= OFF_KHAT, "Gram operand reads reach Kh");
 static_assert(OFF_AF >= OFF_TB + 16 * KB && OFF_AF + 64 * LDA * 4 <= OFF_TF, "A overlaps T Diag(beta) or T");
 static_assert(OFF_TF + 64 * LDT * 4 <= OFF_KHAT, "T overlaps Kh");
 static_assert(OFF_KHAT + 16 * KB <= OFF_MISC, "Kh overflows the L region");
@@ -240,7 +242,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     const uint32_t sbase = smem_u32(sm);
     uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     uint64_t *bar_mma = bar_tma + 1;
-    uint64_t *bar_gram = bar_tma + 2;  // 4 arrivals: one commit per Gram column block
+    uint64_t *bar_gram = bar_tma + 2;  // 2 arrivals: one commit per Gram column block
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + OFF_TMEMADDR);
     float *sBeta = reinterpret_cast<float *>(sm + OFF_BETA);
     float *sD = reinterpret_cast<float *>(sm + OFF_DSUM);
@@ -273,7 +275,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (tid == 0) {
         mbar_init(bar_tma, 1);
         mbar_init(bar_mma, 1);
-        mbar_init(bar_gram, NSUB);
+        mbar_init(bar_gram, kGramChains);
         fence_mbar_init();
         tma_prefetch_desc(&tm_q);
         tma_prefetch_desc(&tm_k);
@@ -363,16 +365,17 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
 
     // thread roles for the token-parallel passes: subtile ti (a pair of warps), half hh of
     // the subtile (rows 8hh..8hh+7), and a quad of channels (4 consecutive channels, 8 bytes)
-    // subtile of each warp pair; warps w and w + 4 share a scheduler, and subtile i
-    // writes i + 1 Gram left-operand rows per token, so pair subtiles 0 with 3 and 1 with 2
-    const int ti = (0x22331100 >> (4 * warp)) & 0xF;  // warps 0..7 -> 0,0,1,1,3,3,2,2
+    // subtile of each warp pair; warps w and w + 4 share a scheduler, and subtiles 0, 1
+    // write one Gram left-operand row pair per token, subtiles 2, 3 two, so each scheduler
+    // gets one of each
+    const int ti = warp >> 1;  // warps 0..7 -> 0,0,1,1,2,2,3,3
     const int hh = lane >> 4;                     // which 8 rows of the subtile
     const int cq = (warp & 1) * 16 + (lane & 15); // channel quad 0..31 (the two warps of a pair)
     const int c0 = 4 * cq;                        // first channel
     const int cblk = c0 >> 6;                     // 64-wide block of the channel
     const int cin = c0 & 63;                      // channel inside the block
     constexpr int HR = SUB / 2;                   // rows per thread
-    constexpr uint32_t idG = idesc_bf16_f32(128, 16, 0, 0);     // Gram: K-major x K-major, N = 16
+    constexpr uint32_t idG = idesc_bf16_f32(128, 32, 0, 0);     // Gram: K-major x K-major, N = 32
     constexpr uint32_t idKM = idesc_bf16_f32(128, 128, 0, 1);   // K-major A, MN-major B, N = 128
     constexpr uint32_t idMM = idesc_bf16_f32(128, 128, 1, 1);   // MN-major A and B, N = 128
 
@@ -502,17 +505,19 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                     make_float4(ed[0][0] * ed[1][0] * ed[2][0] * ed[3][0], ed[0][1] * ed[1][1] * ed[2][1] * ed[3][1],
                                 ed[0][2] * ed[1][2] * ed[2][2] * ed[3][2], ed[0][3] * ed[1][3] * ed[2][3] * ed[3][3]);
             }
-            float E[NSUB][4];  // E[j] = exp(G_start(ti) - G_start(j)) for j = 1..ti (1 for j = ti)
+            // column block b (tokens 32b..32b+31) is referenced to its middle token 32b + 16:
+            // its left operand rows are x_r e^{G_r - G_mid(b)} (r >= 32b), its right operand
+            // rows k_s e^{G_mid(b) - G_s}; every factor lies in [e^-80, e^80] within a block.
+            // Here as multiples of this subtile's own factors (relative to its start):
+            //   el0 = e^{G_start(ti) - G_16}, el1 = e^{G_start(ti) - G_48} (ti >= 2),
+            //   er  = e^{G_mid(block of ti) - G_start(ti)}
+            float el0[4], el1[4], er[4];
 #pragma unroll
-            for (int j = 0; j < NSUB; ++j)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    float acc = 1.f;
-#pragma unroll
-                    for (int m = 0; m < NSUB; ++m)
-                        if (m >= j && m < ti) acc *= ed[m][e];
-                    E[j][e] = acc;
-                }
+            for (int e = 0; e < 4; ++e) {
+                el0[e] = ti == 0 ? ex2(-Dm[0][e]) : ti == 1 ? 1.f : ti == 2 ? ed[1][e] : ed[1][e] * ed[2][e];
+                el1[e] = ti == 2 ? ex2(-Dm[2][e]) : 1.f;
+                er[e] = ti == 0 ? ed[0][e] : ti == 2 ? ed[2][e] : 1.f;
+            }
 #pragma unroll
             for (int rr = 0; rr < HR; ++rr)
 #pragma unroll
@@ -551,27 +556,29 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         qx[e] *= iq;
                     }
                 }
-                // right operand row r (column block ti): k_r e^{G_start(ti) - G_r}; and Kh row r:
+                // right operand row r: k_r e^{G_mid - G_r}; and Kh row r:
                 // k_r e^{G_C - G_r} = (k_r e^{G_start(ti) - G_r}) e^{G_C - G_start(ti)}, both factors bounded
                 float kr[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) kr[e] = kx[e] * Fi[rr][e];
-                st4(rrow + off_r, kr[0], kr[1], kr[2], kr[3]);
+                st4(rrow + off_r, kr[0] * er[0], kr[1] * er[1], kr[2] * er[2], kr[3] * er[3]);
                 st4(khrow + off_r, kr[0] * post[0], kr[1] * post[1], kr[2] * post[2], kr[3] * post[3]);
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     kf[e] = kx[e] * F[rr][e];
                     qf[e] = qx[e] * F[rr][e];
                 }
-#pragma unroll
-                for (int j = 1; j < NSUB; ++j) {
-                    if (j > ti) continue;
-                    const uint32_t rows = l_rows(j), hr = rows / 2;
-                    uint8_t *Lb = sm + OFF_L + l_off(j) + cblk * rows * 128;
-                    st4(Lb + sw128_offset(r - 16 * j, cin), kf[0] * E[j][0], kf[1] * E[j][1], kf[2] * E[j][2],
-                        kf[3] * E[j][3]);
-                    st4(Lb + sw128_offset(hr + r - 16 * j, cin), qf[0] * E[j][0], qf[1] * E[j][1],
-                        qf[2] * E[j][2], qf[3] * E[j][3]);
+                {  // left operands: block 0 (every row), block 1 (rows >= 32)
+                    uint8_t *L0 = sm + OFF_L + L0_OFF + cblk * 16 * KB;
+                    st4(L0 + off_r, kf[0] * el0[0], kf[1] * el0[1], kf[2] * el0[2], kf[3] * el0[3]);
+                    st4(L0 + off_q, qf[0] * el0[0], qf[1] * el0[1], qf[2] * el0[2], qf[3] * el0[3]);
+                    if (ti >= 2) {
+                        uint8_t *L1 = sm + OFF_L + L1_OFF + cblk * 8 * KB;
+                        st4(L1 + sw128_offset(r - 32, cin), kf[0] * el1[0], kf[1] * el1[1], kf[2] * el1[2],
+                            kf[3] * el1[3]);
+                        st4(L1 + sw128_offset(r, cin), qf[0] * el1[0], qf[1] * el1[1], qf[2] * el1[2],
+                            qf[3] * el1[3]);
+                    }
                 }
                 st4(qrow + off_q, qf[0] * pg[0], qf[1] * pg[1], qf[2] * pg[2], qf[3] * pg[3]);  // Gamma * q
                 st4(qrow + off_r, kf[0] * pg[0], kf[1] * pg[1], kf[2] * pg[2], kf[3] * pg[3]);  // Gamma * k, row r
@@ -580,14 +587,14 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         fence_proxy_async_smem();
         __syncthreads();
 
-        // ---- Gram MMAs: column block j -> TMEM columns 16j..16j+15, issued by lane 0 of warp j
-        if (lane == 0 && warp < NSUB) {
+        // ---- Gram MMAs: column block j -> TMEM columns 32j..32j+31, issued by lane 0 of warp j
+        if (lane == 0 && warp < kGramChains) {
             const int j = warp;
             tc_fence_after();
-            Opnd A = (j == 0) ? Opnd{sbase + OFF_WQ, false, 16 * KB, 0}
-                              : Opnd{sbase + OFF_L + l_off(j), false, l_rows(j) * 128u, 0};
-            Opnd B{sbase + OFF_R + 16u * j * 128u, false, 8 * KB, 0};
-            mma_chain<D / 16>(tmem + TM_GRAM + 16u * j, A, B, idG, false);
+            Opnd A = (j == 0) ? Opnd{sbase + OFF_L + L0_OFF, false, 16 * KB, 0}
+                              : Opnd{sbase + OFF_L + L1_OFF, false, 8 * KB, 0};
+            Opnd B{sbase + OFF_R + 32u * j * 128u, false, 8 * KB, 0};
+            mma_chain<D / 16>(tmem + TM_GRAM + 32u * j, A, B, idG, false);
             mma_commit(bar_gram);
         }
         if (more && tid == 0) issue_k(tokn);  // the k tile is consumed (Kh is written with the Gram operands)
@@ -598,40 +605,40 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             if (__syncthreads_or(!ok)) { aborted = true; break; }
         }
 
-        // ---- phase 2: Gram readout -> A (fp32, strictly lower, times beta_r), P (bf16, lower)
+        // ---- phase 2: Gram readout -> A (fp32, strictly lower, times beta_r), P (bf16, lower).
+        // Warps of column half j read block j's 32 columns; the masks select (never multiply)
+        // so that the upper-triangle entries, which may overflow, are dropped.
         {
             float v2[2][16];
-            tmem_ld16(tmem + tlane + TM_GRAM + 16u * (2 * half), v2[0]);
-            tmem_ld16(tmem + tlane + TM_GRAM + 16u * (2 * half + 1), v2[1]);
+            tmem_ld16(tmem + tlane + TM_GRAM + 32u * half, v2[0]);
+            tmem_ld16(tmem + tlane + TM_GRAM + 32u * half + 16u, v2[1]);
             tmem_wait_ld();
+            const int j = half;
+            const int m = 32 * quarter + lane;
+            const int kr = 64 - 32 * j;  // k rows of block j's left operand (rows >= 32j)
+            if (m < kr) {
+                const int r = 32 * j + m;
+                const float b = sBeta[r];
+                float4 *arow = reinterpret_cast<float4 *>(AF + r * LDA + 32 * j);
 #pragma unroll
-            for (int jj = 0; jj < 2; ++jj) {
-                const int j = 2 * half + jj;
-                const float *v = v2[jj];
-                const int m = 32 * quarter + lane;
-                const int kr = 64 - 16 * j;
-                if (m < kr) {
-                    const int r = 16 * j + m;
-                    const float b = sBeta[r];
-                    float4 *arow = reinterpret_cast<float4 *>(AF + r * LDA + 16 * j);
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float *v = v2[q4 >> 2] + 4 * (q4 & 3);
+                    const int s = 32 * j + 4 * q4;
+                    arow[q4] = make_float4((s < r) ? b * v[0] : 0.f, (s + 1 < r) ? b * v[1] : 0.f,
+                                           (s + 2 < r) ? b * v[2] : 0.f, (s + 3 < r) ? b * v[3] : 0.f);
+                }
+            } else if (m < 2 * kr) {
+                const int r = 32 * j + (m - kr);
+                uint8_t *prow = sm + OFF_PB;
 #pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        const int s = 16 * j + 4 * q4;
-                        arow[q4] = make_float4((s < r) ? b * v[4 * q4] : 0.f, (s + 1 < r) ? b * v[4 * q4 + 1] : 0.f,
-                                               (s + 2 < r) ? b * v[4 * q4 + 2] : 0.f, (s + 3 < r) ? b * v[4 * q4 + 3] : 0.f);
-                    }
-                } else if (m < 2 * kr) {
-                    const int r = 16 * j + (m - kr);
-                    uint8_t *prow = sm + OFF_PB;
-#pragma unroll
-                    for (int s2 = 0; s2 < 16; s2 += 2) {
-                        const int s = 16 * j + s2;
-                        st_bf2(prow + sw128_offset(r, s), (s <= r) ? v[s2] : 0.f, (s + 1 <= r) ? v[s2 + 1] : 0.f);
-                    }
-                    if (r < 16 * (j + 1)) {  // diagonal block: zero the blocks to its right
-                        for (int s = 16 * (j + 1); s < C; s += 8)
-                            *reinterpret_cast<uint4 *>(prow + sw128_offset(r, s)) = make_uint4(0, 0, 0, 0);
-                    }
+                for (int s2 = 0; s2 < 32; s2 += 2) {
+                    const int s = 32 * j + s2;
+                    const float *v = v2[s2 >> 4] + (s2 & 15);
+                    st_bf2(prow + sw128_offset(r, s), (s <= r) ? v[0] : 0.f, (s + 1 <= r) ? v[1] : 0.f);
+                }
+                if (j == 0 && r < 32) {  // diagonal block of block 0: zero block 1's columns
+                    for (int s = 32; s < C; s += 8)
+                        *reinterpret_cast<uint4 *>(prow + sw128_offset(r, s)) = make_uint4(0, 0, 0, 0);
                 }
             }
         }
