@@ -18,6 +18,7 @@
 // packed sequences. M_p is a dk x dk matrix kept in the state layout
 // ([column][dk], so pass A runs with dv = dk).
 #include "kda_internal.cuh"
+#include "kda_sm100.cuh"
 
 namespace kda {
 namespace {
@@ -54,36 +55,64 @@ __global__ void kda_segment_init_kernel(int32_t *cu_seg, float *Mbuf, int B, int
 // columns ci + 16 c, so a warp's reads of Ms are consecutive and of X a broadcast.
 constexpr int kRowsPerCta = 16;
 
+// The steps of a scan are sequential, so each step's transition Ms_p (DK x DK) and this
+// CTA's rows of Zs_p are brought into shared memory two steps ahead by bulk copies (two
+// buffers, one mbarrier each; no tensor map, no multicast): the copies of steps p + 1 and
+// p + 2 are in flight while step p computes. The waits are bounded; a timeout sets
+// KDA_ERR_TIMEOUT in the status word and the CTA stops (its copies in flight land first).
+constexpr long long kScanWaitCycles = 2000000000LL;  // ~1 s at 2 GHz
+
 template <int DK, int DV>
 __global__ void __launch_bounds__(kSegThreads)
-kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float *Sin, float *ST, int P, int H) {
+kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float *Sin, float *ST, int P, int H,
+                    int *dev_status) {
+    using namespace sm100;
     constexpr int TI = DK / 16;                      // columns per thread
     constexpr int RPI = kSegThreads / 16;            // rows covered per pass of the threads (16)
     constexpr int RP = kRowsPerCta / RPI;            // rows per thread (1)
-    extern __shared__ float smem[];
+    constexpr uint32_t kMBytes = DK * DK * sizeof(float), kZBytes = kRowsPerCta * DK * sizeof(float);
+    extern __shared__ __align__(16) float smem[];
     float *Xs = smem;                                // [kRowsPerCta][DK]
-    float *Ms = smem + kRowsPerCta * DK;             // [DK][DK]
+    float *Ms = Xs + kRowsPerCta * DK;               // 2 x [DK][DK]
+    float *Zs = Ms + 2 * DK * DK;                    // 2 x [kRowsPerCta][DK]
+    uint64_t *bar = reinterpret_cast<uint64_t *>(Zs + 2 * kRowsPerCta * DK);
     const int b = blockIdx.x / H, h = blockIdx.x % H, j0 = blockIdx.y * kRowsPerCta, tid = threadIdx.x;
     const int r0 = tid / 16, ci = tid % 16;
     const size_t sbase = (((size_t)b * H + h) * DV + j0) * DK;
-    for (int e = tid; e < kRowsPerCta * DK; e += kSegThreads) Xs[e] = S0 ? S0[sbase + e] : 0.f;
-    for (int p = 0; p < P; ++p) {
+    auto fetch = [&](int p) {  // step p's Ms and Zs rows -> buffer p & 1 (one thread)
         const size_t u = (size_t)b * P + p;
-        const size_t xbase = ((u * H + h) * DV + j0) * DK, mbase = (u * H + h) * DK * DK;
-        for (int e = 4 * tid; e < DK * DK; e += 4 * kSegThreads)
-            *reinterpret_cast<float4 *>(Ms + e) = *reinterpret_cast<const float4 *>(Mbuf + mbase + e);
-        __syncthreads();
+        const int buf = p & 1;
+        mbar_arrive_expect_tx(&bar[buf], kMBytes + kZBytes);
+        bulk_load(Ms + buf * DK * DK, Mbuf + (u * H + h) * DK * DK, kMBytes, &bar[buf]);
+        bulk_load(Zs + buf * kRowsPerCta * DK, Zbuf + ((u * H + h) * DV + j0) * DK, kZBytes, &bar[buf]);
+    };
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        fence_mbar_init();
+        for (int p = 0; p < 2 && p < P; ++p) fetch(p);
+    }
+    for (int e = tid; e < kRowsPerCta * DK; e += kSegThreads) Xs[e] = S0 ? S0[sbase + e] : 0.f;
+    __syncthreads();
+    int p = 0;
+    bool ok = true;
+    for (; p < P; ++p) {
+        const int buf = p & 1;
+        const bool got = mbar_wait_bounded(&bar[buf], (uint32_t)(p >> 1) & 1u, kScanWaitCycles);
+        if (__syncthreads_or(!got)) { ok = false; break; }
+        const float *M = Ms + buf * DK * DK, *Z = Zs + buf * kRowsPerCta * DK;
+        const size_t xbase = ((((size_t)b * P + p) * H + h) * DV + j0) * DK;
         for (int e = tid; e < kRowsPerCta * DK; e += kSegThreads) Sin[xbase + e] = Xs[e];
         float acc[RP][TI];
 #pragma unroll
         for (int rr = 0; rr < RP; ++rr)
 #pragma unroll
-            for (int c = 0; c < TI; ++c) acc[rr][c] = Zbuf[xbase + (size_t)(r0 + RPI * rr) * DK + ci + 16 * c];
+            for (int c = 0; c < TI; ++c) acc[rr][c] = Z[(r0 + RPI * rr) * DK + ci + 16 * c];
 #pragma unroll 8
         for (int a = 0; a < DK; ++a) {
             float mv[TI];
 #pragma unroll
-            for (int c = 0; c < TI; ++c) mv[c] = Ms[a * DK + ci + 16 * c];
+            for (int c = 0; c < TI; ++c) mv[c] = M[a * DK + ci + 16 * c];
 #pragma unroll
             for (int rr = 0; rr < RP; ++rr) {
                 const float xv = Xs[(r0 + RPI * rr) * DK + a];
@@ -91,12 +120,24 @@ kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float
                 for (int c = 0; c < TI; ++c) acc[rr][c] = fmaf(xv, mv[c], acc[rr][c]);
             }
         }
-        __syncthreads();  // every thread has read X and Ms_p
+        __syncthreads();  // every thread has read X and this step's buffer
+        if (tid == 0 && p + 2 < P) {
+            fence_proxy_async_smem();
+            fetch(p + 2);
+        }
 #pragma unroll
         for (int rr = 0; rr < RP; ++rr)
 #pragma unroll
             for (int c = 0; c < TI; ++c) Xs[(r0 + RPI * rr) * DK + ci + 16 * c] = acc[rr][c];
         __syncthreads();
+    }
+    if (!ok) {
+        if (tid == 0) {
+            if (dev_status) atomicExch(dev_status, (int)KDA_ERR_TIMEOUT);
+            const int issued = p + 2 < P ? p + 2 : P;  // steps p .. issued - 1 may be in flight
+            for (int i = p; i < issued; ++i) mbar_wait_bounded(&bar[i & 1], (uint32_t)(i >> 1) & 1u, kScanWaitCycles);
+        }
+        return;
     }
     if (ST)
         for (int e = tid; e < kRowsPerCta * DK; e += kSegThreads) ST[sbase + e] = Xs[e];
@@ -104,12 +145,13 @@ kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float
 
 template <int DK, int DV>
 cudaError_t launch_scan_t(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin) {
-    const size_t smem = (size_t)(kRowsPerCta * DK + DK * DK) * sizeof(float);
+    const size_t smem = (size_t)(kRowsPerCta * DK + 2 * DK * DK + 2 * kRowsPerCta * DK) * sizeof(float) + 16;
     cudaError_t e = cudaFuncSetAttribute(kda_kcp_scan_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)(s.B * s.H), DV / kRowsPerCta);
-    kda_kcp_scan_kernel<DK, DV><<<grid, kSegThreads, smem, s.stream>>>(s.S0, Mbuf, Zbuf, Sin, s.ST, s.P, s.H);
+    kda_kcp_scan_kernel<DK, DV><<<grid, kSegThreads, smem, s.stream>>>(s.S0, Mbuf, Zbuf, Sin, s.ST, s.P, s.H,
+                                                                      s.dev_status);
     return cudaGetLastError();
 }
 
