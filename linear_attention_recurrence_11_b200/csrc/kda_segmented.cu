@@ -52,8 +52,10 @@ __global__ void kda_segment_init_kernel(int32_t *cu_seg, float *Mbuf, int B, int
 // Ms[a][i] = M[i][a]. So one CTA per (sequence b, head h, block of kRowsPerCta rows)
 // runs the whole scan for its rows: X <- S0 rows (or 0); for p = 0..P-1 { Sin[p] = X;
 // X = X Ms_p + Zs_p }; S_T = X. fp32. Thread (r, ci) owns row r of the block and the
-// columns ci + 16 c, so a warp's reads of Ms are consecutive and of X a broadcast.
-constexpr int kRowsPerCta = 16;
+// columns ci + 32 c, so a warp's reads of Ms are consecutive and of X a broadcast.
+// Blocks of 8 rows: 128 CTAs for 8 heads x 128 rows.
+constexpr int kRowsPerCta = 8;
+constexpr int kScanTpr = kSegThreads / kRowsPerCta;  // threads per row (32)
 
 // The steps of a scan are sequential, so each step's transition Ms_p (DK x DK) and this
 // CTA's rows of Zs_p are brought into shared memory two steps ahead by bulk copies (two
@@ -67,9 +69,10 @@ __global__ void __launch_bounds__(kSegThreads)
 kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float *Sin, float *ST, int P, int H,
                     int *dev_status) {
     using namespace sm100;
-    constexpr int TI = DK / 16;                      // columns per thread
-    constexpr int RPI = kSegThreads / 16;            // rows covered per pass of the threads (16)
+    constexpr int TI = DK / kScanTpr;                // columns per thread
+    constexpr int RPI = kSegThreads / kScanTpr;      // rows covered per pass of the threads (8)
     constexpr int RP = kRowsPerCta / RPI;            // rows per thread (1)
+    static_assert(TI >= 1 && RP == 1, "scan thread mapping");
     constexpr uint32_t kMBytes = DK * DK * sizeof(float), kZBytes = kRowsPerCta * DK * sizeof(float);
     extern __shared__ __align__(16) float smem[];
     float *Xs = smem;                                // [kRowsPerCta][DK]
@@ -77,7 +80,7 @@ kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float
     float *Zs = Ms + 2 * DK * DK;                    // 2 x [kRowsPerCta][DK]
     uint64_t *bar = reinterpret_cast<uint64_t *>(Zs + 2 * kRowsPerCta * DK);
     const int b = blockIdx.x / H, h = blockIdx.x % H, j0 = blockIdx.y * kRowsPerCta, tid = threadIdx.x;
-    const int r0 = tid / 16, ci = tid % 16;
+    const int r0 = tid / kScanTpr, ci = tid % kScanTpr;
     const size_t sbase = (((size_t)b * H + h) * DV + j0) * DK;
     auto fetch = [&](int p) {  // step p's Ms and Zs rows -> buffer p & 1 (one thread)
         const size_t u = (size_t)b * P + p;
@@ -107,12 +110,12 @@ kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float
 #pragma unroll
         for (int rr = 0; rr < RP; ++rr)
 #pragma unroll
-            for (int c = 0; c < TI; ++c) acc[rr][c] = Z[(r0 + RPI * rr) * DK + ci + 16 * c];
+            for (int c = 0; c < TI; ++c) acc[rr][c] = Z[(r0 + RPI * rr) * DK + ci + kScanTpr * c];
 #pragma unroll 8
         for (int a = 0; a < DK; ++a) {
             float mv[TI];
 #pragma unroll
-            for (int c = 0; c < TI; ++c) mv[c] = M[a * DK + ci + 16 * c];
+            for (int c = 0; c < TI; ++c) mv[c] = M[a * DK + ci + kScanTpr * c];
 #pragma unroll
             for (int rr = 0; rr < RP; ++rr) {
                 const float xv = Xs[(r0 + RPI * rr) * DK + a];
@@ -128,7 +131,7 @@ kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float
 #pragma unroll
         for (int rr = 0; rr < RP; ++rr)
 #pragma unroll
-            for (int c = 0; c < TI; ++c) Xs[(r0 + RPI * rr) * DK + ci + 16 * c] = acc[rr][c];
+            for (int c = 0; c < TI; ++c) Xs[(r0 + RPI * rr) * DK + ci + kScanTpr * c] = acc[rr][c];
         __syncthreads();
     }
     if (!ok) {
