@@ -478,6 +478,18 @@ def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):
     return res
 
 
+def multi_decode_algorithmic(B, H, T, dk, dv, accepted):
+    """Bytes one speculative round must move (bf16 inputs and outputs, fp32 states):
+    the verification reads every state and the inputs of all T tokens and writes all
+    outputs; the commit reads and writes the states of the requests with an accepted
+    token and reads the accepted tokens' inputs."""
+    state = dk * dv * 4
+    per_tok = (3 * dk + dv + 1) * 2
+    written = sum(1 for a in accepted if a > 0)
+    return ((B + 2 * written) * H * state + (B * T + sum(accepted)) * H * per_tok
+            + B * T * H * dv * 2)
+
+
 def multi_decode_measure(args, device, peaks, max_ranks, world, w, S, rounds=10):
     """Speculative decoding rounds on the same states: T draft tokens per request,
     a verification call (outputs of all T, states untouched) then a commit call
@@ -509,14 +521,8 @@ def multi_decode_measure(args, device, peaks, max_ranks, world, w, S, rounds=10)
     b.record(stream)
     torch.cuda.synchronize(device)
     ms = max_ranks(a.elapsed_time(b)) / rounds
-    state = w.dk * w.dv * 4
-    per_tok = (3 * w.dk + w.dv + 1) * 2
-    written = int((acc > 0).sum().item())
     accepted = int(acc.sum().item())
-    # verify: every state read, the inputs of all T tokens, all outputs; commit: the states of
-    # requests with an accepted token read and written, the inputs of the accepted tokens
-    bytes_round = ((w.B + 2 * written) * w.H * state
-                   + (w.B * T + accepted) * w.H * per_tok + w.B * T * w.H * w.dv * 2)
+    bytes_round = multi_decode_algorithmic(w.B, w.H, T, w.dk, w.dv, acc.tolist())
     gbs = bytes_round / (ms / 1e3) / 1e9
     return {"draft_tokens": T, "ms_per_round": ms, "accepted_tokens_per_round": accepted * world,
             "accepted_tokens_per_s": world * accepted / (ms / 1e3),

@@ -36,3 +36,15 @@ def test_algorithmic_counts():
     bd, _ = bench.decode_algorithmic(256, 96, 128, 128, 2)
     assert bd == 256 * 96 * (2 * 128 * 128 * 4 + 4 * 128 * 2 + 2 + 128 * 2)
     assert bench.weak_scaling_value(100, 10, 1000.0, 4) == 4000.0
+
+
+def test_multi_decode_algorithmic_bytes():
+    import bench
+    state = 128 * 128 * 4
+    per_tok = (3 * 128 + 128 + 1) * 2
+    # nothing accepted: the verification alone (states read once, all inputs, all outputs)
+    assert bench.multi_decode_algorithmic(2, 3, 4, 128, 128, [0, 0]) == \
+        2 * 3 * state + 2 * 4 * 3 * per_tok + 2 * 4 * 3 * 128 * 2
+    # one request commits 3 tokens: its states read and written, 3 more tokens' inputs
+    assert bench.multi_decode_algorithmic(2, 3, 4, 128, 128, [3, 0]) - \
+        bench.multi_decode_algorithmic(2, 3, 4, 128, 128, [0, 0]) == 2 * 3 * state + 3 * 3 * per_tok
