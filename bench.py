@@ -352,7 +352,6 @@ def run_ours(args, rank, world, device):
     if not args.no_decode and args.workload == "prefill":
         res["decode"] = decode_measure(args, device, peaks, barrier, max_ranks, world,
                                        steps=args.decode_steps)
-        res["gpu_launches"] += res["decode"]["gpu_launches"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline_prefill(inp, w, args.cpu_seconds)
     return res
@@ -474,7 +473,6 @@ def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):
             "requests": w.B, "l2": f"state {w.B * w.H * w.dk * w.dv * 4 / 1e9:.2f} GB per step, larger than L2"}
     if args.draft_tokens > 0:
         res["multi_token"] = multi_decode_measure(args, device, peaks, max_ranks, world, w, S)
-        res["gpu_launches"] += res["multi_token"]["gpu_launches"]
     return res
 
 
