@@ -8,7 +8,7 @@ import torch
 
 from linear_attention_recurrence_11_b200.inputs import WORKLOADS, make_inputs, to_f64, workload_inputs
 
-from kda_testutil import TOL, case, compare_units, oracle_forward, rel
+from kda_testutil import TOL, case, compare_units, oracle_forward, parity_streamed, rel
 
 pytestmark = pytest.mark.gpu
 
@@ -41,7 +41,7 @@ def check_full(K, oracle_mod, inp, chunk, dtype, path, cu=None):
     o, ST = run(K, inp, chunk, path)
     o_ref, ST_ref = oracle_forward(oracle_mod, inp)
     N, H = ST.shape[0], ST.shape[1]
-    e_o, e_s = compare_units(o, ST, o_ref, ST_ref, all_units(N, H), cu)
+    e_o, e_s = compare_units(o, ST, o_ref, ST_ref, all_units(N, H), cu, tol=TOL[dtype])
     assert e_o < TOL[dtype] and e_s < TOL[dtype], (e_o, e_s)
     return e_o, e_s
 
@@ -79,7 +79,7 @@ def test_varlen_with_edge_lengths(K, oracle_mod, path):
     inp["cu_seqlens"] = torch.tensor(cu, device="cuda")
     o, ST = run(K, inp, 64, path)
     o_ref, ST_ref = oracle_forward(oracle_mod, inp)
-    e_o, e_s = compare_units(o, ST, o_ref, ST_ref, all_units(len(lens), 2), cu)
+    e_o, e_s = compare_units(o, ST, o_ref, ST_ref, all_units(len(lens), 2), cu, tol=TOL["bf16"])
     assert e_o < TOL["bf16"] and e_s < TOL["bf16"], (e_o, e_s)
     # the empty sequence passes its state through untouched
     assert torch.equal(ST[3], inp["S0"][3])
@@ -103,7 +103,7 @@ def test_varlen_many_sequences(K, oracle_mod, nseq):
     picks = [int(i) for i in np.argsort(-lens)[:3]] + [int(np.argmin(lens)), nseq - 1]
     units = [(n, h) for n in picks for h in range(H)]
     o_ref, ST_ref = oracle_forward(oracle_mod, inp, units=units)
-    e_o, e_s = compare_units(o, ST, o_ref, ST_ref, units, cu)
+    e_o, e_s = compare_units(o, ST, o_ref, ST_ref, units, cu, tol=TOL["bf16"])
     assert e_o < TOL["bf16"] and e_s < TOL["bf16"], (e_o, e_s)
     zero = np.nonzero(lens == 0)[0]
     assert torch.equal(ST[zero], inp["S0"][zero])
@@ -226,29 +226,26 @@ def test_decode_full_size_1000_steps_sampled(K, oracle_mod):
 
 # ------------------------------------------------------- full-size prefill
 
-def test_prefill_h96_T8192_sampled_heads(K, oracle_mod):
+def test_prefill_h96_T8192_all_heads(K, oracle_mod):
     """The layer-shape workload at full size, in the launch configuration the
-    benchmark times; three seeded heads recomputed by the oracle in full."""
+    benchmark times: every one of the 96 heads recomputed by the oracle in
+    full (on all host cores), the pooled and the worst per-head error gated."""
     w = WORKLOADS["prefill_h96_T8192_d128_bf16"]
     inp = workload_inputs(w, device="cuda")
     o, ST = run(K, inp, w.chunk, "auto")
     assert torch.isfinite(o).all() and torch.isfinite(ST).all()
-    units = [(0, 0), (0, 47), (0, 95)]
-    o_ref, ST_ref = oracle_forward(oracle_mod, inp, units=units)
-    e_o, e_s = compare_units(o, ST, o_ref, ST_ref, units)
-    assert e_o < TOL["bf16"] and e_s < TOL["bf16"], (e_o, e_s)
+    parity_streamed(oracle_mod, inp, o, ST, all_units(1, w.H), TOL["bf16"], label="h96_T8192")
 
 
 def test_varlen_full_size_sampled(K, oracle_mod):
-    """Eight packed long sequences (log-uniform lengths in [4096, 131072]);
-    the oracle follows a seeded subset of (sequence, head) units end to end."""
+    """Eight packed long sequences (log-uniform lengths in [4096, 131072]); the
+    oracle follows at least one head of every sequence end to end (a different
+    head for each), plus two more heads of the longest and the shortest."""
     w = WORKLOADS["varlen_h96_8seq_d128_bf16"]
     inp = workload_inputs(w, device="cuda")
     o, ST = run(K, inp, w.chunk, "auto")
     assert torch.isfinite(ST).all()
-    cu = w.cu_seqlens()
     order = sorted(range(w.num_seqs), key=lambda n: w.seqlens[n])
-    units = [(order[0], 5), (order[1], 60), (order[-1], 17)]
-    o_ref, ST_ref = oracle_forward(oracle_mod, inp, units=units)
-    e_o, e_s = compare_units(o, ST, o_ref, ST_ref, units, cu)
-    assert e_o < TOL["bf16"] and e_s < TOL["bf16"], (e_o, e_s)
+    units = [(n, (13 * n + 5) % w.H) for n in range(w.num_seqs)]
+    units += [(order[0], 60), (order[-1], 17)]
+    parity_streamed(oracle_mod, inp, o, ST, units, TOL["bf16"], label="varlen_8seq")

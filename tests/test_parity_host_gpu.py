@@ -76,7 +76,7 @@ def test_oracle_parity_through_host_buffers(K, oracle_mod, dtype):
     o, S_T = run_host(K, to_host(inp), 64 if dtype == "bf16" else 32, 128 if dtype == "bf16" else 64)
     o_ref, S_ref = oracle_forward(oracle_mod, inp)
     units = [(b, h) for b in range(2) for h in range(2)]
-    e_o, e_s = compare_units(o, S_T, o_ref, S_ref, units)
+    e_o, e_s = compare_units(o, S_T, o_ref, S_ref, units, tol=TOL[dtype])
     assert e_o < TOL[dtype] and e_s < TOL[dtype], (e_o, e_s)
 
 
@@ -124,5 +124,5 @@ def test_benchmark_workload_sampled(K, oracle_mod):
     assert torch.equal(o, o_d) and torch.equal(S_T, S_d)
     units = [(0, 0), (0, 57)]
     o_ref, S_ref = oracle_forward(oracle_mod, inp, units=units)
-    e_o, e_s = compare_units(o, S_T, o_ref, S_ref, units)
+    e_o, e_s = compare_units(o, S_T, o_ref, S_ref, units, tol=TOL["bf16"])
     assert e_o < TOL["bf16"] and e_s < TOL["bf16"], (e_o, e_s)

@@ -39,7 +39,7 @@ def test_snapshots(K, oracle_mod, dtype, dk, dv, chunk, T, every, path):
     ns = T // every
     assert Ssn.shape == (B, ns, H, dv, dk)
     o_ref, ST_ref = oracle_forward(oracle_mod, inp)
-    e_o, e_s = compare_units(o, ST, o_ref, ST_ref, [(b, h) for b in range(B) for h in range(H)])
+    e_o, e_s = compare_units(o, ST, o_ref, ST_ref, [(b, h) for b in range(B) for h in range(H)], tol=TOL[dtype])
     assert e_o < TOL[dtype] and e_s < TOL[dtype], (e_o, e_s)
     for b in range(B):
         for h in range(H):
