@@ -51,11 +51,16 @@ def test_kcp_composition_error_at_machine_precision(oracle_mod):
     S_in = oracle_mod.kcp_scan(np.stack(Ms), np.stack(Ss))
     err_scan = np.max(np.abs(S_in[-1] - S_seq))
     eps = np.finfo(np.float64).eps
-    # the pages' figures are themselves ~1e2 eps-scaled errors on O(0.1) values
-    assert fig["kcp_composition_max_error"] < 100 * eps
-    assert fig["kcp_scan_4ranks_max_error"] < 100 * eps
+    # The pages print absolute errors (6.94e-18 for one composition, 1.39e-17 for
+    # the 4-rank scan) on a case of unstated size and magnitude; read as "exact up
+    # to rounding", they fix the level, not the digits. The oracle's own errors,
+    # measured here on a case of its own, must sit at that level: a few ulp of the
+    # state's magnitude, and the scan (three compositions in a row) no more than a
+    # few times the single composition, as in the pages' pair of figures.
     assert err_comp <= 64 * eps * max(scale, 1.0)
     assert err_scan <= 64 * eps * max(scale, 1.0)
+    ratio_pages = fig["kcp_scan_4ranks_max_error"] / fig["kcp_composition_max_error"]
+    assert err_scan <= 4 * ratio_pages * max(err_comp, eps * scale)
 
 
 def test_state_size_figure():

@@ -12,7 +12,7 @@ from fractions import Fraction
 import numpy as np
 import pytest
 
-TOL = 1e-13
+TOL = 1e-14
 
 
 def rel(x, ref):
