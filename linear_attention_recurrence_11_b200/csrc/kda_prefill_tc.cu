@@ -354,10 +354,19 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     tc_fence_after();
 
     uint32_t tma_phase = 0, mma_phase = 0, gram_phase = 0;
-    bool aborted = false, tma_pending = nchunks > 0;
+    // Unwinding state (meaningful in thread 0, which issues every copy and MMA):
+    // tma_armed: the transaction count of phase tma_phase is armed and not yet consumed;
+    // tma_issued: which of the next tiles (1 g, 2 k, 4 v, 8 q) have been requested for it;
+    // mma_bar / mma_bar_phase: a commit that was waited for without success.
+    bool aborted = false, tma_armed = nchunks > 0;
+    uint32_t tma_issued = nchunks > 0 ? 15u : 0u;
+    long long tma_tok = t_begin;
+    uint64_t *mma_bar = nullptr;
+    uint32_t mma_bar_phase = 0;
     // wait for an MMA commit; every thread takes part
     auto wait_mma = [&]() -> bool {
         const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
+        if (!ok) { mma_bar = bar_mma; mma_bar_phase = mma_phase; }
         mma_phase ^= 1u;
         tc_fence_after();
         return __syncthreads_or(!ok) == 0;
@@ -389,7 +398,8 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         {
             const bool ok = mbar_wait_bounded(bar_tma, tma_phase, kWaitCycles);
             tma_phase ^= 1u;
-            tma_pending = false;
+            if (ok) tma_armed = false;
+            else tma_phase ^= 1u;  // still the phase to drain on the way out
             if (__syncthreads_or(!ok)) { aborted = true; break; }
         }
         if (tid < C) {
@@ -475,6 +485,9 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         if (more && tid == 0) {  // g tile consumed: start the next chunk's loads
             mbar_arrive_expect_tx(bar_tma, tma_bytes);
             issue_g(tokn);
+            tma_armed = true;
+            tma_tok = tokn;
+            tma_issued = 1u;
         }
 
         // ---- phase 1b: Gram operands, Gamma * q and Gamma * k; keep the factors for Kh
@@ -597,9 +610,13 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mma_chain<D / 16>(tmem + TM_GRAM + 32u * j, A, B, idG, false);
             mma_commit(bar_gram);
         }
-        if (more && tid == 0) issue_k(tokn);  // the k tile is consumed (Kh is written with the Gram operands)
+        if (more && tid == 0) {  // the k tile is consumed (Kh is written with the Gram operands)
+            issue_k(tokn);
+            tma_issued |= 2u;
+        }
         {
             const bool ok = mbar_wait_bounded(bar_gram, gram_phase, kWaitCycles);
+            if (!ok) { mma_bar = bar_gram; mma_bar_phase = gram_phase; }
             gram_phase ^= 1u;
             tc_fence_after();
             if (__syncthreads_or(!ok)) { aborted = true; break; }
@@ -720,8 +737,10 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mma_commit(bar_mma);
         }
         if (!wait_mma()) { aborted = true; break; }
-        if (more && tid == 0) issue_v(tokn);
-        tma_pending = more;
+        if (more && tid == 0) {
+            issue_v(tokn);
+            tma_issued |= 4u;
+        }
 
         // ---- phase 4: -W (rows 0..63) into the [-W ; Qt] operand
         if (quarter < 2) {
@@ -769,7 +788,10 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tc_fence_before();
         }
         if (!wait_mma()) { aborted = true; break; }
-        if (more && tid == 0) issue_q(tokn);  // rows 64..127 of the [-W ; Qt] operand are free
+        if (more && tid == 0) {  // rows 64..127 of the [-W ; Qt] operand are free
+            issue_q(tokn);
+            tma_issued |= 8u;
+        }
 
         // ---- phase 5: U (rows 0..63) -> bf16 B operand, MN-major [tok][dv]
         if (quarter < 2) {
@@ -869,8 +891,20 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (tid == 0) bulk_wait_all();  // the output stores are complete before the CTA exits
 
     if (aborted) {
-        if (tid == 0 && p.dev_status) atomicExch(p.dev_status, (int)KDA_ERR_TIMEOUT);
-        if (tma_pending && tid == 0) mbar_wait_bounded(bar_tma, tma_phase, kWaitCycles);
+        // Unwind without leaving work in flight: complete the armed transaction count by
+        // requesting the tiles not yet requested and wait (bounded) for the copies, then
+        // wait (bounded) for a commit that timed out, before TMEM is freed below.
+        if (tid == 0) {
+            if (p.dev_status) atomicExch(p.dev_status, (int)KDA_ERR_TIMEOUT);
+            if (tma_armed) {
+                if (!(tma_issued & 1u)) issue_g(tma_tok);
+                if (!(tma_issued & 2u)) issue_k(tma_tok);
+                if (!(tma_issued & 4u)) issue_v(tma_tok);
+                if (!(tma_issued & 8u)) issue_q(tma_tok);
+                mbar_wait_bounded(bar_tma, tma_phase, kWaitCycles);
+            }
+            if (mma_bar) mbar_wait_bounded(mma_bar, mma_bar_phase, kWaitCycles);
+        }
     } else if (p.ST) {
         tc_fence_after();
 #pragma unroll
