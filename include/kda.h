@@ -197,12 +197,16 @@ int kda_forward_host(const void *q, const void *k, const void *v, const void *g,
  * sequences returns KDA_ERR_SCRATCH_LIMIT and launches nothing; dense batches
  * have no limit. This entry point itself allocates nothing.
  *
- * The first call on each device looks up the array's device address (with
- * that device current) and caches it; make that first call before any stream
- * capture. Every call shares the one array per device and leaves its contents
- * behind (each call overwrites what it reads, so stale contents are harmless);
- * calls that overlap on the GPU race on it, so do not run two at once on one
- * device.
+ * The array belongs to the current device: make the device that owns the
+ * tensors current before the call, and pass a stream of that device. Each call
+ * made outside a stream capture looks up the array's device address (with that
+ * device current), so an address never outlives a context reset; a call made
+ * while the stream is being captured reuses the address from the last call on
+ * that device outside a capture, so make one call on each device before any
+ * stream capture. Every call shares the one array per device and leaves its
+ * contents behind (each call overwrites what it reads, so stale contents are
+ * harmless); calls that overlap on the GPU race on it, so do not run two at
+ * once on one device.
  */
 int kda_forward_noalloc(const void *q, const void *k, const void *v, const void *g,
                         const void *beta, const float *S0, void *o, float *S_T, int B, int T,

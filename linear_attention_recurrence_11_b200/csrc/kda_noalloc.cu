@@ -25,13 +25,18 @@ std::mutex g_scratch_mu;
 void *g_scratch_addr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device. In host code the
-// array's name only stands in for the symbol; the address has to be looked up
-// once per device, with that device current.
-int scratch_address(void **out) {
+// array's name only stands in for the symbol; the address is looked up with the
+// device current. It is looked up again on every call made outside a stream
+// capture, so a context torn down and rebuilt (after cudaDeviceReset) never
+// leaves a stale address behind; inside a capture the address from the last
+// uncaptured call on that device is used (the lookup is not made during capture).
+int scratch_address(cudaStream_t stream, void **out) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess) return KDA_ERR_CUDA;
     std::lock_guard<std::mutex> lock(g_scratch_mu);
-    if (g_scratch_addr[dev] == nullptr) {
+    if (cap == cudaStreamCaptureStatusNone || g_scratch_addr[dev] == nullptr) {
         void *p = nullptr;
         if (cudaGetSymbolAddress(&p, kda_noalloc_scratch) != cudaSuccess || p == nullptr) return KDA_ERR_CUDA;
         g_scratch_addr[dev] = p;
@@ -48,7 +53,7 @@ extern "C" int kda_forward_noalloc(const void *q, const void *k, const void *v, 
                                    int num_seqs, int *dev_status, void *stream) {
     if (cu_seqlens != nullptr && num_seqs > kda::kMaxOrderedSeqs) return KDA_ERR_SCRATCH_LIMIT;
     void *scratch = nullptr;
-    const int st = scratch_address(&scratch);
+    const int st = scratch_address(static_cast<cudaStream_t>(stream), &scratch);
     if (st != KDA_OK) return st;
     return kda_forward(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, dtype, cu_seqlens, num_seqs,
                        scratch, sizeof(kda_noalloc_scratch), dev_status, stream);

@@ -192,10 +192,11 @@ def kda_forward_noalloc(q, k, v, g, beta, S0, o, S_T, *, chunk: int = 64, cu_seq
     _need(o, "o", dtype, (B, T, H, dv), dev)
     if S_T is not None:
         _need(S_T, "S_T", torch.float32, (N, H, dv, dk), dev)
-    rc = _lib.kda_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
-                                  _ptr(S_T), B, T, H, dk, dv, int(chunk), DTYPES[dtype],
-                                  _ptr(cu_seqlens), N if cu_seqlens is not None else 0,
-                                  _ptr(dev_status), _stream_handle(stream, dev))
+    with torch.cuda.device(dev):  # the library's scratch array is the current device's
+        rc = _lib.kda_forward_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                      _ptr(S_T), B, T, H, dk, dv, int(chunk), DTYPES[dtype],
+                                      _ptr(cu_seqlens), N if cu_seqlens is not None else 0,
+                                      _ptr(dev_status), _stream_handle(stream, dev))
     if rc != KDA_OK:
         raise KdaError(rc, "kda_forward_noalloc")
     return o, S_T

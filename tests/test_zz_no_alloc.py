@@ -2,8 +2,9 @@
 memory (engines that pre-plan all device memory in their own pools, hosts that
 hand over raw device pointers without an allocator): called through the C ABI,
 it must give the same results as kda_forward with a caller-provided workspace,
-on two calls in a row (the second one finds the previous call's schedule in
-the shared scratch array), and refuse packed batches larger than that array.
+on two calls in a row with different batches (the second one finds the
+previous call's schedule in the shared scratch array), and refuse packed
+batches larger than that array.
 
 This file is named to be collected last, so a run that stops at its first
 failure has already run every other test."""
@@ -48,18 +49,27 @@ def _noalloc_c(K, inp, o, ST, chunk=64):
 
 @pytest.mark.parametrize("dtype,dk,chunk", [("bf16", 128, 64), ("f32", 64, 32)])
 def test_noalloc_matches_forward_two_calls(K, dtype, dk, chunk):
-    lens = [130, 0, 7, 64, 200, 1, 65, 0, 33, 300, 12, 90]
-    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
-    inp = case(1, int(cu[-1]), 3, dk, dk, dtype, seed=77, s0_std=0.1, num_states=len(lens))
-    inp["cu_seqlens"] = torch.tensor(cu, device="cuda")
-    o_ref, S_ref = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"],
-                                 chunk=chunk, cu_seqlens=inp["cu_seqlens"])
-    torch.cuda.synchronize()
-    for call in range(2):
+    """Two calls in a row with different packed batches: the second has more
+    sequences, in another length order, so its longest-first schedule differs
+    from the one the first call leaves in the shared array (every stale entry is
+    still a valid sequence index of the second batch, so a call that read the
+    array without writing it would run some sequences twice and others never,
+    and its NaN-filled outputs would show it). Each call is compared with
+    kda_forward (caller-provided workspace) on the same inputs."""
+    batches = [[7, 130, 0, 200, 1, 65, 33],
+               [300, 1, 90, 0, 12, 65, 200, 7, 0, 130, 33, 64]]
+    for call, lens in enumerate(batches):
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        inp = case(1, int(cu[-1]), 3, dk, dk, dtype, seed=77 + call, s0_std=0.1, num_states=len(lens))
+        inp["cu_seqlens"] = torch.tensor(cu, device="cuda")
+        o_ref, S_ref = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"],
+                                     chunk=chunk, cu_seqlens=inp["cu_seqlens"])
+        torch.cuda.synchronize()
         o = torch.full_like(o_ref, float("nan"))
         ST = torch.full_like(S_ref, float("nan"))
         rc, status = _noalloc_c(K, inp, o, ST, chunk)
         assert rc == 0 and status == 0, (call, rc, status)
+        assert torch.isfinite(o).all() and torch.isfinite(ST).all(), call
         assert rel(to_f64(o), to_f64(o_ref)) < TOL[dtype], call
         assert rel(to_f64(ST), to_f64(S_ref)) < TOL[dtype], call
 
