@@ -46,7 +46,7 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="prefill", choices=sorted(WORKLOAD_ALIASES))
-    p.add_argument("--path", default="auto", choices=["auto", "simt", "tc"])
+    p.add_argument("--path", default="auto", choices=["auto", "simt", "tc", "tc_single", "tc_split"])
     p.add_argument("--snap-every", type=int, default=1024,
                    help="prefill leg saving the state every N tokens (0: skip)")
     p.add_argument("--draft-tokens", type=int, default=4,
@@ -279,14 +279,19 @@ def run_ours(args, rank, world, device):
     tokens = w.total_tokens
     value = weak_scaling_value(tokens, K, ms_total, world)
     alg_bytes, alg_flops = prefill_algorithmic(w, elem)
-    kern_src = ("linear_attention_recurrence_11_b200/csrc/kda_prefill_tc.cu" if path_used == "tc"
-                else "linear_attention_recurrence_11_b200/csrc/kda_prefill_simt.cu")
+    if path_used == "tc":  # the split form runs when the workspace holds its records
+        split = seg == 0 and args.path in ("auto", "tc", "tc_split")
+        kern_src = ("linear_attention_recurrence_11_b200/csrc/kda_prefill_split.cu" if split
+                    else "linear_attention_recurrence_11_b200/csrc/kda_prefill_tc.cu")
+        path_used = "tc_split" if split else "tc_single"
+    else:
+        kern_src = "linear_attention_recurrence_11_b200/csrc/kda_prefill_simt.cu"
     achieved = alg_bytes / (kern_ms / 1e3) / 1e9
     traffic = traffic_for(kern_src, wname)
     res.update({
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16" if path_used == "tc" else ("f32" if elem == 4 else "bf16-storage/f32-compute"),
+        "vs_baseline": None, "dtype": "bf16" if path_used.startswith("tc") else ("f32" if elem == 4 else "bf16-storage/f32-compute"),
         "data": "synthetic (seeded: q,k unit-norm N(0,1); v N(0,1); beta sigmoid(N); g -5*sigmoid(N))",
         "config": {"workload": wname, "B": B, "T": T, "H": w.H, "dk": w.dk, "dv": w.dv,
                    "chunk": w.chunk, "num_seqs": N, "kernel_path": path_used,

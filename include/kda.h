@@ -73,10 +73,28 @@ typedef enum { KDA_DTYPE_F32 = 0, KDA_DTYPE_BF16 = 1 } kda_dtype;
  *   not print its formula; this is the plainest map onto that range. */
 typedef enum { KDA_FUSE_NORM_QK = 1, KDA_FUSE_GATE_LOGITS = 2 } kda_fuse;
 
-/* Which prefill kernel kda_forward_ex runs. AUTO picks the tensor-core kernel
- * where it is built (bf16, dk = dv = 128, chunk = 64) and the SIMT kernel
- * otherwise. */
-typedef enum { KDA_PATH_AUTO = 0, KDA_PATH_SIMT = 1, KDA_PATH_TC = 2 } kda_path;
+/* Which prefill kernels kda_forward_ex runs. The tensor cores cover bf16,
+ * dk = dv = 128, chunk = 64; the SIMT kernel covers every supported shape.
+ * On the tensor cores there are two forms of the same computation:
+ *  - split: a chunk-parallel kernel computes, for every (sequence, head,
+ *    chunk), the part of the chunk that does not depend on the incoming state
+ *    (decayed Grams, triangular solve, W, Ut; "Exercices", Q21: a chunk's KCP
+ *    pair depends on its own inputs only) into the workspace, then a second
+ *    kernel carries each unit's state across its chunks. Needs the workspace
+ *    kda_forward_workspace_size reports (about 72.5 KiB per chunk per head).
+ *  - single: one kernel per (sequence, head) computes everything chunk after
+ *    chunk; it needs no workspace beyond the packed-batch schedule.
+ * AUTO and TC run the split form when the workspace passed holds it and the
+ * single form otherwise (TC returns KDA_ERR_UNSUPPORTED off the tensor-core
+ * shapes, AUTO falls back to SIMT); TC_SINGLE and TC_SPLIT force one form
+ * (TC_SPLIT returns KDA_ERR_WORKSPACE if the workspace is too small). */
+typedef enum {
+    KDA_PATH_AUTO = 0,
+    KDA_PATH_SIMT = 1,
+    KDA_PATH_TC = 2,
+    KDA_PATH_TC_SINGLE = 3,
+    KDA_PATH_TC_SPLIT = 4
+} kda_path;
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char *kda_status_string(int status);
@@ -85,20 +103,26 @@ const char *kda_status_string(int status);
 int kda_abi_version(void);
 
 /*
- * Bytes of device workspace kda_forward needs for these sizes (0 if none).
- * num_seqs is the number of packed sequences when cu_seqlens is used, else B
- * (B == 1 with num_seqs > 1 means packed sequences). Packed batches of 2 to
- * 2048 sequences use a few bytes per sequence for a longest-first schedule
- * (a small kernel ranks the sequences by length so the longest start first);
- * nothing else needs workspace. The workspace is scratch: its contents on
- * entry do not matter and it may be reused after the stream reaches the end
- * of the call. Returns (size_t)-1 if the sizes are invalid.
+ * Bytes of device workspace kda_forward needs for these sizes (0 if none):
+ * the scratch of the chunked prefill of "Exercices", Q7 with the KCP
+ * composition of Q21-Q22. num_seqs is the number of packed sequences when
+ * cu_seqlens is used, else B (B == 1 with num_seqs > 1 means packed
+ * sequences). On the tensor-core shapes it is the split form's per-chunk
+ * records (74,240 bytes per chunk per head; for packed batches counted for
+ * at most T / 64 + num_seqs chunks per head) plus, for packed batches, the
+ * sequences' chunk offsets and a longest-first schedule of up to 2048
+ * sequences. A smaller workspace still works on the tensor cores (the single
+ * form, see kda_path). The workspace is scratch: its contents on entry do not
+ * matter and it may be reused after the stream reaches the end of the call.
+ * Returns (size_t)-1 if the sizes are invalid.
  */
 size_t kda_forward_workspace_size(int B, int T, int H, int dk, int dv, int chunk,
                                   int num_seqs, int dtype);
 
 /*
- * Chunked prefill with KCP inter-chunk state composition.
+ * Chunked prefill with KCP inter-chunk state composition: the recurrence of
+ * "Exercices", Q7 evaluated chunk by chunk, the state carried across chunks
+ * by the pair composition of Q21-Q22.
  *
  *   q, k, g, v, beta : inputs (layouts above).
  *   S0   : [N, H, dv, dk] fp32 initial states, or NULL for zeros.
@@ -140,7 +164,8 @@ int kda_forward_fused(const void *q, const void *k, const void *v, const void *g
                       size_t workspace_bytes, int *dev_status, void *stream, int path, int flags);
 
 /* Number of kernel launches one kda_forward_ex call with these arguments
- * enqueues (0 when T = 0 and no state is copied), or -1 if invalid. */
+ * enqueues (0 when T = 0 and no state is copied), or -1 if invalid. For AUTO
+ * and TC it assumes the workspace kda_forward_workspace_size reports. */
 int kda_forward_launches(int B, int T, int H, int dk, int dv, int chunk, int dtype,
                          int has_cu_seqlens, int num_seqs, int path);
 
@@ -164,7 +189,8 @@ int kda_forward_launches(int B, int T, int H, int dk, int dv, int chunk, int dty
  *          about T / 8 rounded up to whole chunks.
  *   workspace / workspace_bytes : DEVICE memory, 256-byte aligned, of at least
  *          kda_forward_host_workspace_size(...) bytes: two slots for one
- *          piece's inputs and outputs, and the state.
+ *          piece's inputs and outputs, the state, and the device prefill's
+ *          workspace for one piece (kda_forward_workspace_size of a piece).
  *   dev_status, path : as for kda_forward_ex. stream : the caller's stream;
  *          the launches run on it, and it is made to wait for the last
  *          download, so the host outputs are complete once the stream is.

@@ -17,8 +17,8 @@ int check_prefill_sizes(int B, int T, int H, int dk, int dv, int chunk, int dtyp
     if (!dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;
     if (!head_dim_ok(dk) || !head_dim_ok(dv) || !chunk_ok(chunk)) return KDA_ERR_UNSUPPORTED;
     if (has_cu && (B != 1 || num_seqs <= 0)) return KDA_ERR_INVALID_ARG;
-    if (path != KDA_PATH_AUTO && path != KDA_PATH_SIMT && path != KDA_PATH_TC) return KDA_ERR_INVALID_ARG;
-    if (path == KDA_PATH_TC && !kda::prefill_tc_supported(dk, dv, chunk, dtype)) return KDA_ERR_UNSUPPORTED;
+    if (path < KDA_PATH_AUTO || path > KDA_PATH_TC_SPLIT) return KDA_ERR_INVALID_ARG;
+    if (path >= KDA_PATH_TC && !kda::prefill_tc_supported(dk, dv, chunk, dtype)) return KDA_ERR_UNSUPPORTED;
     // the kernels index tokens with size_t and units with 32-bit grid indices
     const size_t units = (size_t)(has_cu ? num_seqs : B) * (size_t)H;
     if (units * (size_t)(dv / 32) > 0x7fffffffu) return KDA_ERR_UNSUPPORTED;
@@ -34,6 +34,33 @@ const int32_t kPackedMarker = 0;
 bool use_tc(const kda::PrefillArgs &a, int path) {
     if (path == KDA_PATH_SIMT) return false;
     return kda::prefill_tc_supported(a.dk, a.dv, a.chunk, a.dtype);
+}
+
+// The prefill form a call runs (kda_path): the SIMT kernel, the single tensor-core kernel, or
+// the split tensor-core form, which AUTO and TC take when the workspace holds its records.
+enum class Form { Simt, Single, Split };
+Form choose_form(const kda::PrefillArgs &a, int path, size_t workspace_bytes, bool workspace_known) {
+    if (!use_tc(a, path)) return Form::Simt;
+    if (path == KDA_PATH_TC_SINGLE) return Form::Single;
+    if (path == KDA_PATH_TC_SPLIT) return Form::Split;
+    if (!workspace_known) return Form::Split;  // size queries assume the reported workspace
+    return workspace_bytes >= kda::prefill_split_workspace(a) ? Form::Split : Form::Single;
+}
+
+size_t form_workspace(const kda::PrefillArgs &a, Form f) {
+    switch (f) {
+        case Form::Simt: return kda::prefill_simt_workspace(a);
+        case Form::Single: return kda::prefill_tc_workspace(a);
+        default: return kda::prefill_split_workspace(a);
+    }
+}
+
+cudaError_t form_launch(const kda::PrefillArgs &a, Form f) {
+    switch (f) {
+        case Form::Simt: return kda::launch_prefill_simt(a);
+        case Form::Single: return kda::launch_prefill_tc(a);
+        default: return kda::launch_prefill_split(a);
+    }
 }
 
 }  // namespace
@@ -74,7 +101,9 @@ size_t kda_forward_workspace_size(int B, int T, int H, int dk, int dv, int chunk
     size_t ws = kda::prefill_simt_workspace(a);
     if (kda::prefill_tc_supported(dk, dv, chunk, dtype)) {
         const size_t t = kda::prefill_tc_workspace(a);
+        const size_t sp = kda::prefill_split_workspace(a);
         ws = t > ws ? t : ws;
+        ws = sp > ws ? sp : ws;
     }
     return ws;
 }
@@ -85,7 +114,11 @@ int kda_forward_launches(int B, int T, int H, int dk, int dv, int chunk, int dty
     if (check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, has_cu_seqlens != 0, num_seqs, path, &a))
         return -1;
     a.cu_seqlens = has_cu_seqlens ? &kPackedMarker : nullptr;
-    return use_tc(a, path) ? kda::prefill_tc_launches(a) : kda::prefill_simt_launches(a);
+    switch (choose_form(a, path, 0, false)) {
+        case Form::Simt: return kda::prefill_simt_launches(a);
+        case Form::Single: return kda::prefill_tc_launches(a);
+        default: return kda::prefill_split_launches(a);
+    }
 }
 
 int kda_forward_ex(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -104,10 +137,10 @@ int kda_forward_ex(const void *q, const void *k, const void *v, const void *g, c
     a.S0 = S0; a.o = o; a.ST = S_T; a.cu_seqlens = cu_seqlens;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.dev_status = dev_status;
     a.stream = static_cast<cudaStream_t>(stream);
-    const bool tc = use_tc(a, path);
-    const size_t need = tc ? kda::prefill_tc_workspace(a) : kda::prefill_simt_workspace(a);
+    const Form f = choose_form(a, path, workspace == nullptr ? 0 : workspace_bytes, true);
+    const size_t need = form_workspace(a, f);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
-    const cudaError_t e = tc ? kda::launch_prefill_tc(a) : kda::launch_prefill_simt(a);
+    const cudaError_t e = form_launch(a, f);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
 }
 
@@ -129,6 +162,7 @@ int kda_forward_snapshots(const void *q, const void *k, const void *v, const voi
     a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.dev_status = dev_status;
     a.stream = static_cast<cudaStream_t>(stream);
     a.S_snap = S_snap; a.snap_every = T / snap_every > 0 ? snap_every : 0;
+    if (path == KDA_PATH_TC_SPLIT) return KDA_ERR_UNSUPPORTED;  // snapshots come from the single form
     const bool tc = use_tc(a, path);
     const cudaError_t e = tc ? kda::launch_prefill_tc(a) : kda::launch_prefill_simt(a);
     return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
@@ -151,6 +185,10 @@ int kda_forward_fused(const void *q, const void *k, const void *v, const void *g
     a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.dev_status = dev_status;
     a.stream = static_cast<cudaStream_t>(stream);
     a.fuse = flags;
+    if (flags && path == KDA_PATH_TC_SPLIT) return KDA_ERR_UNSUPPORTED;  // fused pre-operations: single form
+    if (!flags)
+        return kda_forward_ex(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, dtype, cu_seqlens, num_seqs,
+                              workspace, workspace_bytes, dev_status, stream, path);
     const bool tc = use_tc(a, path);
     const size_t need = tc ? kda::prefill_tc_workspace(a) : kda::prefill_simt_workspace(a);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
@@ -178,7 +216,7 @@ int check_segmented(int B, int T, int H, int dk, int dv, int chunk, int dtype, i
     if (P > 1) {  // the segments run as packed sequences of one flat token axis
         if ((long long)B * T > 0x7fffffffLL || (long long)B * P > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
         if ((size_t)(B * P) * (size_t)H * (size_t)(dv > dk ? dv : dk) / 32 > 0x7fffffffu) return KDA_ERR_UNSUPPORTED;
-        if (path == KDA_PATH_TC && !kda::prefill_tc_supported(dk, dk, chunk, dtype)) return KDA_ERR_UNSUPPORTED;
+        if (path >= KDA_PATH_TC && !kda::prefill_tc_supported(dk, dk, chunk, dtype)) return KDA_ERR_UNSUPPORTED;
     }
     *s = kda::SegmentedArgs{};
     s->B = B; s->T = T; s->H = H; s->dk = dk; s->dv = dv; s->chunk = chunk; s->dtype = dtype;
@@ -261,7 +299,7 @@ int kda_segment_pair(const void *q, const void *k, const void *v, const void *g,
     kda::PrefillArgs a{};
     int st = check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, false, 0, path, &a);
     if (st) return st;
-    if (path == KDA_PATH_TC && !kda::prefill_tc_supported(dk, dk, chunk, dtype)) return KDA_ERR_UNSUPPORTED;
+    if (path >= KDA_PATH_TC && !kda::prefill_tc_supported(dk, dk, chunk, dtype)) return KDA_ERR_UNSUPPORTED;
     if (!M || !Z || (T > 0 && (!q || !k || !v || !g || !beta))) return KDA_ERR_INVALID_ARG;
     for (const void *p : {q, k, v, g, beta, (const void *)M, (const void *)Z, (const void *)dev_status})
         if (!aligned16(p)) return KDA_ERR_ALIGNMENT;

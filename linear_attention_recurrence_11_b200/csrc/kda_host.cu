@@ -56,10 +56,11 @@ struct HostLayout {
     size_t q, k, v, g, beta, o;  // bytes of one piece of each tensor
     size_t slot;                 // one slot: the six tensors, 256-byte aligned each
     size_t state;                // [B, H, dv, dk] fp32
+    size_t scratch;              // the device prefill's workspace for one piece (pieces run in turn)
     size_t total;
 };
 
-HostLayout host_layout(int B, int Lp, int H, int dk, int dv, int dtype) {
+HostLayout host_layout(int B, int Lp, int H, int dk, int dv, int chunk, int dtype) {
     const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
     const size_t tok = (size_t)B * (size_t)Lp * (size_t)H;
     HostLayout L{};
@@ -68,7 +69,9 @@ HostLayout host_layout(int B, int Lp, int H, int dk, int dv, int dtype) {
     L.beta = tok * es;
     L.slot = round_up(L.q) + round_up(L.k) + round_up(L.v) + round_up(L.g) + round_up(L.beta) + round_up(L.o);
     L.state = round_up((size_t)B * H * dv * dk * sizeof(float));
-    L.total = 2 * L.slot + L.state;
+    const size_t ws = Lp > 0 ? kda_forward_workspace_size(B, Lp, H, dk, dv, chunk, B, dtype) : 0;
+    L.scratch = ws == (size_t)-1 ? 0 : round_up(ws);
+    L.total = 2 * L.slot + L.state + L.scratch;
     return L;
 }
 
@@ -101,7 +104,7 @@ size_t kda_forward_host_workspace_size(int B, int T, int H, int dk, int dv, int 
     if (piece_len < 0 || (piece_len > 0 && piece_len % chunk != 0)) return (size_t)-1;
     const int Lp0 = piece_len > 0 ? piece_len : default_piece(T, chunk);
     const int Lp = T < Lp0 ? T : Lp0;
-    return host_layout(B, Lp, H, dk, dv, dtype).total;
+    return host_layout(B, Lp, H, dk, dv, chunk, dtype).total;
 }
 
 int kda_forward_host(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -114,7 +117,7 @@ int kda_forward_host(const void *q, const void *k, const void *v, const void *g,
     if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
     const int Lp0 = piece_len > 0 ? piece_len : default_piece(T, chunk);
     const int Lp = T < Lp0 ? T : Lp0;
-    const HostLayout L = host_layout(B, Lp, H, dk, dv, dtype);
+    const HostLayout L = host_layout(B, Lp, H, dk, dv, chunk, dtype);
     if (!workspace || workspace_bytes < L.total) return KDA_ERR_WORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_ALIGNMENT;
 
@@ -139,6 +142,7 @@ int kda_forward_host(const void *q, const void *k, const void *v, const void *g,
         slot[s].o = b;
     }
     float *state = reinterpret_cast<float *>(ws + 2 * L.slot);
+    void *scratch = L.scratch ? ws + 2 * L.slot + L.state : nullptr;
     const size_t state_bytes = (size_t)B * H * dv * dk * sizeof(float);
 
 #define KDA_TRY(x)                                   \
@@ -171,7 +175,7 @@ int kda_forward_host(const void *q, const void *k, const void *v, const void *g,
         if (p >= 2) KDA_TRY(cudaStreamWaitEvent(cs, hp.ev_down[s], 0));
         st = kda_forward_ex(slot[s].q, slot[s].k, slot[s].v, slot[s].g, slot[s].beta,
                             (p == 0 && !S0) ? nullptr : state, slot[s].o, state, B, n, H, dk, dv, chunk, dtype,
-                            nullptr, 0, nullptr, 0, dev_status, cs, path);
+                            nullptr, 0, scratch, L.scratch, dev_status, cs, path);
         if (st) return st;
         KDA_TRY(cudaEventRecord(hp.ev_comp[s], cs));
         // its outputs back to the host

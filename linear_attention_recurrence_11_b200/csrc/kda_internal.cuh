@@ -108,6 +108,10 @@ cudaError_t launch_kcp_scan(const SegmentedArgs &s, const float *Mbuf, const flo
 cudaError_t launch_prefill_tc(const PrefillArgs &a);
 size_t prefill_tc_workspace(const PrefillArgs &a);
 int prefill_tc_launches(const PrefillArgs &a);
+// the split tensor-core form: chunk-parallel records in the workspace, then the state chains
+cudaError_t launch_prefill_split(const PrefillArgs &a);
+size_t prefill_split_workspace(const PrefillArgs &a);
+int prefill_split_launches(const PrefillArgs &a);
 
 cudaError_t launch_decode(const DecodeArgs &a);
 cudaError_t launch_decode_multi(const MultiDecodeArgs &a);

@@ -1,0 +1,1007 @@
+// Split tensor-core prefill (sm_100a): bf16 q/k/v/g/beta, fp32 state,
+// dk = dv = 128, chunks of C = 64 tokens, in two kernels.
+//
+// Only a small part of a chunk's work depends on the state S it receives: the
+// KCP pair of the chunk ("Exercices", Q21-Q22) is (Diag(Gamma_C) - Kh^T W, Kh^T Ut),
+// and everything in it (the decayed Grams, the triangular solve, W, Ut, Kh) is a
+// function of the chunk's own q, k, v, g, beta. So:
+//
+//  1. kda_prep_kernel runs every (sequence, head, chunk) task independently,
+//     persistent CTAs striding over the tasks (two CTAs per SM): the cumulative
+//     log-decay inside 16-token subtiles ("Exercices", Q8), the Gram operands
+//     referenced to the middle of each 32-token column block, the Gram products
+//     A and P on tcgen05, T = (I + A)^{-1} (diagonal 16 x 16 blocks by forward
+//     substitution, merges with warp-level TF32 MMAs), and [W | Ut] =
+//     T Diag(beta) [Gamma k | v] on tcgen05. It writes one record per task to the
+//     workspace: [-W ; Gamma q] (the A operand of the state product), Kh, Ut, P
+//     and Gamma_C, each as the image of the shared-memory tile the second kernel
+//     feeds to its tensor cores.
+//  2. kda_chain_kernel walks each (sequence, head) unit's chunks in order with
+//     the fp32 state resident in TMEM (the KCP left fold): per chunk one bulk
+//     copy brings the record (double-buffered, a chunk ahead), then
+//        [U ; Gamma Q S] = [-W ; Gamma Q] S        (the record's Ut added at readout)
+//        O = Gamma Q S + P U,   S <- Diag(Gamma_C) S + Kh^T U
+//     with the U / O accumulator alternating between two TMEM regions so that the
+//     next chunk's state product runs while this chunk's outputs are read out.
+//
+// The state-independent work, most of a chunk's cycles, is thereby spread over
+// all SMs instead of sitting on each unit's serial chain. No cluster multicast
+// is used; every copy is a plain TMA tile load, a bulk copy or a tensor store.
+#include "kda_internal.cuh"
+#include "kda_sm100.cuh"
+#include "kda_tc_common.cuh"
+
+namespace kda {
+namespace {
+
+using namespace sm100;
+using namespace tc;
+
+constexpr int NT = 256;
+constexpr uint32_t KB = 1024;
+
+// ------------------------------------------------ per-task record in the workspace
+constexpr uint32_t REC_WQ = 0;         // 32 KB [-W ; Gamma q], K-major, 128 rows x 128, K-blocks 16 KB apart
+constexpr uint32_t REC_KH = 32 * KB;   // 16 KB Kh = e^{G_C - G} k, MN-major [tok][dk], 64-channel blocks 8 KB apart
+constexpr uint32_t REC_UT = 48 * KB;   // 16 KB Ut (bf16), MN-major [tok][dv], N-blocks 8 KB apart
+constexpr uint32_t REC_P = 64 * KB;    // 8 KB  P (bf16, s <= r), K-major [r][s]
+constexpr uint32_t REC_GC = 72 * KB;   // 512 B Gamma_C (fp32, one per channel)
+constexpr uint32_t REC_BYTES = 72 * KB + 512;
+static_assert(REC_BYTES % 128 == 0, "records keep 128-byte alignment");
+
+// ------------------------------------------------------------ prep smem layout
+constexpr uint32_t P_L0 = 0;          // 32 KB k (rows 0..63) and q (rows 64..127) tiles, the Gram left operand L0 in place
+constexpr uint32_t P_L1 = 32 * KB;    // 16 KB Gram left operand L1 ([k ; q] rows 32..63, K-blocks 8 KB apart)
+constexpr uint32_t P_R = 48 * KB;     // 16 KB Gram right operand, K-major [s][dk]
+constexpr uint32_t P_GK = 64 * KB;    // 16 KB Gamma k, B operand MN-major [tok][dk]
+constexpr uint32_t P_GV = 80 * KB;    // 16 KB g (plain [64][128] bf16), then v (B operand MN-major [tok][dv])
+constexpr uint32_t P_MISC = 96 * KB;
+// aliases once the Gram products are done (L0, L1, R free)
+constexpr uint32_t P_TB = 0;                          // 8 KB A operand T Diag(beta) rows 0..63 (the MMA reads 16 KB)
+constexpr uint32_t P_AF = 8 * KB;                     // 64 x LDA fp32 A
+constexpr uint32_t P_TF = P_AF + 64 * LDA * 4;        // 64 x LDT fp32 T
+constexpr uint32_t P_XS = P_TF + 64 * LDT * 4;        // 32 x LDX fp32 scratch
+constexpr uint32_t P_PST = 48 * KB;                   // 8 KB P staging (record image)
+// once the W / Ut product is done (T Diag(beta), Gamma k, v free)
+constexpr uint32_t P_WST = 32 * KB;                   // 16 KB -W staging: the record's two K-blocks, rows 0..63
+constexpr uint32_t P_UST = 56 * KB;                   // 16 KB Ut staging (record image)
+static_assert(P_XS + 32 * LDX * 4 <= P_PST, "inverse scratch reaches the P staging");
+static_assert(P_WST + 16 * KB <= P_PST && P_PST + 8 * KB <= P_UST, "staging tiles overlap");
+static_assert(P_L1 + 8 * KB + 16 * KB <= P_GK, "L1 read as a 128-row operand reaches Gamma k");
+constexpr uint32_t P_BAR = P_MISC;                    // 4 mbarriers
+constexpr uint32_t P_TMEMADDR = P_MISC + 64;
+constexpr uint32_t P_BETA = P_MISC + 128;             // 64 fp32
+constexpr uint32_t P_DSUM = P_BETA + 256;             // 4 x 128 fp32 subtile totals of g (log2 units)
+constexpr uint32_t P_SMEM_USED = P_DSUM + 2048;
+constexpr uint32_t P_SMEM_BYTES = P_SMEM_USED + 1024;  // slack for 1024-byte alignment
+static_assert(2 * (P_SMEM_BYTES + 1024) <= 233472, "two prep CTAs per SM");
+constexpr uint32_t P_TM_W = 0, P_TM_UT = 128, P_TM_COLS = 256;  // the Gram uses columns 0..63 first
+
+// ----------------------------------------------------------- chain smem layout
+constexpr uint32_t C_RECSTRIDE = 73 * KB;             // >= REC_BYTES, 1 KB aligned
+constexpr uint32_t C_SB = 2 * C_RECSTRIDE;            // 32 KB S (bf16), B operand MN-major [dk][dv], N-blocks 16 KB apart
+constexpr uint32_t C_MISC = C_SB + 32 * KB;
+constexpr uint32_t C_BAR = C_MISC;                    // 3 mbarriers
+constexpr uint32_t C_TMEMADDR = C_MISC + 64;
+constexpr uint32_t C_SMEM_BYTES = C_MISC + 128 + 1024;
+static_assert(REC_BYTES <= C_RECSTRIDE && C_SMEM_BYTES <= 232448, "chain shared memory budget");
+constexpr uint32_t C_TM_U0 = 0, C_TM_U1 = 128, C_TM_S = 256, C_TM_COLS = 512;
+
+struct SplitParams {
+    PrefillArgs a;
+    uint8_t *rec;               // records, REC_BYTES each, task t at rec + t * REC_BYTES
+    const int32_t *chunk_base;  // packed batches: [num_units + 1] first task chunk of each sequence
+    int nch;                    // dense batches: chunks per sequence
+    long long tasks;            // dense batches: number of tasks (units x chunks)
+};
+
+// Task t = (global chunk index) * H + head. The global chunk index runs over the
+// chunks of sequence 0, then sequence 1, ...; heads vary fastest, so CTAs that
+// run neighbouring tasks read neighbouring rows of the [tokens, H, d] inputs.
+struct Task {
+    long long t, tok0;
+    int n, h, Lc;
+};
+
+__device__ __forceinline__ Task task_at(const SplitParams &sp, long long t) {
+    const PrefillArgs &p = sp.a;
+    Task k;
+    k.t = t;
+    k.h = (int)(t % p.H);
+    const long long gc = t / p.H;
+    long long c, end;
+    if (sp.chunk_base) {  // largest n with chunk_base[n] <= gc (empty sequences share a base)
+        int lo = 0, hi = p.num_units;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (sp.chunk_base[mid] <= gc) lo = mid; else hi = mid;
+        }
+        k.n = lo;
+        c = gc - sp.chunk_base[lo];
+        k.tok0 = (long long)p.cu_seqlens[lo] + c * C;
+        end = p.cu_seqlens[lo + 1];
+    } else {
+        k.n = (int)(gc / sp.nch);
+        c = gc % sp.nch;
+        k.tok0 = (long long)k.n * p.T + c * C;
+        end = (long long)k.n * p.T + p.T;
+    }
+    k.Lc = (int)((end - k.tok0) < C ? (end - k.tok0) : C);
+    return k;
+}
+
+// First task chunk of every packed sequence: base[n] = sum over m < n of ceil(len_m / C),
+// base[num] = the total. One block, tiles of blockDim.x sequences with a running carry.
+__global__ void chunk_base_kernel(const int32_t *cu, int num, int32_t *base) {
+    __shared__ int32_t warp_sums[32];
+    __shared__ int32_t carry_s;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
+    if (tid == 0) carry_s = 0;
+    __syncthreads();
+    for (int start = 0; start < num; start += blockDim.x) {
+        const int i = start + tid;
+        int v = 0;
+        if (i < num) {
+            const int len = cu[i + 1] - cu[i];
+            v = len > 0 ? (len + C - 1) / C : 0;
+        }
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_sums[wid] = x;
+        __syncthreads();
+        if (wid == 0) {
+            int w = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            warp_sums[lane] = w;
+        }
+        __syncthreads();
+        const int carry = carry_s;
+        const int incl = carry + (wid ? warp_sums[wid - 1] : 0) + x;
+        if (i < num) base[i] = incl - v;
+        __syncthreads();
+        if (tid == blockDim.x - 1) carry_s = incl;
+        __syncthreads();
+    }
+    if (tid == 0) base[num] = carry_s;
+}
+
+// ======================================================================= prep
+__global__ void __launch_bounds__(NT, 2)
+kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                const SplitParams sp) {
+    const PrefillArgs &p = sp.a;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + P_BAR);  // k, q, g of a task
+    uint64_t *bar_v = bar_ld + 1;
+    uint64_t *bar_gram = bar_ld + 2;                               // 2 arrivals
+    uint64_t *bar_mma = bar_ld + 3;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + P_TMEMADDR);
+    float *sBeta = reinterpret_cast<float *>(sm + P_BETA);
+    float *sD = reinterpret_cast<float *>(sm + P_DSUM);
+    float *AF = reinterpret_cast<float *>(sm + P_AF);
+    float *TF = reinterpret_cast<float *>(sm + P_TF);
+    float *XS = reinterpret_cast<float *>(sm + P_XS);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const size_t H = (size_t)p.H;
+    const __nv_bfloat16 *beta = static_cast<const __nv_bfloat16 *>(p.beta);
+    const long long total = sp.chunk_base ? (long long)sp.chunk_base[p.num_units] * p.H : sp.tasks;
+
+    if (tid == 0) {
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_v, 1);
+        mbar_init(bar_gram, 2);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_v);
+        tma_prefetch_desc(&tm_g);
+    }
+    if (warp == 0) {
+        tmem_alloc(s_tmem, P_TM_COLS);
+        tmem_relinquish();
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t tlane = (uint32_t)(32 * quarter) << 16;
+
+    auto issue_kqg = [&](const Task &k) {
+        tma_load_3d(sm + P_L0, &tm_k, bar_ld, 0, k.h, (int)k.tok0);
+        tma_load_3d(sm + P_L0 + 16 * KB, &tm_k, bar_ld, 64, k.h, (int)k.tok0);
+        tma_load_3d(sm + P_L0 + 8 * KB, &tm_q, bar_ld, 0, k.h, (int)k.tok0);
+        tma_load_3d(sm + P_L0 + 24 * KB, &tm_q, bar_ld, 64, k.h, (int)k.tok0);
+        tma_load_3d(sm + P_GV, &tm_g, bar_ld, 0, k.h, (int)k.tok0);
+    };
+    auto issue_v = [&](const Task &k) {
+        tma_load_3d(sm + P_GV, &tm_v, bar_v, 0, k.h, (int)k.tok0);
+        tma_load_3d(sm + P_GV + 8 * KB, &tm_v, bar_v, 64, k.h, (int)k.tok0);
+    };
+    const bool has_v = p.v != nullptr;  // all-zero values (a segment's transition): no v, Ut = 0
+
+    long long t = blockIdx.x;
+    bool have = t < total;
+    Task cur{};
+    if (have) cur = task_at(sp, t);
+    // unwinding state (thread 0): armed transaction counts and a commit whose wait ran out
+    bool ld_armed = false, v_armed = false;
+    uint64_t *mma_bar = nullptr;
+    uint32_t mma_bar_phase = 0;
+    uint32_t ld_phase = 0, v_phase = 0, gram_phase = 0, mma_phase = 0;
+    bool aborted = false;
+    if (have && tid == 0) {
+        mbar_arrive_expect_tx(bar_ld, 48 * KB);
+        issue_kqg(cur);
+        ld_armed = true;
+    }
+    __nv_bfloat16 bcur = __float2bfloat16(0.f);
+    if (have && tid < C && tid < cur.Lc) bcur = beta[(size_t)(cur.tok0 + tid) * H + cur.h];
+
+    // thread roles of the token-parallel passes (as in the single-kernel prefill): subtile ti,
+    // half hh of it (8 rows), a quad of channels c0..c0+3
+    const int ti = warp >> 1;
+    const int hh = lane >> 4;
+    const int cq = (warp & 1) * 16 + (lane & 15);
+    const int c0 = 4 * cq;
+    const int cblk = c0 >> 6;
+    const int cin = c0 & 63;
+    constexpr int HR = SUB / 2;
+    constexpr uint32_t idG = idesc_bf16_f32(128, 32, 0, 0);
+    constexpr uint32_t idKM = idesc_bf16_f32(128, 128, 0, 1);
+
+    while (have) {
+        const long long tn = t + gridDim.x;
+        const bool more = tn < total;
+        Task nxt{};
+        if (more) nxt = task_at(sp, tn);
+        uint8_t *rec = sp.rec + (size_t)cur.t * REC_BYTES;
+        const int Lc = cur.Lc;
+
+        // ---- this task's k, q, g
+        {
+            const bool ok = mbar_wait_bounded(bar_ld, ld_phase, kWaitCycles);
+            if (ok) { ld_phase ^= 1u; ld_armed = false; }
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+        }
+        __nv_bfloat16 bnext = __float2bfloat16(0.f);
+        if (tid < C) {
+            sBeta[tid] = (tid < Lc) ? __bfloat162float(bcur) : 0.f;
+            if (more && tid < nxt.Lc) bnext = beta[(size_t)(nxt.tok0 + tid) * H + nxt.h];
+        }
+        if (Lc < C) {  // zero the k and q rows past the end of the sequence
+            for (int idx = tid; idx < (C - Lc) * 16; idx += NT) {
+                const int r = Lc + idx / 16, q16 = idx % 16;
+                const int blk = q16 >> 3, pc = (q16 & 7) * 8;
+                const uint4 z = make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4 *>(sm + P_L0 + blk * 16 * KB + sw128_offset(r, pc)) = z;
+                *reinterpret_cast<uint4 *>(sm + P_L0 + blk * 16 * KB + sw128_offset(64 + r, pc)) = z;
+            }
+        }
+
+        // ---- cumulative log2-decay inside subtile ti for channels c0..c0+3
+        float gl[HR][4];
+        {
+            float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int rr = 0; rr < HR; ++rr) {
+                const int row = SUB * ti + HR * hh + rr;  // rows past the end decay by 1
+                const uint2 raw = row < Lc ? *reinterpret_cast<const uint2 *>(sm + P_GV + row * 256 + c0 * 2)
+                                           : make_uint2(0, 0);
+                const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+                const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+                a[0] = fmaf(g01.x, kLog2e, a[0]);
+                a[1] = fmaf(g01.y, kLog2e, a[1]);
+                a[2] = fmaf(g23.x, kLog2e, a[2]);
+                a[3] = fmaf(g23.y, kLog2e, a[3]);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) gl[rr][e] = a[e];
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float lo = __shfl_sync(0xffffffffu, a[e], lane & 15);
+                if (hh) {
+#pragma unroll
+                    for (int rr = 0; rr < HR; ++rr) gl[rr][e] += lo;
+                }
+            }
+            if (hh) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sD[ti * D + c0 + e] = gl[HR - 1][e];
+            }
+        }
+        if (tid == 0) bulk_wait_read_all();  // the previous task's record stores have read their staging
+        __syncthreads();
+        if (tid == 0 && has_v) {  // g consumed: v lands in its tile
+            mbar_arrive_expect_tx(bar_v, 16 * KB);
+            issue_v(cur);
+            v_armed = true;
+        }
+
+        // ---- Gram operands (L0 in place, L1, R), Gamma k; Gamma q, Kh and Gamma_C to the record
+        {
+            float Dm[NSUB][4], ed[NSUB][4];
+#pragma unroll
+            for (int m = 0; m < NSUB; ++m) {
+                const float4 d4 = *reinterpret_cast<const float4 *>(sD + m * D + c0);
+                Dm[m][0] = d4.x; Dm[m][1] = d4.y; Dm[m][2] = d4.z; Dm[m][3] = d4.w;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ed[m][e] = ex2(Dm[m][e]);
+            }
+            float pg[4], post[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float a = 1.f, b = 1.f;
+#pragma unroll
+                for (int m = 0; m < NSUB; ++m) {
+                    if (m < ti) a *= ed[m][e];
+                    if (m >= ti) b *= ed[m][e];
+                }
+                pg[e] = a;    // Gamma at the start of subtile ti
+                post[e] = b;  // decay from the start of subtile ti to the end of the chunk
+            }
+            if (ti == 0 && hh == 0) {
+                *reinterpret_cast<float4 *>(rec + REC_GC + 4 * c0) =
+                    make_float4(ed[0][0] * ed[1][0] * ed[2][0] * ed[3][0], ed[0][1] * ed[1][1] * ed[2][1] * ed[3][1],
+                                ed[0][2] * ed[1][2] * ed[2][2] * ed[3][2], ed[0][3] * ed[1][3] * ed[2][3] * ed[3][3]);
+            }
+            // column block b (tokens 32b..32b+31) referenced to its middle token 32b + 16:
+            //   el0 = e^{G_start(ti) - G_16}, el1 = e^{G_start(ti) - G_48} (ti >= 2),
+            //   er  = e^{G_mid(block of ti) - G_start(ti)}
+            float el0[4], el1[4], er[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                el0[e] = ti == 0 ? ex2(-Dm[0][e]) : ti == 1 ? 1.f : ti == 2 ? ed[1][e] : ed[1][e] * ed[2][e];
+                el1[e] = ti == 2 ? ex2(-Dm[2][e]) : 1.f;
+                er[e] = ti == 0 ? ed[0][e] : ti == 2 ? ed[2][e] : 1.f;
+            }
+            uint8_t *const l0 = sm + P_L0 + cblk * 16 * KB;
+            uint8_t *const l1 = sm + P_L1 + cblk * 8 * KB;
+            uint8_t *const rrow = sm + P_R + cblk * 8 * KB;
+            uint8_t *const gkrow = sm + P_GK + cblk * 8 * KB;
+            uint8_t *const gq_rec = rec + REC_WQ + cblk * 16 * KB + 8 * KB;
+            uint8_t *const kh_rec = rec + REC_KH + cblk * 8 * KB;
+            auto pk4 = [](float a, float b, float c, float d) { return make_uint2(pack_bf2(a, b), pack_bf2(c, d)); };
+            auto ld4 = [](const uint8_t *ptr, float (&v)[4]) {
+                const uint2 raw = *reinterpret_cast<const uint2 *>(ptr);
+                const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+                const float2 y = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+                v[0] = x.x; v[1] = x.y; v[2] = y.x; v[3] = y.y;
+            };
+#pragma unroll
+            for (int rr = 0; rr < HR; ++rr) {
+                const int r = SUB * ti + HR * hh + rr;
+                const uint32_t off_r = sw128_offset(r, cin);
+                const uint32_t off_q = sw128_offset(64 + r, cin);
+                float kx[4], qx[4];
+                ld4(l0 + off_r, kx);
+                ld4(l0 + off_q, qx);
+                float F[4], Fi[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    F[e] = ex2(gl[rr][e]);    // e^{G_r - G_start(ti)}, in [e^-80, 1]
+                    Fi[e] = ex2(-gl[rr][e]);  // e^{G_start(ti) - G_r}, in [1, e^80]
+                }
+                float kr[4], kf[4], qf[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    kr[e] = kx[e] * Fi[e];
+                    kf[e] = kx[e] * F[e];
+                    qf[e] = qx[e] * F[e];
+                }
+                *reinterpret_cast<uint2 *>(rrow + off_r) = pk4(kr[0] * er[0], kr[1] * er[1], kr[2] * er[2], kr[3] * er[3]);
+                *reinterpret_cast<uint2 *>(kh_rec + off_r) =
+                    pk4(kr[0] * post[0], kr[1] * post[1], kr[2] * post[2], kr[3] * post[3]);
+                *reinterpret_cast<uint2 *>(l0 + off_r) = pk4(kf[0] * el0[0], kf[1] * el0[1], kf[2] * el0[2], kf[3] * el0[3]);
+                *reinterpret_cast<uint2 *>(l0 + off_q) = pk4(qf[0] * el0[0], qf[1] * el0[1], qf[2] * el0[2], qf[3] * el0[3]);
+                if (ti >= 2) {
+                    *reinterpret_cast<uint2 *>(l1 + sw128_offset(r - 32, cin)) =
+                        pk4(kf[0] * el1[0], kf[1] * el1[1], kf[2] * el1[2], kf[3] * el1[3]);
+                    *reinterpret_cast<uint2 *>(l1 + sw128_offset(r, cin)) =
+                        pk4(qf[0] * el1[0], qf[1] * el1[1], qf[2] * el1[2], qf[3] * el1[3]);
+                }
+                *reinterpret_cast<uint2 *>(gq_rec + off_r) = pk4(qf[0] * pg[0], qf[1] * pg[1], qf[2] * pg[2], qf[3] * pg[3]);
+                *reinterpret_cast<uint2 *>(gkrow + off_r) = pk4(kf[0] * pg[0], kf[1] * pg[1], kf[2] * pg[2], kf[3] * pg[3]);
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // ---- Gram MMAs: column block j -> TMEM columns 32j..32j+31, issued by lane 0 of warp j
+        if (lane == 0 && warp < 2) {
+            const int j = warp;
+            tc_fence_after();
+            Opnd A = (j == 0) ? Opnd{sbase + P_L0, false, 16 * KB, 0} : Opnd{sbase + P_L1, false, 8 * KB, 0};
+            Opnd B{sbase + P_R + 32u * j * 128u, false, 8 * KB, 0};
+            mma_chain<D / 16>(tmem + P_TM_W + 32u * j, A, B, idG, false);
+            mma_commit(bar_gram);
+        }
+        {
+            const bool ok = mbar_wait_bounded(bar_gram, gram_phase, kWaitCycles);
+            if (!ok) { mma_bar = bar_gram; mma_bar_phase = gram_phase; }
+            gram_phase ^= 1u;
+            tc_fence_after();
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+        }
+
+        // ---- Gram readout -> A (fp32, strictly lower, times beta_r), P (bf16, lower) staging.
+        // The masks select (never multiply), so upper-triangle entries that overflow are dropped.
+        {
+            float v2[2][16];
+            tmem_ld16(tmem + tlane + P_TM_W + 32u * half, v2[0]);
+            tmem_ld16(tmem + tlane + P_TM_W + 32u * half + 16u, v2[1]);
+            tmem_wait_ld();
+            const int j = half;
+            const int m = 32 * quarter + lane;
+            const int kr = 64 - 32 * j;
+            if (m < kr) {
+                const int r = 32 * j + m;
+                const float b = sBeta[r];
+                float4 *arow = reinterpret_cast<float4 *>(AF + r * LDA + 32 * j);
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    const float *v = v2[q4 >> 2] + 4 * (q4 & 3);
+                    const int s = 32 * j + 4 * q4;
+                    arow[q4] = make_float4((s < r) ? b * v[0] : 0.f, (s + 1 < r) ? b * v[1] : 0.f,
+                                           (s + 2 < r) ? b * v[2] : 0.f, (s + 3 < r) ? b * v[3] : 0.f);
+                }
+            } else if (m < 2 * kr) {
+                const int r = 32 * j + (m - kr);
+                uint8_t *prow = sm + P_PST;
+#pragma unroll
+                for (int s2 = 0; s2 < 32; s2 += 2) {
+                    const int s = 32 * j + s2;
+                    const float *v = v2[s2 >> 4] + (s2 & 15);
+                    st_bf2(prow + sw128_offset(r, s), (s <= r) ? v[0] : 0.f, (s + 1 <= r) ? v[1] : 0.f);
+                }
+                if (j == 0 && r < 32) {  // the diagonal block of block 0: zero block 1's columns
+                    for (int s = 32; s < C; s += 8)
+                        *reinterpret_cast<uint4 *>(prow + sw128_offset(r, s)) = make_uint4(0, 0, 0, 0);
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            bulk_store(rec + REC_P, sm + P_PST, 8 * KB);
+            bulk_commit();
+        }
+
+        // ---- T = (I + A)^{-1} (unit lower triangular) by 16 x 16 blocks
+        if (warp < NSUB && lane < 16) {
+            const int o0 = 16 * warp, cc = lane;
+            float x[16];
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                float a[16];
+                const float4 *arow = reinterpret_cast<const float4 *>(AF + (o0 + rr) * LDA + o0);
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    if (4 * q4 < rr) {
+                        const float4 tt = arow[q4];
+                        a[4 * q4] = tt.x; a[4 * q4 + 1] = tt.y; a[4 * q4 + 2] = tt.z; a[4 * q4 + 3] = tt.w;
+                    }
+                }
+                float acc[4] = {(rr == cc) ? 1.f : 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ss = 0; ss < rr; ++ss) acc[ss & 3] = fmaf(-a[ss], x[ss], acc[ss & 3]);
+                x[rr] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+            }
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) TF[(o0 + rr) * LDT + o0 + cc] = x[rr];
+            if ((warp & 1) == 0) {
+#pragma unroll
+                for (int rr = 0; rr < 16; ++rr) TF[(o0 + rr) * LDT + o0 + 16 + cc] = 0.f;
+            }
+        }
+        __syncthreads();
+        tri_inverse_offdiag(AF, TF, XS, tid);
+        // T Diag(beta) -> bf16 A operand, rows 0..63 (rows 64..127 of the product are never read)
+        {
+            const int r = tid >> 3, pc = (tid & 7) * 8;
+            const float4 b0 = *reinterpret_cast<const float4 *>(sBeta + pc);
+            const float4 b1 = *reinterpret_cast<const float4 *>(sBeta + pc + 4);
+            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+                const int ri = r + 32 * i;
+                const float4 t0 = *reinterpret_cast<const float4 *>(TF + ri * LDT + pc);
+                const float4 t1 = *reinterpret_cast<const float4 *>(TF + ri * LDT + pc + 4);
+                const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
+                float u[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) u[e] = (pc + e <= ri) ? tv[e] * bb[e] : 0.f;
+                uint4 w;
+                w.x = pack_bf2(u[0], u[1]);
+                w.y = pack_bf2(u[2], u[3]);
+                w.z = pack_bf2(u[4], u[5]);
+                w.w = pack_bf2(u[6], u[7]);
+                *reinterpret_cast<uint4 *>(sm + P_TB + sw128_offset(ri, pc)) = w;
+            }
+        }
+        // ---- v of this task (zero rows past the end; all zero for a transition pass)
+        if (has_v) {
+            const bool ok = mbar_wait_bounded(bar_v, v_phase, kWaitCycles);
+            if (ok) { v_phase ^= 1u; v_armed = false; }
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+            if (Lc < C) {
+                for (int idx = tid; idx < (C - Lc) * 16; idx += NT) {
+                    const int r = Lc + idx / 16, q16 = idx % 16;
+                    *reinterpret_cast<uint4 *>(sm + P_GV + (q16 >> 3) * 8 * KB + sw128_offset(r, (q16 & 7) * 8)) =
+                        make_uint4(0, 0, 0, 0);
+                }
+            }
+        } else {
+            for (int idx = tid; idx < 16 * KB / 16; idx += NT)
+                *reinterpret_cast<uint4 *>(sm + P_GV + 16 * idx) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+
+        // ---- [W | Ut] = T Diag(beta) [Gamma K | V]
+        if (tid == 0) {
+            tc_fence_after();
+            Opnd A{sbase + P_TB, false, 16 * KB, 0};
+            Opnd BK{sbase + P_GK, true, 0, 8 * KB};
+            Opnd BV{sbase + P_GV, true, 0, 8 * KB};
+            mma_chain<C / 16>(tmem + P_TM_W, A, BK, idKM, false);
+            mma_chain<C / 16>(tmem + P_TM_UT, A, BV, idKM, false);
+            mma_commit(bar_mma);
+        }
+        {
+            const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
+            if (!ok) { mma_bar = bar_mma; mma_bar_phase = mma_phase; }
+            mma_phase ^= 1u;
+            tc_fence_after();
+            if (__syncthreads_or(!ok)) { aborted = true; break; }
+        }
+        // the next task's k, q, g: L0 and the g / v tile are free
+        if (more && tid == 0) {
+            mbar_arrive_expect_tx(bar_ld, 48 * KB);
+            issue_kqg(nxt);
+            ld_armed = true;
+        }
+
+        // ---- -W and Ut (rows 0..63) -> staging -> record
+        if (quarter < 2) {
+            const int r = 32 * quarter + lane;
+            float v[4][16];
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + P_TM_W + 64u * half + 16u * gq, v[gq]);
+            tmem_wait_ld();
+            uint8_t *wst = sm + P_WST + half * 8 * KB;
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) {
+                uint4 w0, w1;
+                pack16(v[gq], -1.f, w0, w1);
+                *reinterpret_cast<uint4 *>(wst + sw128_offset(r, 16 * gq)) = w0;
+                *reinterpret_cast<uint4 *>(wst + sw128_offset(r, 16 * gq + 8)) = w1;
+            }
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + P_TM_UT + 64u * half + 16u * gq, v[gq]);
+            tmem_wait_ld();
+            uint8_t *ust = sm + P_UST + half * 8 * KB;
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) {
+                uint4 w0, w1;
+                pack16(v[gq], 1.f, w0, w1);
+                *reinterpret_cast<uint4 *>(ust + sw128_offset(r, 16 * gq)) = w0;
+                *reinterpret_cast<uint4 *>(ust + sw128_offset(r, 16 * gq + 8)) = w1;
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            bulk_store(rec + REC_WQ, sm + P_WST, 8 * KB);
+            bulk_store(rec + REC_WQ + 16 * KB, sm + P_WST + 8 * KB, 8 * KB);
+            bulk_store(rec + REC_UT, sm + P_UST, 16 * KB);
+            bulk_commit();
+        }
+        cur = nxt;
+        t = tn;
+        have = more;
+        bcur = bnext;
+    }
+    if (tid == 0) bulk_wait_all();  // record stores complete (the direct stores are ordinary writes)
+    if (aborted && tid == 0) {
+        // unwind with nothing in flight: armed copies complete (bounded), a timed-out commit is
+        // waited for (bounded) before TMEM is freed
+        if (p.dev_status) atomicExch(p.dev_status, (int)KDA_ERR_TIMEOUT);
+        if (ld_armed) mbar_wait_bounded(bar_ld, ld_phase, kWaitCycles);
+        if (v_armed) mbar_wait_bounded(bar_v, v_phase, kWaitCycles);
+        if (mma_bar) mbar_wait_bounded(mma_bar, mma_bar_phase, kWaitCycles);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, P_TM_COLS);
+    }
+}
+
+// ====================================================================== chain
+__global__ void __launch_bounds__(NT, 1)
+kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp) {
+    const PrefillArgs &p = sp.a;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bar_rec = reinterpret_cast<uint64_t *>(sm + C_BAR);  // [2]: the record of buffer b
+    uint64_t *bar_mma = bar_rec + 2;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + C_TMEMADDR);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int h = blockIdx.x % p.H;
+    const int n = unit_seq(p, blockIdx.x / p.H);
+    const size_t H = (size_t)p.H;
+    long long t_begin, len, cbase;
+    if (p.cu_seqlens) {
+        t_begin = p.cu_seqlens[n];
+        len = (long long)p.cu_seqlens[n + 1] - t_begin;
+        cbase = sp.chunk_base[n];
+    } else {
+        t_begin = (long long)n * p.T;
+        len = p.T;
+        cbase = (long long)n * sp.nch;
+    }
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
+    const size_t state_base = ((size_t)n * H + h) * (size_t)(D * D);
+    const long long nchunks = (len + C - 1) / C;
+    auto record = [&](long long c) -> const uint8_t * {
+        return sp.rec + ((size_t)(cbase + c) * H + (size_t)h) * REC_BYTES;
+    };
+
+    if (tid == 0) {
+        mbar_init(&bar_rec[0], 1);
+        mbar_init(&bar_rec[1], 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_o);
+    }
+    if (warp == 0) {
+        tmem_alloc(s_tmem, C_TM_COLS);
+        tmem_relinquish();
+    }
+    __syncthreads();
+    // bit b: buffer b has a record load armed and not yet waited for / the parity of its next phase
+    uint32_t rec_armed = 0, rec_phase = 0;
+    if (tid == 0) {
+        for (int b = 0; b < 2 && b < nchunks; ++b) {
+            mbar_arrive_expect_tx(&bar_rec[b], REC_BYTES);
+            bulk_load(sm + b * C_RECSTRIDE, record(b), REC_BYTES, &bar_rec[b]);
+            rec_armed |= 1u << b;
+        }
+    }
+    // incoming state -> TMEM (fp32, lane = dk row, column = dv) and its bf16 copy
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t tlane = (uint32_t)(32 * quarter) << 16;
+    const int si = 32 * quarter + lane;
+    {
+        uint8_t *sb = sm + C_SB + half * 16 * KB;
+#pragma unroll
+        for (int gq = 0; gq < 4; ++gq) {
+            float v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int j = 64 * half + 16 * gq + e;
+                v[e] = p.S0 ? p.S0[state_base + (size_t)j * D + si] : 0.f;
+            }
+            tmem_st16(tmem + tlane + C_TM_S + 64u * half + 16u * gq, v);
+            uint4 w0, w1;
+            pack16(v, 1.f, w0, w1);
+            *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq)) = w0;
+            *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq + 8)) = w1;
+        }
+        tmem_wait_st();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    constexpr uint32_t idKM = idesc_bf16_f32(128, 128, 0, 1);
+    constexpr uint32_t idMM = idesc_bf16_f32(128, 128, 1, 1);
+    uint32_t mma_phase = 0;
+    bool aborted = false, mma_pending = false;
+    auto wait_rec = [&](int b) -> bool {  // every thread takes part
+        const bool ok = mbar_wait_bounded(&bar_rec[b], (rec_phase >> b) & 1u, kWaitCycles);
+        if (ok) { rec_phase ^= 1u << b; rec_armed &= ~(1u << b); }
+        return __syncthreads_or(!ok) == 0;
+    };
+    auto wait_mma = [&]() -> bool {
+        const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
+        if (ok) { mma_phase ^= 1u; mma_pending = false; }
+        tc_fence_after();
+        return __syncthreads_or(!ok) == 0;
+    };
+    auto issue_u = [&](int b) {  // [U ; Gamma Q S] = [-W ; Gamma Q] S into the accumulator of buffer b
+        tc_fence_after();
+        Opnd A{sbase + b * C_RECSTRIDE + REC_WQ, false, 16 * KB, 0};
+        Opnd B{sbase + C_SB, true, 0, 16 * KB};
+        mma_chain<D / 16>(tmem + (b ? C_TM_U1 : C_TM_U0), A, B, idKM, false);
+        mma_commit(bar_mma);
+    };
+
+    if (nchunks > 0) {
+        if (!wait_rec(0)) aborted = true;
+        else if (tid == 0) { issue_u(0); mma_pending = true; }
+    }
+    for (long long ch = 0; ch < nchunks && !aborted; ++ch) {
+        const int b = (int)(ch & 1);
+        uint8_t *buf = sm + b * C_RECSTRIDE;
+        const uint32_t tmu = b ? C_TM_U1 : C_TM_U0;
+        const long long tok0 = t_begin + ch * C;
+        const int Lc = (int)((len - ch * C) < C ? (len - ch * C) : C);
+        const bool more = ch + 1 < nchunks;
+
+        // S <- Diag(Gamma_C) S in TMEM while the state product runs, so that Kh^T U
+        // accumulates onto the state directly
+        {
+            const float gam = reinterpret_cast<const float *>(buf + REC_GC)[si];
+            float sv[4][16];
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + C_TM_S + 64u * half + 16u * gq, sv[gq]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) sv[gq][e] *= gam;
+                tmem_st16(tmem + tlane + C_TM_S + 64u * half + 16u * gq, sv[gq]);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+        }
+        if (!wait_mma()) { aborted = true; break; }
+
+        // U = Ut - W S (rows 0..63) -> bf16 B operand, written over the record's Ut tile
+        if (quarter < 2) {
+            const int r = 32 * quarter + lane;
+            uint8_t *ut = buf + REC_UT + half * 8 * KB;
+            float v[4][16];
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + tmu + 64u * half + 16u * gq, v[gq]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) {
+#pragma unroll
+                for (int pc = 0; pc < 2; ++pc) {
+                    uint4 *slot = reinterpret_cast<uint4 *>(ut + sw128_offset(r, 16 * gq + 8 * pc));
+                    const uint4 w = *slot;
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                    float *x = v[gq] + 8 * pc;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ws[e]));
+                        x[2 * e] += f.x;
+                        x[2 * e + 1] += f.y;
+                    }
+                    uint4 o4;
+                    o4.x = pack_bf2(x[0], x[1]);
+                    o4.y = pack_bf2(x[2], x[3]);
+                    o4.z = pack_bf2(x[4], x[5]);
+                    o4.w = pack_bf2(x[6], x[7]);
+                    *slot = o4;
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // O = Gamma Q S + P U (rows 64..127 of the accumulator), S += Kh^T U
+        if (tid == 0) {
+            tc_fence_after();
+            Opnd AK{sbase + b * C_RECSTRIDE + REC_KH, true, 0, 8 * KB};
+            Opnd BU{sbase + b * C_RECSTRIDE + REC_UT, true, 0, 8 * KB};
+            Opnd AP{sbase + b * C_RECSTRIDE + REC_P - 8 * KB, false, 16 * KB, 0};
+            mma_chain<C / 16>(tmem + C_TM_S, AK, BU, idMM, true);
+            mma_chain<C / 16>(tmem + tmu, AP, BU, idKM, true);
+            mma_commit(bar_mma);
+            mma_pending = true;
+        }
+        if (!wait_mma()) { aborted = true; break; }
+
+        // the bf16 copy of the updated state: the next chunk's state product waits on it
+        {
+            uint8_t *sb = sm + C_SB + half * 16 * KB;
+            float sv[4][16];
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + C_TM_S + 64u * half + 16u * gq, sv[gq]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) {
+                uint4 w0, w1;
+                pack16(sv[gq], 1.f, w0, w1);
+                *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq)) = w0;
+                *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq + 8)) = w1;
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (more) {
+            if (!wait_rec(b ^ 1)) { aborted = true; break; }
+            if (tid == 0) { issue_u(b ^ 1); mma_pending = true; }
+        }
+
+        // outputs (rows 64..127 of this chunk's accumulator) while the next product runs. A
+        // full chunk is staged over the U tile (its products are done) and leaves by two
+        // tensor stores; the rows of a partial chunk are stored directly.
+        if (quarter >= 2 && p.o) {
+            const int r = 32 * quarter + lane - 64;
+            float v[4][16];
+#pragma unroll
+            for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + tmu + 64u * half + 16u * gq, v[gq]);
+            tmem_wait_ld();
+            if (Lc == C) {
+                uint8_t *base = buf + REC_UT + half * 8 * KB;
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) {
+                    uint4 w0, w1;
+                    pack16(v[gq], 1.f, w0, w1);
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, 16 * gq)) = w0;
+                    *reinterpret_cast<uint4 *>(base + sw128_offset(r, 16 * gq + 8)) = w1;
+                }
+            } else if (r < Lc) {
+                uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(tok0 + r) * H + h) * D + 64 * half);
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq) {
+                    uint4 w0, w1;
+                    pack16(v[gq], 1.f, w0, w1);
+                    dst[2 * gq] = w0;
+                    dst[2 * gq + 1] = w1;
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            if (Lc == C && p.o) {
+                tma_store_3d(&tm_o, buf + REC_UT, 0, h, (int)tok0);
+                tma_store_3d(&tm_o, buf + REC_UT + 8 * KB, 64, h, (int)tok0);
+                bulk_commit();
+            }
+            if (ch + 2 < nchunks) {  // the record two chunks ahead goes into this buffer once the
+                bulk_wait_read_all();  // output stores have read it
+                mbar_arrive_expect_tx(&bar_rec[b], REC_BYTES);
+                bulk_load(buf, record(ch + 2), REC_BYTES, &bar_rec[b]);
+                rec_armed |= 1u << b;
+            }
+        }
+    }
+    if (tid == 0) bulk_wait_all();
+
+    if (aborted) {
+        if (tid == 0) {
+            if (p.dev_status) atomicExch(p.dev_status, (int)KDA_ERR_TIMEOUT);
+            for (int b = 0; b < 2; ++b)
+                if ((rec_armed >> b) & 1u) mbar_wait_bounded(&bar_rec[b], (rec_phase >> b) & 1u, kWaitCycles);
+            if (mma_pending) mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
+        }
+    } else if (p.ST) {
+        tc_fence_after();
+#pragma unroll
+        for (int gq = 0; gq < 4; ++gq) {
+            float sv[16];
+            tmem_ld16(tmem + tlane + C_TM_S + 64u * half + 16u * gq, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int j = 64 * half + 16 * gq + e;
+                p.ST[state_base + (size_t)j * D + si] = sv[e];
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C_TM_COLS);
+    }
+}
+
+int num_sms() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+            n = v;
+        else
+            n = 148;
+    }
+    return n;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// One packed sequence (cu_seqlens = [0, T]) is the dense batch B = 1; the split form treats it
+// so, which keeps its workspace the size kda_forward_workspace_size reports for num_seqs = 1.
+bool packed(const PrefillArgs &a) { return a.cu_seqlens != nullptr && a.num_units > 1; }
+
+// Upper bound of the number of tasks: dense batches exactly, packed ones by
+// sum ceil(len / C) <= T / C + num_seqs.
+long long split_tasks_bound(const PrefillArgs &a) {
+    if (packed(a)) return ((long long)(a.T + C - 1) / C + a.num_units) * a.H;
+    return (long long)a.B * ((a.T + C - 1) / C) * a.H;
+}
+
+}  // namespace
+
+size_t prefill_split_workspace(const PrefillArgs &a) {
+    size_t ws = align256((size_t)split_tasks_bound(a) * REC_BYTES);
+    if (packed(a)) ws += align256((size_t)(a.num_units + 1) * sizeof(int32_t)) + align256(seq_order_bytes(a.num_units));
+    return ws;
+}
+
+int prefill_split_launches(const PrefillArgs &a) {
+    if (a.num_units <= 0 || a.H <= 0) return 0;
+    const size_t tokens = a.cu_seqlens ? (size_t)a.T : (size_t)a.B * (size_t)a.T;
+    if (tokens == 0) return prefill_simt_launches(a);
+    return 2 + (packed(a) ? 1 + (seq_order_bytes(a.num_units) > 0 ? 1 : 0) : 0);
+}
+
+cudaError_t launch_prefill_split(const PrefillArgs &a) {
+    if (a.num_units == 0) return cudaSuccess;
+    const size_t tokens = a.cu_seqlens ? (size_t)a.T : (size_t)a.B * (size_t)a.T;
+    if (tokens == 0) return launch_prefill_simt(a);
+    CUtensorMap mq, mk, mv, mg, mo;
+    if (!make_map(&mq, a.q, tokens, a.H, 64, true) || !make_map(&mk, a.k, tokens, a.H, 64, true) ||
+        !make_map(&mv, a.v ? a.v : a.q, tokens, a.H, 64, true) || !make_map(&mg, a.g, tokens, a.H, 128, false) ||
+        !make_map(&mo, a.o ? a.o : a.q, tokens, a.H, 64, true))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kda_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    SplitParams sp{};
+    sp.a = a;
+    if (!packed(a)) sp.a.cu_seqlens = nullptr;  // dense, or one packed sequence = B = 1 of T tokens
+    uint8_t *ws = static_cast<uint8_t *>(a.workspace);
+    sp.rec = ws;
+    const long long bound = split_tasks_bound(a);
+    size_t off = align256((size_t)bound * REC_BYTES);
+    if (packed(a)) {
+        int32_t *base = reinterpret_cast<int32_t *>(ws + off);
+        off += align256((size_t)(a.num_units + 1) * sizeof(int32_t));
+        chunk_base_kernel<<<1, 1024, 0, a.stream>>>(a.cu_seqlens, a.num_units, base);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        sp.chunk_base = base;
+        if (seq_order_bytes(a.num_units) > 0) {
+            int32_t *order = reinterpret_cast<int32_t *>(ws + off);
+            e = launch_seq_order(a.cu_seqlens, a.num_units, order, a.stream);
+            if (e != cudaSuccess) return e;
+            sp.a.seq_order = order;
+        }
+    } else {
+        sp.nch = (a.T + C - 1) / C;
+        sp.tasks = bound;
+    }
+    const long long grid_p = bound < 2LL * num_sms() ? bound : 2LL * num_sms();
+    kda_prep_kernel<<<(unsigned)grid_p, NT, P_SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, sp);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const unsigned grid_c = (unsigned)((size_t)a.num_units * a.H);
+    kda_chain_kernel<<<grid_c, NT, C_SMEM_BYTES, a.stream>>>(mo, sp);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

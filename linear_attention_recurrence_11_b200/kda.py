@@ -67,7 +67,7 @@ _lib.kda_forward_host.restype = _i
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT = 0, 1, 2, 3
 KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_SCRATCH_LIMIT = 4, 5, 6, 7
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
-PATHS = {"auto": 0, "simt": 1, "tc": 2}
+PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_single": 3, "tc_split": 4}
 KDA_FUSE_NORM_QK, KDA_FUSE_GATE_LOGITS = 1, 2  # fused pre-operations (see include/kda.h)
 
 

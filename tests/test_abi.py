@@ -110,20 +110,35 @@ def test_decode_rejects_bad_args(K):
 
 
 def test_workspace_and_launch_queries(K):
-    assert K.kda_forward_workspace_size(1, 8192, 96, 128, 128, 64, 1, 1) == 0
-    assert K.kda_forward_workspace_size(2, 8192, 96, 128, 128, 64, 2, 1) == 0
-    # packed sequences: a small longest-first schedule (up to 2048 sequences)
-    assert K.kda_forward_workspace_size(1, 352549, 96, 128, 128, 64, 8, 1) == 256
+    # tensor-core shapes: the split form's per-chunk records, 74,240 bytes per chunk per head
+    # ([-W ; Gamma q] 32 KiB, Kh 16 KiB, Ut 16 KiB, P 8 KiB, Gamma_C 512 B)
+    rec = 74240
+    al = lambda x: (x + 255) // 256 * 256
+    assert K.kda_forward_workspace_size(1, 8192, 96, 128, 128, 64, 1, 1) == 128 * 96 * rec
+    assert K.kda_forward_workspace_size(2, 8192, 96, 128, 128, 64, 2, 1) == 2 * 128 * 96 * rec
+    assert K.kda_forward_workspace_size(2, 100, 3, 128, 128, 64, 2, 1) == 2 * 2 * 3 * rec
+    # packed sequences: records for at most T / 64 + N chunks per head, the sequences' chunk
+    # offsets, and a small longest-first schedule (up to 2048 sequences)
+    n_ch = -(-352549 // 64) + 8
+    assert K.kda_forward_workspace_size(1, 352549, 96, 128, 128, 64, 8, 1) == \
+        al(n_ch * 96 * rec) + al(9 * 4) + 256
+    # other shapes (SIMT kernel): only the schedule
     assert K.kda_forward_workspace_size(1, 100000, 2, 64, 64, 32, 2048, 0) == 8192
     assert K.kda_forward_workspace_size(1, 100000, 2, 64, 64, 32, 2049, 0) == 0
-    assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8) == 2
+    # launches: split = prep + chains (+ chunk offsets and schedule for packed batches)
+    assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8) == 4
+    assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8, "tc_single") == 2
     assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8, "simt") == 2
-    assert K.kda_forward_launches(1, 8192, 96, 128, 128, 64, 1, 0, 1) == 1
+    assert K.kda_forward_launches(1, 8192, 96, 128, 128, 64, 1, 0, 1) == 2
+    assert K.kda_forward_launches(1, 8192, 96, 128, 128, 64, 1, 0, 1, "tc_split") == 2
+    assert K.kda_forward_launches(1, 8192, 96, 128, 128, 64, 1, 0, 1, "tc_single") == 1
     with pytest.raises(K.KdaError):
         K.kda_forward_workspace_size(1, 8192, 96, 100, 128, 64, 1, 1)
-    assert K.kda_forward_launches(1, 8192, 96, 128, 128, 64, 1, 0, 1) >= 1
     assert K.kda_forward_launches(1, 256, 1, 32, 32, 16, 0, 0, 1, "simt") == 1
     assert K.kda_forward_launches(1, 256, 1, 48, 32, 16, 0, 0, 1) == -1
+    # forcing a tensor-core form off its shapes is refused
+    assert K.kda_forward_launches(1, 256, 1, 32, 32, 16, 0, 0, 1, "tc_split") == -1
+    assert K.kda_forward_launches(1, 256, 1, 32, 32, 16, 0, 0, 1, "tc_single") == -1
 
 
 def test_python_binding_refuses_cpu_tensors(K):
@@ -166,9 +181,9 @@ def test_segmented_queries(K):
     # the transition of a dk = 64 segment is 64 x 64 whatever dv is
     n2 = K.kda_forward_segmented_workspace_size(1, 1000, 2, 64, 128, 64, 1, 256)
     assert n2 >= 4 * 2 * (64 * 64 + 2 * 128 * 64) * 4
-    # one segment: the plain prefill's needs (none for a dense batch)
-    assert K.kda_forward_segmented_workspace_size(2, 1000, 2, 128, 128, 64, 1, 1024) == 0
-    assert K.kda_forward_segmented_launches(2, 1000, 2, 128, 128, 64, 1, 1024) == 1
+    # one segment: the plain prefill's needs (the split form's records for a dense batch)
+    assert K.kda_forward_segmented_workspace_size(2, 1000, 2, 128, 128, 64, 1, 1024) == 2 * 16 * 2 * 74240
+    assert K.kda_forward_segmented_launches(2, 1000, 2, 128, 128, 64, 1, 1024) == 2
     # init, three passes each with a longest-first schedule, scan
     assert K.kda_forward_segmented_launches(1, 1000, 2, 128, 128, 64, 1, 256) == 8
     with pytest.raises(K.KdaError):
@@ -249,14 +264,17 @@ def test_host_entry_point_validates_before_any_cuda_call(K):
 
 
 def test_host_workspace_size_is_two_piece_slots_and_the_state(K):
-    # two slots of one piece's q, k, v, g, beta and o (each rounded up to 256 bytes) plus the fp32 state
+    # two slots of one piece's q, k, v, g, beta and o (each rounded up to 256 bytes), the fp32
+    # state, and the device prefill's workspace for one piece (the split form's records)
     B, T, H, d, L = 1, 8192, 96, 128, 1024
     piece = B * L * H * d * 2
     slot = 5 * piece + B * L * H * 2
     state = B * H * d * d * 4
-    assert K.kda_forward_host_workspace_size(B, T, H, d, d, 64, 1, L) == 2 * slot + state
+    records = K.kda_forward_workspace_size(B, L, H, d, d, 64, B, 1)
+    assert records == B * (L // 64) * H * 74240
+    assert K.kda_forward_host_workspace_size(B, T, H, d, d, 64, 1, L) == 2 * slot + state + records
     # piece_len 0: about T / 8 in whole chunks; a piece never exceeds the sequence
-    assert K.kda_forward_host_workspace_size(B, T, H, d, d, 64, 1, 0) == 2 * slot + state
+    assert K.kda_forward_host_workspace_size(B, T, H, d, d, 64, 1, 0) == 2 * slot + state + records
     small = K.kda_forward_host_workspace_size(2, 100, 3, 64, 32, 32, 0, 256)
     tok = 2 * 100 * 3
     rnd = lambda x: (x + 255) // 256 * 256

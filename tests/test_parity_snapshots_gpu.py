@@ -54,8 +54,9 @@ def test_resume_from_a_snapshot(K):
     o, ST, Ssn = K.kda_forward_snapshots(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"],
                                          snap_every=256, chunk=64)
     rest = {x: inp[x][:, 512:].contiguous() for x in ("q", "k", "v", "g", "beta")}
+    # snapshots come from the single-kernel form; resume on the same form
     o2, S2 = K.kda_forward(rest["q"], rest["k"], rest["v"], rest["g"], rest["beta"], Ssn[:, 1].contiguous(),
-                           chunk=64)
+                           chunk=64, path="tc_single")
     torch.cuda.synchronize()
     assert rel(to_f64(o2), to_f64(o[:, 512:])) < 1e-5 and rel(to_f64(S2), to_f64(ST)) < 1e-5
 
@@ -65,6 +66,6 @@ def test_no_snapshot_due(K, oracle_mod):
     inp = case(1, 100, 2, 128, 128, "bf16", seed=63)
     o, ST, Ssn = K.kda_forward_snapshots(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None,
                                          snap_every=128, chunk=64)
-    o2, S2 = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None, chunk=64)
+    o2, S2 = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None, chunk=64, path="tc_single")
     torch.cuda.synchronize()
     assert Ssn.shape[1] == 0 and torch.equal(o, o2) and torch.equal(ST, S2)

@@ -1,0 +1,110 @@
+"""GPU parity of the two tensor-core prefill forms against each other and the
+oracle: the split form (a chunk-parallel kernel writes every chunk's
+state-independent operands to the workspace, a second kernel carries each
+unit's state) and the single-kernel form compute the same chunked recurrence
+("Exercices", Q7, Q21-Q22) and must agree with the fp64 oracle and with each
+other; the workspace passed decides which form AUTO runs."""
+import numpy as np
+import pytest
+import torch
+
+from kda_testutil import TOL, case, compare_units, oracle_forward, rel
+from linear_attention_recurrence_11_b200.inputs import to_f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def K():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from linear_attention_recurrence_11_b200 import kda
+    return kda
+
+
+def fwd(K, inp, path, **kw):
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    o, ST = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp.get("S0"), chunk=64,
+                          cu_seqlens=inp.get("cu_seqlens"), path=path, dev_status=status, **kw)
+    torch.cuda.synchronize()
+    assert int(status[0]) == 0
+    return o, ST
+
+
+@pytest.mark.parametrize("B,T,H", [(1, 64, 1), (2, 200, 3), (1, 1, 2), (3, 127, 2), (1, 64 * 9 + 5, 4)])
+def test_split_matches_oracle_and_single(K, oracle_mod, B, T, H):
+    inp = case(B, T, H, 128, 128, "bf16", seed=1000 + T + B, s0_std=0.05, g_min_frac=0.1)
+    o_s, S_s = fwd(K, inp, "tc_split")
+    o_f, S_f = fwd(K, inp, "tc_single")
+    o_ref, S_ref = oracle_forward(oracle_mod, inp)
+    units = [(b, h) for b in range(B) for h in range(H)]
+    compare_units(o_s, S_s, o_ref, S_ref, units, tol=TOL["bf16"], label="split")
+    compare_units(o_f, S_f, o_ref, S_ref, units, tol=TOL["bf16"], label="single")
+    # the two forms round at slightly different points (Ut reaches the state product in bf16
+    # in the split form), so they agree to the bf16 level, not bit for bit
+    assert rel(to_f64(o_s), to_f64(o_f)) < 5e-3 and rel(to_f64(S_s), to_f64(S_f)) < 5e-3
+
+
+@pytest.mark.parametrize("lens", [[1, 65, 130, 0, 64, 7, 200], [0, 0, 3], [500], [64] * 40 + [0, 129]])
+def test_split_packed(K, oracle_mod, lens):
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    H = 3
+    inp = case(1, int(cu[-1]), H, 128, 128, "bf16", seed=len(lens) + int(cu[-1]), s0_std=0.1,
+               num_states=len(lens))
+    inp["cu_seqlens"] = torch.tensor(cu, device="cuda")
+    o, ST = fwd(K, inp, "tc_split")
+    o_ref, S_ref = oracle_forward(oracle_mod, inp)
+    units = [(n, h) for n in range(len(lens)) for h in range(H)]
+    compare_units(o, ST, o_ref, S_ref, units, cu, tol=TOL["bf16"], label="split packed")
+    zero = [n for n, L in enumerate(lens) if L == 0]
+    if zero:
+        assert torch.equal(ST[zero], inp["S0"][zero])
+
+
+def test_split_identity_transition_is_exact(K):
+    """beta = 0, g = 0: every record's W, Ut and P-columns vanish and Gamma_C = 1, so the
+    state passes through bit for bit."""
+    inp = case(2, 150, 2, 128, 128, "bf16", seed=21, s0_std=0.5)
+    inp["g"].zero_(); inp["beta"].zero_()
+    o, ST = fwd(K, inp, "tc_split")
+    assert torch.equal(ST, inp["S0"])
+    ref = torch.einsum("bthi,bhji->bthj", inp["q"].double(), inp["S0"].double())
+    assert rel(to_f64(o), ref.cpu().numpy()) < TOL["bf16"]
+
+
+def test_split_g_min_runs(K, oracle_mod):
+    """Whole channels and 128-token runs at g = g_min = -5 (the e^80 subtile bound)."""
+    inp = case(1, 256, 2, 128, 128, "bf16", seed=11, s0_std=0.1)
+    inp["g"][:, :, :, ::3] = -5.0
+    inp["g"][:, 64:192] = -5.0
+    o, ST = fwd(K, inp, "tc_split")
+    o_ref, S_ref = oracle_forward(oracle_mod, inp)
+    compare_units(o, ST, o_ref, S_ref, [(0, 0), (0, 1)], tol=TOL["bf16"], label="split g_min")
+
+
+def test_workspace_decides_the_form(K):
+    """AUTO with the reported workspace runs the split form; with only the packed schedule's
+    few bytes (or none) it runs the single form; TC_SPLIT with too small a workspace is refused."""
+    inp = case(1, 300, 2, 128, 128, "bf16", seed=5, s0_std=0.1)
+    o_split, S_split = fwd(K, inp, "tc_split")
+    o_single, S_single = fwd(K, inp, "tc_single")
+    o_a, S_a = fwd(K, inp, "auto")
+    assert torch.equal(o_a, o_split) and torch.equal(S_a, S_split)
+    small = torch.empty(256, dtype=torch.uint8, device="cuda")
+    o_b, S_b = fwd(K, inp, "auto", workspace=small)
+    assert torch.equal(o_b, o_single) and torch.equal(S_b, S_single)
+    with pytest.raises(K.KdaError) as e:
+        fwd(K, inp, "tc_split", workspace=small)
+    assert e.value.code == K.KDA_ERR_WORKSPACE
+
+
+def test_split_two_calls_reuse_workspace(K, oracle_mod):
+    """The records are scratch: a second call with other inputs in the same workspace gives
+    its own results (every record is rewritten before it is read)."""
+    ws = torch.empty(K.kda_forward_workspace_size(2, 256, 2, 128, 128, 64, 2, torch.bfloat16),
+                     dtype=torch.uint8, device="cuda")
+    for seed in (1, 2):
+        inp = case(2, 256, 2, 128, 128, "bf16", seed=seed, s0_std=0.1)
+        o, ST = fwd(K, inp, "auto", workspace=ws)
+        o_ref, S_ref = oracle_forward(oracle_mod, inp)
+        compare_units(o, ST, o_ref, S_ref, [(b, h) for b in range(2) for h in range(2)], tol=TOL["bf16"])
