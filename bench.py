@@ -46,12 +46,15 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=5)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--workload", default="prefill", choices=sorted(WORKLOAD_ALIASES))
-    p.add_argument("--path", default="auto", choices=["auto", "simt", "tc", "tc_single", "tc_split"])
+    p.add_argument("--path", default="auto", choices=["auto", "simt", "tc", "tc_single", "tc_split", "tc_pipe"])
     p.add_argument("--snap-every", type=int, default=1024,
                    help="prefill leg saving the state every N tokens (0: skip)")
     p.add_argument("--draft-tokens", type=int, default=4,
                    help="draft tokens per request in the speculative decode leg (0: skip)")
-    p.add_argument("--decode-steps", type=int, default=50)
+    p.add_argument("--decode-steps", type=int, default=0,
+                   help="decode steps timed (0: the decode workload's own count, 1000)")
+    p.add_argument("--no-varlen", action="store_true",
+                   help="skip the packed-sequence leg of the default run")
     p.add_argument("--tokens", type=int, default=0,
                    help="override T of the dense prefill workload (smaller only for profiling captures)")
     p.add_argument("--decode-requests", type=int, default=256,
@@ -280,10 +283,10 @@ def run_ours(args, rank, world, device):
     value = weak_scaling_value(tokens, K, ms_total, world)
     alg_bytes, alg_flops = prefill_algorithmic(w, elem)
     if path_used == "tc":  # the split form runs when the workspace holds its records
-        split = seg == 0 and args.path in ("auto", "tc", "tc_split")
+        split = seg == 0 and args.path in ("auto", "tc", "tc_split", "tc_pipe")
         kern_src = ("linear_attention_recurrence_11_b200/csrc/kda_prefill_split.cu" if split
                     else "linear_attention_recurrence_11_b200/csrc/kda_prefill_tc.cu")
-        path_used = "tc_split" if split else "tc_single"
+        path_used = ("tc_pipe" if args.path == "tc_pipe" else "tc_split") if split else "tc_single"
     else:
         kern_src = "linear_attention_recurrence_11_b200/csrc/kda_prefill_simt.cu"
     achieved = alg_bytes / (kern_ms / 1e3) / 1e9
@@ -354,12 +357,84 @@ def run_ours(args, rank, world, device):
     if not args.no_e2e:
         res["e2e"] = e2e_prefill(args, device, inp, w, forward, o, ST, world, barrier, max_ranks,
                                  dense=not seg and not w.seqlens)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline_prefill(inp, w, args.cpu_seconds)
+        res["cpu_baseline_all_cores"] = cpu_baseline_all_cores(inp, w)
+    default_run = args.workload == "prefill" and not args.tokens
+    del inp, o, ST, ws
+    torch.cuda.empty_cache()
+    if default_run and not args.no_varlen:
+        res["varlen"] = varlen_measure(args, device, peaks, barrier, max_ranks, world, rank)
+        torch.cuda.empty_cache()
     if not args.no_decode and args.workload == "prefill":
         res["decode"] = decode_measure(args, device, peaks, barrier, max_ranks, world,
                                        steps=args.decode_steps)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline_prefill(inp, w, args.cpu_seconds)
     return res
+
+
+def varlen_measure(args, device, peaks, barrier, max_ranks, world, rank):
+    """The packed long-context workload (8 sequences, log-uniform lengths in
+    [4096, 131072], 96 heads) through kda_forward with cu_seqlens, inputs
+    resident in HBM; and, for the chain-bound question, the longest sequence
+    alone through the same entry point (its time over the batch's time)."""
+    import torch
+    from linear_attention_recurrence_11_b200 import kda
+    from linear_attention_recurrence_11_b200.inputs import WORKLOADS, workload_inputs
+    w = rank_workload(WORKLOADS["varlen_h96_8seq_d128_bf16"], rank)
+    inp = workload_inputs(w, device=device)
+    T, N = w.total_tokens, w.num_seqs
+    dt = inp["k"].dtype
+    o = torch.empty((1, T, w.H, w.dv), dtype=dt, device=device)
+    ST = torch.empty((N, w.H, w.dv, w.dk), dtype=torch.float32, device=device)
+    ws = torch.empty(max(1, kda.kda_forward_workspace_size(1, T, w.H, w.dk, w.dv, w.chunk, N, dt)),
+                     dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream(device)
+
+    def step():
+        kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], chunk=w.chunk,
+                        cu_seqlens=inp["cu_seqlens"], o=o, S_T=ST, workspace=ws, path=args.path)
+
+    def timed(fn, K):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize(device)
+        barrier()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(K):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        return max_ranks(a.elapsed_time(b)) / K
+
+    K = max(3, min(args.steps, 5))
+    with ClockSampler(device.index) as clk:
+        ms = timed(step, K)
+    # the longest sequence alone (dense B = 1), the same kernels
+    cu = w.cu_seqlens()
+    nl = max(range(N), key=lambda n: w.seqlens[n])
+    sl = {x: inp[x][:, cu[nl]:cu[nl + 1]].contiguous() for x in ("q", "k", "v", "g", "beta")}
+    o1 = torch.empty_like(sl["v"])
+    ST1 = torch.empty((1, w.H, w.dv, w.dk), dtype=torch.float32, device=device)
+
+    def longest():
+        kda.kda_forward(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], None, chunk=w.chunk, o=o1, S_T=ST1,
+                        workspace=ws, path=args.path)
+    ms_long = timed(longest, K)
+    alg_bytes, alg_flops = prefill_algorithmic(w, dt.itemsize)
+    gbs = alg_bytes / (ms / 1e3) / 1e9
+    return {"workload": w.name, "tokens": T, "sequences": N, "lengths": list(w.seqlens),
+            "ms_per_step": ms, "tokens_per_s": world * T / (ms / 1e3),
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "algorithmic_bytes_per_step": alg_bytes,
+                         "peak_source": peaks["source"] + " (hbm_gbs)"},
+            "tensor_frac": alg_flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+            "longest_sequence": {"tokens": w.seqlens[nl], "ms": ms_long, "ratio_to_batch": ms_long / ms,
+                                 "note": "the longest sequence alone (all 96 heads) through kda_forward; "
+                                         "near 1 means the batch is bound by that sequence's chain"},
+            "gpu_launches": K * kda.kda_forward_launches(1, T, w.H, w.dk, w.dv, w.chunk, dt, True, N, args.path),
+            "steps": K, "clocks": clk.summary(),
+            "l2": f"inputs larger than L2 ({4 * inp['q'].numel() * dt.itemsize / 1e9:.1f} GB read per step)"}
 
 
 def e2e_prefill(args, device, inp, w, forward, o, ST, world, barrier, max_ranks, dense):
@@ -427,9 +502,10 @@ def e2e_prefill(args, device, inp, w, forward, o, ST, world, barrier, max_ranks,
 
 
 def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):
-    """Decode step over 256 requests x 96 heads (1.61 GB of fp32 state, larger
-    than L2), states updated in place; per-step inputs cycle over 8 pre-drawn
-    sets."""
+    """Decode steps over 256 requests x 96 heads (1.61 GB of fp32 state, larger
+    than L2), states updated in place, for the workload's step count (1000)
+    unless --decode-steps says otherwise; every step has its own seeded inputs
+    (drawn before the timed region)."""
     import torch
     from linear_attention_recurrence_11_b200 import kda
     from linear_attention_recurrence_11_b200.inputs import WORKLOADS, workload_inputs
@@ -437,19 +513,21 @@ def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):
     w = WORKLOADS["decode_n256_h96_d128"]
     if args.decode_requests != w.B:
         w = dataclasses.replace(w, B=args.decode_requests)
+    steps = steps or w.decode_steps
     S = workload_inputs(w, device=device, step=0)["S0"]
+    warm = max(3, args.warmup)
     sets = []
-    for s in range(8):
+    for s in range(warm + steps):
         d = workload_inputs(w, device=device, step=s)
         sets.append({k: d[k][:, 0].contiguous() for k in ("q", "k", "v", "g", "beta")})
     o = torch.empty((w.B, w.H, w.dv), dtype=sets[0]["k"].dtype, device=device)
     stream = torch.cuda.current_stream(device)
 
     def step(i):
-        d = sets[i % 8]
+        d = sets[i]
         kda.kda_decode_step(d["q"], d["k"], d["v"], d["g"], d["beta"], S, o)
 
-    for i in range(max(3, args.warmup)):
+    for i in range(warm):
         step(i)
     torch.cuda.synchronize(device)
     barrier()
@@ -457,11 +535,12 @@ def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):
     with ClockSampler(device.index) as clk:
         a.record(stream)
         for i in range(steps):
-            step(i)
+            step(warm + i)
         b.record(stream)
         torch.cuda.synchronize(device)
     ms = max_ranks(a.elapsed_time(b)) / steps
     elem = sets[0]["k"].element_size()
+    del sets
     alg_bytes, _ = decode_algorithmic(w.B, w.H, w.dk, w.dv, elem)
     gbs = alg_bytes / (ms / 1e3) / 1e9
     res = {"metric": f"KDA decode step GB/s ({w.B} req x {w.H} heads, fp32 state)",
@@ -577,6 +656,34 @@ def cpu_baseline_prefill(inp, w, seconds):
             "sample": f"{heads} of {w.H} heads x {T} tokens of {w.name}, sequential fp64 oracle, "
                       f"one thread; tokens/s = token-heads/s / {w.H}",
             "host_cpus": os.cpu_count(), "seconds": el}
+
+
+def cpu_baseline_all_cores(inp, w):
+    """The same oracle over all host cores: one whole head per task on a thread
+    pool (the oracle is a C library called through ctypes, which releases the
+    GIL, so the heads run in parallel), every head of the workload at up to 8192
+    tokens; the wall time includes each head's copy to fp64."""
+    import oracle
+    from concurrent.futures import ThreadPoolExecutor
+    from linear_attention_recurrence_11_b200.inputs import to_f64
+    oracle.build()
+    T = min(w.total_tokens if w.seqlens else w.T, 8192)
+    host = {x: inp[x][0, :T].cpu() for x in ("q", "k", "v", "g", "beta")}
+    cores = os.cpu_count() or 1
+
+    def one(h):
+        a = [to_f64(host[x][:, h]) for x in ("q", "k", "v", "g", "beta")]
+        oracle.forward(*a)
+
+    t = time.perf_counter()
+    with ThreadPoolExecutor(max_workers=cores) as ex:
+        list(ex.map(one, range(w.H)))
+    el = time.perf_counter() - t
+    return {"value": T * w.H / w.H / el, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "label": "CPU baseline, all cores",
+            "sample": f"all {w.H} heads x {T} tokens of {w.name}, sequential fp64 oracle per head, "
+                      f"{cores} threads (one head per task); tokens/s = token-heads/s / {w.H}",
+            "seconds": el}
 
 
 def run_reference(args, rank, world):

@@ -75,25 +75,32 @@ typedef enum { KDA_FUSE_NORM_QK = 1, KDA_FUSE_GATE_LOGITS = 2 } kda_fuse;
 
 /* Which prefill kernels kda_forward_ex runs. The tensor cores cover bf16,
  * dk = dv = 128, chunk = 64; the SIMT kernel covers every supported shape.
- * On the tensor cores there are two forms of the same computation:
- *  - split: a chunk-parallel kernel computes, for every (sequence, head,
- *    chunk), the part of the chunk that does not depend on the incoming state
- *    (decayed Grams, triangular solve, W, Ut; "Exercices", Q21: a chunk's KCP
- *    pair depends on its own inputs only) into the workspace, then a second
- *    kernel carries each unit's state across its chunks. Needs the workspace
- *    kda_forward_workspace_size reports (about 72.5 KiB per chunk per head).
- *  - single: one kernel per (sequence, head) computes everything chunk after
- *    chunk; it needs no workspace beyond the packed-batch schedule.
- * AUTO and TC run the split form when the workspace passed holds it and the
- * single form otherwise (TC returns KDA_ERR_UNSUPPORTED off the tensor-core
- * shapes, AUTO falls back to SIMT); TC_SINGLE and TC_SPLIT force one form
- * (TC_SPLIT returns KDA_ERR_WORKSPACE if the workspace is too small). */
+ * On the tensor cores there are three forms of the same computation. The part
+ * of a chunk that does not depend on the state it receives (decayed Grams,
+ * triangular solve, W, Ut; "Exercices", Q21: a chunk's KCP pair depends on
+ * its own inputs only) is either computed on each unit's serial path or by
+ * chunk-parallel producers that hand a 73 KiB record per chunk to the state
+ * chains:
+ *  - single (TC_SINGLE): one kernel per (sequence, head) computes everything
+ *    chunk after chunk; no workspace beyond the packed-batch schedule.
+ *  - split (TC_SPLIT): a chunk-parallel kernel writes every chunk's record to
+ *    the workspace, then a second kernel carries each unit's state across its
+ *    chunks (73 KiB of workspace per chunk per head).
+ *  - pipe (TC_PIPE): one cooperative launch runs the chains and the producers
+ *    at once, the records passing through a ring of 4 per unit; for at most
+ *    two thirds of twice the SM count of units (197 on 148 SMs), else
+ *    KDA_ERR_UNSUPPORTED. Workspace: about 292 KiB per unit.
+ * AUTO and TC run the split form when the workspace holds it, then the pipe
+ * form when its ring fits, else the single form (TC returns
+ * KDA_ERR_UNSUPPORTED off the tensor-core shapes, AUTO falls back to SIMT);
+ * a forced form returns KDA_ERR_WORKSPACE if the workspace is too small. */
 typedef enum {
     KDA_PATH_AUTO = 0,
     KDA_PATH_SIMT = 1,
     KDA_PATH_TC = 2,
     KDA_PATH_TC_SINGLE = 3,
-    KDA_PATH_TC_SPLIT = 4
+    KDA_PATH_TC_SPLIT = 4,
+    KDA_PATH_TC_PIPE = 5
 } kda_path;
 
 /* Human-readable name of a status code (static string, never NULL). */
@@ -102,17 +109,21 @@ const char *kda_status_string(int status);
 /* ABI version of this header (bumped when a signature changes). */
 int kda_abi_version(void);
 
+/* Name of the CUDA error behind the last KDA_ERR_CUDA this thread received
+ * from an entry point (a static string, "none" if there was none). */
+const char *kda_last_cuda_error(void);
+
 /*
  * Bytes of device workspace kda_forward needs for these sizes (0 if none):
  * the scratch of the chunked prefill of "Exercices", Q7 with the KCP
  * composition of Q21-Q22. num_seqs is the number of packed sequences when
  * cu_seqlens is used, else B (B == 1 with num_seqs > 1 means packed
- * sequences). On the tensor-core shapes it is the split form's per-chunk
- * records (74,240 bytes per chunk per head; for packed batches counted for
- * at most T / 64 + num_seqs chunks per head) plus, for packed batches, the
- * sequences' chunk offsets and a longest-first schedule of up to 2048
- * sequences. A smaller workspace still works on the tensor cores (the single
- * form, see kda_path). The workspace is scratch: its contents on entry do not
+ * sequences). On the tensor-core shapes it covers every tensor-core form
+ * (kda_path): the split form's per-chunk records (74,752 bytes per chunk per
+ * head; for packed batches counted for at most T / 64 + num_seqs chunks per
+ * head, plus the sequences' chunk offsets and a longest-first schedule of up
+ * to 2048 sequences), or the pipe form's ring where that is larger. A smaller
+ * workspace still works on the tensor cores (see kda_path). The workspace is scratch: its contents on entry do not
  * matter and it may be reused after the stream reaches the end of the call.
  * Returns (size_t)-1 if the sizes are invalid.
  */

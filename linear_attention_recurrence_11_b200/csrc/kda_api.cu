@@ -17,13 +17,14 @@ int check_prefill_sizes(int B, int T, int H, int dk, int dv, int chunk, int dtyp
     if (!dtype_ok(dtype)) return KDA_ERR_INVALID_ARG;
     if (!head_dim_ok(dk) || !head_dim_ok(dv) || !chunk_ok(chunk)) return KDA_ERR_UNSUPPORTED;
     if (has_cu && (B != 1 || num_seqs <= 0)) return KDA_ERR_INVALID_ARG;
-    if (path < KDA_PATH_AUTO || path > KDA_PATH_TC_SPLIT) return KDA_ERR_INVALID_ARG;
+    if (path < KDA_PATH_AUTO || path > KDA_PATH_TC_PIPE) return KDA_ERR_INVALID_ARG;
     if (path >= KDA_PATH_TC && !kda::prefill_tc_supported(dk, dv, chunk, dtype)) return KDA_ERR_UNSUPPORTED;
     // the kernels index tokens with size_t and units with 32-bit grid indices
     const size_t units = (size_t)(has_cu ? num_seqs : B) * (size_t)H;
     if (units * (size_t)(dv / 32) > 0x7fffffffu) return KDA_ERR_UNSUPPORTED;
     a->B = B; a->T = T; a->H = H; a->dk = dk; a->dv = dv; a->chunk = chunk; a->dtype = dtype;
     a->num_units = has_cu ? num_seqs : B;
+    if (path == KDA_PATH_TC_PIPE && !kda::prefill_pipe_supported(*a)) return KDA_ERR_UNSUPPORTED;
     return KDA_OK;
 }
 
@@ -36,21 +37,26 @@ bool use_tc(const kda::PrefillArgs &a, int path) {
     return kda::prefill_tc_supported(a.dk, a.dv, a.chunk, a.dtype);
 }
 
-// The prefill form a call runs (kda_path): the SIMT kernel, the single tensor-core kernel, or
-// the split tensor-core form, which AUTO and TC take when the workspace holds its records.
-enum class Form { Simt, Single, Split };
+// The prefill form a call runs (kda_path): the SIMT kernel or one of the three tensor-core
+// forms. AUTO and TC take the two-kernel split form when the workspace holds its records, then
+// the one-launch form when its ring fits, then the single kernel.
+enum class Form { Simt, Single, Split, Pipe };
 Form choose_form(const kda::PrefillArgs &a, int path, size_t workspace_bytes, bool workspace_known) {
     if (!use_tc(a, path)) return Form::Simt;
     if (path == KDA_PATH_TC_SINGLE) return Form::Single;
     if (path == KDA_PATH_TC_SPLIT) return Form::Split;
+    if (path == KDA_PATH_TC_PIPE) return Form::Pipe;
     if (!workspace_known) return Form::Split;  // size queries assume the reported workspace
-    return workspace_bytes >= kda::prefill_split_workspace(a) ? Form::Split : Form::Single;
+    if (workspace_bytes >= kda::prefill_split_workspace(a)) return Form::Split;
+    if (kda::prefill_pipe_supported(a) && workspace_bytes >= kda::prefill_pipe_workspace(a)) return Form::Pipe;
+    return Form::Single;
 }
 
 size_t form_workspace(const kda::PrefillArgs &a, Form f) {
     switch (f) {
         case Form::Simt: return kda::prefill_simt_workspace(a);
         case Form::Single: return kda::prefill_tc_workspace(a);
+        case Form::Pipe: return kda::prefill_pipe_workspace(a);
         default: return kda::prefill_split_workspace(a);
     }
 }
@@ -59,6 +65,7 @@ cudaError_t form_launch(const kda::PrefillArgs &a, Form f) {
     switch (f) {
         case Form::Simt: return kda::launch_prefill_simt(a);
         case Form::Single: return kda::launch_prefill_tc(a);
+        case Form::Pipe: return kda::launch_prefill_pipe(a);
         default: return kda::launch_prefill_split(a);
     }
 }
@@ -66,6 +73,14 @@ cudaError_t form_launch(const kda::PrefillArgs &a, Form f) {
 }  // namespace
 
 namespace kda {
+namespace {
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+}
+int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return KDA_OK;
+    g_last_cuda_error = e;
+    return KDA_ERR_CUDA;
+}
 int validate_prefill(int B, int T, int H, int dk, int dv, int chunk, int dtype, int path) {
     PrefillArgs a{};
     return check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, false, 0, path, &a);
@@ -90,6 +105,11 @@ const char *kda_status_string(int status) {
 
 int kda_abi_version(void) { return 2; }
 
+const char *kda_last_cuda_error(void) {
+    const cudaError_t e = kda::g_last_cuda_error;
+    return e == cudaSuccess ? "none" : cudaGetErrorName(e);
+}
+
 size_t kda_forward_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int num_seqs,
                                   int dtype) {
     kda::PrefillArgs a{};
@@ -102,8 +122,10 @@ size_t kda_forward_workspace_size(int B, int T, int H, int dk, int dv, int chunk
     if (kda::prefill_tc_supported(dk, dv, chunk, dtype)) {
         const size_t t = kda::prefill_tc_workspace(a);
         const size_t sp = kda::prefill_split_workspace(a);
+        const size_t pi = kda::prefill_pipe_supported(a) ? kda::prefill_pipe_workspace(a) : 0;
         ws = t > ws ? t : ws;
         ws = sp > ws ? sp : ws;
+        ws = pi > ws ? pi : ws;
     }
     return ws;
 }
@@ -117,6 +139,7 @@ int kda_forward_launches(int B, int T, int H, int dk, int dv, int chunk, int dty
     switch (choose_form(a, path, 0, false)) {
         case Form::Simt: return kda::prefill_simt_launches(a);
         case Form::Single: return kda::prefill_tc_launches(a);
+        case Form::Pipe: return kda::prefill_pipe_launches(a);
         default: return kda::prefill_split_launches(a);
     }
 }
@@ -141,7 +164,7 @@ int kda_forward_ex(const void *q, const void *k, const void *v, const void *g, c
     const size_t need = form_workspace(a, f);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
     const cudaError_t e = form_launch(a, f);
-    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return kda::cuda_status(e);
 }
 
 int kda_forward_snapshots(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -162,10 +185,10 @@ int kda_forward_snapshots(const void *q, const void *k, const void *v, const voi
     a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.dev_status = dev_status;
     a.stream = static_cast<cudaStream_t>(stream);
     a.S_snap = S_snap; a.snap_every = T / snap_every > 0 ? snap_every : 0;
-    if (path == KDA_PATH_TC_SPLIT) return KDA_ERR_UNSUPPORTED;  // snapshots come from the single form
+    if (path == KDA_PATH_TC_SPLIT || path == KDA_PATH_TC_PIPE) return KDA_ERR_UNSUPPORTED;  // single form only
     const bool tc = use_tc(a, path);
     const cudaError_t e = tc ? kda::launch_prefill_tc(a) : kda::launch_prefill_simt(a);
-    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return kda::cuda_status(e);
 }
 
 int kda_forward_fused(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -185,7 +208,8 @@ int kda_forward_fused(const void *q, const void *k, const void *v, const void *g
     a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.dev_status = dev_status;
     a.stream = static_cast<cudaStream_t>(stream);
     a.fuse = flags;
-    if (flags && path == KDA_PATH_TC_SPLIT) return KDA_ERR_UNSUPPORTED;  // fused pre-operations: single form
+    if (flags && (path == KDA_PATH_TC_SPLIT || path == KDA_PATH_TC_PIPE))
+        return KDA_ERR_UNSUPPORTED;  // fused pre-operations: single form
     if (!flags)
         return kda_forward_ex(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, dtype, cu_seqlens, num_seqs,
                               workspace, workspace_bytes, dev_status, stream, path);
@@ -193,7 +217,7 @@ int kda_forward_fused(const void *q, const void *k, const void *v, const void *g
     const size_t need = tc ? kda::prefill_tc_workspace(a) : kda::prefill_simt_workspace(a);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
     const cudaError_t e = tc ? kda::launch_prefill_tc(a) : kda::launch_prefill_simt(a);
-    return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return kda::cuda_status(e);
 }
 
 int kda_forward(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -264,7 +288,7 @@ int kda_forward_segmented(const void *q, const void *k, const void *v, const voi
     s.workspace = workspace; s.workspace_bytes = workspace_bytes; s.dev_status = dev_status;
     s.stream = static_cast<cudaStream_t>(stream);
     if (workspace == nullptr || workspace_bytes < kda::segmented_workspace(s)) return KDA_ERR_WORKSPACE;
-    return kda::launch_segmented(s, tc_pair, tc_state) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return kda::cuda_status(kda::launch_segmented(s, tc_pair, tc_state));
 }
 
 int kda_decode_step_fused(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -278,7 +302,7 @@ int kda_decode_step_fused(const void *q, const void *k, const void *v, const voi
         if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
     kda::DecodeArgs a{q, k, v, g, beta, S, o, N, H, dk, dv, dtype, static_cast<cudaStream_t>(stream)};
     a.fuse = flags;
-    return kda::launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return kda::cuda_status(kda::launch_decode(a));
 }
 
 int kda_decode_step(const void *q, const void *k, const void *v, const void *g, const void *beta,
@@ -290,7 +314,7 @@ int kda_decode_step(const void *q, const void *k, const void *v, const void *g, 
     for (const void *p : {q, k, v, g, beta, (const void *)S, (const void *)o})
         if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
     kda::DecodeArgs a{q, k, v, g, beta, S, o, N, H, dk, dv, dtype, static_cast<cudaStream_t>(stream)};
-    return kda::launch_decode(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return kda::cuda_status(kda::launch_decode(a));
 }
 
 int kda_segment_pair(const void *q, const void *k, const void *v, const void *g, const void *beta, float *M,
@@ -309,7 +333,7 @@ int kda_segment_pair(const void *q, const void *k, const void *v, const void *g,
     s.dev_status = dev_status; s.stream = static_cast<cudaStream_t>(stream);
     const bool tc_pair = path != KDA_PATH_SIMT && kda::prefill_tc_supported(dk, dk, chunk, dtype);
     const bool tc_state = path != KDA_PATH_SIMT && kda::prefill_tc_supported(dk, dv, chunk, dtype);
-    return kda::launch_segment_pair(s, M, Z, tc_pair, tc_state) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return kda::cuda_status(kda::launch_segment_pair(s, M, Z, tc_pair, tc_state));
 }
 
 int kda_kcp_scan(const float *S0, const float *M, const float *Z, float *S_in, float *S_T, int B, int P, int H,
@@ -323,7 +347,7 @@ int kda_kcp_scan(const float *S0, const float *M, const float *Z, float *S_in, f
     kda::SegmentedArgs s{};
     s.S0 = S0; s.ST = S_T; s.B = B; s.P = P; s.H = H; s.dk = dk; s.dv = dv;
     s.stream = static_cast<cudaStream_t>(stream);
-    return kda::launch_kcp_scan(s, M, Z, S_in) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return kda::cuda_status(kda::launch_kcp_scan(s, M, Z, S_in));
 }
 
 int kda_decode_multi(const void *q, const void *k, const void *v, const void *g, const void *beta, float *S,
@@ -339,7 +363,7 @@ int kda_decode_multi(const void *q, const void *k, const void *v, const void *g,
         if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
     kda::MultiDecodeArgs a{q, k, v, g, beta, S, o, n_accept, dev_status, N, T, H, dk, dv, dtype,
                            static_cast<cudaStream_t>(stream)};
-    return kda::launch_decode_multi(a) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    return kda::cuda_status(kda::launch_decode_multi(a));
 }
 
 }  // extern "C"

@@ -112,9 +112,16 @@ int prefill_tc_launches(const PrefillArgs &a);
 cudaError_t launch_prefill_split(const PrefillArgs &a);
 size_t prefill_split_workspace(const PrefillArgs &a);
 int prefill_split_launches(const PrefillArgs &a);
+// the one-launch form: chains and record producers in one cooperative launch, records in a ring
+bool prefill_pipe_supported(const PrefillArgs &a);
+cudaError_t launch_prefill_pipe(const PrefillArgs &a);
+size_t prefill_pipe_workspace(const PrefillArgs &a);
+int prefill_pipe_launches(const PrefillArgs &a);
 
 cudaError_t launch_decode(const DecodeArgs &a);
 cudaError_t launch_decode_multi(const MultiDecodeArgs &a);
+// KDA_OK for cudaSuccess; otherwise KDA_ERR_CUDA, the error kept for kda_last_cuda_error
+int cuda_status(cudaError_t e);
 // KDA_OK, or the status kda_forward_ex returns for these sizes (dense batches)
 int validate_prefill(int B, int T, int H, int dk, int dv, int chunk, int dtype, int path);
 

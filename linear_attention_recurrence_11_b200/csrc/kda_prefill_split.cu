@@ -41,13 +41,21 @@ constexpr int NT = 256;
 constexpr uint32_t KB = 1024;
 
 // ------------------------------------------------ per-task record in the workspace
-constexpr uint32_t REC_WQ = 0;         // 32 KB [-W ; Gamma q], K-major, 128 rows x 128, K-blocks 16 KB apart
-constexpr uint32_t REC_KH = 32 * KB;   // 16 KB Kh = e^{G_C - G} k, MN-major [tok][dk], 64-channel blocks 8 KB apart
-constexpr uint32_t REC_UT = 48 * KB;   // 16 KB Ut (bf16), MN-major [tok][dv], N-blocks 8 KB apart
-constexpr uint32_t REC_P = 64 * KB;    // 8 KB  P (bf16, s <= r), K-major [r][s]
-constexpr uint32_t REC_GC = 72 * KB;   // 512 B Gamma_C (fp32, one per channel)
-constexpr uint32_t REC_BYTES = 72 * KB + 512;
-static_assert(REC_BYTES % 128 == 0, "records keep 128-byte alignment");
+// Three contiguous pieces, each the image of the shared-memory tiles its consumer feeds to
+// the tensor cores, in the order the state chain needs them: A = [-W ; Gamma q] and Gamma_C
+// (the state product and the state's decay), B = Ut and P (the U readout and the output
+// product), C = Kh (the state update).
+constexpr uint32_t REC_WQ = 0;          // 32 KB [-W ; Gamma q], K-major, 128 rows x 128, K-blocks 16 KB apart
+constexpr uint32_t REC_GC = 32 * KB;    // 512 B Gamma_C (fp32, one per channel)
+constexpr uint32_t REC_UT = 33 * KB;    // 16 KB Ut (bf16), MN-major [tok][dv], N-blocks 8 KB apart
+constexpr uint32_t REC_P = 49 * KB;     // 8 KB  P (bf16, s <= r), K-major [r][s]
+constexpr uint32_t REC_KH = 57 * KB;    // 16 KB Kh = e^{G_C - G} k, MN-major [tok][dk], 64-channel blocks 8 KB apart
+constexpr uint32_t REC_BYTES = 73 * KB;
+constexpr uint32_t REC_A_BYTES = 32 * KB + 512;  // piece A: [REC_WQ, REC_GC + 512)
+constexpr uint32_t REC_B_BYTES = 24 * KB;        // piece B: [REC_UT, REC_KH)
+constexpr uint32_t REC_C_BYTES = 16 * KB;        // piece C: [REC_KH, REC_BYTES)
+static_assert(REC_UT + REC_B_BYTES == REC_KH && REC_KH + REC_C_BYTES == REC_BYTES, "record pieces");
+static_assert(REC_UT % 1024 == 0 && REC_P % 1024 == 0 && REC_KH % 1024 == 0, "tiles stay 1 KB aligned");
 
 // ------------------------------------------------------------ prep smem layout
 constexpr uint32_t P_L0 = 0;          // 32 KB k (rows 0..63) and q (rows 64..127) tiles, the Gram left operand L0 in place
@@ -78,7 +86,7 @@ static_assert(2 * (P_SMEM_BYTES + 1024) <= 233472, "two prep CTAs per SM");
 constexpr uint32_t P_TM_W = 0, P_TM_UT = 128, P_TM_COLS = 256;  // the Gram uses columns 0..63 first
 
 // ----------------------------------------------------------- chain smem layout
-constexpr uint32_t C_RECSTRIDE = 73 * KB;             // >= REC_BYTES, 1 KB aligned
+constexpr uint32_t C_RECSTRIDE = REC_BYTES;           // 1 KB aligned
 constexpr uint32_t C_SB = 2 * C_RECSTRIDE;            // 32 KB S (bf16), B operand MN-major [dk][dv], N-blocks 16 KB apart
 constexpr uint32_t C_MISC = C_SB + 32 * KB;
 constexpr uint32_t C_BAR = C_MISC;                    // 3 mbarriers
@@ -101,6 +109,8 @@ struct SplitParams {
 struct Task {
     long long t, tok0;
     int n, h, Lc;
+    int chain;      // ring-buffer form: the chain that consumes the record, and its index there
+    long long tau;
 };
 
 __device__ __forceinline__ Task task_at(const SplitParams &sp, long long t) {
@@ -174,13 +184,38 @@ __global__ void chunk_base_kernel(const int32_t *cu, int num, int32_t *base) {
 }
 
 // ======================================================================= prep
-__global__ void __launch_bounds__(NT, 2)
-kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
-                const SplitParams sp) {
+// Every task of the batch, strided over the grid; the record of task t is the t-th of the
+// workspace (the two-kernel form: the chains run after this kernel has finished).
+struct StaticTasks {
+    static constexpr bool kPublish = false;
+    const SplitParams *sp;
+    long long t, total;
+    __device__ bool first(Task &k) {
+        total = sp->chunk_base ? (long long)sp->chunk_base[sp->a.num_units] * sp->a.H : sp->tasks;
+        t = blockIdx.x;
+        if (t >= total) return false;
+        k = task_at(*sp, t);
+        return true;
+    }
+    __device__ bool next(Task &k) {
+        t += gridDim.x;
+        if (t >= total) return false;
+        k = task_at(*sp, t);
+        return true;
+    }
+    __device__ uint8_t *record(const Task &k) const { return sp->rec + (size_t)k.t * REC_BYTES; }
+    __device__ bool acquire(const Task &) { return true; }
+    __device__ void release(const Task &) {}
+};
+
+// The persistent loop of a record-producing CTA over the tasks its source hands out.
+// Src::acquire (thread 0) returns once the task's record may be written, before its first
+// store; Src::release (thread 0) publishes a record whose stores have completed (kPublish).
+template <class Src>
+__device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
+                                          const CUtensorMap &tm_g, const SplitParams &sp, Src &src, uint8_t *sm,
+                                          const Group &grp) {
     const PrefillArgs &p = sp.a;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
     uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + P_BAR);  // k, q, g of a task
     uint64_t *bar_v = bar_ld + 1;
@@ -193,11 +228,10 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float *TF = reinterpret_cast<float *>(sm + P_TF);
     float *XS = reinterpret_cast<float *>(sm + P_XS);
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = grp.tid, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, half = warp >> 2;
     const size_t H = (size_t)p.H;
     const __nv_bfloat16 *beta = static_cast<const __nv_bfloat16 *>(p.beta);
-    const long long total = sp.chunk_base ? (long long)sp.chunk_base[p.num_units] * p.H : sp.tasks;
 
     if (tid == 0) {
         mbar_init(bar_ld, 1);
@@ -212,9 +246,9 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
     if (warp == 0) {
         tmem_alloc(s_tmem, P_TM_COLS);
-        tmem_relinquish();
+        if (grp.relinquish) tmem_relinquish();
     }
-    __syncthreads();
+    grp.sync();
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
     const uint32_t tlane = (uint32_t)(32 * quarter) << 16;
@@ -232,10 +266,10 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     };
     const bool has_v = p.v != nullptr;  // all-zero values (a segment's transition): no v, Ut = 0
 
-    long long t = blockIdx.x;
-    bool have = t < total;
     Task cur{};
-    if (have) cur = task_at(sp, t);
+    bool have = src.first(cur);
+    Task pend{};  // a record whose stores were issued and that is not yet published
+    bool has_pend = false;
     // unwinding state (thread 0): armed transaction counts and a commit whose wait ran out
     bool ld_armed = false, v_armed = false;
     uint64_t *mma_bar = nullptr;
@@ -263,18 +297,16 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     constexpr uint32_t idKM = idesc_bf16_f32(128, 128, 0, 1);
 
     while (have) {
-        const long long tn = t + gridDim.x;
-        const bool more = tn < total;
         Task nxt{};
-        if (more) nxt = task_at(sp, tn);
-        uint8_t *rec = sp.rec + (size_t)cur.t * REC_BYTES;
+        const bool more = src.next(nxt);
+        uint8_t *rec = src.record(cur);
         const int Lc = cur.Lc;
 
         // ---- this task's k, q, g
         {
             const bool ok = mbar_wait_bounded(bar_ld, ld_phase, kWaitCycles);
             if (ok) { ld_phase ^= 1u; ld_armed = false; }
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
+            if (grp.sync_or(!ok)) { aborted = true; break; }
         }
         __nv_bfloat16 bnext = __float2bfloat16(0.f);
         if (tid < C) {
@@ -322,8 +354,20 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int e = 0; e < 4; ++e) sD[ti * D + c0 + e] = gl[HR - 1][e];
             }
         }
-        if (tid == 0) bulk_wait_read_all();  // the previous task's record stores have read their staging
-        __syncthreads();
+        // the previous task's record stores have read their staging (and, where records are
+        // published, completed: then that record is published); this task's record may be written
+        bool slot_ok = true;
+        if (tid == 0) {
+            if (Src::kPublish) {
+                bulk_wait_all();
+                if (has_pend) src.release(pend);
+                has_pend = false;
+            } else {
+                bulk_wait_read_all();
+            }
+            slot_ok = src.acquire(cur);
+        }
+        if (grp.sync_or(!slot_ok)) { aborted = true; break; }
         if (tid == 0 && has_v) {  // g consumed: v lands in its tile
             mbar_arrive_expect_tx(bar_v, 16 * KB);
             issue_v(cur);
@@ -416,8 +460,9 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 *reinterpret_cast<uint2 *>(gkrow + off_r) = pk4(kf[0] * pg[0], kf[1] * pg[1], kf[2] * pg[2], kf[3] * pg[3]);
             }
         }
+        if (Src::kPublish) __threadfence();  // this thread's record stores before the publication
         fence_proxy_async_smem();
-        __syncthreads();
+        grp.sync();
 
         // ---- Gram MMAs: column block j -> TMEM columns 32j..32j+31, issued by lane 0 of warp j
         if (lane == 0 && warp < 2) {
@@ -433,7 +478,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!ok) { mma_bar = bar_gram; mma_bar_phase = gram_phase; }
             gram_phase ^= 1u;
             tc_fence_after();
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
+            if (grp.sync_or(!ok)) { aborted = true; break; }
         }
 
         // ---- Gram readout -> A (fp32, strictly lower, times beta_r), P (bf16, lower) staging.
@@ -474,7 +519,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        grp.sync();
         if (tid == 0) {
             bulk_store(rec + REC_P, sm + P_PST, 8 * KB);
             bulk_commit();
@@ -507,8 +552,8 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 for (int rr = 0; rr < 16; ++rr) TF[(o0 + rr) * LDT + o0 + 16 + cc] = 0.f;
             }
         }
-        __syncthreads();
-        tri_inverse_offdiag(AF, TF, XS, tid);
+        grp.sync();
+        tri_inverse_offdiag(AF, TF, XS, tid, grp.id);
         // T Diag(beta) -> bf16 A operand, rows 0..63 (rows 64..127 of the product are never read)
         {
             const int r = tid >> 3, pc = (tid & 7) * 8;
@@ -536,7 +581,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (has_v) {
             const bool ok = mbar_wait_bounded(bar_v, v_phase, kWaitCycles);
             if (ok) { v_phase ^= 1u; v_armed = false; }
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
+            if (grp.sync_or(!ok)) { aborted = true; break; }
             if (Lc < C) {
                 for (int idx = tid; idx < (C - Lc) * 16; idx += NT) {
                     const int r = Lc + idx / 16, q16 = idx % 16;
@@ -549,7 +594,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 *reinterpret_cast<uint4 *>(sm + P_GV + 16 * idx) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
-        __syncthreads();
+        grp.sync();
 
         // ---- [W | Ut] = T Diag(beta) [Gamma K | V]
         if (tid == 0) {
@@ -566,7 +611,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (!ok) { mma_bar = bar_mma; mma_bar_phase = mma_phase; }
             mma_phase ^= 1u;
             tc_fence_after();
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
+            if (grp.sync_or(!ok)) { aborted = true; break; }
         }
         // the next task's k, q, g: L0 and the g / v tile are free
         if (more && tid == 0) {
@@ -604,19 +649,23 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        grp.sync();
         if (tid == 0) {
             bulk_store(rec + REC_WQ, sm + P_WST, 8 * KB);
             bulk_store(rec + REC_WQ + 16 * KB, sm + P_WST + 8 * KB, 8 * KB);
             bulk_store(rec + REC_UT, sm + P_UST, 16 * KB);
             bulk_commit();
         }
+        pend = cur;
+        has_pend = true;
         cur = nxt;
-        t = tn;
         have = more;
         bcur = bnext;
     }
-    if (tid == 0) bulk_wait_all();  // record stores complete (the direct stores are ordinary writes)
+    if (tid == 0) {
+        bulk_wait_all();  // record stores complete (the direct stores are ordinary writes)
+        if (Src::kPublish && has_pend && !aborted) src.release(pend);
+    }
     if (aborted && tid == 0) {
         // unwind with nothing in flight: armed copies complete (bounded), a timed-out commit is
         // waited for (bounded) before TMEM is freed
@@ -626,11 +675,21 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (mma_bar) mbar_wait_bounded(mma_bar, mma_bar_phase, kWaitCycles);
     }
     tc_fence_before();
-    __syncthreads();
+    grp.sync();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, P_TM_COLS);
     }
+}
+
+__global__ void __launch_bounds__(NT, 2)
+kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                const SplitParams sp) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    StaticTasks src{&sp, 0, 0};
+    prep_loop(tm_q, tm_k, tm_v, tm_g, sp, src, sm, Group{(int)threadIdx.x, 0u, true});
 }
 
 // ====================================================================== chain
@@ -917,6 +976,466 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
     }
 }
 
+// ================================================= persistent pipeline (one launch)
+// With no more (sequence, head) units than a GPU-wide fraction of its CTA slots, one
+// cooperative launch runs both roles at once: CTA c < NC carries unit c's state chain, the
+// other CTAs produce records into a ring of R slots per chain. A record's slot is free once
+// its chain has copied all three pieces of the record R places before it into shared memory
+// (consumed[c]); a record is ready once its stores have completed (ready[c][slot] = tau + 1).
+// Both flags only grow, are written with release and read with acquire semantics at GPU
+// scope, and every wait is bounded. The producers take tasks in order of (record index, chain),
+// so the earliest unfinished task can always proceed (its slot's earlier record belongs to an
+// older, finished task), and the chains consume in order: no cycle of waits can form. The
+// ring (NC x R x 73 KB, 28 MB for 96 units) stays in L2, so records do not cost HBM traffic.
+constexpr int kRingSlots = 4;
+
+// pipeline chain-role smem layout (the record pieces at their record offsets, then S bf16)
+constexpr uint32_t X_SB = REC_BYTES;                  // 32 KB S (bf16), B operand MN-major
+constexpr uint32_t X_BAR = X_SB + 32 * KB;            // 4 mbarriers (pieces A, B, C; MMA)
+constexpr uint32_t X_TMEMADDR = X_BAR + 64;
+constexpr uint32_t X_SMEM_USED = X_BAR + 128;
+constexpr uint32_t X_TM_U = 0, X_TM_S = 128, X_TM_COLS = 256;
+
+struct PipeParams {
+    SplitParams sp;
+    uint8_t *ring;        // [NC][R] records
+    unsigned *ready;      // [NC][R]: record tau of chain c is in slot tau % R once ready >= tau + 1
+    unsigned *consumed;   // [NC]: records 0 .. consumed - 1 of chain c have been copied out
+    int NC, nprep;        // chains (one per unit) and producing CTAs
+    long long ntasks;     // NC x the most chunks a unit can have
+};
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *ptr) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned *ptr, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+// Bounded wait until a monotonic counter reaches `target`.
+__device__ __forceinline__ bool wait_counter(const unsigned *ptr, unsigned target, long long max_cycles) {
+    if (ld_acquire_gpu(ptr) >= target) return true;
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(ptr) < target) {
+        if (clock64() - t0 > max_cycles) return false;
+        __nanosleep(100);
+    }
+    return true;
+}
+
+// Task t of the ring form: record tau = t / NC of chain c = t % NC (unit c: sequence c / H,
+// head c % H); tasks past the end of a unit's sequence are skipped.
+struct RingTasks {
+    static constexpr bool kPublish = true;
+    const PipeParams *pp;
+    long long t;     // the next candidate task
+    long long rank;  // this producer's index among the pp->nprep producers
+    __device__ bool valid(long long tt, Task &k) const {
+        const PrefillArgs &p = pp->sp.a;
+        const int c = (int)(tt % pp->NC);
+        const long long tau = tt / pp->NC;
+        const int n = c / p.H;
+        long long b, e;
+        if (p.cu_seqlens) {
+            b = p.cu_seqlens[n];
+            e = p.cu_seqlens[n + 1];
+        } else {
+            b = (long long)n * p.T;
+            e = b + p.T;
+        }
+        const long long tok0 = b + tau * C;
+        if (tok0 >= e) return false;
+        k.t = tt;
+        k.n = n;
+        k.h = c % p.H;
+        k.tok0 = tok0;
+        k.Lc = (int)((e - tok0) < C ? (e - tok0) : C);
+        k.chain = c;
+        k.tau = tau;
+        return true;
+    }
+    __device__ bool advance(Task &k) {
+        for (; t < pp->ntasks; t += pp->nprep)
+            if (valid(t, k)) return true;
+        return false;
+    }
+    __device__ bool first(Task &k) {
+        t = rank;
+        return advance(k);
+    }
+    __device__ bool next(Task &k) {
+        t += pp->nprep;
+        return advance(k);
+    }
+    __device__ uint8_t *record(const Task &k) const {
+        return pp->ring + ((size_t)k.chain * kRingSlots + (size_t)(k.tau % kRingSlots)) * REC_BYTES;
+    }
+    __device__ bool acquire(const Task &k) {
+        if (k.tau < kRingSlots) return true;
+        const bool ok = wait_counter(pp->consumed + k.chain, (unsigned)(k.tau - kRingSlots + 1), kWaitCycles);
+        fence_proxy_async_global();  // the slot's bulk stores come after the chain's copies out of it
+        return ok;
+    }
+    __device__ void release(const Task &k) {
+        fence_proxy_async_global();
+        __threadfence();
+        st_release_gpu(pp->ready + (size_t)k.chain * kRingSlots + (size_t)(k.tau % kRingSlots), (unsigned)(k.tau + 1));
+    }
+};
+
+// The state chain of unit c, its records read from the ring piece by piece as
+// their shared-memory tiles free up: A (state product operand, decay) once the state product
+// is done, B (Ut, P) once the output product is done, C (Kh) once the outputs staged over it
+// have left.
+__device__ __forceinline__ void chain_role(const PipeParams &pp, const CUtensorMap &tm_o, uint8_t *sm, const Group &grp,
+                                           int c) {
+    const PrefillArgs &p = pp.sp.a;
+    const uint32_t sbase = smem_u32(sm);
+    uint64_t *bar_a = reinterpret_cast<uint64_t *>(sm + X_BAR);
+    uint64_t *bar_b = bar_a + 1;
+    uint64_t *bar_c = bar_a + 2;
+    uint64_t *bar_mma = bar_a + 3;
+    uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + X_TMEMADDR);
+
+    const int tid = grp.tid, warp = tid >> 5, lane = tid & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int n = c / p.H, h = c % p.H;
+    const size_t H = (size_t)p.H;
+    long long t_begin, len;
+    if (p.cu_seqlens) {
+        t_begin = p.cu_seqlens[n];
+        len = (long long)p.cu_seqlens[n + 1] - t_begin;
+    } else {
+        t_begin = (long long)n * p.T;
+        len = p.T;
+    }
+    __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
+    const size_t state_base = ((size_t)n * H + h) * (size_t)(D * D);
+    const long long nchunks = (len + C - 1) / C;
+    const unsigned *ready = pp.ready + (size_t)c * kRingSlots;
+    auto slot = [&](long long tau) -> const uint8_t * {
+        return pp.ring + ((size_t)c * kRingSlots + (size_t)(tau % kRingSlots)) * REC_BYTES;
+    };
+
+    if (tid == 0) {
+        mbar_init(bar_a, 1);
+        mbar_init(bar_b, 1);
+        mbar_init(bar_c, 1);
+        mbar_init(bar_mma, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_o);
+    }
+    if (warp == 0) {
+        tmem_alloc(s_tmem, X_TM_COLS);
+        if (grp.relinquish) tmem_relinquish();
+    }
+    grp.sync();
+    // thread-0 state of the copies: armed bits (1 A, 2 B, 4 C) and the phase of each barrier
+    uint32_t armed = 0, ph_a = 0, ph_b = 0, ph_c = 0, mma_phase = 0;
+    bool flag_fail = false, aborted = false, mma_pending = false;
+    auto load_a = [&](long long tau) {
+        mbar_arrive_expect_tx(bar_a, REC_A_BYTES);
+        bulk_load(sm + REC_WQ, slot(tau) + REC_WQ, REC_A_BYTES, bar_a);
+        armed |= 1u;
+    };
+    auto load_b = [&](long long tau) {
+        mbar_arrive_expect_tx(bar_b, REC_B_BYTES);
+        bulk_load(sm + REC_UT, slot(tau) + REC_UT, REC_B_BYTES, bar_b);
+        armed |= 2u;
+    };
+    auto load_c = [&](long long tau) {
+        mbar_arrive_expect_tx(bar_c, REC_C_BYTES);
+        bulk_load(sm + REC_KH, slot(tau) + REC_KH, REC_C_BYTES, bar_c);
+        armed |= 4u;
+    };
+    if (tid == 0 && nchunks > 0) {
+        if (!wait_counter(&ready[0], 1u, kWaitCycles)) {
+            flag_fail = true;
+        } else {
+            fence_proxy_async_global();
+            load_a(0);
+            load_b(0);
+            load_c(0);
+        }
+    }
+    // incoming state -> TMEM (fp32, lane = dk row, column = dv) and its bf16 copy
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t tlane = (uint32_t)(32 * quarter) << 16;
+    const int si = 32 * quarter + lane;
+    {
+        uint8_t *sb = sm + X_SB + half * 16 * KB;
+#pragma unroll
+        for (int gq = 0; gq < 4; ++gq) {
+            float v[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int j = 64 * half + 16 * gq + e;
+                v[e] = p.S0 ? p.S0[state_base + (size_t)j * D + si] : 0.f;
+            }
+            tmem_st16(tmem + tlane + X_TM_S + 64u * half + 16u * gq, v);
+            uint4 w0, w1;
+            pack16(v, 1.f, w0, w1);
+            *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq)) = w0;
+            *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq + 8)) = w1;
+        }
+        tmem_wait_st();
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    if (grp.sync_or(flag_fail)) aborted = true;
+    tc_fence_after();
+
+    constexpr uint32_t idKM = idesc_bf16_f32(128, 128, 0, 1);
+    constexpr uint32_t idMM = idesc_bf16_f32(128, 128, 1, 1);
+    // bounded waits every thread takes part in; a failure anywhere (or a failed flag wait in
+    // thread 0) aborts the chain on every thread
+    auto wait_piece = [&](uint64_t *bar, uint32_t &ph, uint32_t bit) -> bool {
+        const bool ok = mbar_wait_bounded(bar, ph, kWaitCycles);
+        if (ok) { ph ^= 1u; armed &= ~bit; }
+        return grp.sync_or(!ok || flag_fail) == 0;
+    };
+    auto wait_mma = [&]() -> bool {
+        const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
+        if (ok) { mma_phase ^= 1u; mma_pending = false; }
+        tc_fence_after();
+        return grp.sync_or(!ok) == 0;
+    };
+    auto issue_u = [&]() {  // [U ; Gamma Q S] = [-W ; Gamma Q] S
+        tc_fence_after();
+        Opnd A{sbase + REC_WQ, false, 16 * KB, 0};
+        Opnd B{sbase + X_SB, true, 0, 16 * KB};
+        mma_chain<D / 16>(tmem + X_TM_U, A, B, idKM, false);
+        mma_commit(bar_mma);
+        mma_pending = true;
+    };
+
+    if (!aborted && nchunks > 0) {
+        if (!wait_piece(bar_a, ph_a, 1u)) aborted = true;
+        else if (tid == 0) issue_u();
+    }
+    for (long long tau = 0; tau < nchunks && !aborted; ++tau) {
+        const long long tok0 = t_begin + tau * C;
+        const int Lc = (int)((len - tau * C) < C ? (len - tau * C) : C);
+        const bool more = tau + 1 < nchunks;
+
+        // S <- Diag(Gamma_C) S while the state product runs
+        {
+            const float gam = reinterpret_cast<const float *>(sm + REC_GC)[si];
+#pragma unroll
+            for (int g2 = 0; g2 < 2; ++g2) {
+                float sv[2][16];
+#pragma unroll
+                for (int gq = 0; gq < 2; ++gq)
+                    tmem_ld16(tmem + tlane + X_TM_S + 64u * half + 32u * g2 + 16u * gq, sv[gq]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int gq = 0; gq < 2; ++gq) {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) sv[gq][e] *= gam;
+                    tmem_st16(tmem + tlane + X_TM_S + 64u * half + 32u * g2 + 16u * gq, sv[gq]);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+        }
+        if (!wait_mma()) { aborted = true; break; }
+        // piece A of the next record (the state product's operand and Gamma_C are consumed)
+        if (tid == 0 && more) {
+            if (!wait_counter(&ready[(tau + 1) % kRingSlots], (unsigned)(tau + 2), kWaitCycles)) {
+                flag_fail = true;
+            } else {
+                fence_proxy_async_global();
+                load_a(tau + 1);
+            }
+        }
+        if (!wait_piece(bar_b, ph_b, 2u)) { aborted = true; break; }
+
+        // U = Ut - W S (rows 0..63) -> bf16 B operand, written over the record's Ut tile
+        if (quarter < 2) {
+            const int r = 32 * quarter + lane;
+            uint8_t *ut = sm + REC_UT + half * 8 * KB;
+#pragma unroll
+            for (int g2 = 0; g2 < 2; ++g2) {
+            float v[2][16];
+#pragma unroll
+            for (int gq = 0; gq < 2; ++gq) tmem_ld16(tmem + tlane + X_TM_U + 64u * half + 32u * g2 + 16u * gq, v[gq]);
+            tmem_wait_ld();
+#pragma unroll
+            for (int gq = 0; gq < 2; ++gq) {
+#pragma unroll
+                for (int pc = 0; pc < 2; ++pc) {
+                    uint4 *sl = reinterpret_cast<uint4 *>(ut + sw128_offset(r, 32 * g2 + 16 * gq + 8 * pc));
+                    const uint4 w = *sl;
+                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                    float *x = v[gq] + 8 * pc;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ws[e]));
+                        x[2 * e] += f.x;
+                        x[2 * e + 1] += f.y;
+                    }
+                    uint4 o4;
+                    o4.x = pack_bf2(x[0], x[1]);
+                    o4.y = pack_bf2(x[2], x[3]);
+                    o4.z = pack_bf2(x[4], x[5]);
+                    o4.w = pack_bf2(x[6], x[7]);
+                    *sl = o4;
+                }
+            }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        if (!wait_piece(bar_c, ph_c, 4u)) { aborted = true; break; }
+        if (tid == 0) {
+            // every piece of record tau is in shared memory: its slot may be refilled
+            st_release_gpu(pp.consumed + c, (unsigned)(tau + 1));
+            tc_fence_after();
+            Opnd AK{sbase + REC_KH, true, 0, 8 * KB};
+            Opnd BU{sbase + REC_UT, true, 0, 8 * KB};
+            Opnd AP{sbase + REC_P - 8 * KB, false, 16 * KB, 0};
+            mma_chain<C / 16>(tmem + X_TM_S, AK, BU, idMM, true);
+            mma_chain<C / 16>(tmem + X_TM_U, AP, BU, idKM, true);
+            mma_commit(bar_mma);
+            mma_pending = true;
+        }
+        if (!wait_mma()) { aborted = true; break; }
+        if (tid == 0 && more && !flag_fail) load_b(tau + 1);  // Ut, U and P are consumed
+
+        // the bf16 copy of the updated state, and this chunk's outputs into registers, before
+        // the next state product overwrites the accumulator
+        // the bf16 copy of the updated state, and this chunk's outputs (rows 64..127 of the
+        // accumulator) out of TMEM before the next state product overwrites it: a full chunk is
+        // staged over the Kh tile (its product is done) for two tensor stores, the rows of a
+        // partial chunk are stored directly
+        {
+            uint8_t *sb = sm + X_SB + half * 16 * KB;
+#pragma unroll
+            for (int g2 = 0; g2 < 2; ++g2) {
+                float sv[2][16];
+#pragma unroll
+                for (int gq = 0; gq < 2; ++gq)
+                    tmem_ld16(tmem + tlane + X_TM_S + 64u * half + 32u * g2 + 16u * gq, sv[gq]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int gq = 0; gq < 2; ++gq) {
+                    uint4 w0, w1;
+                    pack16(sv[gq], 1.f, w0, w1);
+                    *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 32 * g2 + 16 * gq)) = w0;
+                    *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 32 * g2 + 16 * gq + 8)) = w1;
+                }
+            }
+        }
+        if (quarter >= 2 && p.o) {
+            const int r = 32 * quarter + lane - 64;
+#pragma unroll
+            for (int g2 = 0; g2 < 2; ++g2) {
+                float ov[2][16];
+#pragma unroll
+                for (int gq = 0; gq < 2; ++gq)
+                    tmem_ld16(tmem + tlane + X_TM_U + 64u * half + 32u * g2 + 16u * gq, ov[gq]);
+                tmem_wait_ld();
+                if (Lc == C) {
+                    uint8_t *base = sm + REC_KH + half * 8 * KB;
+#pragma unroll
+                    for (int gq = 0; gq < 2; ++gq) {
+                        uint4 w0, w1;
+                        pack16(ov[gq], 1.f, w0, w1);
+                        *reinterpret_cast<uint4 *>(base + sw128_offset(r, 32 * g2 + 16 * gq)) = w0;
+                        *reinterpret_cast<uint4 *>(base + sw128_offset(r, 32 * g2 + 16 * gq + 8)) = w1;
+                    }
+                } else if (r < Lc) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(tok0 + r) * H + h) * D + 64 * half + 32 * g2);
+#pragma unroll
+                    for (int gq = 0; gq < 2; ++gq) {
+                        uint4 w0, w1;
+                        pack16(ov[gq], 1.f, w0, w1);
+                        dst[2 * gq] = w0;
+                        dst[2 * gq + 1] = w1;
+                    }
+                }
+            }
+        }
+        fence_proxy_async_smem();
+        tc_fence_before();
+        grp.sync();
+        if (more) {
+            if (!wait_piece(bar_a, ph_a, 1u)) { aborted = true; break; }
+            if (tid == 0) issue_u();
+        }
+        if (tid == 0) {
+            if (Lc == C && p.o) {
+                tma_store_3d(&tm_o, sm + REC_KH, 0, h, (int)tok0);
+                tma_store_3d(&tm_o, sm + REC_KH + 8 * KB, 64, h, (int)tok0);
+                bulk_commit();
+            }
+            if (more && !flag_fail) {  // Kh of the next record, once the outputs have left its tile
+                bulk_wait_read_all();
+                load_c(tau + 1);
+            }
+        }
+    }
+    if (tid == 0) bulk_wait_all();
+
+    if (aborted) {
+        if (tid == 0) {
+            if (p.dev_status) atomicExch(p.dev_status, (int)KDA_ERR_TIMEOUT);
+            if (armed & 1u) mbar_wait_bounded(bar_a, ph_a, kWaitCycles);
+            if (armed & 2u) mbar_wait_bounded(bar_b, ph_b, kWaitCycles);
+            if (armed & 4u) mbar_wait_bounded(bar_c, ph_c, kWaitCycles);
+            if (mma_pending) mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
+        }
+    } else if (p.ST) {
+        tc_fence_after();
+#pragma unroll
+        for (int gq = 0; gq < 4; ++gq) {
+            float sv[16];
+            tmem_ld16(tmem + tlane + X_TM_S + 64u * half + 16u * gq, sv);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const int j = 64 * half + 16 * gq + e;
+                p.ST[state_base + (size_t)j * D + si] = sv[e];
+            }
+        }
+    }
+    tc_fence_before();
+    grp.sync();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, X_TM_COLS);
+    }
+}
+
+// One CTA of two 256-thread groups per SM, each with half of the shared memory and its own 256
+// TMEM columns (the occupancy calculator counts a CTA that allocates tensor memory once per
+// SM, so a cooperative launch of two CTAs per SM is refused; two groups in one CTA are not).
+// Group slot G = gi * gridDim.x + blockIdx.x: the first NC slots carry the chains (group 0 of
+// the first NC CTAs, one chain per SM while there are SMs), the others produce records.
+constexpr uint32_t PIPE_GROUP_BYTES = ((X_SMEM_USED > P_SMEM_USED ? X_SMEM_USED : P_SMEM_USED) + 1023) / 1024 * 1024;
+constexpr uint32_t PIPE_SMEM = 2 * PIPE_GROUP_BYTES + 1024;
+static_assert(PIPE_SMEM <= 232448, "two groups in one CTA");
+
+__global__ void __launch_bounds__(2 * NT, 1)
+kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                const __grid_constant__ CUtensorMap tm_o, const PipeParams pp) {
+    extern __shared__ uint8_t smem_raw[];
+    const int gi = (int)(threadIdx.x >> 8);
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u) + gi * PIPE_GROUP_BYTES;
+    const Group grp{(int)(threadIdx.x & (NT - 1)), 1u + (uint32_t)gi, false};
+    const int G = gi * (int)gridDim.x + (int)blockIdx.x;
+    if (G < pp.NC) {
+        chain_role(pp, tm_o, sm, grp, G);
+    } else {
+        RingTasks src{&pp, 0, G - pp.NC};
+        prep_loop(tm_q, tm_k, tm_v, tm_g, pp.sp, src, sm, grp);
+    }
+}
+
 int num_sms() {
     static int n = 0;
     if (n == 0) {
@@ -943,6 +1462,46 @@ long long split_tasks_bound(const PrefillArgs &a) {
     return (long long)a.B * ((a.T + C - 1) / C) * a.H;
 }
 
+// The one-launch form: one chain CTA per (sequence, head) unit, at most two thirds of the
+// grid's CTA slots (two per SM), so that at least a third produce records.
+long long pipe_units(const PrefillArgs &a) { return (long long)a.num_units * a.H; }
+bool pipe_ok(const PrefillArgs &a) {
+    const long long units = pipe_units(a);
+    return units >= 1 && 3 * units <= 2 * (2LL * num_sms());
+}
+size_t pipe_ring_bytes(const PrefillArgs &a) { return align256((size_t)pipe_units(a) * kRingSlots * REC_BYTES); }
+size_t pipe_flag_bytes(const PrefillArgs &a) {
+    return align256((size_t)pipe_units(a) * (kRingSlots + 1) * sizeof(unsigned));
+}
+
+cudaError_t launch_pipe(const PrefillArgs &a, const CUtensorMap &mq, const CUtensorMap &mk, const CUtensorMap &mv,
+                        const CUtensorMap &mg, const CUtensorMap &mo) {
+    const int grid = num_sms();  // one CTA of two groups per SM, all resident (cooperative launch)
+    int per_sm = 0;
+    cudaError_t e = cudaFuncSetAttribute(kda_pipe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)PIPE_SMEM);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kda_pipe_kernel, 2 * NT, PIPE_SMEM);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+    PipeParams pp{};
+    pp.sp.a = a;
+    if (!packed(a)) pp.sp.a.cu_seqlens = nullptr;
+    pp.sp.nch = (a.T + C - 1) / C;
+    uint8_t *ws = static_cast<uint8_t *>(a.workspace);
+    pp.ring = ws;
+    pp.ready = reinterpret_cast<unsigned *>(ws + pipe_ring_bytes(a));
+    pp.NC = (int)pipe_units(a);
+    pp.consumed = pp.ready + (size_t)pp.NC * kRingSlots;
+    pp.nprep = 2 * grid - pp.NC;
+    pp.ntasks = (long long)pp.NC * pp.sp.nch;  // a unit has at most ceil(T / C) chunks
+    e = cudaMemsetAsync(pp.ready, 0, pipe_flag_bytes(a), a.stream);
+    if (e != cudaSuccess) return e;
+    void *args[] = {const_cast<CUtensorMap *>(&mq), const_cast<CUtensorMap *>(&mk), const_cast<CUtensorMap *>(&mv),
+                    const_cast<CUtensorMap *>(&mg), const_cast<CUtensorMap *>(&mo), &pp};
+    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(kda_pipe_kernel), dim3(grid), dim3(2 * NT), args,
+                                       PIPE_SMEM, a.stream);
+}
+
 }  // namespace
 
 size_t prefill_split_workspace(const PrefillArgs &a) {
@@ -958,6 +1517,27 @@ int prefill_split_launches(const PrefillArgs &a) {
     return 2 + (packed(a) ? 1 + (seq_order_bytes(a.num_units) > 0 ? 1 : 0) : 0);
 }
 
+bool prefill_pipe_supported(const PrefillArgs &a) { return pipe_ok(a); }
+size_t prefill_pipe_workspace(const PrefillArgs &a) { return pipe_ring_bytes(a) + pipe_flag_bytes(a); }
+int prefill_pipe_launches(const PrefillArgs &a) {
+    if (a.num_units <= 0 || a.H <= 0) return 0;
+    const size_t tokens = a.cu_seqlens ? (size_t)a.T : (size_t)a.B * (size_t)a.T;
+    return tokens == 0 ? prefill_simt_launches(a) : 1;
+}
+
+cudaError_t launch_prefill_pipe(const PrefillArgs &a) {
+    if (a.num_units == 0) return cudaSuccess;
+    const size_t tokens = a.cu_seqlens ? (size_t)a.T : (size_t)a.B * (size_t)a.T;
+    if (tokens == 0) return launch_prefill_simt(a);
+    if (!pipe_ok(a)) return cudaErrorInvalidConfiguration;
+    CUtensorMap mq, mk, mv, mg, mo;
+    if (!make_map(&mq, a.q, tokens, a.H, 64, true) || !make_map(&mk, a.k, tokens, a.H, 64, true) ||
+        !make_map(&mv, a.v ? a.v : a.q, tokens, a.H, 64, true) || !make_map(&mg, a.g, tokens, a.H, 128, false) ||
+        !make_map(&mo, a.o ? a.o : a.q, tokens, a.H, 64, true))
+        return cudaErrorInvalidValue;
+    return launch_pipe(a, mq, mk, mv, mg, mo);
+}
+
 cudaError_t launch_prefill_split(const PrefillArgs &a) {
     if (a.num_units == 0) return cudaSuccess;
     const size_t tokens = a.cu_seqlens ? (size_t)a.T : (size_t)a.B * (size_t)a.T;
@@ -968,6 +1548,9 @@ cudaError_t launch_prefill_split(const PrefillArgs &a) {
         !make_map(&mo, a.o ? a.o : a.q, tokens, a.H, 64, true))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C_SMEM_BYTES);
     if (e != cudaSuccess) return e;

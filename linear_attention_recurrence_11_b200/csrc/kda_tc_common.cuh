@@ -45,6 +45,31 @@ __device__ __forceinline__ void pack16(const float *v, float scale, uint4 &w0, u
     w1.w = pack_bf2(scale * v[14], scale * v[15]);
 }
 
+// ------------------------------------------------------------- thread groups
+// A group of 256 threads that synchronise among themselves on named barrier `id` (0 is the
+// CTA barrier, the same as __syncthreads for a 256-thread CTA); a 512-thread CTA can run two
+// groups side by side on barriers 1 and 2.
+__device__ __forceinline__ void group_sync(uint32_t id) { asm volatile("bar.sync %0, 256;" ::"r"(id) : "memory"); }
+__device__ __forceinline__ bool group_sync_or(uint32_t id, bool pred) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.or.pred p, %2, 256, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(id)
+        : "memory");
+    return r != 0;
+}
+struct Group {
+    int tid;           // 0..255 within the group
+    uint32_t id;       // named barrier
+    bool relinquish;   // the group is the whole CTA: give up the TMEM allocation permit after allocating
+    __device__ __forceinline__ void sync() const { group_sync(id); }
+    __device__ __forceinline__ bool sync_or(bool p) const { return group_sync_or(id, p); }
+};
+
 // ------------------------------------------------------------- MMA issue
 // Operand tile in shared memory (128-byte swizzled rows): K-major tiles keep
 // 64-wide K blocks `kblk` bytes apart; MN-major tiles keep 64-wide M/N blocks
@@ -118,7 +143,8 @@ __device__ __forceinline__ void warp_store_16x8(float *Dm, int ldd, int dr, int 
 // i.e. the 2 x 2 block inverse applied twice; each product is a handful of
 // warp-level TF32 MMAs. A: 64 x LDA fp32 (strictly lower), T: 64 x LDT fp32,
 // XS: scratch of 32 x 36 fp32.
-__device__ __forceinline__ void tri_inverse_offdiag(const float *AF, float *TF, float *XS, int tid) {
+__device__ __forceinline__ void tri_inverse_offdiag(const float *AF, float *TF, float *XS, int tid,
+                                                    uint32_t bar_id = 0) {
     const int warp = tid >> 5;
     float c[4];
     // level 1: 2 blocks x 2 column tiles of 8 -> warps 0..3
@@ -128,20 +154,20 @@ __device__ __forceinline__ void tri_inverse_offdiag(const float *AF, float *TF, 
         warp_mma_16x8<16>(AF, LDA, i1, j1, TF, LDT, j1, j1 + 8 * nt, c);     // X = A_ij T_jj
         warp_store_16x8(XS, LDX, 16 * b, 8 * nt, c, 1.f);
     }
-    __syncthreads();
+    group_sync(bar_id);
     if (warp < 4) {
         warp_mma_16x8<16>(TF, LDT, i1, i1, XS, LDX, 16 * b, 8 * nt, c);       // T_ij = -T_ii X
         warp_store_16x8(TF, LDT, i1, j1 + 8 * nt, c, -1.f);
     }
-    __syncthreads();
+    group_sync(bar_id);
     // level 2: 2 row tiles x 4 column tiles -> warps 0..7
     const int mt = warp >> 2, n2 = warp & 3;
     warp_mma_16x8<32>(AF, LDA, 32 + 16 * mt, 0, TF, LDT, 0, 8 * n2, c);        // X = A21 T_lo
     warp_store_16x8(XS, LDX, 16 * mt, 8 * n2, c, 1.f);
-    __syncthreads();
+    group_sync(bar_id);
     warp_mma_16x8<32>(TF, LDT, 32 + 16 * mt, 32, XS, LDX, 0, 8 * n2, c);       // T21 = -T_hi X
     warp_store_16x8(TF, LDT, 32 + 16 * mt, 8 * n2, c, -1.f);
-    __syncthreads();
+    group_sync(bar_id);
 }
 
 // ------------------------------------------------------------------ host side

@@ -26,6 +26,7 @@ _vp, _i, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 _lib.kda_status_string.argtypes = [_i]
 _lib.kda_status_string.restype = ctypes.c_char_p
 _lib.kda_abi_version.restype = _i
+_lib.kda_last_cuda_error.restype = ctypes.c_char_p
 _lib.kda_forward_workspace_size.argtypes = [_i] * 8
 _lib.kda_forward_workspace_size.restype = _sz
 _lib.kda_forward_launches.argtypes = [_i] * 10
@@ -67,14 +68,15 @@ _lib.kda_forward_host.restype = _i
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT = 0, 1, 2, 3
 KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_SCRATCH_LIMIT = 4, 5, 6, 7
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
-PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_single": 3, "tc_split": 4}
+PATHS = {"auto": 0, "simt": 1, "tc": 2, "tc_single": 3, "tc_split": 4, "tc_pipe": 5}
 KDA_FUSE_NORM_QK, KDA_FUSE_GATE_LOGITS = 1, 2  # fused pre-operations (see include/kda.h)
 
 
 class KdaError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
-        super().__init__(f"{where}: {kda_status_string(code)} (status {code})")
+        detail = f": {_lib.kda_last_cuda_error().decode()}" if code == KDA_ERR_CUDA else ""
+        super().__init__(f"{where}: {kda_status_string(code)}{detail} (status {code})")
 
 
 def kda_status_string(code: int) -> str:

@@ -109,36 +109,46 @@ def test_decode_rejects_bad_args(K):
     assert d(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 96, 128, 128, 3, None) == K.KDA_ERR_INVALID_ARG
 
 
+REC = 74752  # bytes of one chunk's record: [-W ; Gamma q] + Gamma_C, Ut + P, Kh (73 KiB)
+
+
+def al(x):
+    return (x + 255) // 256 * 256
+
+
 def test_workspace_and_launch_queries(K):
-    # tensor-core shapes: the split form's per-chunk records, 74,240 bytes per chunk per head
-    # ([-W ; Gamma q] 32 KiB, Kh 16 KiB, Ut 16 KiB, P 8 KiB, Gamma_C 512 B)
-    rec = 74240
-    al = lambda x: (x + 255) // 256 * 256
-    assert K.kda_forward_workspace_size(1, 8192, 96, 128, 128, 64, 1, 1) == 128 * 96 * rec
-    assert K.kda_forward_workspace_size(2, 8192, 96, 128, 128, 64, 2, 1) == 2 * 128 * 96 * rec
-    assert K.kda_forward_workspace_size(2, 100, 3, 128, 128, 64, 2, 1) == 2 * 2 * 3 * rec
+    # tensor-core shapes: the split form's per-chunk records
+    assert K.kda_forward_workspace_size(1, 8192, 96, 128, 128, 64, 1, 1) == 128 * 96 * REC
+    assert K.kda_forward_workspace_size(2, 8192, 96, 128, 128, 64, 2, 1) == 2 * 128 * 96 * REC
+    # a short batch: the pipe form's ring (4 records and 5 flags per unit) is the larger need
+    assert K.kda_forward_workspace_size(2, 100, 3, 128, 128, 64, 2, 1) == \
+        max(2 * 2 * 3 * REC, al(6 * 4 * REC) + al(6 * 5 * 4))
     # packed sequences: records for at most T / 64 + N chunks per head, the sequences' chunk
     # offsets, and a small longest-first schedule (up to 2048 sequences)
     n_ch = -(-352549 // 64) + 8
     assert K.kda_forward_workspace_size(1, 352549, 96, 128, 128, 64, 8, 1) == \
-        al(n_ch * 96 * rec) + al(9 * 4) + 256
+        al(n_ch * 96 * REC) + al(9 * 4) + 256
     # other shapes (SIMT kernel): only the schedule
     assert K.kda_forward_workspace_size(1, 100000, 2, 64, 64, 32, 2048, 0) == 8192
     assert K.kda_forward_workspace_size(1, 100000, 2, 64, 64, 32, 2049, 0) == 0
-    # launches: split = prep + chains (+ chunk offsets and schedule for packed batches)
+    # launches: split = records + chains (+ chunk offsets and schedule for packed batches);
+    # pipe = one launch, only for up to 197 units on 148 SMs
     assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8) == 4
     assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8, "tc_single") == 2
     assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8, "simt") == 2
+    assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8, "tc_pipe") == -1
     assert K.kda_forward_launches(1, 8192, 96, 128, 128, 64, 1, 0, 1) == 2
     assert K.kda_forward_launches(1, 8192, 96, 128, 128, 64, 1, 0, 1, "tc_split") == 2
+    assert K.kda_forward_launches(1, 8192, 96, 128, 128, 64, 1, 0, 1, "tc_pipe") == 1
     assert K.kda_forward_launches(1, 8192, 96, 128, 128, 64, 1, 0, 1, "tc_single") == 1
+    assert K.kda_forward_launches(2, 8192, 99, 128, 128, 64, 1, 0, 2, "tc_pipe") == -1  # 198 units
     with pytest.raises(K.KdaError):
         K.kda_forward_workspace_size(1, 8192, 96, 100, 128, 64, 1, 1)
     assert K.kda_forward_launches(1, 256, 1, 32, 32, 16, 0, 0, 1, "simt") == 1
     assert K.kda_forward_launches(1, 256, 1, 48, 32, 16, 0, 0, 1) == -1
     # forcing a tensor-core form off its shapes is refused
-    assert K.kda_forward_launches(1, 256, 1, 32, 32, 16, 0, 0, 1, "tc_split") == -1
-    assert K.kda_forward_launches(1, 256, 1, 32, 32, 16, 0, 0, 1, "tc_single") == -1
+    for f in ("tc_split", "tc_single", "tc_pipe"):
+        assert K.kda_forward_launches(1, 256, 1, 32, 32, 16, 0, 0, 1, f) == -1
 
 
 def test_python_binding_refuses_cpu_tensors(K):
@@ -182,7 +192,8 @@ def test_segmented_queries(K):
     n2 = K.kda_forward_segmented_workspace_size(1, 1000, 2, 64, 128, 64, 1, 256)
     assert n2 >= 4 * 2 * (64 * 64 + 2 * 128 * 64) * 4
     # one segment: the plain prefill's needs (the split form's records for a dense batch)
-    assert K.kda_forward_segmented_workspace_size(2, 1000, 2, 128, 128, 64, 1, 1024) == 2 * 16 * 2 * 74240
+    assert K.kda_forward_segmented_workspace_size(2, 1000, 2, 128, 128, 64, 1, 1024) == \
+        max(2 * 16 * 2 * REC, al(4 * 4 * REC) + al(4 * 5 * 4))
     assert K.kda_forward_segmented_launches(2, 1000, 2, 128, 128, 64, 1, 1024) == 2
     # init, three passes each with a longest-first schedule, scan
     assert K.kda_forward_segmented_launches(1, 1000, 2, 128, 128, 64, 1, 256) == 8
@@ -271,7 +282,7 @@ def test_host_workspace_size_is_two_piece_slots_and_the_state(K):
     slot = 5 * piece + B * L * H * 2
     state = B * H * d * d * 4
     records = K.kda_forward_workspace_size(B, L, H, d, d, 64, B, 1)
-    assert records == B * (L // 64) * H * 74240
+    assert records == B * (L // 64) * H * REC
     assert K.kda_forward_host_workspace_size(B, T, H, d, d, 64, 1, L) == 2 * slot + state + records
     # piece_len 0: about T / 8 in whole chunks; a piece never exceeds the sequence
     assert K.kda_forward_host_workspace_size(B, T, H, d, d, 64, 1, 0) == 2 * slot + state + records

@@ -1,7 +1,8 @@
-"""GPU parity of the two tensor-core prefill forms against each other and the
+"""GPU parity of the tensor-core prefill forms against each other and the
 oracle: the split form (a chunk-parallel kernel writes every chunk's
 state-independent operands to the workspace, a second kernel carries each
-unit's state) and the single-kernel form compute the same chunked recurrence
+unit's state), the pipe form (both roles in one cooperative launch, records
+through a ring) and the single-kernel form compute the same chunked recurrence
 ("Exercices", Q7, Q21-Q22) and must agree with the fp64 oracle and with each
 other; the workspace passed decides which form AUTO runs."""
 import numpy as np
@@ -31,10 +32,14 @@ def fwd(K, inp, path, **kw):
     return o, ST
 
 
+FORMS = ["tc_split", "tc_pipe"]
+
+
+@pytest.mark.parametrize("form", FORMS)
 @pytest.mark.parametrize("B,T,H", [(1, 64, 1), (2, 200, 3), (1, 1, 2), (3, 127, 2), (1, 64 * 9 + 5, 4)])
-def test_split_matches_oracle_and_single(K, oracle_mod, B, T, H):
+def test_split_matches_oracle_and_single(K, oracle_mod, B, T, H, form):
     inp = case(B, T, H, 128, 128, "bf16", seed=1000 + T + B, s0_std=0.05, g_min_frac=0.1)
-    o_s, S_s = fwd(K, inp, "tc_split")
+    o_s, S_s = fwd(K, inp, form)
     o_f, S_f = fwd(K, inp, "tc_single")
     o_ref, S_ref = oracle_forward(oracle_mod, inp)
     units = [(b, h) for b in range(B) for h in range(H)]
@@ -45,66 +50,98 @@ def test_split_matches_oracle_and_single(K, oracle_mod, B, T, H):
     assert rel(to_f64(o_s), to_f64(o_f)) < 5e-3 and rel(to_f64(S_s), to_f64(S_f)) < 5e-3
 
 
+@pytest.mark.parametrize("form", FORMS)
 @pytest.mark.parametrize("lens", [[1, 65, 130, 0, 64, 7, 200], [0, 0, 3], [500], [64] * 40 + [0, 129]])
-def test_split_packed(K, oracle_mod, lens):
+def test_split_packed(K, oracle_mod, lens, form):
     cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     H = 3
     inp = case(1, int(cu[-1]), H, 128, 128, "bf16", seed=len(lens) + int(cu[-1]), s0_std=0.1,
                num_states=len(lens))
     inp["cu_seqlens"] = torch.tensor(cu, device="cuda")
-    o, ST = fwd(K, inp, "tc_split")
+    o, ST = fwd(K, inp, form)
     o_ref, S_ref = oracle_forward(oracle_mod, inp)
     units = [(n, h) for n in range(len(lens)) for h in range(H)]
-    compare_units(o, ST, o_ref, S_ref, units, cu, tol=TOL["bf16"], label="split packed")
+    compare_units(o, ST, o_ref, S_ref, units, cu, tol=TOL["bf16"], label=form + " packed")
     zero = [n for n, L in enumerate(lens) if L == 0]
     if zero:
         assert torch.equal(ST[zero], inp["S0"][zero])
 
 
-def test_split_identity_transition_is_exact(K):
+@pytest.mark.parametrize("form", FORMS)
+def test_split_identity_transition_is_exact(K, form):
     """beta = 0, g = 0: every record's W, Ut and P-columns vanish and Gamma_C = 1, so the
     state passes through bit for bit."""
     inp = case(2, 150, 2, 128, 128, "bf16", seed=21, s0_std=0.5)
     inp["g"].zero_(); inp["beta"].zero_()
-    o, ST = fwd(K, inp, "tc_split")
+    o, ST = fwd(K, inp, form)
     assert torch.equal(ST, inp["S0"])
     ref = torch.einsum("bthi,bhji->bthj", inp["q"].double(), inp["S0"].double())
     assert rel(to_f64(o), ref.cpu().numpy()) < TOL["bf16"]
 
 
-def test_split_g_min_runs(K, oracle_mod):
+@pytest.mark.parametrize("form", FORMS)
+def test_split_g_min_runs(K, oracle_mod, form):
     """Whole channels and 128-token runs at g = g_min = -5 (the e^80 subtile bound)."""
     inp = case(1, 256, 2, 128, 128, "bf16", seed=11, s0_std=0.1)
     inp["g"][:, :, :, ::3] = -5.0
     inp["g"][:, 64:192] = -5.0
-    o, ST = fwd(K, inp, "tc_split")
+    o, ST = fwd(K, inp, form)
     o_ref, S_ref = oracle_forward(oracle_mod, inp)
     compare_units(o, ST, o_ref, S_ref, [(0, 0), (0, 1)], tol=TOL["bf16"], label="split g_min")
 
 
 def test_workspace_decides_the_form(K):
-    """AUTO with the reported workspace runs the split form; with only the packed schedule's
-    few bytes (or none) it runs the single form; TC_SPLIT with too small a workspace is refused."""
+    """AUTO with the reported workspace runs the split form; with only the pipe form's ring it
+    runs the pipe form; with a few bytes (or none) the single form; a forced form with too
+    small a workspace is refused."""
     inp = case(1, 300, 2, 128, 128, "bf16", seed=5, s0_std=0.1)
     o_split, S_split = fwd(K, inp, "tc_split")
+    o_pipe, S_pipe = fwd(K, inp, "tc_pipe")
     o_single, S_single = fwd(K, inp, "tc_single")
     o_a, S_a = fwd(K, inp, "auto")
     assert torch.equal(o_a, o_split) and torch.equal(S_a, S_split)
+    # the two record forms compute the same records and the same chain: bit for bit
+    assert torch.equal(o_pipe, o_split) and torch.equal(S_pipe, S_split)
+    ring = torch.empty(2 * 4 * 74752 + 256, dtype=torch.uint8, device="cuda")
+    o_r, S_r = fwd(K, inp, "auto", workspace=ring)
+    assert torch.equal(o_r, o_pipe) and torch.equal(S_r, S_pipe)
     small = torch.empty(256, dtype=torch.uint8, device="cuda")
     o_b, S_b = fwd(K, inp, "auto", workspace=small)
     assert torch.equal(o_b, o_single) and torch.equal(S_b, S_single)
-    with pytest.raises(K.KdaError) as e:
-        fwd(K, inp, "tc_split", workspace=small)
-    assert e.value.code == K.KDA_ERR_WORKSPACE
+    for form in FORMS:
+        with pytest.raises(K.KdaError) as e:
+            fwd(K, inp, form, workspace=small)
+        assert e.value.code == K.KDA_ERR_WORKSPACE
 
 
-def test_split_two_calls_reuse_workspace(K, oracle_mod):
+@pytest.mark.parametrize("form", ["auto", "tc_pipe"])
+def test_split_two_calls_reuse_workspace(K, oracle_mod, form):
     """The records are scratch: a second call with other inputs in the same workspace gives
-    its own results (every record is rewritten before it is read)."""
+    its own results (every record is rewritten before it is read, the ring's flags are
+    reset by every call)."""
     ws = torch.empty(K.kda_forward_workspace_size(2, 256, 2, 128, 128, 64, 2, torch.bfloat16),
                      dtype=torch.uint8, device="cuda")
     for seed in (1, 2):
         inp = case(2, 256, 2, 128, 128, "bf16", seed=seed, s0_std=0.1)
-        o, ST = fwd(K, inp, "auto", workspace=ws)
+        o, ST = fwd(K, inp, form, workspace=ws)
         o_ref, S_ref = oracle_forward(oracle_mod, inp)
         compare_units(o, ST, o_ref, S_ref, [(b, h) for b in range(2) for h in range(2)], tol=TOL["bf16"])
+
+
+@pytest.mark.parametrize("B,T,H,lens", [(3, 130, 70, None), (1, 0, 6, [64] * 40 + [0, 129])])
+def test_split_two_kernel_form(K, oracle_mod, B, T, H, lens):
+    """More (sequence, head) units than the one-launch form takes (two thirds of two CTAs per
+    SM): every chunk's record goes to the workspace, then the chains run (dense and packed)."""
+    if lens is None:
+        inp = case(B, T, H, 128, 128, "bf16", seed=77, s0_std=0.05)
+        units = [(b, h) for b in range(B) for h in range(H)]
+        cu = None
+    else:
+        cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+        inp = case(1, int(cu[-1]), H, 128, 128, "bf16", seed=78, s0_std=0.05, num_states=len(lens))
+        inp["cu_seqlens"] = torch.tensor(cu, device="cuda")
+        units = [(n, h) for n in range(len(lens)) for h in range(H)]
+    assert len(units) * 3 > 2 * 2 * torch.cuda.get_device_properties(0).multi_processor_count
+    o, ST = fwd(K, inp, "tc_split")
+    o_ref, S_ref = oracle_forward(oracle_mod, inp, units=units)
+    compare_units(o, ST, o_ref, S_ref, units, cu, tol=TOL["bf16"], label="split two-kernel")
