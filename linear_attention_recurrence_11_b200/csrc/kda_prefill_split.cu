@@ -117,8 +117,10 @@ __device__ __forceinline__ Task task_at(const SplitParams &sp, long long t) {
     const PrefillArgs &p = sp.a;
     Task k;
     k.t = t;
-    k.h = (int)(t % p.H);
-    const long long gc = t / p.H;
+    // 32-bit quotients: the number of tasks is below 2^31 (checked when the call is validated)
+    const unsigned t32 = (unsigned)t;
+    k.h = (int)(t32 % (unsigned)p.H);
+    const unsigned gc = t32 / (unsigned)p.H;
     long long c, end;
     if (sp.chunk_base) {  // largest n with chunk_base[n] <= gc (empty sequences share a base)
         int lo = 0, hi = p.num_units;
@@ -131,8 +133,8 @@ __device__ __forceinline__ Task task_at(const SplitParams &sp, long long t) {
         k.tok0 = (long long)p.cu_seqlens[lo] + c * C;
         end = p.cu_seqlens[lo + 1];
     } else {
-        k.n = (int)(gc / sp.nch);
-        c = gc % sp.nch;
+        k.n = (int)(gc / (unsigned)sp.nch);
+        c = gc % (unsigned)sp.nch;
         k.tok0 = (long long)k.n * p.T + c * C;
         end = (long long)k.n * p.T + p.T;
     }
@@ -301,6 +303,17 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
         const bool more = src.next(nxt);
         uint8_t *rec = src.record(cur);
         const int Lc = cur.Lc;
+        if (more && tid == 0) {  // the next task's tiles into L2 now; its loads come late (below)
+            tma_prefetch_l2_3d(&tm_k, 0, nxt.h, (int)nxt.tok0);
+            tma_prefetch_l2_3d(&tm_k, 64, nxt.h, (int)nxt.tok0);
+            tma_prefetch_l2_3d(&tm_q, 0, nxt.h, (int)nxt.tok0);
+            tma_prefetch_l2_3d(&tm_q, 64, nxt.h, (int)nxt.tok0);
+            tma_prefetch_l2_3d(&tm_g, 0, nxt.h, (int)nxt.tok0);
+            if (has_v) {
+                tma_prefetch_l2_3d(&tm_v, 0, nxt.h, (int)nxt.tok0);
+                tma_prefetch_l2_3d(&tm_v, 64, nxt.h, (int)nxt.tok0);
+            }
+        }
 
         // ---- this task's k, q, g
         {
@@ -411,13 +424,17 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
                 el1[e] = ti == 2 ? ex2(-Dm[2][e]) : 1.f;
                 er[e] = ti == 0 ? ed[0][e] : ti == 2 ? ed[2][e] : 1.f;
             }
+            const float2 er2[2] = {make_float2(er[0], er[1]), make_float2(er[2], er[3])};
+            const float2 post2[2] = {make_float2(post[0], post[1]), make_float2(post[2], post[3])};
+            const float2 el02[2] = {make_float2(el0[0], el0[1]), make_float2(el0[2], el0[3])};
+            const float2 el12[2] = {make_float2(el1[0], el1[1]), make_float2(el1[2], el1[3])};
+            const float2 pg2[2] = {make_float2(pg[0], pg[1]), make_float2(pg[2], pg[3])};
             uint8_t *const l0 = sm + P_L0 + cblk * 16 * KB;
             uint8_t *const l1 = sm + P_L1 + cblk * 8 * KB;
             uint8_t *const rrow = sm + P_R + cblk * 8 * KB;
             uint8_t *const gkrow = sm + P_GK + cblk * 8 * KB;
             uint8_t *const gq_rec = rec + REC_WQ + cblk * 16 * KB + 8 * KB;
             uint8_t *const kh_rec = rec + REC_KH + cblk * 8 * KB;
-            auto pk4 = [](float a, float b, float c, float d) { return make_uint2(pack_bf2(a, b), pack_bf2(c, d)); };
             auto ld4 = [](const uint8_t *ptr, float (&v)[4]) {
                 const uint2 raw = *reinterpret_cast<const uint2 *>(ptr);
                 const float2 x = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
@@ -432,32 +449,38 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
                 float kx[4], qx[4];
                 ld4(l0 + off_r, kx);
                 ld4(l0 + off_q, qx);
-                float F[4], Fi[4];
+                // paired fp32 products (two channels per instruction, each the same IEEE product)
+                float2 F[2], Fi[2];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    F[e] = ex2(gl[rr][e]);    // e^{G_r - G_start(ti)}, in [e^-80, 1]
-                    Fi[e] = ex2(-gl[rr][e]);  // e^{G_start(ti) - G_r}, in [1, e^80]
+                for (int e = 0; e < 2; ++e) {
+                    F[e] = make_float2(ex2(gl[rr][2 * e]), ex2(gl[rr][2 * e + 1]));      // e^{G_r - G_start(ti)}
+                    Fi[e] = make_float2(ex2(-gl[rr][2 * e]), ex2(-gl[rr][2 * e + 1]));  // e^{G_start(ti) - G_r}
                 }
-                float kr[4], kf[4], qf[4];
+                float2 kr[2], kf[2], qf[2];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    kr[e] = kx[e] * Fi[e];
-                    kf[e] = kx[e] * F[e];
-                    qf[e] = qx[e] * F[e];
+                for (int e = 0; e < 2; ++e) {
+                    const float2 k2 = make_float2(kx[2 * e], kx[2 * e + 1]);
+                    const float2 q2 = make_float2(qx[2 * e], qx[2 * e + 1]);
+                    kr[e] = __fmul2_rn(k2, Fi[e]);
+                    kf[e] = __fmul2_rn(k2, F[e]);
+                    qf[e] = __fmul2_rn(q2, F[e]);
                 }
-                *reinterpret_cast<uint2 *>(rrow + off_r) = pk4(kr[0] * er[0], kr[1] * er[1], kr[2] * er[2], kr[3] * er[3]);
-                *reinterpret_cast<uint2 *>(kh_rec + off_r) =
-                    pk4(kr[0] * post[0], kr[1] * post[1], kr[2] * post[2], kr[3] * post[3]);
-                *reinterpret_cast<uint2 *>(l0 + off_r) = pk4(kf[0] * el0[0], kf[1] * el0[1], kf[2] * el0[2], kf[3] * el0[3]);
-                *reinterpret_cast<uint2 *>(l0 + off_q) = pk4(qf[0] * el0[0], qf[1] * el0[1], qf[2] * el0[2], qf[3] * el0[3]);
+                auto st2 = [](uint8_t *ptr, const float2 (&x)[2], const float2 (&f)[2]) {
+                    const __nv_bfloat162 a = __float22bfloat162_rn(__fmul2_rn(x[0], f[0]));
+                    const __nv_bfloat162 b = __float22bfloat162_rn(__fmul2_rn(x[1], f[1]));
+                    *reinterpret_cast<uint2 *>(ptr) =
+                        make_uint2(*reinterpret_cast<const uint32_t *>(&a), *reinterpret_cast<const uint32_t *>(&b));
+                };
+                st2(rrow + off_r, kr, er2);
+                st2(kh_rec + off_r, kr, post2);
+                st2(l0 + off_r, kf, el02);
+                st2(l0 + off_q, qf, el02);
                 if (ti >= 2) {
-                    *reinterpret_cast<uint2 *>(l1 + sw128_offset(r - 32, cin)) =
-                        pk4(kf[0] * el1[0], kf[1] * el1[1], kf[2] * el1[2], kf[3] * el1[3]);
-                    *reinterpret_cast<uint2 *>(l1 + sw128_offset(r, cin)) =
-                        pk4(qf[0] * el1[0], qf[1] * el1[1], qf[2] * el1[2], qf[3] * el1[3]);
+                    st2(l1 + sw128_offset(r - 32, cin), kf, el12);
+                    st2(l1 + sw128_offset(r, cin), qf, el12);
                 }
-                *reinterpret_cast<uint2 *>(gq_rec + off_r) = pk4(qf[0] * pg[0], qf[1] * pg[1], qf[2] * pg[2], qf[3] * pg[3]);
-                *reinterpret_cast<uint2 *>(gkrow + off_r) = pk4(kf[0] * pg[0], kf[1] * pg[1], kf[2] * pg[2], kf[3] * pg[3]);
+                st2(gq_rec + off_r, qf, pg2);
+                st2(gkrow + off_r, kf, pg2);
             }
         }
         if (Src::kPublish) __threadfence();  // this thread's record stores before the publication
@@ -693,6 +716,37 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 }
 
 // ====================================================================== chain
+// U = (-W S from TMEM) + Ut for one row r of a 64-column half, written as bf16 over the Ut tile
+// (MN-major [tok][dv], 128-byte rows): all of the row's Ut is loaded before any of it is
+// overwritten, in two passes of 32 columns.
+__device__ __forceinline__ void u_readout(uint8_t *ut, int r, uint32_t taddr) {
+#pragma unroll
+    for (int g2 = 0; g2 < 2; ++g2) {
+        float v[2][16];
+        tmem_ld16(taddr + 32u * g2, v[0]);
+        tmem_ld16(taddr + 32u * g2 + 16u, v[1]);
+        uint4 w[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) w[i] = *reinterpret_cast<const uint4 *>(ut + sw128_offset(r, 32 * g2 + 8 * i));
+        tmem_wait_ld();
+        uint4 o4[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t ws[4] = {w[i].x, w[i].y, w[i].z, w[i].w};
+            float *x = v[i >> 1] + 8 * (i & 1);
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ws[e]));
+                pk[e] = pack_bf2(x[2 * e] + f.x, x[2 * e + 1] + f.y);
+            }
+            o4[i] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4 *>(ut + sw128_offset(r, 32 * g2 + 8 * i)) = o4[i];
+    }
+}
+
 __global__ void __launch_bounds__(NT, 1)
 kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp) {
     const PrefillArgs &p = sp.a;
@@ -827,38 +881,17 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
             tc_fence_before();
         }
         if (!wait_mma()) { aborted = true; break; }
+        if (tid == 0 && ch >= 1 && ch + 1 < nchunks) {
+            // the record one chunk ahead goes into the other buffer, whose outputs (staged by the
+            // previous chunk) have been read by their stores by now
+            bulk_wait_read_all();
+            mbar_arrive_expect_tx(&bar_rec[b ^ 1], REC_BYTES);
+            bulk_load(sm + (b ^ 1) * C_RECSTRIDE, record(ch + 1), REC_BYTES, &bar_rec[b ^ 1]);
+            rec_armed |= 1u << (b ^ 1);
+        }
 
         // U = Ut - W S (rows 0..63) -> bf16 B operand, written over the record's Ut tile
-        if (quarter < 2) {
-            const int r = 32 * quarter + lane;
-            uint8_t *ut = buf + REC_UT + half * 8 * KB;
-            float v[4][16];
-#pragma unroll
-            for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + tmu + 64u * half + 16u * gq, v[gq]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int gq = 0; gq < 4; ++gq) {
-#pragma unroll
-                for (int pc = 0; pc < 2; ++pc) {
-                    uint4 *slot = reinterpret_cast<uint4 *>(ut + sw128_offset(r, 16 * gq + 8 * pc));
-                    const uint4 w = *slot;
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                    float *x = v[gq] + 8 * pc;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ws[e]));
-                        x[2 * e] += f.x;
-                        x[2 * e + 1] += f.y;
-                    }
-                    uint4 o4;
-                    o4.x = pack_bf2(x[0], x[1]);
-                    o4.y = pack_bf2(x[2], x[3]);
-                    o4.z = pack_bf2(x[4], x[5]);
-                    o4.w = pack_bf2(x[6], x[7]);
-                    *slot = o4;
-                }
-            }
-        }
+        if (quarter < 2) u_readout(buf + REC_UT + half * 8 * KB, 32 * quarter + lane, tmem + tlane + tmu + 64u * half);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -937,12 +970,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
                 tma_store_3d(&tm_o, buf + REC_UT + 8 * KB, 64, h, (int)tok0);
                 bulk_commit();
             }
-            if (ch + 2 < nchunks) {  // the record two chunks ahead goes into this buffer once the
-                bulk_wait_read_all();  // output stores have read it
-                mbar_arrive_expect_tx(&bar_rec[b], REC_BYTES);
-                bulk_load(buf, record(ch + 2), REC_BYTES, &bar_rec[b]);
-                rec_armed |= 1u << b;
-            }
+
         }
     }
     if (tid == 0) bulk_wait_all();
@@ -1254,39 +1282,7 @@ __device__ __forceinline__ void chain_role(const PipeParams &pp, const CUtensorM
         if (!wait_piece(bar_b, ph_b, 2u)) { aborted = true; break; }
 
         // U = Ut - W S (rows 0..63) -> bf16 B operand, written over the record's Ut tile
-        if (quarter < 2) {
-            const int r = 32 * quarter + lane;
-            uint8_t *ut = sm + REC_UT + half * 8 * KB;
-#pragma unroll
-            for (int g2 = 0; g2 < 2; ++g2) {
-            float v[2][16];
-#pragma unroll
-            for (int gq = 0; gq < 2; ++gq) tmem_ld16(tmem + tlane + X_TM_U + 64u * half + 32u * g2 + 16u * gq, v[gq]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int gq = 0; gq < 2; ++gq) {
-#pragma unroll
-                for (int pc = 0; pc < 2; ++pc) {
-                    uint4 *sl = reinterpret_cast<uint4 *>(ut + sw128_offset(r, 32 * g2 + 16 * gq + 8 * pc));
-                    const uint4 w = *sl;
-                    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-                    float *x = v[gq] + 8 * pc;
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ws[e]));
-                        x[2 * e] += f.x;
-                        x[2 * e + 1] += f.y;
-                    }
-                    uint4 o4;
-                    o4.x = pack_bf2(x[0], x[1]);
-                    o4.y = pack_bf2(x[2], x[3]);
-                    o4.z = pack_bf2(x[4], x[5]);
-                    o4.w = pack_bf2(x[6], x[7]);
-                    *sl = o4;
-                }
-            }
-            }
-        }
+        if (quarter < 2) u_readout(sm + REC_UT + half * 8 * KB, 32 * quarter + lane, tmem + tlane + X_TM_U + 64u * half);
         fence_proxy_async_smem();
         tc_fence_before();
         if (!wait_piece(bar_c, ph_c, 4u)) { aborted = true; break; }
