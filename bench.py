@@ -282,7 +282,10 @@ def run_ours(args, rank, world, device):
     tokens = w.total_tokens
     value = weak_scaling_value(tokens, K, ms_total, world)
     alg_bytes, alg_flops = prefill_algorithmic(w, elem)
-    if path_used == "tc":  # the split form runs when the workspace holds its records
+    if path_used == "tc" and seg:  # segments: records once, three chain passes, a scan
+        kern_src = "linear_attention_recurrence_11_b200/csrc/kda_prefill_split.cu"
+        path_used = "tc_segmented"
+    elif path_used == "tc":  # the split form runs when the workspace holds its records
         split = seg == 0 and args.path in ("auto", "tc", "tc_split", "tc_pipe")
         kern_src = ("linear_attention_recurrence_11_b200/csrc/kda_prefill_split.cu" if split
                     else "linear_attention_recurrence_11_b200/csrc/kda_prefill_tc.cu")

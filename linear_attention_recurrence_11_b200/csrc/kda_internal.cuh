@@ -110,6 +110,17 @@ size_t prefill_tc_workspace(const PrefillArgs &a);
 int prefill_tc_launches(const PrefillArgs &a);
 // the split tensor-core form: chunk-parallel records in the workspace, then the state chains
 cudaError_t launch_prefill_split(const PrefillArgs &a);
+// its two stages: the records of every chunk of `a` (in a.workspace), and one pass of the
+// state chains over them with pass's S0 / S_T / o (the q, k, g, beta, sizes and layout of
+// `a`; pass.v == nullptr leaves every record's Ut out: all-zero values)
+struct SplitRecords {
+    uint8_t *rec;
+    const int32_t *chunk_base, *seq_order;
+    int nch;
+    long long tasks;
+};
+cudaError_t launch_split_records(const PrefillArgs &a, SplitRecords *out);
+cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r);
 size_t prefill_split_workspace(const PrefillArgs &a);
 int prefill_split_launches(const PrefillArgs &a);
 // the one-launch form: chains and record producers in one cooperative launch, records in a ring

@@ -719,7 +719,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 // U = (-W S from TMEM) + Ut for one row r of a 64-column half, written as bf16 over the Ut tile
 // (MN-major [tok][dv], 128-byte rows): all of the row's Ut is loaded before any of it is
 // overwritten, in two passes of 32 columns.
-__device__ __forceinline__ void u_readout(uint8_t *ut, int r, uint32_t taddr) {
+__device__ __forceinline__ void u_readout(uint8_t *ut, int r, uint32_t taddr, bool add_ut = true) {
 #pragma unroll
     for (int g2 = 0; g2 < 2; ++g2) {
         float v[2][16];
@@ -737,7 +737,8 @@ __device__ __forceinline__ void u_readout(uint8_t *ut, int r, uint32_t taddr) {
             uint32_t pk[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ws[e]));
+                const float2 f = add_ut ? __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&ws[e]))
+                                        : make_float2(0.f, 0.f);
                 pk[e] = pack_bf2(x[2 * e] + f.x, x[2 * e + 1] + f.y);
             }
             o4[i] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
@@ -891,7 +892,9 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
         }
 
         // U = Ut - W S (rows 0..63) -> bf16 B operand, written over the record's Ut tile
-        if (quarter < 2) u_readout(buf + REC_UT + half * 8 * KB, 32 * quarter + lane, tmem + tlane + tmu + 64u * half);
+        // (all-zero values, the transition pass of a segment: the record's Ut is left out)
+        if (quarter < 2)
+            u_readout(buf + REC_UT + half * 8 * KB, 32 * quarter + lane, tmem + tlane + tmu + 64u * half, p.v != nullptr);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -1534,21 +1537,19 @@ cudaError_t launch_prefill_pipe(const PrefillArgs &a) {
     return launch_pipe(a, mq, mk, mv, mg, mo);
 }
 
-cudaError_t launch_prefill_split(const PrefillArgs &a) {
+cudaError_t launch_split_records(const PrefillArgs &a, SplitRecords *out) {
+    *out = SplitRecords{};
     if (a.num_units == 0) return cudaSuccess;
     const size_t tokens = a.cu_seqlens ? (size_t)a.T : (size_t)a.B * (size_t)a.T;
-    if (tokens == 0) return launch_prefill_simt(a);
-    CUtensorMap mq, mk, mv, mg, mo;
+    if (tokens == 0) return cudaSuccess;
+    CUtensorMap mq, mk, mv, mg;
     if (!make_map(&mq, a.q, tokens, a.H, 64, true) || !make_map(&mk, a.k, tokens, a.H, 64, true) ||
-        !make_map(&mv, a.v ? a.v : a.q, tokens, a.H, 64, true) || !make_map(&mg, a.g, tokens, a.H, 128, false) ||
-        !make_map(&mo, a.o ? a.o : a.q, tokens, a.H, 64, true))
+        !make_map(&mv, a.v ? a.v : a.q, tokens, a.H, 64, true) || !make_map(&mg, a.g, tokens, a.H, 128, false))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM_BYTES);
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                              (int)cudaSharedmemCarveoutMaxShared);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kda_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C_SMEM_BYTES);
     if (e != cudaSuccess) return e;
     SplitParams sp{};
     sp.a = a;
@@ -1578,9 +1579,43 @@ cudaError_t launch_prefill_split(const PrefillArgs &a) {
     kda_prep_kernel<<<(unsigned)grid_p, NT, P_SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, sp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const unsigned grid_c = (unsigned)((size_t)a.num_units * a.H);
-    kda_chain_kernel<<<grid_c, NT, C_SMEM_BYTES, a.stream>>>(mo, sp);
+    out->rec = sp.rec;
+    out->chunk_base = sp.chunk_base;
+    out->seq_order = sp.a.seq_order;
+    out->nch = sp.nch;
+    out->tasks = sp.tasks;
+    return cudaSuccess;
+}
+
+cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r) {
+    if (pass.num_units == 0) return cudaSuccess;
+    const size_t tokens = pass.cu_seqlens ? (size_t)pass.T : (size_t)pass.B * (size_t)pass.T;
+    if (tokens == 0) return launch_prefill_simt(pass);
+    CUtensorMap mo;
+    if (!make_map(&mo, pass.o ? pass.o : pass.q, tokens, pass.H, 64, true)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(kda_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    SplitParams sp{};
+    sp.a = pass;
+    if (!packed(pass)) sp.a.cu_seqlens = nullptr;
+    sp.a.seq_order = r.seq_order;
+    sp.rec = r.rec;
+    sp.chunk_base = r.chunk_base;
+    sp.nch = r.nch;
+    sp.tasks = r.tasks;
+    const unsigned grid_c = (unsigned)((size_t)pass.num_units * pass.H);
+    kda_chain_kernel<<<grid_c, NT, C_SMEM_BYTES, pass.stream>>>(mo, sp);
     return cudaGetLastError();
+}
+
+cudaError_t launch_prefill_split(const PrefillArgs &a) {
+    if (a.num_units == 0) return cudaSuccess;
+    const size_t tokens = a.cu_seqlens ? (size_t)a.T : (size_t)a.B * (size_t)a.T;
+    if (tokens == 0) return launch_prefill_simt(a);
+    SplitRecords r;
+    cudaError_t e = launch_split_records(a, &r);
+    if (e != cudaSuccess) return e;
+    return launch_split_chain(a, r);
 }
 
 }  // namespace kda

@@ -14,8 +14,11 @@
 //   scan    S_in,0 = S0, S_in,p+1 = M_p S_in,p + S~_p (fp32, one CTA per
 //           (sequence, head), sequential over segments; the last one is S_T);
 //   pass C  the recurrence run over every segment from S_in,p, writing o.
-// Passes A-C are the ordinary prefill kernels over the segments laid out as
-// packed sequences. M_p is a dk x dk matrix kept in the state layout
+// On the tensor-core shapes (bf16, dk = dv = 128, chunks of 64) the state-independent
+// part of every chunk is computed once, as the split prefill's records, and passes
+// A-C are three runs of its state-chain kernel over them (pass A leaves the records'
+// Ut out); elsewhere passes A-C are the ordinary prefill kernels over the segments
+// laid out as packed sequences. M_p is a dk x dk matrix kept in the state layout
 // ([column][dk], so pass A runs with dv = dk).
 #include "kda_internal.cuh"
 #include "kda_sm100.cuh"
@@ -179,9 +182,26 @@ cudaError_t launch_scan(const SegmentedArgs &s, const float *Mbuf, const float *
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
-// Workspace carve-up (all pieces 256-byte aligned).
+// The segments of the B sequences as one packed batch (cu_seqlens filled on the device).
+PrefillArgs segments_as_packed(const SegmentedArgs &s, const int32_t *cu_seg) {
+    PrefillArgs a{};
+    a.q = s.q; a.k = s.k; a.v = s.v; a.g = s.g; a.beta = s.beta;
+    a.cu_seqlens = cu_seg;
+    a.B = 1; a.T = s.B * s.T; a.H = s.H; a.dk = s.dk; a.dv = s.dv; a.chunk = s.chunk; a.dtype = s.dtype;
+    a.num_units = s.B * s.P;
+    a.dev_status = s.dev_status; a.stream = s.stream;
+    return a;
+}
+
+// Whether passes A-C run on the split prefill's records (both tensor-core shapes).
+bool records_path(const SegmentedArgs &s) {
+    return prefill_tc_supported(s.dk, s.dk, s.chunk, s.dtype) && prefill_tc_supported(s.dk, s.dv, s.chunk, s.dtype);
+}
+
+// Workspace carve-up (all pieces 256-byte aligned): segment offsets, the longest-first
+// schedule, M, S~ and S_in of every (segment, head), and the records where they are used.
 struct SegLayout {
-    size_t cu, order, M, Z, Sin, total;
+    size_t cu, order, M, Z, Sin, rec, total;
 };
 SegLayout seg_layout(const SegmentedArgs &s) {
     const size_t units = (size_t)s.B * s.P;
@@ -191,7 +211,12 @@ SegLayout seg_layout(const SegmentedArgs &s) {
     L.M = L.order + seq_order_bytes((int)units);
     L.Z = L.M + align256(units * s.H * s.dk * s.dk * sizeof(float));
     L.Sin = L.Z + align256(units * s.H * s.dv * s.dk * sizeof(float));
-    L.total = L.Sin + align256(units * s.H * s.dv * s.dk * sizeof(float));
+    L.rec = L.Sin + align256(units * s.H * s.dv * s.dk * sizeof(float));
+    L.total = L.rec;
+    if (records_path(s)) {
+        static const int32_t marker = 0;  // compared against null only
+        L.total += align256(prefill_split_workspace(segments_as_packed(s, &marker)));
+    }
     return L;
 }
 
@@ -224,6 +249,8 @@ cudaError_t launch_segment_pair(const SegmentedArgs &s, float *M, float *Z, bool
 
 int segmented_launches(const SegmentedArgs &s) {
     const int order = seq_order_bytes(s.B * s.P) > 0 ? 1 : 0;
+    if (records_path(s))  // init, chunk offsets (+ schedule), records, three chain passes, scan
+        return 1 + 1 + order + 1 + 3 + 1;
     return 1 /* init */ + 3 * (1 + order) /* passes A, B, C */ + 1 /* scan */;
 }
 
@@ -239,6 +266,26 @@ cudaError_t launch_segmented(const SegmentedArgs &s, bool tc_pair, bool tc_state
     kda_segment_init_kernel<<<296, kSegThreads, 0, s.stream>>>(cu_seg, Mbuf, s.B, s.T, s.P, s.seg_len, s.H, s.dk);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+
+    if (records_path(s)) {
+        PrefillArgs a = segments_as_packed(s, cu_seg);
+        a.workspace = ws + L.rec;
+        a.workspace_bytes = L.total - L.rec;
+        SplitRecords r;
+        if ((e = launch_split_records(a, &r)) != cudaSuccess) return e;
+        // pass A: M_p from the identity with zero values; pass B: S~_p from zero
+        PrefillArgs pa = a;
+        pa.v = nullptr; pa.o = nullptr; pa.S0 = Mbuf; pa.ST = Mbuf; pa.dv = s.dk;
+        if ((e = launch_split_chain(pa, r)) != cudaSuccess) return e;
+        PrefillArgs pb = a;
+        pb.o = nullptr; pb.S0 = nullptr; pb.ST = Zbuf;
+        if ((e = launch_split_chain(pb, r)) != cudaSuccess) return e;
+        if ((e = launch_scan(s, Mbuf, Zbuf, Sin)) != cudaSuccess) return e;
+        // pass C: outputs, every segment from its incoming state
+        PrefillArgs pc = a;
+        pc.o = s.o; pc.S0 = Sin; pc.ST = nullptr;
+        return launch_split_chain(pc, r);
+    }
 
     PrefillArgs a{};
     a.q = s.q; a.k = s.k; a.g = s.g; a.beta = s.beta;

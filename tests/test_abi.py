@@ -185,9 +185,13 @@ def test_segmented_rejects_bad_arguments(K):
 
 
 def test_segmented_queries(K):
-    # 4 segments x 2 heads: three fp32 128 x 128 states per (segment, head) plus offsets
+    # 4 segments x 2 heads: three fp32 128 x 128 states per (segment, head), offsets, and on
+    # the tensor-core shapes the records of every chunk of the segments (at most T / 64 + 4
+    # chunks per head, 73 KiB each, with their own chunk offsets and schedule)
     n = K.kda_forward_segmented_workspace_size(1, 1000, 2, 128, 128, 64, 1, 256)
-    assert n >= 3 * 4 * 2 * 128 * 128 * 4 and n < 3 * 4 * 2 * 128 * 128 * 4 + 4096
+    states = 3 * 4 * 2 * 128 * 128 * 4
+    records = al((-(-1000 // 64) + 4) * 2 * REC)
+    assert n >= states + records and n < states + records + 4096
     # the transition of a dk = 64 segment is 64 x 64 whatever dv is
     n2 = K.kda_forward_segmented_workspace_size(1, 1000, 2, 64, 128, 64, 1, 256)
     assert n2 >= 4 * 2 * (64 * 64 + 2 * 128 * 64) * 4
@@ -195,8 +199,10 @@ def test_segmented_queries(K):
     assert K.kda_forward_segmented_workspace_size(2, 1000, 2, 128, 128, 64, 1, 1024) == \
         max(2 * 16 * 2 * REC, al(4 * 4 * REC) + al(4 * 5 * 4))
     assert K.kda_forward_segmented_launches(2, 1000, 2, 128, 128, 64, 1, 1024) == 2
-    # init, three passes each with a longest-first schedule, scan
+    # tensor-core shapes: init, chunk offsets, schedule, records, three chain passes, scan
     assert K.kda_forward_segmented_launches(1, 1000, 2, 128, 128, 64, 1, 256) == 8
+    # elsewhere: init, three prefill passes each with a longest-first schedule, scan
+    assert K.kda_forward_segmented_launches(1, 1000, 2, 64, 64, 64, 1, 256) == 8
     with pytest.raises(K.KdaError):
         K.kda_forward_segmented_workspace_size(1, 1000, 2, 128, 128, 64, 1, 96)
 
