@@ -285,11 +285,14 @@ def run_ours(args, rank, world, device):
     if path_used == "tc" and seg:  # segments: records once, three chain passes, a scan
         kern_src = "linear_attention_recurrence_11_b200/csrc/kda_prefill_split.cu"
         path_used = "tc_segmented"
-    elif path_used == "tc":  # the split form runs when the workspace holds its records
-        split = seg == 0 and args.path in ("auto", "tc", "tc_split", "tc_pipe")
-        kern_src = ("linear_attention_recurrence_11_b200/csrc/kda_prefill_split.cu" if split
-                    else "linear_attention_recurrence_11_b200/csrc/kda_prefill_tc.cu")
-        path_used = ("tc_pipe" if args.path == "tc_pipe" else "tc_split") if split else "tc_single"
+    elif path_used == "tc":  # AUTO: the split form up to three units per SM, else the single kernel
+        sms = torch.cuda.get_device_properties(device).multi_processor_count
+        if args.path in ("tc_split", "tc_pipe", "tc_single"):
+            path_used = args.path
+        else:
+            path_used = "tc_split" if N * w.H <= 3 * sms else "tc_single"
+        kern_src = ("linear_attention_recurrence_11_b200/csrc/kda_prefill_tc.cu" if path_used == "tc_single"
+                    else "linear_attention_recurrence_11_b200/csrc/kda_prefill_split.cu")
     else:
         kern_src = "linear_attention_recurrence_11_b200/csrc/kda_prefill_simt.cu"
     achieved = alg_bytes / (kern_ms / 1e3) / 1e9
@@ -420,9 +423,12 @@ def varlen_measure(args, device, peaks, barrier, max_ranks, world, rank):
     o1 = torch.empty_like(sl["v"])
     ST1 = torch.empty((1, w.H, w.dv, w.dk), dtype=torch.float32, device=device)
 
+    ws1 = torch.empty(max(1, kda.kda_forward_workspace_size(1, w.seqlens[nl], w.H, w.dk, w.dv, w.chunk, 1, dt,
+                                                           path=args.path)), dtype=torch.uint8, device=device)
+
     def longest():
         kda.kda_forward(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], None, chunk=w.chunk, o=o1, S_T=ST1,
-                        workspace=ws, path=args.path)
+                        workspace=ws1, path=args.path)
     ms_long = timed(longest, K)
     alg_bytes, alg_flops = prefill_algorithmic(w, dt.itemsize)
     gbs = alg_bytes / (ms / 1e3) / 1e9

@@ -90,10 +90,13 @@ typedef enum { KDA_FUSE_NORM_QK = 1, KDA_FUSE_GATE_LOGITS = 2 } kda_fuse;
  *    at once, the records passing through a ring of 4 per unit; for at most
  *    two thirds of twice the SM count of units (197 on 148 SMs), else
  *    KDA_ERR_UNSUPPORTED. Workspace: about 292 KiB per unit.
- * AUTO and TC run the split form when the workspace holds it, then the pipe
- * form when its ring fits, else the single form (TC returns
- * KDA_ERR_UNSUPPORTED off the tensor-core shapes, AUTO falls back to SIMT);
- * a forced form returns KDA_ERR_WORKSPACE if the workspace is too small. */
+ * AUTO and TC run the single form for batches of more than three units per
+ * SM (all SMs are busy and records would only add traffic); otherwise the
+ * split form when the workspace holds it, then the pipe form when its ring
+ * fits, else the single form (TC returns KDA_ERR_UNSUPPORTED off the
+ * tensor-core shapes, AUTO falls back to SIMT); a forced form returns
+ * KDA_ERR_WORKSPACE if the workspace is too small
+ * (kda_forward_workspace_size_ex gives each path's need). */
 typedef enum {
     KDA_PATH_AUTO = 0,
     KDA_PATH_SIMT = 1,
@@ -118,17 +121,24 @@ const char *kda_last_cuda_error(void);
  * the scratch of the chunked prefill of "Exercices", Q7 with the KCP
  * composition of Q21-Q22. num_seqs is the number of packed sequences when
  * cu_seqlens is used, else B (B == 1 with num_seqs > 1 means packed
- * sequences). On the tensor-core shapes it covers every tensor-core form
- * (kda_path): the split form's per-chunk records (74,752 bytes per chunk per
- * head; for packed batches counted for at most T / 64 + num_seqs chunks per
- * head, plus the sequences' chunk offsets and a longest-first schedule of up
- * to 2048 sequences), or the pipe form's ring where that is larger. A smaller
- * workspace still works on the tensor cores (see kda_path). The workspace is scratch: its contents on entry do not
+ * sequences). On the tensor-core shapes it is what AUTO runs (kda_path): for
+ * batches of up to three (sequence, head) units per SM, the split form's
+ * per-chunk records (74,752 bytes per chunk per head; for packed batches
+ * counted for at most T / 64 + num_seqs chunks per head, plus the sequences'
+ * chunk offsets and a longest-first schedule of up to 2048 sequences); for
+ * larger batches, the single form's schedule only. A smaller workspace still
+ * works on the tensor cores (see kda_path). The workspace is scratch: its contents on entry do not
  * matter and it may be reused after the stream reaches the end of the call.
  * Returns (size_t)-1 if the sizes are invalid.
  */
 size_t kda_forward_workspace_size(int B, int T, int H, int dk, int dv, int chunk,
                                   int num_seqs, int dtype);
+
+/* The workspace kda_forward_ex needs with an explicit path (kda_path): the form
+ * that path runs with that workspace; kda_forward_workspace_size is this with
+ * KDA_PATH_AUTO. (size_t)-1 if the sizes or the path are invalid. */
+size_t kda_forward_workspace_size_ex(int B, int T, int H, int dk, int dv, int chunk,
+                                     int num_seqs, int dtype, int path);
 
 /*
  * Chunked prefill with KCP inter-chunk state composition: the recurrence of

@@ -38,14 +38,18 @@ bool use_tc(const kda::PrefillArgs &a, int path) {
 }
 
 // The prefill form a call runs (kda_path): the SIMT kernel or one of the three tensor-core
-// forms. AUTO and TC take the two-kernel split form when the workspace holds its records, then
-// the one-launch form when its ring fits, then the single kernel.
+// forms. AUTO and TC take the single kernel for batches of more (sequence, head) units than
+// three per SM (they keep every SM busy and add no record traffic); otherwise the two-kernel
+// split form when the workspace holds its records, then the one-launch form when its ring
+// fits, then the single kernel.
 enum class Form { Simt, Single, Split, Pipe };
+bool many_units(const kda::PrefillArgs &a) { return (long long)a.num_units * a.H > 3LL * kda::device_sm_count(); }
 Form choose_form(const kda::PrefillArgs &a, int path, size_t workspace_bytes, bool workspace_known) {
     if (!use_tc(a, path)) return Form::Simt;
     if (path == KDA_PATH_TC_SINGLE) return Form::Single;
     if (path == KDA_PATH_TC_SPLIT) return Form::Split;
     if (path == KDA_PATH_TC_PIPE) return Form::Pipe;
+    if (many_units(a)) return Form::Single;
     if (!workspace_known) return Form::Split;  // size queries assume the reported workspace
     if (workspace_bytes >= kda::prefill_split_workspace(a)) return Form::Split;
     if (kda::prefill_pipe_supported(a) && workspace_bytes >= kda::prefill_pipe_workspace(a)) return Form::Pipe;
@@ -110,24 +114,23 @@ const char *kda_last_cuda_error(void) {
     return e == cudaSuccess ? "none" : cudaGetErrorName(e);
 }
 
-size_t kda_forward_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int num_seqs,
-                                  int dtype) {
+size_t kda_forward_workspace_size_ex(int B, int T, int H, int dk, int dv, int chunk, int num_seqs, int dtype,
+                                     int path) {
     kda::PrefillArgs a{};
     // packed sequences (cu_seqlens) are recognised by B == 1 and num_seqs > 1
     const bool has_cu = B == 1 && num_seqs > 1;
-    if (check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, has_cu, num_seqs, KDA_PATH_AUTO, &a))
-        return (size_t)-1;
+    if (check_prefill_sizes(B, T, H, dk, dv, chunk, dtype, has_cu, num_seqs, path, &a)) return (size_t)-1;
     a.cu_seqlens = has_cu ? &kPackedMarker : nullptr;
-    size_t ws = kda::prefill_simt_workspace(a);
-    if (kda::prefill_tc_supported(dk, dv, chunk, dtype)) {
-        const size_t t = kda::prefill_tc_workspace(a);
-        const size_t sp = kda::prefill_split_workspace(a);
-        const size_t pi = kda::prefill_pipe_supported(a) ? kda::prefill_pipe_workspace(a) : 0;
-        ws = t > ws ? t : ws;
-        ws = sp > ws ? sp : ws;
-        ws = pi > ws ? pi : ws;
-    }
-    return ws;
+    const Form f = choose_form(a, path, 0, false);
+    size_t ws = form_workspace(a, f);
+    if (f == Form::Simt) return ws;
+    // the SIMT kernel is the fallback of every tensor-core form (empty batches)
+    const size_t s = kda::prefill_simt_workspace(a);
+    return s > ws ? s : ws;
+}
+
+size_t kda_forward_workspace_size(int B, int T, int H, int dk, int dv, int chunk, int num_seqs, int dtype) {
+    return kda_forward_workspace_size_ex(B, T, H, dk, dv, chunk, num_seqs, dtype, KDA_PATH_AUTO);
 }
 
 int kda_forward_launches(int B, int T, int H, int dk, int dv, int chunk, int dtype,

@@ -131,6 +131,9 @@ int prefill_pipe_launches(const PrefillArgs &a);
 
 cudaError_t launch_decode(const DecodeArgs &a);
 cudaError_t launch_decode_multi(const MultiDecodeArgs &a);
+// SMs of the current device (148 when no device answers, e.g. size queries on a host
+// without a GPU); cached after the first call
+int device_sm_count();
 // KDA_OK for cudaSuccess; otherwise KDA_ERR_CUDA, the error kept for kda_last_cuda_error
 int cuda_status(cudaError_t e);
 // KDA_OK, or the status kda_forward_ex returns for these sizes (dense batches)

@@ -1116,13 +1116,41 @@ struct RingTasks {
     }
 };
 
-// The state chain of unit c, its records read from the ring piece by piece as
-// their shared-memory tiles free up: A (state product operand, decay) once the state product
-// is done, B (Ut, P) once the output product is done, C (Kh) once the outputs staged over it
-// have left.
-__device__ __forceinline__ void chain_role(const PipeParams &pp, const CUtensorMap &tm_o, uint8_t *sm, const Group &grp,
-                                           int c) {
-    const PrefillArgs &p = pp.sp.a;
+// Where a chain's records come from. The ring (pipe form): record tau of chain c is in slot
+// tau % R once the producers have published it, and its slot is handed back once all three
+// pieces are in shared memory. The array (split form): every record is in the workspace,
+// written by an earlier kernel.
+struct RingRecords {
+    const PipeParams *pp;
+    int c;
+    __device__ const uint8_t *slot(long long tau) const {
+        return pp->ring + ((size_t)c * kRingSlots + (size_t)(tau % kRingSlots)) * REC_BYTES;
+    }
+    __device__ bool wait_ready(long long tau) const {  // thread 0
+        const bool ok = wait_counter(pp->ready + (size_t)c * kRingSlots + (size_t)(tau % kRingSlots),
+                                     (unsigned)(tau + 1), kWaitCycles);
+        fence_proxy_async_global();
+        return ok;
+    }
+    __device__ void release(long long tau) const { st_release_gpu(pp->consumed + c, (unsigned)(tau + 1)); }
+};
+struct ArrayRecords {
+    const uint8_t *rec;
+    size_t H;
+    int h;
+    long long cbase;
+    __device__ const uint8_t *slot(long long tau) const { return rec + ((size_t)(cbase + tau) * H + (size_t)h) * REC_BYTES; }
+    __device__ bool wait_ready(long long) const { return true; }
+    __device__ void release(long long) const {}
+};
+
+// The state chain of unit (sequence n, head h) with its records read piece by piece into one
+// buffer as their shared-memory tiles free up: A (state product operand, decay) once the state
+// product is done, B (Ut, P) once the output product is done, C (Kh) once the outputs staged
+// over it have left. One 256-thread group, ~106 KB of shared memory, 256 TMEM columns.
+template <class Rec>
+__device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorMap &tm_o, uint8_t *sm, const Group &grp,
+                                           int n, int h, const Rec &recs) {
     const uint32_t sbase = smem_u32(sm);
     uint64_t *bar_a = reinterpret_cast<uint64_t *>(sm + X_BAR);
     uint64_t *bar_b = bar_a + 1;
@@ -1132,7 +1160,6 @@ __device__ __forceinline__ void chain_role(const PipeParams &pp, const CUtensorM
 
     const int tid = grp.tid, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, half = warp >> 2;
-    const int n = c / p.H, h = c % p.H;
     const size_t H = (size_t)p.H;
     long long t_begin, len;
     if (p.cu_seqlens) {
@@ -1145,10 +1172,7 @@ __device__ __forceinline__ void chain_role(const PipeParams &pp, const CUtensorM
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
     const size_t state_base = ((size_t)n * H + h) * (size_t)(D * D);
     const long long nchunks = (len + C - 1) / C;
-    const unsigned *ready = pp.ready + (size_t)c * kRingSlots;
-    auto slot = [&](long long tau) -> const uint8_t * {
-        return pp.ring + ((size_t)c * kRingSlots + (size_t)(tau % kRingSlots)) * REC_BYTES;
-    };
+    auto slot = [&](long long tau) -> const uint8_t * { return recs.slot(tau); };
 
     if (tid == 0) {
         mbar_init(bar_a, 1);
@@ -1182,10 +1206,9 @@ __device__ __forceinline__ void chain_role(const PipeParams &pp, const CUtensorM
         armed |= 4u;
     };
     if (tid == 0 && nchunks > 0) {
-        if (!wait_counter(&ready[0], 1u, kWaitCycles)) {
+        if (!recs.wait_ready(0)) {
             flag_fail = true;
         } else {
-            fence_proxy_async_global();
             load_a(0);
             load_b(0);
             load_c(0);
@@ -1275,23 +1298,20 @@ __device__ __forceinline__ void chain_role(const PipeParams &pp, const CUtensorM
         if (!wait_mma()) { aborted = true; break; }
         // piece A of the next record (the state product's operand and Gamma_C are consumed)
         if (tid == 0 && more) {
-            if (!wait_counter(&ready[(tau + 1) % kRingSlots], (unsigned)(tau + 2), kWaitCycles)) {
-                flag_fail = true;
-            } else {
-                fence_proxy_async_global();
-                load_a(tau + 1);
-            }
+            if (!recs.wait_ready(tau + 1)) flag_fail = true;
+            else load_a(tau + 1);
         }
         if (!wait_piece(bar_b, ph_b, 2u)) { aborted = true; break; }
 
         // U = Ut - W S (rows 0..63) -> bf16 B operand, written over the record's Ut tile
-        if (quarter < 2) u_readout(sm + REC_UT + half * 8 * KB, 32 * quarter + lane, tmem + tlane + X_TM_U + 64u * half);
+        if (quarter < 2)
+            u_readout(sm + REC_UT + half * 8 * KB, 32 * quarter + lane, tmem + tlane + X_TM_U + 64u * half, p.v != nullptr);
         fence_proxy_async_smem();
         tc_fence_before();
         if (!wait_piece(bar_c, ph_c, 4u)) { aborted = true; break; }
         if (tid == 0) {
             // every piece of record tau is in shared memory: its slot may be refilled
-            st_release_gpu(pp.consumed + c, (unsigned)(tau + 1));
+            recs.release(tau);
             tc_fence_after();
             Opnd AK{sbase + REC_KH, true, 0, 8 * KB};
             Opnd BU{sbase + REC_UT, true, 0, 8 * KB};
@@ -1428,25 +1448,29 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const Group grp{(int)(threadIdx.x & (NT - 1)), 1u + (uint32_t)gi, false};
     const int G = gi * (int)gridDim.x + (int)blockIdx.x;
     if (G < pp.NC) {
-        chain_role(pp, tm_o, sm, grp, G);
+        const RingRecords recs{&pp, G};
+        chain_role(pp.sp.a, tm_o, sm, grp, G / pp.sp.a.H, G % pp.sp.a.H, recs);
     } else {
         RingTasks src{&pp, 0, G - pp.NC};
         prep_loop(tm_q, tm_k, tm_v, tm_g, pp.sp, src, sm, grp);
     }
 }
 
-int num_sms() {
-    static int n = 0;
-    if (n == 0) {
-        int dev = 0, v = 0;
-        if (cudaGetDevice(&dev) == cudaSuccess &&
-            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-            n = v;
-        else
-            n = 148;
-    }
-    return n;
+// The state chains over the record array with one record buffer: ~106 KB of shared memory and
+// 256 TMEM columns, so two chains share an SM (for batches of more units than SMs).
+__global__ void __launch_bounds__(NT, 2)
+kda_chain2_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const PrefillArgs &p = sp.a;
+    const int h = blockIdx.x % p.H;
+    const int n = unit_seq(p, blockIdx.x / p.H);
+    const ArrayRecords recs{sp.rec, (size_t)p.H, h, sp.chunk_base ? (long long)sp.chunk_base[n] : (long long)n * sp.nch};
+    chain_role(p, tm_o, sm, Group{(int)threadIdx.x, 0u, true}, n, h, recs);
 }
+constexpr uint32_t CHAIN2_SMEM = X_SMEM_USED + 1024;
+
+int num_sms() { return device_sm_count(); }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -1502,6 +1526,19 @@ cudaError_t launch_pipe(const PrefillArgs &a, const CUtensorMap &mq, const CUten
 }
 
 }  // namespace
+
+int device_sm_count() {
+    static int n = 0;
+    if (n == 0) {
+        int dev = 0, v = 0;
+        if (cudaGetDevice(&dev) == cudaSuccess &&
+            cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+            n = v;
+        else
+            n = 148;
+    }
+    return n;
+}
 
 size_t prefill_split_workspace(const PrefillArgs &a) {
     size_t ws = align256((size_t)split_tasks_bound(a) * REC_BYTES);
@@ -1593,7 +1630,12 @@ cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r) {
     if (tokens == 0) return launch_prefill_simt(pass);
     CUtensorMap mo;
     if (!make_map(&mo, pass.o ? pass.o : pass.q, tokens, pass.H, 64, true)) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(kda_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C_SMEM_BYTES);
+    // more units than SMs: the one-buffer chains, two per SM; otherwise the double-buffered ones
+    const bool compact = (long long)pass.num_units * pass.H > num_sms();
+    cudaError_t e = compact ? cudaFuncSetAttribute(kda_chain2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)CHAIN2_SMEM)
+                            : cudaFuncSetAttribute(kda_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   (int)C_SMEM_BYTES);
     if (e != cudaSuccess) return e;
     SplitParams sp{};
     sp.a = pass;
@@ -1604,7 +1646,14 @@ cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r) {
     sp.nch = r.nch;
     sp.tasks = r.tasks;
     const unsigned grid_c = (unsigned)((size_t)pass.num_units * pass.H);
-    kda_chain_kernel<<<grid_c, NT, C_SMEM_BYTES, pass.stream>>>(mo, sp);
+    if (compact) {
+        e = cudaFuncSetAttribute(kda_chain2_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+        kda_chain2_kernel<<<grid_c, NT, CHAIN2_SMEM, pass.stream>>>(mo, sp);
+    } else {
+        kda_chain_kernel<<<grid_c, NT, C_SMEM_BYTES, pass.stream>>>(mo, sp);
+    }
     return cudaGetLastError();
 }
 

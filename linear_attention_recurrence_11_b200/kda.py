@@ -29,6 +29,8 @@ _lib.kda_abi_version.restype = _i
 _lib.kda_last_cuda_error.restype = ctypes.c_char_p
 _lib.kda_forward_workspace_size.argtypes = [_i] * 8
 _lib.kda_forward_workspace_size.restype = _sz
+_lib.kda_forward_workspace_size_ex.argtypes = [_i] * 9
+_lib.kda_forward_workspace_size_ex.restype = _sz
 _lib.kda_forward_launches.argtypes = [_i] * 10
 _lib.kda_forward_launches.restype = _i
 _FWD = [_vp] * 8 + [_i] * 7 + [_vp, _i, _vp, _sz, _vp, _vp]
@@ -87,10 +89,11 @@ def kda_abi_version() -> int:
     return _lib.kda_abi_version()
 
 
-def kda_forward_workspace_size(B, T, H, dk, dv, chunk, num_seqs, dtype) -> int:
-    n = _lib.kda_forward_workspace_size(B, T, H, dk, dv, chunk, num_seqs, DTYPES.get(dtype, dtype))
+def kda_forward_workspace_size(B, T, H, dk, dv, chunk, num_seqs, dtype, path="auto") -> int:
+    n = _lib.kda_forward_workspace_size_ex(B, T, H, dk, dv, chunk, num_seqs, DTYPES.get(dtype, dtype), PATHS[path])
     if n == ctypes.c_size_t(-1).value:
-        raise KdaError(KDA_ERR_INVALID_ARG, "kda_forward_workspace_size")
+        raise KdaError(KDA_ERR_UNSUPPORTED if path.startswith("tc") else KDA_ERR_INVALID_ARG,
+                       "kda_forward_workspace_size")
     return int(n)
 
 
@@ -155,9 +158,10 @@ def kda_forward(q, k, v, g, beta, S0=None, *, chunk: int = 64, cu_seqlens=None, 
         S_T = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
     if S_T is not None:
         _need(S_T, "S_T", torch.float32, (N, H, dv, dk), dev)
-    ws_need = kda_forward_workspace_size(B, T, H, dk, dv, chunk, N, dtype)
-    if workspace is None and ws_need > 0:
-        workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
+    if workspace is None:
+        ws_need = _lib.kda_forward_workspace_size_ex(B, T, H, dk, dv, int(chunk), N, DTYPES[dtype], PATHS[path])
+        if ws_need not in (0, ctypes.c_size_t(-1).value):
+            workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     args = (_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o), _ptr(S_T), B, T, H, dk, dv,
             int(chunk), DTYPES[dtype], _ptr(cu_seqlens), N if cu_seqlens is not None else 0,

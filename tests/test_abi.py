@@ -120,20 +120,32 @@ def test_workspace_and_launch_queries(K):
     # tensor-core shapes: the split form's per-chunk records
     assert K.kda_forward_workspace_size(1, 8192, 96, 128, 128, 64, 1, 1) == 128 * 96 * REC
     assert K.kda_forward_workspace_size(2, 8192, 96, 128, 128, 64, 2, 1) == 2 * 128 * 96 * REC
-    # a short batch: the pipe form's ring (4 records and 5 flags per unit) is the larger need
-    assert K.kda_forward_workspace_size(2, 100, 3, 128, 128, 64, 2, 1) == \
-        max(2 * 2 * 3 * REC, al(6 * 4 * REC) + al(6 * 5 * 4))
-    # packed sequences: records for at most T / 64 + N chunks per head, the sequences' chunk
-    # offsets, and a small longest-first schedule (up to 2048 sequences)
+    assert K.kda_forward_workspace_size(2, 100, 3, 128, 128, 64, 2, 1) == 2 * 2 * 3 * REC
+    # the pipe form: a ring of 4 records and 5 flags per unit
+    assert K.kda_forward_workspace_size(2, 100, 3, 128, 128, 64, 2, 1, "tc_pipe") == \
+        al(6 * 4 * REC) + al(6 * 5 * 4)
+    assert K.kda_forward_workspace_size(2, 100, 3, 128, 128, 64, 2, 1, "tc_single") == 0
+    # packed sequences, up to three units per SM: records for at most T / 64 + N chunks per
+    # head, the sequences' chunk offsets, and a small longest-first schedule (up to 2048)
+    n_ch = -(-100000 // 64) + 3
+    assert K.kda_forward_workspace_size(1, 100000, 96, 128, 128, 64, 3, 1) == \
+        al(n_ch * 96 * REC) + al(4 * 4) + 256
+    # more units than three per SM (8 x 96 = 768): AUTO runs the single form (its schedule only);
+    # a forced split form still reports its records
     n_ch = -(-352549 // 64) + 8
-    assert K.kda_forward_workspace_size(1, 352549, 96, 128, 128, 64, 8, 1) == \
+    assert K.kda_forward_workspace_size(1, 352549, 96, 128, 128, 64, 8, 1) == 256
+    assert K.kda_forward_workspace_size(1, 352549, 96, 128, 128, 64, 8, 1, "tc_split") == \
         al(n_ch * 96 * REC) + al(9 * 4) + 256
+    with pytest.raises(K.KdaError):
+        K.kda_forward_workspace_size(1, 352549, 96, 128, 128, 64, 8, 1, "tc_pipe")
     # other shapes (SIMT kernel): only the schedule
     assert K.kda_forward_workspace_size(1, 100000, 2, 64, 64, 32, 2048, 0) == 8192
     assert K.kda_forward_workspace_size(1, 100000, 2, 64, 64, 32, 2049, 0) == 0
     # launches: split = records + chains (+ chunk offsets and schedule for packed batches);
     # pipe = one launch, only for up to 197 units on 148 SMs
-    assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8) == 4
+    assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8) == 2
+    assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8, "tc_split") == 4
+    assert K.kda_forward_launches(1, 100000, 96, 128, 128, 64, 1, 1, 3) == 4
     assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8, "tc_single") == 2
     assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8, "simt") == 2
     assert K.kda_forward_launches(1, 352549, 96, 128, 128, 64, 1, 1, 8, "tc_pipe") == -1
@@ -196,8 +208,7 @@ def test_segmented_queries(K):
     n2 = K.kda_forward_segmented_workspace_size(1, 1000, 2, 64, 128, 64, 1, 256)
     assert n2 >= 4 * 2 * (64 * 64 + 2 * 128 * 64) * 4
     # one segment: the plain prefill's needs (the split form's records for a dense batch)
-    assert K.kda_forward_segmented_workspace_size(2, 1000, 2, 128, 128, 64, 1, 1024) == \
-        max(2 * 16 * 2 * REC, al(4 * 4 * REC) + al(4 * 5 * 4))
+    assert K.kda_forward_segmented_workspace_size(2, 1000, 2, 128, 128, 64, 1, 1024) == 2 * 16 * 2 * REC
     assert K.kda_forward_segmented_launches(2, 1000, 2, 128, 128, 64, 1, 1024) == 2
     # tensor-core shapes: init, chunk offsets, schedule, records, three chain passes, scan
     assert K.kda_forward_segmented_launches(1, 1000, 2, 128, 128, 64, 1, 256) == 8

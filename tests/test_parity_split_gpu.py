@@ -119,7 +119,7 @@ def test_split_two_calls_reuse_workspace(K, oracle_mod, form):
     """The records are scratch: a second call with other inputs in the same workspace gives
     its own results (every record is rewritten before it is read, the ring's flags are
     reset by every call)."""
-    ws = torch.empty(K.kda_forward_workspace_size(2, 256, 2, 128, 128, 64, 2, torch.bfloat16),
+    ws = torch.empty(K.kda_forward_workspace_size(2, 256, 2, 128, 128, 64, 2, torch.bfloat16, path=form),
                      dtype=torch.uint8, device="cuda")
     for seed in (1, 2):
         inp = case(2, 256, 2, 128, 128, "bf16", seed=seed, s0_std=0.1)
