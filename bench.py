@@ -612,6 +612,19 @@ def multi_decode_measure(args, device, peaks, max_ranks, world, w, S, rounds=10)
     b.record(stream)
     torch.cuda.synchronize(device)
     ms = max_ranks(a.elapsed_time(b)) / rounds
+    # each call alone: the verification (repeatable, states untouched), then the commit
+    parts = {}
+    for name, call in (("verify", lambda: kda.kda_decode_multi(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                                                               S, o, n_accept=zeros)),
+                       ("commit", lambda: kda.kda_decode_multi(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"],
+                                                               S, None, n_accept=acc, outputs=False))):
+        torch.cuda.synchronize(device)
+        a.record(stream)
+        for _ in range(rounds):
+            call()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        parts[name + "_ms"] = max_ranks(a.elapsed_time(b)) / rounds
     accepted = int(acc.sum().item())
     bytes_round = multi_decode_algorithmic(w.B, w.H, T, w.dk, w.dv, acc.tolist())
     gbs = bytes_round / (ms / 1e3) / 1e9
@@ -620,7 +633,7 @@ def multi_decode_measure(args, device, peaks, max_ranks, world, w, S, rounds=10)
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "kernel": "kda_decode_multi.cu",
                          "algorithmic_bytes_per_round": bytes_round, "peak_source": peaks["source"] + " (hbm_gbs)"},
-            "gpu_launches": 2 * rounds,
+            **parts, "gpu_launches": 2 * rounds,
             "note": "per round: verify (outputs of all draft tokens) + commit (accepted prefixes); "
                     "kda_decode_step would move the state twice per accepted token instead"}
 

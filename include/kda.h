@@ -365,6 +365,10 @@ int kda_decode_step_fused(const void *q, const void *k, const void *v, const voi
  * once and written at most once, whatever T is.
  * Typical use: verify T draft tokens with n_accept all zero (outputs only),
  * then commit with the accepted counts and o = NULL.
+ * A request with outputs and nothing accepted, T <= 16, is computed in the
+ * chunked form ("Exercices", Q21-Q22, applied to the T tokens): two dot
+ * products per token with every state column, then a T x T triangular
+ * system per column; the results equal the sequential steps' up to rounding.
  *
  *   q, k, g : [N, T, H, dk];  v, o : [N, T, H, dv];  beta : [N, T, H]   (dtype)
  *   S        : [N, H, dv, dk] fp32, read, and written where n_accept > 0.

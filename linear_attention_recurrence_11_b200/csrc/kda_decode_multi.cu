@@ -27,6 +27,21 @@
 // are collected there and written as contiguous rows at the end. Without
 // outputs (o = NULL) only the first n_acc tokens are applied, and a request
 // with n_acc = 0 reads nothing.
+//
+// A verification (outputs of all T tokens, n_acc = 0, T <= kVerifyMaxT) does
+// not need the intermediate states at all. With G_t the cumulative log-decay
+// up to token t, the decayed state seen by token t is
+//   S'_t = Diag(e^{G_t}) S + sum_{tau < t} Diag(e^{G_t - G_tau}) k_tau u_tau^T,
+// so per column j of S, with a_t = (e^{G_t} k_t)^T S[:, j] and
+// b_t = (e^{G_t} q_t)^T S[:, j],
+//   u_t[j] = beta_t (v_t[j] - a_t - sum_{tau < t} A_{t tau} u_tau[j]),
+//   o_t[j] = b_t + sum_{tau < t} P_{t tau} u_tau[j] + u_t[j] (k_t^T q_t),
+// A_{t tau} = sum_i k_t[i] k_tau[i] e^{G_t[i] - G_tau[i]} and P likewise with
+// q_t: the chunked form of the recurrence ("Exercices", Q21-Q22) applied to the
+// T draft tokens. Each state element then takes 2T multiply-adds (two dot
+// products per token, no dependency between tokens) instead of the four
+// operations of a sequential step, and the T x T systems are solved per column
+// after the state has streamed through.
 #include "kda_internal.cuh"
 #include "kda_sm100.cuh"
 
@@ -41,6 +56,9 @@ constexpr int kMtRowsPerPass = (kMtThreads / 32) * (32 / kMtLanesPerRow);  // 16
 constexpr int kMtRowsInFlight = 2;
 constexpr int kMtCols = kMtRowsPerPass * kMtRowsInFlight;                  // 32 columns per pass
 constexpr long long kMtWaitCycles = 2000000000LL;                          // ~1 s at 2 GHz
+constexpr int kVerifyMaxT = 16;  // verifications of up to this many tokens take the chunked form
+constexpr int kVerifyGroup = 4;  // tokens per sweep over the columns held in registers
+static_assert(kMtRowsInFlight * 2 * kVerifyGroup == 16 && kMtLanesPerRow == 8, "reduce_scatter8 layout");
 
 // 16 bytes of elements -> floats (8 bf16 or 4 fp32)
 __device__ __forceinline__ void unpack16(const uint4 &r, float (&x)[8]) {
@@ -55,6 +73,23 @@ __device__ __forceinline__ void unpack16(const uint4 &r, float (&x)[8]) {
 __device__ __forceinline__ void unpack16(const uint4 &r, float (&x)[4]) {
     x[0] = __uint_as_float(r.x); x[1] = __uint_as_float(r.y);
     x[2] = __uint_as_float(r.z); x[3] = __uint_as_float(r.w);
+}
+
+// Sums of 16 values over the 8 lanes of a column group (xor 4, 2, 1), scattered: the lane whose
+// index in the group has bits b2 b1 b0 ends with the complete sums of entries
+// 8 b2 + 4 b1 + 2 b0 + {0, 1} in y[0], y[1] (14 shuffles instead of 48).
+__device__ __forceinline__ void reduce_scatter8(const float (&v)[16], float (&y)[2], int sub) {
+    const bool u4 = sub & 4, u2 = sub & 2, u1 = sub & 1;
+    float w[8], x[4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        w[i] = (u4 ? v[i + 8] : v[i]) + __shfl_xor_sync(0xffffffffu, u4 ? v[i] : v[i + 8], 4);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        x[i] = (u2 ? w[i + 4] : w[i]) + __shfl_xor_sync(0xffffffffu, u2 ? w[i] : w[i + 4], 2);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        y[i] = (u1 ? x[i + 2] : x[i]) + __shfl_xor_sync(0xffffffffu, u1 ? x[i] : x[i + 2], 1);
 }
 
 template <typename Tin, int DK, int DV>
@@ -82,6 +117,7 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
     int n_acc = p.n_accept ? p.n_accept[n] : T;
     n_acc = n_acc < 0 ? 0 : (n_acc > T ? T : n_acc);
     const int t_end = o ? T : n_acc;  // tokens whose effect is needed
+    const bool verify = o != nullptr && n_acc == 0 && T <= kVerifyMaxT;  // the chunked form
     float *Su = p.S + unit * (size_t)DV * DK;
     if (t_end > 0 && tid == 0) {  // the first two passes' columns -> shared memory
         mbar_init(&bar[0], 1);
@@ -127,7 +163,7 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
                 if (base + u * kMtThreads >= total) continue;
                 float x[VEC];
                 unpack16(raw[u], x);
-                if (is_g[u]) {
+                if (is_g[u] && !verify) {  // the chunked form keeps g and sums it
 #pragma unroll
                     for (int e = 0; e < VEC; ++e) x[e] = __expf(x[e]);
                 }
@@ -138,8 +174,55 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
         }
         if (tid < t_end) sIn[tid * TOK + 3 * DK + DV] = ld_elem(beta, ((size_t)n * T + tid) * H + h);
     }
-    float *sOut = sIn + T * TOK;
+    float *sOut = sIn + T * TOK;  // outputs [T][DV]; the chunked form first keeps b_t there
+    float *sA0 = sOut + T * DV;   // chunked form: a_t [T][DV], then A and P [T][T] each
+    float *sAm = sA0 + T * DV, *sPm = sAm + T * T;
     __syncthreads();
+    if (verify) {
+        // G_t (cumulative log-decay, in place of g), then A and P (P_tt = k_t^T q_t), then the
+        // decayed e^{G_t} q_t, e^{G_t} k_t in place of q_t, k_t
+        for (int i = tid; i < DK; i += kMtThreads) {
+            float acc = 0.f;
+            for (int t = 0; t < T; ++t) {
+                acc += sIn[t * TOK + 2 * DK + i];
+                sIn[t * TOK + 2 * DK + i] = acc;
+            }
+        }
+        __syncthreads();
+        int pidx = 0;
+        for (int t = 0; t < T; ++t) {
+            const float *it = sIn + t * TOK;
+            for (int tau = 0; tau <= t; ++tau, ++pidx) {
+                if ((pidx & 3) != warp) continue;
+                const float *iu = sIn + tau * TOK;
+                float sa = 0.f, sp = 0.f;
+#pragma unroll
+                for (int i = lane; i < DK; i += 32) {
+                    const float w = tau == t ? iu[DK + i] : iu[DK + i] * __expf(it[2 * DK + i] - iu[2 * DK + i]);
+                    sa = fmaf(it[DK + i], w, sa);
+                    sp = fmaf(it[i], w, sp);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    sa += __shfl_xor_sync(0xffffffffu, sa, off);
+                    sp += __shfl_xor_sync(0xffffffffu, sp, off);
+                }
+                if (lane == 0) {
+                    sAm[t * T + tau] = sa;
+                    sPm[t * T + tau] = sp;
+                }
+            }
+        }
+        __syncthreads();
+        for (int idx = tid; idx < T * DK; idx += kMtThreads) {
+            const int t = idx / DK, i = idx % DK;
+            float *it = sIn + t * TOK;
+            const float e = __expf(it[2 * DK + i]);
+            it[i] *= e;
+            it[DK + i] *= e;
+        }
+        __syncthreads();
+    }
 
     int pass = 0;
     bool ok = true;
@@ -161,6 +244,56 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
             fence_proxy_async_smem();
             mbar_arrive_expect_tx(&bar[b], kPassBytes);
             bulk_load(sBuf + b * kMtCols * DK, Su + (size_t)(pass + 2) * kMtCols * DK, kPassBytes, &bar[b]);
+        }
+        if (verify) {
+            // a_t, b_t of this pass's columns, kVerifyGroup tokens per sweep over the registers
+            for (int t0 = 0; t0 < T; t0 += kVerifyGroup) {
+                float2 acc[kMtRowsInFlight][2][kVerifyGroup];
+#pragma unroll
+                for (int r = 0; r < kMtRowsInFlight; ++r)
+#pragma unroll
+                    for (int w = 0; w < 2; ++w)
+#pragma unroll
+                        for (int t4 = 0; t4 < kVerifyGroup; ++t4) acc[r][w][t4] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int t4 = 0; t4 < kVerifyGroup; ++t4) {
+                    if (t0 + t4 >= T) break;
+                    const float *in = sIn + (t0 + t4) * TOK;
+#pragma unroll
+                    for (int m = 0; m < F4; ++m) {
+                        const int c = 4 * (sub + kMtLanesPerRow * m);
+                        const float4 qd = *reinterpret_cast<const float4 *>(in + c);
+                        const float4 kd = *reinterpret_cast<const float4 *>(in + DK + c);
+#pragma unroll
+                        for (int r = 0; r < kMtRowsInFlight; ++r) {
+                            const float2 x0 = make_float2(s[r][m].x, s[r][m].y);
+                            const float2 x1 = make_float2(s[r][m].z, s[r][m].w);
+                            acc[r][0][t4] = __ffma2_rn(x0, make_float2(kd.x, kd.y), acc[r][0][t4]);
+                            acc[r][0][t4] = __ffma2_rn(x1, make_float2(kd.z, kd.w), acc[r][0][t4]);
+                            acc[r][1][t4] = __ffma2_rn(x0, make_float2(qd.x, qd.y), acc[r][1][t4]);
+                            acc[r][1][t4] = __ffma2_rn(x1, make_float2(qd.z, qd.w), acc[r][1][t4]);
+                        }
+                    }
+                }
+                float v16[16];
+#pragma unroll
+                for (int r = 0; r < kMtRowsInFlight; ++r)
+#pragma unroll
+                    for (int w = 0; w < 2; ++w)
+#pragma unroll
+                        for (int t4 = 0; t4 < kVerifyGroup; ++t4)
+                            v16[8 * r + 4 * w + t4] = acc[r][w][t4].x + acc[r][w][t4].y;
+                float y[2];
+                reduce_scatter8(v16, y, sub);
+                const int r = (sub >> 2) & 1, w = (sub >> 1) & 1;
+                const int j = pass * kMtCols + warp * (32 / kMtLanesPerRow) + rw + r * kMtRowsPerPass;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    const int t = t0 + 2 * (sub & 1) + i;
+                    if (t < T) (w ? sOut : sA0)[t * DV + j] = y[i];
+                }
+            }
+            continue;
         }
         for (int t = 0; t < t_end; ++t) {
             const float *in = sIn + t * TOK;
@@ -243,6 +376,25 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
         }
         return;
     }
+    if (verify) {  // the T x T systems, one column per thread
+        __syncthreads();
+        for (int j = tid; j < DV; j += kMtThreads) {
+            float u[kVerifyMaxT];
+#pragma unroll
+            for (int t = 0; t < kVerifyMaxT; ++t) {
+                if (t >= T) break;
+                const float *in = sIn + t * TOK;
+                float a = sA0[t * DV + j], b = sOut[t * DV + j];
+#pragma unroll
+                for (int tau = 0; tau < t; ++tau) {
+                    a = fmaf(sAm[t * T + tau], u[tau], a);
+                    b = fmaf(sPm[t * T + tau], u[tau], b);
+                }
+                u[t] = in[3 * DK + DV] * (in[3 * DK + j] - a);
+                sOut[t * DV + j] = fmaf(u[t], sPm[t * T + t], b);
+            }
+        }
+    }
     if (o) {  // outputs, one contiguous dv row per token
         __syncthreads();
         for (int idx = tid; idx < T * DV; idx += kMtThreads) {
@@ -255,7 +407,8 @@ __global__ void __launch_bounds__(kMtThreads) kda_decode_multi_kernel(const Mult
 template <typename Tin, int DK, int DV>
 cudaError_t launch_mt(const MultiDecodeArgs &a) {
     const size_t smem = 2 * (size_t)kMtCols * DK * sizeof(float) + 16 +
-                        (size_t)a.T * (3 * DK + DV + 4 + DV) * sizeof(float);
+                        (size_t)a.T * (3 * DK + DV + 4 + DV) * sizeof(float) +
+                        (a.T <= kVerifyMaxT ? (size_t)a.T * (DV + 2 * a.T) * sizeof(float) : 0);
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kda_decode_multi_kernel<Tin, DK, DV>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -104,3 +104,28 @@ def test_commit_without_outputs_equals_the_full_call(K):
     assert K.kda_decode_multi(*args, S2, n_accept=acc, outputs=False, dev_status=status) is None
     torch.cuda.synchronize()
     assert torch.equal(S1, S2) and int(status[0]) == 0
+
+
+@pytest.mark.parametrize("dtype,dk,dv,T", [("bf16", 128, 128, 1), ("bf16", 128, 128, 2), ("f32", 128, 128, 5),
+                                           ("bf16", 64, 128, 7), ("f32", 32, 32, 13), ("bf16", 128, 64, 16),
+                                           ("f32", 64, 64, 16), ("bf16", 128, 128, 17)])
+def test_verification_form(K, oracle_mod, dtype, dk, dv, T):
+    """Verification calls (outputs of all T tokens, nothing accepted): up to 16 tokens they
+    take the chunked form (dot products of every state column with the decayed k_t and
+    q_t, then T x T systems per column), beyond it the sequential steps; both against the
+    oracle's sequential steps, with g at g_min on whole channels, and the states untouched."""
+    N, H = 5, 3
+    inp = make_inputs(N, T, H, dk, dv, dtype, seed=7 * T + dk + dv, device="cuda")
+    g = inp["g"].clone()
+    g[..., : dk // 4] = -5.0
+    inp["g"] = g
+    S = (0.05 * torch.randn(N, H, dv, dk, generator=torch.Generator().manual_seed(T + 100))).cuda()
+    S_before = S.clone()
+    zeros = np.zeros(N, dtype=np.int32)
+    o_ref, _ = oracle_multi(oracle_mod, inp, S, zeros)
+    o = K.kda_decode_multi(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], S,
+                           n_accept=torch.tensor(zeros, device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.equal(S, S_before)
+    worst = max(rel(to_f64(o[n, :, h]), o_ref[n, :, h]) for n in range(N) for h in range(H))
+    assert worst < TOL[dtype], worst
