@@ -430,6 +430,20 @@ def varlen_measure(args, device, peaks, barrier, max_ranks, world, rank):
         kda.kda_forward(sl["q"], sl["k"], sl["v"], sl["g"], sl["beta"], None, chunk=w.chunk, o=o1, S_T=ST1,
                         workspace=ws1, path=args.path)
     ms_long = timed(longest, K)
+    del o1, ST1, ws1, sl
+    # the same batch through the segment-parallel prefill (sequences cut every seg_len
+    # tokens; the short ones stay one segment each)
+    seg_len = 16384
+    wss = torch.empty(max(1, kda.kda_forward_segmented_varlen_workspace_size(T, w.H, w.dk, w.dv, w.chunk, dt, N,
+                                                                             seg_len)),
+                      dtype=torch.uint8, device=device)
+
+    def segmented():
+        kda.kda_forward_segmented(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], seg_len=seg_len,
+                                  chunk=w.chunk, cu_seqlens=inp["cu_seqlens"], o=o, S_T=ST, workspace=wss,
+                                  path=args.path)
+    ms_seg = timed(segmented, 3)
+    del wss
     alg_bytes, alg_flops = prefill_algorithmic(w, dt.itemsize)
     gbs = alg_bytes / (ms / 1e3) / 1e9
     return {"workload": w.name, "tokens": T, "sequences": N, "lengths": list(w.seqlens),
@@ -441,6 +455,11 @@ def varlen_measure(args, device, peaks, barrier, max_ranks, world, rank):
             "longest_sequence": {"tokens": w.seqlens[nl], "ms": ms_long, "ratio_to_batch": ms_long / ms,
                                  "note": "the longest sequence alone (all 96 heads) through kda_forward; "
                                          "near 1 means the batch is bound by that sequence's chain"},
+            "segmented": {"seg_len": seg_len, "ms_per_step": ms_seg, "tokens_per_s": world * T / (ms_seg / 1e3),
+                          "launches": kda.kda_forward_segmented_varlen_launches(T, w.H, w.dk, w.dv, w.chunk, dt, N,
+                                                                                seg_len, args.path),
+                          "note": "kda_forward_segmented with cu_seqlens: segment pairs, scan, replay; three "
+                                  "passes over the inputs, outside the leg's timed steps"},
             "gpu_launches": K * kda.kda_forward_launches(1, T, w.H, w.dk, w.dv, w.chunk, dt, True, N, args.path),
             "steps": K, "clocks": clk.summary(),
             "l2": f"inputs larger than L2 ({4 * inp['q'].numel() * dt.itemsize / 1e9:.1f} GB read per step)"}

@@ -312,6 +312,33 @@ int kda_forward_segmented(const void *q, const void *k, const void *v, const voi
                           void *stream, int path);
 
 /*
+ * kda_forward_segmented for a packed batch (the cu_seqlens layout of kda_forward:
+ * q, k, g [1, T, H, dk], v, o [1, T, H, dv], beta [1, T, H], num_seqs sequences
+ * at device offsets cu_seqlens[0..num_seqs], S0 / S_T [num_seqs, H, dv, dk]).
+ * Every sequence longer than seg_len is cut into ceil(len / seg_len) segments
+ * starting at multiples of seg_len from its first token; shorter ones (empty
+ * ones included) are one segment each and go through the same passes as
+ * ordinary units. The segment table is built on the device from cu_seqlens
+ * (the lengths need not be known on the host): the workspace is sized for the
+ * bound T / seg_len + num_seqs on the number of segments. With T <= seg_len
+ * no sequence is cut and the call is kda_forward_ex with cu_seqlens.
+ *
+ *   seg_len : tokens per segment, a positive multiple of chunk.
+ *   workspace / workspace_bytes : at least
+ *             kda_forward_segmented_varlen_workspace_size(...) bytes.
+ *   path    : kda_path, as in kda_forward_ex.
+ * Other arguments, results and errors as kda_forward with cu_seqlens.
+ */
+size_t kda_forward_segmented_varlen_workspace_size(int T, int H, int dk, int dv, int chunk, int dtype, int num_seqs,
+                                                   int seg_len);
+int kda_forward_segmented_varlen_launches(int T, int H, int dk, int dv, int chunk, int dtype, int num_seqs,
+                                          int seg_len, int path);
+int kda_forward_segmented_varlen(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                                 const float *S0, void *o, float *S_T, int T, int H, int dk, int dv, int chunk,
+                                 int dtype, const int32_t *cu_seqlens, int num_seqs, int seg_len, void *workspace,
+                                 size_t workspace_bytes, int *dev_status, void *stream, int path);
+
+/*
  * One decode step: one new token for each of N requests, states in place.
  * Same recurrence with T = 1 ("Exercices", Q4: decode is bound by memory
  * bandwidth; each state is read and written exactly once).

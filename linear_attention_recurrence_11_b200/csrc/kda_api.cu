@@ -247,7 +247,31 @@ int check_segmented(int B, int T, int H, int dk, int dv, int chunk, int dtype, i
     }
     *s = kda::SegmentedArgs{};
     s->B = B; s->T = T; s->H = H; s->dk = dk; s->dv = dv; s->chunk = chunk; s->dtype = dtype;
-    s->seg_len = seg_len; s->P = (int)P;
+    s->seg_len = seg_len; s->P = (int)P; s->units = B * (int)P;
+    *tc_pair = path != KDA_PATH_SIMT && kda::prefill_tc_supported(dk, dk, chunk, dtype);
+    *tc_state = path != KDA_PATH_SIMT && kda::prefill_tc_supported(dk, dv, chunk, dtype);
+    return KDA_OK;
+}
+
+// The same for packed batches: num_seqs sequences over T tokens in all. *cut is false when no
+// sequence can be longer than seg_len (T <= seg_len): the call is then kda_forward_ex.
+int check_segmented_varlen(int T, int H, int dk, int dv, int chunk, int dtype, int num_seqs, int seg_len,
+                           int path, kda::SegmentedArgs *s, bool *tc_pair, bool *tc_state, bool *cut) {
+    kda::PrefillArgs a{};
+    int st = check_prefill_sizes(1, T, H, dk, dv, chunk, dtype, true, num_seqs, path, &a);
+    if (st) return st;
+    if (seg_len <= 0 || seg_len % chunk != 0) return KDA_ERR_INVALID_ARG;
+    *cut = T > seg_len;
+    const long long units = (long long)T / seg_len + num_seqs;  // bound on the number of segments
+    if (*cut) {
+        if (units >= 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+        if ((size_t)units * (size_t)H * (size_t)(dv > dk ? dv : dk) / 32 > 0x7fffffffu) return KDA_ERR_UNSUPPORTED;
+        if (path >= KDA_PATH_TC && !kda::prefill_tc_supported(dk, dk, chunk, dtype)) return KDA_ERR_UNSUPPORTED;
+    }
+    *s = kda::SegmentedArgs{};
+    s->B = num_seqs; s->T = T; s->H = H; s->dk = dk; s->dv = dv; s->chunk = chunk; s->dtype = dtype;
+    s->seg_len = seg_len; s->P = 0; s->units = (int)units;
+    s->cu_seqlens = &kPackedMarker;  // replaced by the caller's offsets in the call itself
     *tc_pair = path != KDA_PATH_SIMT && kda::prefill_tc_supported(dk, dk, chunk, dtype);
     *tc_state = path != KDA_PATH_SIMT && kda::prefill_tc_supported(dk, dv, chunk, dtype);
     return KDA_OK;
@@ -288,6 +312,50 @@ int kda_forward_segmented(const void *q, const void *k, const void *v, const voi
                           (const void *)workspace, (const void *)dev_status})
         if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
     s.q = q; s.k = k; s.v = v; s.g = g; s.beta = beta; s.S0 = S0; s.o = o; s.ST = S_T;
+    s.workspace = workspace; s.workspace_bytes = workspace_bytes; s.dev_status = dev_status;
+    s.stream = static_cast<cudaStream_t>(stream);
+    if (workspace == nullptr || workspace_bytes < kda::segmented_workspace(s)) return KDA_ERR_WORKSPACE;
+    return kda::cuda_status(kda::launch_segmented(s, tc_pair, tc_state));
+}
+
+size_t kda_forward_segmented_varlen_workspace_size(int T, int H, int dk, int dv, int chunk, int dtype, int num_seqs,
+                                                   int seg_len) {
+    kda::SegmentedArgs s;
+    bool tp, ts, cut;
+    if (check_segmented_varlen(T, H, dk, dv, chunk, dtype, num_seqs, seg_len, KDA_PATH_AUTO, &s, &tp, &ts, &cut))
+        return (size_t)-1;
+    if (!cut) return kda_forward_workspace_size(1, T, H, dk, dv, chunk, num_seqs, dtype);
+    return kda::segmented_workspace(s);
+}
+
+int kda_forward_segmented_varlen_launches(int T, int H, int dk, int dv, int chunk, int dtype, int num_seqs,
+                                          int seg_len, int path) {
+    kda::SegmentedArgs s;
+    bool tp, ts, cut;
+    if (check_segmented_varlen(T, H, dk, dv, chunk, dtype, num_seqs, seg_len, path, &s, &tp, &ts, &cut)) return -1;
+    if (!cut) return kda_forward_launches(1, T, H, dk, dv, chunk, dtype, 1, num_seqs, path);
+    return kda::segmented_launches(s);
+}
+
+int kda_forward_segmented_varlen(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                                 const float *S0, void *o, float *S_T, int T, int H, int dk, int dv, int chunk,
+                                 int dtype, const int32_t *cu_seqlens, int num_seqs, int seg_len, void *workspace,
+                                 size_t workspace_bytes, int *dev_status, void *stream, int path) {
+    kda::SegmentedArgs s;
+    bool tc_pair, tc_state, cut;
+    int st = check_segmented_varlen(T, H, dk, dv, chunk, dtype, num_seqs, seg_len, path, &s, &tc_pair, &tc_state,
+                                    &cut);
+    if (st) return st;
+    if (!cu_seqlens) return KDA_ERR_INVALID_ARG;
+    if (!cut)  // no sequence is longer than a segment: the plain prefill
+        return kda_forward_ex(q, k, v, g, beta, S0, o, S_T, 1, T, H, dk, dv, chunk, dtype, cu_seqlens, num_seqs,
+                              workspace, workspace_bytes, dev_status, stream, path);
+    if (!q || !k || !v || !g || !beta || !o) return KDA_ERR_INVALID_ARG;
+    for (const void *p : {q, k, v, g, beta, (const void *)S0, (const void *)o, (const void *)S_T,
+                          (const void *)workspace, (const void *)dev_status})
+        if (!aligned16(p)) return KDA_ERR_ALIGNMENT;
+    s.q = q; s.k = k; s.v = v; s.g = g; s.beta = beta; s.S0 = S0; s.o = o; s.ST = S_T;
+    s.cu_seqlens = cu_seqlens;
     s.workspace = workspace; s.workspace_bytes = workspace_bytes; s.dev_status = dev_status;
     s.stream = static_cast<cudaStream_t>(stream);
     if (workspace == nullptr || workspace_bytes < kda::segmented_workspace(s)) return KDA_ERR_WORKSPACE;

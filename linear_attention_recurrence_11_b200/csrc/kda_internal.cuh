@@ -45,6 +45,10 @@ struct SegmentedArgs {
     size_t workspace_bytes;
     int *dev_status;
     cudaStream_t stream;
+    // kda_forward_segmented_varlen: B = num_seqs packed sequences (device offsets) over T tokens
+    // in all, every one cut into max(1, ceil(len / seg_len)) segments; P is unused
+    const int32_t *cu_seqlens = nullptr;
+    int units = 0;  // segment slots: B * P for dense batches, T / seg_len + B for packed ones
 };
 
 struct DecodeArgs {
@@ -104,7 +108,9 @@ cudaError_t launch_segmented(const SegmentedArgs &s, bool tc_pair, bool tc_state
 // one segment per sequence: M [B, H, dk, dk] (from the identity, zero values), Z [B, H, dv, dk] (from 0)
 cudaError_t launch_segment_pair(const SegmentedArgs &s, float *M, float *Z, bool tc_pair, bool tc_state);
 // s.S0 / s.ST / s.B / s.P / s.H / s.dk / s.dv / s.stream: incoming states of P segments per sequence
-cudaError_t launch_kcp_scan(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin);
+// (seg_base non-null: sequence b has the segments seg_base[b] .. seg_base[b + 1] - 1)
+cudaError_t launch_kcp_scan(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin,
+                            const int32_t *seg_base = nullptr);
 cudaError_t launch_prefill_tc(const PrefillArgs &a);
 size_t prefill_tc_workspace(const PrefillArgs &a);
 int prefill_tc_launches(const PrefillArgs &a);

@@ -14,11 +14,13 @@
 //   scan    S_in,0 = S0, S_in,p+1 = M_p S_in,p + S~_p (fp32, one CTA per
 //           (sequence, head), sequential over segments; the last one is S_T);
 //   pass C  the recurrence run over every segment from S_in,p, writing o.
-// On the tensor-core shapes (bf16, dk = dv = 128, chunks of 64) the state-independent
-// part of every chunk is computed once, as the split prefill's records, and passes
-// A-C are three runs of its state-chain kernel over them (pass A leaves the records'
-// Ut out); elsewhere passes A-C are the ordinary prefill kernels over the segments
-// laid out as packed sequences. M_p is a dk x dk matrix kept in the state layout
+// On the tensor-core shapes (bf16, dk = dv = 128, chunks of 64) with at most three
+// (segment, head) units per SM, the state-independent part of every chunk is computed
+// once, as the split prefill's records, and passes A-C are three runs of its
+// state-chain kernel over them (pass A leaves the records' Ut out); elsewhere passes
+// A-C are the ordinary prefill kernels over the segments laid out as packed sequences.
+// Packed batches (cu_seqlens) are planned on the device: every sequence is cut into
+// max(1, ceil(len / seg_len)) segments and the scan walks each sequence's own count. M_p is a dk x dk matrix kept in the state layout
 // ([column][dk], so pass A runs with dv = dk).
 #include "kda_internal.cuh"
 #include "kda_sm100.cuh"
@@ -28,11 +30,11 @@ namespace {
 
 constexpr int kSegThreads = 256;
 
-// cu_seg[u] for the B * P segments (segment p of sequence b is unit b * P + p) and the
-// identity as the starting "state" of pass A, [B * P, H, dk, dk] in the state layout.
-__global__ void kda_segment_init_kernel(int32_t *cu_seg, float *Mbuf, int B, int T, int P, int seg_len,
-                                        int H, int dk) {
-    const int units = B * P;
+// cu_seg[u] for the B * P segments of a dense batch (segment p of sequence b is unit b * P + p;
+// cu_seg null: none) and the identity as the starting "state" of pass A, [units, H, dk, dk] in
+// the state layout.
+__global__ void kda_segment_init_kernel(int32_t *cu_seg, float *Mbuf, int units, int B, int T, int P,
+                                        int seg_len, int H, int dk) {
     const size_t gid = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
     const size_t stride = (size_t)gridDim.x * blockDim.x;
     for (size_t u = gid; cu_seg && u <= (size_t)units; u += stride) {
@@ -48,6 +50,59 @@ __global__ void kda_segment_init_kernel(int32_t *cu_seg, float *Mbuf, int B, int
         const size_t e = i % ((size_t)dk * dk);
         Mbuf[i] = (e / dk == e % dk) ? 1.f : 0.f;
     }
+}
+
+// The segments of a packed batch (one block): sequence n of length len_n gets
+// P_n = max(1, ceil(len_n / seg_len)) segments, seg_base[n] = sum of P_m over m < n, and
+// segment p of it starts at cu[n] + p seg_len (the last ends at cu[n + 1]; an empty sequence is
+// one empty segment). The units past the last segment, up to `units`, are empty segments at the
+// end of the token axis. units >= seg_base[num] holds because P_n <= len_n / seg_len + 1.
+__global__ void kda_segment_plan_kernel(const int32_t *cu, int num, int seg_len, int units, int32_t *seg_base,
+                                        int32_t *cu_seg) {
+    __shared__ int32_t warp_sums[32];
+    __shared__ int32_t carry_s;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
+    if (tid == 0) carry_s = 0;
+    __syncthreads();
+    for (int start = 0; start < num; start += blockDim.x) {
+        const int i = start + tid;
+        int v = 0;
+        if (i < num) {
+            const int len = cu[i + 1] - cu[i];
+            v = len > seg_len ? (len + seg_len - 1) / seg_len : 1;
+        }
+        int x = v;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_sums[wid] = x;
+        __syncthreads();
+        if (wid == 0) {
+            int w = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, w, o);
+                if (lane >= o) w += y;
+            }
+            warp_sums[lane] = w;
+        }
+        __syncthreads();
+        const int carry = carry_s;
+        const int incl = carry + (wid ? warp_sums[wid - 1] : 0) + x;
+        if (i < num) {  // clamped to the slots, should offsets past the token count ever arrive
+            const int first = min(incl - v, units), last = min(incl, units);
+            seg_base[i] = first;
+            for (int u = first; u < last; ++u) cu_seg[u] = cu[i] + (u - first) * seg_len;
+        }
+        __syncthreads();
+        if (tid == blockDim.x - 1) carry_s = incl;
+        __syncthreads();
+    }
+    const int used = min(carry_s, units);
+    if (tid == 0) seg_base[num] = used;
+    for (int u = used + tid; u <= units; u += blockDim.x) cu_seg[u] = cu[num];
 }
 
 // Rows of the stored state (X[j][i] = S[i][j], [dv][dk]) evolve independently through
@@ -70,7 +125,7 @@ constexpr long long kScanWaitCycles = 2000000000LL;  // ~1 s at 2 GHz
 template <int DK, int DV>
 __global__ void __launch_bounds__(kSegThreads)
 kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float *Sin, float *ST, int P, int H,
-                    int *dev_status) {
+                    const int32_t *seg_base, int *dev_status) {
     using namespace sm100;
     constexpr int TI = DK / kScanTpr;                // columns per thread
     constexpr int RPI = kSegThreads / kScanTpr;      // rows covered per pass of the threads (8)
@@ -85,8 +140,11 @@ kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float
     const int b = blockIdx.x / H, h = blockIdx.x % H, j0 = blockIdx.y * kRowsPerCta, tid = threadIdx.x;
     const int r0 = tid / kScanTpr, ci = tid % kScanTpr;
     const size_t sbase = (((size_t)b * H + h) * DV + j0) * DK;
+    // this sequence's segments: units u0 .. u0 + P - 1
+    const size_t u0 = seg_base ? (size_t)seg_base[b] : (size_t)b * P;
+    if (seg_base) P = seg_base[b + 1] - seg_base[b];
     auto fetch = [&](int p) {  // step p's Ms and Zs rows -> buffer p & 1 (one thread)
-        const size_t u = (size_t)b * P + p;
+        const size_t u = u0 + p;
         const int buf = p & 1;
         mbar_arrive_expect_tx(&bar[buf], kMBytes + kZBytes);
         bulk_load(Ms + buf * DK * DK, Mbuf + (u * H + h) * DK * DK, kMBytes, &bar[buf]);
@@ -107,7 +165,7 @@ kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float
         const bool got = mbar_wait_bounded(&bar[buf], (uint32_t)(p >> 1) & 1u, kScanWaitCycles);
         if (__syncthreads_or(!got)) { ok = false; break; }
         const float *M = Ms + buf * DK * DK, *Z = Zs + buf * kRowsPerCta * DK;
-        const size_t xbase = ((((size_t)b * P + p) * H + h) * DV + j0) * DK;
+        const size_t xbase = (((u0 + p) * H + h) * DV + j0) * DK;
         for (int e = tid; e < kRowsPerCta * DK; e += kSegThreads) Sin[xbase + e] = Xs[e];
         float acc[RP][TI];
 #pragma unroll
@@ -150,64 +208,75 @@ kda_kcp_scan_kernel(const float *S0, const float *Mbuf, const float *Zbuf, float
 }
 
 template <int DK, int DV>
-cudaError_t launch_scan_t(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin) {
+cudaError_t launch_scan_t(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin,
+                          const int32_t *seg_base) {
     const size_t smem = (size_t)(kRowsPerCta * DK + 2 * DK * DK + 2 * kRowsPerCta * DK) * sizeof(float) + 16;
     cudaError_t e = cudaFuncSetAttribute(kda_kcp_scan_kernel<DK, DV>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)(s.B * s.H), DV / kRowsPerCta);
     kda_kcp_scan_kernel<DK, DV><<<grid, kSegThreads, smem, s.stream>>>(s.S0, Mbuf, Zbuf, Sin, s.ST, s.P, s.H,
-                                                                      s.dev_status);
+                                                                      seg_base, s.dev_status);
     return cudaGetLastError();
 }
 
 template <int DK>
-cudaError_t launch_scan_dv(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin) {
+cudaError_t launch_scan_dv(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin,
+                           const int32_t *seg_base) {
     switch (s.dv) {
-        case 32: return launch_scan_t<DK, 32>(s, Mbuf, Zbuf, Sin);
-        case 64: return launch_scan_t<DK, 64>(s, Mbuf, Zbuf, Sin);
-        case 128: return launch_scan_t<DK, 128>(s, Mbuf, Zbuf, Sin);
+        case 32: return launch_scan_t<DK, 32>(s, Mbuf, Zbuf, Sin, seg_base);
+        case 64: return launch_scan_t<DK, 64>(s, Mbuf, Zbuf, Sin, seg_base);
+        case 128: return launch_scan_t<DK, 128>(s, Mbuf, Zbuf, Sin, seg_base);
         default: return cudaErrorInvalidValue;
     }
 }
 
-cudaError_t launch_scan(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin) {
+cudaError_t launch_scan(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin,
+                        const int32_t *seg_base) {
     switch (s.dk) {
-        case 32: return launch_scan_dv<32>(s, Mbuf, Zbuf, Sin);
-        case 64: return launch_scan_dv<64>(s, Mbuf, Zbuf, Sin);
-        case 128: return launch_scan_dv<128>(s, Mbuf, Zbuf, Sin);
+        case 32: return launch_scan_dv<32>(s, Mbuf, Zbuf, Sin, seg_base);
+        case 64: return launch_scan_dv<64>(s, Mbuf, Zbuf, Sin, seg_base);
+        case 128: return launch_scan_dv<128>(s, Mbuf, Zbuf, Sin, seg_base);
         default: return cudaErrorInvalidValue;
     }
 }
 
 size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Tokens on the flat axis: B dense sequences of T, or the T tokens of a packed batch.
+long long seg_tokens(const SegmentedArgs &s) { return s.cu_seqlens ? (long long)s.T : (long long)s.B * s.T; }
+
 // The segments of the B sequences as one packed batch (cu_seqlens filled on the device).
 PrefillArgs segments_as_packed(const SegmentedArgs &s, const int32_t *cu_seg) {
     PrefillArgs a{};
     a.q = s.q; a.k = s.k; a.v = s.v; a.g = s.g; a.beta = s.beta;
     a.cu_seqlens = cu_seg;
-    a.B = 1; a.T = s.B * s.T; a.H = s.H; a.dk = s.dk; a.dv = s.dv; a.chunk = s.chunk; a.dtype = s.dtype;
-    a.num_units = s.B * s.P;
+    a.B = 1; a.T = (int)seg_tokens(s); a.H = s.H; a.dk = s.dk; a.dv = s.dv; a.chunk = s.chunk; a.dtype = s.dtype;
+    a.num_units = s.units;
     a.dev_status = s.dev_status; a.stream = s.stream;
     return a;
 }
 
-// Whether passes A-C run on the split prefill's records (both tensor-core shapes).
+// Whether passes A-C run on the split prefill's records: both tensor-core shapes, and no more
+// (segment, head) units than three per SM (beyond that the single-kernel passes keep every SM
+// busy on their own and the records would only add their traffic, as in kda_forward's choice).
 bool records_path(const SegmentedArgs &s) {
-    return prefill_tc_supported(s.dk, s.dk, s.chunk, s.dtype) && prefill_tc_supported(s.dk, s.dv, s.chunk, s.dtype);
+    return prefill_tc_supported(s.dk, s.dk, s.chunk, s.dtype) && prefill_tc_supported(s.dk, s.dv, s.chunk, s.dtype) &&
+           (long long)s.units * s.H <= 3LL * device_sm_count();
 }
 
-// Workspace carve-up (all pieces 256-byte aligned): segment offsets, the longest-first
-// schedule, M, S~ and S_in of every (segment, head), and the records where they are used.
+// Workspace carve-up (all pieces 256-byte aligned): segment offsets (and, for packed batches,
+// each sequence's first segment), the longest-first schedule, M, S~ and S_in of every
+// (segment, head), and the records where they are used.
 struct SegLayout {
-    size_t cu, order, M, Z, Sin, rec, total;
+    size_t cu, base, order, M, Z, Sin, rec, total;
 };
 SegLayout seg_layout(const SegmentedArgs &s) {
-    const size_t units = (size_t)s.B * s.P;
+    const size_t units = (size_t)s.units;
     SegLayout L;
     L.cu = 0;
-    L.order = L.cu + align256((units + 1) * sizeof(int32_t));
+    L.base = L.cu + align256((units + 1) * sizeof(int32_t));
+    L.order = L.base + (s.cu_seqlens ? align256(((size_t)s.B + 1) * sizeof(int32_t)) : 0);
     L.M = L.order + seq_order_bytes((int)units);
     L.Z = L.M + align256(units * s.H * s.dk * s.dk * sizeof(float));
     L.Sin = L.Z + align256(units * s.H * s.dv * s.dk * sizeof(float));
@@ -224,15 +293,18 @@ cudaError_t run_pass(const PrefillArgs &a, bool tc) { return tc ? launch_prefill
 
 }  // namespace
 
-size_t segmented_workspace(const SegmentedArgs &s) { return s.P <= 1 ? 0 : seg_layout(s).total; }
+size_t segmented_workspace(const SegmentedArgs &s) {
+    return s.cu_seqlens == nullptr && s.P <= 1 ? 0 : seg_layout(s).total;
+}
 
-cudaError_t launch_kcp_scan(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin) {
-    return launch_scan(s, Mbuf, Zbuf, Sin);
+cudaError_t launch_kcp_scan(const SegmentedArgs &s, const float *Mbuf, const float *Zbuf, float *Sin,
+                            const int32_t *seg_base) {
+    return launch_scan(s, Mbuf, Zbuf, Sin, seg_base);
 }
 
 cudaError_t launch_segment_pair(const SegmentedArgs &s, float *M, float *Z, bool tc_pair, bool tc_state) {
     // identity start for the transition pass (no offsets needed: one segment per sequence)
-    kda_segment_init_kernel<<<296, kSegThreads, 0, s.stream>>>(nullptr, M, s.B, s.T, 1, s.T, s.H, s.dk);
+    kda_segment_init_kernel<<<296, kSegThreads, 0, s.stream>>>(nullptr, M, s.B, s.B, s.T, 1, s.T, s.H, s.dk);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     PrefillArgs a{};
@@ -248,22 +320,30 @@ cudaError_t launch_segment_pair(const SegmentedArgs &s, float *M, float *Z, bool
 }
 
 int segmented_launches(const SegmentedArgs &s) {
-    const int order = seq_order_bytes(s.B * s.P) > 0 ? 1 : 0;
+    const int order = seq_order_bytes(s.units) > 0 ? 1 : 0;
+    const int init = s.cu_seqlens ? 2 : 1;  // (segment plan +) identity start
     if (records_path(s))  // init, chunk offsets (+ schedule), records, three chain passes, scan
-        return 1 + 1 + order + 1 + 3 + 1;
-    return 1 /* init */ + 3 * (1 + order) /* passes A, B, C */ + 1 /* scan */;
+        return init + 1 + order + 1 + 3 + 1;
+    return init + 3 * (1 + order) /* passes A, B, C */ + 1 /* scan */;
 }
 
 cudaError_t launch_segmented(const SegmentedArgs &s, bool tc_pair, bool tc_state) {
     const SegLayout L = seg_layout(s);
     uint8_t *ws = static_cast<uint8_t *>(s.workspace);
     int32_t *cu_seg = reinterpret_cast<int32_t *>(ws + L.cu);
+    int32_t *seg_base = s.cu_seqlens ? reinterpret_cast<int32_t *>(ws + L.base) : nullptr;
     float *Mbuf = reinterpret_cast<float *>(ws + L.M);
     float *Zbuf = reinterpret_cast<float *>(ws + L.Z);
     float *Sin = reinterpret_cast<float *>(ws + L.Sin);
-    const int units = s.B * s.P;
+    const int units = s.units;
 
-    kda_segment_init_kernel<<<296, kSegThreads, 0, s.stream>>>(cu_seg, Mbuf, s.B, s.T, s.P, s.seg_len, s.H, s.dk);
+    if (s.cu_seqlens) {
+        kda_segment_plan_kernel<<<1, 1024, 0, s.stream>>>(s.cu_seqlens, s.B, s.seg_len, units, seg_base, cu_seg);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    kda_segment_init_kernel<<<296, kSegThreads, 0, s.stream>>>(s.cu_seqlens ? nullptr : cu_seg, Mbuf, units, s.B,
+                                                               s.T, s.P, s.seg_len, s.H, s.dk);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -280,7 +360,7 @@ cudaError_t launch_segmented(const SegmentedArgs &s, bool tc_pair, bool tc_state
         PrefillArgs pb = a;
         pb.o = nullptr; pb.S0 = nullptr; pb.ST = Zbuf;
         if ((e = launch_split_chain(pb, r)) != cudaSuccess) return e;
-        if ((e = launch_scan(s, Mbuf, Zbuf, Sin)) != cudaSuccess) return e;
+        if ((e = launch_scan(s, Mbuf, Zbuf, Sin, seg_base)) != cudaSuccess) return e;
         // pass C: outputs, every segment from its incoming state
         PrefillArgs pc = a;
         pc.o = s.o; pc.S0 = Sin; pc.ST = nullptr;
@@ -290,7 +370,7 @@ cudaError_t launch_segmented(const SegmentedArgs &s, bool tc_pair, bool tc_state
     PrefillArgs a{};
     a.q = s.q; a.k = s.k; a.g = s.g; a.beta = s.beta;
     a.cu_seqlens = cu_seg;
-    a.B = 1; a.T = s.B * s.T; a.H = s.H; a.dk = s.dk; a.chunk = s.chunk; a.dtype = s.dtype;
+    a.B = 1; a.T = (int)seg_tokens(s); a.H = s.H; a.dk = s.dk; a.chunk = s.chunk; a.dtype = s.dtype;
     a.num_units = units;
     a.workspace = ws + L.order; a.workspace_bytes = seq_order_bytes(units);
     a.dev_status = s.dev_status; a.stream = s.stream;
@@ -304,7 +384,7 @@ cudaError_t launch_segmented(const SegmentedArgs &s, bool tc_pair, bool tc_state
     pb.v = s.v; pb.o = nullptr; pb.S0 = nullptr; pb.ST = Zbuf; pb.dv = s.dv;
     if ((e = run_pass(pb, tc_state)) != cudaSuccess) return e;
     // scan: incoming state of every segment, and S_T
-    if ((e = launch_scan(s, Mbuf, Zbuf, Sin)) != cudaSuccess) return e;
+    if ((e = launch_scan(s, Mbuf, Zbuf, Sin, seg_base)) != cudaSuccess) return e;
     // pass C: outputs, every segment from its incoming state
     PrefillArgs pc = a;
     pc.v = s.v; pc.o = s.o; pc.S0 = Sin; pc.ST = nullptr; pc.dv = s.dv;

@@ -48,6 +48,12 @@ _lib.kda_forward_segmented_launches.argtypes = [_i] * 9
 _lib.kda_forward_segmented_launches.restype = _i
 _lib.kda_forward_segmented.argtypes = [_vp] * 8 + [_i] * 8 + [_vp, _sz, _vp, _vp, _i]
 _lib.kda_forward_segmented.restype = _i
+_lib.kda_forward_segmented_varlen_workspace_size.argtypes = [_i] * 8
+_lib.kda_forward_segmented_varlen_workspace_size.restype = _sz
+_lib.kda_forward_segmented_varlen_launches.argtypes = [_i] * 9
+_lib.kda_forward_segmented_varlen_launches.restype = _i
+_lib.kda_forward_segmented_varlen.argtypes = [_vp] * 8 + [_i] * 6 + [_vp, _i, _i, _vp, _sz, _vp, _vp, _i]
+_lib.kda_forward_segmented_varlen.restype = _i
 _lib.kda_decode_multi.argtypes = [_vp] * 8 + [_i] * 6 + [_vp, _vp]
 _lib.kda_decode_multi.restype = _i
 _lib.kda_forward_snapshots.argtypes = [_vp] * 9 + [_i] * 8 + [_vp, _sz, _vp, _vp, _i]
@@ -285,12 +291,26 @@ def kda_forward_segmented_launches(B, T, H, dk, dv, chunk, dtype, seg_len, path=
                                                PATHS[path])
 
 
-def kda_forward_segmented(q, k, v, g, beta, S0=None, *, seg_len: int, chunk: int = 64, o=None,
+def kda_forward_segmented_varlen_workspace_size(T, H, dk, dv, chunk, dtype, num_seqs, seg_len) -> int:
+    n = _lib.kda_forward_segmented_varlen_workspace_size(T, H, dk, dv, chunk, DTYPES.get(dtype, dtype), num_seqs,
+                                                         seg_len)
+    if n == ctypes.c_size_t(-1).value:
+        raise KdaError(KDA_ERR_INVALID_ARG, "kda_forward_segmented_varlen_workspace_size")
+    return int(n)
+
+
+def kda_forward_segmented_varlen_launches(T, H, dk, dv, chunk, dtype, num_seqs, seg_len, path="auto") -> int:
+    return _lib.kda_forward_segmented_varlen_launches(T, H, dk, dv, chunk, DTYPES.get(dtype, dtype), num_seqs,
+                                                      seg_len, PATHS[path])
+
+
+def kda_forward_segmented(q, k, v, g, beta, S0=None, *, seg_len: int, chunk: int = 64, cu_seqlens=None, o=None,
                           S_T=None, return_state: bool = True, workspace=None, dev_status=None,
                           stream=None, path: str = "auto"):
-    """kda_forward on B dense sequences, each cut into segments of ``seg_len``
-    tokens that run as independent units (segment pairs, a scan, a replay).
-    Same shapes and results as kda_forward without cu_seqlens."""
+    """kda_forward with every sequence cut into segments of ``seg_len`` tokens
+    that run as independent units (segment pairs, a scan, a replay). Same shapes
+    and results as kda_forward: B dense sequences, or (cu_seqlens, B = 1) a
+    packed batch whose sequences longer than seg_len are cut."""
     _need(k, "k")
     dtype, dev = k.dtype, k.device
     if dtype not in DTYPES:
@@ -301,23 +321,38 @@ def kda_forward_segmented(q, k, v, g, beta, S0=None, *, seg_len: int, chunk: int
     _need(g, "g", dtype, (B, T, H, dk), dev)
     _need(v, "v", dtype, (B, T, H, dv), dev)
     _need(beta, "beta", dtype, (B, T, H), dev)
+    N = B
+    if cu_seqlens is not None:
+        _need(cu_seqlens, "cu_seqlens", torch.int32, None, dev)
+        N = cu_seqlens.numel() - 1
     if S0 is not None:
-        _need(S0, "S0", torch.float32, (B, H, dv, dk), dev)
+        _need(S0, "S0", torch.float32, (N, H, dv, dk), dev)
     if o is None:
         o = torch.empty((B, T, H, dv), dtype=dtype, device=dev)
     _need(o, "o", dtype, (B, T, H, dv), dev)
     if return_state and S_T is None:
-        S_T = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+        S_T = torch.empty((N, H, dv, dk), dtype=torch.float32, device=dev)
     if S_T is not None:
-        _need(S_T, "S_T", torch.float32, (B, H, dv, dk), dev)
-    ws_need = kda_forward_segmented_workspace_size(B, T, H, dk, dv, chunk, dtype, seg_len)
+        _need(S_T, "S_T", torch.float32, (N, H, dv, dk), dev)
+    if cu_seqlens is not None:
+        ws_need = kda_forward_segmented_varlen_workspace_size(T, H, dk, dv, chunk, dtype, N, seg_len)
+    else:
+        ws_need = kda_forward_segmented_workspace_size(B, T, H, dk, dv, chunk, dtype, seg_len)
     if workspace is None and ws_need > 0:
         workspace = torch.empty(ws_need, dtype=torch.uint8, device=dev)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    rc = _lib.kda_forward_segmented(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
-                                    _ptr(S_T), B, T, H, dk, dv, int(chunk), DTYPES[dtype], int(seg_len),
-                                    _ptr(workspace), ws_bytes, _ptr(dev_status),
-                                    _stream_handle(stream, dev), PATHS[path])
+    if cu_seqlens is not None:
+        if B != 1:
+            raise ValueError("cu_seqlens needs B == 1")
+        rc = _lib.kda_forward_segmented_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                               _ptr(S_T), T, H, dk, dv, int(chunk), DTYPES[dtype],
+                                               _ptr(cu_seqlens), N, int(seg_len), _ptr(workspace), ws_bytes,
+                                               _ptr(dev_status), _stream_handle(stream, dev), PATHS[path])
+    else:
+        rc = _lib.kda_forward_segmented(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                        _ptr(S_T), B, T, H, dk, dv, int(chunk), DTYPES[dtype], int(seg_len),
+                                        _ptr(workspace), ws_bytes, _ptr(dev_status),
+                                        _stream_handle(stream, dev), PATHS[path])
     if rc != KDA_OK:
         raise KdaError(rc, "kda_forward_segmented")
     return o, S_T

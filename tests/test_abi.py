@@ -218,6 +218,53 @@ def test_segmented_queries(K):
         K.kda_forward_segmented_workspace_size(1, 1000, 2, 128, 128, 64, 1, 96)
 
 
+def segv(K, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, S0=None, o=FAKE, S_T=None, T=1000, H=2,
+             dk=128, dv=128, chunk=64, dtype=1, cu=FAKE, num=3, seg_len=256, ws=None, ws_bytes=0, status=None,
+             stream=None, path=0)
+    a.update(kw)
+    return K._lib.kda_forward_segmented_varlen(a["q"], a["k"], a["v"], a["g"], a["beta"], a["S0"], a["o"],
+                                               a["S_T"], a["T"], a["H"], a["dk"], a["dv"], a["chunk"], a["dtype"],
+                                               a["cu"], a["num"], a["seg_len"], a["ws"], a["ws_bytes"],
+                                               a["status"], a["stream"], a["path"])
+
+
+def test_segmented_varlen_rejects_bad_arguments(K):
+    assert segv(K, seg_len=0) == K.KDA_ERR_INVALID_ARG
+    assert segv(K, seg_len=100) == K.KDA_ERR_INVALID_ARG
+    assert segv(K, num=0) == K.KDA_ERR_INVALID_ARG
+    assert segv(K, cu=None) == K.KDA_ERR_INVALID_ARG
+    assert segv(K, dk=48) == K.KDA_ERR_UNSUPPORTED
+    assert segv(K, o=None) == K.KDA_ERR_INVALID_ARG
+    assert segv(K, k=FAKE + 4) == K.KDA_ERR_ALIGNMENT
+    assert segv(K) == K.KDA_ERR_WORKSPACE
+    assert segv(K, ws=FAKE, ws_bytes=4096) == K.KDA_ERR_WORKSPACE
+    assert segv(K, dtype=0, path=K.PATHS["tc"]) == K.KDA_ERR_UNSUPPORTED
+
+
+def test_segmented_varlen_queries(K):
+    # T = 1000 over 3 sequences cut every 256 tokens: at most 1000 // 256 + 3 = 6 segments;
+    # three fp32 states per (segment, head), and the records of every chunk (6 x 2 units)
+    n = K.kda_forward_segmented_varlen_workspace_size(1000, 2, 128, 128, 64, 1, 3, 256)
+    states = 3 * 6 * 2 * 128 * 128 * 4
+    records = al((-(-1000 // 64) + 6) * 2 * REC)
+    assert n >= states + records and n < states + records + 8192
+    # segment plan, identity start, chunk offsets, schedule, records, three chain passes, scan
+    assert K.kda_forward_segmented_varlen_launches(1000, 2, 128, 128, 64, 1, 3, 256) == 9
+    # elsewhere: plan, identity start, three prefill passes each with a schedule, scan
+    assert K.kda_forward_segmented_varlen_launches(1000, 2, 64, 64, 64, 1, 3, 256) == 9
+    # more (segment, head) units than three per SM: single-kernel passes, no records
+    big = K.kda_forward_segmented_varlen_workspace_size(100000, 96, 128, 128, 64, 1, 8, 4096)
+    assert big < 3 * (100000 // 4096 + 8) * 96 * 128 * 128 * 4 + (1 << 20)
+    # T <= seg_len: no sequence is cut, the plain packed prefill's needs
+    assert K.kda_forward_segmented_varlen_workspace_size(1000, 2, 128, 128, 64, 1, 3, 1024) == \
+        K.kda_forward_workspace_size(1, 1000, 2, 128, 128, 64, 3, 1)
+    assert K.kda_forward_segmented_varlen_launches(1000, 2, 128, 128, 64, 1, 3, 1024, "auto") == \
+        K.kda_forward_launches(1, 1000, 2, 128, 128, 64, 1, 1, 3)
+    with pytest.raises(K.KdaError):
+        K.kda_forward_segmented_varlen_workspace_size(1000, 2, 128, 128, 64, 1, 3, 96)
+
+
 def test_decode_multi_rejects_bad_args(K):
     d = K._lib.kda_decode_multi
     args = lambda **kw: [kw.get(n, FAKE) for n in ("q", "k", "v", "g", "beta", "S", "o", "acc")] + \

@@ -134,3 +134,76 @@ def test_context_parallel_module_one_rank_nccl(K):
     o2, S2 = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], chunk=64)
     torch.cuda.synchronize()
     assert rel(to_f64(o), to_f64(o2)) < 1e-5 and rel(to_f64(S_T), to_f64(S2)) < 1e-2
+
+
+def run_seg_packed(K, inp, chunk, seg_len, path="auto"):
+    status = torch.zeros(4, dtype=torch.int32, device=inp["k"].device)
+    o, ST = K.kda_forward_segmented(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp.get("S0"),
+                                    seg_len=seg_len, chunk=chunk, cu_seqlens=inp["cu_seqlens"], path=path,
+                                    dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status[0]) == 0, f"device status {int(status[0])}"
+    return o, ST
+
+
+def packed_case(lens, H, dk, dv, dtype, seed, s0_std=0.1):
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    inp = case(1, int(cu[-1]), H, dk, dv, dtype, seed=seed, s0_std=s0_std, num_states=len(lens))
+    inp["cu_seqlens"] = torch.tensor(cu, device="cuda")
+    return inp, [int(x) for x in cu]
+
+
+@pytest.mark.parametrize("path", ["auto", "simt"])
+@pytest.mark.parametrize("lens,seg_len", [([1, 65, 700, 0, 64, 300, 256], 128), ([900, 0, 3], 256),
+                                          ([640], 64), ([500, 501], 192), ([0, 0, 130], 64)])
+def test_packed_segments(K, oracle_mod, path, lens, seg_len):
+    """Packed sequences, each cut into ceil(len / seg_len) segments (one for the short and
+    the empty ones): ragged last segments and chunks, a length that is a multiple of
+    seg_len, empty sequences (their state passes through bit for bit)."""
+    H = 2
+    inp, cu = packed_case(lens, H, 128, 128, "bf16", seed=sum(lens) + seg_len)
+    o, ST = run_seg_packed(K, inp, 64, seg_len, path)
+    o_ref, ST_ref = oracle_forward(oracle_mod, inp)
+    units = [(n, h) for n in range(len(lens)) for h in range(H)]
+    compare_units(o, ST, o_ref, ST_ref, units, cu, tol=TOL["bf16"], label=f"packed segments {path}")
+    zero = [n for n, L in enumerate(lens) if L == 0]
+    if zero:
+        assert torch.equal(ST[zero], inp["S0"][zero])
+
+
+@pytest.mark.parametrize("dtype,dk,dv,chunk,lens,seg_len", [
+    ("f32", 32, 32, 16, [300, 17, 0, 96], 64), ("f32", 64, 128, 32, [257, 400], 96),
+    ("bf16", 64, 32, 16, [33, 200, 64], 48)])
+def test_packed_segments_simt_shapes(K, oracle_mod, dtype, dk, dv, chunk, lens, seg_len):
+    inp, cu = packed_case(lens, 2, dk, dv, dtype, seed=dk + dv + seg_len)
+    o, ST = run_seg_packed(K, inp, chunk, seg_len)
+    o_ref, ST_ref = oracle_forward(oracle_mod, inp)
+    units = [(n, h) for n in range(len(lens)) for h in range(2)]
+    compare_units(o, ST, o_ref, ST_ref, units, cu, tol=TOL[dtype], label="packed segments simt shapes")
+
+
+def test_packed_segments_uncut_is_the_plain_prefill(K):
+    """T <= seg_len: no sequence is cut, the call is kda_forward_ex with cu_seqlens."""
+    inp, cu = packed_case([100, 0, 200], 2, 128, 128, "bf16", seed=29)
+    o1, S1 = run_seg_packed(K, inp, 64, 320)
+    o2, S2 = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], chunk=64,
+                           cu_seqlens=inp["cu_seqlens"])
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+def test_varlen_workload_segmented_sampled(K, oracle_mod):
+    """The packed 8-sequence workload (96 heads, 352,549 tokens) through the
+    segment-parallel prefill with 16,384-token segments (its two longest sequences
+    become 6 and 7 segments; more (segment, head) units than three per SM, so the
+    passes run the single-kernel prefill): oracle parity on units of the two longest
+    sequences and of a short one, streamed over the host cores."""
+    from kda_testutil import parity_streamed
+    w = WORKLOADS["varlen_h96_8seq_d128_bf16"]
+    inp = workload_inputs(w, device="cuda")
+    o, ST = run_seg_packed(K, inp, w.chunk, 16384)
+    assert torch.isfinite(o).all() and torch.isfinite(ST).all()
+    lens = np.diff(inp["cu_seqlens"].cpu().numpy())
+    order = [int(i) for i in np.argsort(-lens)]
+    units = [(order[0], 0), (order[0], 95), (order[1], 47), (order[-1], 3)]
+    parity_streamed(oracle_mod, inp, o, ST, units, TOL["bf16"], label="varlen segmented")
