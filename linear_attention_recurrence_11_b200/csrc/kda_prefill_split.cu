@@ -719,7 +719,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 // U = (-W S from TMEM) + Ut for one row r of a 64-column half, written as bf16 over the Ut tile
 // (MN-major [tok][dv], 128-byte rows): all of the row's Ut is loaded before any of it is
 // overwritten, in two passes of 32 columns.
-__device__ __forceinline__ void u_readout(uint8_t *ut, int r, uint32_t taddr, bool add_ut = true) {
+__device__ __forceinline__ void u_readout(const uint8_t *ut, uint8_t *dst, int r, uint32_t taddr, bool add_ut = true) {
 #pragma unroll
     for (int g2 = 0; g2 < 2; ++g2) {
         float v[2][16];
@@ -744,7 +744,7 @@ __device__ __forceinline__ void u_readout(uint8_t *ut, int r, uint32_t taddr, bo
             o4[i] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
         }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4 *>(ut + sw128_offset(r, 32 * g2 + 8 * i)) = o4[i];
+        for (int i = 0; i < 4; ++i) *reinterpret_cast<uint4 *>(dst + sw128_offset(r, 32 * g2 + 8 * i)) = o4[i];
     }
 }
 
@@ -894,7 +894,8 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
         // U = Ut - W S (rows 0..63) -> bf16 B operand, written over the record's Ut tile
         // (all-zero values, the transition pass of a segment: the record's Ut is left out)
         if (quarter < 2)
-            u_readout(buf + REC_UT + half * 8 * KB, 32 * quarter + lane, tmem + tlane + tmu + 64u * half, p.v != nullptr);
+            u_readout(buf + REC_UT + half * 8 * KB, buf + REC_UT + half * 8 * KB, 32 * quarter + lane,
+                      tmem + tlane + tmu + 64u * half, p.v != nullptr);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncthreads();
@@ -1022,9 +1023,14 @@ constexpr int kRingSlots = 4;
 
 // pipeline chain-role smem layout (the record pieces at their record offsets, then S bf16)
 constexpr uint32_t X_SB = REC_BYTES;                  // 32 KB S (bf16), B operand MN-major
-constexpr uint32_t X_BAR = X_SB + 32 * KB;            // 4 mbarriers (pieces A, B, C; MMA)
+constexpr uint32_t X_BAR = X_SB + 32 * KB;            // 5 mbarriers (pieces A, B or Ut, C; MMA; P)
 constexpr uint32_t X_TMEMADDR = X_BAR + 64;
 constexpr uint32_t X_SMEM_USED = X_BAR + 128;
+// the compact chains add a U / O tile (16 KB, [tok][dv] MN-major bf16, N-blocks 8 KB apart): U
+// goes there instead of over the record's Ut and the outputs are staged there instead of over
+// Kh, so that every record piece is reloaded as soon as its own tile is consumed
+constexpr uint32_t X_UO = X_BAR + 1024;
+constexpr uint32_t X2_SMEM_USED = X_UO + 16 * KB;
 constexpr uint32_t X_TM_U = 0, X_TM_S = 128, X_TM_COLS = 256;
 
 struct PipeParams {
@@ -1148,14 +1154,22 @@ struct ArrayRecords {
 // buffer as their shared-memory tiles free up: A (state product operand, decay) once the state
 // product is done, B (Ut, P) once the output product is done, C (Kh) once the outputs staged
 // over it have left. One 256-thread group, ~106 KB of shared memory, 256 TMEM columns.
-template <class Rec>
+// kUO (the compact chain kernel): U and the staged outputs live in their own tile (X_UO,
+// 16 KB more), and B is loaded as Ut (once U has been read out) and P (once the output
+// product is done), C once the output product is done: each piece then arrives about a chunk
+// before it is needed.
+template <class Rec, bool kUO = false>
 __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorMap &tm_o, uint8_t *sm, const Group &grp,
                                            int n, int h, const Rec &recs) {
     const uint32_t sbase = smem_u32(sm);
     uint64_t *bar_a = reinterpret_cast<uint64_t *>(sm + X_BAR);
-    uint64_t *bar_b = bar_a + 1;
+    uint64_t *bar_b = bar_a + 1;  // B, or (kUO) Ut
     uint64_t *bar_c = bar_a + 2;
     uint64_t *bar_mma = bar_a + 3;
+    uint64_t *bar_p = bar_a + 4;  // kUO: P
+    uint8_t *const uo = kUO ? sm + X_UO : sm + REC_UT;  // where U goes
+    const uint32_t uo_addr = sbase + (kUO ? X_UO : REC_UT);
+    uint8_t *const ostage = kUO ? sm + X_UO : sm + REC_KH;  // where a full chunk's outputs are staged
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + X_TMEMADDR);
 
     const int tid = grp.tid, warp = tid >> 5, lane = tid & 31;
@@ -1179,6 +1193,7 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
         mbar_init(bar_b, 1);
         mbar_init(bar_c, 1);
         mbar_init(bar_mma, 1);
+        if (kUO) mbar_init(bar_p, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_o);
     }
@@ -1187,18 +1202,24 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
         if (grp.relinquish) tmem_relinquish();
     }
     grp.sync();
-    // thread-0 state of the copies: armed bits (1 A, 2 B, 4 C) and the phase of each barrier
-    uint32_t armed = 0, ph_a = 0, ph_b = 0, ph_c = 0, mma_phase = 0;
+    // thread-0 state of the copies: armed bits (1 A, 2 B or Ut, 4 C, 8 P) and the phase of each barrier
+    uint32_t armed = 0, ph_a = 0, ph_b = 0, ph_c = 0, ph_p = 0, mma_phase = 0;
     bool flag_fail = false, aborted = false, mma_pending = false;
     auto load_a = [&](long long tau) {
         mbar_arrive_expect_tx(bar_a, REC_A_BYTES);
         bulk_load(sm + REC_WQ, slot(tau) + REC_WQ, REC_A_BYTES, bar_a);
         armed |= 1u;
     };
-    auto load_b = [&](long long tau) {
-        mbar_arrive_expect_tx(bar_b, REC_B_BYTES);
-        bulk_load(sm + REC_UT, slot(tau) + REC_UT, REC_B_BYTES, bar_b);
+    auto load_b = [&](long long tau) {  // B, or (kUO) its Ut part
+        const uint32_t bytes = kUO ? REC_P - REC_UT : REC_B_BYTES;
+        mbar_arrive_expect_tx(bar_b, bytes);
+        bulk_load(sm + REC_UT, slot(tau) + REC_UT, bytes, bar_b);
         armed |= 2u;
+    };
+    auto load_p = [&](long long tau) {  // kUO: the P part of B
+        mbar_arrive_expect_tx(bar_p, REC_KH - REC_P);
+        bulk_load(sm + REC_P, slot(tau) + REC_P, REC_KH - REC_P, bar_p);
+        armed |= 8u;
     };
     auto load_c = [&](long long tau) {
         mbar_arrive_expect_tx(bar_c, REC_C_BYTES);
@@ -1211,6 +1232,7 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
         } else {
             load_a(0);
             load_b(0);
+            if (kUO) load_p(0);
             load_c(0);
         }
     }
@@ -1301,20 +1323,25 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
             if (!recs.wait_ready(tau + 1)) flag_fail = true;
             else load_a(tau + 1);
         }
+        // (kUO) the previous chunk's output stores have read the U / O tile
+        if (kUO && tid == 0) bulk_wait_read_all();
         if (!wait_piece(bar_b, ph_b, 2u)) { aborted = true; break; }
 
-        // U = Ut - W S (rows 0..63) -> bf16 B operand, written over the record's Ut tile
+        // U = Ut - W S (rows 0..63) -> bf16 B operand (over the record's Ut tile, or kUO in its own)
         if (quarter < 2)
-            u_readout(sm + REC_UT + half * 8 * KB, 32 * quarter + lane, tmem + tlane + X_TM_U + 64u * half, p.v != nullptr);
+            u_readout(sm + REC_UT + half * 8 * KB, uo + half * 8 * KB, 32 * quarter + lane,
+                      tmem + tlane + X_TM_U + 64u * half, p.v != nullptr);
         fence_proxy_async_smem();
         tc_fence_before();
         if (!wait_piece(bar_c, ph_c, 4u)) { aborted = true; break; }
+        if (kUO && !wait_piece(bar_p, ph_p, 8u)) { aborted = true; break; }
         if (tid == 0) {
             // every piece of record tau is in shared memory: its slot may be refilled
             recs.release(tau);
+            if (kUO && more && !flag_fail) load_b(tau + 1);  // Ut is consumed
             tc_fence_after();
             Opnd AK{sbase + REC_KH, true, 0, 8 * KB};
-            Opnd BU{sbase + REC_UT, true, 0, 8 * KB};
+            Opnd BU{uo_addr, true, 0, 8 * KB};
             Opnd AP{sbase + REC_P - 8 * KB, false, 16 * KB, 0};
             mma_chain<C / 16>(tmem + X_TM_S, AK, BU, idMM, true);
             mma_chain<C / 16>(tmem + X_TM_U, AP, BU, idKM, true);
@@ -1322,7 +1349,14 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
             mma_pending = true;
         }
         if (!wait_mma()) { aborted = true; break; }
-        if (tid == 0 && more && !flag_fail) load_b(tau + 1);  // Ut, U and P are consumed
+        if (tid == 0 && more && !flag_fail) {
+            if (kUO) {  // P and Kh are consumed
+                load_p(tau + 1);
+                load_c(tau + 1);
+            } else {
+                load_b(tau + 1);  // Ut, U and P are consumed
+            }
+        }
 
         // the bf16 copy of the updated state, and this chunk's outputs into registers, before
         // the next state product overwrites the accumulator
@@ -1358,7 +1392,7 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
                     tmem_ld16(tmem + tlane + X_TM_U + 64u * half + 32u * g2 + 16u * gq, ov[gq]);
                 tmem_wait_ld();
                 if (Lc == C) {
-                    uint8_t *base = sm + REC_KH + half * 8 * KB;
+                    uint8_t *base = ostage + half * 8 * KB;
 #pragma unroll
                     for (int gq = 0; gq < 2; ++gq) {
                         uint4 w0, w1;
@@ -1387,11 +1421,11 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
         }
         if (tid == 0) {
             if (Lc == C && p.o) {
-                tma_store_3d(&tm_o, sm + REC_KH, 0, h, (int)tok0);
-                tma_store_3d(&tm_o, sm + REC_KH + 8 * KB, 64, h, (int)tok0);
+                tma_store_3d(&tm_o, ostage, 0, h, (int)tok0);
+                tma_store_3d(&tm_o, ostage + 8 * KB, 64, h, (int)tok0);
                 bulk_commit();
             }
-            if (more && !flag_fail) {  // Kh of the next record, once the outputs have left its tile
+            if (!kUO && more && !flag_fail) {  // Kh of the next record, once the outputs have left its tile
                 bulk_wait_read_all();
                 load_c(tau + 1);
             }
@@ -1404,6 +1438,7 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
             if (p.dev_status) atomicExch(p.dev_status, (int)KDA_ERR_TIMEOUT);
             if (armed & 1u) mbar_wait_bounded(bar_a, ph_a, kWaitCycles);
             if (armed & 2u) mbar_wait_bounded(bar_b, ph_b, kWaitCycles);
+            if (armed & 8u) mbar_wait_bounded(bar_p, ph_p, kWaitCycles);
             if (armed & 4u) mbar_wait_bounded(bar_c, ph_c, kWaitCycles);
             if (mma_pending) mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
         }
@@ -1466,9 +1501,10 @@ kda_chain2_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp
     const int h = blockIdx.x % p.H;
     const int n = unit_seq(p, blockIdx.x / p.H);
     const ArrayRecords recs{sp.rec, (size_t)p.H, h, sp.chunk_base ? (long long)sp.chunk_base[n] : (long long)n * sp.nch};
-    chain_role(p, tm_o, sm, Group{(int)threadIdx.x, 0u, true}, n, h, recs);
+    chain_role<ArrayRecords, true>(p, tm_o, sm, Group{(int)threadIdx.x, 0u, true}, n, h, recs);
 }
-constexpr uint32_t CHAIN2_SMEM = X_SMEM_USED + 1024;
+constexpr uint32_t CHAIN2_SMEM = X2_SMEM_USED + 1024;
+static_assert(2 * 1024 + P_SMEM_BYTES + CHAIN2_SMEM <= 233472, "a prep CTA and a compact chain share an SM");
 
 int num_sms() { return device_sm_count(); }
 
