@@ -296,7 +296,7 @@ def run_ours(args, rank, world, device):
     else:
         kern_src = "linear_attention_recurrence_11_b200/csrc/kda_prefill_simt.cu"
     achieved = alg_bytes / (kern_ms / 1e3) / 1e9
-    traffic = traffic_for(kern_src, wname)
+    traffic = traffic_for(kern_src, f"{wname}/{path_used}")
     res.update({
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
