@@ -34,6 +34,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "KDA prefill tokens/s (H=96,d=128) & % tensor peak; decode GB/s vs HBM"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL_HBM_GBS = 7700.0  # HGX B200 HBM3e, for context beside the measured / fallback copy bandwidth
 WORKLOAD_ALIASES = {"prefill": "prefill_h96_T8192_d128_bf16", "varlen": "varlen_h96_8seq_d128_bf16",
                     "b2": "b2_h4_T2048_d128_bf16", "small": "small_f32_T256_d32",
                     "decode": "decode_n256_h96_d128", "long": "long_h8_T65536_d128_bf16"}
@@ -567,6 +568,28 @@ def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):
         b.record(stream)
         torch.cuda.synchronize(device)
     ms = max_ranks(a.elapsed_time(b)) / steps
+    # the same steps captured once in a CUDA graph and replayed (launch cost off the host)
+    graph_ms = None
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(device)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for i in range(steps):
+                    step(warm + i)
+        stream.wait_stream(side)
+        g.replay()
+        torch.cuda.synchronize(device)
+        barrier()
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        graph_ms = max_ranks(a.elapsed_time(b)) / steps
+        del g
+    except RuntimeError:
+        graph_ms = None
     elem = sets[0]["k"].element_size()
     del sets
     alg_bytes, _ = decode_algorithmic(w.B, w.H, w.dk, w.dv, elem)
@@ -582,6 +605,8 @@ def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):
                          "algorithmic_bytes_per_launch": alg_bytes,
                          "peak_source": peaks["source"] + " (hbm_gbs)"},
             "gpu_launches": steps, "clocks": clk.summary(),
+            "graph_ms_per_step": graph_ms,
+            "frac_of_nominal_hbm": gbs / NOMINAL_HBM_GBS,
             "requests": w.B, "l2": f"state {w.B * w.H * w.dk * w.dv * 4 / 1e9:.2f} GB per step, larger than L2"}
     if args.draft_tokens > 0:
         res["multi_token"] = multi_decode_measure(args, device, peaks, max_ranks, world, w, S)
@@ -691,12 +716,23 @@ def _oracle_sample(inp, w, seconds, max_heads=None):
     return done, el, heads, T
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_baseline_prefill(inp, w, seconds):
     done, el, heads, T = _oracle_sample(inp, w, seconds)
     return {"value": done / w.H / el, "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{heads} of {w.H} heads x {T} tokens of {w.name}, sequential fp64 oracle, "
                       f"one thread; tokens/s = token-heads/s / {w.H}",
-            "host_cpus": os.cpu_count(), "seconds": el}
+            "host_cpus": os.cpu_count(), "cpu_model": cpu_model(), "seconds": el}
 
 
 def cpu_baseline_all_cores(inp, w):

@@ -88,7 +88,8 @@ constexpr uint32_t P_TM_W = 0, P_TM_UT = 128, P_TM_COLS = 256;  // the Gram uses
 // ----------------------------------------------------------- chain smem layout
 constexpr uint32_t C_RECSTRIDE = REC_BYTES;           // 1 KB aligned
 constexpr uint32_t C_SB = 2 * C_RECSTRIDE;            // 32 KB S (bf16), B operand MN-major [dk][dv], N-blocks 16 KB apart
-constexpr uint32_t C_MISC = C_SB + 32 * KB;
+constexpr uint32_t C_OST = C_SB + 32 * KB;            // 16 KB output staging ([tok][dv], N-blocks 8 KB apart)
+constexpr uint32_t C_MISC = C_OST + 16 * KB;
 constexpr uint32_t C_BAR = C_MISC;                    // 3 mbarriers
 constexpr uint32_t C_TMEMADDR = C_MISC + 64;
 constexpr uint32_t C_SMEM_BYTES = C_MISC + 128 + 1024;
@@ -794,7 +795,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
     __syncthreads();
     // bit b: buffer b has a record load armed and not yet waited for / the parity of its next phase
     uint32_t rec_armed = 0, rec_phase = 0;
-    if (tid == 0) {
+    if (tid == 0) {  // records 0 and 1; record c + 2 is requested once chunk c's products are done
         for (int b = 0; b < 2 && b < nchunks; ++b) {
             mbar_arrive_expect_tx(&bar_rec[b], REC_BYTES);
             bulk_load(sm + b * C_RECSTRIDE, record(b), REC_BYTES, &bar_rec[b]);
@@ -882,14 +883,6 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
             tc_fence_before();
         }
         if (!wait_mma()) { aborted = true; break; }
-        if (tid == 0 && ch >= 1 && ch + 1 < nchunks) {
-            // the record one chunk ahead goes into the other buffer, whose outputs (staged by the
-            // previous chunk) have been read by their stores by now
-            bulk_wait_read_all();
-            mbar_arrive_expect_tx(&bar_rec[b ^ 1], REC_BYTES);
-            bulk_load(sm + (b ^ 1) * C_RECSTRIDE, record(ch + 1), REC_BYTES, &bar_rec[b ^ 1]);
-            rec_armed |= 1u << (b ^ 1);
-        }
 
         // U = Ut - W S (rows 0..63) -> bf16 B operand, written over the record's Ut tile
         // (all-zero values, the transition pass of a segment: the record's Ut is left out)
@@ -912,6 +905,11 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
             mma_pending = true;
         }
         if (!wait_mma()) { aborted = true; break; }
+        if (tid == 0 && ch + 2 < nchunks) {  // this buffer's record is consumed: the one two chunks ahead
+            mbar_arrive_expect_tx(&bar_rec[b], REC_BYTES);
+            bulk_load(buf, record(ch + 2), REC_BYTES, &bar_rec[b]);
+            rec_armed |= 1u << b;
+        }
 
         // the bf16 copy of the updated state: the next chunk's state product waits on it
         {
@@ -930,6 +928,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
         }
         fence_proxy_async_smem();
         tc_fence_before();
+        if (tid == 0) bulk_wait_read_all();  // the previous chunk's output stores have read their staging
         __syncthreads();
         if (more) {
             if (!wait_rec(b ^ 1)) { aborted = true; break; }
@@ -937,8 +936,8 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
         }
 
         // outputs (rows 64..127 of this chunk's accumulator) while the next product runs. A
-        // full chunk is staged over the U tile (its products are done) and leaves by two
-        // tensor stores; the rows of a partial chunk are stored directly.
+        // full chunk is staged in its own tile and leaves by two tensor stores; the rows of a
+        // partial chunk are stored directly.
         if (quarter >= 2 && p.o) {
             const int r = 32 * quarter + lane - 64;
             float v[4][16];
@@ -946,7 +945,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
             for (int gq = 0; gq < 4; ++gq) tmem_ld16(tmem + tlane + tmu + 64u * half + 16u * gq, v[gq]);
             tmem_wait_ld();
             if (Lc == C) {
-                uint8_t *base = buf + REC_UT + half * 8 * KB;
+                uint8_t *base = sm + C_OST + half * 8 * KB;
 #pragma unroll
                 for (int gq = 0; gq < 4; ++gq) {
                     uint4 w0, w1;
@@ -970,8 +969,8 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
         __syncthreads();
         if (tid == 0) {
             if (Lc == C && p.o) {
-                tma_store_3d(&tm_o, buf + REC_UT, 0, h, (int)tok0);
-                tma_store_3d(&tm_o, buf + REC_UT + 8 * KB, 64, h, (int)tok0);
+                tma_store_3d(&tm_o, sm + C_OST, 0, h, (int)tok0);
+                tma_store_3d(&tm_o, sm + C_OST + 8 * KB, 64, h, (int)tok0);
                 bulk_commit();
             }
 
