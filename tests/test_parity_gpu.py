@@ -205,7 +205,7 @@ def test_decode_full_size_1000_steps_sampled(K, oracle_mod):
     inp0 = workload_inputs(w, device="cuda", step=0)
     S = inp0["S0"]
     S_init = to_f64(S)
-    refs = [np.ascontiguousarray(S_init[n, h]) for n, h in picks]
+    refs = [S_init[n, h].copy() for n, h in picks]  # copies: the oracle steps them in place
     for t in range(w.decode_steps):
         inp = inp0 if t == 0 else workload_inputs(w, device="cuda", step=t)
         d = {k: inp[k][:, 0].contiguous() for k in ("q", "k", "v", "g", "beta")}
@@ -222,7 +222,7 @@ def test_decode_full_size_1000_steps_sampled(K, oracle_mod):
             worst_s = worst_o = 0.0
             for n in range(w.B):
                 for h in range(w.H):
-                    St = np.ascontiguousarray(S_init[n, h])
+                    St = S_init[n, h].copy()
                     ot = oracle_mod.decode_step(hd["q"][n, h], hd["k"][n, h], hd["v"][n, h],
                                                 hd["g"][n, h], hd["beta"][n, h], St)
                     es, ds = np.sum((S1[n, h] - St) ** 2), np.sum(St ** 2)
