@@ -568,6 +568,8 @@ def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):
         b.record(stream)
         torch.cuda.synchronize(device)
     ms = max_ranks(a.elapsed_time(b)) / steps
+    # speculative rounds on the states as the timed steps left them
+    multi = multi_decode_measure(args, device, peaks, max_ranks, world, w, S) if args.draft_tokens > 0 else None
     # the same steps captured once in a CUDA graph and replayed (launch cost off the host)
     graph_ms = None
     try:
@@ -608,8 +610,8 @@ def decode_measure(args, device, peaks, barrier, max_ranks, world, steps):
             "graph_ms_per_step": graph_ms,
             "frac_of_nominal_hbm": gbs / NOMINAL_HBM_GBS,
             "requests": w.B, "l2": f"state {w.B * w.H * w.dk * w.dv * 4 / 1e9:.2f} GB per step, larger than L2"}
-    if args.draft_tokens > 0:
-        res["multi_token"] = multi_decode_measure(args, device, peaks, max_ranks, world, w, S)
+    if multi is not None:
+        res["multi_token"] = multi
     return res
 
 
