@@ -271,8 +271,12 @@ int kda_forward_noalloc(const void *q, const void *k, const void *v, const void 
  *                the state after its first (p + 1) snap_every tokens, in the
  *                S0 layout of one sequence (it can be passed back as S0 to
  *                resume from that prefix). May be NULL when T < snap_every.
- * Other arguments, results and errors as kda_forward_ex (no workspace is
- * needed for dense batches; pass NULL, 0).
+ * Other arguments, results and errors as kda_forward_ex. The workspace decides
+ * the tensor-core form as there: with kda_forward_workspace_size_ex(..., path)
+ * bytes the split form runs (its chains store the snapshots; dense batches of
+ * up to one (sequence, head) unit per SM), with NULL, 0 the single form.
+ * KDA_PATH_TC_PIPE is refused (KDA_ERR_UNSUPPORTED), and so is
+ * KDA_PATH_TC_SPLIT for more units than SMs.
  */
 int kda_forward_snapshots(const void *q, const void *k, const void *v, const void *g, const void *beta,
                           const float *S0, void *o, float *S_T, float *S_snap, int snap_every, int B, int T,

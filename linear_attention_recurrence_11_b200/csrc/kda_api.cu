@@ -188,7 +188,16 @@ int kda_forward_snapshots(const void *q, const void *k, const void *v, const voi
     a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.dev_status = dev_status;
     a.stream = static_cast<cudaStream_t>(stream);
     a.S_snap = S_snap; a.snap_every = T / snap_every > 0 ? snap_every : 0;
-    if (path == KDA_PATH_TC_SPLIT || path == KDA_PATH_TC_PIPE) return KDA_ERR_UNSUPPORTED;  // single form only
+    // the split form (when it is the form kda_forward_ex would run and its chains can store the
+    // snapshots) or the single form; the pipe form does not write snapshots
+    if (path == KDA_PATH_TC_PIPE) return KDA_ERR_UNSUPPORTED;
+    const bool split_ok = use_tc(a, path) && kda::prefill_split_snapshots_ok(a);
+    if (path == KDA_PATH_TC_SPLIT && !split_ok) return KDA_ERR_UNSUPPORTED;
+    const Form f = choose_form(a, path, workspace_bytes, true);
+    if (f == Form::Split && split_ok) {
+        if (workspace == nullptr || workspace_bytes < kda::prefill_split_workspace(a)) return KDA_ERR_WORKSPACE;
+        return kda::cuda_status(kda::launch_prefill_split(a));
+    }
     const bool tc = use_tc(a, path);
     const cudaError_t e = tc ? kda::launch_prefill_tc(a) : kda::launch_prefill_simt(a);
     return kda::cuda_status(e);

@@ -129,6 +129,8 @@ cudaError_t launch_split_records(const PrefillArgs &a, SplitRecords *out);
 cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r);
 size_t prefill_split_workspace(const PrefillArgs &a);
 int prefill_split_launches(const PrefillArgs &a);
+// the split form writes S_snap (dense batches of up to one unit per SM: the double-buffered chains)
+bool prefill_split_snapshots_ok(const PrefillArgs &a);
 // the one-launch form: chains and record producers in one cooperative launch, records in a ring
 bool prefill_pipe_supported(const PrefillArgs &a);
 cudaError_t launch_prefill_pipe(const PrefillArgs &a);

@@ -925,6 +925,17 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
                 *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq)) = w0;
                 *reinterpret_cast<uint4 *>(sb + sw128_offset(si, 16 * gq + 8)) = w1;
             }
+            // a snapshot of the state after this chunk (dense batches; fp32, the S0 layout of one
+            // sequence), from the values just read for the bf16 copy
+            const long long done = (ch + 1) * C;
+            if (p.snap_every && Lc == C && done % p.snap_every == 0) {
+                const long long nsnap = p.T / p.snap_every;
+                float *dst = p.S_snap + (((size_t)n * nsnap + (size_t)(done / p.snap_every - 1)) * H + h) * (size_t)(D * D);
+#pragma unroll
+                for (int gq = 0; gq < 4; ++gq)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) dst[(size_t)(64 * half + 16 * gq + e) * D + si] = sv[gq][e];
+            }
         }
         fence_proxy_async_smem();
         tc_fence_before();
@@ -1659,8 +1670,13 @@ cudaError_t launch_split_records(const PrefillArgs &a, SplitRecords *out) {
     return cudaSuccess;
 }
 
+bool prefill_split_snapshots_ok(const PrefillArgs &a) {
+    return !packed(a) && (long long)a.num_units * a.H <= num_sms();
+}
+
 cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r) {
     if (pass.num_units == 0) return cudaSuccess;
+    if (pass.snap_every && !prefill_split_snapshots_ok(pass)) return cudaErrorInvalidValue;
     const size_t tokens = pass.cu_seqlens ? (size_t)pass.T : (size_t)pass.B * (size_t)pass.T;
     if (tokens == 0) return launch_prefill_simt(pass);
     CUtensorMap mo;

@@ -415,7 +415,8 @@ def kda_decode_multi(q, k, v, g, beta, S, o=None, *, n_accept=None, outputs: boo
 
 
 def kda_forward_snapshots(q, k, v, g, beta, S0=None, *, snap_every: int, chunk: int = 64, o=None,
-                          S_T=None, S_snap=None, dev_status=None, stream=None, path: str = "auto"):
+                          S_T=None, S_snap=None, workspace=None, dev_status=None, stream=None,
+                          path: str = "auto"):
     """kda_forward on B dense sequences that also returns the state every
     ``snap_every`` tokens: S_snap fp32 ``[B, T // snap_every, H, dv, dk]`` (slot p =
     the state after (p + 1) * snap_every tokens, usable as S0 of one sequence).
@@ -442,10 +443,15 @@ def kda_forward_snapshots(q, k, v, g, beta, S0=None, *, snap_every: int, chunk: 
     if S_snap is None:
         S_snap = torch.empty((B, nsnap, H, dv, dk), dtype=torch.float32, device=dev)
     _need(S_snap, "S_snap", torch.float32, (B, nsnap, H, dv, dk), dev)
+    if workspace is None and path != "tc_single":  # the split form where it applies (the single form without)
+        n = kda_forward_workspace_size(B, T, H, dk, dv, chunk, B, dtype, path=path)
+        if n > 0:
+            workspace = torch.empty(n, dtype=torch.uint8, device=dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     rc = _lib.kda_forward_snapshots(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
                                     _ptr(S_T), _ptr(S_snap) if nsnap > 0 else None, int(snap_every), B, T, H,
-                                    dk, dv, int(chunk), DTYPES[dtype], None, 0, _ptr(dev_status),
-                                    _stream_handle(stream, dev), PATHS[path])
+                                    dk, dv, int(chunk), DTYPES[dtype], _ptr(workspace), ws_bytes,
+                                    _ptr(dev_status), _stream_handle(stream, dev), PATHS[path])
     if rc != KDA_OK:
         raise KdaError(rc, "kda_forward_snapshots")
     return o, S_T, S_snap

@@ -291,6 +291,11 @@ def test_snapshots_reject_bad_arguments(K):
     assert call(snap=None) == K.KDA_ERR_INVALID_ARG     # 3 snapshots are due
     assert call(snap=FAKE + 4) == K.KDA_ERR_ALIGNMENT
     assert call(dk=48) == K.KDA_ERR_UNSUPPORTED
+    # the pipe form writes no snapshots; the split form stores them for up to one unit per SM
+    assert call(path=K.PATHS["tc_pipe"]) == K.KDA_ERR_UNSUPPORTED
+    assert call(path=K.PATHS["tc_split"], B=2, H=75) == K.KDA_ERR_UNSUPPORTED
+    # a forced split form needs its records
+    assert call(path=K.PATHS["tc_split"]) == K.KDA_ERR_WORKSPACE
 
 
 def test_pair_and_scan_reject_bad_arguments(K):

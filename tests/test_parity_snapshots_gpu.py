@@ -27,6 +27,7 @@ def prefix_states(oracle_mod, inp, b, h, ends):
 
 @pytest.mark.parametrize("dtype,dk,dv,chunk,T,every,path", [
     ("bf16", 128, 128, 64, 1000, 256, "auto"), ("bf16", 128, 128, 64, 1000, 256, "simt"),
+    ("bf16", 128, 128, 64, 1000, 256, "tc_single"), ("bf16", 128, 128, 64, 512, 64, "tc_split"),
     ("bf16", 128, 128, 64, 512, 64, "auto"), ("f32", 32, 32, 16, 256, 48, "auto"),
     ("f32", 64, 128, 32, 300, 96, "auto"),
 ])
@@ -48,24 +49,34 @@ def test_snapshots(K, oracle_mod, dtype, dk, dv, chunk, T, every, path):
             assert rel(got, np.stack(refs)) < TOL[dtype]
 
 
-def test_resume_from_a_snapshot(K):
-    """A snapshot is a valid S0: resuming from it reproduces the rest of the run."""
+@pytest.mark.parametrize("path", ["auto", "tc_single"])
+def test_resume_from_a_snapshot(K, path):
+    """A snapshot is a valid S0: resuming from it on the same form reproduces the rest of
+    the run (the split form's chains and the single kernel both save the fp32 state they
+    carry)."""
     inp = case(1, 768, 2, 128, 128, "bf16", seed=61, s0_std=0.1)
     o, ST, Ssn = K.kda_forward_snapshots(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"],
-                                         snap_every=256, chunk=64)
+                                         snap_every=256, chunk=64, path=path)
     rest = {x: inp[x][:, 512:].contiguous() for x in ("q", "k", "v", "g", "beta")}
-    # snapshots come from the single-kernel form; resume on the same form
     o2, S2 = K.kda_forward(rest["q"], rest["k"], rest["v"], rest["g"], rest["beta"], Ssn[:, 1].contiguous(),
-                           chunk=64, path="tc_single")
+                           chunk=64, path=path)
     torch.cuda.synchronize()
     assert rel(to_f64(o2), to_f64(o[:, 512:])) < 1e-5 and rel(to_f64(S2), to_f64(ST)) < 1e-5
 
 
-def test_no_snapshot_due(K, oracle_mod):
-    """T < snap_every: no snapshot, the plain prefill results."""
+@pytest.mark.parametrize("path", ["auto", "tc_single"])
+def test_no_snapshot_due(K, oracle_mod, path):
+    """T < snap_every: no snapshot, the plain prefill results of the same form."""
     inp = case(1, 100, 2, 128, 128, "bf16", seed=63)
     o, ST, Ssn = K.kda_forward_snapshots(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None,
-                                         snap_every=128, chunk=64)
-    o2, S2 = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None, chunk=64, path="tc_single")
+                                         snap_every=128, chunk=64, path=path)
+    o2, S2 = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None, chunk=64, path=path)
     torch.cuda.synchronize()
     assert Ssn.shape[1] == 0 and torch.equal(o, o2) and torch.equal(ST, S2)
+
+
+def test_snapshots_refused_on_the_pipe_form(K):
+    inp = case(1, 256, 2, 128, 128, "bf16", seed=65)
+    with pytest.raises(K.KdaError):
+        K.kda_forward_snapshots(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None, snap_every=128,
+                                chunk=64, path="tc_pipe")
