@@ -346,7 +346,7 @@ def run_ours(args, rank, world, device):
         def snap():
             kda.kda_forward_snapshots(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"],
                                       snap_every=args.snap_every, chunk=w.chunk, o=o, S_T=ST, S_snap=Ssn,
-                                      path=args.path)
+                                      workspace=ws, path=args.path)
         for _ in range(2):
             snap()
         torch.cuda.synchronize(device)
@@ -361,6 +361,26 @@ def run_ours(args, rank, world, device):
                             "ms_per_step": ms_snap, "overhead_vs_step": ms_snap / kern_ms - 1.0,
                             "snapshot_bytes_per_step": Ssn.numel() * 4,
                             "note": "kda_forward_snapshots on the same inputs, outside the timed region"}
+    if not seg and not w.seqlens:
+        # the same step with the fused pre-operations (q, k normalised per row and g computed from
+        # gate logits inside the kernels; the synthetic g read as logits, for timing only)
+        def fused():
+            kda.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], chunk=w.chunk, o=o,
+                            S_T=ST, workspace=ws, path=args.path,
+                            fuse=kda.KDA_FUSE_NORM_QK | kda.KDA_FUSE_GATE_LOGITS)
+        for _ in range(2):
+            fused()
+        torch.cuda.synchronize(device)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(5):
+            fused()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        ms_fused = a.elapsed_time(b) / 5
+        res["fused"] = {"ms_per_step": ms_fused, "overhead_vs_step": ms_fused / kern_ms - 1.0,
+                        "note": "kda_forward with KDA_FUSE_NORM_QK | KDA_FUSE_GATE_LOGITS on the same inputs, "
+                                "outside the timed region"}
     if not args.no_e2e:
         res["e2e"] = e2e_prefill(args, device, inp, w, forward, o, ST, world, barrier, max_ranks,
                                  dense=not seg and not w.seqlens)

@@ -220,12 +220,17 @@ int kda_forward_fused(const void *q, const void *k, const void *v, const void *g
     a.workspace = workspace; a.workspace_bytes = workspace_bytes; a.dev_status = dev_status;
     a.stream = static_cast<cudaStream_t>(stream);
     a.fuse = flags;
-    if (flags && (path == KDA_PATH_TC_SPLIT || path == KDA_PATH_TC_PIPE))
-        return KDA_ERR_UNSUPPORTED;  // fused pre-operations: single form
     if (!flags)
         return kda_forward_ex(q, k, v, g, beta, S0, o, S_T, B, T, H, dk, dv, chunk, dtype, cu_seqlens, num_seqs,
                               workspace, workspace_bytes, dev_status, stream, path);
-    const bool tc = use_tc(a, path);
+    if (path == KDA_PATH_TC_PIPE) return KDA_ERR_UNSUPPORTED;  // the pipe form has no fused variant
+    // the form kda_forward_ex would run (the pipe form's place taken by the single form)
+    const Form f = choose_form(a, path, workspace_bytes, true);
+    if (f == Form::Split) {
+        if (workspace == nullptr || workspace_bytes < kda::prefill_split_workspace(a)) return KDA_ERR_WORKSPACE;
+        return kda::cuda_status(kda::launch_prefill_split(a));
+    }
+    const bool tc = f != Form::Simt;
     const size_t need = tc ? kda::prefill_tc_workspace(a) : kda::prefill_simt_workspace(a);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return KDA_ERR_WORKSPACE;
     const cudaError_t e = tc ? kda::launch_prefill_tc(a) : kda::launch_prefill_simt(a);

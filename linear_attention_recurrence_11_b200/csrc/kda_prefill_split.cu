@@ -80,7 +80,8 @@ constexpr uint32_t P_BAR = P_MISC;                    // 4 mbarriers
 constexpr uint32_t P_TMEMADDR = P_MISC + 64;
 constexpr uint32_t P_BETA = P_MISC + 128;             // 64 fp32
 constexpr uint32_t P_DSUM = P_BETA + 256;             // 4 x 128 fp32 subtile totals of g (log2 units)
-constexpr uint32_t P_SMEM_USED = P_DSUM + 2048;
+constexpr uint32_t P_NORM = P_DSUM + 2048;            // fused variant: 2 x 64 x 2 fp32 partial squared norms of k, q
+constexpr uint32_t P_SMEM_USED = P_NORM + 1024;
 constexpr uint32_t P_SMEM_BYTES = P_SMEM_USED + 1024;  // slack for 1024-byte alignment
 static_assert(2 * (P_SMEM_BYTES + 1024) <= 233472, "two prep CTAs per SM");
 constexpr uint32_t P_TM_W = 0, P_TM_UT = 128, P_TM_COLS = 256;  // the Gram uses columns 0..63 first
@@ -214,11 +215,17 @@ struct StaticTasks {
 // The persistent loop of a record-producing CTA over the tasks its source hands out.
 // Src::acquire (thread 0) returns once the task's record may be written, before its first
 // store; Src::release (thread 0) publishes a record whose stores have completed (kPublish).
-template <class Src>
+// kFused: the variant with the fused pre-operations (p.fuse: q, k normalised per row inside the
+// operand pass, g computed from gate logits in the cumulative decay), a separate instantiation
+// so that the plain variant carries none of it.
+template <bool kFused, class Src>
 __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtensorMap &tm_k, const CUtensorMap &tm_v,
                                           const CUtensorMap &tm_g, const SplitParams &sp, Src &src, uint8_t *sm,
                                           const Group &grp) {
     const PrefillArgs &p = sp.a;
+    const bool fuse_gate = kFused && (p.fuse & KDA_FUSE_GATE_LOGITS) != 0;
+    const bool fuse_norm = kFused && (p.fuse & KDA_FUSE_NORM_QK) != 0;
+    float *sNorm = reinterpret_cast<float *>(sm + P_NORM);
     const uint32_t sbase = smem_u32(sm);
     uint64_t *bar_ld = reinterpret_cast<uint64_t *>(sm + P_BAR);  // k, q, g of a task
     uint64_t *bar_v = bar_ld + 1;
@@ -346,8 +353,12 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
                 const int row = SUB * ti + HR * hh + rr;  // rows past the end decay by 1
                 const uint2 raw = row < Lc ? *reinterpret_cast<const uint2 *>(sm + P_GV + row * 256 + c0 * 2)
                                            : make_uint2(0, 0);
-                const float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
-                const float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+                float2 g01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.x));
+                float2 g23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&raw.y));
+                if (fuse_gate && row < Lc) {  // g holds gate logits
+                    g01 = make_float2(gate_from_logit(g01.x), gate_from_logit(g01.y));
+                    g23 = make_float2(gate_from_logit(g23.x), gate_from_logit(g23.y));
+                }
                 a[0] = fmaf(g01.x, kLog2e, a[0]);
                 a[1] = fmaf(g01.y, kLog2e, a[1]);
                 a[2] = fmaf(g23.x, kLog2e, a[2]);
@@ -367,6 +378,35 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
 #pragma unroll
                 for (int e = 0; e < 4; ++e) sD[ti * D + c0 + e] = gl[HR - 1][e];
             }
+        }
+        if (fuse_norm) {
+            // squared norms of this thread's 8 k and 8 q rows over its 4 channels, summed over the
+            // 16 lanes of the half-warp (64 channels) by a reduce-scatter: lane l ends with the sum
+            // of value l (k row l, or q row l - 8); the partner warp holds the other 64 channels
+            const uint8_t *l0 = sm + P_L0 + cblk * 16 * KB;
+            float nv[2 * HR];
+#pragma unroll
+            for (int rr = 0; rr < HR; ++rr) {
+                const int r = SUB * ti + HR * hh + rr;
+                const uint2 kr = *reinterpret_cast<const uint2 *>(l0 + sw128_offset(r, cin));
+                const uint2 qr = *reinterpret_cast<const uint2 *>(l0 + sw128_offset(64 + r, cin));
+                const float2 k01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kr.x));
+                const float2 k23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&kr.y));
+                const float2 q01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qr.x));
+                const float2 q23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&qr.y));
+                nv[rr] = r < Lc ? k01.x * k01.x + k01.y * k01.y + k23.x * k23.x + k23.y * k23.y : 0.f;
+                nv[HR + rr] = r < Lc ? q01.x * q01.x + q01.y * q01.y + q23.x * q23.x + q23.y * q23.y : 0.f;
+            }
+            const int l16 = lane & 15;
+#pragma unroll
+            for (int w = 8; w >= 1; w >>= 1) {  // keep half of the values, add the partner's copies
+                const bool up = l16 & w;
+#pragma unroll
+                for (int i = 0; i < w; ++i)
+                    nv[i] = (up ? nv[i + w] : nv[i]) + __shfl_xor_sync(0xffffffffu, up ? nv[i] : nv[i + w], w);
+            }
+            const int r = SUB * ti + HR * hh + (l16 & 7);
+            sNorm[((l16 >> 3) * C + r) * 2 + (warp & 1)] = nv[0];
         }
         // the previous task's record stores have read their staging (and, where records are
         // published, completed: then that record is published); this task's record may be written
@@ -450,6 +490,16 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
                 float kx[4], qx[4];
                 ld4(l0 + off_r, kx);
                 ld4(l0 + off_q, qx);
+                if (fuse_norm) {  // k and q normalised per row (rows past the end stay zero)
+                    const float nk = sNorm[(0 * C + r) * 2] + sNorm[(0 * C + r) * 2 + 1];
+                    const float nq = sNorm[(1 * C + r) * 2] + sNorm[(1 * C + r) * 2 + 1];
+                    const float ik = nk > 0.f ? rsqrtf(nk) : 0.f, iq = nq > 0.f ? rsqrtf(nq) : 0.f;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        kx[e] *= ik;
+                        qx[e] *= iq;
+                    }
+                }
                 // paired fp32 products (two channels per instruction, each the same IEEE product)
                 float2 F[2], Fi[2];
 #pragma unroll
@@ -706,6 +756,7 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
     }
 }
 
+template <bool kFused>
 __global__ void __launch_bounds__(NT, 2)
 kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -713,7 +764,7 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     StaticTasks src{&sp, 0, 0};
-    prep_loop(tm_q, tm_k, tm_v, tm_g, sp, src, sm, Group{(int)threadIdx.x, 0u, true});
+    prep_loop<kFused>(tm_q, tm_k, tm_v, tm_g, sp, src, sm, Group{(int)threadIdx.x, 0u, true});
 }
 
 // ====================================================================== chain
@@ -1497,7 +1548,7 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         chain_role(pp.sp.a, tm_o, sm, grp, G / pp.sp.a.H, G % pp.sp.a.H, recs);
     } else {
         RingTasks src{&pp, 0, G - pp.NC};
-        prep_loop(tm_q, tm_k, tm_v, tm_g, pp.sp, src, sm, grp);
+        prep_loop<false>(tm_q, tm_k, tm_v, tm_g, pp.sp, src, sm, grp);
     }
 }
 
@@ -1629,10 +1680,10 @@ cudaError_t launch_split_records(const PrefillArgs &a, SplitRecords *out) {
     if (!make_map(&mq, a.q, tokens, a.H, 64, true) || !make_map(&mk, a.k, tokens, a.H, 64, true) ||
         !make_map(&mv, a.v ? a.v : a.q, tokens, a.H, 64, true) || !make_map(&mg, a.g, tokens, a.H, 128, false))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM_BYTES);
+    const auto prep = a.fuse ? kda_prep_kernel<true> : kda_prep_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(kda_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             (int)cudaSharedmemCarveoutMaxShared);
+    e = cudaFuncSetAttribute(prep, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     SplitParams sp{};
     sp.a = a;
@@ -1659,7 +1710,7 @@ cudaError_t launch_split_records(const PrefillArgs &a, SplitRecords *out) {
         sp.tasks = bound;
     }
     const long long grid_p = bound < 2LL * num_sms() ? bound : 2LL * num_sms();
-    kda_prep_kernel<<<(unsigned)grid_p, NT, P_SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, sp);
+    prep<<<(unsigned)grid_p, NT, P_SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, sp);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     out->rec = sp.rec;

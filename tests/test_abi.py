@@ -315,6 +315,9 @@ def test_fused_entry_points_reject_unknown_flags(K):
     base = [FAKE] * 5 + [None, FAKE, None, 1, 64, 2, 128, 128, 64, 1, None, 0, None, 0, None, None, 0]
     assert f(*base, 4) == K.KDA_ERR_INVALID_ARG
     assert f(*(base[:8] + [0] + base[9:]), 1) == K.KDA_ERR_INVALID_ARG  # B = 0
+    # the pipe form has no fused variant; a forced split form needs its records
+    assert f(*(base[:-1] + [K.PATHS["tc_pipe"]]), 1) == K.KDA_ERR_UNSUPPORTED
+    assert f(*(base[:-1] + [K.PATHS["tc_split"]]), 1) == K.KDA_ERR_WORKSPACE
     d = K._lib.kda_decode_step_fused
     assert d(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 4, 96, 128, 128, 1, None, 8) == K.KDA_ERR_INVALID_ARG
 

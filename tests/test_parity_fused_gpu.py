@@ -48,7 +48,8 @@ def reference_inputs(inp):
 
 @pytest.mark.parametrize("dtype,dk,dv,chunk,T,path", [
     ("bf16", 128, 128, 64, 300, "auto"), ("bf16", 128, 128, 64, 300, "simt"), ("f32", 64, 32, 32, 150, "auto"),
-    ("bf16", 32, 64, 16, 100, "auto"),
+    ("bf16", 32, 64, 16, 100, "auto"), ("bf16", 128, 128, 64, 300, "tc_split"),
+    ("bf16", 128, 128, 64, 300, "tc_single"),
 ])
 def test_fused_prefill(K, oracle_mod, dtype, dk, dv, chunk, T, path):
     B, H = 2, 2
@@ -95,3 +96,36 @@ def test_unfused_call_is_unchanged(K):
     o2, S2 = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], None, chunk=64, fuse=0)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2) and torch.equal(S1, S2)
+
+
+@pytest.mark.parametrize("flags", ["norm", "gate"])
+def test_fused_packed_split_form(K, oracle_mod, flags):
+    """Packed sequences through the split form's record producer with one fused
+    pre-operation at a time (the other input given as the plain entry points take it)."""
+    lens = [130, 0, 64, 257]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    H = 2
+    inp = raw_inputs(1, int(cu[-1]), H, 128, 128, "bf16", seed=97)
+    S0 = (0.1 * torch.randn(len(lens), H, 128, 128, generator=torch.Generator().manual_seed(5))).cuda()
+    r = reference_inputs(inp)
+    if flags == "norm":
+        f = K.KDA_FUSE_NORM_QK
+        g_in = (-5.0 * torch.sigmoid(inp["g"].float())).to(inp["g"].dtype)
+        r["g"] = to_f64(g_in)
+    else:
+        f = K.KDA_FUSE_GATE_LOGITS
+        g_in = inp["g"]
+        for x in ("q", "k"):
+            inp[x] = torch.nn.functional.normalize(inp[x].float(), dim=-1).to(inp[x].dtype)
+            r[x] = to_f64(inp[x])
+    o, ST = K.kda_forward(inp["q"], inp["k"], inp["v"], g_in, inp["beta"], S0, chunk=64,
+                          cu_seqlens=torch.tensor(cu, device="cuda"), path="tc_split", fuse=f)
+    torch.cuda.synchronize()
+    S0f = to_f64(S0)
+    for n in range(len(lens)):
+        for h in range(H):
+            a, b = int(cu[n]), int(cu[n + 1])
+            ou, su = oracle_mod.forward(*(r[x][0, a:b, h] for x in ("q", "k", "v", "g", "beta")), S0=S0f[n, h])
+            if b > a:
+                assert rel(to_f64(o[0, a:b, h]), ou) < TOL["bf16"], (n, h)
+            assert rel(to_f64(ST[n, h]), su) < TOL["bf16"], (n, h)
