@@ -800,6 +800,8 @@ __device__ __forceinline__ void u_readout(const uint8_t *ut, uint8_t *dst, int r
     }
 }
 
+// kSnap: the instantiation that also stores the state every p.snap_every tokens
+template <bool kSnap>
 __global__ void __launch_bounds__(NT, 1)
 kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp) {
     const PrefillArgs &p = sp.a;
@@ -979,7 +981,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
             // a snapshot of the state after this chunk (dense batches; fp32, the S0 layout of one
             // sequence), from the values just read for the bf16 copy
             const long long done = (ch + 1) * C;
-            if (p.snap_every && Lc == C && done % p.snap_every == 0) {
+            if (kSnap && p.snap_every && Lc == C && done % p.snap_every == 0) {
                 const long long nsnap = p.T / p.snap_every;
                 float *dst = p.S_snap + (((size_t)n * nsnap + (size_t)(done / p.snap_every - 1)) * H + h) * (size_t)(D * D);
 #pragma unroll
@@ -1736,8 +1738,8 @@ cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r) {
     const bool compact = (long long)pass.num_units * pass.H > num_sms();
     cudaError_t e = compact ? cudaFuncSetAttribute(kda_chain2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                    (int)CHAIN2_SMEM)
-                            : cudaFuncSetAttribute(kda_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)C_SMEM_BYTES);
+                            : cudaFuncSetAttribute(pass.snap_every ? kda_chain_kernel<true> : kda_chain_kernel<false>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C_SMEM_BYTES);
     if (e != cudaSuccess) return e;
     SplitParams sp{};
     sp.a = pass;
@@ -1754,7 +1756,10 @@ cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r) {
         if (e != cudaSuccess) return e;
         kda_chain2_kernel<<<grid_c, NT, CHAIN2_SMEM, pass.stream>>>(mo, sp);
     } else {
-        kda_chain_kernel<<<grid_c, NT, C_SMEM_BYTES, pass.stream>>>(mo, sp);
+        if (pass.snap_every)
+            kda_chain_kernel<true><<<grid_c, NT, C_SMEM_BYTES, pass.stream>>>(mo, sp);
+        else
+            kda_chain_kernel<false><<<grid_c, NT, C_SMEM_BYTES, pass.stream>>>(mo, sp);
     }
     return cudaGetLastError();
 }
