@@ -178,7 +178,10 @@ int kda_forward_ex(const void *q, const void *k, const void *v, const void *g, c
                    int path);
 
 /* kda_forward_ex with fused pre-operations (flags: kda_fuse bits; 0 = kda_forward_ex).
- * Unknown bits return KDA_ERR_INVALID_ARG. */
+ * Unknown bits return KDA_ERR_INVALID_ARG. The form is chosen as by
+ * kda_forward_ex (the split form's record producer and the single form both have
+ * a fused variant); KDA_PATH_TC_PIPE with flags returns KDA_ERR_UNSUPPORTED, and
+ * where AUTO would run the pipe form the single form runs. */
 int kda_forward_fused(const void *q, const void *k, const void *v, const void *g, const void *beta,
                       const float *S0, void *o, float *S_T, int B, int T, int H, int dk, int dv, int chunk,
                       int dtype, const int32_t *cu_seqlens, int num_seqs, void *workspace,
