@@ -232,6 +232,28 @@ int kda_forward_host(const void *q, const void *k, const void *v, const void *g,
                      int *dev_status, void *stream, int path);
 
 /*
+ * kda_forward_host for a packed batch (the cu_seqlens layout of kda_forward:
+ * q, k, g [T, H, dk], v, o [T, H, dv], beta [T, H], S0 / S_T [num_seqs, H, dv,
+ * dk], all in HOST memory; cu_seqlens a HOST int32 array [num_seqs + 1] with
+ * cu_seqlens[0] = 0, non-decreasing, cu_seqlens[num_seqs] = T). The flat token
+ * axis is cut into pieces of about piece_len tokens (0: about T / 8), each cut
+ * moved down onto the chunk grid of the sequence it falls in, so every part of
+ * a sequence starts at one of its own chunk boundaries; piece p is one packed
+ * kda_forward_ex launch over the sequences it touches, from and to their fp32
+ * states in a device buffer (in place). Uploads, launches and downloads
+ * overlap as in kda_forward_host. Results equal one device call's up to
+ * rounding (a piece may run a different tensor-core form than the whole batch).
+ * workspace: at least kda_forward_host_varlen_workspace_size(...) bytes,
+ * 256-byte aligned. Other arguments and errors as kda_forward_host.
+ */
+size_t kda_forward_host_varlen_workspace_size(int T, int H, int dk, int dv, int chunk, int dtype,
+                                              const int32_t *cu_seqlens, int num_seqs, int piece_len);
+int kda_forward_host_varlen(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                            const float *S0, void *o, float *S_T, int T, int H, int dk, int dv, int chunk,
+                            int dtype, const int32_t *cu_seqlens, int num_seqs, int piece_len, void *workspace,
+                            size_t workspace_bytes, int *dev_status, void *stream, int path);
+
+/*
  * kda_forward without a workspace argument, for callers that cannot allocate
  * device memory: engines that reserve all device memory in their own pools at
  * start-up and treat any other allocation as an error, hosts that hand a

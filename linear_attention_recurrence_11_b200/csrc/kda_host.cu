@@ -20,6 +20,7 @@
 // for it, so that anything the caller enqueues after the call (an event, a
 // synchronisation) sees the host outputs complete.
 #include <mutex>
+#include <vector>
 
 #include "kda_internal.cuh"
 
@@ -87,6 +88,71 @@ cudaError_t copy_piece(void *dst, const void *src, int B, int T, long long t0, i
     return cudaMemcpy2DAsync(static_cast<char *>(dst) + off, full, src, width, width, B, cudaMemcpyDeviceToHost,
                              s);
 }
+
+// Packed batches: the flat token axis [0, T) is cut into pieces of about Lp tokens, each
+// boundary moved down onto the chunk grid of the sequence it falls in (that sequence's chunks
+// start at cu[n]), so that every part of a sequence inside a piece starts at one of its own
+// chunk boundaries. Piece i covers tokens [cut[i], cut[i + 1]) and sequences first[i] ..
+// last[i] (the ones with a token in it); local[i] are its offsets relative to cut[i].
+struct PackedPlan {
+    std::vector<long long> cut;
+    std::vector<int> first, last;
+    std::vector<int32_t> local;    // all pieces' local offsets, piece i's at local_at[i]
+    std::vector<size_t> local_at;
+    int max_tokens = 0, max_seqs = 0;
+};
+
+// the sequence holding token t (cu[n] <= t < cu[n + 1]; empty sequences hold none)
+int seq_of(const int32_t *cu, int num, long long t) {
+    int lo = 0, hi = num;  // cu[lo] <= t < cu[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) / 2;
+        if (cu[mid] <= t) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+bool plan_packed(const int32_t *cu, int num, long long T, int Lp, int chunk, PackedPlan &P) {
+    P = PackedPlan{};
+    P.cut.push_back(0);
+    while (P.cut.back() < T) {
+        const long long t0 = P.cut.back();
+        long long b = t0 + Lp;
+        if (b < T) {
+            const int n = seq_of(cu, num, b);
+            const long long aligned = cu[n] + (b - cu[n]) / chunk * chunk;
+            b = aligned > t0 ? aligned : (long long)(cu[n] + ((t0 - cu[n]) / chunk + 1) * chunk);
+            if (b > cu[n + 1]) b = cu[n + 1];
+            if (b <= t0 || b > T) return false;
+        } else {
+            b = T;
+        }
+        P.cut.push_back(b);
+    }
+    const size_t pieces = P.cut.size() - 1;
+    for (size_t i = 0; i < pieces; ++i) {
+        const long long t0 = P.cut[i], t1 = P.cut[i + 1];
+        const int f = seq_of(cu, num, t0), l = seq_of(cu, num, t1 - 1);
+        P.first.push_back(f);
+        P.last.push_back(l);
+        P.local_at.push_back(P.local.size());
+        for (int n = f; n <= l + 1; ++n) {
+            long long x = n == f ? t0 : (n == l + 1 ? t1 : (long long)cu[n]);
+            P.local.push_back((int32_t)(x - t0));
+        }
+        while (P.local.size() % 4) P.local.push_back(0);  // each piece's offsets 16-byte aligned
+        if (t1 - t0 > P.max_tokens) P.max_tokens = (int)(t1 - t0);
+        if (l - f + 1 > P.max_seqs) P.max_seqs = l - f + 1;
+    }
+    return true;
+}
+
+// Device workspace of the packed form: two slots of max_tokens, every sequence's state, the
+// pieces' local offsets, and the device prefill's workspace for the largest piece.
+struct PackedLayout {
+    HostLayout slots;  // slot sizes for B = 1 and max_tokens (its state / scratch fields unused)
+    size_t state, local, scratch, total;
+};
 
 int default_piece(int T, int chunk) {
     // about eight pieces, whole chunks, at least one chunk
@@ -183,6 +249,138 @@ int kda_forward_host(const void *q, const void *k, const void *v, const void *g,
         if (n > 0) KDA_TRY(copy_piece(o, slot[s].o, B, T, t0, n, (size_t)H * dv, es, false, hp.down));
         KDA_TRY(cudaEventRecord(hp.ev_down[s], hp.down));
     }
+    if (S_T) KDA_TRY(cudaMemcpyAsync(S_T, state, state_bytes, cudaMemcpyDeviceToHost, hp.down));
+    KDA_TRY(cudaEventRecord(hp.ev_done, hp.down));
+    KDA_TRY(cudaStreamWaitEvent(cs, hp.ev_done, 0));
+#undef KDA_TRY
+    return KDA_OK;
+}
+
+namespace {
+PackedLayout packed_layout(const PackedPlan &P, int num, int H, int dk, int dv, int chunk, int dtype) {
+    PackedLayout L{};
+    L.slots = host_layout(1, P.max_tokens, H, dk, dv, chunk, dtype);
+    L.state = round_up((size_t)num * H * dv * dk * sizeof(float));
+    L.local = round_up(P.local.size() * sizeof(int32_t));
+    const size_t ws = P.max_tokens > 0 ? kda_forward_workspace_size(1, P.max_tokens, H, dk, dv, chunk,
+                                                                     P.max_seqs > 1 ? P.max_seqs : 1, dtype)
+                                       : 0;
+    L.scratch = ws == (size_t)-1 ? 0 : round_up(ws);
+    L.total = 2 * L.slots.slot + L.state + L.local + L.scratch;
+    return L;
+}
+
+int check_host_varlen(int T, int H, int dk, int dv, int chunk, int dtype, const int32_t *cu, int num,
+                      int piece_len, int path) {
+    int st = kda::validate_prefill(1, T, H, dk, dv, chunk, dtype, path);
+    if (st) return st;
+    if (!cu || num <= 0) return KDA_ERR_INVALID_ARG;
+    if (cu[0] != 0 || cu[num] != T) return KDA_ERR_INVALID_ARG;
+    for (int n = 0; n < num; ++n)
+        if (cu[n + 1] < cu[n]) return KDA_ERR_INVALID_ARG;
+    if (piece_len < 0 || (piece_len > 0 && piece_len % chunk != 0)) return KDA_ERR_INVALID_ARG;
+    return KDA_OK;
+}
+}  // namespace
+
+size_t kda_forward_host_varlen_workspace_size(int T, int H, int dk, int dv, int chunk, int dtype,
+                                              const int32_t *cu_seqlens, int num_seqs, int piece_len) {
+    if (check_host_varlen(T, H, dk, dv, chunk, dtype, cu_seqlens, num_seqs, piece_len, KDA_PATH_AUTO) != KDA_OK)
+        return (size_t)-1;
+    PackedPlan P;
+    if (!plan_packed(cu_seqlens, num_seqs, T, piece_len > 0 ? piece_len : default_piece(T, chunk), chunk, P))
+        return (size_t)-1;
+    return packed_layout(P, num_seqs, H, dk, dv, chunk, dtype).total;
+}
+
+int kda_forward_host_varlen(const void *q, const void *k, const void *v, const void *g, const void *beta,
+                            const float *S0, void *o, float *S_T, int T, int H, int dk, int dv, int chunk,
+                            int dtype, const int32_t *cu_seqlens, int num_seqs, int piece_len, void *workspace,
+                            size_t workspace_bytes, int *dev_status, void *stream, int path) {
+    int st = check_host_varlen(T, H, dk, dv, chunk, dtype, cu_seqlens, num_seqs, piece_len, path);
+    if (st) return st;
+    if (T > 0 && (!q || !k || !v || !g || !beta || !o)) return KDA_ERR_INVALID_ARG;
+    PackedPlan P;
+    if (!plan_packed(cu_seqlens, num_seqs, T, piece_len > 0 ? piece_len : default_piece(T, chunk), chunk, P))
+        return KDA_ERR_INVALID_ARG;
+    const PackedLayout L = packed_layout(P, num_seqs, H, dk, dv, chunk, dtype);
+    if (!workspace || workspace_bytes < L.total) return KDA_ERR_WORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return KDA_ERR_ALIGNMENT;
+
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return KDA_ERR_CUDA;
+    HostPipe &hp = g_pipes[dev];
+    std::call_once(hp.once, [&hp] { hp.init_error = pipe_init(hp); });
+    if (hp.init_error != cudaSuccess) return KDA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(hp.mu);
+
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const size_t es = dtype == KDA_DTYPE_BF16 ? 2 : 4;
+    char *ws = static_cast<char *>(workspace);
+    struct Slot { char *q, *k, *v, *g, *beta, *o; } slot[2];
+    const HostLayout &S = L.slots;
+    for (int i = 0; i < 2; ++i) {
+        char *b = ws + i * S.slot;
+        slot[i].q = b; b += round_up(S.q);
+        slot[i].k = b; b += round_up(S.k);
+        slot[i].v = b; b += round_up(S.v);
+        slot[i].g = b; b += round_up(S.g);
+        slot[i].beta = b; b += round_up(S.beta);
+        slot[i].o = b;
+    }
+    float *state = reinterpret_cast<float *>(ws + 2 * S.slot);
+    int32_t *local = reinterpret_cast<int32_t *>(ws + 2 * S.slot + L.state);
+    void *scratch = L.scratch ? ws + 2 * S.slot + L.state + L.local : nullptr;
+    const size_t unit_state = (size_t)H * dv * dk;
+    const size_t state_bytes = (size_t)num_seqs * unit_state * sizeof(float);
+
+#define KDA_TRY(x)                                   \
+    do {                                             \
+        if ((x) != cudaSuccess) return KDA_ERR_CUDA; \
+    } while (0)
+    KDA_TRY(cudaEventRecord(hp.ev_start, cs));
+    KDA_TRY(cudaStreamWaitEvent(hp.up, hp.ev_start, 0));
+    KDA_TRY(cudaStreamWaitEvent(hp.down, hp.ev_start, 0));
+    // every sequence's state (S0 or zeros) and the pieces' local offsets, once
+    if (S0) KDA_TRY(cudaMemcpyAsync(state, S0, state_bytes, cudaMemcpyHostToDevice, hp.up));
+    else KDA_TRY(cudaMemsetAsync(state, 0, state_bytes, hp.up));
+    KDA_TRY(cudaMemcpyAsync(local, P.local.data(), P.local.size() * sizeof(int32_t), cudaMemcpyHostToDevice, hp.up));
+
+    const size_t rowq = (size_t)H * dk * es, rowv = (size_t)H * dv * es, rowb = (size_t)H * es;
+    const char *hq = static_cast<const char *>(q), *hk = static_cast<const char *>(k);
+    const char *hv = static_cast<const char *>(v), *hg = static_cast<const char *>(g);
+    const char *hb = static_cast<const char *>(beta);
+    char *ho = static_cast<char *>(o);
+    const size_t pieces = P.cut.size() - 1;
+    for (size_t p = 0; p < pieces; ++p) {
+        const int s = (int)(p & 1);
+        const long long t0 = P.cut[p];
+        const int n = (int)(P.cut[p + 1] - t0);
+        // upload piece p once the launch of piece p - 2 has consumed the slot: contiguous rows
+        if (p >= 2) KDA_TRY(cudaStreamWaitEvent(hp.up, hp.ev_comp[s], 0));
+        KDA_TRY(cudaMemcpyAsync(slot[s].q, hq + t0 * rowq, n * rowq, cudaMemcpyHostToDevice, hp.up));
+        KDA_TRY(cudaMemcpyAsync(slot[s].k, hk + t0 * rowq, n * rowq, cudaMemcpyHostToDevice, hp.up));
+        KDA_TRY(cudaMemcpyAsync(slot[s].v, hv + t0 * rowv, n * rowv, cudaMemcpyHostToDevice, hp.up));
+        KDA_TRY(cudaMemcpyAsync(slot[s].g, hg + t0 * rowq, n * rowq, cudaMemcpyHostToDevice, hp.up));
+        KDA_TRY(cudaMemcpyAsync(slot[s].beta, hb + t0 * rowb, n * rowb, cudaMemcpyHostToDevice, hp.up));
+        KDA_TRY(cudaEventRecord(hp.ev_up[s], hp.up));
+        // the packed prefill of piece p: its sequences' states in place
+        KDA_TRY(cudaStreamWaitEvent(cs, hp.ev_up[s], 0));
+        if (p >= 2) KDA_TRY(cudaStreamWaitEvent(cs, hp.ev_down[s], 0));
+        float *st_p = state + (size_t)P.first[p] * unit_state;
+        const int ns = P.last[p] - P.first[p] + 1;
+        st = kda_forward_ex(slot[s].q, slot[s].k, slot[s].v, slot[s].g, slot[s].beta, st_p, slot[s].o, st_p, 1, n,
+                            H, dk, dv, chunk, dtype, local + P.local_at[p], ns, scratch, L.scratch, dev_status, cs,
+                            path);
+        if (st) return st;
+        KDA_TRY(cudaEventRecord(hp.ev_comp[s], cs));
+        KDA_TRY(cudaStreamWaitEvent(hp.down, hp.ev_comp[s], 0));
+        KDA_TRY(cudaMemcpyAsync(ho + t0 * rowv, slot[s].o, n * rowv, cudaMemcpyDeviceToHost, hp.down));
+        KDA_TRY(cudaEventRecord(hp.ev_down[s], hp.down));
+    }
+    // the state copies above were on the upload stream: the download waits for them
+    KDA_TRY(cudaEventRecord(hp.ev_up[0], hp.up));
+    KDA_TRY(cudaStreamWaitEvent(hp.down, hp.ev_up[0], 0));
     if (S_T) KDA_TRY(cudaMemcpyAsync(S_T, state, state_bytes, cudaMemcpyDeviceToHost, hp.down));
     KDA_TRY(cudaEventRecord(hp.ev_done, hp.down));
     KDA_TRY(cudaStreamWaitEvent(cs, hp.ev_done, 0));

@@ -72,6 +72,10 @@ _lib.kda_forward_host_workspace_size.argtypes = [_i] * 8
 _lib.kda_forward_host_workspace_size.restype = _sz
 _lib.kda_forward_host.argtypes = [_vp] * 8 + [_i] * 8 + [_vp, _sz, _vp, _vp, _i]
 _lib.kda_forward_host.restype = _i
+_lib.kda_forward_host_varlen_workspace_size.argtypes = [_i] * 6 + [_vp, _i, _i]
+_lib.kda_forward_host_varlen_workspace_size.restype = _sz
+_lib.kda_forward_host_varlen.argtypes = [_vp] * 8 + [_i] * 6 + [_vp, _i, _i, _vp, _sz, _vp, _vp, _i]
+_lib.kda_forward_host_varlen.restype = _i
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_ALIGNMENT = 0, 1, 2, 3
 KDA_ERR_WORKSPACE, KDA_ERR_CUDA, KDA_ERR_TIMEOUT, KDA_ERR_SCRATCH_LIMIT = 4, 5, 6, 7
@@ -234,15 +238,29 @@ def kda_forward_host_workspace_size(B, T, H, dk, dv, chunk, dtype, piece_len=0) 
     return int(n)
 
 
-def kda_forward_host(q, k, v, g, beta, S0=None, *, chunk: int = 64, piece_len: int = 0, o=None, S_T=None,
-                     return_state: bool = True, workspace=None, device=None, dev_status=None, stream=None,
+def kda_forward_host_varlen_workspace_size(T, H, dk, dv, chunk, dtype, cu_seqlens, piece_len=0) -> int:
+    cu = torch.as_tensor(cu_seqlens, dtype=torch.int32).contiguous()
+    n = _lib.kda_forward_host_varlen_workspace_size(T, H, dk, dv, chunk, DTYPES.get(dtype, dtype), _ptr(cu),
+                                                    cu.numel() - 1, int(piece_len))
+    if n == ctypes.c_size_t(-1).value:
+        raise KdaError(KDA_ERR_INVALID_ARG, "kda_forward_host_varlen_workspace_size")
+    return int(n)
+
+
+def kda_forward_host(q, k, v, g, beta, S0=None, *, chunk: int = 64, piece_len: int = 0, cu_seqlens=None, o=None,
+                     S_T=None, return_state: bool = True, workspace=None, device=None, dev_status=None, stream=None,
                      path: str = "auto"):
-    """Dense-batch prefill with inputs and outputs in host memory (CPU tensors,
-    pinned for overlapped copies): the library uploads, runs and downloads the
-    sequence in pieces of ``piece_len`` tokens (0: about T / 8). Outputs are
-    allocated on the host (pinned when k is) unless given. Returns ``(o, S_T)``;
-    they are complete once ``stream`` (default: the current stream of
-    ``device``) has finished."""
+    """Prefill with inputs and outputs in host memory (CPU tensors, pinned for
+    overlapped copies): the library uploads, runs and downloads the tokens in
+    pieces of about ``piece_len`` (0: about T / 8). Dense batches ``[B, T, H, d]``,
+    or with ``cu_seqlens`` (a CPU int32 tensor ``[N + 1]``, B must be 1) a packed
+    batch whose states are ``[N, H, dv, dk]``. Outputs are allocated on the host
+    (pinned when k is) unless given. Returns ``(o, S_T)``; they are complete once
+    ``stream`` (default: the current stream of ``device``) has finished."""
+    if cu_seqlens is not None:
+        return _forward_host_varlen(q, k, v, g, beta, S0, chunk=chunk, piece_len=piece_len, cu_seqlens=cu_seqlens,
+                                    o=o, S_T=S_T, return_state=return_state, workspace=workspace, device=device,
+                                    dev_status=dev_status, stream=stream, path=path)
     _need_host(k, "k")
     dtype = k.dtype
     if dtype not in DTYPES:
@@ -276,6 +294,50 @@ def kda_forward_host(q, k, v, g, beta, S0=None, *, chunk: int = 64, piece_len: i
                                    workspace.numel(), _ptr(dev_status), _stream_handle(stream, dev), PATHS[path])
     if rc != KDA_OK:
         raise KdaError(rc, "kda_forward_host")
+    return o, S_T
+
+
+def _forward_host_varlen(q, k, v, g, beta, S0, *, chunk, piece_len, cu_seqlens, o, S_T, return_state, workspace,
+                         device, dev_status, stream, path):
+    _need_host(k, "k")
+    dtype = k.dtype
+    if dtype not in DTYPES:
+        raise ValueError(f"unsupported dtype {dtype}")
+    B, T, H, dk = k.shape
+    if B != 1:
+        raise ValueError("cu_seqlens needs B == 1")
+    dv = v.shape[-1]
+    _need_host(q, "q", dtype, (B, T, H, dk))
+    _need_host(g, "g", dtype, (B, T, H, dk))
+    _need_host(v, "v", dtype, (B, T, H, dv))
+    _need_host(beta, "beta", dtype, (B, T, H))
+    cu = cu_seqlens
+    _need_host(cu, "cu_seqlens", torch.int32, None)
+    N = cu.numel() - 1
+    if S0 is not None:
+        _need_host(S0, "S0", torch.float32, (N, H, dv, dk))
+    pin = k.is_pinned()
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=dtype, pin_memory=pin)
+    _need_host(o, "o", dtype, (B, T, H, dv))
+    if return_state and S_T is None:
+        S_T = torch.empty((N, H, dv, dk), dtype=torch.float32, pin_memory=pin)
+    if S_T is not None:
+        _need_host(S_T, "S_T", torch.float32, (N, H, dv, dk))
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if workspace is None:
+        workspace = torch.empty(kda_forward_host_varlen_workspace_size(T, H, dk, dv, chunk, dtype, cu, piece_len),
+                                dtype=torch.uint8, device=dev)
+    _need(workspace, "workspace", torch.uint8, None, dev)
+    if dev_status is not None:
+        _need(dev_status, "dev_status", torch.int32, None, dev)
+    with torch.cuda.device(dev):
+        rc = _lib.kda_forward_host_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(S0), _ptr(o),
+                                          _ptr(S_T), T, H, dk, dv, int(chunk), DTYPES[dtype], _ptr(cu), N,
+                                          int(piece_len), _ptr(workspace), workspace.numel(), _ptr(dev_status),
+                                          _stream_handle(stream, dev), PATHS[path])
+    if rc != KDA_OK:
+        raise KdaError(rc, "kda_forward_host_varlen")
     return o, S_T
 
 

@@ -364,3 +364,29 @@ def test_host_workspace_size_is_two_piece_slots_and_the_state(K):
     assert small == 2 * (3 * rnd(tok * 64 * 4) + 2 * rnd(tok * 32 * 4) + rnd(tok * 4)) + rnd(2 * 3 * 32 * 64 * 4)
     with pytest.raises(K.KdaError):
         K.kda_forward_host_workspace_size(1, 64, 2, 128, 128, 64, 1, 96)
+
+
+def test_host_varlen_validates_offsets_before_any_cuda_call(K):
+    import ctypes
+    f = K._lib.kda_forward_host_varlen
+
+    def call(cu, T=1000, num=None, **kw):
+        arr = (ctypes.c_int32 * len(cu))(*cu)
+        a = dict(ws=FAKE, ws_bytes=1 << 40, piece=256, path=0)
+        a.update(kw)
+        return f(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, None, T, 2, 128, 128, 64, 1, arr,
+                 len(cu) - 1 if num is None else num, a["piece"], a["ws"], a["ws_bytes"], None, None, a["path"])
+    assert call([1, 500, 1000]) == K.KDA_ERR_INVALID_ARG       # does not start at 0
+    assert call([0, 600, 500, 1000]) == K.KDA_ERR_INVALID_ARG  # decreasing
+    assert call([0, 500, 999]) == K.KDA_ERR_INVALID_ARG        # does not end at T
+    assert call([0, 1000], num=0) == K.KDA_ERR_INVALID_ARG
+    assert call([0, 500, 1000], piece=100) == K.KDA_ERR_INVALID_ARG  # not whole chunks
+    assert call([0, 500, 1000], ws=None) == K.KDA_ERR_WORKSPACE
+    assert call([0, 500, 1000], ws=FAKE + 16) == K.KDA_ERR_ALIGNMENT
+    # the workspace: two slots of the largest piece, every sequence's state, the pieces'
+    # offsets, the device prefill's scratch for the largest piece
+    n2 = K.kda_forward_host_varlen_workspace_size(1000, 2, 128, 128, 64, 1, [0, 500, 1000], 256)
+    n8 = K.kda_forward_host_varlen_workspace_size(1000, 2, 128, 128, 64, 1, [0] + [125 * i for i in range(1, 9)], 256)
+    assert n2 > 2 * 256 * 2 * 128 * 2 * 5 and n8 > n2
+    with pytest.raises(K.KdaError):
+        K.kda_forward_host_varlen_workspace_size(1000, 2, 128, 128, 64, 1, [0, 500, 900], 256)

@@ -2,12 +2,13 @@
 copied up, run from the carried state and copied down, give the same o and
 S_T as one device-resident kda_forward_ex call over the whole sequence (bit
 for bit, pieces being whole chunks), and meet the oracle's bars."""
+import numpy as np
 import pytest
 import torch
 
-from linear_attention_recurrence_11_b200.inputs import WORKLOADS, workload_inputs
+from linear_attention_recurrence_11_b200.inputs import WORKLOADS, to_f64, workload_inputs
 
-from kda_testutil import TOL, case, compare_units, oracle_forward
+from kda_testutil import TOL, case, compare_units, oracle_forward, rel
 
 pytestmark = pytest.mark.gpu
 
@@ -126,3 +127,60 @@ def test_benchmark_workload_sampled(K, oracle_mod):
     o_ref, S_ref = oracle_forward(oracle_mod, inp, units=units)
     e_o, e_s = compare_units(o, S_T, o_ref, S_ref, units, tol=TOL["bf16"])
     assert e_o < TOL["bf16"] and e_s < TOL["bf16"], (e_o, e_s)
+
+
+def packed_host_case(lens, H, dk, dv, dtype, seed, s0_std):
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    inp = case(1, int(cu[-1]), H, dk, dv, dtype, seed=seed, s0_std=s0_std, num_states=len(lens))
+    inp["cu_seqlens"] = torch.tensor(cu, device="cuda")
+    return inp, cu
+
+
+@pytest.mark.parametrize("lens,piece_len,s0", [
+    ([300, 0, 700, 64, 5, 1000], 256, 0.1),   # cuts inside sequences, snapped to their chunk grids
+    ([100, 200, 0], 128, 0.0),               # an empty sequence at the end; no S0
+    ([64] * 10 + [0, 129], 192, 0.1),         # many short sequences per piece
+    ([2048], 0, 0.1),                         # one sequence, default piece length
+])
+def test_packed_host_pieces(K, oracle_mod, lens, piece_len, s0):
+    """Packed batches from host memory (kda_forward_host with cu_seqlens): pieces of the
+    flat token axis, every cut on the chunk grid of the sequence it falls in, each a packed
+    launch over the states of the sequences it touches. Against one device call over the
+    whole batch (equal up to rounding: a piece may run another tensor-core form) and the
+    oracle, every unit gated; empty sequences keep S0 bit for bit."""
+    H = 2
+    inp, cu = packed_host_case(lens, H, 128, 128, "bf16", seed=len(lens) + int(cu_sum(lens)), s0_std=s0)
+    h = to_host(inp)
+    status = torch.zeros(4, dtype=torch.int32, device="cuda")
+    o, S_T = K.kda_forward_host(*(h[n] for n in NAMES), h.get("S0"), chunk=64, piece_len=piece_len,
+                                cu_seqlens=torch.tensor(cu), dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status[0]) == 0
+    o_d, S_d = K.kda_forward(*(inp[n] for n in NAMES), inp.get("S0"), chunk=64, cu_seqlens=inp["cu_seqlens"])
+    torch.cuda.synchronize()
+    o_d, S_d = o_d.cpu(), S_d.cpu()
+    units = [(n, hh) for n in range(len(lens)) for hh in range(H)]
+    o_ref, S_ref = oracle_forward(oracle_mod, inp)
+    compare_units(o, S_T, o_ref, S_ref, units, [int(x) for x in cu], tol=TOL["bf16"], label="packed host")
+    assert rel(to_f64(o), to_f64(o_d)) < 1e-2 and rel(to_f64(S_T), to_f64(S_d)) < 1e-2
+    for n, L in enumerate(lens):
+        if L == 0:
+            want = inp["S0"][n].cpu() if inp.get("S0") is not None else torch.zeros_like(S_T[n])
+            assert torch.equal(S_T[n], want)
+
+
+def test_packed_host_fp32_simt(K, oracle_mod):
+    lens = [90, 33, 0, 160]
+    H = 2
+    inp, cu = packed_host_case(lens, H, 64, 32, "f32", seed=5, s0_std=0.1)
+    h = to_host(inp)
+    o, S_T = K.kda_forward_host(*(h[n] for n in NAMES), h.get("S0"), chunk=32, piece_len=64,
+                                cu_seqlens=torch.tensor(cu))
+    torch.cuda.synchronize()
+    units = [(n, hh) for n in range(len(lens)) for hh in range(H)]
+    o_ref, S_ref = oracle_forward(oracle_mod, inp)
+    compare_units(o, S_T, o_ref, S_ref, units, [int(x) for x in cu], tol=TOL["f32"], label="packed host f32")
+
+
+def cu_sum(lens):
+    return sum(lens)
