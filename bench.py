@@ -339,7 +339,7 @@ def run_ours(args, rank, world, device):
         res["plain_prefill"] = {"ms_per_step": a.elapsed_time(b) / 3,
                                 "tokens_per_s": tokens / (a.elapsed_time(b) / 3 / 1e3),
                                 "note": "kda_forward on the same inputs, one unit per (sequence, head); outside the timed region"}
-    if args.snap_every > 0 and not seg and not w.seqlens and T >= args.snap_every:
+    if args.snap_every > 0 and not seg and not w.seqlens and T >= args.snap_every and args.path != "tc_pipe":
         # the same prefill saving the state every snap_every tokens (prefix cache)
         Ssn = torch.empty((B, T // args.snap_every, w.H, w.dv, w.dk), dtype=torch.float32, device=device)
 
@@ -361,7 +361,7 @@ def run_ours(args, rank, world, device):
                             "ms_per_step": ms_snap, "overhead_vs_step": ms_snap / kern_ms - 1.0,
                             "snapshot_bytes_per_step": Ssn.numel() * 4,
                             "note": "kda_forward_snapshots on the same inputs, outside the timed region"}
-    if not seg and not w.seqlens:
+    if not seg and not w.seqlens and args.path != "tc_pipe":  # the pipe form has no fused variant
         # the same step with the fused pre-operations (q, k normalised per row and g computed from
         # gate logits inside the kernels; the synthetic g read as logits, for timing only)
         def fused():
