@@ -51,11 +51,14 @@ constexpr uint32_t REC_UT = 33 * KB;    // 16 KB Ut (bf16), MN-major [tok][dv], 
 constexpr uint32_t REC_P = 49 * KB;     // 8 KB  P (bf16, s <= r), K-major [r][s]
 constexpr uint32_t REC_KH = 57 * KB;    // 16 KB Kh = e^{G_C - G} k, MN-major [tok][dk], 64-channel blocks 8 KB apart
 constexpr uint32_t REC_BYTES = 73 * KB;
+// a publication flag in the padding after Gamma_C, for records produced beside their chain
+constexpr uint32_t REC_FLAG = REC_GC + 512;
 constexpr uint32_t REC_A_BYTES = 32 * KB + 512;  // piece A: [REC_WQ, REC_GC + 512)
 constexpr uint32_t REC_B_BYTES = 24 * KB;        // piece B: [REC_UT, REC_KH)
 constexpr uint32_t REC_C_BYTES = 16 * KB;        // piece C: [REC_KH, REC_BYTES)
 static_assert(REC_UT + REC_B_BYTES == REC_KH && REC_KH + REC_C_BYTES == REC_BYTES, "record pieces");
 static_assert(REC_UT % 1024 == 0 && REC_P % 1024 == 0 && REC_KH % 1024 == 0, "tiles stay 1 KB aligned");
+static_assert(REC_FLAG + 4 <= REC_UT, "the flag lies outside every tile");
 
 // ------------------------------------------------------------ prep smem layout
 constexpr uint32_t P_L0 = 0;          // 32 KB k (rows 0..63) and q (rows 64..127) tiles, the Gram left operand L0 in place
@@ -103,6 +106,7 @@ struct SplitParams {
     const int32_t *chunk_base;  // packed batches: [num_units + 1] first task chunk of each sequence
     int nch;                    // dense batches: chunks per sequence
     long long tasks;            // dense batches: number of tasks (units x chunks)
+    long long flag_from = 0, flag_to = 0;  // prep kernel: clear the flags of records flag_from .. flag_to - 1
 };
 
 // Task t = (global chunk index) * H + head. The global chunk index runs over the
@@ -142,6 +146,27 @@ __device__ __forceinline__ Task task_at(const SplitParams &sp, long long t) {
     }
     k.Lc = (int)((end - k.tok0) < C ? (end - k.tok0) : C);
     return k;
+}
+
+// Flags and counters written with release and read with acquire semantics at GPU scope.
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *ptr) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned *ptr, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+// Bounded wait until a monotonic counter reaches `target`.
+__device__ __forceinline__ bool wait_counter(const unsigned *ptr, unsigned target, long long max_cycles) {
+    if (ld_acquire_gpu(ptr) >= target) return true;
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(ptr) < target) {
+        if (clock64() - t0 > max_cycles) return false;
+        __nanosleep(100);
+    }
+    return true;
 }
 
 // First task chunk of every packed sequence: base[n] = sum over m < n of ceil(len_m / C),
@@ -191,7 +216,7 @@ __global__ void chunk_base_kernel(const int32_t *cu, int num, int32_t *base) {
 // Every task of the batch, strided over the grid; the record of task t is the t-th of the
 // workspace (the two-kernel form: the chains run after this kernel has finished).
 struct StaticTasks {
-    static constexpr bool kPublish = false;
+    static constexpr bool kPublish = false, kLatePublish = false;
     const SplitParams *sp;
     long long t, total;
     __device__ bool first(Task &k) {
@@ -212,9 +237,39 @@ struct StaticTasks {
     __device__ void release(const Task &) {}
 };
 
+// Tasks first_task .. sp->tasks - 1 of a dense batch, strided over `stride` producers: the
+// last chunks' records, produced beside the chains that consume them. A record is published by
+// its flag once all of its stores have completed.
+struct TailTasks {
+    static constexpr bool kPublish = true, kLatePublish = true;
+    const SplitParams *sp;
+    long long first_task, rank, stride, t;
+    __device__ bool first(Task &k) {
+        t = first_task + rank;
+        if (t >= sp->tasks) return false;
+        k = task_at(*sp, t);
+        return true;
+    }
+    __device__ bool next(Task &k) {
+        t += stride;
+        if (t >= sp->tasks) return false;
+        k = task_at(*sp, t);
+        return true;
+    }
+    __device__ uint8_t *record(const Task &k) const { return sp->rec + (size_t)k.t * REC_BYTES; }
+    __device__ bool acquire(const Task &) { return true; }
+    __device__ void release(const Task &k) {
+        fence_proxy_async_global();
+        __threadfence();
+        st_release_gpu(reinterpret_cast<unsigned *>(record(k) + REC_FLAG), 1u);
+    }
+};
+
 // The persistent loop of a record-producing CTA over the tasks its source hands out.
 // Src::acquire (thread 0) returns once the task's record may be written, before its first
-// store; Src::release (thread 0) publishes a record whose stores have completed (kPublish).
+// store; Src::release (thread 0) publishes a record whose stores have completed (kPublish):
+// at the next task's acquire, or (kLatePublish, for sources whose acquire never waits on a
+// consumer) after that task's first bulk store, by which time the record's stores are done.
 // kFused: the variant with the fused pre-operations (p.fuse: q, k normalised per row inside the
 // operand pass, g computed from gate logits in the cumulative decay), a separate instantiation
 // so that the plain variant carries none of it.
@@ -409,10 +464,11 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
             sNorm[((l16 >> 3) * C + r) * 2 + (warp & 1)] = nv[0];
         }
         // the previous task's record stores have read their staging (and, where records are
-        // published, completed: then that record is published); this task's record may be written
+        // published at this point, completed: then that record is published); this task's
+        // record may be written
         bool slot_ok = true;
         if (tid == 0) {
-            if (Src::kPublish) {
+            if (Src::kPublish && !Src::kLatePublish) {
                 bulk_wait_all();
                 if (has_pend) src.release(pend);
                 has_pend = false;
@@ -534,7 +590,8 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
                 st2(gkrow + off_r, kf, pg2);
             }
         }
-        if (Src::kPublish) __threadfence();  // this thread's record stores before the publication
+        // this thread's record stores before the publication (late publication: fenced then)
+        if (Src::kPublish && !Src::kLatePublish) __threadfence();
         fence_proxy_async_smem();
         grp.sync();
 
@@ -591,12 +648,20 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
                 }
             }
         }
+        // (late publication) the previous record's direct stores, issued a task ago, before the
+        // sync after which it is published
+        if (Src::kLatePublish) __threadfence();
         fence_proxy_async_smem();
         tc_fence_before();
         grp.sync();
         if (tid == 0) {
             bulk_store(rec + REC_P, sm + P_PST, 8 * KB);
             bulk_commit();
+            if (Src::kLatePublish && has_pend) {  // every group but this P store: the previous record
+                bulk_wait_all_but_last();
+                src.release(pend);
+                has_pend = false;
+            }
         }
 
         // ---- T = (I + A)^{-1} (unit lower triangular) by 16 x 16 blocks
@@ -763,6 +828,10 @@ kda_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 const SplitParams sp) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    // the flags of the records that a later launch produces beside its chains start cleared
+    for (long long t = sp.flag_from + (long long)blockIdx.x * NT + threadIdx.x; t < sp.flag_to;
+         t += (long long)gridDim.x * NT)
+        *reinterpret_cast<unsigned *>(sp.rec + (size_t)t * REC_BYTES + REC_FLAG) = 0u;
     StaticTasks src{&sp, 0, 0};
     prep_loop<kFused>(tm_q, tm_k, tm_v, tm_g, sp, src, sm, Group{(int)threadIdx.x, 0u, true});
 }
@@ -800,22 +869,47 @@ __device__ __forceinline__ void u_readout(const uint8_t *ut, uint8_t *dst, int r
     }
 }
 
-// kSnap: the instantiation that also stores the state every p.snap_every tokens
-template <bool kSnap>
-__global__ void __launch_bounds__(NT, 1)
-kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp) {
+// When a chain's records are complete: all of them (an earlier kernel wrote the array), or
+// (records produced beside the chains) those of tasks below `first`, the others once their
+// flag is set. ready_now is a test, wait a bounded wait (thread 0).
+struct AllReady {
+    __device__ bool ready_now(long long) const { return true; }
+    __device__ bool wait(long long) const { return true; }
+};
+struct FlagReady {
+    const uint8_t *rec;
+    long long first;
+    __device__ const unsigned *flag(long long t) const {
+        return reinterpret_cast<const unsigned *>(rec + (size_t)t * REC_BYTES + REC_FLAG);
+    }
+    __device__ bool ready_now(long long t) const {
+        if (t < first) return true;
+        if (ld_acquire_gpu(flag(t)) == 0u) return false;
+        fence_proxy_async_global();  // the bulk copy out of the record follows its publication
+        return true;
+    }
+    __device__ bool wait(long long t) const {
+        if (t < first) return true;
+        const bool ok = wait_counter(flag(t), 1u, kWaitCycles);
+        fence_proxy_async_global();  // the bulk copy out of the record follows its publication
+        return ok;
+    }
+};
+
+// The state chain of unit (sequence n, head h) over the record array, one 256-thread group:
+// fp32 state resident in TMEM (all 512 columns), records double-buffered a chunk ahead.
+// kSnap: the instantiation that also stores the state every p.snap_every tokens.
+template <bool kSnap, class Rdy>
+__device__ __forceinline__ void chain_dbuf(const SplitParams &sp, const CUtensorMap &tm_o, uint8_t *sm, const Group &grp,
+                                           int n, int h, const Rdy &rdy) {
     const PrefillArgs &p = sp.a;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = smem_u32(sm);
     uint64_t *bar_rec = reinterpret_cast<uint64_t *>(sm + C_BAR);  // [2]: the record of buffer b
     uint64_t *bar_mma = bar_rec + 2;
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + C_TMEMADDR);
 
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = grp.tid, warp = tid >> 5, lane = tid & 31;
     const int quarter = warp & 3, half = warp >> 2;
-    const int h = blockIdx.x % p.H;
-    const int n = unit_seq(p, blockIdx.x / p.H);
     const size_t H = (size_t)p.H;
     long long t_begin, len, cbase;
     if (p.cu_seqlens) {
@@ -830,9 +924,8 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
     __nv_bfloat16 *o = static_cast<__nv_bfloat16 *>(p.o);
     const size_t state_base = ((size_t)n * H + h) * (size_t)(D * D);
     const long long nchunks = (len + C - 1) / C;
-    auto record = [&](long long c) -> const uint8_t * {
-        return sp.rec + ((size_t)(cbase + c) * H + (size_t)h) * REC_BYTES;
-    };
+    auto task = [&](long long c) -> long long { return (cbase + c) * (long long)H + h; };
+    auto record = [&](long long c) -> const uint8_t * { return sp.rec + (size_t)task(c) * REC_BYTES; };
 
     if (tid == 0) {
         mbar_init(&bar_rec[0], 1);
@@ -843,16 +936,25 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
     }
     if (warp == 0) {
         tmem_alloc(s_tmem, C_TM_COLS);
-        tmem_relinquish();
+        if (grp.relinquish) tmem_relinquish();
     }
-    __syncthreads();
+    grp.sync();
     // bit b: buffer b has a record load armed and not yet waited for / the parity of its next phase
     uint32_t rec_armed = 0, rec_phase = 0;
+    // (thread 0) per buffer, a record whose flag was not yet set when the buffer freed up: loaded
+    // just before it is needed; flag_fail: a flag wait gave up
+    long long rec_late[2] = {-1, -1};
+    bool flag_fail = false;
+    auto load_rec = [&](long long c) {
+        const int b = (int)(c & 1);
+        mbar_arrive_expect_tx(&bar_rec[b], REC_BYTES);
+        bulk_load(sm + b * C_RECSTRIDE, record(c), REC_BYTES, &bar_rec[b]);
+        rec_armed |= 1u << b;
+    };
     if (tid == 0) {  // records 0 and 1; record c + 2 is requested once chunk c's products are done
         for (int b = 0; b < 2 && b < nchunks; ++b) {
-            mbar_arrive_expect_tx(&bar_rec[b], REC_BYTES);
-            bulk_load(sm + b * C_RECSTRIDE, record(b), REC_BYTES, &bar_rec[b]);
-            rec_armed |= 1u << b;
+            if (!rdy.wait(task(b))) { flag_fail = true; break; }
+            load_rec(b);
         }
     }
     // incoming state -> TMEM (fp32, lane = dk row, column = dv) and its bf16 copy
@@ -880,7 +982,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
     }
     fence_proxy_async_smem();
     tc_fence_before();
-    __syncthreads();
+    grp.sync();
     tc_fence_after();
 
     constexpr uint32_t idKM = idesc_bf16_f32(128, 128, 0, 1);
@@ -888,15 +990,15 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
     uint32_t mma_phase = 0;
     bool aborted = false, mma_pending = false;
     auto wait_rec = [&](int b) -> bool {  // every thread takes part
-        const bool ok = mbar_wait_bounded(&bar_rec[b], (rec_phase >> b) & 1u, kWaitCycles);
+        const bool ok = !flag_fail && mbar_wait_bounded(&bar_rec[b], (rec_phase >> b) & 1u, kWaitCycles);
         if (ok) { rec_phase ^= 1u << b; rec_armed &= ~(1u << b); }
-        return __syncthreads_or(!ok) == 0;
+        return !grp.sync_or(!ok);
     };
     auto wait_mma = [&]() -> bool {
         const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
         if (ok) { mma_phase ^= 1u; mma_pending = false; }
         tc_fence_after();
-        return __syncthreads_or(!ok) == 0;
+        return !grp.sync_or(!ok);
     };
     auto issue_u = [&](int b) {  // [U ; Gamma Q S] = [-W ; Gamma Q] S into the accumulator of buffer b
         tc_fence_after();
@@ -944,7 +1046,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
                       tmem + tlane + tmu + 64u * half, p.v != nullptr);
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        grp.sync();
 
         // O = Gamma Q S + P U (rows 64..127 of the accumulator), S += Kh^T U
         if (tid == 0) {
@@ -959,9 +1061,8 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
         }
         if (!wait_mma()) { aborted = true; break; }
         if (tid == 0 && ch + 2 < nchunks) {  // this buffer's record is consumed: the one two chunks ahead
-            mbar_arrive_expect_tx(&bar_rec[b], REC_BYTES);
-            bulk_load(buf, record(ch + 2), REC_BYTES, &bar_rec[b]);
-            rec_armed |= 1u << b;
+            if (rdy.ready_now(task(ch + 2))) load_rec(ch + 2);
+            else rec_late[b] = ch + 2;
         }
 
         // the bf16 copy of the updated state: the next chunk's state product waits on it
@@ -992,8 +1093,15 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        if (tid == 0) bulk_wait_read_all();  // the previous chunk's output stores have read their staging
-        __syncthreads();
+        if (tid == 0) {
+            bulk_wait_read_all();  // the previous chunk's output stores have read their staging
+            if (rec_late[b ^ 1] == ch + 1) {  // the next record, requested late: it is needed now
+                if (rdy.wait(task(ch + 1))) load_rec(ch + 1);
+                else flag_fail = true;
+                rec_late[b ^ 1] = -1;
+            }
+        }
+        grp.sync();
         if (more) {
             if (!wait_rec(b ^ 1)) { aborted = true; break; }
             if (tid == 0) { issue_u(b ^ 1); mma_pending = true; }
@@ -1030,7 +1138,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        grp.sync();
         if (tid == 0) {
             if (Lc == C && p.o) {
                 tma_store_3d(&tm_o, sm + C_OST, 0, h, (int)tok0);
@@ -1045,6 +1153,7 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
     if (aborted) {
         if (tid == 0) {
             if (p.dev_status) atomicExch(p.dev_status, (int)KDA_ERR_TIMEOUT);
+            // a record still unpublished when the chain gave up is never requested
             for (int b = 0; b < 2; ++b)
                 if ((rec_armed >> b) & 1u) mbar_wait_bounded(&bar_rec[b], (rec_phase >> b) & 1u, kWaitCycles);
             if (mma_pending) mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
@@ -1064,11 +1173,21 @@ kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp)
         }
     }
     tc_fence_before();
-    __syncthreads();
+    grp.sync();
     if (warp == 0) {
         tc_fence_after();
         tmem_dealloc(tmem, C_TM_COLS);
     }
+}
+
+template <bool kSnap>
+__global__ void __launch_bounds__(NT, 1)
+kda_chain_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const PrefillArgs &p = sp.a;
+    chain_dbuf<kSnap>(sp, tm_o, sm, Group{(int)threadIdx.x, 0u, true}, unit_seq(p, blockIdx.x / p.H),
+                      (int)(blockIdx.x % p.H), AllReady{});
 }
 
 // ================================================= persistent pipeline (one launch)
@@ -1105,30 +1224,11 @@ struct PipeParams {
     long long ntasks;     // NC x the most chunks a unit can have
 };
 
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *ptr) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release_gpu(unsigned *ptr, unsigned v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
-// Bounded wait until a monotonic counter reaches `target`.
-__device__ __forceinline__ bool wait_counter(const unsigned *ptr, unsigned target, long long max_cycles) {
-    if (ld_acquire_gpu(ptr) >= target) return true;
-    const long long t0 = clock64();
-    while (ld_acquire_gpu(ptr) < target) {
-        if (clock64() - t0 > max_cycles) return false;
-        __nanosleep(100);
-    }
-    return true;
-}
 
 // Task t of the ring form: record tau = t / NC of chain c = t % NC (unit c: sequence c / H,
 // head c % H); tasks past the end of a unit's sequence are skipped.
 struct RingTasks {
-    static constexpr bool kPublish = true;
+    static constexpr bool kPublish = true, kLatePublish = false;
     const PipeParams *pp;
     long long t;     // the next candidate task
     long long rank;  // this producer's index among the pp->nprep producers
@@ -1567,6 +1667,42 @@ kda_chain2_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp
     chain_role<ArrayRecords, true>(p, tm_o, sm, Group{(int)threadIdx.x, 0u, true}, n, h, recs);
 }
 constexpr uint32_t CHAIN2_SMEM = X2_SMEM_USED + 1024;
+
+// The tail form (dense batches of one sequence with SMs to spare beside its units): the prep
+// kernel writes the records of the first chunks, then one cooperative launch runs every unit's
+// chain on an SM of its own (CTA c < nchain, one 256-thread group) while the other CTAs, two
+// producing groups each, write the last chunks' records; a chain waits for such a record by its
+// flag. The chains use SMs the two-kernel form leaves idle while they run.
+struct TailParams {
+    SplitParams sp;   // the records; sp.tasks = every task of the batch
+    long long first;  // the first task produced in this launch (its flag and all later ones cleared)
+    int nchain;       // (sequence, head) units = chain CTAs
+};
+constexpr uint32_t TAIL_GROUP_BYTES = (P_SMEM_USED + 1023) / 1024 * 1024;
+constexpr uint32_t TAIL_SMEM_USED = C_SMEM_BYTES - 1024 > 2 * TAIL_GROUP_BYTES ? C_SMEM_BYTES - 1024 : 2 * TAIL_GROUP_BYTES;
+constexpr uint32_t TAIL_SMEM = TAIL_SMEM_USED + 1024;
+static_assert(TAIL_SMEM <= 232448, "a chain, or two producing groups, in one CTA");
+
+template <bool kFused>
+__global__ void __launch_bounds__(2 * NT, 1)
+kda_tail_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
+                const __grid_constant__ CUtensorMap tm_o, const TailParams tp) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    const int gi = (int)(threadIdx.x >> 8);
+    const PrefillArgs &p = tp.sp.a;
+    if ((int)blockIdx.x < tp.nchain) {
+        if (gi != 0) return;  // one group carries the chain, with all of the CTA's TMEM
+        chain_dbuf<false>(tp.sp, tm_o, base, Group{(int)threadIdx.x, 1u, true}, unit_seq(p, blockIdx.x / p.H),
+                          (int)(blockIdx.x % p.H), FlagReady{tp.sp.rec, tp.first});
+    } else {
+        TailTasks src{&tp.sp, tp.first, 2LL * ((int)blockIdx.x - tp.nchain) + gi,
+                      2LL * ((int)gridDim.x - tp.nchain), 0};
+        prep_loop<kFused>(tm_q, tm_k, tm_v, tm_g, tp.sp, src, base + gi * TAIL_GROUP_BYTES,
+                          Group{(int)(threadIdx.x & (NT - 1)), 1u + (uint32_t)gi, false});
+    }
+}
 static_assert(2 * 1024 + P_SMEM_BYTES + CHAIN2_SMEM <= 233472, "a prep CTA and a compact chain share an SM");
 
 int num_sms() { return device_sm_count(); }
@@ -1764,10 +1900,78 @@ cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r) {
     return cudaGetLastError();
 }
 
+// The tail form's split of the tasks: P producing groups keep pace with the chains over the
+// last r x P x nch / units chunks, r the ratio of a chain's cycles per chunk to a producing
+// group's cycles per task. Measured on B200 (96 heads, 8192 tokens): about 4.4K and 23K (two
+// groups of one CTA per SM; a step of the two-kernel form is fastest at r = 0.19, 0.610 ms
+// against 0.636, with 26 of 128 chunks in the tail); the prep kernel does the other chunks.
+bool tail_ok(const PrefillArgs &a) {
+    const long long units = (long long)a.num_units * a.H;
+    return !packed(a) && a.num_units == 1 && a.snap_every == 0 && units + 8 <= num_sms() &&
+           (a.T + C - 1) / C >= 4;
+}
+long long tail_first_task(const PrefillArgs &a) {
+    const long long units = a.H, nch = (a.T + C - 1) / C;
+    const long long producers = 2LL * (num_sms() - units);
+    long long tail = (long long)((double)producers * (double)nch * 0.19 / (double)units);
+    tail = tail < 1 ? 1 : (tail > nch - 1 ? nch - 1 : tail);
+    return (nch - tail) * units;
+}
+
+// whether the tail kernel runs as one cooperative launch of a CTA per SM here
+bool tail_launchable(bool fused) {
+    const auto tail = fused ? kda_tail_kernel<true> : kda_tail_kernel<false>;
+    if (cudaFuncSetAttribute(tail, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TAIL_SMEM) != cudaSuccess)
+        return false;
+    int per_sm = 0, dev = 0, coop = 0;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, tail, 2 * NT, TAIL_SMEM) == cudaSuccess && per_sm >= 1 &&
+           cudaGetDevice(&dev) == cudaSuccess &&
+           cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev) == cudaSuccess && coop != 0;
+}
+
+cudaError_t launch_split_tail(const PrefillArgs &a) {
+    const size_t tokens = (size_t)a.T;
+    CUtensorMap mq, mk, mv, mg, mo;
+    if (!make_map(&mq, a.q, tokens, a.H, 64, true) || !make_map(&mk, a.k, tokens, a.H, 64, true) ||
+        !make_map(&mv, a.v ? a.v : a.q, tokens, a.H, 64, true) || !make_map(&mg, a.g, tokens, a.H, 128, false) ||
+        !make_map(&mo, a.o ? a.o : a.q, tokens, a.H, 64, true))
+        return cudaErrorInvalidValue;
+    SplitParams sp{};
+    sp.a = a;
+    sp.a.cu_seqlens = nullptr;  // dense, or one packed sequence = B = 1 of T tokens
+    sp.rec = static_cast<uint8_t *>(a.workspace);
+    sp.nch = (a.T + C - 1) / C;
+    const long long total = split_tasks_bound(a), first = tail_first_task(a);
+    // the first chunks' records, clearing the flags of the others
+    const auto prep = a.fuse ? kda_prep_kernel<true> : kda_prep_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)P_SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(prep, cudaFuncAttributePreferredSharedMemoryCarveout, (int)cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    SplitParams s1 = sp;
+    s1.tasks = first;
+    s1.flag_from = first;
+    s1.flag_to = total;
+    const long long grid_p = first < 2LL * num_sms() ? first : 2LL * num_sms();
+    prep<<<(unsigned)grid_p, NT, P_SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, s1);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // the chains, and the last chunks' records beside them
+    const auto tail = a.fuse ? kda_tail_kernel<true> : kda_tail_kernel<false>;
+    TailParams tp{};
+    tp.sp = sp;
+    tp.sp.tasks = total;
+    tp.first = first;
+    tp.nchain = a.H;
+    void *args[] = {&mq, &mk, &mv, &mg, &mo, &tp};
+    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(tail), dim3(num_sms()), dim3(2 * NT), args,
+                                       TAIL_SMEM, a.stream);
+}
+
 cudaError_t launch_prefill_split(const PrefillArgs &a) {
     if (a.num_units == 0) return cudaSuccess;
     const size_t tokens = a.cu_seqlens ? (size_t)a.T : (size_t)a.B * (size_t)a.T;
     if (tokens == 0) return launch_prefill_simt(a);
+    if (tail_ok(a) && tail_launchable(a.fuse != 0)) return launch_split_tail(a);
     SplitRecords r;
     cudaError_t e = launch_split_records(a, &r);
     if (e != cudaSuccess) return e;

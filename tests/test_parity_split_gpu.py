@@ -90,6 +90,24 @@ def test_split_g_min_runs(K, oracle_mod, form):
     compare_units(o, ST, o_ref, S_ref, [(0, 0), (0, 1)], tol=TOL["bf16"], label="split g_min")
 
 
+@pytest.mark.parametrize("spare", [8, 60])
+def test_split_one_sequence_records_beside_the_chains(K, oracle_mod, spare):
+    """One sequence whose heads leave `spare` SMs beside their chains: the prep kernel writes
+    the first chunks' records and the last ones are produced on the spare SMs while the chains
+    run (each chain waits for such a record by its flag). Sampled heads against the oracle,
+    every head bit for bit against the pipe form (the same records and chain arithmetic), and
+    a ragged last chunk."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    H = sms - spare
+    inp = case(1, 64 * 11 + 37, H, 128, 128, "bf16", seed=90 + spare, s0_std=0.1, g_min_frac=0.1)
+    o, ST = fwd(K, inp, "tc_split")
+    units = [(0, h) for h in (0, 1, H // 2, H - 2, H - 1)]
+    o_ref, S_ref = oracle_forward(oracle_mod, inp, units=units)
+    compare_units(o, ST, o_ref, S_ref, units, tol=TOL["bf16"], label=f"split, {spare} spare SMs")
+    o_p, S_p = fwd(K, inp, "tc_pipe")
+    assert torch.equal(o, o_p) and torch.equal(ST, S_p)
+
+
 def test_workspace_decides_the_form(K):
     """AUTO with the reported workspace runs the split form; with only the pipe form's ring it
     runs the pipe form; with a few bytes (or none) the single form; a forced form with too
