@@ -1683,7 +1683,8 @@ constexpr uint32_t TAIL_SMEM_USED = C_SMEM_BYTES - 1024 > 2 * TAIL_GROUP_BYTES ?
 constexpr uint32_t TAIL_SMEM = TAIL_SMEM_USED + 1024;
 static_assert(TAIL_SMEM <= 232448, "a chain, or two producing groups, in one CTA");
 
-template <bool kFused>
+// kFused: the producers' fused pre-operations; kSnap: the chains' state snapshots
+template <bool kFused, bool kSnap>
 __global__ void __launch_bounds__(2 * NT, 1)
 kda_tail_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -1694,7 +1695,7 @@ kda_tail_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const PrefillArgs &p = tp.sp.a;
     if ((int)blockIdx.x < tp.nchain) {
         if (gi != 0) return;  // one group carries the chain, with all of the CTA's TMEM
-        chain_dbuf<false>(tp.sp, tm_o, base, Group{(int)threadIdx.x, 1u, true}, unit_seq(p, blockIdx.x / p.H),
+        chain_dbuf<kSnap>(tp.sp, tm_o, base, Group{(int)threadIdx.x, 1u, true}, unit_seq(p, blockIdx.x / p.H),
                           (int)(blockIdx.x % p.H), FlagReady{tp.sp.rec, tp.first});
     } else {
         TailTasks src{&tp.sp, tp.first, 2LL * ((int)blockIdx.x - tp.nchain) + gi,
@@ -1903,24 +1904,31 @@ cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r) {
 // The tail form's split of the tasks: P producing groups keep pace with the chains over the
 // last r x P x nch / units chunks, r the ratio of a chain's cycles per chunk to a producing
 // group's cycles per task. Measured on B200 (96 heads, 8192 tokens): about 4.4K and 23K (two
-// groups of one CTA per SM; a step of the two-kernel form is fastest at r = 0.19, 0.610 ms
-// against 0.636, with 26 of 128 chunks in the tail); the prep kernel does the other chunks.
+// groups of one CTA per SM; the step is fastest at r = 0.19, 0.610 ms against 0.636 for the
+// two-kernel form, with 26 of 128 chunks in the tail; the producers with fused pre-operations
+// take about 1.4 times as long per task); the prep kernel does the other chunks.
 bool tail_ok(const PrefillArgs &a) {
     const long long units = (long long)a.num_units * a.H;
-    return !packed(a) && a.num_units == 1 && a.snap_every == 0 && units + 8 <= num_sms() &&
+    return !packed(a) && a.num_units == 1 && !(a.fuse && a.snap_every) && units + 8 <= num_sms() &&
            (a.T + C - 1) / C >= 4;
+}
+const void *tail_kernel_for(const PrefillArgs &a) {
+    if (a.snap_every) return reinterpret_cast<const void *>(kda_tail_kernel<false, true>);
+    return a.fuse ? reinterpret_cast<const void *>(kda_tail_kernel<true, false>)
+                  : reinterpret_cast<const void *>(kda_tail_kernel<false, false>);
 }
 long long tail_first_task(const PrefillArgs &a) {
     const long long units = a.H, nch = (a.T + C - 1) / C;
     const long long producers = 2LL * (num_sms() - units);
-    long long tail = (long long)((double)producers * (double)nch * 0.19 / (double)units);
+    const double r = a.fuse ? 0.14 : 0.19;
+    long long tail = (long long)((double)producers * (double)nch * r / (double)units);
     tail = tail < 1 ? 1 : (tail > nch - 1 ? nch - 1 : tail);
     return (nch - tail) * units;
 }
 
 // whether the tail kernel runs as one cooperative launch of a CTA per SM here
-bool tail_launchable(bool fused) {
-    const auto tail = fused ? kda_tail_kernel<true> : kda_tail_kernel<false>;
+bool tail_launchable(const PrefillArgs &a) {
+    const void *tail = tail_kernel_for(a);
     if (cudaFuncSetAttribute(tail, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TAIL_SMEM) != cudaSuccess)
         return false;
     int per_sm = 0, dev = 0, coop = 0;
@@ -1956,22 +1964,21 @@ cudaError_t launch_split_tail(const PrefillArgs &a) {
     prep<<<(unsigned)grid_p, NT, P_SMEM_BYTES, a.stream>>>(mq, mk, mv, mg, s1);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     // the chains, and the last chunks' records beside them
-    const auto tail = a.fuse ? kda_tail_kernel<true> : kda_tail_kernel<false>;
+    const void *tail = tail_kernel_for(a);
     TailParams tp{};
     tp.sp = sp;
     tp.sp.tasks = total;
     tp.first = first;
     tp.nchain = a.H;
     void *args[] = {&mq, &mk, &mv, &mg, &mo, &tp};
-    return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(tail), dim3(num_sms()), dim3(2 * NT), args,
-                                       TAIL_SMEM, a.stream);
+    return cudaLaunchCooperativeKernel(tail, dim3(num_sms()), dim3(2 * NT), args, TAIL_SMEM, a.stream);
 }
 
 cudaError_t launch_prefill_split(const PrefillArgs &a) {
     if (a.num_units == 0) return cudaSuccess;
     const size_t tokens = a.cu_seqlens ? (size_t)a.T : (size_t)a.B * (size_t)a.T;
     if (tokens == 0) return launch_prefill_simt(a);
-    if (tail_ok(a) && tail_launchable(a.fuse != 0)) return launch_split_tail(a);
+    if (tail_ok(a) && tail_launchable(a)) return launch_split_tail(a);
     SplitRecords r;
     cudaError_t e = launch_split_records(a, &r);
     if (e != cudaSuccess) return e;

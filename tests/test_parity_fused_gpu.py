@@ -89,6 +89,21 @@ def test_fused_decode(K, oracle_mod, dtype):
     assert rel(to_f64(S), S_ref) < TOL[dtype]
 
 
+def test_fused_one_sequence_split_form(K, oracle_mod):
+    """One sequence on the split form: the producers of the last chunks' records, beside the
+    chains, apply the fused pre-operations too."""
+    B, T, H = 1, 64 * 12 + 9, 3
+    inp = raw_inputs(B, T, H, 128, 128, "bf16", seed=71)
+    o, ST = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], chunk=64,
+                          path="tc_split", fuse=K.KDA_FUSE_NORM_QK | K.KDA_FUSE_GATE_LOGITS)
+    torch.cuda.synchronize()
+    r = reference_inputs(inp)
+    S0 = to_f64(inp["S0"])
+    for h in range(H):
+        ou, su = oracle_mod.forward(*(r[x][0, :, h] for x in ("q", "k", "v", "g", "beta")), S0=S0[0, h])
+        assert rel(to_f64(o[0, :, h]), ou) < TOL["bf16"] and rel(to_f64(ST[0, h]), su) < TOL["bf16"], h
+
+
 def test_unfused_call_is_unchanged(K):
     """fuse = 0 takes the plain entry point (normalised inputs, g as log-decays)."""
     inp = make_inputs(1, 200, 2, 128, 128, "bf16", seed=93, device="cuda")
