@@ -108,6 +108,28 @@ def test_split_one_sequence_records_beside_the_chains(K, oracle_mod, spare):
     assert torch.equal(o, o_p) and torch.equal(ST, S_p)
 
 
+def test_split_one_sequence_in_a_cuda_graph(K):
+    """The one-sequence split step (a cooperative launch beside the prep kernel) captured in a
+    CUDA graph and replayed: the same outputs as the eager call, bit for bit."""
+    inp = case(1, 64 * 9 + 3, 4, 128, 128, "bf16", seed=93, s0_std=0.1)
+    o_e, S_e = fwd(K, inp, "tc_split")
+    o = torch.empty_like(o_e)
+    ST = torch.empty_like(S_e)
+    ws = torch.empty(K.kda_forward_workspace_size(1, inp["k"].shape[1], 4, 128, 128, 64, 1, torch.bfloat16),
+                     dtype=torch.uint8, device="cuda")
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], chunk=64, o=o, S_T=ST,
+                      workspace=ws, path="tc_split")
+    for _ in range(2):
+        o.zero_()
+        g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(o, o_e) and torch.equal(ST, S_e)
+
+
 def test_workspace_decides_the_form(K):
     """AUTO with the reported workspace runs the split form; with only the pipe form's ring it
     runs the pipe form; with a few bytes (or none) the single form; a forced form with too
