@@ -85,7 +85,12 @@ typedef enum { KDA_FUSE_NORM_QK = 1, KDA_FUSE_GATE_LOGITS = 2 } kda_fuse;
  *    chunk after chunk; no workspace beyond the packed-batch schedule.
  *  - split (TC_SPLIT): a chunk-parallel kernel writes every chunk's record to
  *    the workspace, then a second kernel carries each unit's state across its
- *    chunks (73 KiB of workspace per chunk per head).
+ *    chunks (73 KiB of workspace per chunk per head). For one sequence whose
+ *    heads leave at least 8 SMs free (and 4 or more chunks), the first kernel
+ *    writes the first chunks' records only and the second is a cooperative
+ *    launch in which the free SMs write the last ones beside the chains (the
+ *    same records and arithmetic, bit for bit; the same workspace). Where a
+ *    cooperative launch is not possible, the two-kernel order runs.
  *  - pipe (TC_PIPE): one cooperative launch runs the chains and the producers
  *    at once, the records passing through a ring of 4 per unit; for at most
  *    two thirds of twice the SM count of units (197 on 148 SMs), else
