@@ -359,7 +359,8 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
     const int cin = c0 & 63;
     constexpr int HR = SUB / 2;
     constexpr uint32_t idG = idesc_bf16_f32(128, 32, 0, 0);
-    constexpr uint32_t idKM = idesc_bf16_f32(128, 128, 0, 1);
+    constexpr uint32_t idWU = idesc_bf16_f32(128, 256, 0, 1);
+    static_assert(P_GV == P_GK + 16 * KB && P_TM_UT == P_TM_W + 128, "[Gamma k | v] and [W | Ut] are contiguous");
 
     while (have) {
         Task nxt{};
@@ -735,14 +736,14 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
         fence_proxy_async_smem();
         grp.sync();
 
-        // ---- [W | Ut] = T Diag(beta) [Gamma K | V]
+        // ---- [W | Ut] = T Diag(beta) [Gamma K | V]: one N = 256 chain, Gamma k and v being four
+        // consecutive 64-column blocks and W, Ut consecutive accumulators (an MMA instruction
+        // costs about as much at N = 128 as at N = 256, so this halves the instructions)
         if (tid == 0) {
             tc_fence_after();
             Opnd A{sbase + P_TB, false, 16 * KB, 0};
-            Opnd BK{sbase + P_GK, true, 0, 8 * KB};
-            Opnd BV{sbase + P_GV, true, 0, 8 * KB};
-            mma_chain<C / 16>(tmem + P_TM_W, A, BK, idKM, false);
-            mma_chain<C / 16>(tmem + P_TM_UT, A, BV, idKM, false);
+            Opnd BKV{sbase + P_GK, true, 0, 8 * KB};
+            mma_chain<C / 16>(tmem + P_TM_W, A, BKV, idWU, false);
             mma_commit(bar_mma);
         }
         {
