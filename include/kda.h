@@ -85,8 +85,8 @@ typedef enum { KDA_FUSE_NORM_QK = 1, KDA_FUSE_GATE_LOGITS = 2 } kda_fuse;
  *    chunk after chunk; no workspace beyond the packed-batch schedule.
  *  - split (TC_SPLIT): a chunk-parallel kernel writes every chunk's record to
  *    the workspace, then a second kernel carries each unit's state across its
- *    chunks (73 KiB of workspace per chunk per head). For one sequence whose
- *    heads leave at least 8 SMs free (and 4 or more chunks), the first kernel
+ *    chunks (73 KiB of workspace per chunk per head). For one sequence of 32 or
+ *    more heads that leave at least 8 SMs free (and 4 or more chunks), the first kernel
  *    writes the first chunks' records only and the second is a cooperative
  *    launch in which the free SMs write the last ones beside the chains (the
  *    same records and arithmetic, bit for bit; the same workspace). Where a

@@ -1908,10 +1908,12 @@ cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r) {
 // groups of one CTA per SM; the step is fastest at r = 0.19, 0.610 ms against 0.636 for the
 // two-kernel form, with 26 of 128 chunks in the tail; the producers with fused pre-operations
 // take about 1.4 times as long per task); the prep kernel does the other chunks.
+// With few units the chains dominate the step (8 heads x 65,536 tokens: 2.7 ms, the prep of all
+// records 0.27 ms), and the tail form only adds its flag checks to them.
 bool tail_ok(const PrefillArgs &a) {
     const long long units = (long long)a.num_units * a.H;
-    return !packed(a) && a.num_units == 1 && !(a.fuse && a.snap_every) && units + 8 <= num_sms() &&
-           (a.T + C - 1) / C >= 4;
+    return !packed(a) && a.num_units == 1 && !(a.fuse && a.snap_every) && units >= 32 &&
+           units + 8 <= num_sms() && (a.T + C - 1) / C >= 4;
 }
 const void *tail_kernel_for(const PrefillArgs &a) {
     if (a.snap_every) return reinterpret_cast<const void *>(kda_tail_kernel<false, true>);

@@ -90,9 +90,9 @@ def test_fused_decode(K, oracle_mod, dtype):
 
 
 def test_fused_one_sequence_split_form(K, oracle_mod):
-    """One sequence on the split form: the producers of the last chunks' records, beside the
-    chains, apply the fused pre-operations too."""
-    B, T, H = 1, 64 * 12 + 9, 3
+    """One sequence of 40 heads on the split form: the producers of the last chunks' records,
+    beside the chains, apply the fused pre-operations too."""
+    B, T, H = 1, 64 * 12 + 9, 40
     inp = raw_inputs(B, T, H, 128, 128, "bf16", seed=71)
     o, ST = K.kda_forward(inp["q"], inp["k"], inp["v"], inp["g"], inp["beta"], inp["S0"], chunk=64,
                           path="tc_split", fuse=K.KDA_FUSE_NORM_QK | K.KDA_FUSE_GATE_LOGITS)

@@ -109,13 +109,14 @@ def test_split_one_sequence_records_beside_the_chains(K, oracle_mod, spare):
 
 
 def test_split_one_sequence_in_a_cuda_graph(K):
-    """The one-sequence split step (a cooperative launch beside the prep kernel) captured in a
-    CUDA graph and replayed: the same outputs as the eager call, bit for bit."""
-    inp = case(1, 64 * 9 + 3, 4, 128, 128, "bf16", seed=93, s0_std=0.1)
+    """The one-sequence split step (40 heads: a cooperative launch beside the prep kernel)
+    captured in a CUDA graph and replayed: the same outputs as the eager call, bit for bit."""
+    H = 40
+    inp = case(1, 64 * 9 + 3, H, 128, 128, "bf16", seed=93, s0_std=0.1)
     o_e, S_e = fwd(K, inp, "tc_split")
     o = torch.empty_like(o_e)
     ST = torch.empty_like(S_e)
-    ws = torch.empty(K.kda_forward_workspace_size(1, inp["k"].shape[1], 4, 128, 128, 64, 1, torch.bfloat16),
+    ws = torch.empty(K.kda_forward_workspace_size(1, inp["k"].shape[1], H, 128, 128, 64, 1, torch.bfloat16),
                      dtype=torch.uint8, device="cuda")
     side = torch.cuda.Stream()
     side.wait_stream(torch.cuda.current_stream())
