@@ -444,12 +444,15 @@ int kda_decode_multi(const void *q, const void *k, const void *v, const void *g,
                      int *dev_status, void *stream);
 
 /*
- * Diagnostic: one CTA waits, through the same bounded-wait helper the
- * tensor-core prefill uses for every mbarrier wait, on an mbarrier that
- * nothing arrives on; after max_cycles SM clocks (1 .. 4e9) it gives up,
- * stores KDA_ERR_TIMEOUT into *dev_status (device int, 16-byte aligned) and
- * returns. Nothing faults or hangs and the stream stays usable; used to test
- * failure reporting without a GPU fault.
+ * Diagnostic: one CTA waits, through the same bounded-wait helpers the
+ * tensor-core prefill uses, on an mbarrier that nothing arrives on (every wait
+ * on a copy or an MMA) and then on a flag in global memory that nothing sets
+ * (a chain waiting for a record produced beside it). After max_cycles SM clocks
+ * (1 .. 4e9) each wait gives up. dev_status is 4 device ints, 16-byte aligned:
+ * [0] receives KDA_ERR_TIMEOUT from the mbarrier wait, [1] is the flag (the
+ * caller sets it to zero), [2] receives KDA_ERR_TIMEOUT from the flag wait.
+ * Nothing faults or hangs and the stream stays usable; used to test failure
+ * reporting without a GPU fault.
  */
 int kda_selftest_wait_timeout(int *dev_status, long long max_cycles, void *stream);
 

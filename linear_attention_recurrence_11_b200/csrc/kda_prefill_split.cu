@@ -148,27 +148,6 @@ __device__ __forceinline__ Task task_at(const SplitParams &sp, long long t) {
     return k;
 }
 
-// Flags and counters written with release and read with acquire semantics at GPU scope.
-__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *ptr) {
-    unsigned v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
-    return v;
-}
-__device__ __forceinline__ void st_release_gpu(unsigned *ptr, unsigned v) {
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
-}
-__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
-// Bounded wait until a monotonic counter reaches `target`.
-__device__ __forceinline__ bool wait_counter(const unsigned *ptr, unsigned target, long long max_cycles) {
-    if (ld_acquire_gpu(ptr) >= target) return true;
-    const long long t0 = clock64();
-    while (ld_acquire_gpu(ptr) < target) {
-        if (clock64() - t0 > max_cycles) return false;
-        __nanosleep(100);
-    }
-    return true;
-}
-
 // First task chunk of every packed sequence: base[n] = sum over m < n of ceil(len_m / C),
 // base[num] = the total. One block, tiles of blockDim.x sequences with a running carry.
 __global__ void chunk_base_kernel(const int32_t *cu, int num, int32_t *base) {

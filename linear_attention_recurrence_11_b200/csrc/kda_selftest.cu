@@ -1,9 +1,11 @@
-// Self-test of the bounded waits that every mbarrier wait of the tensor-core
-// prefill goes through: a kernel waits, with the same helper and the same
-// reporting, on an mbarrier that nothing ever arrives on. The wait gives up
-// after max_cycles SM clocks, the kernel records KDA_ERR_TIMEOUT in the status
-// word and returns; nothing faults, traps or hangs, and the context stays
-// usable. Used by the failure-detection tests.
+// Self-test of the bounded waits of the tensor-core prefill: a kernel waits, with
+// the same helpers and the same reporting, on an mbarrier that nothing ever
+// arrives on (every wait on a copy or an MMA), then on a flag in global memory
+// that nothing ever sets (a chain waiting for a record produced by another CTA
+// of its launch). Each wait gives up after max_cycles SM clocks and the kernel
+// records KDA_ERR_TIMEOUT, for the mbarrier in dev_status[0] and for the flag in
+// dev_status[2] (dev_status[1] is the flag, zero on entry); nothing faults, traps
+// or hangs, and the context stays usable. Used by the failure-detection tests.
 #include "kda_internal.cuh"
 #include "kda_sm100.cuh"
 
@@ -19,7 +21,11 @@ __global__ void kda_wait_selftest_kernel(int *dev_status, long long max_cycles) 
     __syncthreads();
     // phase 0 never completes: no thread arrives and no copy is in flight
     const bool ok = sm100::mbar_wait_bounded(&bar, 0, max_cycles);
-    if (__syncthreads_or(!ok) && threadIdx.x == 0 && dev_status) atomicExch(dev_status, (int)KDA_ERR_TIMEOUT);
+    if (__syncthreads_or(!ok) && threadIdx.x == 0) atomicExch(dev_status, (int)KDA_ERR_TIMEOUT);
+    // the flag stays zero: nothing in this launch sets it
+    if (threadIdx.x == 0 &&
+        !sm100::wait_counter(reinterpret_cast<const unsigned *>(dev_status + 1), 1u, max_cycles))
+        atomicExch(dev_status + 2, (int)KDA_ERR_TIMEOUT);
 }
 
 }  // namespace

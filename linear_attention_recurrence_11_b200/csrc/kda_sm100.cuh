@@ -60,6 +60,30 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
     return true;
 }
 
+// Flags and counters in global memory, written with release and read with acquire semantics
+// at GPU scope (records and states handed between CTAs of one launch).
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned *ptr) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(ptr) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(unsigned *ptr, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(ptr), "r"(v) : "memory");
+}
+// orders this thread's earlier generic accesses to global memory with its later async-proxy ones
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+// Bounded wait until a monotonic counter reaches `target`: false if it did not within
+// `max_cycles` SM clock cycles (the caller records the timeout and unwinds).
+__device__ __forceinline__ bool wait_counter(const unsigned *ptr, unsigned target, long long max_cycles) {
+    if (ld_acquire_gpu(ptr) >= target) return true;
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(ptr) < target) {
+        if (clock64() - t0 > max_cycles) return false;
+        __nanosleep(100);
+    }
+    return true;
+}
+
 // Bulk copy (no tensor map, no multicast) of `bytes` contiguous bytes from global to
 // shared memory, completing on `bar` as transaction bytes. Both addresses 16-byte
 // aligned, bytes a multiple of 16.

@@ -1,7 +1,9 @@
 """Failure detection on the GPU without a fault: a kernel waits (bounded) on an
 mbarrier that nothing arrives on, through the same helper as every mbarrier
-wait of the tensor-core prefill; it must give up, report KDA_ERR_TIMEOUT in the
-status word and leave the context usable for the next call."""
+wait of the tensor-core prefill, and on a flag in global memory that nothing
+sets, through the same helper as a chain waiting for a record produced beside
+it; it must give up on both, report KDA_ERR_TIMEOUT for each and leave the
+context usable for the next call."""
 import pytest
 import torch
 
@@ -20,9 +22,10 @@ def K():
 
 def test_wait_runs_out_and_reports(K, oracle_mod):
     status = torch.zeros(4, dtype=torch.int32, device="cuda")
-    K.kda_selftest_wait_timeout(status, max_cycles=20_000_000)  # ~10 ms of SM clocks
+    K.kda_selftest_wait_timeout(status, max_cycles=20_000_000)  # ~10 ms of SM clocks per wait
     torch.cuda.synchronize()
-    assert int(status[0]) == K.KDA_ERR_TIMEOUT
+    assert int(status[0]) == K.KDA_ERR_TIMEOUT  # the mbarrier wait
+    assert int(status[1]) == 0 and int(status[2]) == K.KDA_ERR_TIMEOUT  # the flag wait
     # the context is intact: a prefill right after runs and matches the oracle
     inp = case(1, 200, 2, 128, 128, "bf16", seed=81, s0_std=0.1)
     st2 = torch.zeros(4, dtype=torch.int32, device="cuda")
