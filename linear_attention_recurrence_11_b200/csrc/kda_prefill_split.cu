@@ -627,6 +627,10 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
                         *reinterpret_cast<uint4 *>(prow + sw128_offset(r, s)) = make_uint4(0, 0, 0, 0);
                 }
             }
+            // T Diag(beta) (bf16, rows 0..63) starts as zeros: the inverse writes its lower blocks
+            // (L0 is free: the Gram products are done)
+            *reinterpret_cast<uint4 *>(sm + P_TB + 16 * tid) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4 *>(sm + P_TB + 16 * NT + 16 * tid) = make_uint4(0, 0, 0, 0);
         }
         // (late publication) the previous record's direct stores, issued a task ago, before the
         // sync after which it is published
@@ -664,38 +668,23 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
                 for (int ss = 0; ss < rr; ++ss) acc[ss & 3] = fmaf(-a[ss], x[ss], acc[ss & 3]);
                 x[rr] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             }
+            // T_ii, and its column times beta into T Diag(beta) (x is 0 above the diagonal)
+            const float bcol = sBeta[o0 + cc];
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) TF[(o0 + rr) * LDT + o0 + cc] = x[rr];
+            for (int rr = 0; rr < 16; ++rr) {
+                TF[(o0 + rr) * LDT + o0 + cc] = x[rr];
+                *reinterpret_cast<__nv_bfloat16 *>(sm + P_TB + sw128_offset(o0 + rr, o0 + cc)) =
+                    __float2bfloat16_rn(x[rr] * bcol);
+            }
             if ((warp & 1) == 0) {
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) TF[(o0 + rr) * LDT + o0 + 16 + cc] = 0.f;
             }
         }
         grp.sync();
-        tri_inverse_offdiag(AF, TF, XS, tid, grp.id);
-        // T Diag(beta) -> bf16 A operand, rows 0..63 (rows 64..127 of the product are never read)
-        {
-            const int r = tid >> 3, pc = (tid & 7) * 8;
-            const float4 b0 = *reinterpret_cast<const float4 *>(sBeta + pc);
-            const float4 b1 = *reinterpret_cast<const float4 *>(sBeta + pc + 4);
-            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int ri = r + 32 * i;
-                const float4 t0 = *reinterpret_cast<const float4 *>(TF + ri * LDT + pc);
-                const float4 t1 = *reinterpret_cast<const float4 *>(TF + ri * LDT + pc + 4);
-                const float tv[8] = {t0.x, t0.y, t0.z, t0.w, t1.x, t1.y, t1.z, t1.w};
-                float u[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) u[e] = (pc + e <= ri) ? tv[e] * bb[e] : 0.f;
-                uint4 w;
-                w.x = pack_bf2(u[0], u[1]);
-                w.y = pack_bf2(u[2], u[3]);
-                w.z = pack_bf2(u[4], u[5]);
-                w.w = pack_bf2(u[6], u[7]);
-                *reinterpret_cast<uint4 *>(sm + P_TB + sw128_offset(ri, pc)) = w;
-            }
-        }
+        // the off-diagonal blocks of T, each also written times beta into T Diag(beta): the bf16
+        // A operand of [W | Ut], rows 0..63 (rows 64..127 of the product are never read)
+        tri_inverse_offdiag(AF, TF, XS, tid, grp.id, sm + P_TB, sBeta);
         // ---- v of this task (zero rows past the end; all zero for a transition pass)
         if (has_v) {
             const bool ok = mbar_wait_bounded(bar_v, v_phase, kWaitCycles);

@@ -127,12 +127,19 @@ __device__ __forceinline__ void warp_mma_16x8(const float *A, int lda, int ar, i
     }
 }
 
-// Store a C fragment of warp_mma_16x8 (times `scale`) at D[dr + .., dc + ..].
+// Store a C fragment of warp_mma_16x8 (times `scale`) at D[dr + .., dc + ..]; with tb, also
+// the same values times beta[column] as bf16 at (row, column) of tb, a 128-byte swizzled tile.
 __device__ __forceinline__ void warp_store_16x8(float *Dm, int ldd, int dr, int dc, const float (&c)[4],
-                                                float scale) {
+                                                float scale, uint8_t *tb = nullptr, const float *beta = nullptr) {
     const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
-    *reinterpret_cast<float2 *>(Dm + (dr + g) * ldd + dc + 2 * t) = make_float2(scale * c[0], scale * c[1]);
-    *reinterpret_cast<float2 *>(Dm + (dr + g + 8) * ldd + dc + 2 * t) = make_float2(scale * c[2], scale * c[3]);
+    const float2 lo = make_float2(scale * c[0], scale * c[1]), hi = make_float2(scale * c[2], scale * c[3]);
+    *reinterpret_cast<float2 *>(Dm + (dr + g) * ldd + dc + 2 * t) = lo;
+    *reinterpret_cast<float2 *>(Dm + (dr + g + 8) * ldd + dc + 2 * t) = hi;
+    if (tb) {
+        const float b0 = beta[dc + 2 * t], b1 = beta[dc + 2 * t + 1];
+        st_bf2(tb + sw128_offset(dr + g, dc + 2 * t), lo.x * b0, lo.y * b1);
+        st_bf2(tb + sw128_offset(dr + g + 8, dc + 2 * t), hi.x * b0, hi.y * b1);
+    }
 }
 
 // Off-diagonal part of T = (I + A)^{-1} (64 x 64 unit lower triangular) once the
@@ -142,9 +149,11 @@ __device__ __forceinline__ void warp_store_16x8(float *Dm, int ldd, int dr, int 
 //   level 2:  T[32:64, 0:32] = -T[32:64, 32:64] A[32:64, 0:32] T[0:32, 0:32]  (32 x 32)
 // i.e. the 2 x 2 block inverse applied twice; each product is a handful of
 // warp-level TF32 MMAs. A: 64 x LDA fp32 (strictly lower), T: 64 x LDT fp32,
-// XS: scratch of 32 x 36 fp32.
+// XS: scratch of 32 x 36 fp32. With tb, every block of T computed here is also written
+// times beta[column] as bf16 into tb (the A operand T Diag(beta), 128-byte swizzled rows).
 __device__ __forceinline__ void tri_inverse_offdiag(const float *AF, float *TF, float *XS, int tid,
-                                                    uint32_t bar_id = 0) {
+                                                    uint32_t bar_id = 0, uint8_t *tb = nullptr,
+                                                    const float *beta = nullptr) {
     const int warp = tid >> 5;
     float c[4];
     // level 1: 2 blocks x 2 column tiles of 8 -> warps 0..3
@@ -157,7 +166,7 @@ __device__ __forceinline__ void tri_inverse_offdiag(const float *AF, float *TF, 
     group_sync(bar_id);
     if (warp < 4) {
         warp_mma_16x8<16>(TF, LDT, i1, i1, XS, LDX, 16 * b, 8 * nt, c);       // T_ij = -T_ii X
-        warp_store_16x8(TF, LDT, i1, j1 + 8 * nt, c, -1.f);
+        warp_store_16x8(TF, LDT, i1, j1 + 8 * nt, c, -1.f, tb, beta);
     }
     group_sync(bar_id);
     // level 2: 2 row tiles x 4 column tiles -> warps 0..7
@@ -166,7 +175,7 @@ __device__ __forceinline__ void tri_inverse_offdiag(const float *AF, float *TF, 
     warp_store_16x8(XS, LDX, 16 * mt, 8 * n2, c, 1.f);
     group_sync(bar_id);
     warp_mma_16x8<32>(TF, LDT, 32 + 16 * mt, 32, XS, LDX, 0, 8 * n2, c);       // T21 = -T_hi X
-    warp_store_16x8(TF, LDT, 32 + 16 * mt, 8 * n2, c, -1.f);
+    warp_store_16x8(TF, LDT, 32 + 16 * mt, 8 * n2, c, -1.f, tb, beta);
     group_sync(bar_id);
 }
 
