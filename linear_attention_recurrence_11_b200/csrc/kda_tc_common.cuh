@@ -162,9 +162,7 @@ __device__ __forceinline__ void tri_inverse_offdiag(const float *AF, float *TF, 
     if (warp < 4) {
         warp_mma_16x8<16>(AF, LDA, i1, j1, TF, LDT, j1, j1 + 8 * nt, c);     // X = A_ij T_jj
         warp_store_16x8(XS, LDX, 16 * b, 8 * nt, c, 1.f);
-    }
-    group_sync(bar_id);
-    if (warp < 4) {
+        __syncwarp();  // the product below reads only the 16 x 8 tile of X this warp wrote
         warp_mma_16x8<16>(TF, LDT, i1, i1, XS, LDX, 16 * b, 8 * nt, c);       // T_ij = -T_ii X
         warp_store_16x8(TF, LDT, i1, j1 + 8 * nt, c, -1.f, tb, beta);
     }
