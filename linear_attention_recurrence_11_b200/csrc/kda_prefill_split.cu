@@ -685,12 +685,14 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
         // the off-diagonal blocks of T, each also written times beta into T Diag(beta): the bf16
         // A operand of [W | Ut], rows 0..63 (rows 64..127 of the product are never read)
         tri_inverse_offdiag(AF, TF, XS, tid, grp.id, sm + P_TB, sBeta);
-        // ---- v of this task (zero rows past the end; all zero for a transition pass)
+        // ---- v of this task (zero rows past the end; all zero for a transition pass). Every
+        // thread has seen the copy complete before it zeroes rows of it, and one barrier both
+        // publishes the tile to the tensor cores and agrees on a wait that ran out.
+        bool v_ok = true;
         if (has_v) {
-            const bool ok = mbar_wait_bounded(bar_v, v_phase, kWaitCycles);
-            if (ok) { v_phase ^= 1u; v_armed = false; }
-            if (grp.sync_or(!ok)) { aborted = true; break; }
-            if (Lc < C) {
+            v_ok = mbar_wait_bounded(bar_v, v_phase, kWaitCycles);
+            if (v_ok) { v_phase ^= 1u; v_armed = false; }
+            if (v_ok && Lc < C) {
                 for (int idx = tid; idx < (C - Lc) * 16; idx += NT) {
                     const int r = Lc + idx / 16, q16 = idx % 16;
                     *reinterpret_cast<uint4 *>(sm + P_GV + (q16 >> 3) * 8 * KB + sw128_offset(r, (q16 & 7) * 8)) =
@@ -702,7 +704,7 @@ __device__ __forceinline__ void prep_loop(const CUtensorMap &tm_q, const CUtenso
                 *reinterpret_cast<uint4 *>(sm + P_GV + 16 * idx) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
-        grp.sync();
+        if (grp.sync_or(!v_ok)) { aborted = true; break; }
 
         // ---- [W | Ut] = T Diag(beta) [Gamma K | V]: one N = 256 chain, Gamma k and v being four
         // consecutive 64-column blocks and W, Ut consecutive accumulators (an MMA instruction
