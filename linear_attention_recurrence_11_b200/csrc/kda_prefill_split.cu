@@ -965,12 +965,6 @@ __device__ __forceinline__ void chain_dbuf(const SplitParams &sp, const CUtensor
         if (ok) { rec_phase ^= 1u << b; rec_armed &= ~(1u << b); }
         return !grp.sync_or(!ok);
     };
-    auto wait_mma = [&]() -> bool {
-        const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
-        if (ok) { mma_phase ^= 1u; mma_pending = false; }
-        tc_fence_after();
-        return !grp.sync_or(!ok);
-    };
     auto issue_u = [&](int b) {  // [U ; Gamma Q S] = [-W ; Gamma Q] S into the accumulator of buffer b
         tc_fence_after();
         Opnd A{sbase + b * C_RECSTRIDE + REC_WQ, false, 16 * KB, 0};
@@ -1008,16 +1002,20 @@ __device__ __forceinline__ void chain_dbuf(const SplitParams &sp, const CUtensor
             tmem_wait_st();
             tc_fence_before();
         }
-        if (!wait_mma()) { aborted = true; break; }
+        // every thread sees the state product complete; one barrier then both publishes U and
+        // agrees on a wait that ran out
+        bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
+        if (ok) { mma_phase ^= 1u; mma_pending = false; }
+        tc_fence_after();
 
         // U = Ut - W S (rows 0..63) -> bf16 B operand, written over the record's Ut tile
         // (all-zero values, the transition pass of a segment: the record's Ut is left out)
-        if (quarter < 2)
+        if (ok && quarter < 2)
             u_readout(buf + REC_UT + half * 8 * KB, buf + REC_UT + half * 8 * KB, 32 * quarter + lane,
                       tmem + tlane + tmu + 64u * half, p.v != nullptr);
         fence_proxy_async_smem();
         tc_fence_before();
-        grp.sync();
+        if (grp.sync_or(!ok)) { aborted = true; break; }
 
         // O = Gamma Q S + P U (rows 64..127 of the accumulator), S += Kh^T U
         if (tid == 0) {
@@ -1030,14 +1028,18 @@ __device__ __forceinline__ void chain_dbuf(const SplitParams &sp, const CUtensor
             mma_commit(bar_mma);
             mma_pending = true;
         }
-        if (!wait_mma()) { aborted = true; break; }
-        if (tid == 0 && ch + 2 < nchunks) {  // this buffer's record is consumed: the one two chunks ahead
+        ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
+        if (ok) { mma_phase ^= 1u; mma_pending = false; }
+        tc_fence_after();
+        // this buffer's record is consumed (its generic reads were before the barrier above, the
+        // products that read it are complete): the record two chunks ahead
+        if (ok && tid == 0 && ch + 2 < nchunks) {
             if (rdy.ready_now(task(ch + 2))) load_rec(ch + 2);
             else rec_late[b] = ch + 2;
         }
 
         // the bf16 copy of the updated state: the next chunk's state product waits on it
-        {
+        if (ok) {
             uint8_t *sb = sm + C_SB + half * 16 * KB;
             float sv[4][16];
 #pragma unroll
@@ -1072,11 +1074,16 @@ __device__ __forceinline__ void chain_dbuf(const SplitParams &sp, const CUtensor
                 rec_late[b ^ 1] = -1;
             }
         }
-        grp.sync();
+        // every thread sees the next record land; one barrier then publishes the state's copy,
+        // and agrees on both waits
+        bool rok = true;
         if (more) {
-            if (!wait_rec(b ^ 1)) { aborted = true; break; }
-            if (tid == 0) { issue_u(b ^ 1); mma_pending = true; }
+            const int nb = b ^ 1;
+            rok = !flag_fail && mbar_wait_bounded(&bar_rec[nb], (rec_phase >> nb) & 1u, kWaitCycles);
+            if (rok) { rec_phase ^= 1u << nb; rec_armed &= ~(1u << nb); }
         }
+        if (grp.sync_or(!ok || !rok)) { aborted = true; break; }
+        if (more && tid == 0) { issue_u(b ^ 1); mma_pending = true; }
 
         // outputs (rows 64..127 of this chunk's accumulator) while the next product runs. A
         // full chunk is staged in its own tile and leaves by two tensor stores; the rows of a

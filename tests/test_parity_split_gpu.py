@@ -108,6 +108,22 @@ def test_split_one_sequence_records_beside_the_chains(K, oracle_mod, spare):
     assert torch.equal(o, o_p) and torch.equal(ST, S_p)
 
 
+@pytest.mark.parametrize("T", [64 * 3 + 61, 64 * 2 + 61])
+def test_split_one_sequence_fewest_heads(K, oracle_mod, T):
+    """32 heads, the fewest that take the records-beside-chains launch. At 4 chunks (the fewest
+    it takes) every chunk but the first is produced beside the chains, the ragged last one
+    included; at 3 chunks the two-kernel form runs. Every head against the oracle, and bit for
+    bit against the pipe form."""
+    H = 32
+    inp = case(1, T, H, 128, 128, "bf16", seed=95 + T, s0_std=0.1, g_min_frac=0.1)
+    o, ST = fwd(K, inp, "tc_split")
+    units = [(0, h) for h in range(H)]
+    o_ref, S_ref = oracle_forward(oracle_mod, inp, units=units)
+    compare_units(o, ST, o_ref, S_ref, units, tol=TOL["bf16"], label=f"split, 32 heads, T={T}")
+    o_p, S_p = fwd(K, inp, "tc_pipe")
+    assert torch.equal(o, o_p) and torch.equal(ST, S_p)
+
+
 def test_split_one_sequence_in_a_cuda_graph(K):
     """The one-sequence split step (40 heads: a cooperative launch beside the prep kernel)
     captured in a CUDA graph and replayed: the same outputs as the eager call, bit for bit."""
