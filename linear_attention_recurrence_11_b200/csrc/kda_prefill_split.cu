@@ -1882,9 +1882,10 @@ cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r) {
 // The tail form's split of the tasks: P producing groups keep pace with the chains over the
 // last r x P x nch / units chunks, r the ratio of a chain's cycles per chunk to a producing
 // group's cycles per task. Measured on B200 (96 heads, 8192 tokens): about 4.4K and 23K (two
-// groups of one CTA per SM; the step is fastest at r = 0.19, 0.610 ms against 0.636 for the
+// groups of one CTA per SM; the step is fastest at r = 0.19, 0.59 ms against 0.636 for the
 // two-kernel form, with 26 of 128 chunks in the tail; the producers with fused pre-operations
-// take about 1.4 times as long per task); the prep kernel does the other chunks.
+// take about 1.4 times as long per task, and that step is fastest at r = 0.12, 16 chunks in the
+// tail, 0.74 ms against 0.76 at 0.14); the prep kernel does the other chunks.
 // With few units the chains dominate the step (8 heads x 65,536 tokens: 2.7 ms, the prep of all
 // records 0.27 ms), and the tail form only adds its flag checks to them.
 bool tail_ok(const PrefillArgs &a) {
@@ -1900,7 +1901,7 @@ const void *tail_kernel_for(const PrefillArgs &a) {
 long long tail_first_task(const PrefillArgs &a) {
     const long long units = a.H, nch = (a.T + C - 1) / C;
     const long long producers = 2LL * (num_sms() - units);
-    const double r = a.fuse ? 0.14 : 0.19;
+    const double r = a.fuse ? 0.12 : 0.19;
     long long tail = (long long)((double)producers * (double)nch * r / (double)units);
     tail = tail < 1 ? 1 : (tail > nch - 1 ? nch - 1 : tail);
     return (nch - tail) * units;
