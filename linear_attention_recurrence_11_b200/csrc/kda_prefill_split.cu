@@ -193,7 +193,9 @@ __global__ void chunk_base_kernel(const int32_t *cu, int num, int32_t *base) {
 
 // ======================================================================= prep
 // Every task of the batch, strided over the grid; the record of task t is the t-th of the
-// workspace (the two-kernel form: the chains run after this kernel has finished).
+// workspace (the two-kernel form: the chains run after this kernel has finished). The tasks
+// are taken from the last to the first, so that the records still in L2 when the chains start
+// are those of the first chunks, which the chains read first.
 struct StaticTasks {
     static constexpr bool kPublish = false, kLatePublish = false;
     const SplitParams *sp;
@@ -202,13 +204,13 @@ struct StaticTasks {
         total = sp->chunk_base ? (long long)sp->chunk_base[sp->a.num_units] * sp->a.H : sp->tasks;
         t = blockIdx.x;
         if (t >= total) return false;
-        k = task_at(*sp, t);
+        k = task_at(*sp, total - 1 - t);
         return true;
     }
     __device__ bool next(Task &k) {
         t += gridDim.x;
         if (t >= total) return false;
-        k = task_at(*sp, t);
+        k = task_at(*sp, total - 1 - t);
         return true;
     }
     __device__ uint8_t *record(const Task &k) const { return sp->rec + (size_t)k.t * REC_BYTES; }
