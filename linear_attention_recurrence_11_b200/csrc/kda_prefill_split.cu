@@ -1185,14 +1185,9 @@ constexpr int kRingSlots = 4;
 
 // pipeline chain-role smem layout (the record pieces at their record offsets, then S bf16)
 constexpr uint32_t X_SB = REC_BYTES;                  // 32 KB S (bf16), B operand MN-major
-constexpr uint32_t X_BAR = X_SB + 32 * KB;            // 5 mbarriers (pieces A, B or Ut, C; MMA; P)
+constexpr uint32_t X_BAR = X_SB + 32 * KB;            // 4 mbarriers (pieces A, B, C; MMA)
 constexpr uint32_t X_TMEMADDR = X_BAR + 64;
 constexpr uint32_t X_SMEM_USED = X_BAR + 128;
-// the compact chains add a U / O tile (16 KB, [tok][dv] MN-major bf16, N-blocks 8 KB apart): U
-// goes there instead of over the record's Ut and the outputs are staged there instead of over
-// Kh, so that every record piece is reloaded as soon as its own tile is consumed
-constexpr uint32_t X_UO = X_BAR + 1024;
-constexpr uint32_t X2_SMEM_USED = X_UO + 16 * KB;
 constexpr uint32_t X_TM_U = 0, X_TM_S = 128, X_TM_COLS = 256;
 
 struct PipeParams {
@@ -1265,10 +1260,9 @@ struct RingTasks {
     }
 };
 
-// Where a chain's records come from. The ring (pipe form): record tau of chain c is in slot
-// tau % R once the producers have published it, and its slot is handed back once all three
-// pieces are in shared memory. The array (split form): every record is in the workspace,
-// written by an earlier kernel.
+// Where the pipe form's chains find their records: record tau of chain c is in slot tau % R
+// of the ring once the producers have published it, and its slot is handed back once all
+// three pieces are in shared memory.
 struct RingRecords {
     const PipeParams *pp;
     int c;
@@ -1283,36 +1277,22 @@ struct RingRecords {
     }
     __device__ void release(long long tau) const { st_release_gpu(pp->consumed + c, (unsigned)(tau + 1)); }
 };
-struct ArrayRecords {
-    const uint8_t *rec;
-    size_t H;
-    int h;
-    long long cbase;
-    __device__ const uint8_t *slot(long long tau) const { return rec + ((size_t)(cbase + tau) * H + (size_t)h) * REC_BYTES; }
-    __device__ bool wait_ready(long long) const { return true; }
-    __device__ void release(long long) const {}
-};
 
 // The state chain of unit (sequence n, head h) with its records read piece by piece into one
 // buffer as their shared-memory tiles free up: A (state product operand, decay) once the state
 // product is done, B (Ut, P) once the output product is done, C (Kh) once the outputs staged
 // over it have left. One 256-thread group, ~106 KB of shared memory, 256 TMEM columns.
-// kUO (the compact chain kernel): U and the staged outputs live in their own tile (X_UO,
-// 16 KB more), and B is loaded as Ut (once U has been read out) and P (once the output
-// product is done), C once the output product is done: each piece then arrives about a chunk
-// before it is needed.
-template <class Rec, bool kUO = false>
+template <class Rec>
 __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorMap &tm_o, uint8_t *sm, const Group &grp,
                                            int n, int h, const Rec &recs) {
     const uint32_t sbase = smem_u32(sm);
     uint64_t *bar_a = reinterpret_cast<uint64_t *>(sm + X_BAR);
-    uint64_t *bar_b = bar_a + 1;  // B, or (kUO) Ut
+    uint64_t *bar_b = bar_a + 1;  // B: Ut and P
     uint64_t *bar_c = bar_a + 2;
     uint64_t *bar_mma = bar_a + 3;
-    uint64_t *bar_p = bar_a + 4;  // kUO: P
-    uint8_t *const uo = kUO ? sm + X_UO : sm + REC_UT;  // where U goes
-    const uint32_t uo_addr = sbase + (kUO ? X_UO : REC_UT);
-    uint8_t *const ostage = kUO ? sm + X_UO : sm + REC_KH;  // where a full chunk's outputs are staged
+    uint8_t *const uo = sm + REC_UT;  // U goes over the record's Ut
+    const uint32_t uo_addr = sbase + REC_UT;
+    uint8_t *const ostage = sm + REC_KH;  // a full chunk's outputs are staged over Kh
     uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + X_TMEMADDR);
 
     const int tid = grp.tid, warp = tid >> 5, lane = tid & 31;
@@ -1336,7 +1316,6 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
         mbar_init(bar_b, 1);
         mbar_init(bar_c, 1);
         mbar_init(bar_mma, 1);
-        if (kUO) mbar_init(bar_p, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_o);
     }
@@ -1345,24 +1324,18 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
         if (grp.relinquish) tmem_relinquish();
     }
     grp.sync();
-    // thread-0 state of the copies: armed bits (1 A, 2 B or Ut, 4 C, 8 P) and the phase of each barrier
-    uint32_t armed = 0, ph_a = 0, ph_b = 0, ph_c = 0, ph_p = 0, mma_phase = 0;
+    // thread-0 state of the copies: armed bits (1 A, 2 B, 4 C) and the phase of each barrier
+    uint32_t armed = 0, ph_a = 0, ph_b = 0, ph_c = 0, mma_phase = 0;
     bool flag_fail = false, aborted = false, mma_pending = false;
     auto load_a = [&](long long tau) {
         mbar_arrive_expect_tx(bar_a, REC_A_BYTES);
         bulk_load(sm + REC_WQ, slot(tau) + REC_WQ, REC_A_BYTES, bar_a);
         armed |= 1u;
     };
-    auto load_b = [&](long long tau) {  // B, or (kUO) its Ut part
-        const uint32_t bytes = kUO ? REC_P - REC_UT : REC_B_BYTES;
-        mbar_arrive_expect_tx(bar_b, bytes);
-        bulk_load(sm + REC_UT, slot(tau) + REC_UT, bytes, bar_b);
+    auto load_b = [&](long long tau) {
+        mbar_arrive_expect_tx(bar_b, REC_B_BYTES);
+        bulk_load(sm + REC_UT, slot(tau) + REC_UT, REC_B_BYTES, bar_b);
         armed |= 2u;
-    };
-    auto load_p = [&](long long tau) {  // kUO: the P part of B
-        mbar_arrive_expect_tx(bar_p, REC_KH - REC_P);
-        bulk_load(sm + REC_P, slot(tau) + REC_P, REC_KH - REC_P, bar_p);
-        armed |= 8u;
     };
     auto load_c = [&](long long tau) {
         mbar_arrive_expect_tx(bar_c, REC_C_BYTES);
@@ -1375,7 +1348,6 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
         } else {
             load_a(0);
             load_b(0);
-            if (kUO) load_p(0);
             load_c(0);
         }
     }
@@ -1466,22 +1438,18 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
             if (!recs.wait_ready(tau + 1)) flag_fail = true;
             else load_a(tau + 1);
         }
-        // (kUO) the previous chunk's output stores have read the U / O tile
-        if (kUO && tid == 0) bulk_wait_read_all();
         if (!wait_piece(bar_b, ph_b, 2u)) { aborted = true; break; }
 
-        // U = Ut - W S (rows 0..63) -> bf16 B operand (over the record's Ut tile, or kUO in its own)
+        // U = Ut - W S (rows 0..63) -> bf16 B operand, over the record's Ut tile
         if (quarter < 2)
             u_readout(sm + REC_UT + half * 8 * KB, uo + half * 8 * KB, 32 * quarter + lane,
                       tmem + tlane + X_TM_U + 64u * half, p.v != nullptr);
         fence_proxy_async_smem();
         tc_fence_before();
         if (!wait_piece(bar_c, ph_c, 4u)) { aborted = true; break; }
-        if (kUO && !wait_piece(bar_p, ph_p, 8u)) { aborted = true; break; }
         if (tid == 0) {
             // every piece of record tau is in shared memory: its slot may be refilled
             recs.release(tau);
-            if (kUO && more && !flag_fail) load_b(tau + 1);  // Ut is consumed
             tc_fence_after();
             Opnd AK{sbase + REC_KH, true, 0, 8 * KB};
             Opnd BU{uo_addr, true, 0, 8 * KB};
@@ -1492,17 +1460,8 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
             mma_pending = true;
         }
         if (!wait_mma()) { aborted = true; break; }
-        if (tid == 0 && more && !flag_fail) {
-            if (kUO) {  // P and Kh are consumed
-                load_p(tau + 1);
-                load_c(tau + 1);
-            } else {
-                load_b(tau + 1);  // Ut, U and P are consumed
-            }
-        }
+        if (tid == 0 && more && !flag_fail) load_b(tau + 1);  // Ut, U and P are consumed
 
-        // the bf16 copy of the updated state, and this chunk's outputs into registers, before
-        // the next state product overwrites the accumulator
         // the bf16 copy of the updated state, and this chunk's outputs (rows 64..127 of the
         // accumulator) out of TMEM before the next state product overwrites it: a full chunk is
         // staged over the Kh tile (its product is done) for two tensor stores, the rows of a
@@ -1568,7 +1527,7 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
                 tma_store_3d(&tm_o, ostage + 8 * KB, 64, h, (int)tok0);
                 bulk_commit();
             }
-            if (!kUO && more && !flag_fail) {  // Kh of the next record, once the outputs have left its tile
+            if (more && !flag_fail) {  // Kh of the next record, once the outputs have left its tile
                 bulk_wait_read_all();
                 load_c(tau + 1);
             }
@@ -1581,7 +1540,6 @@ __device__ __forceinline__ void chain_role(const PrefillArgs &p, const CUtensorM
             if (p.dev_status) atomicExch(p.dev_status, (int)KDA_ERR_TIMEOUT);
             if (armed & 1u) mbar_wait_bounded(bar_a, ph_a, kWaitCycles);
             if (armed & 2u) mbar_wait_bounded(bar_b, ph_b, kWaitCycles);
-            if (armed & 8u) mbar_wait_bounded(bar_p, ph_p, kWaitCycles);
             if (armed & 4u) mbar_wait_bounded(bar_c, ph_c, kWaitCycles);
             if (mma_pending) mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
         }
@@ -1634,20 +1592,6 @@ kda_pipe_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 }
 
-// The state chains over the record array with one record buffer: ~106 KB of shared memory and
-// 256 TMEM columns, so two chains share an SM (for batches of more units than SMs).
-__global__ void __launch_bounds__(NT, 2)
-kda_chain2_kernel(const __grid_constant__ CUtensorMap tm_o, const SplitParams sp) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const PrefillArgs &p = sp.a;
-    const int h = blockIdx.x % p.H;
-    const int n = unit_seq(p, blockIdx.x / p.H);
-    const ArrayRecords recs{sp.rec, (size_t)p.H, h, sp.chunk_base ? (long long)sp.chunk_base[n] : (long long)n * sp.nch};
-    chain_role<ArrayRecords, true>(p, tm_o, sm, Group{(int)threadIdx.x, 0u, true}, n, h, recs);
-}
-constexpr uint32_t CHAIN2_SMEM = X2_SMEM_USED + 1024;
-
 // The tail form (dense batches of one sequence with SMs to spare beside its units): the prep
 // kernel writes the records of the first chunks, then one cooperative launch runs every unit's
 // chain on an SM of its own (CTA c < nchain, one 256-thread group) while the other CTAs, two
@@ -1684,7 +1628,6 @@ kda_tail_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                           Group{(int)(threadIdx.x & (NT - 1)), 1u + (uint32_t)gi, false});
     }
 }
-static_assert(2 * 1024 + P_SMEM_BYTES + CHAIN2_SMEM <= 233472, "a prep CTA and a compact chain share an SM");
 
 int num_sms() { return device_sm_count(); }
 
@@ -1851,12 +1794,11 @@ cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r) {
     if (tokens == 0) return launch_prefill_simt(pass);
     CUtensorMap mo;
     if (!make_map(&mo, pass.o ? pass.o : pass.q, tokens, pass.H, 64, true)) return cudaErrorInvalidValue;
-    // more units than SMs: the one-buffer chains, two per SM; otherwise the double-buffered ones
-    const bool compact = (long long)pass.num_units * pass.H > num_sms();
-    cudaError_t e = compact ? cudaFuncSetAttribute(kda_chain2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                   (int)CHAIN2_SMEM)
-                            : cudaFuncSetAttribute(pass.snap_every ? kda_chain_kernel<true> : kda_chain_kernel<false>,
-                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C_SMEM_BYTES);
+    // the double-buffered chains, one per SM, in as many waves as the units need (with more
+    // units than SMs they beat one-buffer chains two per SM: 2 x 96 heads x 8192 tokens took
+    // 1.22 ms per step against 1.39)
+    cudaError_t e = cudaFuncSetAttribute(pass.snap_every ? kda_chain_kernel<true> : kda_chain_kernel<false>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C_SMEM_BYTES);
     if (e != cudaSuccess) return e;
     SplitParams sp{};
     sp.a = pass;
@@ -1867,17 +1809,10 @@ cudaError_t launch_split_chain(const PrefillArgs &pass, const SplitRecords &r) {
     sp.nch = r.nch;
     sp.tasks = r.tasks;
     const unsigned grid_c = (unsigned)((size_t)pass.num_units * pass.H);
-    if (compact) {
-        e = cudaFuncSetAttribute(kda_chain2_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                 (int)cudaSharedmemCarveoutMaxShared);
-        if (e != cudaSuccess) return e;
-        kda_chain2_kernel<<<grid_c, NT, CHAIN2_SMEM, pass.stream>>>(mo, sp);
-    } else {
-        if (pass.snap_every)
-            kda_chain_kernel<true><<<grid_c, NT, C_SMEM_BYTES, pass.stream>>>(mo, sp);
-        else
-            kda_chain_kernel<false><<<grid_c, NT, C_SMEM_BYTES, pass.stream>>>(mo, sp);
-    }
+    if (pass.snap_every)
+        kda_chain_kernel<true><<<grid_c, NT, C_SMEM_BYTES, pass.stream>>>(mo, sp);
+    else
+        kda_chain_kernel<false><<<grid_c, NT, C_SMEM_BYTES, pass.stream>>>(mo, sp);
     return cudaGetLastError();
 }
 
