@@ -95,8 +95,9 @@ typedef enum { KDA_FUSE_NORM_QK = 1, KDA_FUSE_GATE_LOGITS = 2 } kda_fuse;
  *    at once, the records passing through a ring of 4 per unit; for at most
  *    two thirds of twice the SM count of units (197 on 148 SMs), else
  *    KDA_ERR_UNSUPPORTED. Workspace: about 292 KiB per unit.
- * AUTO and TC run the single form for batches of more than three units per
- * SM (all SMs are busy and records would only add traffic); otherwise the
+ * AUTO and TC run the single form for batches of more than eight units per
+ * SM in dense batches, three in packed ones (all SMs are busy and records
+ * would only add traffic); otherwise the
  * split form when the workspace holds it, then the pipe form when its ring
  * fits, else the single form (TC returns KDA_ERR_UNSUPPORTED off the
  * tensor-core shapes, AUTO falls back to SIMT); a forced form returns
@@ -127,7 +128,8 @@ const char *kda_last_cuda_error(void);
  * composition of Q21-Q22. num_seqs is the number of packed sequences when
  * cu_seqlens is used, else B (B == 1 with num_seqs > 1 means packed
  * sequences). On the tensor-core shapes it is what AUTO runs (kda_path): for
- * batches of up to three (sequence, head) units per SM, the split form's
+ * batches of up to eight (sequence, head) units per SM (dense) or three
+ * (packed), the split form's
  * per-chunk records (74,752 bytes per chunk per head; for packed batches
  * counted for at most T / 64 + num_seqs chunks per head, plus the sequences'
  * chunk offsets and a longest-first schedule of up to 2048 sequences); for

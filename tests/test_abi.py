@@ -125,6 +125,11 @@ def test_workspace_and_launch_queries(K):
     assert K.kda_forward_workspace_size(2, 100, 3, 128, 128, 64, 2, 1, "tc_pipe") == \
         al(6 * 4 * REC) + al(6 * 5 * 4)
     assert K.kda_forward_workspace_size(2, 100, 3, 128, 128, 64, 2, 1, "tc_single") == 0
+    # dense batches take the split form up to eight units per SM (1184 on 148 SMs), then the
+    # single kernel (no workspace)
+    assert K.kda_forward_workspace_size(12, 8192, 96, 128, 128, 64, 12, 1) == 12 * 128 * 96 * REC
+    assert K.kda_forward_workspace_size(13, 8192, 96, 128, 128, 64, 13, 1) == 0
+    assert K.kda_forward_launches(12, 8192, 96, 128, 128, 64, 1, 0, 12) == 2
     # packed sequences, up to three units per SM: records for at most T / 64 + N chunks per
     # head, the sequences' chunk offsets, and a small longest-first schedule (up to 2048)
     n_ch = -(-100000 // 64) + 3

@@ -124,6 +124,22 @@ def test_split_one_sequence_fewest_heads(K, oracle_mod, T):
     assert torch.equal(o, o_p) and torch.equal(ST, S_p)
 
 
+def test_auto_dense_many_units_takes_split(K, oracle_mod):
+    """A dense batch of more units than three per SM (5 x 96 = 480, under the eight per SM of
+    dense batches): AUTO runs the split form, its chains in waves of one per SM. The same
+    outputs as a forced split call bit for bit (the single kernel rounds differently), and
+    sampled units against the oracle."""
+    B, T, H = 5, 130, 96
+    assert B * H > 3 * torch.cuda.get_device_properties(0).multi_processor_count
+    inp = case(B, T, H, 128, 128, "bf16", seed=97, s0_std=0.05)
+    o, ST = fwd(K, inp, "auto")
+    o_s, S_s = fwd(K, inp, "tc_split")
+    assert torch.equal(o, o_s) and torch.equal(ST, S_s)
+    units = [(0, 0), (1, 17), (2, 50), (4, 95)]
+    o_ref, S_ref = oracle_forward(oracle_mod, inp, units=units)
+    compare_units(o, ST, o_ref, S_ref, units, tol=TOL["bf16"], label="auto, 480 dense units")
+
+
 def test_split_one_sequence_in_a_cuda_graph(K):
     """The one-sequence split step (40 heads: a cooperative launch beside the prep kernel)
     captured in a CUDA graph and replayed: the same outputs as the eager call, bit for bit."""
