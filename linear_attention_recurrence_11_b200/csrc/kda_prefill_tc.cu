@@ -239,13 +239,14 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     long long tma_tok = t_begin;
     uint64_t *mma_bar = nullptr;
     uint32_t mma_bar_phase = 0;
-    // wait for an MMA commit; every thread takes part
+    // wait for an MMA commit in every thread; the barrier after the readout that follows both
+    // publishes it and agrees on a wait that ran out
     auto wait_mma = [&]() -> bool {
         const bool ok = mbar_wait_bounded(bar_mma, mma_phase, kWaitCycles);
         if (!ok) { mma_bar = bar_mma; mma_bar_phase = mma_phase; }
         mma_phase ^= 1u;
         tc_fence_after();
-        return __syncthreads_or(!ok) == 0;
+        return ok;
     };
 
     // thread roles for the token-parallel passes: subtile ti (a pair of warps), half hh of
@@ -490,18 +491,15 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             issue_k(tokn);
             tma_issued |= 2u;
         }
-        {
-            const bool ok = mbar_wait_bounded(bar_gram, gram_phase, kWaitCycles);
-            if (!ok) { mma_bar = bar_gram; mma_bar_phase = gram_phase; }
-            gram_phase ^= 1u;
-            tc_fence_after();
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
-        }
+        const bool ok_gram = mbar_wait_bounded(bar_gram, gram_phase, kWaitCycles);
+        if (!ok_gram) { mma_bar = bar_gram; mma_bar_phase = gram_phase; }
+        gram_phase ^= 1u;
+        tc_fence_after();
 
         // ---- phase 2: Gram readout -> A (fp32, strictly lower, times beta_r), P (bf16, lower).
         // Warps of column half j read block j's 32 columns; the masks select (never multiply)
         // so that the upper-triangle entries, which may overflow, are dropped.
-        {
+        if (ok_gram) {
             float v2[2][16];
             tmem_ld16(tmem + tlane + TM_GRAM + 32u * half, v2[0]);
             tmem_ld16(tmem + tlane + TM_GRAM + 32u * half + 16u, v2[1]);
@@ -536,7 +534,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
         }
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(!ok_gram)) { aborted = true; break; }
 
         // ---- phase 3: T = (I + A)^{-1} (unit lower triangular) by 16 x 16 blocks
         if (warp < NSUB && lane < 16) {
@@ -612,14 +610,14 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mma_chain<C / 16>(tmem + TM_U, A, BV, idKM, false);
             mma_commit(bar_mma);
         }
-        if (!wait_mma()) { aborted = true; break; }
-        if (more && tid == 0) {
+        const bool ok_wu = wait_mma();
+        if (ok_wu && more && tid == 0) {
             issue_v(tokn);
             tma_issued |= 4u;
         }
 
         // ---- phase 4: -W (rows 0..63) into the [-W ; Qt] operand
-        if (quarter < 2) {
+        if (ok_wu && quarter < 2) {
             const int r = 32 * quarter + lane;
             uint8_t *base = sm + OFF_WQ + half * 16 * KB;
             float v[4][16];
@@ -636,7 +634,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(!ok_wu)) { aborted = true; break; }
 
         // ---- [U ; Qt S] = [Ut ; 0] + [-W ; Qt] S
         if (tid == 0) {
@@ -663,14 +661,14 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             tmem_wait_st();
             tc_fence_before();
         }
-        if (!wait_mma()) { aborted = true; break; }
-        if (more && tid == 0) {  // rows 64..127 of the [-W ; Qt] operand are free
+        const bool ok_u = wait_mma();
+        if (ok_u && more && tid == 0) {  // rows 64..127 of the [-W ; Qt] operand are free
             issue_q(tokn);
             tma_issued |= 8u;
         }
 
         // ---- phase 5: U (rows 0..63) -> bf16 B operand, MN-major [tok][dv]
-        if (quarter < 2) {
+        if (ok_u && quarter < 2) {
             const int r = 32 * quarter + lane;
             uint8_t *base = sm + OFF_UB + half * 8 * KB;
             float v[4][16];
@@ -687,7 +685,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(!ok_u)) { aborted = true; break; }
 
         // ---- O = Qt S + P U (rows 64..127 of the same accumulator), S += dS = Kh^T U
         if (tid == 0) {
@@ -699,13 +697,13 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             mma_chain<C / 16>(tmem + TM_U, AP, BU, idKM, true);
             mma_commit(bar_mma);
         }
-        if (!wait_mma()) { aborted = true; break; }
+        const bool ok_o = wait_mma();
 
         // ---- phase 6: outputs, and the bf16 copy of the updated state. A full chunk of
         // outputs is staged in the U tile (free now, and already in the 128-byte swizzled
         // [token][dv] layout a tensor store reads) and written by two TMA stores; the
         // rows of a partial chunk are stored directly, so nothing lands past the sequence.
-        if (quarter >= 2 && p.o) {
+        if (ok_o && quarter >= 2 && p.o) {
             const int r = 32 * quarter + lane - 64;
             float v[4][16];
 #pragma unroll
@@ -731,7 +729,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 }
             }
         }
-        {
+        if (ok_o) {
             uint8_t *sb = sm + OFF_SB + half * 16 * KB;
             float sv[4][16];
 #pragma unroll
@@ -757,7 +755,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         fence_proxy_async_smem();
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(!ok_o)) { aborted = true; break; }
         if (Lc == C && tid == 0 && p.o) {
             tma_store_3d(&tm_o, sm + OFF_UB, 0, h, (int)tok0);
             tma_store_3d(&tm_o, sm + OFF_UB + 8 * KB, 64, h, (int)tok0);
