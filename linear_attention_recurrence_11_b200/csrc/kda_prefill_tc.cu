@@ -271,13 +271,12 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         const bool more = ch + 1 < nchunks;
         const long long tokn = tok0 + C;
 
-        // ---- wait for this chunk's tiles
-        {
-            const bool ok = mbar_wait_bounded(bar_tma, tma_phase, kWaitCycles);
+        // ---- wait for this chunk's tiles (every thread; the barrier after the decay pass agrees
+        // on a wait that ran out, and on failure the phase stays the one to drain on the way out)
+        const bool ok_tile = mbar_wait_bounded(bar_tma, tma_phase, kWaitCycles);
+        if (ok_tile) {
             tma_phase ^= 1u;
-            if (ok) tma_armed = false;
-            else tma_phase ^= 1u;  // still the phase to drain on the way out
-            if (__syncthreads_or(!ok)) { aborted = true; break; }
+            tma_armed = false;
         }
         if (tid < C) {
             sBeta[tid] = (tid < Lc) ? __bfloat162float(bnext) : 0.f;
@@ -358,7 +357,7 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             }
         }
         if (tid == 0) bulk_wait_read_all();  // the previous chunk's staged outputs have been read
-        __syncthreads();
+        if (__syncthreads_or(!ok_tile)) { aborted = true; break; }
         if (more && tid == 0) {  // g tile consumed: start the next chunk's loads
             mbar_arrive_expect_tx(bar_tma, tma_bytes);
             issue_g(tokn);
@@ -532,6 +531,12 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                         *reinterpret_cast<uint4 *>(prow + sw128_offset(r, s)) = make_uint4(0, 0, 0, 0);
                 }
             }
+            // T Diag(beta) (bf16, 128 rows) starts as zeros: the inverse writes its lower blocks,
+            // and rows 64..127 stay zero, the [Ut ; 0] the state product accumulates onto (the
+            // Gram products that read this tile are done)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<uint4 *>(sm + OFF_TB + 16 * (tid + NT * i)) = make_uint4(0, 0, 0, 0);
         }
         tc_fence_before();
         if (__syncthreads_or(!ok_gram)) { aborted = true; break; }
@@ -559,44 +564,23 @@ kda_prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
                 for (int ss = 0; ss < rr; ++ss) acc[ss & 3] = fmaf(-a[ss], x[ss], acc[ss & 3]);
                 x[rr] = (acc[0] + acc[1]) + (acc[2] + acc[3]);
             }
+            // T_ii, and its column times beta into T Diag(beta) (x is 0 above the diagonal)
+            const float bcol = sBeta[o0 + cc];
 #pragma unroll
-            for (int rr = 0; rr < 16; ++rr) TF[(o0 + rr) * LDT + o0 + cc] = x[rr];
+            for (int rr = 0; rr < 16; ++rr) {
+                TF[(o0 + rr) * LDT + o0 + cc] = x[rr];
+                *reinterpret_cast<__nv_bfloat16 *>(sm + OFF_TB + sw128_offset(o0 + rr, o0 + cc)) =
+                    __float2bfloat16_rn(x[rr] * bcol);
+            }
             if ((warp & 1) == 0) {  // the 16 x 16 block right of it, inside its 32 x 32 diagonal block
 #pragma unroll
                 for (int rr = 0; rr < 16; ++rr) TF[(o0 + rr) * LDT + o0 + 16 + cc] = 0.f;
             }
         }
         __syncthreads();
-        tri_inverse_offdiag(AF, TF, XS, tid);
-        // T Diag(beta) -> bf16 A operand (rows 0..63), zero rows 64..127: every thread converts
-        // two 8-column pieces of T (rows r and r + 32, same columns) and zeroes two pieces
-        {
-            const int r = tid >> 3, pc = (tid & 7) * 8;
-            const float4 b0 = *reinterpret_cast<const float4 *>(sBeta + pc);
-            const float4 b1 = *reinterpret_cast<const float4 *>(sBeta + pc + 4);
-            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-            float4 t[2][2];
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                t[i][0] = *reinterpret_cast<const float4 *>(TF + (r + 32 * i) * LDT + pc);
-                t[i][1] = *reinterpret_cast<const float4 *>(TF + (r + 32 * i) * LDT + pc + 4);
-            }
-#pragma unroll
-            for (int i = 0; i < 2; ++i) {
-                const int ri = r + 32 * i;
-                const float tv[8] = {t[i][0].x, t[i][0].y, t[i][0].z, t[i][0].w, t[i][1].x, t[i][1].y, t[i][1].z, t[i][1].w};
-                float u[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) u[e] = (pc + e <= ri) ? tv[e] * bb[e] : 0.f;
-                uint4 w;
-                w.x = pack_bf2(u[0], u[1]);
-                w.y = pack_bf2(u[2], u[3]);
-                w.z = pack_bf2(u[4], u[5]);
-                w.w = pack_bf2(u[6], u[7]);
-                *reinterpret_cast<uint4 *>(sm + OFF_TB + sw128_offset(ri, pc)) = w;
-                *reinterpret_cast<uint4 *>(sm + OFF_TB + sw128_offset(ri + 64, pc)) = make_uint4(0, 0, 0, 0);
-            }
-        }
+        // the off-diagonal blocks of T, each also written times beta into T Diag(beta): the bf16
+        // A operand of [W | Ut]
+        tri_inverse_offdiag(AF, TF, XS, tid, 0, sm + OFF_TB, sBeta);
         fence_proxy_async_smem();
         __syncthreads();
 
